@@ -1,0 +1,195 @@
+"""ctypes loader for the float64 selective-scan oracle in ``selscan_oracle.c``.
+
+TEST INFRASTRUCTURE ONLY: the test suite, the smoke check and the benchmark's
+CPU-baseline leg are the only callers. The CUDA library never imports this
+module and this module never imports the CUDA library.
+
+All array arguments are numpy arrays of any real dtype; they are widened to
+float64 (exact for fp32 and bf16 values) before the call. Layouts follow the
+pages' statement of the selective SSM ("Mamba & State Space Models — Guide
+Complet", §4 "Implémentation du SSM sélectif (S6)"): x, delta, z, y
+[batch, L, D]; B, C [batch, L, N]; A [D, N]; D, delta_bias [D]; states
+[batch, D, N].
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from typing import Optional
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+SOURCE = os.path.join(_HERE, "selscan_oracle.c")
+LIBRARY = os.path.join(_HERE, "_build", "libselscan_oracle.so")
+
+BBAR_DELTA = 0  # B_bar = Δ·B (the hot path's input term)
+BBAR_ZOH = 1  # B_bar = (exp(Δ·A) − 1)/A·B (diagonal zero-order hold)
+
+_dp = ctypes.POINTER(ctypes.c_double)
+_i64 = ctypes.c_int64
+
+
+def build(source: str = SOURCE, out: str = LIBRARY) -> str:
+    """Compile the oracle with gcc (IEEE float64, no fast-math)."""
+    os.makedirs(os.path.dirname(out), exist_ok=True)
+    tmp = out + f".tmp{os.getpid()}"
+    cmd = ["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11",
+           "-o", tmp, source, "-lm"]
+    subprocess.run(cmd, check=True)
+    os.replace(tmp, out)
+    return out
+
+
+def _ptr(a: Optional[np.ndarray]):
+    if a is None:
+        return None
+    return a.ctypes.data_as(_dp)
+
+
+def _f64(a, shape=None) -> Optional[np.ndarray]:
+    if a is None:
+        return None
+    arr = np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+    if shape is not None and arr.shape != tuple(shape):
+        raise ValueError(f"expected shape {tuple(shape)}, got {arr.shape}")
+    return arr
+
+
+def default_threads() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:  # pragma: no cover
+        return os.cpu_count() or 1
+
+
+class Oracle:
+    """Handle on one compiled oracle library (the default one, or a variant
+    compiled from edited source by the planted-mistake tests)."""
+
+    def __init__(self, lib_path: Optional[str] = None):
+        if lib_path is None:
+            lib_path = LIBRARY
+            if (not os.path.exists(lib_path)
+                    or os.path.getmtime(lib_path) < os.path.getmtime(SOURCE)):
+                build()
+        self.path = lib_path
+        lib = ctypes.CDLL(lib_path)
+        lib.oracle_selscan_fwd.restype = None
+        lib.oracle_selscan_fwd.argtypes = [
+            _dp, _dp, _dp, _dp, _dp, _dp, _dp, _dp, ctypes.c_int, ctypes.c_int,
+            _dp, _dp, _dp, _i64, _i64, _i64, _i64, ctypes.c_int]
+        lib.oracle_selscan_fwd_chunked.restype = None
+        lib.oracle_selscan_fwd_chunked.argtypes = [
+            _dp, _dp, _dp, _dp, _dp, _dp, _dp, _dp, ctypes.c_int, ctypes.c_int,
+            _dp, _dp, _dp, _i64, _i64, _i64, _i64, _i64, ctypes.c_int]
+        lib.oracle_state_update.restype = None
+        lib.oracle_state_update.argtypes = [
+            _dp, _dp, _dp, _dp, _dp, _dp, _dp, _dp, _dp, ctypes.c_int, _dp,
+            _i64, _i64, _i64]
+        lib.oracle_compose.restype = None
+        lib.oracle_compose.argtypes = [ctypes.c_double] * 4 + [_dp, _dp]
+        lib.oracle_zoh_discretize.restype = None
+        lib.oracle_zoh_discretize.argtypes = [ctypes.c_double, _dp, _dp, _dp,
+                                              _dp, _i64]
+        self.lib = lib
+
+    # -- whole-sequence scan -------------------------------------------------
+    def _fwd_args(self, x, delta, A, B, C, D, z, delta_bias, h0):
+        x = _f64(x)
+        if x.ndim != 3:
+            raise ValueError("x must be [batch, L, D]")
+        batch, L, dim = x.shape
+        A = _f64(A)
+        if A.ndim != 2 or A.shape[0] != dim:
+            raise ValueError("A must be [D, N]")
+        N = A.shape[1]
+        args = dict(
+            x=x,
+            delta=_f64(delta, x.shape),
+            A=A,
+            B=_f64(B, (batch, L, N)),
+            C=_f64(C, (batch, L, N)),
+            D=_f64(D, (dim,)),
+            z=_f64(z, x.shape),
+            delta_bias=_f64(delta_bias, (dim,)),
+            h0=_f64(h0, (batch, dim, N)),
+        )
+        return args, (batch, L, dim, N)
+
+    def fwd(self, x, delta, A, B, C, D=None, z=None, delta_bias=None,
+            softplus=True, bbar=BBAR_DELTA, h0=None, threads=None):
+        """Return (y, final_state) as float64 arrays."""
+        a, (batch, L, dim, N) = self._fwd_args(x, delta, A, B, C, D, z,
+                                               delta_bias, h0)
+        y = np.empty((batch, L, dim), dtype=np.float64)
+        hs = np.empty((batch, dim, N), dtype=np.float64)
+        self.lib.oracle_selscan_fwd(
+            _ptr(a["x"]), _ptr(a["delta"]), _ptr(a["A"]), _ptr(a["B"]),
+            _ptr(a["C"]), _ptr(a["D"]), _ptr(a["z"]), _ptr(a["delta_bias"]),
+            int(bool(softplus)), int(bbar), _ptr(a["h0"]), _ptr(y), _ptr(hs),
+            batch, L, dim, N, int(threads or default_threads()))
+        return y, hs
+
+    def fwd_chunked(self, x, delta, A, B, C, D=None, z=None, delta_bias=None,
+                    softplus=True, bbar=BBAR_DELTA, h0=None, chunk=256,
+                    threads=None):
+        """Chunk-aggregate / carry / rescan form; returns (y, final_state)."""
+        a, (batch, L, dim, N) = self._fwd_args(x, delta, A, B, C, D, z,
+                                               delta_bias, h0)
+        y = np.empty((batch, L, dim), dtype=np.float64)
+        hs = np.empty((batch, dim, N), dtype=np.float64)
+        self.lib.oracle_selscan_fwd_chunked(
+            _ptr(a["x"]), _ptr(a["delta"]), _ptr(a["A"]), _ptr(a["B"]),
+            _ptr(a["C"]), _ptr(a["D"]), _ptr(a["z"]), _ptr(a["delta_bias"]),
+            int(bool(softplus)), int(bbar), _ptr(a["h0"]), _ptr(y), _ptr(hs),
+            batch, L, dim, N, int(chunk), int(threads or default_threads()))
+        return y, hs
+
+    # -- single-token decode -------------------------------------------------
+    def state_update(self, state, x, delta, A, B, C, D=None, z=None,
+                     delta_bias=None, softplus=True):
+        """One recurrent step. Returns (y [batch, D], new_state); the input
+        state array is not modified."""
+        st = np.array(state, dtype=np.float64, copy=True, order="C")
+        if st.ndim != 3:
+            raise ValueError("state must be [batch, D, N]")
+        batch, dim, N = st.shape
+        x = _f64(x, (batch, dim))
+        y = np.empty((batch, dim), dtype=np.float64)
+        self.lib.oracle_state_update(
+            _ptr(st), _ptr(x), _ptr(_f64(delta, (batch, dim))),
+            _ptr(_f64(A, (dim, N))), _ptr(_f64(B, (batch, N))),
+            _ptr(_f64(C, (batch, N))), _ptr(_f64(D, (dim,))),
+            _ptr(_f64(z, (batch, dim))), _ptr(_f64(delta_bias, (dim,))),
+            int(bool(softplus)), _ptr(y), batch, dim, N)
+        return y, st
+
+    # -- pieces exposed for the pins -----------------------------------------
+    def compose(self, a_later, b_later, a_earlier, b_earlier):
+        ao = ctypes.c_double()
+        bo = ctypes.c_double()
+        self.lib.oracle_compose(float(a_later), float(b_later),
+                                float(a_earlier), float(b_earlier),
+                                ctypes.byref(ao), ctypes.byref(bo))
+        return ao.value, bo.value
+
+    def zoh_discretize(self, dt, A, B):
+        A = _f64(A)
+        B = _f64(B, A.shape)
+        Ab = np.empty_like(A)
+        Bb = np.empty_like(A)
+        self.lib.oracle_zoh_discretize(float(dt), _ptr(A), _ptr(B), _ptr(Ab),
+                                       _ptr(Bb), A.shape[0])
+        return Ab, Bb
+
+
+_DEFAULT: Optional[Oracle] = None
+
+
+def default() -> Oracle:
+    global _DEFAULT
+    if _DEFAULT is None:
+        _DEFAULT = Oracle()
+    return _DEFAULT

@@ -1,0 +1,278 @@
+/*
+ * selscan_oracle.c -- plain float64 CPU reference of the Mamba-1 selective
+ * scan and of its single-token recurrent state update.
+ *
+ * TEST INFRASTRUCTURE ONLY. This file is the ground truth the CUDA library is
+ * checked against. Only the test suite, the smoke check and the benchmark's
+ * CPU-baseline leg load it. It shares no code, header, table or constant with
+ * the CUDA sources, and the product path never calls it.
+ *
+ * Every loop below is the plain definition, one (batch, channel) chain at a
+ * time, each chain strictly sequential in t. OpenMP only spreads independent
+ * chains over cores; it does not reorder any chain's arithmetic.
+ *
+ * Pages followed (title, section):
+ *  [Guide] "Mamba & State Space Models — Guide Complet" (skillsmp.com skill
+ *          "mamba-ssm"):
+ *          §1 "Discrétisation": ZOH, A_bar = exp(Δ·A),
+ *             B_bar = (exp(Δ·A) − I)·A⁻¹·B; h_k = A_bar·h_{k−1} + B_bar·u_k,
+ *             y_k = C·h_k + D·u_k.
+ *          §4 "Implémentation du SSM sélectif (S6)": Δ = softplus(dt_proj(x))
+ *             with the bias inside the softplus; per token A_bar = exp(Δ_t·A)
+ *             with A diagonal per channel; h starts at zero; y_t = h·C_t + D·x_t
+ *             with D a per-channel vector.
+ *          §4 "Parallel Associative Scan": (a,b)⊕(a',b') = (a·a', a·b' + b).
+ *  [Johe]  "Mamba и State Space Models: альтернатива Transformer"
+ *          (johe.ru/blog/mamba-ssm):
+ *          "SSM as RNN": input term scaled by delta, y read after the update.
+ *          "Discretization": delta_bias added to the projected Δ.
+ *          "Hardware-Aware Scan": the state is carried across fixed-size
+ *             blocks of the sequence.
+ *          "Mamba Block": output gated by silu(gate).
+ *
+ * Readings where the pages are garbled or silent (each listed in the design doc):
+ *  - The input term on the hot path is B_bar·x = Δ·B·x (the delta-scaled B of
+ *    [Johe] "SSM as RNN"), with the x that page's ssm_step drops restored.
+ *    The ZOH coefficient (exp(Δ·A) − 1)/A of [Guide] §1 is kept as a second
+ *    mode (bbar_mode = 1) for the discretization pins.
+ *  - A is used as given (negative for a stable scan); no epsilon or clamp is
+ *    added to Δ; D·x is added before the gate; silu is applied once.
+ *
+ * Layouts (row-major, last index fastest): x, delta, z, y [batch, L, D];
+ * B, C [batch, L, N]; A [D, N]; Dv, delta_bias [D]; states [batch, D, N].
+ * Null Dv / delta_bias / h0 mean zero; null z means no gate; null
+ * final_state means the final state is not returned.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+
+#define ORACLE_BBAR_DELTA 0 /* B_bar = Δ·B   ([Johe] "SSM as RNN")        */
+#define ORACLE_BBAR_ZOH 1   /* B_bar = (exp(Δ·A) − 1)/A·B ([Guide] §1)    */
+
+/* softplus(v) = log(1 + e^v), written so that neither branch overflows. */
+static double softplus(double v)
+{
+    return v > 0.0 ? v + log1p(exp(-v)) : log1p(exp(v));
+}
+
+/* silu(z) = z·sigmoid(z) ([Johe] "Mamba Block", y * silu(gate)). */
+static double silu(double z)
+{
+    return z / (1.0 + exp(-z));
+}
+
+/* Δ for one (token, channel): bias inside the softplus ([Guide] §4,
+ * [Johe] "Discretization"). */
+static double step_size(double delta, const double *delta_bias, int64_t d,
+                        int softplus_flag)
+{
+    double v = delta + (delta_bias ? delta_bias[d] : 0.0);
+    return softplus_flag ? softplus(v) : v;
+}
+
+/* Input coefficient multiplying B[n]·x: Δ, or the diagonal ZOH factor
+ * (exp(Δ·a) − 1)/a, whose a → 0 limit is Δ. */
+static double bbar_coeff(double dt, double a, int bbar_mode)
+{
+    if (bbar_mode == ORACLE_BBAR_ZOH)
+        return a == 0.0 ? dt : expm1(dt * a) / a;
+    return dt;
+}
+
+/*
+ * One token of one channel: the discrete recurrence of [Guide] §1/§4 with the
+ * selective (per-token) Δ, B, C. Updates h[0..N) in place and returns the
+ * gated output.
+ */
+static double token_update(double *h, double xv, double dt, const double *Arow,
+                           const double *Bt, const double *Ct, double dskip,
+                           const double *zv, int64_t N, int bbar_mode)
+{
+    double acc = 0.0;
+    for (int64_t n = 0; n < N; ++n) {
+        double a_bar = exp(dt * Arow[n]);
+        double b_bar = bbar_coeff(dt, Arow[n], bbar_mode) * Bt[n];
+        h[n] = a_bar * h[n] + b_bar * xv;
+        acc += Ct[n] * h[n]; /* y reads the state after the update */
+    }
+    double out = acc + dskip * xv;
+    if (zv)
+        out *= silu(*zv);
+    return out;
+}
+
+/*
+ * Selective scan over a whole sequence.
+ * h0 (nullable, [batch, D, N]) is the state before token 0 (zero if null).
+ */
+void oracle_selscan_fwd(const double *x, const double *delta, const double *A,
+                        const double *B, const double *C, const double *Dv,
+                        const double *z, const double *delta_bias,
+                        int softplus_flag, int bbar_mode, const double *h0,
+                        double *y, double *final_state, int64_t batch,
+                        int64_t L, int64_t D, int64_t N, int nthreads)
+{
+    if (nthreads < 1)
+        nthreads = 1;
+#pragma omp parallel for collapse(2) schedule(dynamic, 1) num_threads(nthreads)
+    for (int64_t b = 0; b < batch; ++b) {
+        for (int64_t d = 0; d < D; ++d) {
+            double *h = (double *)malloc((size_t)N * sizeof(double));
+            for (int64_t n = 0; n < N; ++n)
+                h[n] = h0 ? h0[(b * D + d) * N + n] : 0.0;
+            const double *Arow = A + d * N;
+            double dskip = Dv ? Dv[d] : 0.0;
+            for (int64_t t = 0; t < L; ++t) {
+                int64_t i = (b * L + t) * D + d;
+                int64_t j = (b * L + t) * N;
+                double dt = step_size(delta[i], delta_bias, d, softplus_flag);
+                y[i] = token_update(h, x[i], dt, Arow, B + j, C + j, dskip,
+                                    z ? z + i : NULL, N, bbar_mode);
+            }
+            if (final_state)
+                for (int64_t n = 0; n < N; ++n)
+                    final_state[(b * D + d) * N + n] = h[n];
+            free(h);
+        }
+    }
+}
+
+/*
+ * Single-token recurrent update used at inference: the same token step,
+ * applied in place to a carried state ([Johe] "SSM as Convolution":
+ * recurrent mode for inference; [Guide] §6: O(1) state instead of a cache).
+ * x, delta, z [batch, D]; B, C [batch, N]; state [batch, D, N]; y [batch, D].
+ */
+void oracle_state_update(double *state, const double *x, const double *delta,
+                         const double *A, const double *B, const double *C,
+                         const double *Dv, const double *z,
+                         const double *delta_bias, int softplus_flag,
+                         double *y, int64_t batch, int64_t D, int64_t N)
+{
+    for (int64_t b = 0; b < batch; ++b) {
+        for (int64_t d = 0; d < D; ++d) {
+            int64_t i = b * D + d;
+            double dt = step_size(delta[i], delta_bias, d, softplus_flag);
+            y[i] = token_update(state + i * N, x[i], dt, A + d * N, B + b * N,
+                                C + b * N, Dv ? Dv[d] : 0.0, z ? z + i : NULL, N,
+                                ORACLE_BBAR_DELTA);
+        }
+    }
+}
+
+/*
+ * The associative operator of [Guide] §4 "Parallel Associative Scan" for the
+ * affine maps h -> a·h + b. The page writes (a,b)⊕(a',b') = (a·a', a·b' + b),
+ * which composes correctly when the left operand is the LATER element; here
+ * the later element is named explicitly: the result applies `earlier` first,
+ * then `later`.
+ */
+void oracle_compose(double a_later, double b_later, double a_earlier,
+                    double b_earlier, double *a_out, double *b_out)
+{
+    *a_out = a_later * a_earlier;
+    *b_out = a_later * b_earlier + b_later;
+}
+
+/*
+ * Chunked form of the same scan ([Johe] "Hardware-Aware Scan": fixed-size
+ * blocks with the state carried between them; [Guide] §4 operator):
+ *   1. per chunk c, from a zero state: P_c[n] = product of A_bar over the
+ *      chunk, H_c[n] = the chunk's own final state;
+ *   2. carry: hin_0 = h0, hin_{c+1} = (P_c, H_c) ∘ hin_c;
+ *   3. rescan every chunk from hin_c to produce y.
+ * The final state is hin after the last chunk. Must equal oracle_selscan_fwd
+ * up to rounding order.
+ */
+void oracle_selscan_fwd_chunked(const double *x, const double *delta,
+                                const double *A, const double *B,
+                                const double *C, const double *Dv,
+                                const double *z, const double *delta_bias,
+                                int softplus_flag, int bbar_mode,
+                                const double *h0, double *y,
+                                double *final_state, int64_t batch, int64_t L,
+                                int64_t D, int64_t N, int64_t chunk,
+                                int nthreads)
+{
+    if (chunk < 1)
+        chunk = 1;
+    if (nthreads < 1)
+        nthreads = 1;
+    int64_t nchunks = (L + chunk - 1) / chunk;
+#pragma omp parallel for collapse(2) schedule(dynamic, 1) num_threads(nthreads)
+    for (int64_t b = 0; b < batch; ++b) {
+        for (int64_t d = 0; d < D; ++d) {
+            const double *Arow = A + d * N;
+            double dskip = Dv ? Dv[d] : 0.0;
+            double *P = (double *)malloc((size_t)(nchunks * N) * sizeof(double));
+            double *H = (double *)malloc((size_t)(nchunks * N) * sizeof(double));
+            double *hin = (double *)malloc((size_t)((nchunks + 1) * N) * sizeof(double));
+            /* 1. chunk aggregates from a zero state */
+            for (int64_t c = 0; c < nchunks; ++c) {
+                double *Pc = P + c * N, *Hc = H + c * N;
+                for (int64_t n = 0; n < N; ++n) {
+                    Pc[n] = 1.0;
+                    Hc[n] = 0.0;
+                }
+                int64_t t1 = (c + 1) * chunk < L ? (c + 1) * chunk : L;
+                for (int64_t t = c * chunk; t < t1; ++t) {
+                    int64_t i = (b * L + t) * D + d;
+                    int64_t j = (b * L + t) * N;
+                    double dt = step_size(delta[i], delta_bias, d, softplus_flag);
+                    for (int64_t n = 0; n < N; ++n) {
+                        double a_bar = exp(dt * Arow[n]);
+                        double b_bar = bbar_coeff(dt, Arow[n], bbar_mode) * B[j + n];
+                        /* (a_bar, b_bar·x) ∘ (P, H): this token comes later */
+                        oracle_compose(a_bar, b_bar * x[i], Pc[n], Hc[n],
+                                       &Pc[n], &Hc[n]);
+                    }
+                }
+            }
+            /* 2. carry across chunks */
+            for (int64_t n = 0; n < N; ++n)
+                hin[n] = h0 ? h0[(b * D + d) * N + n] : 0.0;
+            for (int64_t c = 0; c < nchunks; ++c) {
+                for (int64_t n = 0; n < N; ++n) {
+                    double a_unused;
+                    oracle_compose(P[c * N + n], H[c * N + n], 1.0,
+                                   hin[c * N + n], &a_unused,
+                                   &hin[(c + 1) * N + n]);
+                }
+            }
+            /* 3. rescan each chunk from its carried-in state (hin[c] is
+             *    consumed in place; hin[c + 1] was already read above) */
+            for (int64_t c = 0; c < nchunks; ++c) {
+                double *h = hin + c * N;
+                int64_t t1 = (c + 1) * chunk < L ? (c + 1) * chunk : L;
+                for (int64_t t = c * chunk; t < t1; ++t) {
+                    int64_t i = (b * L + t) * D + d;
+                    int64_t j = (b * L + t) * N;
+                    double dt = step_size(delta[i], delta_bias, d, softplus_flag);
+                    y[i] = token_update(h, x[i], dt, Arow, B + j, C + j, dskip,
+                                        z ? z + i : NULL, N, bbar_mode);
+                }
+            }
+            if (final_state)
+                for (int64_t n = 0; n < N; ++n)
+                    final_state[(b * D + d) * N + n] = hin[nchunks * N + n];
+            free(P);
+            free(H);
+            free(hin);
+        }
+    }
+}
+
+/*
+ * Diagonal ZOH input matrix for one step ([Guide] §1 "Discrétisation"):
+ * B_bar[n] = (exp(Δ·A[n]) − 1)/A[n] · B[n], the a → 0 limit being Δ·B[n].
+ * Also returns A_bar[n] = exp(Δ·A[n]).
+ */
+void oracle_zoh_discretize(double dt, const double *A, const double *B,
+                           double *A_bar, double *B_bar, int64_t N)
+{
+    for (int64_t n = 0; n < N; ++n) {
+        A_bar[n] = exp(dt * A[n]);
+        B_bar[n] = bbar_coeff(dt, A[n], ORACLE_BBAR_ZOH) * B[n];
+    }
+}

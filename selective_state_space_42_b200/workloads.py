@@ -1,0 +1,204 @@
+"""Seeded synthetic inputs for the selective scan.
+
+This module only draws random tensors with the shapes and distributions of
+Mamba-1 layers; it holds none of the scan's arithmetic. Both the CUDA path and
+the float64 oracle are fed from here, so the two see bit-identical values.
+
+Shapes: x, delta, z [batch, L, D] in the workload dtype; B, C [batch, L, N] in
+the workload dtype (one per token, shared by every channel); A [D, N] fp32;
+D (skip) and delta_bias [D] fp32; states [batch, D, N] fp32.
+
+Distributions (the pages fix d_state = 16 and give A's diagonal as −(n+1);
+"Mamba & State Space Models — Guide Complet" §2 HiPPO diagonal and §4
+A = −exp(A_log) with A_log = log(1..N)):
+  x, z, B, C ~ N(0, 1); delta ~ 0.5·N(0, 1); delta_bias[d] = log(expm1(U)) with
+  U ~ U[1e-3, 1e-1], so that softplus(delta_bias) = U; A[d, n] = −(n+1);
+  D = 1 (tiny workload) or 1 + 0.1·N(0, 1).
+"""
+from __future__ import annotations
+
+import dataclasses
+from typing import Dict, Optional, Sequence
+
+import torch
+
+DTYPES = {"f32": torch.float32, "bf16": torch.bfloat16}
+
+
+@dataclasses.dataclass(frozen=True)
+class ScanWorkload:
+    name: str
+    batch: int
+    seqlen: int
+    dim: int
+    dstate: int
+    dtype: str  # "f32" | "bf16"
+    gate: bool
+    seed: int
+    skip_ones: bool = False  # D = 1.0 instead of 1 + 0.1·N(0,1)
+    softplus: bool = True
+    final_state: bool = True
+
+    @property
+    def elements(self) -> int:
+        """Scan elements B·L·D·N."""
+        return self.batch * self.seqlen * self.dim * self.dstate
+
+    def algorithmic_bytes(self) -> int:
+        """Minimum HBM bytes a fused single pass must move: x, delta, z in and
+        y out per (b, l, d); B and C per (b, l); final state out; A, D and
+        delta_bias once."""
+        es = 4 if self.dtype == "f32" else 2
+        per_bld = (3 if self.gate else 2) * es + es
+        per_bl = 2 * self.dstate * es
+        fixed = self.dim * self.dstate * 4 + 2 * self.dim * 4
+        if self.final_state:
+            fixed += self.batch * self.dim * self.dstate * 4
+        return (self.batch * self.seqlen * self.dim * per_bld
+                + self.batch * self.seqlen * per_bl + fixed)
+
+    def scaled(self, **kw) -> "ScanWorkload":
+        return dataclasses.replace(self, **kw)
+
+
+@dataclasses.dataclass(frozen=True)
+class DecodeWorkload:
+    name: str
+    batch: int
+    dim: int
+    dstate: int
+    steps: int
+    dtype: str
+    gate: bool
+    seed: int
+
+    def algorithmic_bytes_per_step(self) -> int:
+        es = 4 if self.dtype == "f32" else 2
+        per_bd = (3 if self.gate else 2) * es + es + 2 * self.dstate * 4
+        return (self.batch * self.dim * per_bd
+                + self.batch * 2 * self.dstate * es
+                + self.dim * self.dstate * 4 + 2 * self.dim * 4)
+
+    @property
+    def elements_per_step(self) -> int:
+        return self.batch * self.dim * self.dstate
+
+
+WORKLOADS: Dict[str, ScanWorkload] = {
+    # tiny fp32 scan, no gate, D = 1
+    "tiny_f32": ScanWorkload("tiny_f32", 1, 256, 64, 16, "f32", gate=False,
+                             seed=0, skip_ones=True),
+    # Mamba-130M-shaped layer (d_model 768, expand 2)
+    "mamba130m_layer": ScanWorkload("mamba130m_layer", 8, 2048, 1536, 16,
+                                    "bf16", gate=True, seed=1),
+    # Mamba-2.8B-shaped layer (d_model 2560, expand 2)
+    "mamba2p8b_layer": ScanWorkload("mamba2p8b_layer", 4, 8192, 5120, 16,
+                                    "bf16", gate=True, seed=2),
+    # one 1M-token sequence
+    "long_1m": ScanWorkload("long_1m", 1, 1 << 20, 2048, 16, "bf16",
+                            gate=True, seed=3),
+}
+
+DECODE = DecodeWorkload("decode_b256", 256, 5120, 16, 1000, "bf16", gate=True,
+                        seed=4)
+
+
+def _gen(seed: int, device) -> torch.Generator:
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    return g
+
+
+def _randn(shape, g, device, scale=1.0) -> torch.Tensor:
+    t = torch.randn(shape, generator=g, device=device, dtype=torch.float32)
+    return t.mul_(scale) if scale != 1.0 else t
+
+
+def param_tensors(dim: int, dstate: int, g, device, skip_ones: bool):
+    """A, D (skip) and delta_bias for `dim` channels."""
+    A = -torch.arange(1, dstate + 1, dtype=torch.float32, device=device)
+    A = A.repeat(dim, 1).contiguous()
+    u = torch.rand(dim, generator=g, device=device, dtype=torch.float64)
+    u = 1e-3 + (1e-1 - 1e-3) * u
+    delta_bias = torch.log(torch.expm1(u)).to(torch.float32)
+    if skip_ones:
+        Dv = torch.ones(dim, dtype=torch.float32, device=device)
+    else:
+        Dv = _randn((dim,), g, device, 0.1).add_(1.0)
+    return A, Dv, delta_bias
+
+
+def make_scan_inputs(w: ScanWorkload, device="cpu") -> Dict[str, torch.Tensor]:
+    """All inputs of one selective-scan call, drawn in a fixed order from one
+    generator seeded with ``w.seed`` (generator on ``device``)."""
+    dt = DTYPES[w.dtype]
+    g = _gen(w.seed, device)
+    shp = (w.batch, w.seqlen, w.dim)
+    bshp = (w.batch, w.seqlen, w.dstate)
+    out = {}
+    out["x"] = _randn(shp, g, device).to(dt)
+    out["delta"] = _randn(shp, g, device, 0.5).to(dt)
+    out["z"] = _randn(shp, g, device).to(dt) if w.gate else None
+    out["B"] = _randn(bshp, g, device).to(dt)
+    out["C"] = _randn(bshp, g, device).to(dt)
+    out["A"], out["D"], out["delta_bias"] = param_tensors(
+        w.dim, w.dstate, g, device, w.skip_ones)
+    return out
+
+
+def make_decode_state(w: DecodeWorkload, device="cpu") -> torch.Tensor:
+    g = _gen(w.seed, device)
+    return _randn((w.batch, w.dim, w.dstate), g, device, 0.1)
+
+
+def make_decode_params(w: DecodeWorkload, device="cpu"):
+    g = _gen(w.seed + 7919, device)
+    return param_tensors(w.dim, w.dstate, g, device, skip_ones=False)
+
+
+def make_decode_step(w: DecodeWorkload, step: int,
+                     device="cpu") -> Dict[str, Optional[torch.Tensor]]:
+    """Per-token inputs of decode step ``step`` (seed w.seed + 1 + step)."""
+    dt = DTYPES[w.dtype]
+    g = _gen(w.seed + 1 + step, device)
+    shp = (w.batch, w.dim)
+    out = {}
+    out["x"] = _randn(shp, g, device).to(dt)
+    out["delta"] = _randn(shp, g, device, 0.5).to(dt)
+    out["z"] = _randn(shp, g, device).to(dt) if w.gate else None
+    out["B"] = _randn((w.batch, w.dstate), g, device).to(dt)
+    out["C"] = _randn((w.batch, w.dstate), g, device).to(dt)
+    return out
+
+
+def channel_subset(dim: int, stride: int = 64) -> Sequence[int]:
+    """Deterministic channel sample: first, second, last and every
+    ``stride``-th channel."""
+    s = set(range(0, dim, stride)) | {0, 1 % max(dim, 1), dim - 1}
+    return sorted(c for c in s if 0 <= c < dim)
+
+
+def ragged_shapes():
+    """Small shapes that span several tiles with ragged tails."""
+    return [
+        (1, 1, 1, 1), (1, 3, 5, 4), (2, 31, 33, 16), (1, 33, 130, 16),
+        (3, 257, 72, 8), (2, 255, 257, 16), (1, 600, 96, 1),
+    ]
+
+
+def nbytes(t: Optional[torch.Tensor]) -> int:
+    return 0 if t is None else t.numel() * t.element_size()
+
+
+def gib(x: float) -> float:
+    return x / float(1 << 30)
+
+
+def ceil_div(a: int, b: int) -> int:
+    return -(-a // b)
+
+
+__all__ = ["ScanWorkload", "DecodeWorkload", "WORKLOADS", "DECODE",
+           "make_scan_inputs", "make_decode_state", "make_decode_params",
+           "make_decode_step", "channel_subset", "ragged_shapes", "DTYPES",
+           "nbytes", "gib", "ceil_div"]
