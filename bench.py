@@ -1,0 +1,386 @@
+#!/usr/bin/env python
+"""Benchmark of the selective scan (libselscan) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl selscan|reference]
+
+One step = one selscan_fwd call over one batch of the Mamba-2.8B-shaped layer
+(batch 4, L 8192, d_inner 5120, d_state 16; bf16 x/delta/z/B/C, fp32 state,
+softplus and silu gate on, final state returned). Inputs are synthetic and
+seeded, and stay resident in HBM; at 1.35 GB per step they are ~10x the L2,
+so no L2 flush is needed between steps.
+
+Prints ONE JSON line (rank 0). Under torchrun each rank runs its own replica
+(independent batches: weak scaling, no collective on the data path); time is
+the max over ranks of the CUDA-event time of the K timed steps.
+
+--impl reference times the float64 CPU oracle (the only reference there is)
+on a bounded sample of the same workload, on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "selective-scan elems (B·L·D·N)/s"
+UNIT = "elems/s"
+WORKLOAD = "mamba2p8b_layer"
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["selscan", "reference"], default="selscan")
+    ap.add_argument("--workload", default=WORKLOAD)
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0,
+                    help="target duration of the oracle CPU-baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-clocks", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            j = json.load(f)
+        return float(j["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+# ---- clocks sampled during the timed region -----------------------------------
+class ClockSampler:
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,"
+              "clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.t0 = self.t1 = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self._reader = threading.Thread(target=self._read, daemon=True)
+        self._reader.start()
+        time.sleep(0.6)  # nvidia-smi start-up
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line.strip()))
+
+    def mark_start(self):
+        self.t0 = time.time()
+
+    def mark_end(self):
+        self.t1 = time.time()
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, mx, reasons, n = [], None, set(), 0
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown",
+                 "sw_power_cap"]
+        for ts, line in self.lines:
+            if self.t0 is None or ts < self.t0 or ts > self.t1 + 0.15:
+                continue
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 10:
+                continue
+            try:
+                sm.append(float(parts[2]))
+                mx = float(parts[3])
+            except ValueError:
+                continue
+            n += 1
+            for name, v in zip(names, parts[6:10]):
+                if v.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                    "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": n}
+
+
+# ---- CPU baseline: the float64 oracle on a bounded sample ------------------------
+def _oracle_args(inp, rows, nch):
+    """Host float64 copies of batch rows `rows` and channels 0..nch-1."""
+    import torch
+    sel = list(rows)
+    bl = lambda t: None if t is None else t[sel][:, :, :nch].to("cpu", torch.float64).numpy()  # noqa
+    ch = lambda t: t[:nch].to("cpu", torch.float64).numpy()  # noqa
+    return (bl(inp["x"]), bl(inp["delta"]), ch(inp["A"]),
+            inp["B"][sel].to("cpu", torch.float64).numpy(),
+            inp["C"][sel].to("cpu", torch.float64).numpy(), ch(inp["D"]),
+            bl(inp.get("z")), ch(inp["delta_bias"]))
+
+
+def _sample_channels(w, rate, seconds, cores, rows=1):
+    per_channel = rows * w.seqlen * w.dstate
+    n = int(rate * seconds / per_channel)
+    if n >= cores:
+        n = n // cores * cores
+    return max(1, min(w.dim, n))
+
+
+def oracle_cpu_baseline(inp, w, target_s):
+    """The oracle, as it stands, on batch row 0 and a channel subset sized to
+    take about target_s seconds of the host's cores. Returns the
+    cpu_baseline object (elements/s over the sample)."""
+    import oracle
+    orc = oracle.default()
+    cores = oracle.default_threads()
+    probe = max(cores, 8)
+    t = time.perf_counter()
+    orc.fwd(*_oracle_args(inp, (0,), probe), softplus=True, threads=cores)
+    rate = probe * w.seqlen * w.dstate / max(time.perf_counter() - t, 1e-9)
+    nch = _sample_channels(w, rate, target_s, cores)
+    args = _oracle_args(inp, (0,), nch)
+    t = time.perf_counter()
+    orc.fwd(*args, softplus=True, threads=cores)
+    dt = time.perf_counter() - t
+    el = nch * w.seqlen * w.dstate
+    return {"value": el / dt, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": (f"{w.name}: batch row 0, channels 0..{nch - 1} of {w.dim}, all "
+                       f"{w.seqlen} tokens, d_state {w.dstate}: {el:.3e} scan "
+                       f"elements in {dt:.2f} s (float64, OpenMP over channels)")}
+
+
+def run_reference(args):
+    """--impl reference: the oracle timed on the host cores; each step is a
+    bounded sample (batch row 0, a channel subset) of the workload."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import oracle
+    from selective_state_space_42_b200 import workloads as wl
+    w = wl.WORKLOADS[args.workload]
+    cores = oracle.default_threads()
+    sub = w.scaled(batch=1, dim=min(w.dim, 4 * max(cores, 8) * 8))
+    inp = wl.make_scan_inputs(sub, device="cpu")
+    orc = oracle.default()
+    per_step_s = min(args.cpu_seconds, 150.0 / max(args.steps + args.warmup, 1))
+    probe = max(cores, 8)
+    t = time.perf_counter()
+    orc.fwd(*_oracle_args(inp, (0,), probe), softplus=True, threads=cores)
+    rate = probe * w.seqlen * w.dstate / max(time.perf_counter() - t, 1e-9)
+    nch = min(_sample_channels(w, rate, per_step_s, cores), sub.dim)
+    a = _oracle_args(inp, (0,), nch)
+    times = []
+    for i in range(args.warmup + args.steps):
+        t = time.perf_counter()
+        orc.fwd(*a, softplus=True, threads=cores)
+        if i >= args.warmup:
+            times.append(time.perf_counter() - t)
+    total = sum(times)
+    elems = len(times) * nch * w.seqlen * w.dstate
+    value = elems / total
+    sample = (f"{w.name}: per step batch row 0, channels 0..{nch - 1}, all {w.seqlen} "
+              f"tokens, d_state {w.dstate}; float64 oracle, OpenMP over channels")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * total / max(len(times), 1), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_block(w, 1),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores,
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_block(w, world):
+    return {"workload": w.name, "batch_per_gpu": w.batch, "seqlen": w.seqlen,
+            "d_inner": w.dim, "d_state": w.dstate, "io_dtype": w.dtype,
+            "state_dtype": "f32", "gate": w.gate, "delta_softplus": w.softplus,
+            "final_state": w.final_state, "A": "-(n+1)",
+            "parallelism": f"replicas x{world}" if world > 1 else "single",
+            "l2": "no flush: inputs (1.35 GB/step) >> 126 MB L2"}
+
+
+# ---- the GPU arm ---------------------------------------------------------------
+def smi_id(torch, dev, local):
+    """nvidia-smi id of a torch device: its PCI bus id when torch exposes it."""
+    p = torch.cuda.get_device_properties(dev)
+    try:
+        return f"{p.pci_domain_id:08X}:{p.pci_bus_id:02X}:{p.pci_device_id:02X}.0"
+    except AttributeError:
+        return str(local)
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    import torch.distributed as dist
+
+    import selective_state_space_42_b200 as ss
+    from selective_state_space_42_b200 import workloads as wl
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", device_id=dev,
+                                timeout=datetime.timedelta(seconds=120))
+    ss.load_library()
+
+    w = wl.WORKLOADS[args.workload]
+    plan = ss.selscan_fwd_plan(w.batch, w.seqlen, w.dim, w.dstate)
+    inp = wl.make_scan_inputs(w.scaled(seed=w.seed + 1000 * rank), device=dev)
+    y = torch.empty_like(inp["x"])
+    fs = torch.empty(w.batch, w.dim, w.dstate, device=dev, dtype=torch.float32)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        ss.selscan_fwd(inp["x"], inp["delta"], inp["A"], inp["B"], inp["C"], inp["D"],
+                       inp["z"], inp["delta_bias"], softplus=True, y=y, final_state=fs,
+                       stream=stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier(device_ids=[local])
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize(dev)
+
+    sampler = None if args.no_clocks else ClockSampler(smi_id(torch, dev, local))
+    if sampler:
+        sampler.start()
+    barrier()
+    torch.cuda.synchronize(dev)
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    if sampler:
+        sampler.mark_start()
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    if sampler:
+        sampler.mark_end()
+    barrier()
+    ms = ev0.elapsed_time(ev1)
+    clocks = sampler.stop() if sampler else None
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+
+    # end to end through the public call: pinned host inputs -> device ->
+    # selscan_fwd -> y and final state back to pinned host memory, every step
+    names = ["x", "delta", "z", "B", "C"]
+    host = {k: inp[k].to("cpu").pin_memory() for k in names}
+    y_h = torch.empty(y.shape, dtype=y.dtype, pin_memory=True)
+    fs_h = torch.empty(fs.shape, dtype=fs.dtype, pin_memory=True)
+    dbuf = {k: torch.empty_like(inp[k]) for k in names}
+
+    def e2e_step():
+        for k in names:
+            dbuf[k].copy_(host[k], non_blocking=True)
+        ss.selscan_fwd(dbuf["x"], dbuf["delta"], inp["A"], dbuf["B"], dbuf["C"],
+                       inp["D"], dbuf["z"], inp["delta_bias"], softplus=True, y=y,
+                       final_state=fs, stream=stream)
+        y_h.copy_(y, non_blocking=True)
+        fs_h.copy_(fs, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    h2d = sum(host[k].numel() * host[k].element_size() for k in names)
+    d2h = y_h.numel() * y_h.element_size() + fs_h.numel() * fs_h.element_size()
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = oracle_cpu_baseline(inp, w, args.cpu_seconds)
+
+    if world > 1:
+        dist.barrier(device_ids=[local])
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    elems = w.elements * world * args.steps
+    value = elems / (ms / 1e3)
+    per_launch_s = ms / 1e3 / args.steps
+    alg_bytes = w.algorithmic_bytes()
+    achieved = alg_bytes / per_launch_s / 1e9
+    peak, peak_kind = peaks()
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic (seeded N(0,1) inputs, Mamba-2.8B layer shapes, no weights)",
+        "config": config_block(w, world),
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "peak_kind": peak_kind,
+                     "frac_of_8TBps": achieved / 8000.0,
+                     "algorithmic_bytes_per_launch": alg_bytes,
+                     "kernel": "scan_kernel<bf16, gate, scan>", "traffic": None},
+        "e2e": {"value": w.elements * world * args.e2e_steps / (e2e_ms / 1e3),
+                "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": e2e_ms / args.e2e_steps},
+        "gpu_launches": args.steps * plan["launches"],
+        "plan": plan,
+        "cpu_baseline": cpu,
+        "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,158 @@
+/*
+ * selscan.h -- C ABI of libselscan, the Mamba-1 selective scan for B200
+ * (sm_100a).
+ *
+ * The operation (pages: "Mamba & State Space Models — Guide Complet" §1
+ * "Discrétisation" and §4 "Implémentation du SSM sélectif (S6)";
+ * "Mamba и State Space Models: альтернатива Transformer", "SSM as RNN",
+ * "Discretization" and "Mamba Block"). For every batch row b, channel d and
+ * state index n, with h = 0 before the first token:
+ *
+ *     Δ_t      = softplus(delta[b,t,d] + delta_bias[d])   (or no softplus)
+ *     Abar_t   = exp(Δ_t · A[d,n])
+ *     h_t[n]   = Abar_t · h_{t-1}[n] + Δ_t · B[b,t,n] · x[b,t,d]
+ *     y[b,t,d] = (Σ_n C[b,t,n] · h_t[n] + D[d] · x[b,t,d]) · silu(z[b,t,d])
+ *
+ * Δ, B and C vary per token (the "selection"); A is diagonal per channel and
+ * fixed; the input term is Δ·B ("SSM as RNN" scales B by delta); y reads the
+ * state after the token's update; D·x is added before the gate.
+ *
+ * Conventions shared by every entry point:
+ *  - All tensor pointers are DEVICE pointers on the current CUDA device,
+ *    row-major and contiguous, last index fastest. The caller owns every
+ *    buffer; the library keeps no pointer after a call returns.
+ *  - `dtype` is the element type of x, delta, z, B, C and y. A, D,
+ *    delta_bias and all states are always float32. Arithmetic is float32.
+ *    bf16 results are rounded to nearest even.
+ *  - Pointers must be aligned to their element size; y must not overlap any
+ *    input.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *    default stream). The return value reports argument validation and
+ *    launch errors (cudaGetLastError after the launches), not completion.
+ *  - "required" pointers may be NULL only when their tensor has zero
+ *    elements.
+ *  - Return values: SELSCAN_OK (0) or one of the negative SELSCAN_ERR_*
+ *    codes; nothing is launched when validation fails.
+ */
+#ifndef SELSCAN_H_
+#define SELSCAN_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define SELSCAN_API __attribute__((visibility("default")))
+#else
+#define SELSCAN_API
+#endif
+
+/* Same type as cudaStream_t; spelled out so that this header needs no CUDA
+ * header. */
+typedef struct CUstream_st *selscan_stream_t;
+
+typedef enum {
+    SELSCAN_F32 = 0,  /* float32 x, delta, z, B, C, y */
+    SELSCAN_BF16 = 1  /* bfloat16 x, delta, z, B, C, y */
+} selscan_dtype_t;
+
+enum {
+    SELSCAN_OK = 0,
+    SELSCAN_ERR_NULL_ARG = -1,           /* a required pointer is NULL */
+    SELSCAN_ERR_BAD_DIM = -2,            /* a size is negative or too large */
+    SELSCAN_ERR_BAD_DTYPE = -3,          /* dtype is not a selscan_dtype_t */
+    SELSCAN_ERR_MISALIGNED = -4,         /* a pointer is not element-aligned */
+    SELSCAN_ERR_DSTATE_UNSUPPORTED = -5, /* dstate outside 1..16 */
+    SELSCAN_ERR_CUDA = -6,               /* a CUDA call failed */
+    SELSCAN_ERR_ALIAS = -7               /* y overlaps an input */
+};
+
+#define SELSCAN_MAX_DSTATE 16
+
+/*
+ * selscan_fwd -- selective scan over whole sequences (the forward pass).
+ *
+ *   x, delta      [batch, seqlen, dim]      dtype        required
+ *   A             [dim, dstate]             float32      required
+ *   B, C          [batch, seqlen, dstate]   dtype        required; shared by
+ *                                                        all channels
+ *   D             [dim]                     float32      NULL -> no skip term
+ *   z             [batch, seqlen, dim]      dtype        NULL -> no gate
+ *   delta_bias    [dim]                     float32      NULL -> zero bias
+ *   softplus_flag nonzero -> Δ = softplus(delta + bias), zero -> Δ = delta + bias
+ *   y             [batch, seqlen, dim]      dtype        required output
+ *   final_state   [batch, dim, dstate]      float32      NULL -> not written;
+ *                                                        else h after the
+ *                                                        last token (zeros if
+ *                                                        seqlen == 0)
+ *   batch, seqlen, dim >= 0 (any of them 0 -> nothing to compute);
+ *   1 <= dstate <= SELSCAN_MAX_DSTATE.
+ *
+ * Long sequences with few channels are split into chunks scanned in
+ * parallel, then joined by carrying each chunk's final state (the pages'
+ * blockwise scan with its state carried across blocks, "Hardware-Aware
+ * Scan", and the associative operator of Guide Complet §4 "Parallel
+ * Associative Scan"). That plan takes a stream-ordered device workspace
+ * (cudaMallocAsync / cudaFreeAsync on `stream`) of
+ * 2 · batch · chunks · dim · 16 floats (states padded to 16); no other memory
+ * is allocated.
+ */
+SELSCAN_API int selscan_fwd(const void *x, const void *delta, const float *A,
+                const void *B, const void *C, const float *D, const void *z,
+                const float *delta_bias, int softplus_flag, void *y,
+                float *final_state, int64_t batch, int64_t seqlen, int64_t dim,
+                int64_t dstate, selscan_dtype_t dtype, selscan_stream_t stream);
+
+/*
+ * selscan_fwd_plan -- the launch plan selscan_fwd would use for these sizes
+ * (host only; no CUDA work). Writes, through each non-NULL pointer, the
+ * number of sequence chunks (0 when there is nothing to compute), the number
+ * of kernel launches (1 single pass; 3 chunked: chunk aggregates, carry,
+ * rescan) and the bytes of stream-ordered workspace that call allocates.
+ * Returns SELSCAN_OK or the size errors of selscan_fwd. The plan depends on
+ * the current device's SM count.
+ */
+SELSCAN_API int selscan_fwd_plan(int64_t batch, int64_t seqlen, int64_t dim,
+                                 int64_t dstate, int64_t *chunks, int64_t *launches,
+                                 int64_t *workspace_bytes);
+
+/*
+ * selscan_state_update -- one token of recurrent inference, in place
+ * ("SSM as Convolution": recurrent mode for inference; Guide Complet §6: a
+ * constant-size state instead of a growing cache).
+ *
+ *   state         [batch, dim, dstate]      float32      required, read and
+ *                                                        overwritten with h_t
+ *   x, delta      [batch, dim]              dtype        required
+ *   A             [dim, dstate]             float32      required
+ *   B, C          [batch, dstate]           dtype        required
+ *   D             [dim]                     float32      NULL -> no skip term
+ *   z             [batch, dim]              dtype        NULL -> no gate
+ *   delta_bias    [dim]                     float32      NULL -> zero bias
+ *   softplus_flag as for selscan_fwd
+ *   y             [batch, dim]              dtype        required output
+ *
+ * A final_state from selscan_fwd is a valid `state`: steps continue the
+ * sequence exactly where the scan stopped. No memory is allocated.
+ */
+SELSCAN_API int selscan_state_update(float *state, const void *x, const void *delta,
+                         const float *A, const void *B, const void *C,
+                         const float *D, const void *z,
+                         const float *delta_bias, int softplus_flag, void *y,
+                         int64_t batch, int64_t dim, int64_t dstate,
+                         selscan_dtype_t dtype, selscan_stream_t stream);
+
+/* Static, NUL-terminated description of a status code (never NULL). */
+SELSCAN_API const char *selscan_status_string(int status);
+
+/* Text of the CUDA error behind the calling thread's last SELSCAN_ERR_CUDA
+ * (static storage; "no error" if none). */
+SELSCAN_API const char *selscan_last_cuda_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SELSCAN_H_ */

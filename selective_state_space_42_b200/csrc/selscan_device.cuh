@@ -1,0 +1,100 @@
+// selscan_device.cuh -- device-side helpers shared by the libselscan kernels:
+// element loads/stores for the two I/O dtypes, the MUFU wrappers, softplus
+// and silu in float32, and the launch-parameter structs.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace selscan {
+
+constexpr int kMaxN = 16;           // largest supported d_state
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+// ---- element I/O -------------------------------------------------------------
+__device__ __forceinline__ float to_f32(float v) { return v; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 v) { return __bfloat162float(v); }
+
+template <typename T> __device__ __forceinline__ T from_f32(float v);
+template <> __device__ __forceinline__ float from_f32<float>(float v) { return v; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float v) {
+    return __float2bfloat16_rn(v);  // round to nearest even
+}
+
+template <typename T>
+__device__ __forceinline__ float ldg_f32(const T *p) { return to_f32(__ldg(p)); }
+
+// ---- special-function unit (MUFU) instructions ----------------------------------
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float lg2_approx(float x) {
+    float y;
+    asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float rcp_approx(float x) {
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// softplus(v) = max(v, 0) + log1p(w), w = exp(-|v|) in (0, 1].
+// log1p(w): for w < 1/16 the alternating series w − w²/2 + … + w⁷/7 (truncation
+// below w⁸/8 < 1e-10 relative); otherwise log2(1 + w)·ln 2, where 1 + w ≥ 1.0625
+// keeps lg2's absolute error small relative to the result. Both branches are
+// evaluated and one is selected, so warps never diverge here.
+__device__ __forceinline__ float softplus_f32(float v) {
+    const float w = ex2_approx(-fabsf(v) * kLog2e);
+    float s = fmaf(w, -1.0f / 7.0f, 1.0f / 6.0f);
+    s = fmaf(w, -s, 1.0f / 5.0f);
+    s = fmaf(w, -s, 1.0f / 4.0f);
+    s = fmaf(w, -s, 1.0f / 3.0f);
+    s = fmaf(w, -s, 1.0f / 2.0f);
+    s = fmaf(w, -s, 1.0f);
+    const float series = w * s;
+    const float viaLog = lg2_approx(1.0f + w) * kLn2;
+    return fmaxf(v, 0.0f) + (w < 0.0625f ? series : viaLog);
+}
+
+// silu(z) = z · sigmoid(z) = z / (1 + e^-z); e^-z overflowing to +inf gives 0.
+__device__ __forceinline__ float silu_f32(float z) {
+    return z * rcp_approx(1.0f + ex2_approx(-z * kLog2e));
+}
+
+// ---- launch parameters -------------------------------------------------------------
+struct ScanParams {
+    const void *x, *delta, *z, *B, *C;
+    const float *A, *Dskip, *delta_bias;
+    void *y;
+    float *final_state;
+    int64_t batch, seqlen, dim;
+    int dstate;
+    int softplus;
+    int64_t chunk_len;   // tokens per chunk (== seqlen when not chunked)
+    int nchunks;         // chunks per sequence
+    int ntiles;          // channel tiles per batch row
+    // chunk workspace, [batch][nchunks][dim][kMaxN] each (NULL if nchunks == 1):
+    float *ws_P;         // pass 1: product of Abar over the chunk
+    float *ws_H;         // pass 1: chunk state from zero; after carry: state entering the chunk
+};
+
+struct StepParams {
+    float *state;
+    const void *x, *delta, *z, *B, *C;
+    const float *A, *Dskip, *delta_bias;
+    void *y;
+    int64_t batch, dim;
+    int dstate;
+    int softplus;
+};
+
+// Host-side launchers (one translation unit per kernel family).
+cudaError_t launch_scan(const ScanParams &p, bool bf16, cudaStream_t stream);
+cudaError_t launch_state_update(const StepParams &p, bool bf16, cudaStream_t stream);
+
+}  // namespace selscan

@@ -1,0 +1,219 @@
+"""Python binding of libselscan (include/selscan.h): argument marshalling only.
+
+Every function here checks that the tensors it is handed are what the C ABI
+expects (device, dtype, contiguity, shape) and passes raw pointers, sizes and
+the current CUDA stream to the library. All computation runs in the CUDA
+kernels behind the ABI. If the shared library is missing, every call raises
+(``SelscanUnavailable``); there is no fallback implementation.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libselscan.so")
+
+SELSCAN_F32 = 0
+SELSCAN_BF16 = 1
+SELSCAN_MAX_DSTATE = 16
+
+STATUS = {
+    0: "SELSCAN_OK", -1: "SELSCAN_ERR_NULL_ARG", -2: "SELSCAN_ERR_BAD_DIM",
+    -3: "SELSCAN_ERR_BAD_DTYPE", -4: "SELSCAN_ERR_MISALIGNED",
+    -5: "SELSCAN_ERR_DSTATE_UNSUPPORTED", -6: "SELSCAN_ERR_CUDA",
+    -7: "SELSCAN_ERR_ALIAS",
+}
+
+_vp = ctypes.c_void_p
+_i64 = ctypes.c_int64
+_int = ctypes.c_int
+
+# name -> (restype, argtypes), mirroring include/selscan.h
+SIGNATURES = {
+    "selscan_fwd": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _int, _vp, _vp,
+                           _i64, _i64, _i64, _i64, _int, _vp]),
+    "selscan_state_update": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                    _int, _vp, _i64, _i64, _i64, _int, _vp]),
+    "selscan_fwd_plan": (_int, [_i64, _i64, _i64, _i64, ctypes.POINTER(_i64),
+                                ctypes.POINTER(_i64), ctypes.POINTER(_i64)]),
+    "selscan_status_string": (ctypes.c_char_p, [_int]),
+    "selscan_last_cuda_error": (ctypes.c_char_p, []),
+}
+
+
+class SelscanUnavailable(RuntimeError):
+    """libselscan.so is not built or cannot be loaded."""
+
+
+class SelscanError(RuntimeError):
+    def __init__(self, status: int, detail: str = ""):
+        self.status = status
+        msg = f"{STATUS.get(status, status)}: {detail}"
+        super().__init__(msg)
+
+
+_lib: Optional[ctypes.CDLL] = None
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load (once) and type the shared library; raises if it is missing."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise SelscanUnavailable(
+            f"{path} is missing: build it with `python -m "
+            f"selective_state_space_42_b200.build` (nvcc, sm_100a)")
+    try:
+        lib = ctypes.CDLL(path)
+    except OSError as e:  # pragma: no cover
+        raise SelscanUnavailable(f"cannot load {path}: {e}") from e
+    for name, (res, args) in SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = lib
+    return lib
+
+
+def selscan_status_string(status: int) -> str:
+    return load_library().selscan_status_string(int(status)).decode()
+
+
+def selscan_last_cuda_error() -> str:
+    return load_library().selscan_last_cuda_error().decode()
+
+
+def _check(status: int):
+    if status != 0:
+        detail = selscan_status_string(status)
+        if status == -6:
+            detail += f" ({selscan_last_cuda_error()})"
+        raise SelscanError(status, detail)
+
+
+# ---- tensor marshalling ----------------------------------------------------------
+def _torch():
+    import torch
+    return torch
+
+
+def _dtype_code(t) -> int:
+    torch = _torch()
+    if t.dtype == torch.float32:
+        return SELSCAN_F32
+    if t.dtype == torch.bfloat16:
+        return SELSCAN_BF16
+    raise TypeError(f"unsupported dtype {t.dtype} (float32 or bfloat16)")
+
+
+def _ptr(t, name, shape=None, dtype=None, device=None, required=True):
+    if t is None:
+        if required:
+            raise ValueError(f"{name} is required")
+        return None
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    return t.data_ptr()
+
+
+def _stream_ptr(stream, device):
+    torch = _torch()
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def selscan_fwd_plan(batch: int, seqlen: int, dim: int, dstate: int) -> dict:
+    """Launch plan of selscan_fwd for these sizes (C ABI ``selscan_fwd_plan``):
+    {"chunks", "launches", "workspace_bytes"}."""
+    c, n, w = _i64(), _i64(), _i64()
+    _check(load_library().selscan_fwd_plan(batch, seqlen, dim, dstate, ctypes.byref(c),
+                                           ctypes.byref(n), ctypes.byref(w)))
+    return {"chunks": c.value, "launches": n.value, "workspace_bytes": w.value}
+
+
+def selscan_fwd(x, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=True,
+                y=None, final_state=None, return_final_state=False, stream=None):
+    """Selective scan over whole sequences (C ABI ``selscan_fwd``).
+
+    x, delta, z: [batch, L, dim]; B, C: [batch, L, dstate] (same dtype as x,
+    float32 or bfloat16); A: [dim, dstate] float32; D, delta_bias: [dim]
+    float32. Returns y (allocated if not given) or (y, final_state)."""
+    torch = _torch()
+    if x.dim() != 3:
+        raise ValueError("x must be [batch, L, dim]")
+    batch, L, dim = x.shape
+    if A.dim() != 2 or A.shape[0] != dim:
+        raise ValueError("A must be [dim, dstate]")
+    N = A.shape[1]
+    dev, dt = x.device, x.dtype
+    code = _dtype_code(x)
+    if y is None:
+        y = torch.empty_like(x)
+    if final_state is None and return_final_state:
+        final_state = torch.empty(batch, dim, N, device=dev, dtype=torch.float32)
+    f32 = torch.float32
+    args = [
+        _ptr(x, "x", (batch, L, dim), dt, dev),
+        _ptr(delta, "delta", (batch, L, dim), dt, dev),
+        _ptr(A, "A", (dim, N), f32, dev),
+        _ptr(B, "B", (batch, L, N), dt, dev),
+        _ptr(C, "C", (batch, L, N), dt, dev),
+        _ptr(D, "D", (dim,), f32, dev, required=False),
+        _ptr(z, "z", (batch, L, dim), dt, dev, required=False),
+        _ptr(delta_bias, "delta_bias", (dim,), f32, dev, required=False),
+        int(bool(softplus)),
+        _ptr(y, "y", (batch, L, dim), dt, dev),
+        _ptr(final_state, "final_state", (batch, dim, N), f32, dev, required=False),
+        batch, L, dim, N, code, _stream_ptr(stream, dev),
+    ]
+    _check(load_library().selscan_fwd(*args))
+    if return_final_state:
+        return y, final_state
+    return y
+
+
+def selscan_state_update(state, x, delta, A, B, C, D=None, z=None, delta_bias=None,
+                         softplus=True, y=None, stream=None):
+    """One recurrent step in place on ``state`` (C ABI ``selscan_state_update``).
+
+    state: [batch, dim, dstate] float32 (updated); x, delta, z: [batch, dim];
+    B, C: [batch, dstate]. Returns y [batch, dim]."""
+    torch = _torch()
+    if state.dim() != 3:
+        raise ValueError("state must be [batch, dim, dstate]")
+    batch, dim, N = state.shape
+    dev, dt = x.device, x.dtype
+    code = _dtype_code(x)
+    if y is None:
+        y = torch.empty_like(x)
+    f32 = torch.float32
+    args = [
+        _ptr(state, "state", (batch, dim, N), f32, dev),
+        _ptr(x, "x", (batch, dim), dt, dev),
+        _ptr(delta, "delta", (batch, dim), dt, dev),
+        _ptr(A, "A", (dim, N), f32, dev),
+        _ptr(B, "B", (batch, N), dt, dev),
+        _ptr(C, "C", (batch, N), dt, dev),
+        _ptr(D, "D", (dim,), f32, dev, required=False),
+        _ptr(z, "z", (batch, dim), dt, dev, required=False),
+        _ptr(delta_bias, "delta_bias", (dim,), f32, dev, required=False),
+        int(bool(softplus)),
+        _ptr(y, "y", (batch, dim), dt, dev),
+        batch, dim, N, code, _stream_ptr(stream, dev),
+    ]
+    _check(load_library().selscan_state_update(*args))
+    return y

@@ -1,0 +1,123 @@
+"""The C ABI without a GPU: the library loads, exports every function that
+include/*.h declares, and its host-side validation returns the documented
+status codes before any CUDA call (CPU only; no kernel is launched)."""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+import selective_state_space_42_b200 as ss
+from selective_state_space_42_b200 import build as ssbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    ssbuild.build()
+    return ss.load_library()
+
+
+def declared_functions():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = open(h).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", "", text)
+        names |= set(re.findall(r"\b(selscan_\w+)\s*\(", text))
+    return sorted(names)
+
+
+def test_header_declares_entry_points():
+    names = declared_functions()
+    for n in ("selscan_fwd", "selscan_state_update", "selscan_status_string"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert names
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in include/ but not exported"
+        assert n in ss.selscan.SIGNATURES, f"{n} has no binding signature"
+
+
+def test_only_declared_symbols_are_exported(lib):
+    out = os.popen(f"nm -D --defined-only {ss.LIB_PATH}").read()
+    exported = set(re.findall(r"\b(selscan_\w+)\b", out))
+    assert exported == set(declared_functions())
+
+
+def test_status_strings(lib):
+    for code in [0, -1, -2, -3, -4, -5, -6, -7]:
+        s = ss.selscan_status_string(code)
+        assert s and s != "unknown status"
+    assert ss.selscan_status_string(12345) == "unknown status"
+
+
+P = 1 << 20  # a fake, aligned, non-null device address (never dereferenced)
+
+
+def fwd(lib, **kw):
+    a = dict(x=P, delta=P + 4096, A=P + 8192, B=P + 12288, C=P + 16384, D=None,
+             z=None, delta_bias=None, softplus=1, y=P + 65536, final_state=None,
+             batch=0, seqlen=8, dim=4, dstate=16, dtype=1, stream=None)
+    a.update(kw)
+    return lib.selscan_fwd(a["x"], a["delta"], a["A"], a["B"], a["C"], a["D"], a["z"],
+                           a["delta_bias"], a["softplus"], a["y"], a["final_state"],
+                           a["batch"], a["seqlen"], a["dim"], a["dstate"], a["dtype"],
+                           a["stream"])
+
+
+def step(lib, **kw):
+    a = dict(state=P + 131072, x=P, delta=P + 4096, A=P + 8192, B=P + 12288,
+             C=P + 16384, D=None, z=None, delta_bias=None, softplus=1, y=P + 65536,
+             batch=0, dim=4, dstate=16, dtype=1, stream=None)
+    a.update(kw)
+    return lib.selscan_state_update(a["state"], a["x"], a["delta"], a["A"], a["B"],
+                                    a["C"], a["D"], a["z"], a["delta_bias"],
+                                    a["softplus"], a["y"], a["batch"], a["dim"],
+                                    a["dstate"], a["dtype"], a["stream"])
+
+
+def test_fwd_validation(lib):
+    assert fwd(lib) == 0  # batch = 0: nothing to do, no CUDA call
+    assert fwd(lib, batch=2, dim=0) == 0
+    assert fwd(lib, batch=2, seqlen=0) == 0  # no final_state to clear
+    assert fwd(lib, x=None) == 0  # empty tensors may be NULL
+    assert fwd(lib, batch=1, x=None) == -1
+    assert fwd(lib, batch=1, y=None) == -1
+    assert fwd(lib, batch=1, B=None) == -1
+    assert fwd(lib, batch=1, A=None) == -1
+    assert fwd(lib, dtype=7) == -3
+    assert fwd(lib, batch=-1) == -2
+    assert fwd(lib, seqlen=-5) == -2
+    assert fwd(lib, batch=1 << 30, seqlen=1 << 30, dim=1 << 30) == -2
+    assert fwd(lib, dstate=0) == -5
+    assert fwd(lib, dstate=17) == -5
+    assert fwd(lib, x=P + 1) == -4  # bf16 needs 2-byte alignment
+    assert fwd(lib, x=P + 2, dtype=0) == -4  # fp32 needs 4-byte alignment
+    assert fwd(lib, A=P + 2) == -4
+    assert fwd(lib, batch=1, y=P) == -7  # y == x
+    assert fwd(lib, batch=1, y=P + 12288 - 2) == -7  # y runs into B
+
+
+def test_state_update_validation(lib):
+    assert step(lib) == 0
+    assert step(lib, state=None) == 0  # batch = 0: empty
+    assert step(lib, batch=1, state=None) == -1
+    assert step(lib, dtype=-1) == -3
+    assert step(lib, dim=-1) == -2
+    assert step(lib, dstate=20) == -5
+    assert step(lib, state=P + 2) == -4
+    assert step(lib, batch=1, y=P + 131072) == -7  # y overlaps the state
+
+
+def test_binding_rejects_cpu_tensors(lib):
+    torch = pytest.importorskip("torch")
+    x = torch.zeros(1, 4, 8)
+    with pytest.raises(ValueError):
+        ss.selscan_fwd(x, x, torch.zeros(8, 16), torch.zeros(1, 4, 16),
+                       torch.zeros(1, 4, 16))
