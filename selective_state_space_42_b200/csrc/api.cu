@@ -9,19 +9,9 @@
 #include "selscan.h"
 #include "selscan_device.cuh"
 
-namespace selscan {
-int scan_channels_per_cta();
-int scan_tile_tokens();
-}
-
 namespace {
 
 thread_local cudaError_t g_last_cuda_error = cudaSuccess;
-
-int cuda_fail(cudaError_t e) {
-    g_last_cuda_error = e;
-    return SELSCAN_ERR_CUDA;
-}
 
 bool misaligned(const void *p, size_t a) {
     return p != nullptr && (reinterpret_cast<uintptr_t>(p) % a) != 0;
@@ -99,6 +89,79 @@ size_t workspace_bytes(int64_t batch, int64_t dim, int nchunks) {
 
 }  // namespace
 
+namespace selscan {
+
+int cuda_fail(cudaError_t e) {
+    g_last_cuda_error = e;
+    return SELSCAN_ERR_CUDA;
+}
+
+// Argument validation and launch plan shared by the selscan_fwd entry points.
+// On SELSCAN_OK fills *p (workspace pointers left NULL) and *ws_bytes, the
+// chunk workspace the plan needs; *done is set when no kernel has to run
+// (empty sizes; for seqlen == 0 the final state has been cleared on stream).
+int fwd_setup(const void *x, const void *delta, const float *A, const void *B,
+              const void *C, const float *D, const void *z, const float *delta_bias,
+              int softplus_flag, void *y, float *final_state, int64_t batch,
+              int64_t seqlen, int64_t dim, int64_t dstate, int dtype,
+              cudaStream_t stream, ScanParams *p, size_t *ws_bytes, bool *done) {
+    *done = false;
+    *ws_bytes = 0;
+    if (dtype != SELSCAN_F32 && dtype != SELSCAN_BF16) return SELSCAN_ERR_BAD_DTYPE;
+    if (batch < 0 || seqlen < 0 || dim < 0) return SELSCAN_ERR_BAD_DIM;
+    if (dstate < 1 || dstate > SELSCAN_MAX_DSTATE) return SELSCAN_ERR_DSTATE_UNSUPPORTED;
+    if (!mul_le(batch, seqlen, kMaxElems) || !mul_le(batch * seqlen, dim, kMaxElems) ||
+        !mul_le(batch, dim, kMaxElems))
+        return SELSCAN_ERR_BAD_DIM;
+    // A tensor with zero elements may be passed as NULL.
+    const bool has_tokens = batch * seqlen * dim > 0;
+    if (has_tokens && (!x || !delta || !y || !B || !C)) return SELSCAN_ERR_NULL_ARG;
+    if (dim > 0 && !A) return SELSCAN_ERR_NULL_ARG;
+    const size_t es = dtype == SELSCAN_F32 ? 4 : 2;
+    if (misaligned(x, es) || misaligned(delta, es) || misaligned(z, es) ||
+        misaligned(B, es) || misaligned(C, es) || misaligned(y, es) ||
+        misaligned(A, 4) || misaligned(D, 4) || misaligned(delta_bias, 4) ||
+        misaligned(final_state, 4))
+        return SELSCAN_ERR_MISALIGNED;
+    const size_t nx = (size_t)(batch * seqlen * dim) * es;
+    const size_t nbc = (size_t)(batch * seqlen * dstate) * es;
+    if (overlaps(y, nx, x, nx) || overlaps(y, nx, delta, nx) || overlaps(y, nx, z, nx) ||
+        overlaps(y, nx, B, nbc) || overlaps(y, nx, C, nbc))
+        return SELSCAN_ERR_ALIAS;
+
+    if (batch == 0 || dim == 0) {
+        *done = true;
+        return SELSCAN_OK;
+    }
+    if (seqlen == 0) {
+        *done = true;
+        if (final_state) {
+            cudaError_t e = cudaMemsetAsync(final_state, 0,
+                                            (size_t)(batch * dim * dstate) * sizeof(float),
+                                            stream);
+            if (e != cudaSuccess) return cuda_fail(e);
+        }
+        return SELSCAN_OK;
+    }
+
+    p->x = x; p->delta = delta; p->z = z; p->B = B; p->C = C;
+    p->A = A; p->Dskip = D; p->delta_bias = delta_bias;
+    p->y = y; p->final_state = final_state;
+    p->batch = batch; p->seqlen = seqlen; p->dim = dim; p->dstate = (int)dstate;
+    p->softplus = softplus_flag ? 1 : 0;
+    const int64_t cpc = scan_channels_per_cta();
+    p->ntiles = (int)((dim + cpc - 1) / cpc);
+    const Plan plan = plan_fwd(batch, seqlen, dim);
+    p->chunk_len = plan.chunk_len;
+    p->nchunks = plan.nchunks;
+    p->ws_P = p->ws_H = nullptr;
+    if (!mul_le(batch * plan.nchunks, p->ntiles, INT32_MAX)) return SELSCAN_ERR_BAD_DIM;
+    *ws_bytes = workspace_bytes(batch, dim, plan.nchunks);
+    return SELSCAN_OK;
+}
+
+}  // namespace selscan
+
 extern "C" {
 
 const char *selscan_status_string(int status) {
@@ -126,66 +189,26 @@ int selscan_fwd(const void *x, const void *delta, const float *A, const void *B,
                 int64_t seqlen, int64_t dim, int64_t dstate, selscan_dtype_t dtype,
                 selscan_stream_t stream_) {
     cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
-    if (dtype != SELSCAN_F32 && dtype != SELSCAN_BF16) return SELSCAN_ERR_BAD_DTYPE;
-    if (batch < 0 || seqlen < 0 || dim < 0) return SELSCAN_ERR_BAD_DIM;
-    if (dstate < 1 || dstate > SELSCAN_MAX_DSTATE) return SELSCAN_ERR_DSTATE_UNSUPPORTED;
-    if (!mul_le(batch, seqlen, kMaxElems) || !mul_le(batch * seqlen, dim, kMaxElems) ||
-        !mul_le(batch, dim, kMaxElems))
-        return SELSCAN_ERR_BAD_DIM;
-    // A tensor with zero elements may be passed as NULL.
-    const bool has_tokens = batch * seqlen * dim > 0;
-    if (has_tokens && (!x || !delta || !y || !B || !C)) return SELSCAN_ERR_NULL_ARG;
-    if (dim > 0 && !A) return SELSCAN_ERR_NULL_ARG;
-    const size_t es = dtype == SELSCAN_F32 ? 4 : 2;
-    if (misaligned(x, es) || misaligned(delta, es) || misaligned(z, es) ||
-        misaligned(B, es) || misaligned(C, es) || misaligned(y, es) ||
-        misaligned(A, 4) || misaligned(D, 4) || misaligned(delta_bias, 4) ||
-        misaligned(final_state, 4))
-        return SELSCAN_ERR_MISALIGNED;
-    const size_t nx = (size_t)(batch * seqlen * dim) * es;
-    const size_t nbc = (size_t)(batch * seqlen * dstate) * es;
-    if (overlaps(y, nx, x, nx) || overlaps(y, nx, delta, nx) || overlaps(y, nx, z, nx) ||
-        overlaps(y, nx, B, nbc) || overlaps(y, nx, C, nbc))
-        return SELSCAN_ERR_ALIAS;
-
-    if (batch == 0 || dim == 0) return SELSCAN_OK;
-    if (seqlen == 0) {
-        if (final_state) {
-            cudaError_t e = cudaMemsetAsync(final_state, 0,
-                                            (size_t)(batch * dim * dstate) * sizeof(float),
-                                            stream);
-            if (e != cudaSuccess) return cuda_fail(e);
-        }
-        return SELSCAN_OK;
-    }
-
     selscan::ScanParams p{};
-    p.x = x; p.delta = delta; p.z = z; p.B = B; p.C = C;
-    p.A = A; p.Dskip = D; p.delta_bias = delta_bias;
-    p.y = y; p.final_state = final_state;
-    p.batch = batch; p.seqlen = seqlen; p.dim = dim; p.dstate = (int)dstate;
-    p.softplus = softplus_flag ? 1 : 0;
-    const int64_t cpc = selscan::scan_channels_per_cta();
-    p.ntiles = (int)((dim + cpc - 1) / cpc);
-    const Plan plan = plan_fwd(batch, seqlen, dim);
-    p.chunk_len = plan.chunk_len;
-    p.nchunks = plan.nchunks;
-    if (!mul_le(batch * plan.nchunks, p.ntiles, INT32_MAX)) return SELSCAN_ERR_BAD_DIM;
-
+    size_t ws_bytes = 0;
+    bool done = false;
+    const int st = selscan::fwd_setup(x, delta, A, B, C, D, z, delta_bias, softplus_flag,
+                                      y, final_state, batch, seqlen, dim, dstate, dtype,
+                                      stream, &p, &ws_bytes, &done);
+    if (st != SELSCAN_OK || done) return st;
     void *ws = nullptr;
-    if (plan.nchunks > 1) {
-        const size_t bytes = workspace_bytes(batch, dim, plan.nchunks);
-        cudaError_t e = cudaMallocAsync(&ws, bytes, stream);
-        if (e != cudaSuccess) return cuda_fail(e);
+    if (ws_bytes > 0) {
+        cudaError_t e = cudaMallocAsync(&ws, ws_bytes, stream);
+        if (e != cudaSuccess) return selscan::cuda_fail(e);
         p.ws_P = static_cast<float *>(ws);
-        p.ws_H = reinterpret_cast<float *>(static_cast<char *>(ws) + bytes / 2);
+        p.ws_H = reinterpret_cast<float *>(static_cast<char *>(ws) + ws_bytes / 2);
     }
     cudaError_t e = selscan::launch_scan(p, dtype == SELSCAN_BF16, stream);
     if (ws) {
         cudaError_t ef = cudaFreeAsync(ws, stream);
         if (e == cudaSuccess) e = ef;
     }
-    return e == cudaSuccess ? SELSCAN_OK : cuda_fail(e);
+    return e == cudaSuccess ? SELSCAN_OK : selscan::cuda_fail(e);
 }
 
 int selscan_fwd_plan(int64_t batch, int64_t seqlen, int64_t dim, int64_t dstate,
@@ -241,7 +264,7 @@ int selscan_state_update(float *state, const void *x, const void *delta, const f
     p.batch = batch; p.dim = dim; p.dstate = (int)dstate;
     p.softplus = softplus_flag ? 1 : 0;
     cudaError_t e = selscan::launch_state_update(p, dtype == SELSCAN_BF16, stream);
-    return e == cudaSuccess ? SELSCAN_OK : cuda_fail(e);
+    return e == cudaSuccess ? SELSCAN_OK : selscan::cuda_fail(e);
 }
 
 }  // extern "C"

@@ -210,6 +210,8 @@ scan_kernel(const ScanParams p) {
 
 // Chunk carry: one thread per (b, d, n), sequential over chunks,
 // hin_0 = 0, hin_{c+1} = P_c · hin_c + H_c; hin_c overwrites H_c in place.
+// Only the aggregates of chunks 0 .. nchunks-2 are read (pass 1 skips the
+// last chunk), so every workspace element is written before it is read.
 __global__ void carry_kernel(const ScanParams p) {
     const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     const int64_t total = p.batch * p.dim * kMaxN;
@@ -221,10 +223,14 @@ __global__ void carry_kernel(const ScanParams p) {
     float h = 0.0f;
     for (int c = 0; c < p.nchunks; ++c) {
         const size_t idx = (((size_t)b * p.nchunks + c) * p.dim + d) * kMaxN + n;
-        const float P = p.ws_P[idx];
-        const float H = p.ws_H[idx];
-        p.ws_H[idx] = h;
-        h = fmaf(P, h, H);
+        if (c + 1 < p.nchunks) {
+            const float P = p.ws_P[idx];
+            const float H = p.ws_H[idx];
+            p.ws_H[idx] = h;
+            h = fmaf(P, h, H);
+        } else {
+            p.ws_H[idx] = h;
+        }
     }
 }
 

@@ -96,5 +96,15 @@ struct StepParams {
 // Host-side launchers (one translation unit per kernel family).
 cudaError_t launch_scan(const ScanParams &p, bool bf16, cudaStream_t stream);
 cudaError_t launch_state_update(const StepParams &p, bool bf16, cudaStream_t stream);
+int scan_channels_per_cta();
+int scan_tile_tokens();
+
+// Host-side helpers of the C ABI (api.cu).
+int cuda_fail(cudaError_t e);  // records e for selscan_last_cuda_error
+int fwd_setup(const void *x, const void *delta, const float *A, const void *B,
+              const void *C, const float *D, const void *z, const float *delta_bias,
+              int softplus_flag, void *y, float *final_state, int64_t batch,
+              int64_t seqlen, int64_t dim, int64_t dstate, int dtype,
+              cudaStream_t stream, ScanParams *p, size_t *ws_bytes, bool *done);
 
 }  // namespace selscan
