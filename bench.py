@@ -230,6 +230,27 @@ def config_block(w, world):
             "l2": "no flush: inputs (1.35 GB/step) >> 126 MB L2"}
 
 
+# ---- multi-rank helpers (host logic; tested with gloo on CPU) ------------------
+def rank_seed(w, rank: int) -> int:
+    """Each rank draws its own independent batch (weak scaling)."""
+    return w.seed + 1000 * rank
+
+
+def max_over_ranks(value: float, dist, device) -> float:
+    """Max of a per-rank float over all ranks (every rank gets it)."""
+    import torch
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_rate(elements_per_rank: int, world: int, steps: int, max_ms: float) -> float:
+    """Whole-job throughput: all ranks' elements over the slowest rank's time."""
+    return elements_per_rank * world * steps / (max_ms / 1e3)
+
+
 # ---- the GPU arm ---------------------------------------------------------------
 def smi_id(torch, dev, local):
     """nvidia-smi id of a torch device: its PCI bus id when torch exposes it."""
@@ -264,7 +285,7 @@ def main():
 
     w = wl.WORKLOADS[args.workload]
     plan = ss.selscan_fwd_plan(w.batch, w.seqlen, w.dim, w.dstate)
-    inp = wl.make_scan_inputs(w.scaled(seed=w.seed + 1000 * rank), device=dev)
+    inp = wl.make_scan_inputs(w.scaled(seed=rank_seed(w, rank)), device=dev)
     y = torch.empty_like(inp["x"])
     fs = torch.empty(w.batch, w.dim, w.dstate, device=dev, dtype=torch.float32)
     stream = torch.cuda.current_stream(dev)
@@ -301,10 +322,7 @@ def main():
     barrier()
     ms = ev0.elapsed_time(ev1)
     clocks = sampler.stop() if sampler else None
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, dist if world > 1 else None, dev)
 
     # end to end through the public call: pinned host inputs -> device ->
     # selscan_fwd -> y and final state back to pinned host memory, every step
@@ -334,11 +352,7 @@ def main():
     e1.record(stream)
     torch.cuda.synchronize(dev)
     barrier()
-    e2e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), dist if world > 1 else None, dev)
     h2d = sum(host[k].numel() * host[k].element_size() for k in names)
     d2h = y_h.numel() * y_h.element_size() + fs_h.numel() * fs_h.element_size()
 
@@ -352,8 +366,7 @@ def main():
     if rank != 0:
         return 0
 
-    elems = w.elements * world * args.steps
-    value = elems / (ms / 1e3)
+    value = job_rate(w.elements, world, args.steps, ms)
     per_launch_s = ms / 1e3 / args.steps
     alg_bytes = w.algorithmic_bytes()
     achieved = alg_bytes / per_launch_s / 1e9
@@ -370,7 +383,7 @@ def main():
                      "frac_of_8TBps": achieved / 8000.0,
                      "algorithmic_bytes_per_launch": alg_bytes,
                      "kernel": "scan_kernel<bf16, gate, scan>", "traffic": None},
-        "e2e": {"value": w.elements * world * args.e2e_steps / (e2e_ms / 1e3),
+        "e2e": {"value": job_rate(w.elements, world, args.e2e_steps, e2e_ms),
                 "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": e2e_ms / args.e2e_steps},
         "gpu_launches": args.steps * plan["launches"],
