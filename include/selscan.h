@@ -66,7 +66,9 @@ enum {
     SELSCAN_ERR_MISALIGNED = -4,         /* a pointer is not element-aligned */
     SELSCAN_ERR_DSTATE_UNSUPPORTED = -5, /* dstate outside 1..16 */
     SELSCAN_ERR_CUDA = -6,               /* a CUDA call failed */
-    SELSCAN_ERR_ALIAS = -7               /* y overlaps an input */
+    SELSCAN_ERR_ALIAS = -7,              /* y overlaps an input */
+    SELSCAN_ERR_WORKSPACE = -8           /* selscan_fwd_noalloc: the plan needs more
+                                            workspace than its static array holds */
 };
 
 #define SELSCAN_MAX_DSTATE 16
@@ -104,6 +106,40 @@ SELSCAN_API int selscan_fwd(const void *x, const void *delta, const float *A,
                 const float *delta_bias, int softplus_flag, void *y,
                 float *final_state, int64_t batch, int64_t seqlen, int64_t dim,
                 int64_t dstate, selscan_dtype_t dtype, selscan_stream_t stream);
+
+/*
+ * selscan_fwd_noalloc -- selscan_fwd without any device allocation.
+ *
+ * The pages have no counterpart of this call; it exists for callers that
+ * cannot allocate device memory while they run: code whose device memory is
+ * all handed out by another allocator (a framework's caching allocator, an
+ * arena reserved at start-up), latency-critical loops where an allocation may
+ * block or fail, and processes without stream-ordered memory pools.
+ *
+ * Same arguments, results and launch plan as selscan_fwd. When the plan is
+ * chunked, the chunk workspace is a fixed array inside the library of
+ * SELSCAN_NOALLOC_WORKSPACE_BYTES bytes, held on every GPU that loads the
+ * library until the process exits; sizes whose workspace (selscan_fwd_plan)
+ * exceeds it are rejected with SELSCAN_ERR_WORKSPACE before anything runs.
+ * This call never calls cudaMalloc, cudaMallocAsync or cudaFree.
+ *  - The first call on a device that needs the workspace looks up the
+ *    array's device address (cudaGetSymbolAddress, once per device, with that
+ *    device current); make that first call before any stream capture.
+ *  - All calls on a device share the one array, and it keeps the contents
+ *    of the last call. Calls that overlap on the GPU (e.g. on two streams
+ *    without ordering between them) race on it and give wrong results; order
+ *    them. No element has to start at zero: each call writes every workspace
+ *    element before reading it.
+ */
+#define SELSCAN_NOALLOC_WORKSPACE_BYTES (16u << 20)
+
+SELSCAN_API int selscan_fwd_noalloc(const void *x, const void *delta, const float *A,
+                                    const void *B, const void *C, const float *D,
+                                    const void *z, const float *delta_bias,
+                                    int softplus_flag, void *y, float *final_state,
+                                    int64_t batch, int64_t seqlen, int64_t dim,
+                                    int64_t dstate, selscan_dtype_t dtype,
+                                    selscan_stream_t stream);
 
 /*
  * selscan_fwd_plan -- the launch plan selscan_fwd would use for these sizes

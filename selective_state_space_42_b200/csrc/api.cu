@@ -174,6 +174,8 @@ const char *selscan_status_string(int status) {
     case SELSCAN_ERR_DSTATE_UNSUPPORTED: return "dstate must be between 1 and 16";
     case SELSCAN_ERR_CUDA: return "a CUDA runtime call failed (see selscan_last_cuda_error)";
     case SELSCAN_ERR_ALIAS: return "the output y overlaps an input";
+    case SELSCAN_ERR_WORKSPACE:
+        return "the sizes need more chunk workspace than the static scratch array holds";
     default: return "unknown status";
     }
 }

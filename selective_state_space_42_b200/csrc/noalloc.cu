@@ -1,0 +1,82 @@
+// noalloc.cu -- selscan_fwd_noalloc: the selective scan with its chunk
+// workspace taken from a fixed device array instead of being allocated.
+//
+// Some callers cannot allocate device memory while they run: code whose whole
+// device memory is handed out by another allocator (a framework's caching
+// allocator, a fixed arena reserved at start-up), latency-critical loops where
+// an allocation may block or fail at the worst moment, and processes where
+// stream-ordered memory pools are unavailable or switched off. This entry
+// point computes exactly what selscan_fwd computes with the same launch plan,
+// but when that plan is chunked its workspace is the file-scope array below,
+// which every GPU that loads the library holds until the process exits.
+//
+// Host code must not use the array's name as a device address: in host code
+// it names a host-side stand-in. The device address is looked up once per
+// device with cudaGetSymbolAddress (with that device current), checked, cached
+// and passed to the kernels as a plain pointer.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <mutex>
+
+#include "selscan.h"
+#include "selscan_device.cuh"
+
+namespace {
+
+constexpr size_t kScratchFloats = (size_t)SELSCAN_NOALLOC_WORKSPACE_BYTES / sizeof(float);
+
+// The shared scratch: pass-1 chunk aggregates and carried states of the
+// chunked plan. Each call writes every element it reads before reading it, so
+// nothing in it has to start at zero; it keeps the last call's contents.
+static __device__ __align__(256) float g_scratch[kScratchFloats];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_mutex;
+float *g_scratch_ptr[kMaxDevices] = {nullptr};
+
+// Device address of g_scratch on the current device (looked up on first use).
+cudaError_t scratch_address(float **out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_mutex);
+    if (g_scratch_ptr[dev] == nullptr) {
+        void *ptr = nullptr;
+        e = cudaGetSymbolAddress(&ptr, g_scratch);
+        if (e != cudaSuccess) return e;
+        g_scratch_ptr[dev] = static_cast<float *>(ptr);
+    }
+    *out = g_scratch_ptr[dev];
+    return cudaSuccess;
+}
+
+}  // namespace
+
+extern "C" int selscan_fwd_noalloc(const void *x, const void *delta, const float *A,
+                                   const void *B, const void *C, const float *D,
+                                   const void *z, const float *delta_bias,
+                                   int softplus_flag, void *y, float *final_state,
+                                   int64_t batch, int64_t seqlen, int64_t dim,
+                                   int64_t dstate, selscan_dtype_t dtype,
+                                   selscan_stream_t stream_) {
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    selscan::ScanParams p{};
+    size_t ws_bytes = 0;
+    bool done = false;
+    const int st = selscan::fwd_setup(x, delta, A, B, C, D, z, delta_bias, softplus_flag,
+                                      y, final_state, batch, seqlen, dim, dstate, dtype,
+                                      stream, &p, &ws_bytes, &done);
+    if (st != SELSCAN_OK || done) return st;
+    if (ws_bytes > (size_t)SELSCAN_NOALLOC_WORKSPACE_BYTES) return SELSCAN_ERR_WORKSPACE;
+    if (ws_bytes > 0) {
+        float *scratch = nullptr;
+        cudaError_t e = scratch_address(&scratch);
+        if (e != cudaSuccess) return selscan::cuda_fail(e);
+        p.ws_P = scratch;
+        p.ws_H = scratch + ws_bytes / 2 / sizeof(float);
+    }
+    cudaError_t e = selscan::launch_scan(p, dtype == SELSCAN_BF16, stream);
+    return e == cudaSuccess ? SELSCAN_OK : selscan::cuda_fail(e);
+}

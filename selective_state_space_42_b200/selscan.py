@@ -23,8 +23,11 @@ STATUS = {
     0: "SELSCAN_OK", -1: "SELSCAN_ERR_NULL_ARG", -2: "SELSCAN_ERR_BAD_DIM",
     -3: "SELSCAN_ERR_BAD_DTYPE", -4: "SELSCAN_ERR_MISALIGNED",
     -5: "SELSCAN_ERR_DSTATE_UNSUPPORTED", -6: "SELSCAN_ERR_CUDA",
-    -7: "SELSCAN_ERR_ALIAS",
+    -7: "SELSCAN_ERR_ALIAS", -8: "SELSCAN_ERR_WORKSPACE",
 }
+
+# bytes of the fixed workspace array behind selscan_fwd_noalloc
+SELSCAN_NOALLOC_WORKSPACE_BYTES = 16 << 20
 
 _vp = ctypes.c_void_p
 _i64 = ctypes.c_int64
@@ -36,6 +39,8 @@ SIGNATURES = {
                            _i64, _i64, _i64, _i64, _int, _vp]),
     "selscan_state_update": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                     _int, _vp, _i64, _i64, _i64, _int, _vp]),
+    "selscan_fwd_noalloc": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _int, _vp,
+                                   _vp, _i64, _i64, _i64, _i64, _int, _vp]),
     "selscan_fwd_plan": (_int, [_i64, _i64, _i64, _i64, ctypes.POINTER(_i64),
                                 ctypes.POINTER(_i64), ctypes.POINTER(_i64)]),
     "selscan_status_string": (ctypes.c_char_p, [_int]),
@@ -152,6 +157,23 @@ def selscan_fwd(x, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=Tru
     x, delta, z: [batch, L, dim]; B, C: [batch, L, dstate] (same dtype as x,
     float32 or bfloat16); A: [dim, dstate] float32; D, delta_bias: [dim]
     float32. Returns y (allocated if not given) or (y, final_state)."""
+    return _fwd("selscan_fwd", x, delta, A, B, C, D, z, delta_bias, softplus, y,
+                final_state, return_final_state, stream)
+
+
+def selscan_fwd_noalloc(x, delta, A, B, C, D=None, z=None, delta_bias=None,
+                        softplus=True, y=None, final_state=None,
+                        return_final_state=False, stream=None):
+    """selscan_fwd whose chunk workspace is the library's fixed device array
+    (C ABI ``selscan_fwd_noalloc``): the library allocates nothing. For
+    callers that cannot allocate device memory, pass y (and final_state)
+    preallocated; otherwise this wrapper allocates them with torch."""
+    return _fwd("selscan_fwd_noalloc", x, delta, A, B, C, D, z, delta_bias, softplus,
+                y, final_state, return_final_state, stream)
+
+
+def _fwd(entry, x, delta, A, B, C, D, z, delta_bias, softplus, y, final_state,
+         return_final_state, stream):
     torch = _torch()
     if x.dim() != 3:
         raise ValueError("x must be [batch, L, dim]")
@@ -180,7 +202,7 @@ def selscan_fwd(x, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=Tru
         _ptr(final_state, "final_state", (batch, dim, N), f32, dev, required=False),
         batch, L, dim, N, code, _stream_ptr(stream, dev),
     ]
-    _check(load_library().selscan_fwd(*args))
+    _check(getattr(load_library(), entry)(*args))
     if return_final_state:
         return y, final_state
     return y
