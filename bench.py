@@ -382,7 +382,7 @@ def main():
                      "frac": achieved / peak, "peak_kind": peak_kind,
                      "frac_of_8TBps": achieved / 8000.0,
                      "algorithmic_bytes_per_launch": alg_bytes,
-                     "kernel": "scan_kernel<bf16, gate, scan>", "traffic": None},
+                     "kernel": "scan_tma_kernel<bf16, gate, seq>", "traffic": None},
         "e2e": {"value": job_rate(w.elements, world, args.e2e_steps, e2e_ms),
                 "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": e2e_ms / args.e2e_steps},

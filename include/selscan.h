@@ -92,14 +92,14 @@ enum {
  *   batch, seqlen, dim >= 0 (any of them 0 -> nothing to compute);
  *   1 <= dstate <= SELSCAN_MAX_DSTATE.
  *
- * Long sequences with few channels are split into chunks scanned in
- * parallel, then joined by carrying each chunk's final state (the pages'
- * blockwise scan with its state carried across blocks, "Hardware-Aware
- * Scan", and the associative operator of Guide Complet §4 "Parallel
- * Associative Scan"). That plan takes a stream-ordered device workspace
- * (cudaMallocAsync / cudaFreeAsync on `stream`) of
- * 2 · batch · chunks · dim · 16 floats (states padded to 16); no other memory
- * is allocated.
+ * The sequence is processed in chunks whose final states are carried to the
+ * next chunk (the pages' blockwise scan with its state carried across blocks,
+ * "Hardware-Aware Scan", and the associative operator of Guide Complet §4
+ * "Parallel Associative Scan"). Depending on the sizes, chunks run one after
+ * another with the state handed over on the device, or in parallel followed
+ * by a carry pass. Either takes a stream-ordered device workspace
+ * (cudaMallocAsync / cudaFreeAsync on `stream`; its size is reported by
+ * selscan_fwd_plan); no other memory is allocated.
  */
 SELSCAN_API int selscan_fwd(const void *x, const void *delta, const float *A,
                 const void *B, const void *C, const float *D, const void *z,
@@ -128,8 +128,9 @@ SELSCAN_API int selscan_fwd(const void *x, const void *delta, const float *A,
  *  - All calls on a device share the one array, and it keeps the contents
  *    of the last call. Calls that overlap on the GPU (e.g. on two streams
  *    without ordering between them) race on it and give wrong results; order
- *    them. No element has to start at zero: each call writes every workspace
- *    element before reading it.
+ *    them. The call itself clears, on `stream` and before its kernels, the
+ *    counters that must start at zero (cudaMemsetAsync, no allocation); every
+ *    other workspace element is written before it is read.
  */
 #define SELSCAN_NOALLOC_WORKSPACE_BYTES (16u << 20)
 
@@ -143,12 +144,12 @@ SELSCAN_API int selscan_fwd_noalloc(const void *x, const void *delta, const floa
 
 /*
  * selscan_fwd_plan -- the launch plan selscan_fwd would use for these sizes
- * (host only; no CUDA work). Writes, through each non-NULL pointer, the
- * number of sequence chunks (0 when there is nothing to compute), the number
- * of kernel launches (1 single pass; 3 chunked: chunk aggregates, carry,
- * rescan) and the bytes of stream-ordered workspace that call allocates.
- * Returns SELSCAN_OK or the size errors of selscan_fwd. The plan depends on
- * the current device's SM count.
+ * with bf16 tensors on 16-byte boundaries (host only; no CUDA work). Writes,
+ * through each non-NULL pointer, the number of sequence chunks (0 when there
+ * is nothing to compute), the number of kernel launches (1 single pass; 3
+ * chunked: chunk aggregates, carry, rescan) and the bytes of stream-ordered
+ * workspace that call allocates. Returns SELSCAN_OK or the size errors of
+ * selscan_fwd. The plan depends on the current device's SM count.
  */
 SELSCAN_API int selscan_fwd_plan(int64_t batch, int64_t seqlen, int64_t dim,
                                  int64_t dstate, int64_t *chunks, int64_t *launches,
@@ -179,6 +180,18 @@ SELSCAN_API int selscan_state_update(float *state, const void *x, const void *de
                          const float *delta_bias, int softplus_flag, void *y,
                          int64_t batch, int64_t dim, int64_t dstate,
                          selscan_dtype_t dtype, selscan_stream_t stream);
+
+/*
+ * selscan_device_status -- the library's sticky device-side error word on
+ * the current device (synchronous: waits for prior work). 0 means no device
+ * wait has given up; otherwise the code of the first one that did (1: a
+ * sequence chunk waited too long for its predecessor's state; 2, 3: a
+ * pipeline stage waited too long). Every device-side wait in the library is
+ * bounded (2 s); a wait that gives up records its code here and the kernel
+ * returns instead of hanging, leaving its outputs undefined. `clear` nonzero
+ * resets the word to 0 after reading it.
+ */
+SELSCAN_API int selscan_device_status(int *status, int clear);
 
 /* Static, NUL-terminated description of a status code (never NULL). */
 SELSCAN_API const char *selscan_status_string(int status);

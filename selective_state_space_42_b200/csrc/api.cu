@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 #include <stdlib.h>
+#include <string.h>
 
 #include "selscan.h"
 #include "selscan_device.cuh"
@@ -45,22 +46,21 @@ int sm_count() {
     return sms;
 }
 
-// Sequence split of one selscan_fwd call. Each (batch row, channel) chain is
-// one thread; when there are too few chains to keep every SM busy, the
-// sequence is split so that chains × chunks reaches a target of resident
-// threads, each chunk at least kMinChunk tokens and a whole number of B/C
-// tiles. SELSCAN_CHUNKS overrides the chunk count (tuning only).
-struct Plan {
-    int nchunks;
-    int64_t chunk_len;
-};
+int64_t env_int(const char *name) {
+    const char *v = getenv(name);
+    return (v && *v) ? atoll(v) : 0;
+}
 
-Plan plan_fwd(int64_t batch, int64_t seqlen, int64_t dim) {
+int64_t round_up(int64_t a, int64_t m) { return (a + m - 1) / m * m; }
+
+// Chunks of the generic kernels' plan. Each (batch row, channel) chain is one
+// thread; with too few chains to keep every SM busy the sequence is split so
+// that chains × chunks reaches a target of resident threads, each chunk at
+// least kMinChunk tokens and a whole number of B/C tiles.
+void plan_generic(int64_t batch, int64_t seqlen, int64_t dim, selscan::FwdPlan *pl) {
     constexpr int64_t kMinChunk = 256;
     constexpr int64_t kSinglePassChains = 16384;
-    const char *env = getenv("SELSCAN_CHUNKS");
-    int64_t n = 0;
-    if (env && *env) n = atoll(env);
+    int64_t n = env_int("SELSCAN_CHUNKS");
     if (n <= 0) {
         const int64_t chains = batch * dim;
         const int64_t target = (int64_t)sm_count() * 512;
@@ -73,18 +73,75 @@ Plan plan_fwd(int64_t batch, int64_t seqlen, int64_t dim) {
     if (n < 1) n = 1;
     if (n > seqlen) n = seqlen > 0 ? seqlen : 1;
     const int64_t tileT = selscan::scan_tile_tokens();
-    int64_t len = (seqlen + n - 1) / n;
-    len = (len + tileT - 1) / tileT * tileT;
+    int64_t len = round_up((seqlen + n - 1) / n, tileT);
     if (len < 1) len = 1;
-    Plan p;
-    p.chunk_len = len;
-    p.nchunks = seqlen > 0 ? (int)((seqlen + len - 1) / len) : 1;
-    return p;
+    selscan::ScanParams &g = pl->gp;
+    g.chunk_len = len;
+    g.nchunks = seqlen > 0 ? (int)((seqlen + len - 1) / len) : 1;
+    const int64_t cpc = selscan::scan_channels_per_cta();
+    g.ntiles = (int)((dim + cpc - 1) / cpc);
+    pl->tma = false;
+    pl->chunks = g.nchunks;
+    pl->launches = g.nchunks > 1 ? 3 : 1;
+    pl->ws_bytes = g.nchunks > 1
+                       ? 2 * (size_t)(batch * g.nchunks * dim) * selscan::kMaxN * sizeof(float)
+                       : 0;
+    pl->ws_clear = 0;
 }
 
-size_t workspace_bytes(int64_t batch, int64_t dim, int nchunks) {
-    if (nchunks <= 1) return 0;
-    return 2 * (size_t)(batch * nchunks * dim) * selscan::kMaxN * sizeof(float);
+// Plan of the TMA kernel. Groups = batch rows × 128-channel tiles. With at
+// least ~60% as many groups as SMs: one pass, units of kUnit tokens handed
+// from chunk to chunk (kModeSeq). With fewer: chunk aggregates, carry and
+// rescan, with about 8 units per SM. SELSCAN_PATH=seq|chunked, SELSCAN_UNIT
+// and SELSCAN_CHUNKS override (tuning only).
+void plan_tma(int64_t batch, int64_t seqlen, int64_t dim, bool bf16, selscan::FwdPlan *pl) {
+    const int64_t tileT = selscan::tma_tile_tokens(bf16);
+    const int64_t cpt = selscan::tma_tile_channels();
+    const int64_t ntiles = (dim + cpt - 1) / cpt;
+    const int64_t groups = batch * ntiles;
+    const int64_t sms = sm_count();
+    const char *path = getenv("SELSCAN_PATH");
+    bool seq = groups * 5 >= sms * 3;
+    if (path && !strcmp(path, "seq")) seq = true;
+    if (path && !strcmp(path, "chunked")) seq = false;
+    int64_t len = 0;
+    if (seq) {
+        len = env_int("SELSCAN_UNIT");
+        if (len <= 0) len = 512;
+    } else {
+        int64_t n = env_int("SELSCAN_CHUNKS");
+        if (n <= 0) n = (8 * sms + groups - 1) / groups;
+        const int64_t nmax = seqlen / 256 > 1 ? seqlen / 256 : 1;
+        n = n < nmax ? n : nmax;
+        if (n < 2) seq = true;
+        len = (seqlen + n - 1) / n;
+    }
+    len = round_up(len < seqlen ? len : seqlen, tileT);
+    const int64_t nchunks = (seqlen + len - 1) / len;
+    if (nchunks <= 1) seq = true;
+    selscan::TmaScanParams &t = pl->tp;
+    t.mode = seq ? selscan::kModeSeq : selscan::kModeAgg;
+    t.ntiles = (int)ntiles;
+    t.chunk_len = len;
+    t.nchunks = (int)nchunks;
+    t.groups = groups;
+    t.timeout_ns = 2000000000ull;
+    const int64_t tmo = env_int("SELSCAN_TIMEOUT_MS");
+    if (tmo > 0) t.timeout_ns = (unsigned long long)tmo * 1000000ull;
+    pl->tma = true;
+    pl->chunks = (int)nchunks;
+    pl->launches = seq ? 1 : 3;
+    // workspace: [0, 256) tickets; SEQ: flags at 256, states after them;
+    // chunked: P and H arrays from 256.
+    if (seq) {
+        const size_t flags_end = round_up(256 + 4 * 4 * groups, 256);  // one per warp
+        pl->ws_clear = flags_end;
+        pl->ws_bytes = flags_end + (size_t)groups * cpt * selscan::kMaxN * sizeof(float);
+    } else {
+        pl->ws_clear = 256;
+        pl->ws_bytes =
+            256 + 2 * (size_t)(batch * nchunks * dim) * selscan::kMaxN * sizeof(float);
+    }
 }
 
 }  // namespace
@@ -96,17 +153,33 @@ int cuda_fail(cudaError_t e) {
     return SELSCAN_ERR_CUDA;
 }
 
+void plan_for_sizes(int64_t batch, int64_t seqlen, int64_t dim, int64_t dstate, int dtype,
+                    bool aligned, FwdPlan *pl) {
+    const bool bf16 = dtype == SELSCAN_BF16;
+    const int64_t es = bf16 ? 2 : 4;
+    const char *path = getenv("SELSCAN_PATH");
+    const bool forced_generic = path && !strcmp(path, "generic");
+    // TMA rows must start on 16-byte boundaries and tiles are 128 channels.
+    const bool eligible = aligned && !forced_generic && dim >= tma_tile_channels() &&
+                          (dim * es) % 16 == 0 && batch * seqlen < ((int64_t)1 << 31) &&
+                          dstate <= kMaxN;
+    pl->bf16 = bf16;
+    if (eligible)
+        plan_tma(batch, seqlen, dim, bf16, pl);
+    else
+        plan_generic(batch, seqlen, dim, pl);
+}
+
 // Argument validation and launch plan shared by the selscan_fwd entry points.
-// On SELSCAN_OK fills *p (workspace pointers left NULL) and *ws_bytes, the
-// chunk workspace the plan needs; *done is set when no kernel has to run
-// (empty sizes; for seqlen == 0 the final state has been cleared on stream).
+// On SELSCAN_OK fills *plan (workspace pointers left NULL); *done is set when
+// no kernel has to run (empty sizes; for seqlen == 0 the final state has
+// been cleared on stream).
 int fwd_setup(const void *x, const void *delta, const float *A, const void *B,
               const void *C, const float *D, const void *z, const float *delta_bias,
               int softplus_flag, void *y, float *final_state, int64_t batch,
               int64_t seqlen, int64_t dim, int64_t dstate, int dtype,
-              cudaStream_t stream, ScanParams *p, size_t *ws_bytes, bool *done) {
+              cudaStream_t stream, FwdPlan *plan, bool *done) {
     *done = false;
-    *ws_bytes = 0;
     if (dtype != SELSCAN_F32 && dtype != SELSCAN_BF16) return SELSCAN_ERR_BAD_DTYPE;
     if (batch < 0 || seqlen < 0 || dim < 0) return SELSCAN_ERR_BAD_DIM;
     if (dstate < 1 || dstate > SELSCAN_MAX_DSTATE) return SELSCAN_ERR_DSTATE_UNSUPPORTED;
@@ -144,20 +217,80 @@ int fwd_setup(const void *x, const void *delta, const float *A, const void *B,
         return SELSCAN_OK;
     }
 
-    p->x = x; p->delta = delta; p->z = z; p->B = B; p->C = C;
-    p->A = A; p->Dskip = D; p->delta_bias = delta_bias;
-    p->y = y; p->final_state = final_state;
-    p->batch = batch; p->seqlen = seqlen; p->dim = dim; p->dstate = (int)dstate;
-    p->softplus = softplus_flag ? 1 : 0;
-    const int64_t cpc = scan_channels_per_cta();
-    p->ntiles = (int)((dim + cpc - 1) / cpc);
-    const Plan plan = plan_fwd(batch, seqlen, dim);
-    p->chunk_len = plan.chunk_len;
-    p->nchunks = plan.nchunks;
-    p->ws_P = p->ws_H = nullptr;
-    if (!mul_le(batch * plan.nchunks, p->ntiles, INT32_MAX)) return SELSCAN_ERR_BAD_DIM;
-    *ws_bytes = workspace_bytes(batch, dim, plan.nchunks);
+    const bool aligned = !misaligned(x, 16) && !misaligned(delta, 16) && !misaligned(z, 16);
+    plan_for_sizes(batch, seqlen, dim, dstate, dtype, aligned, plan);
+    plan->x = x;
+    plan->delta = delta;
+    plan->z = z;
+
+    ScanParams &g = plan->gp;
+    g.x = x; g.delta = delta; g.z = z; g.B = B; g.C = C;
+    g.A = A; g.Dskip = D; g.delta_bias = delta_bias;
+    g.y = y; g.final_state = final_state;
+    g.batch = batch; g.seqlen = seqlen; g.dim = dim; g.dstate = (int)dstate;
+    g.softplus = softplus_flag ? 1 : 0;
+    g.ws_P = g.ws_H = nullptr;
+    if (plan->tma) {
+        TmaScanParams &t = plan->tp;
+        t.B = B; t.C = C; t.A = A; t.Dskip = D; t.delta_bias = delta_bias;
+        t.y = y; t.final_state = final_state;
+        t.batch = batch; t.seqlen = seqlen; t.dim = dim; t.dstate = (int)dstate;
+        t.softplus = g.softplus;
+        const int64_t units = t.groups * t.nchunks;
+        if (units >= INT32_MAX) return SELSCAN_ERR_BAD_DIM;
+        // carry kernel parameters (chunked plan)
+        g.nchunks = t.nchunks;
+        g.chunk_len = t.chunk_len;
+    } else if (!mul_le(batch * g.nchunks, g.ntiles, INT32_MAX)) {
+        return SELSCAN_ERR_BAD_DIM;
+    }
     return SELSCAN_OK;
+}
+
+cudaError_t fwd_run(FwdPlan *plan, void *ws, cudaStream_t stream) {
+    if (!plan->tma) {
+        ScanParams &g = plan->gp;
+        if (g.nchunks > 1) {
+            const size_t half = plan->ws_bytes / 2;
+            g.ws_P = static_cast<float *>(ws);
+            g.ws_H = reinterpret_cast<float *>(static_cast<char *>(ws) + half);
+        }
+        return launch_scan(g, plan->bf16, stream);
+    }
+    TmaScanParams &t = plan->tp;
+    char *w = static_cast<char *>(ws);
+    cudaError_t e = cudaMemsetAsync(w, 0, plan->ws_clear, stream);
+    if (e != cudaSuccess) return e;
+    int *tickets = reinterpret_cast<int *>(w);
+    t.abort_all = tickets + 2;
+    if (t.mode == kModeSeq) {
+        t.ticket = tickets;
+        t.flags = reinterpret_cast<int *>(w + 256);
+        t.ws_state = reinterpret_cast<float *>(w + plan->ws_clear);
+        t.units = (int)(t.groups * t.nchunks);
+        return launch_scan_tma(t, plan->bf16, plan->x, plan->delta, plan->z, stream);
+    }
+    const size_t half = (plan->ws_bytes - 256) / 2;
+    t.ws_P = reinterpret_cast<float *>(w + 256);
+    t.ws_H = reinterpret_cast<float *>(w + 256 + half);
+    // pass 1: aggregates of every chunk but the last
+    t.mode = kModeAgg;
+    t.ticket = tickets;
+    t.units = (int)(t.groups * (t.nchunks - 1));
+    e = launch_scan_tma(t, plan->bf16, plan->x, plan->delta, plan->z, stream);
+    if (e != cudaSuccess) return e;
+    ScanParams &g = plan->gp;
+    g.ws_P = t.ws_P;
+    g.ws_H = t.ws_H;
+    e = launch_carry(g, stream);
+    if (e != cudaSuccess) return e;
+    // pass 2: every chunk from its carried-in state
+    t.mode = kModeRescan;
+    t.ticket = tickets + 1;
+    t.units = (int)(t.groups * t.nchunks);
+    e = launch_scan_tma(t, plan->bf16, plan->x, plan->delta, plan->z, stream);
+    t.mode = kModeAgg;
+    return e;
 }
 
 }  // namespace selscan
@@ -191,21 +324,18 @@ int selscan_fwd(const void *x, const void *delta, const float *A, const void *B,
                 int64_t seqlen, int64_t dim, int64_t dstate, selscan_dtype_t dtype,
                 selscan_stream_t stream_) {
     cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
-    selscan::ScanParams p{};
-    size_t ws_bytes = 0;
+    selscan::FwdPlan plan;
     bool done = false;
     const int st = selscan::fwd_setup(x, delta, A, B, C, D, z, delta_bias, softplus_flag,
                                       y, final_state, batch, seqlen, dim, dstate, dtype,
-                                      stream, &p, &ws_bytes, &done);
+                                      stream, &plan, &done);
     if (st != SELSCAN_OK || done) return st;
     void *ws = nullptr;
-    if (ws_bytes > 0) {
-        cudaError_t e = cudaMallocAsync(&ws, ws_bytes, stream);
+    if (plan.ws_bytes > 0) {
+        cudaError_t e = cudaMallocAsync(&ws, plan.ws_bytes, stream);
         if (e != cudaSuccess) return selscan::cuda_fail(e);
-        p.ws_P = static_cast<float *>(ws);
-        p.ws_H = reinterpret_cast<float *>(static_cast<char *>(ws) + ws_bytes / 2);
     }
-    cudaError_t e = selscan::launch_scan(p, dtype == SELSCAN_BF16, stream);
+    cudaError_t e = selscan::fwd_run(&plan, ws, stream);
     if (ws) {
         cudaError_t ef = cudaFreeAsync(ws, stream);
         if (e == cudaSuccess) e = ef;
@@ -219,18 +349,24 @@ int selscan_fwd_plan(int64_t batch, int64_t seqlen, int64_t dim, int64_t dstate,
     if (dstate < 1 || dstate > SELSCAN_MAX_DSTATE) return SELSCAN_ERR_DSTATE_UNSUPPORTED;
     if (!mul_le(batch, seqlen, kMaxElems) || !mul_le(batch * seqlen, dim, kMaxElems))
         return SELSCAN_ERR_BAD_DIM;
-    int64_t nc = 0, nl = 0;
-    size_t ws = 0;
+    int64_t nc = 0, nl = 0, ws = 0;
     if (batch > 0 && dim > 0 && seqlen > 0) {
-        const Plan plan = plan_fwd(batch, seqlen, dim);
-        nc = plan.nchunks;
-        nl = plan.nchunks > 1 ? 3 : 1;
-        ws = workspace_bytes(batch, dim, plan.nchunks);
+        selscan::FwdPlan plan;
+        selscan::plan_for_sizes(batch, seqlen, dim, dstate, SELSCAN_BF16, true, &plan);
+        nc = plan.chunks;
+        nl = plan.launches;
+        ws = (int64_t)plan.ws_bytes;
     }
     if (chunks) *chunks = nc;
     if (launches) *launches = nl;
-    if (workspace_bytes_out) *workspace_bytes_out = (int64_t)ws;
+    if (workspace_bytes_out) *workspace_bytes_out = ws;
     return SELSCAN_OK;
+}
+
+int selscan_device_status(int *status, int clear) {
+    if (!status) return SELSCAN_ERR_NULL_ARG;
+    cudaError_t e = selscan::read_device_status(status, clear != 0);
+    return e == cudaSuccess ? SELSCAN_OK : selscan::cuda_fail(e);
 }
 
 int selscan_state_update(float *state, const void *x, const void *delta, const float *A,

@@ -26,9 +26,10 @@ namespace {
 
 constexpr size_t kScratchFloats = (size_t)SELSCAN_NOALLOC_WORKSPACE_BYTES / sizeof(float);
 
-// The shared scratch: pass-1 chunk aggregates and carried states of the
-// chunked plan. Each call writes every element it reads before reading it, so
-// nothing in it has to start at zero; it keeps the last call's contents.
+// The shared scratch: the plan's workspace (tickets and completion flags,
+// which each call zeroes on its stream before its kernels run; chunk
+// aggregates and handed-over states, which each call writes before reading).
+// It keeps the last call's contents.
 static __device__ __align__(256) float g_scratch[kScratchFloats];
 
 constexpr int kMaxDevices = 64;
@@ -62,21 +63,18 @@ extern "C" int selscan_fwd_noalloc(const void *x, const void *delta, const float
                                    int64_t dstate, selscan_dtype_t dtype,
                                    selscan_stream_t stream_) {
     cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
-    selscan::ScanParams p{};
-    size_t ws_bytes = 0;
+    selscan::FwdPlan plan;
     bool done = false;
     const int st = selscan::fwd_setup(x, delta, A, B, C, D, z, delta_bias, softplus_flag,
                                       y, final_state, batch, seqlen, dim, dstate, dtype,
-                                      stream, &p, &ws_bytes, &done);
+                                      stream, &plan, &done);
     if (st != SELSCAN_OK || done) return st;
-    if (ws_bytes > (size_t)SELSCAN_NOALLOC_WORKSPACE_BYTES) return SELSCAN_ERR_WORKSPACE;
-    if (ws_bytes > 0) {
-        float *scratch = nullptr;
+    if (plan.ws_bytes > (size_t)SELSCAN_NOALLOC_WORKSPACE_BYTES) return SELSCAN_ERR_WORKSPACE;
+    float *scratch = nullptr;
+    if (plan.ws_bytes > 0) {
         cudaError_t e = scratch_address(&scratch);
         if (e != cudaSuccess) return selscan::cuda_fail(e);
-        p.ws_P = scratch;
-        p.ws_H = scratch + ws_bytes / 2 / sizeof(float);
     }
-    cudaError_t e = selscan::launch_scan(p, dtype == SELSCAN_BF16, stream);
+    cudaError_t e = selscan::fwd_run(&plan, scratch, stream);
     return e == cudaSuccess ? SELSCAN_OK : selscan::cuda_fail(e);
 }

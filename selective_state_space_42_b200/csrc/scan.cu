@@ -259,6 +259,12 @@ cudaError_t launch_typed(const ScanParams &p, cudaStream_t stream) {
 
 }  // namespace
 
+cudaError_t launch_carry(const ScanParams &p, cudaStream_t stream) {
+    const int64_t total = p.batch * p.dim * kMaxN;
+    carry_kernel<<<(unsigned)((total + 255) / 256), 256, 0, stream>>>(p);
+    return cudaGetLastError();
+}
+
 int scan_channels_per_cta() { return kThreads; }
 int scan_tile_tokens() { return kTileT; }
 

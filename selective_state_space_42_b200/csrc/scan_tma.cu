@@ -1,0 +1,554 @@
+// scan_tma.cu -- persistent, TMA-staged selective-scan kernel for sm_100a.
+//
+// Pages: "Mamba & State Space Models — Guide Complet" §4 "Implémentation du
+// SSM sélectif (S6)" (Δ = softplus(·), Abar = exp(Δ·A), h = Abar·h + Bbar·x,
+// y = C·h + D·x) and "Parallel Associative Scan"; "Mamba и State Space Models:
+// альтернатива Transformer", "SSM as RNN" and "Hardware-Aware Scan" (blocks of
+// the sequence with the state carried between them); "Mamba: co potrafią
+// modele przestrzeni stanów", "Cena selekcji" (fuse discretisation and
+// recurrence on chip, never write the expanded state).
+//
+// Organisation. One CTA per SM, 4 consumer warps + 1 producer warp. A unit of
+// work is (batch row b, 128-channel tile, chunk of the sequence). The producer
+// takes units from a global ticket counter, streams each unit's x, delta and
+// z tiles (kTile tokens × 128 channels) into a kStages-deep shared-memory ring
+// with 2-D TMA loads, and converts the unit's B and C rows to float32 in the
+// same ring slot. Each consumer thread owns one channel chain (16 float32
+// states in registers) and walks the tokens of a tile in sub-tiles of kSub:
+// first the per-token scalars (softplus, Δ·x, exp, gate) for all kSub tokens,
+// then the recurrence, packed two states at a time (f32x2).
+//
+// Modes:
+//  kSeq     single pass. Ticket i is chunk i / G of group i % G (G = batch ×
+//           channel tiles), so a unit's predecessor was handed out G tickets
+//           earlier to a running CTA; the unit waits (bounded) for the
+//           predecessor's completion flag, reads its final state from a
+//           per-group buffer in L2, and publishes its own when done. This
+//           balances any number of groups over the SMs without extra work.
+//           Each consumer warp hands over its own 32 channels (one flag per
+//           group and warp), so no barrier spans warps.
+//  kAgg     pass 1 of the chunked plan: chunks from a zero state, storing the
+//           aggregate P = Π Abar = 2^(A·log2 e·ΣΔ) and the chunk state H.
+//  kRescan  pass 2: chunks from the carried-in state; writes y.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "selscan_device.cuh"
+#include "tma_util.cuh"
+
+namespace selscan {
+namespace {
+
+constexpr int kConsumerWarps = 4;
+constexpr int kChannels = 32 * kConsumerWarps;  // channels per tile
+constexpr int kBlock = kChannels + 32;          // + producer warp
+#ifndef SELSCAN_TMA_STAGES
+#define SELSCAN_TMA_STAGES 4
+#endif
+#ifndef SELSCAN_TMA_KSUB
+#define SELSCAN_TMA_KSUB 8
+#endif
+constexpr int kStages = SELSCAN_TMA_STAGES;
+constexpr int kSub = SELSCAN_TMA_KSUB;  // tokens per register sub-tile
+
+template <typename T> struct TileCfg;
+template <> struct TileCfg<__nv_bfloat16> { static constexpr int kTile = 32; };
+template <> struct TileCfg<float> { static constexpr int kTile = 16; };
+
+template <typename T> struct alignas(128) Stage {
+    static constexpr int kTile = TileCfg<T>::kTile;
+    T x[kTile][kChannels];
+    T dl[kTile][kChannels];
+    T z[kTile][kChannels];
+    float B[kTile][kMaxN];
+    float C[kTile][kMaxN];
+};
+
+enum : int { kFirst = 1, kLast = 2, kEnd = 4 };
+
+struct TileInfo {
+    long long b, t0;
+    int tile, chunk, nt, flags;
+};
+
+template <typename T> struct alignas(128) Shared {
+    Stage<T> stage[kStages];
+    TileInfo info[kStages];
+    uint64_t full[kStages];
+    uint64_t empty[kStages];
+    int abort;
+};
+
+}  // namespace
+
+// Sticky device-side error word of this library on each device: 0, or the
+// code of the first wait that gave up (1 predecessor flag, 2 producer ring
+// slot, 3 consumer ring slot). Read and cleared by selscan_device_status.
+__device__ int g_device_status = 0;
+
+namespace {
+
+__device__ const int kNoAbort = 0;
+
+// Records the failure, stops this CTA (shared abort word) and every other CTA
+// of the launch (the launch's abort word in the workspace, polled by waits).
+__device__ __forceinline__ void fail(const TmaScanParams &p, int *abort, int code) {
+    atomicCAS(&g_device_status, 0, code);
+    *reinterpret_cast<volatile int *>(abort) = 1;
+    *reinterpret_cast<volatile int *>(p.abort_all) = 1;
+}
+
+// ---- producer warp -----------------------------------------------------------------
+template <typename T, bool kGate>
+__device__ void produce(Shared<T> &S, const TmaScanParams &p, const CUtensorMap *tm_x,
+                        const CUtensorMap *tm_d, const CUtensorMap *tm_z) {
+    constexpr int kTile = TileCfg<T>::kTile;
+    const int lane = threadIdx.x & 31;
+    if (lane == 0) {
+        prefetch_tmap(tm_x);
+        prefetch_tmap(tm_d);
+        if (kGate) prefetch_tmap(tm_z);
+    }
+    constexpr uint32_t kTileBytes = kTile * kChannels * sizeof(T);
+    const uint32_t tx_bytes = (kGate ? 3u : 2u) * kTileBytes;
+    const T *Bp = static_cast<const T *>(p.B);
+    const T *Cp = static_cast<const T *>(p.C);
+    int s = 0;
+    uint32_t phase = 0;
+    uint32_t issued = 0;  // bit i: stage i has a TMA issued with parity bit (16 + i)
+    for (;;) {
+        int ticket = 0;
+        if (lane == 0) ticket = atomicAdd(p.ticket, 1);
+        ticket = __shfl_sync(0xffffffffu, ticket, 0);
+        const bool end = ticket >= p.units;
+        long long b = 0, t_begin = 0, t_end = 0;
+        int tile = 0, chunk = 0, ntl = 1;
+        if (!end) {
+            const long long g = ticket % p.groups;
+            chunk = (int)(ticket / p.groups);
+            b = g / p.ntiles;
+            tile = (int)(g % p.ntiles);
+            t_begin = (long long)chunk * p.chunk_len;
+            t_end = min(t_begin + p.chunk_len, (long long)p.seqlen);
+            ntl = (int)((t_end - t_begin + kTile - 1) / kTile);
+        }
+        for (int j = 0; j < ntl; ++j) {
+            if (!mbar_wait(&S.empty[s], phase ^ 1u, &S.abort, p.timeout_ns)) {
+                if (lane == 0) {
+                    fail(p, &S.abort, 2);
+                    // wait (bounded) for this warp's own copies still in flight
+                    for (int i = 0; i < kStages; ++i)
+                        if (issued & (1u << i))
+                            mbar_wait(&S.full[i], (issued >> (16 + i)) & 1u, &kNoAbort,
+                                      p.timeout_ns / 16);
+                }
+                __syncwarp();
+                return;
+            }
+            const long long t0 = t_begin + (long long)j * kTile;
+            const int nt = end ? 0 : (int)min((long long)kTile, t_end - t0);
+            if (lane == 0) {
+                TileInfo &inf = S.info[s];
+                inf.b = b;
+                inf.t0 = t0;
+                inf.tile = tile;
+                inf.chunk = chunk;
+                inf.nt = nt;
+                inf.flags = end ? kEnd : ((j == 0 ? kFirst : 0) | (j == ntl - 1 ? kLast : 0));
+                if (!end) {
+                    mbar_expect_tx(&S.full[s], tx_bytes);
+                    const int c0 = tile * kChannels;
+                    const int c1 = (int)(b * p.seqlen + t0);
+                    tma_load_2d(&S.stage[s].x[0][0], tm_x, &S.full[s], c0, c1);
+                    tma_load_2d(&S.stage[s].dl[0][0], tm_d, &S.full[s], c0, c1);
+                    if (kGate) tma_load_2d(&S.stage[s].z[0][0], tm_z, &S.full[s], c0, c1);
+                    issued = (issued | (1u << s)) & ~(1u << (16 + s));
+                    issued |= phase << (16 + s);
+                }
+            }
+            if (!end) {
+                // B and C rows of the tile as float32; rows past the tile's
+                // tokens and states past dstate are zero.
+                const int row = lane % kTile;
+                const bool isC = lane >= kTile;  // only when kTile == 16
+                for (int r = row; r < kTile; r += 32) {
+                    const bool in = r < nt;
+                    const long long gi = (b * p.seqlen + t0 + r) * p.dstate;
+                    float vb[kMaxN], vc[kMaxN];
+#pragma unroll
+                    for (int n = 0; n < kMaxN; ++n) {
+                        const bool ok = in && n < p.dstate;
+                        vb[n] = (ok && (kTile == 32 || !isC)) ? ldg_f32(Bp + gi + n) : 0.0f;
+                        vc[n] = (ok && (kTile == 32 || isC)) ? ldg_f32(Cp + gi + n) : 0.0f;
+                    }
+                    float4 *db = reinterpret_cast<float4 *>(&S.stage[s].B[r][0]);
+                    float4 *dc = reinterpret_cast<float4 *>(&S.stage[s].C[r][0]);
+#pragma unroll
+                    for (int q = 0; q < kMaxN / 4; ++q) {
+                        if (kTile == 32 || !isC)
+                            db[q] = make_float4(vb[4 * q], vb[4 * q + 1], vb[4 * q + 2], vb[4 * q + 3]);
+                        if (kTile == 32 || isC)
+                            dc[q] = make_float4(vc[4 * q], vc[4 * q + 1], vc[4 * q + 2], vc[4 * q + 3]);
+                    }
+                }
+            }
+            __syncwarp();
+            mbar_arrive(&S.full[s]);
+            if (++s == kStages) {
+                s = 0;
+                phase ^= 1u;
+            }
+        }
+        if (end) return;
+    }
+}
+
+// ---- consumer warps ----------------------------------------------------------------
+__device__ __forceinline__ float softplus_fast(float v) {
+    // log(1 + e^v) through the MUFU pair; absolute error ~1e-7, enough for
+    // bf16 I/O. Large v returns v.
+    const float w = ex2_approx(v * kLog2e);
+    const float s = lg2_approx(1.0f + w) * kLn2;
+    return v > 15.0f ? v : s;
+}
+
+template <typename T, bool kGate, int kMode, bool kStruct>
+__device__ __forceinline__ void consume_tile(const Stage<T> &st, int nt, float2 (&h)[kMaxN / 2],
+                                             const float (&A2)[kMaxN], float dskip, float bias,
+                                             int softplus, float &dt_sum, T *yp, long long ybase,
+                                             long long ystride, bool active) {
+    constexpr int kTile = TileCfg<T>::kTile;
+    constexpr bool kFastSp = sizeof(T) == 2;
+    const int c = threadIdx.x;  // channel within the tile
+#pragma unroll 1
+    for (int sub = 0; sub < kTile; sub += kSub) {
+        if (sub >= nt) break;
+        float uu[kSub], rr[kSub], gg[kSub], pp[kSub];
+        // per-token scalars
+#pragma unroll
+        for (int k = 0; k < kSub; ++k) {
+            const int t = sub + k;
+            const bool valid = t < nt;
+            const float xv = to_f32(st.x[t][c]);
+            float dt = to_f32(st.dl[t][c]) + bias;
+            if (softplus) dt = kFastSp ? softplus_fast(dt) : softplus_f32(dt);
+            dt = valid ? dt : 0.0f;  // Abar = 1, no input: the state is unchanged
+            uu[k] = dt * xv;
+            rr[k] = kStruct ? ex2_approx(dt * A2[0]) : dt;
+            if (kMode == kModeAgg) {
+                dt_sum += dt;
+            } else {
+                const float g = kGate ? silu_f32(to_f32(st.z[t][c])) : 1.0f;
+                gg[k] = g;
+                pp[k] = dskip * xv * g;
+            }
+        }
+        // recurrence
+#pragma unroll
+        for (int k = 0; k < kSub; ++k) {
+            const int t = sub + k;
+            float2 a[kMaxN / 2];
+            if (kStruct) {
+                const float r = rr[k];
+                const float r2 = r * r;
+                a[0] = make_float2(r, r2);
+                a[1] = __fmul2_rn(a[0], make_float2(r2, r2));
+                const float r4 = a[1].y;
+                const float2 q4 = make_float2(r4, r4);
+                a[2] = __fmul2_rn(a[0], q4);
+                a[3] = __fmul2_rn(a[1], q4);
+                const float r8 = a[3].y;
+                const float2 q8 = make_float2(r8, r8);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) a[4 + j] = __fmul2_rn(a[j], q8);
+            } else {
+#pragma unroll
+                for (int j = 0; j < kMaxN / 2; ++j)
+                    a[j] = make_float2(ex2_approx(rr[k] * A2[2 * j]),
+                                       ex2_approx(rr[k] * A2[2 * j + 1]));
+            }
+            const float2 u2 = make_float2(uu[k], uu[k]);
+            const float4 *B4 = reinterpret_cast<const float4 *>(&st.B[t][0]);
+            if (kMode == kModeAgg) {
+#pragma unroll
+                for (int q = 0; q < kMaxN / 4; ++q) {
+                    const float4 bq = B4[q];
+                    h[2 * q] = __ffma2_rn(a[2 * q], h[2 * q], __fmul2_rn(u2, make_float2(bq.x, bq.y)));
+                    h[2 * q + 1] =
+                        __ffma2_rn(a[2 * q + 1], h[2 * q + 1], __fmul2_rn(u2, make_float2(bq.z, bq.w)));
+                }
+            } else {
+                const float4 *C4 = reinterpret_cast<const float4 *>(&st.C[t][0]);
+                float2 y0 = make_float2(0.0f, 0.0f), y1 = y0;
+#pragma unroll
+                for (int q = 0; q < kMaxN / 4; ++q) {
+                    const float4 bq = B4[q];
+                    const float4 cq = C4[q];
+                    h[2 * q] = __ffma2_rn(a[2 * q], h[2 * q], __fmul2_rn(u2, make_float2(bq.x, bq.y)));
+                    h[2 * q + 1] =
+                        __ffma2_rn(a[2 * q + 1], h[2 * q + 1], __fmul2_rn(u2, make_float2(bq.z, bq.w)));
+                    y0 = __ffma2_rn(make_float2(cq.x, cq.y), h[2 * q], y0);
+                    y1 = __ffma2_rn(make_float2(cq.z, cq.w), h[2 * q + 1], y1);
+                }
+                const float2 ys = __fadd2_rn(y0, y1);
+                const float out = fmaf(ys.x + ys.y, gg[k], pp[k]);
+                if (active && t < nt) yp[ybase + (long long)t * ystride] = from_f32<T>(out);
+            }
+        }
+    }
+}
+
+template <typename T, bool kGate, int kMode>
+__device__ void consume(Shared<T> &S, const TmaScanParams &p) {
+    const int c = threadIdx.x;  // 0..127
+    const int lane = c & 31;
+    T *yp = static_cast<T *>(p.y);
+    int s = 0;
+    uint32_t phase = 0;
+    int cur_tile = -1;
+    float A2[kMaxN];
+    float dskip = 0.0f, bias = 0.0f;
+    bool structured = false;
+    float2 h[kMaxN / 2];
+#pragma unroll
+    for (int j = 0; j < kMaxN / 2; ++j) h[j] = make_float2(0.0f, 0.0f);
+    float dt_sum = 0.0f;
+    for (;;) {
+        if (!mbar_wait(&S.full[s], phase, &S.abort, p.timeout_ns)) {
+            if (lane == 0) fail(p, &S.abort, 3);
+            return;
+        }
+        const TileInfo inf = S.info[s];
+        if (inf.flags & kEnd) return;
+        const long long d = (long long)inf.tile * kChannels + c;
+        const bool active = d < p.dim;
+        const long long g = inf.b * p.ntiles + inf.tile;
+        if (inf.flags & kFirst) {
+            if (inf.tile != cur_tile) {
+                bool ok = true;
+                if (active) {
+                    const float *Ar = p.A + d * p.dstate;
+                    const float a0 = Ar[0];
+#pragma unroll
+                    for (int n = 0; n < kMaxN; ++n) {
+                        const float an = n < p.dstate ? Ar[n] : 0.0f;
+                        A2[n] = an * kLog2e;
+                        if (n < p.dstate) ok &= (an == (float)(n + 1) * a0);
+                    }
+                    dskip = p.Dskip ? p.Dskip[d] : 0.0f;
+                    bias = p.delta_bias ? p.delta_bias[d] : 0.0f;
+                } else {
+#pragma unroll
+                    for (int n = 0; n < kMaxN; ++n) A2[n] = 0.0f;
+                    dskip = bias = 0.0f;
+                }
+                structured = __all_sync(0xffffffffu, ok);
+                cur_tile = inf.tile;
+            }
+            dt_sum = 0.0f;
+            float hs[kMaxN];
+#pragma unroll
+            for (int n = 0; n < kMaxN; ++n) hs[n] = 0.0f;
+            if (kMode == kModeSeq && inf.chunk > 0) {
+                // every lane acquires this warp's predecessor flag (bounded)
+                const int *flag = p.flags + g * kConsumerWarps + (c >> 5);
+                const uint64_t start = global_ns();
+                while (ld_acquire_gpu(flag) < inf.chunk) {
+                    __nanosleep(64);
+                    if (*reinterpret_cast<volatile int *>(&S.abort) ||
+                        *reinterpret_cast<volatile int *>(p.abort_all) ||
+                        global_ns() - start > p.timeout_ns) {
+                        if (lane == 0) fail(p, &S.abort, 1);
+                        break;
+                    }
+                }
+                __syncwarp();
+                if (active) {
+                    const float *src = p.ws_state + (g * kChannels + c) * kMaxN;
+#pragma unroll
+                    for (int q = 0; q < kMaxN / 4; ++q) {
+                        const float4 v = ld_cg_f4(src + 4 * q);
+                        hs[4 * q] = v.x; hs[4 * q + 1] = v.y; hs[4 * q + 2] = v.z; hs[4 * q + 3] = v.w;
+                    }
+                }
+            } else if (kMode == kModeRescan && p.nchunks > 1 && active) {
+                const float *src = p.ws_H + ((inf.b * p.nchunks + inf.chunk) * p.dim + d) * kMaxN;
+#pragma unroll
+                for (int n = 0; n < kMaxN; ++n) hs[n] = src[n];
+            }
+#pragma unroll
+            for (int j = 0; j < kMaxN / 2; ++j) h[j] = make_float2(hs[2 * j], hs[2 * j + 1]);
+        }
+
+        const long long ybase = (inf.b * p.seqlen + inf.t0) * p.dim + d;
+        if (structured)
+            consume_tile<T, kGate, kMode, true>(S.stage[s], inf.nt, h, A2, dskip, bias, p.softplus,
+                                                dt_sum, yp, ybase, p.dim, active);
+        else
+            consume_tile<T, kGate, kMode, false>(S.stage[s], inf.nt, h, A2, dskip, bias, p.softplus,
+                                                 dt_sum, yp, ybase, p.dim, active);
+
+        if (inf.flags & kLast) {
+            const bool last_chunk = inf.chunk == p.nchunks - 1;
+            if (kMode == kModeAgg) {
+                if (active) {
+                    const long long row = ((inf.b * p.nchunks + inf.chunk) * p.dim + d) * kMaxN;
+#pragma unroll
+                    for (int j = 0; j < kMaxN / 2; ++j) {
+                        p.ws_P[row + 2 * j] = ex2_approx(A2[2 * j] * dt_sum);
+                        p.ws_P[row + 2 * j + 1] = ex2_approx(A2[2 * j + 1] * dt_sum);
+                        p.ws_H[row + 2 * j] = h[j].x;
+                        p.ws_H[row + 2 * j + 1] = h[j].y;
+                    }
+                }
+            } else if (last_chunk) {
+                if (p.final_state && active) {
+                    float *fs = p.final_state + (inf.b * p.dim + d) * p.dstate;
+#pragma unroll
+                    for (int j = 0; j < kMaxN / 2; ++j) {
+                        if (2 * j < p.dstate) fs[2 * j] = h[j].x;
+                        if (2 * j + 1 < p.dstate) fs[2 * j + 1] = h[j].y;
+                    }
+                }
+            } else if (kMode == kModeSeq) {
+                if (active) {
+                    float *dst = p.ws_state + (g * kChannels + c) * kMaxN;
+#pragma unroll
+                    for (int q = 0; q < kMaxN / 4; ++q)
+                        st_cg_f4(dst + 4 * q, make_float4(h[2 * q].x, h[2 * q].y, h[2 * q + 1].x,
+                                                          h[2 * q + 1].y));
+                }
+                __threadfence();
+                __syncwarp();
+                if (lane == 0) st_release_gpu(p.flags + g * kConsumerWarps + (c >> 5), inf.chunk + 1);
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&S.empty[s]);
+        if (++s == kStages) {
+            s = 0;
+            phase ^= 1u;
+        }
+    }
+}
+
+template <typename T, bool kGate, int kMode>
+__global__ void __launch_bounds__(kBlock, 1)
+scan_tma_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_d,
+                const __grid_constant__ CUtensorMap tm_z, const TmaScanParams p) {
+    // Indexed straight off the __shared__ array so that every access compiles
+    // to a shared-memory instruction (no generic addressing, no aliasing with
+    // the global y stores).
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    Shared<T> &S = *reinterpret_cast<Shared<T> *>(smem_raw);
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kStages; ++i) {
+            mbar_init(&S.full[i], 32);              // producer lanes (+ TMA bytes)
+            mbar_init(&S.empty[i], kConsumerWarps);  // one arrival per consumer warp
+        }
+        S.abort = 0;
+        fence_barrier_init();
+    }
+    __syncthreads();
+    if (threadIdx.x >= kChannels)
+        produce<T, kGate>(S, p, &tm_x, &tm_d, &tm_z);
+    else
+        consume<T, kGate, kMode>(S, p);
+}
+
+// ---- host side -----------------------------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        cudaDriverEntryPointQueryResult q;
+        void *ptr = nullptr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    }
+    return fn;
+}
+
+template <typename T>
+bool make_map(CUtensorMap *m, const void *base, long long rows, long long dim) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    const CUtensorMapDataType dt = sizeof(T) == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                                  : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+    cuuint64_t gdim[2] = {(cuuint64_t)dim, (cuuint64_t)rows};
+    cuuint64_t gstride[1] = {(cuuint64_t)(dim * sizeof(T))};
+    cuuint32_t box[2] = {(cuuint32_t)kChannels, (cuuint32_t)TileCfg<T>::kTile};
+    cuuint32_t estride[2] = {1, 1};
+    CUresult r = fn(m, dt, 2, const_cast<void *>(base), gdim, gstride, box, estride,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+int num_sms() {
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    return sms > 0 ? sms : 148;
+}
+
+template <typename T, bool kGate, int kMode>
+cudaError_t launch_mode(const TmaScanParams &p, const void *x, const void *dl, const void *z,
+                        cudaStream_t stream) {
+    if (p.units <= 0) return cudaSuccess;
+    CUtensorMap mx, md, mz;
+    const long long rows = p.batch * p.seqlen;
+    if (!make_map<T>(&mx, x, rows, p.dim) || !make_map<T>(&md, dl, rows, p.dim))
+        return cudaErrorInvalidValue;
+    if (kGate) {
+        if (!make_map<T>(&mz, z, rows, p.dim)) return cudaErrorInvalidValue;
+    } else {
+        mz = md;
+    }
+    const size_t smem = sizeof(Shared<T>);
+    auto kern = scan_tma_kernel<T, kGate, kMode>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    const long long grid = min((long long)num_sms(), (long long)p.units);
+    kern<<<(unsigned)grid, kBlock, smem, stream>>>(mx, md, mz, p);
+    return cudaGetLastError();
+}
+
+template <typename T, bool kGate>
+cudaError_t launch_gate(const TmaScanParams &p, const void *x, const void *dl, const void *z,
+                        cudaStream_t stream) {
+    switch (p.mode) {
+    case kModeSeq: return launch_mode<T, kGate, kModeSeq>(p, x, dl, z, stream);
+    case kModeAgg: return launch_mode<T, false, kModeAgg>(p, x, dl, z, stream);
+    default: return launch_mode<T, kGate, kModeRescan>(p, x, dl, z, stream);
+    }
+}
+
+}  // namespace
+
+cudaError_t read_device_status(int *out, bool clear) {
+    cudaError_t e = cudaMemcpyFromSymbol(out, g_device_status, sizeof(int));
+    if (e == cudaSuccess && clear) {
+        const int zero = 0;
+        e = cudaMemcpyToSymbol(g_device_status, &zero, sizeof(int));
+    }
+    return e;
+}
+
+int tma_tile_channels() { return kChannels; }
+int tma_tile_tokens(bool bf16) {
+    return bf16 ? TileCfg<__nv_bfloat16>::kTile : TileCfg<float>::kTile;
+}
+
+cudaError_t launch_scan_tma(const TmaScanParams &p, bool bf16, const void *x, const void *dl,
+                            const void *z, cudaStream_t stream) {
+    if (bf16)
+        return z ? launch_gate<__nv_bfloat16, true>(p, x, dl, z, stream)
+                 : launch_gate<__nv_bfloat16, false>(p, x, dl, z, stream);
+    return z ? launch_gate<float, true>(p, x, dl, z, stream)
+             : launch_gate<float, false>(p, x, dl, z, stream);
+}
+
+}  // namespace selscan

@@ -93,6 +93,39 @@ struct StepParams {
     int softplus;
 };
 
+// Persistent TMA-staged scan (scan_tma.cu).
+enum : int { kModeSeq = 0, kModeAgg = 1, kModeRescan = 2 };
+
+struct TmaScanParams {
+    const void *B, *C;
+    const float *A, *Dskip, *delta_bias;
+    void *y;
+    float *final_state;
+    long long batch, seqlen, dim;
+    int dstate;
+    int softplus;
+    int mode;             // kModeSeq | kModeAgg | kModeRescan
+    int ntiles;           // 128-channel tiles per batch row
+    long long chunk_len;  // tokens per unit (a multiple of the token tile)
+    int nchunks;          // units per sequence
+    long long groups;     // batch * ntiles
+    int units;            // tickets handed out by this launch
+    // workspace (zeroed counters + arrays)
+    int *ticket;          // next ticket of this launch
+    int *flags;           // kModeSeq: chunks completed, per group and consumer warp
+    int *abort_all;       // set by any CTA whose wait gave up; stops the others
+    float *ws_state;      // kModeSeq: [groups][128][16] state handed between units
+    float *ws_P, *ws_H;   // chunked: [batch][nchunks][dim][16]
+    unsigned long long timeout_ns;  // bound on every device-side wait
+};
+
+cudaError_t launch_scan_tma(const TmaScanParams &p, bool bf16, const void *x, const void *dl,
+                            const void *z, cudaStream_t stream);
+cudaError_t read_device_status(int *out, bool clear);
+int tma_tile_channels();
+int tma_tile_tokens(bool bf16);
+cudaError_t launch_carry(const ScanParams &p, cudaStream_t stream);
+
 // Host-side launchers (one translation unit per kernel family).
 cudaError_t launch_scan(const ScanParams &p, bool bf16, cudaStream_t stream);
 cudaError_t launch_state_update(const StepParams &p, bool bf16, cudaStream_t stream);
@@ -101,10 +134,30 @@ int scan_tile_tokens();
 
 // Host-side helpers of the C ABI (api.cu).
 int cuda_fail(cudaError_t e);  // records e for selscan_last_cuda_error
+
+// A selscan_fwd call after validation: which kernels run, their parameters,
+// and the workspace they need.
+struct FwdPlan {
+    bool tma = false;     // TMA-staged persistent kernel (else the generic kernels)
+    ScanParams gp{};      // generic kernels (and the carry kernel)
+    TmaScanParams tp{};   // TMA kernel
+    const void *x = nullptr, *delta = nullptr, *z = nullptr;
+    bool bf16 = false;
+    int chunks = 1;       // sequence chunks
+    int launches = 0;     // kernel launches
+    size_t ws_bytes = 0;  // workspace bytes
+    size_t ws_clear = 0;  // leading workspace bytes zeroed before the launches
+};
+
 int fwd_setup(const void *x, const void *delta, const float *A, const void *B,
               const void *C, const float *D, const void *z, const float *delta_bias,
               int softplus_flag, void *y, float *final_state, int64_t batch,
               int64_t seqlen, int64_t dim, int64_t dstate, int dtype,
-              cudaStream_t stream, ScanParams *p, size_t *ws_bytes, bool *done);
+              cudaStream_t stream, FwdPlan *plan, bool *done);
+// Plans for the given sizes assuming 16-byte aligned tensors (selscan_fwd_plan).
+void plan_for_sizes(int64_t batch, int64_t seqlen, int64_t dim, int64_t dstate, int dtype,
+                    bool aligned, FwdPlan *plan);
+// Points the plan at a workspace of plan->ws_bytes bytes and launches it.
+cudaError_t fwd_run(FwdPlan *plan, void *ws, cudaStream_t stream);
 
 }  // namespace selscan

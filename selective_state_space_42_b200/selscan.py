@@ -43,6 +43,7 @@ SIGNATURES = {
                                    _vp, _i64, _i64, _i64, _i64, _int, _vp]),
     "selscan_fwd_plan": (_int, [_i64, _i64, _i64, _i64, ctypes.POINTER(_i64),
                                 ctypes.POINTER(_i64), ctypes.POINTER(_i64)]),
+    "selscan_device_status": (_int, [ctypes.POINTER(_int), _int]),
     "selscan_status_string": (ctypes.c_char_p, [_int]),
     "selscan_last_cuda_error": (ctypes.c_char_p, []),
 }
@@ -148,6 +149,14 @@ def selscan_fwd_plan(batch: int, seqlen: int, dim: int, dstate: int) -> dict:
     _check(load_library().selscan_fwd_plan(batch, seqlen, dim, dstate, ctypes.byref(c),
                                            ctypes.byref(n), ctypes.byref(w)))
     return {"chunks": c.value, "launches": n.value, "workspace_bytes": w.value}
+
+
+def selscan_device_status(clear: bool = False) -> int:
+    """The library's sticky device-side error word on the current device (C
+    ABI ``selscan_device_status``); 0 when no device wait has given up."""
+    v = _int()
+    _check(load_library().selscan_device_status(ctypes.byref(v), int(bool(clear))))
+    return v.value
 
 
 def selscan_fwd(x, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=True,

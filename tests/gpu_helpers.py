@@ -90,3 +90,23 @@ def forced_chunks(n):
             del os.environ["SELSCAN_CHUNKS"]
         else:
             os.environ["SELSCAN_CHUNKS"] = old
+
+
+@contextmanager
+def env(**kw):
+    """Temporarily set (value) or unset (None) environment variables read by
+    the library's planner (SELSCAN_PATH, SELSCAN_UNIT, SELSCAN_CHUNKS)."""
+    old = {k: os.environ.get(k) for k in kw}
+    try:
+        for k, v in kw.items():
+            if v is None:
+                os.environ.pop(k, None)
+            else:
+                os.environ[k] = str(v)
+        yield
+    finally:
+        for k, v in old.items():
+            if v is None:
+                os.environ.pop(k, None)
+            else:
+                os.environ[k] = v

@@ -84,6 +84,35 @@ def test_ragged(dtype, shape, variant, chunks):
         _check_fwd(inp, gh.RTOL[dtype], softplus=softplus, what=f"{shape} {variant}")
 
 
+TMA_SHAPES = [(1, 1, 128, 16), (2, 33, 136, 16), (1, 300, 256, 8), (3, 257, 384, 16),
+              (2, 1000, 200, 4), (1, 2049, 128, 1), (4, 96, 1024, 16)]
+TMA_PATHS = {
+    "seq_unit32": dict(SELSCAN_PATH="seq", SELSCAN_UNIT="32", SELSCAN_CHUNKS=None),
+    "seq_default": dict(SELSCAN_PATH="seq", SELSCAN_UNIT=None, SELSCAN_CHUNKS=None),
+    "chunked3": dict(SELSCAN_PATH="chunked", SELSCAN_UNIT=None, SELSCAN_CHUNKS="3"),
+    "chunked_auto": dict(SELSCAN_PATH="chunked", SELSCAN_UNIT=None, SELSCAN_CHUNKS=None),
+}
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("shape", TMA_SHAPES, ids=str)
+@pytest.mark.parametrize("variant", ["structA_gate", "randomA_nogate"])
+@pytest.mark.parametrize("path", list(TMA_PATHS))
+def test_tma_paths(dtype, shape, variant, path):
+    """The TMA-staged kernel in each of its plans, on ragged channel tiles
+    (dim not a multiple of 128), ragged token tiles and d_state 1..16."""
+    batch, L, dim, N = shape
+    w = wl.ScanWorkload("tma", batch, L, dim, N, dtype, gate=variant.endswith("_gate"),
+                        seed=2000 + L + dim + N)
+    inp = wl.make_scan_inputs(w)
+    if variant.startswith("randomA"):
+        inp["A"] = _random_A(dim, N, seed=L * 11 + dim)
+    inp = _cuda(inp)
+    with gh.env(**TMA_PATHS[path]):
+        _check_fwd(inp, gh.RTOL[dtype], what=f"{shape} {variant} {path}")
+    assert ss.selscan_device_status() == 0
+
+
 def test_empty_and_degenerate():
     f32 = torch.float32
     # L = 0: nothing to compute, final state is zero
@@ -166,6 +195,16 @@ def test_long_1m_sampled():
     """One 1M-token sequence: chunk carry across many chunks, state continuity
     over the whole length."""
     _full_size_sampled("long_1m", 512)
+
+
+def test_generic_path_forced_on_bench_shape_sampled():
+    """The generic kernels on the benchmark's workload (planner override)."""
+    with gh.env(SELSCAN_PATH="generic"):
+        _full_size_sampled("mamba2p8b_layer", 1024, batches=[0, 3])
+
+
+def test_no_device_wait_gave_up():
+    assert ss.selscan_device_status(clear=True) == 0
 
 
 def test_cross_entry_fwd_then_decode():
