@@ -90,7 +90,7 @@ void plan_generic(int64_t batch, int64_t seqlen, int64_t dim, selscan::FwdPlan *
 }
 
 // Plan of the TMA kernel. Groups = batch rows × 128-channel tiles. With at
-// least ~60% as many groups as SMs: one pass, units of kUnit tokens handed
+// least ~60% as many groups as SMs: one pass, units of 1024 tokens handed
 // from chunk to chunk (kModeSeq). With fewer: chunk aggregates, carry and
 // rescan, with about 8 units per SM. SELSCAN_PATH=seq|chunked, SELSCAN_UNIT
 // and SELSCAN_CHUNKS override (tuning only).
@@ -107,7 +107,7 @@ void plan_tma(int64_t batch, int64_t seqlen, int64_t dim, bool bf16, selscan::Fw
     int64_t len = 0;
     if (seq) {
         len = env_int("SELSCAN_UNIT");
-        if (len <= 0) len = 512;
+        if (len <= 0) len = 1024;
     } else {
         int64_t n = env_int("SELSCAN_CHUNKS");
         if (n <= 0) n = (8 * sms + groups - 1) / groups;
@@ -134,7 +134,7 @@ void plan_tma(int64_t batch, int64_t seqlen, int64_t dim, bool bf16, selscan::Fw
     // workspace: [0, 256) tickets; SEQ: flags at 256, states after them;
     // chunked: P and H arrays from 256.
     if (seq) {
-        const size_t flags_end = round_up(256 + 4 * 4 * groups, 256);  // one per warp
+        const size_t flags_end = round_up(256 + 4 * 8 * groups, 256);  // one per warp
         pl->ws_clear = flags_end;
         pl->ws_bytes = flags_end + (size_t)groups * cpt * selscan::kMaxN * sizeof(float);
     } else {
@@ -160,9 +160,10 @@ void plan_for_sizes(int64_t batch, int64_t seqlen, int64_t dim, int64_t dstate, 
     const char *path = getenv("SELSCAN_PATH");
     const bool forced_generic = path && !strcmp(path, "generic");
     // TMA rows must start on 16-byte boundaries and tiles are 128 channels.
+    // B/C rows are TMA'd too: dstate·elem must be a multiple of 16 bytes.
     const bool eligible = aligned && !forced_generic && dim >= tma_tile_channels() &&
-                          (dim * es) % 16 == 0 && batch * seqlen < ((int64_t)1 << 31) &&
-                          dstate <= kMaxN;
+                          (dim * es) % 16 == 0 && (dstate * es) % 16 == 0 &&
+                          batch * seqlen < ((int64_t)1 << 31) && dstate <= kMaxN;
     pl->bf16 = bf16;
     if (eligible)
         plan_tma(batch, seqlen, dim, bf16, pl);
@@ -217,7 +218,8 @@ int fwd_setup(const void *x, const void *delta, const float *A, const void *B,
         return SELSCAN_OK;
     }
 
-    const bool aligned = !misaligned(x, 16) && !misaligned(delta, 16) && !misaligned(z, 16);
+    const bool aligned = !misaligned(x, 16) && !misaligned(delta, 16) && !misaligned(z, 16) &&
+                         !misaligned(B, 16) && !misaligned(C, 16);
     plan_for_sizes(batch, seqlen, dim, dstate, dtype, aligned, plan);
     plan->x = x;
     plan->delta = delta;

@@ -40,13 +40,23 @@ namespace selscan {
 namespace {
 
 constexpr int kConsumerWarps = 4;
-constexpr int kChannels = 32 * kConsumerWarps;  // channels per tile
+constexpr int kChannels = 32 * kConsumerWarps;  // channels per tile (one per consumer thread)
 constexpr int kBlock = kChannels + 32;          // + producer warp
+constexpr int kMaxConsumerWarps = 8;            // flags per group in the workspace
 #ifndef SELSCAN_TMA_STAGES
 #define SELSCAN_TMA_STAGES 4
 #endif
 #ifndef SELSCAN_TMA_KSUB
 #define SELSCAN_TMA_KSUB 8
+#endif
+#ifndef SELSCAN_TMA_YTREE
+#define SELSCAN_TMA_YTREE 0
+#endif
+#ifndef SELSCAN_TMA_LATESTORE
+#define SELSCAN_TMA_LATESTORE 0
+#endif
+#ifndef SELSCAN_TMA_SCALAR
+#define SELSCAN_TMA_SCALAR 0
 #endif
 constexpr int kStages = SELSCAN_TMA_STAGES;
 constexpr int kSub = SELSCAN_TMA_KSUB;  // tokens per register sub-tile
@@ -60,9 +70,34 @@ template <typename T> struct alignas(128) Stage {
     T x[kTile][kChannels];
     T dl[kTile][kChannels];
     T z[kTile][kChannels];
-    float B[kTile][kMaxN];
+    T Bs[kTile * kMaxN];  // TMA destination: the tile's B rows, dstate per row
+    T Cs[kTile * kMaxN];
+    float B[kTile][kMaxN];  // float32 copies read by the consumers (zero padded)
     float C[kTile][kMaxN];
 };
+
+// Two-lane float32 arithmetic: packed f32x2 instructions, or two scalar ones.
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
+#if SELSCAN_TMA_SCALAR
+    return make_float2(a.x * b.x, a.y * b.y);
+#else
+    return __fmul2_rn(a, b);
+#endif
+}
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+#if SELSCAN_TMA_SCALAR
+    return make_float2(fmaf(a.x, b.x, c.x), fmaf(a.y, b.y, c.y));
+#else
+    return __ffma2_rn(a, b, c);
+#endif
+}
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+#if SELSCAN_TMA_SCALAR
+    return make_float2(a.x + b.x, a.y + b.y);
+#else
+    return __fadd2_rn(a, b);
+#endif
+}
 
 enum : int { kFirst = 1, kLast = 2, kEnd = 4 };
 
@@ -74,8 +109,9 @@ struct TileInfo {
 template <typename T> struct alignas(128) Shared {
     Stage<T> stage[kStages];
     TileInfo info[kStages];
-    uint64_t full[kStages];
-    uint64_t empty[kStages];
+    uint64_t full[kStages];   // x/delta/z bytes + 32 producer arrivals (after B/C conversion)
+    uint64_t empty[kStages];  // one arrival per consumer warp
+    uint64_t bc[kStages];     // B/C TMA bytes of the stage
     int abort;
 };
 
@@ -99,107 +135,134 @@ __device__ __forceinline__ void fail(const TmaScanParams &p, int *abort, int cod
 }
 
 // ---- producer warp -----------------------------------------------------------------
+// Converts the B and C rows of stage s (landed by TMA as the I/O type, dstate
+// per row) to float32 [kTile][16], zero for rows past nt and states past
+// dstate. Lane l handles float4 slots l, l + 32, ...: consecutive lanes write
+// consecutive 16-byte chunks.
+template <typename T>
+__device__ __forceinline__ void convert_bc(Stage<T> &st, int nt, int dstate, int lane) {
+    constexpr int kTile = TileCfg<T>::kTile;
+    constexpr int kSlots = kTile * kMaxN / 4;
+#pragma unroll
+    for (int i = lane; i < kSlots; i += 32) {
+        const int t = i / (kMaxN / 4);
+        const int n0 = (i % (kMaxN / 4)) * 4;
+        float vb[4], vc[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const bool ok = t < nt && n0 + e < dstate;
+            vb[e] = ok ? to_f32(st.Bs[t * dstate + n0 + e]) : 0.0f;
+            vc[e] = ok ? to_f32(st.Cs[t * dstate + n0 + e]) : 0.0f;
+        }
+        reinterpret_cast<float4 *>(&st.B[0][0])[i] = make_float4(vb[0], vb[1], vb[2], vb[3]);
+        reinterpret_cast<float4 *>(&st.C[0][0])[i] = make_float4(vc[0], vc[1], vc[2], vc[3]);
+    }
+}
+
+// The producer issues every TMA of a stage as soon as the stage is free and
+// converts its B/C kLag stages later, so it never waits on global memory
+// latency itself; the stage is handed to the consumers (32 arrivals on
+// `full`) after its conversion.
 template <typename T, bool kGate>
 __device__ void produce(Shared<T> &S, const TmaScanParams &p, const CUtensorMap *tm_x,
-                        const CUtensorMap *tm_d, const CUtensorMap *tm_z) {
+                        const CUtensorMap *tm_d, const CUtensorMap *tm_z,
+                        const CUtensorMap *tm_b, const CUtensorMap *tm_c) {
     constexpr int kTile = TileCfg<T>::kTile;
+    constexpr int kLag = kStages > 2 ? 2 : 1;
     const int lane = threadIdx.x & 31;
     if (lane == 0) {
         prefetch_tmap(tm_x);
         prefetch_tmap(tm_d);
         if (kGate) prefetch_tmap(tm_z);
+        prefetch_tmap(tm_b);
+        prefetch_tmap(tm_c);
     }
     constexpr uint32_t kTileBytes = kTile * kChannels * sizeof(T);
     const uint32_t tx_bytes = (kGate ? 3u : 2u) * kTileBytes;
-    const T *Bp = static_cast<const T *>(p.B);
-    const T *Cp = static_cast<const T *>(p.C);
-    int s = 0;
+    const uint32_t bc_bytes = 2u * kTile * p.dstate * sizeof(T);
+    int s = 0;                 // next stage to fill
     uint32_t phase = 0;
-    uint32_t issued = 0;  // bit i: stage i has a TMA issued with parity bit (16 + i)
+    int cs = 0;                // oldest stage awaiting conversion
+    uint32_t cphase = 0;
+    int npend = 0;             // stages issued but not yet converted / handed over
+
+    // converts the oldest pending stage and hands it to the consumers
+    auto convert_oldest = [&]() -> bool {
+        if (!mbar_wait(&S.bc[cs], cphase, &S.abort, p.timeout_ns)) return false;
+        convert_bc<T>(S.stage[cs], S.info[cs].nt, p.dstate, lane);
+        __syncwarp();
+        mbar_arrive(&S.full[cs]);
+        if (++cs == kStages) {
+            cs = 0;
+            cphase ^= 1u;
+        }
+        --npend;
+        return true;
+    };
+    // failure: record it, then wait (bounded) for this warp's copies in flight
+    auto bail = [&]() {
+        if (lane == 0) fail(p, &S.abort, 2);
+        for (; npend > 0; --npend) {
+            mbar_wait(&S.bc[cs], cphase, &kNoAbort, p.timeout_ns / 16);
+            mbar_arrive(&S.full[cs]);
+            mbar_wait(&S.full[cs], cphase, &kNoAbort, p.timeout_ns / 16);
+            if (++cs == kStages) {
+                cs = 0;
+                cphase ^= 1u;
+            }
+        }
+        __syncwarp();
+    };
+
     for (;;) {
         int ticket = 0;
         if (lane == 0) ticket = atomicAdd(p.ticket, 1);
         ticket = __shfl_sync(0xffffffffu, ticket, 0);
         const bool end = ticket >= p.units;
-        long long b = 0, t_begin = 0, t_end = 0;
-        int tile = 0, chunk = 0, ntl = 1;
-        if (!end) {
-            const long long g = ticket % p.groups;
-            chunk = (int)(ticket / p.groups);
-            b = g / p.ntiles;
-            tile = (int)(g % p.ntiles);
-            t_begin = (long long)chunk * p.chunk_len;
-            t_end = min(t_begin + p.chunk_len, (long long)p.seqlen);
-            ntl = (int)((t_end - t_begin + kTile - 1) / kTile);
+        if (end) {
+            while (npend > 0)
+                if (!convert_oldest()) return bail();
+            if (!mbar_wait(&S.empty[s], phase ^ 1u, &S.abort, p.timeout_ns)) return bail();
+            if (lane == 0) S.info[s].flags = kEnd;
+            __syncwarp();
+            mbar_arrive(&S.full[s]);
+            return;
         }
+        const long long g = ticket % p.groups;
+        const int chunk = (int)(ticket / p.groups);
+        const long long b = g / p.ntiles;
+        const int tile = (int)(g % p.ntiles);
+        const long long t_begin = (long long)chunk * p.chunk_len;
+        const long long t_end = min(t_begin + p.chunk_len, (long long)p.seqlen);
+        const int ntl = (int)((t_end - t_begin + kTile - 1) / kTile);
         for (int j = 0; j < ntl; ++j) {
-            if (!mbar_wait(&S.empty[s], phase ^ 1u, &S.abort, p.timeout_ns)) {
-                if (lane == 0) {
-                    fail(p, &S.abort, 2);
-                    // wait (bounded) for this warp's own copies still in flight
-                    for (int i = 0; i < kStages; ++i)
-                        if (issued & (1u << i))
-                            mbar_wait(&S.full[i], (issued >> (16 + i)) & 1u, &kNoAbort,
-                                      p.timeout_ns / 16);
-                }
-                __syncwarp();
-                return;
-            }
+            if (!mbar_wait(&S.empty[s], phase ^ 1u, &S.abort, p.timeout_ns)) return bail();
             const long long t0 = t_begin + (long long)j * kTile;
-            const int nt = end ? 0 : (int)min((long long)kTile, t_end - t0);
             if (lane == 0) {
                 TileInfo &inf = S.info[s];
                 inf.b = b;
                 inf.t0 = t0;
                 inf.tile = tile;
                 inf.chunk = chunk;
-                inf.nt = nt;
-                inf.flags = end ? kEnd : ((j == 0 ? kFirst : 0) | (j == ntl - 1 ? kLast : 0));
-                if (!end) {
-                    mbar_expect_tx(&S.full[s], tx_bytes);
-                    const int c0 = tile * kChannels;
-                    const int c1 = (int)(b * p.seqlen + t0);
-                    tma_load_2d(&S.stage[s].x[0][0], tm_x, &S.full[s], c0, c1);
-                    tma_load_2d(&S.stage[s].dl[0][0], tm_d, &S.full[s], c0, c1);
-                    if (kGate) tma_load_2d(&S.stage[s].z[0][0], tm_z, &S.full[s], c0, c1);
-                    issued = (issued | (1u << s)) & ~(1u << (16 + s));
-                    issued |= phase << (16 + s);
-                }
-            }
-            if (!end) {
-                // B and C rows of the tile as float32; rows past the tile's
-                // tokens and states past dstate are zero.
-                const int row = lane % kTile;
-                const bool isC = lane >= kTile;  // only when kTile == 16
-                for (int r = row; r < kTile; r += 32) {
-                    const bool in = r < nt;
-                    const long long gi = (b * p.seqlen + t0 + r) * p.dstate;
-                    float vb[kMaxN], vc[kMaxN];
-#pragma unroll
-                    for (int n = 0; n < kMaxN; ++n) {
-                        const bool ok = in && n < p.dstate;
-                        vb[n] = (ok && (kTile == 32 || !isC)) ? ldg_f32(Bp + gi + n) : 0.0f;
-                        vc[n] = (ok && (kTile == 32 || isC)) ? ldg_f32(Cp + gi + n) : 0.0f;
-                    }
-                    float4 *db = reinterpret_cast<float4 *>(&S.stage[s].B[r][0]);
-                    float4 *dc = reinterpret_cast<float4 *>(&S.stage[s].C[r][0]);
-#pragma unroll
-                    for (int q = 0; q < kMaxN / 4; ++q) {
-                        if (kTile == 32 || !isC)
-                            db[q] = make_float4(vb[4 * q], vb[4 * q + 1], vb[4 * q + 2], vb[4 * q + 3]);
-                        if (kTile == 32 || isC)
-                            dc[q] = make_float4(vc[4 * q], vc[4 * q + 1], vc[4 * q + 2], vc[4 * q + 3]);
-                    }
-                }
+                inf.nt = (int)min((long long)kTile, t_end - t0);
+                inf.flags = (j == 0 ? kFirst : 0) | (j == ntl - 1 ? kLast : 0);
+                const int c1 = (int)(b * p.seqlen + t0);
+                mbar_expect_tx(&S.full[s], tx_bytes);
+                tma_load_2d(&S.stage[s].x[0][0], tm_x, &S.full[s], tile * kChannels, c1);
+                tma_load_2d(&S.stage[s].dl[0][0], tm_d, &S.full[s], tile * kChannels, c1);
+                if (kGate) tma_load_2d(&S.stage[s].z[0][0], tm_z, &S.full[s], tile * kChannels, c1);
+                mbar_arrive_expect_tx(&S.bc[s], bc_bytes);
+                tma_load_2d(&S.stage[s].Bs[0], tm_b, &S.bc[s], 0, c1);
+                tma_load_2d(&S.stage[s].Cs[0], tm_c, &S.bc[s], 0, c1);
             }
             __syncwarp();
-            mbar_arrive(&S.full[s]);
             if (++s == kStages) {
                 s = 0;
                 phase ^= 1u;
             }
+            if (++npend > kLag)
+                if (!convert_oldest()) return bail();
         }
-        if (end) return;
     }
 }
 
@@ -212,10 +275,10 @@ __device__ __forceinline__ float softplus_fast(float v) {
     return v > 15.0f ? v : s;
 }
 
-template <typename T, bool kGate, int kMode, bool kStruct>
+template <typename T, bool kGate, int kMode, bool kStruct, bool kSoftplus>
 __device__ __forceinline__ void consume_tile(const Stage<T> &st, int nt, float2 (&h)[kMaxN / 2],
                                              const float (&A2)[kMaxN], float dskip, float bias,
-                                             int softplus, float &dt_sum, T *yp, long long ybase,
+                                             float &dt_sum, T *yp, long long ybase,
                                              long long ystride, bool active) {
     constexpr int kTile = TileCfg<T>::kTile;
     constexpr bool kFastSp = sizeof(T) == 2;
@@ -231,7 +294,7 @@ __device__ __forceinline__ void consume_tile(const Stage<T> &st, int nt, float2 
             const bool valid = t < nt;
             const float xv = to_f32(st.x[t][c]);
             float dt = to_f32(st.dl[t][c]) + bias;
-            if (softplus) dt = kFastSp ? softplus_fast(dt) : softplus_f32(dt);
+            if (kSoftplus) dt = kFastSp ? softplus_fast(dt) : softplus_f32(dt);
             dt = valid ? dt : 0.0f;  // Abar = 1, no input: the state is unchanged
             uu[k] = dt * xv;
             rr[k] = kStruct ? ex2_approx(dt * A2[0]) : dt;
@@ -252,15 +315,15 @@ __device__ __forceinline__ void consume_tile(const Stage<T> &st, int nt, float2 
                 const float r = rr[k];
                 const float r2 = r * r;
                 a[0] = make_float2(r, r2);
-                a[1] = __fmul2_rn(a[0], make_float2(r2, r2));
+                a[1] = mul2(a[0], make_float2(r2, r2));
                 const float r4 = a[1].y;
                 const float2 q4 = make_float2(r4, r4);
-                a[2] = __fmul2_rn(a[0], q4);
-                a[3] = __fmul2_rn(a[1], q4);
+                a[2] = mul2(a[0], q4);
+                a[3] = mul2(a[1], q4);
                 const float r8 = a[3].y;
                 const float2 q8 = make_float2(r8, r8);
 #pragma unroll
-                for (int j = 0; j < 4; ++j) a[4 + j] = __fmul2_rn(a[j], q8);
+                for (int j = 0; j < 4; ++j) a[4 + j] = mul2(a[j], q8);
             } else {
 #pragma unroll
                 for (int j = 0; j < kMaxN / 2; ++j)
@@ -273,32 +336,67 @@ __device__ __forceinline__ void consume_tile(const Stage<T> &st, int nt, float2 
 #pragma unroll
                 for (int q = 0; q < kMaxN / 4; ++q) {
                     const float4 bq = B4[q];
-                    h[2 * q] = __ffma2_rn(a[2 * q], h[2 * q], __fmul2_rn(u2, make_float2(bq.x, bq.y)));
+                    h[2 * q] = fma2(a[2 * q], h[2 * q], mul2(u2, make_float2(bq.x, bq.y)));
                     h[2 * q + 1] =
-                        __ffma2_rn(a[2 * q + 1], h[2 * q + 1], __fmul2_rn(u2, make_float2(bq.z, bq.w)));
+                        fma2(a[2 * q + 1], h[2 * q + 1], mul2(u2, make_float2(bq.z, bq.w)));
                 }
             } else {
                 const float4 *C4 = reinterpret_cast<const float4 *>(&st.C[t][0]);
+#if SELSCAN_TMA_YTREE
+                float2 acc[4];
+#pragma unroll
+                for (int q = 0; q < kMaxN / 4; ++q) {
+                    const float4 bq = B4[q];
+                    h[2 * q] = fma2(a[2 * q], h[2 * q], mul2(u2, make_float2(bq.x, bq.y)));
+                    h[2 * q + 1] =
+                        fma2(a[2 * q + 1], h[2 * q + 1], mul2(u2, make_float2(bq.z, bq.w)));
+                }
+#pragma unroll
+                for (int q = 0; q < 2; ++q) {
+                    const float4 cq = C4[q];
+                    acc[2 * q] = mul2(make_float2(cq.x, cq.y), h[2 * q]);
+                    acc[2 * q + 1] = mul2(make_float2(cq.z, cq.w), h[2 * q + 1]);
+                }
+#pragma unroll
+                for (int q = 2; q < 4; ++q) {
+                    const float4 cq = C4[q];
+                    acc[2 * q - 4] = fma2(make_float2(cq.x, cq.y), h[2 * q], acc[2 * q - 4]);
+                    acc[2 * q - 3] = fma2(make_float2(cq.z, cq.w), h[2 * q + 1], acc[2 * q - 3]);
+                }
+                const float2 ys = add2(add2(acc[0], acc[1]), add2(acc[2], acc[3]));
+#else
                 float2 y0 = make_float2(0.0f, 0.0f), y1 = y0;
 #pragma unroll
                 for (int q = 0; q < kMaxN / 4; ++q) {
                     const float4 bq = B4[q];
                     const float4 cq = C4[q];
-                    h[2 * q] = __ffma2_rn(a[2 * q], h[2 * q], __fmul2_rn(u2, make_float2(bq.x, bq.y)));
+                    h[2 * q] = fma2(a[2 * q], h[2 * q], mul2(u2, make_float2(bq.x, bq.y)));
                     h[2 * q + 1] =
-                        __ffma2_rn(a[2 * q + 1], h[2 * q + 1], __fmul2_rn(u2, make_float2(bq.z, bq.w)));
-                    y0 = __ffma2_rn(make_float2(cq.x, cq.y), h[2 * q], y0);
-                    y1 = __ffma2_rn(make_float2(cq.z, cq.w), h[2 * q + 1], y1);
+                        fma2(a[2 * q + 1], h[2 * q + 1], mul2(u2, make_float2(bq.z, bq.w)));
+                    y0 = fma2(make_float2(cq.x, cq.y), h[2 * q], y0);
+                    y1 = fma2(make_float2(cq.z, cq.w), h[2 * q + 1], y1);
                 }
-                const float2 ys = __fadd2_rn(y0, y1);
+                const float2 ys = add2(y0, y1);
+#endif
                 const float out = fmaf(ys.x + ys.y, gg[k], pp[k]);
+#if SELSCAN_TMA_LATESTORE
+                gg[k] = out;
+#else
                 if (active && t < nt) yp[ybase + (long long)t * ystride] = from_f32<T>(out);
+#endif
             }
         }
+#if SELSCAN_TMA_LATESTORE
+        if (kMode != kModeAgg) {
+#pragma unroll
+            for (int k = 0; k < kSub; ++k)
+                if (active && sub + k < nt) yp[ybase + (long long)(sub + k) * ystride] = from_f32<T>(gg[k]);
+        }
+#endif
     }
 }
 
-template <typename T, bool kGate, int kMode>
+template <typename T, bool kGate, int kMode, bool kSoftplus>
 __device__ void consume(Shared<T> &S, const TmaScanParams &p) {
     const int c = threadIdx.x;  // 0..127
     const int lane = c & 31;
@@ -351,7 +449,7 @@ __device__ void consume(Shared<T> &S, const TmaScanParams &p) {
             for (int n = 0; n < kMaxN; ++n) hs[n] = 0.0f;
             if (kMode == kModeSeq && inf.chunk > 0) {
                 // every lane acquires this warp's predecessor flag (bounded)
-                const int *flag = p.flags + g * kConsumerWarps + (c >> 5);
+                const int *flag = p.flags + g * kMaxConsumerWarps + (c >> 5);
                 const uint64_t start = global_ns();
                 while (ld_acquire_gpu(flag) < inf.chunk) {
                     __nanosleep(64);
@@ -382,11 +480,11 @@ __device__ void consume(Shared<T> &S, const TmaScanParams &p) {
 
         const long long ybase = (inf.b * p.seqlen + inf.t0) * p.dim + d;
         if (structured)
-            consume_tile<T, kGate, kMode, true>(S.stage[s], inf.nt, h, A2, dskip, bias, p.softplus,
-                                                dt_sum, yp, ybase, p.dim, active);
+            consume_tile<T, kGate, kMode, true, kSoftplus>(S.stage[s], inf.nt, h, A2, dskip, bias,
+                                                           dt_sum, yp, ybase, p.dim, active);
         else
-            consume_tile<T, kGate, kMode, false>(S.stage[s], inf.nt, h, A2, dskip, bias, p.softplus,
-                                                 dt_sum, yp, ybase, p.dim, active);
+            consume_tile<T, kGate, kMode, false, kSoftplus>(S.stage[s], inf.nt, h, A2, dskip, bias,
+                                                            dt_sum, yp, ybase, p.dim, active);
 
         if (inf.flags & kLast) {
             const bool last_chunk = inf.chunk == p.nchunks - 1;
@@ -420,7 +518,8 @@ __device__ void consume(Shared<T> &S, const TmaScanParams &p) {
                 }
                 __threadfence();
                 __syncwarp();
-                if (lane == 0) st_release_gpu(p.flags + g * kConsumerWarps + (c >> 5), inf.chunk + 1);
+                if (lane == 0)
+                    st_release_gpu(p.flags + g * kMaxConsumerWarps + (c >> 5), inf.chunk + 1);
             }
         }
         __syncwarp();
@@ -432,10 +531,11 @@ __device__ void consume(Shared<T> &S, const TmaScanParams &p) {
     }
 }
 
-template <typename T, bool kGate, int kMode>
+template <typename T, bool kGate, int kMode, bool kSoftplus>
 __global__ void __launch_bounds__(kBlock, 1)
 scan_tma_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_d,
-                const __grid_constant__ CUtensorMap tm_z, const TmaScanParams p) {
+                const __grid_constant__ CUtensorMap tm_z, const __grid_constant__ CUtensorMap tm_b,
+                const __grid_constant__ CUtensorMap tm_c, const TmaScanParams p) {
     // Indexed straight off the __shared__ array so that every access compiles
     // to a shared-memory instruction (no generic addressing, no aliasing with
     // the global y stores).
@@ -445,15 +545,16 @@ scan_tma_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
         for (int i = 0; i < kStages; ++i) {
             mbar_init(&S.full[i], 32);              // producer lanes (+ TMA bytes)
             mbar_init(&S.empty[i], kConsumerWarps);  // one arrival per consumer warp
+            mbar_init(&S.bc[i], 1);
         }
         S.abort = 0;
         fence_barrier_init();
     }
     __syncthreads();
     if (threadIdx.x >= kChannels)
-        produce<T, kGate>(S, p, &tm_x, &tm_d, &tm_z);
+        produce<T, kGate>(S, p, &tm_x, &tm_d, &tm_z, &tm_b, &tm_c);
     else
-        consume<T, kGate, kMode>(S, p);
+        consume<T, kGate, kMode, kSoftplus>(S, p);
 }
 
 // ---- host side -----------------------------------------------------------------------
@@ -470,15 +571,18 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
+// 2-D map over a row-major [rows][cols] tensor with boxes of
+// box_cols × TileCfg<T>::kTile rows.
 template <typename T>
-bool make_map(CUtensorMap *m, const void *base, long long rows, long long dim) {
+bool make_map(CUtensorMap *m, const void *base, long long rows, long long cols,
+              int box_cols = kChannels) {
     auto fn = encode_fn();
     if (!fn) return false;
     const CUtensorMapDataType dt = sizeof(T) == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
                                                   : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
-    cuuint64_t gdim[2] = {(cuuint64_t)dim, (cuuint64_t)rows};
-    cuuint64_t gstride[1] = {(cuuint64_t)(dim * sizeof(T))};
-    cuuint32_t box[2] = {(cuuint32_t)kChannels, (cuuint32_t)TileCfg<T>::kTile};
+    cuuint64_t gdim[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t gstride[1] = {(cuuint64_t)(cols * sizeof(T))};
+    cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)TileCfg<T>::kTile};
     cuuint32_t estride[2] = {1, 1};
     CUresult r = fn(m, dt, 2, const_cast<void *>(base), gdim, gstride, box, estride,
                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
@@ -493,13 +597,15 @@ int num_sms() {
     return sms > 0 ? sms : 148;
 }
 
-template <typename T, bool kGate, int kMode>
+template <typename T, bool kGate, int kMode, bool kSoftplus>
 cudaError_t launch_mode(const TmaScanParams &p, const void *x, const void *dl, const void *z,
                         cudaStream_t stream) {
     if (p.units <= 0) return cudaSuccess;
-    CUtensorMap mx, md, mz;
+    CUtensorMap mx, md, mz, mb, mc;
     const long long rows = p.batch * p.seqlen;
-    if (!make_map<T>(&mx, x, rows, p.dim) || !make_map<T>(&md, dl, rows, p.dim))
+    if (!make_map<T>(&mx, x, rows, p.dim) || !make_map<T>(&md, dl, rows, p.dim) ||
+        !make_map<T>(&mb, p.B, rows, p.dstate, p.dstate) ||
+        !make_map<T>(&mc, p.C, rows, p.dstate, p.dstate))
         return cudaErrorInvalidValue;
     if (kGate) {
         if (!make_map<T>(&mz, z, rows, p.dim)) return cudaErrorInvalidValue;
@@ -507,23 +613,30 @@ cudaError_t launch_mode(const TmaScanParams &p, const void *x, const void *dl, c
         mz = md;
     }
     const size_t smem = sizeof(Shared<T>);
-    auto kern = scan_tma_kernel<T, kGate, kMode>;
+    auto kern = scan_tma_kernel<T, kGate, kMode, kSoftplus>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
     const long long grid = min((long long)num_sms(), (long long)p.units);
-    kern<<<(unsigned)grid, kBlock, smem, stream>>>(mx, md, mz, p);
+    kern<<<(unsigned)grid, kBlock, smem, stream>>>(mx, md, mz, mb, mc, p);
     return cudaGetLastError();
+}
+
+template <typename T, bool kGate, bool kSoftplus>
+cudaError_t launch_sp(const TmaScanParams &p, const void *x, const void *dl, const void *z,
+                      cudaStream_t stream) {
+    switch (p.mode) {
+    case kModeSeq: return launch_mode<T, kGate, kModeSeq, kSoftplus>(p, x, dl, z, stream);
+    case kModeAgg: return launch_mode<T, false, kModeAgg, kSoftplus>(p, x, dl, z, stream);
+    default: return launch_mode<T, kGate, kModeRescan, kSoftplus>(p, x, dl, z, stream);
+    }
 }
 
 template <typename T, bool kGate>
 cudaError_t launch_gate(const TmaScanParams &p, const void *x, const void *dl, const void *z,
                         cudaStream_t stream) {
-    switch (p.mode) {
-    case kModeSeq: return launch_mode<T, kGate, kModeSeq>(p, x, dl, z, stream);
-    case kModeAgg: return launch_mode<T, false, kModeAgg>(p, x, dl, z, stream);
-    default: return launch_mode<T, kGate, kModeRescan>(p, x, dl, z, stream);
-    }
+    return p.softplus ? launch_sp<T, kGate, true>(p, x, dl, z, stream)
+                      : launch_sp<T, kGate, false>(p, x, dl, z, stream);
 }
 
 }  // namespace

@@ -36,6 +36,13 @@ __device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes) {
                  : "memory");
 }
 
+// Arrival that also adds `bytes` to the transaction count of the phase.
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+
 // Arrival with release semantics (the caller's prior writes are visible to
 // whoever completes a wait on this phase).
 __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
