@@ -219,7 +219,7 @@ int fwd_setup(const void *x, const void *delta, const float *A, const void *B,
     }
 
     const bool aligned = !misaligned(x, 16) && !misaligned(delta, 16) && !misaligned(z, 16) &&
-                         !misaligned(B, 16) && !misaligned(C, 16);
+                         !misaligned(B, 16) && !misaligned(C, 16) && !misaligned(y, 16);
     plan_for_sizes(batch, seqlen, dim, dstate, dtype, aligned, plan);
     plan->x = x;
     plan->delta = delta;

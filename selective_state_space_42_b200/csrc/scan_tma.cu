@@ -33,6 +33,8 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <atomic>
+
 #include "selscan_device.cuh"
 #include "tma_util.cuh"
 
@@ -48,15 +50,6 @@ constexpr int kMaxConsumerWarps = 8;            // flags per group in the worksp
 #endif
 #ifndef SELSCAN_TMA_KSUB
 #define SELSCAN_TMA_KSUB 8
-#endif
-#ifndef SELSCAN_TMA_YTREE
-#define SELSCAN_TMA_YTREE 0
-#endif
-#ifndef SELSCAN_TMA_LATESTORE
-#define SELSCAN_TMA_LATESTORE 0
-#endif
-#ifndef SELSCAN_TMA_SCALAR
-#define SELSCAN_TMA_SCALAR 0
 #endif
 constexpr int kStages = SELSCAN_TMA_STAGES;
 constexpr int kSub = SELSCAN_TMA_KSUB;  // tokens per register sub-tile
@@ -76,28 +69,11 @@ template <typename T> struct alignas(128) Stage {
     float C[kTile][kMaxN];
 };
 
-// Two-lane float32 arithmetic: packed f32x2 instructions, or two scalar ones.
-__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
-#if SELSCAN_TMA_SCALAR
-    return make_float2(a.x * b.x, a.y * b.y);
-#else
-    return __fmul2_rn(a, b);
-#endif
-}
-__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
-#if SELSCAN_TMA_SCALAR
-    return make_float2(fmaf(a.x, b.x, c.x), fmaf(a.y, b.y, c.y));
-#else
-    return __ffma2_rn(a, b, c);
-#endif
-}
-__device__ __forceinline__ float2 add2(float2 a, float2 b) {
-#if SELSCAN_TMA_SCALAR
-    return make_float2(a.x + b.x, a.y + b.y);
-#else
-    return __fadd2_rn(a, b);
-#endif
-}
+// Two-lane float32 arithmetic (packed f32x2 instructions: one issue slot
+// for two lanes of work).
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+__device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
 
 enum : int { kFirst = 1, kLast = 2, kEnd = 4 };
 
@@ -106,8 +82,12 @@ struct TileInfo {
     int tile, chunk, nt, flags;
 };
 
+constexpr int kYBufs = 2;  // y staging tiles per consumer warp (TMA stores in flight)
+
 template <typename T> struct alignas(128) Shared {
     Stage<T> stage[kStages];
+    // per consumer warp: y of its 32 channels for one full tile, [kTile][32]
+    alignas(128) T ybuf[kConsumerWarps][kYBufs][TileCfg<T>::kTile * 32];
     TileInfo info[kStages];
     uint64_t full[kStages];   // x/delta/z bytes + 32 producer arrivals (after B/C conversion)
     uint64_t empty[kStages];  // one arrival per consumer warp
@@ -275,27 +255,31 @@ __device__ __forceinline__ float softplus_fast(float v) {
     return v > 15.0f ? v : s;
 }
 
-template <typename T, bool kGate, int kMode, bool kStruct, bool kSoftplus>
+// One ring stage for this thread's channel. kFull: the stage holds kTile
+// valid tokens and y goes to this warp's shared-memory tile `ys` (written to
+// global memory by one TMA store per warp); otherwise tokens past nt leave
+// the state unchanged and y goes straight to global memory.
+template <typename T, bool kGate, int kMode, bool kStruct, bool kSoftplus, bool kFull>
 __device__ __forceinline__ void consume_tile(const Stage<T> &st, int nt, float2 (&h)[kMaxN / 2],
                                              const float (&A2)[kMaxN], float dskip, float bias,
-                                             float &dt_sum, T *yp, long long ybase,
+                                             float &dt_sum, T *ys, T *yp, long long ybase,
                                              long long ystride, bool active) {
     constexpr int kTile = TileCfg<T>::kTile;
     constexpr bool kFastSp = sizeof(T) == 2;
     const int c = threadIdx.x;  // channel within the tile
+    const int lane = c & 31;
 #pragma unroll 1
     for (int sub = 0; sub < kTile; sub += kSub) {
-        if (sub >= nt) break;
+        if (!kFull && sub >= nt) break;
         float uu[kSub], rr[kSub], gg[kSub], pp[kSub];
         // per-token scalars
 #pragma unroll
         for (int k = 0; k < kSub; ++k) {
             const int t = sub + k;
-            const bool valid = t < nt;
             const float xv = to_f32(st.x[t][c]);
             float dt = to_f32(st.dl[t][c]) + bias;
             if (kSoftplus) dt = kFastSp ? softplus_fast(dt) : softplus_f32(dt);
-            dt = valid ? dt : 0.0f;  // Abar = 1, no input: the state is unchanged
+            if (!kFull) dt = t < nt ? dt : 0.0f;  // Abar = 1, no input: state unchanged
             uu[k] = dt * xv;
             rr[k] = kStruct ? ex2_approx(dt * A2[0]) : dt;
             if (kMode == kModeAgg) {
@@ -337,69 +321,43 @@ __device__ __forceinline__ void consume_tile(const Stage<T> &st, int nt, float2 
                 for (int q = 0; q < kMaxN / 4; ++q) {
                     const float4 bq = B4[q];
                     h[2 * q] = fma2(a[2 * q], h[2 * q], mul2(u2, make_float2(bq.x, bq.y)));
-                    h[2 * q + 1] =
-                        fma2(a[2 * q + 1], h[2 * q + 1], mul2(u2, make_float2(bq.z, bq.w)));
+                    h[2 * q + 1] = fma2(a[2 * q + 1], h[2 * q + 1], mul2(u2, make_float2(bq.z, bq.w)));
                 }
             } else {
                 const float4 *C4 = reinterpret_cast<const float4 *>(&st.C[t][0]);
-#if SELSCAN_TMA_YTREE
-                float2 acc[4];
-#pragma unroll
-                for (int q = 0; q < kMaxN / 4; ++q) {
-                    const float4 bq = B4[q];
-                    h[2 * q] = fma2(a[2 * q], h[2 * q], mul2(u2, make_float2(bq.x, bq.y)));
-                    h[2 * q + 1] =
-                        fma2(a[2 * q + 1], h[2 * q + 1], mul2(u2, make_float2(bq.z, bq.w)));
-                }
-#pragma unroll
-                for (int q = 0; q < 2; ++q) {
-                    const float4 cq = C4[q];
-                    acc[2 * q] = mul2(make_float2(cq.x, cq.y), h[2 * q]);
-                    acc[2 * q + 1] = mul2(make_float2(cq.z, cq.w), h[2 * q + 1]);
-                }
-#pragma unroll
-                for (int q = 2; q < 4; ++q) {
-                    const float4 cq = C4[q];
-                    acc[2 * q - 4] = fma2(make_float2(cq.x, cq.y), h[2 * q], acc[2 * q - 4]);
-                    acc[2 * q - 3] = fma2(make_float2(cq.z, cq.w), h[2 * q + 1], acc[2 * q - 3]);
-                }
-                const float2 ys = add2(add2(acc[0], acc[1]), add2(acc[2], acc[3]));
-#else
                 float2 y0 = make_float2(0.0f, 0.0f), y1 = y0;
 #pragma unroll
                 for (int q = 0; q < kMaxN / 4; ++q) {
                     const float4 bq = B4[q];
                     const float4 cq = C4[q];
                     h[2 * q] = fma2(a[2 * q], h[2 * q], mul2(u2, make_float2(bq.x, bq.y)));
-                    h[2 * q + 1] =
-                        fma2(a[2 * q + 1], h[2 * q + 1], mul2(u2, make_float2(bq.z, bq.w)));
+                    h[2 * q + 1] = fma2(a[2 * q + 1], h[2 * q + 1], mul2(u2, make_float2(bq.z, bq.w)));
                     y0 = fma2(make_float2(cq.x, cq.y), h[2 * q], y0);
                     y1 = fma2(make_float2(cq.z, cq.w), h[2 * q + 1], y1);
                 }
-                const float2 ys = add2(y0, y1);
-#endif
-                const float out = fmaf(ys.x + ys.y, gg[k], pp[k]);
-#if SELSCAN_TMA_LATESTORE
-                gg[k] = out;
-#else
-                if (active && t < nt) yp[ybase + (long long)t * ystride] = from_f32<T>(out);
-#endif
+                const float2 yv = add2(y0, y1);
+                const T out = from_f32<T>(fmaf(yv.x + yv.y, gg[k], pp[k]));
+                if (kFull)
+                    ys[t * 32 + lane] = out;
+                else if (active && t < nt)
+                    yp[ybase + (long long)t * ystride] = out;
             }
         }
-#if SELSCAN_TMA_LATESTORE
-        if (kMode != kModeAgg) {
-#pragma unroll
-            for (int k = 0; k < kSub; ++k)
-                if (active && sub + k < nt) yp[ybase + (long long)(sub + k) * ystride] = from_f32<T>(gg[k]);
-        }
-#endif
     }
 }
 
 template <typename T, bool kGate, int kMode, bool kSoftplus>
-__device__ void consume(Shared<T> &S, const TmaScanParams &p) {
+__device__ void consume(Shared<T> &S, const TmaScanParams &p, const CUtensorMap *tm_y) {
+    constexpr int kTile = TileCfg<T>::kTile;
     const int c = threadIdx.x;  // 0..127
     const int lane = c & 31;
+    const int warp = c >> 5;
+    int kbuf = 0;
+    // before leaving: this warp's y stores must have finished reading shared memory
+    auto drain = [&]() {
+        if (lane == 0) bulk_wait<0>();
+        __syncwarp();
+    };
     T *yp = static_cast<T *>(p.y);
     int s = 0;
     uint32_t phase = 0;
@@ -414,10 +372,10 @@ __device__ void consume(Shared<T> &S, const TmaScanParams &p) {
     for (;;) {
         if (!mbar_wait(&S.full[s], phase, &S.abort, p.timeout_ns)) {
             if (lane == 0) fail(p, &S.abort, 3);
-            return;
+            return drain();
         }
         const TileInfo inf = S.info[s];
-        if (inf.flags & kEnd) return;
+        if (inf.flags & kEnd) return drain();
         const long long d = (long long)inf.tile * kChannels + c;
         const bool active = d < p.dim;
         const long long g = inf.b * p.ntiles + inf.tile;
@@ -479,12 +437,39 @@ __device__ void consume(Shared<T> &S, const TmaScanParams &p) {
         }
 
         const long long ybase = (inf.b * p.seqlen + inf.t0) * p.dim + d;
-        if (structured)
-            consume_tile<T, kGate, kMode, true, kSoftplus>(S.stage[s], inf.nt, h, A2, dskip, bias,
-                                                           dt_sum, yp, ybase, p.dim, active);
-        else
-            consume_tile<T, kGate, kMode, false, kSoftplus>(S.stage[s], inf.nt, h, A2, dskip, bias,
-                                                            dt_sum, yp, ybase, p.dim, active);
+        if (inf.nt == kTile) {
+            T *ys = S.ybuf[warp][kbuf];
+            if (kMode != kModeAgg) {
+                // the store that last read this staging tile has finished with it
+                if (lane == 0) bulk_wait_read<kYBufs - 1>();
+                __syncwarp();
+            }
+            if (structured)
+                consume_tile<T, kGate, kMode, true, kSoftplus, true>(
+                    S.stage[s], inf.nt, h, A2, dskip, bias, dt_sum, ys, yp, ybase, p.dim, active);
+            else
+                consume_tile<T, kGate, kMode, false, kSoftplus, true>(
+                    S.stage[s], inf.nt, h, A2, dskip, bias, dt_sum, ys, yp, ybase, p.dim, active);
+            if (kMode != kModeAgg) {
+                fence_proxy_async_smem();
+                __syncwarp();
+                const int c0 = inf.tile * kChannels + warp * 32;
+                if (lane == 0 && c0 < p.dim) {
+                    tma_store_2d(tm_y, ys, c0, (int)(inf.b * p.seqlen + inf.t0));
+                    bulk_commit();
+                }
+                kbuf ^= 1;
+            }
+        } else {
+            if (structured)
+                consume_tile<T, kGate, kMode, true, kSoftplus, false>(
+                    S.stage[s], inf.nt, h, A2, dskip, bias, dt_sum, nullptr, yp, ybase, p.dim,
+                    active);
+            else
+                consume_tile<T, kGate, kMode, false, kSoftplus, false>(
+                    S.stage[s], inf.nt, h, A2, dskip, bias, dt_sum, nullptr, yp, ybase, p.dim,
+                    active);
+        }
 
         if (inf.flags & kLast) {
             const bool last_chunk = inf.chunk == p.nchunks - 1;
@@ -535,7 +520,8 @@ template <typename T, bool kGate, int kMode, bool kSoftplus>
 __global__ void __launch_bounds__(kBlock, 1)
 scan_tma_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_d,
                 const __grid_constant__ CUtensorMap tm_z, const __grid_constant__ CUtensorMap tm_b,
-                const __grid_constant__ CUtensorMap tm_c, const TmaScanParams p) {
+                const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_y,
+                const TmaScanParams p) {
     // Indexed straight off the __shared__ array so that every access compiles
     // to a shared-memory instruction (no generic addressing, no aliasing with
     // the global y stores).
@@ -554,7 +540,7 @@ scan_tma_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
     if (threadIdx.x >= kChannels)
         produce<T, kGate>(S, p, &tm_x, &tm_d, &tm_z, &tm_b, &tm_c);
     else
-        consume<T, kGate, kMode, kSoftplus>(S, p);
+        consume<T, kGate, kMode, kSoftplus>(S, p, &tm_y);
 }
 
 // ---- host side -----------------------------------------------------------------------
@@ -591,21 +577,26 @@ bool make_map(CUtensorMap *m, const void *base, long long rows, long long cols,
 }
 
 int num_sms() {
-    int dev = 0, sms = 148;
-    if (cudaGetDevice(&dev) == cudaSuccess)
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    return sms > 0 ? sms : 148;
+    static std::atomic<int> cached[64];
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return 148;
+    if (dev < 64 && (sms = cached[dev].load(std::memory_order_relaxed)) > 0) return sms;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
+        sms = 148;
+    if (dev < 64) cached[dev].store(sms, std::memory_order_relaxed);
+    return sms;
 }
 
 template <typename T, bool kGate, int kMode, bool kSoftplus>
 cudaError_t launch_mode(const TmaScanParams &p, const void *x, const void *dl, const void *z,
                         cudaStream_t stream) {
     if (p.units <= 0) return cudaSuccess;
-    CUtensorMap mx, md, mz, mb, mc;
+    CUtensorMap mx, md, mz, mb, mc, my;
     const long long rows = p.batch * p.seqlen;
     if (!make_map<T>(&mx, x, rows, p.dim) || !make_map<T>(&md, dl, rows, p.dim) ||
         !make_map<T>(&mb, p.B, rows, p.dstate, p.dstate) ||
-        !make_map<T>(&mc, p.C, rows, p.dstate, p.dstate))
+        !make_map<T>(&mc, p.C, rows, p.dstate, p.dstate) ||
+        !make_map<T>(&my, p.y, rows, p.dim, 32))
         return cudaErrorInvalidValue;
     if (kGate) {
         if (!make_map<T>(&mz, z, rows, p.dim)) return cudaErrorInvalidValue;
@@ -614,11 +605,19 @@ cudaError_t launch_mode(const TmaScanParams &p, const void *x, const void *dl, c
     }
     const size_t smem = sizeof(Shared<T>);
     auto kern = scan_tma_kernel<T, kGate, kMode, kSoftplus>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
+    // the shared-memory opt-in is set once per device for this instantiation
+    static std::atomic<unsigned long long> configured{0};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
+    const unsigned long long bit = 1ull << (dev & 63);
+    if (!(configured.load(std::memory_order_acquire) & bit)) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        configured.fetch_or(bit, std::memory_order_acq_rel);
+    }
     const long long grid = min((long long)num_sms(), (long long)p.units);
-    kern<<<(unsigned)grid, kBlock, smem, stream>>>(mx, md, mz, mb, mc, p);
+    kern<<<(unsigned)grid, kBlock, smem, stream>>>(mx, md, mz, mb, mc, my, p);
     return cudaGetLastError();
 }
 
