@@ -5,13 +5,15 @@
 // the recurrence); "Mamba & State Space Models — Guide Complet" §6 (a
 // constant-size state instead of a growing cache) and §4 (the step itself).
 //
-// The step is bound by HBM traffic: the float32 state [batch, dim, dstate] is
-// read and written once, everything else is small. Four consecutive lanes own
-// one (b, d) chain and four consecutive states each, so a warp reads and writes
-// 8 whole chains = 512 contiguous bytes of state per access (16 bytes per lane
-// when dstate == 16). The partial outputs Σ_n C[n]·h[n] are combined across the
-// four lanes with two xor-shuffles. Each element of the state is read and
-// written by the same thread, which makes the in-place update safe.
+// The step is bound by HBM traffic: the float32 state [batch, dim, dstate]
+// is read and written once, everything else is small. Lanes work in quads:
+// the four lanes of a quad hold the four 16-byte quarters of one chain's
+// 16 states, so each warp-wide access covers 8 whole chains = 512 contiguous
+// bytes. Every lane serves kChainsPerLane chains (8 chains apart), issuing
+// all of their state loads before any arithmetic so that enough bytes are in
+// flight to cover DRAM latency. The partial outputs Σ_n C[n]·h[n] are
+// combined across a quad with two xor-shuffles. Each state element is read
+// and written by the same thread, which makes the in-place update safe.
 #include "selscan_device.cuh"
 
 namespace selscan {
@@ -20,8 +22,79 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kLanesPerChain = 4;
 constexpr int kPerLane = kMaxN / kLanesPerChain;  // 4 states per lane
+constexpr int kChainsPerLane = 4;                 // chains per lane, 8 apart
+constexpr int kChainsPerWarp = 32 / kLanesPerChain * kChainsPerLane;  // 32
 
-template <typename T, bool kGate, bool kVec>
+template <typename T, bool kGate>
+__device__ __forceinline__ float token_scalars(const StepParams &p, int64_t chain, int64_t d,
+                                               float &xv, float &zv) {
+    const T *xp = static_cast<const T *>(p.x);
+    const T *dp = static_cast<const T *>(p.delta);
+    xv = ldg_f32(xp + chain);
+    zv = kGate ? ldg_f32(static_cast<const T *>(p.z) + chain) : 0.0f;
+    float dt = ldg_f32(dp + chain) + (p.delta_bias ? p.delta_bias[d] : 0.0f);
+    if (p.softplus) dt = softplus_f32(dt);
+    return dt;
+}
+
+// dstate == 16, state 16-byte aligned: vector path.
+template <typename T, bool kGate>
+__global__ void __launch_bounds__(kThreads)
+state_update_vec_kernel(const StepParams p) {
+    const int lane = threadIdx.x & 31;
+    const int q = lane & 3;         // quarter of the chain's states
+    const int j = lane >> 2;        // chain within an 8-chain group
+    const int64_t warp = ((int64_t)blockIdx.x * kThreads + threadIdx.x) >> 5;
+    const int64_t total = p.batch * p.dim;
+    const int64_t base = warp * kChainsPerWarp;
+
+    float4 st[kChainsPerLane];
+    bool act[kChainsPerLane];
+#pragma unroll
+    for (int k = 0; k < kChainsPerLane; ++k) {
+        const int64_t chain = base + 8 * k + j;
+        act[k] = chain < total;
+        st[k] = act[k] ? *reinterpret_cast<const float4 *>(p.state + chain * kMaxN + 4 * q)
+                       : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    const T *Bp = static_cast<const T *>(p.B);
+    const T *Cp = static_cast<const T *>(p.C);
+#pragma unroll
+    for (int k = 0; k < kChainsPerLane; ++k) {
+        const int64_t chain = act[k] ? base + 8 * k + j : 0;
+        const int64_t b = chain / p.dim;
+        const int64_t d = chain - b * p.dim;
+        float xv = 0.f, zv = 0.f, dt = 0.f;
+        float partial = 0.0f;
+        if (act[k]) {
+            dt = token_scalars<T, kGate>(p, chain, d, xv, zv);
+            const float u = dt * xv;
+            const float4 a4 = *reinterpret_cast<const float4 *>(p.A + d * kMaxN + 4 * q);
+            const float av[4] = {a4.x, a4.y, a4.z, a4.w};
+            float h[4] = {st[k].x, st[k].y, st[k].z, st[k].w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int n = 4 * q + i;
+                const float a = ex2_approx(dt * av[i] * kLog2e);
+                h[i] = fmaf(a, h[i], u * ldg_f32(Bp + b * kMaxN + n));
+                partial = fmaf(ldg_f32(Cp + b * kMaxN + n), h[i], partial);
+            }
+            *reinterpret_cast<float4 *>(p.state + chain * kMaxN + 4 * q) =
+                make_float4(h[0], h[1], h[2], h[3]);
+        }
+        // every lane takes part in the shuffles (inactive chains carry zeros)
+        partial += __shfl_xor_sync(0xffffffffu, partial, 1);
+        partial += __shfl_xor_sync(0xffffffffu, partial, 2);
+        if (act[k] && q == 0) {
+            float out = fmaf(p.Dskip ? p.Dskip[d] : 0.0f, xv, partial);
+            if (kGate) out *= silu_f32(zv);
+            static_cast<T *>(p.y)[chain] = from_f32<T>(out);
+        }
+    }
+}
+
+// Any dstate ≤ 16: one quad of lanes per chain, scalar accesses.
+template <typename T, bool kGate>
 __global__ void __launch_bounds__(kThreads)
 state_update_kernel(const StepParams p) {
     const int64_t gid = (int64_t)blockIdx.x * kThreads + threadIdx.x;
@@ -31,64 +104,48 @@ state_update_kernel(const StepParams p) {
     const int64_t b = active ? chain / p.dim : 0;
     const int64_t d = active ? chain % p.dim : 0;
     const int n0 = q * kPerLane;
+    const T *Bp = static_cast<const T *>(p.B);
+    const T *Cp = static_cast<const T *>(p.C);
 
-    const T *__restrict__ xp = static_cast<const T *>(p.x);
-    const T *__restrict__ dp = static_cast<const T *>(p.delta);
-    const T *__restrict__ Bp = static_cast<const T *>(p.B);
-    const T *__restrict__ Cp = static_cast<const T *>(p.C);
-
-    float partial = 0.0f, xv = 0.0f;
-    float h[kPerLane];
-    float *st = p.state + chain * p.dstate + n0;
+    float partial = 0.0f, xv = 0.0f, zv = 0.0f;
     if (active) {
-        xv = ldg_f32(xp + chain);
-        float dt = ldg_f32(dp + chain) + (p.delta_bias ? p.delta_bias[d] : 0.0f);
-        if (p.softplus) dt = softplus_f32(dt);
+        const float dt = token_scalars<T, kGate>(p, chain, d, xv, zv);
         const float u = dt * xv;
-        if (kVec) {
-            const float4 s = *reinterpret_cast<const float4 *>(st);
-            h[0] = s.x; h[1] = s.y; h[2] = s.z; h[3] = s.w;
-        } else {
-#pragma unroll
-            for (int k = 0; k < kPerLane; ++k) h[k] = n0 + k < p.dstate ? st[k] : 0.0f;
-        }
-        const float *Ar = p.A + d * p.dstate;
+        float *st = p.state + chain * p.dstate + n0;
 #pragma unroll
         for (int k = 0; k < kPerLane; ++k) {
             const int n = n0 + k;
-            if (kVec || n < p.dstate) {
-                const float a = ex2_approx(dt * Ar[n] * kLog2e);
-                h[k] = fmaf(a, h[k], u * ldg_f32(Bp + b * p.dstate + n));
-                partial = fmaf(ldg_f32(Cp + b * p.dstate + n), h[k], partial);
+            if (n < p.dstate) {
+                const float a = ex2_approx(dt * p.A[d * p.dstate + n] * kLog2e);
+                const float h = fmaf(a, st[k], u * ldg_f32(Bp + b * p.dstate + n));
+                st[k] = h;
+                partial = fmaf(ldg_f32(Cp + b * p.dstate + n), h, partial);
             }
         }
-        if (kVec) {
-            *reinterpret_cast<float4 *>(st) = make_float4(h[0], h[1], h[2], h[3]);
-        } else {
-#pragma unroll
-            for (int k = 0; k < kPerLane; ++k)
-                if (n0 + k < p.dstate) st[k] = h[k];
-        }
     }
-    // all 32 lanes take part in the shuffles (inactive lanes carry zeros)
     partial += __shfl_xor_sync(0xffffffffu, partial, 1);
     partial += __shfl_xor_sync(0xffffffffu, partial, 2);
     if (active && q == 0) {
         float out = fmaf(p.Dskip ? p.Dskip[d] : 0.0f, xv, partial);
-        if (kGate) out *= silu_f32(ldg_f32(static_cast<const T *>(p.z) + chain));
+        if (kGate) out *= silu_f32(zv);
         static_cast<T *>(p.y)[chain] = from_f32<T>(out);
     }
 }
 
 template <typename T, bool kGate>
 cudaError_t launch_gate(const StepParams &p, cudaStream_t stream) {
-    const int64_t threads = p.batch * p.dim * kLanesPerChain;
-    const unsigned blocks = (unsigned)((threads + kThreads - 1) / kThreads);
-    const bool vec = p.dstate == kMaxN && (reinterpret_cast<uintptr_t>(p.state) & 15) == 0;
-    if (vec)
-        state_update_kernel<T, kGate, true><<<blocks, kThreads, 0, stream>>>(p);
-    else
-        state_update_kernel<T, kGate, false><<<blocks, kThreads, 0, stream>>>(p);
+    const int64_t chains = p.batch * p.dim;
+    const bool vec = p.dstate == kMaxN && (reinterpret_cast<uintptr_t>(p.state) & 15) == 0 &&
+                     (reinterpret_cast<uintptr_t>(p.A) & 15) == 0;
+    if (vec) {
+        const int64_t warps = (chains + kChainsPerWarp - 1) / kChainsPerWarp;
+        const unsigned blocks = (unsigned)((warps * 32 + kThreads - 1) / kThreads);
+        state_update_vec_kernel<T, kGate><<<blocks, kThreads, 0, stream>>>(p);
+    } else {
+        const int64_t threads = chains * kLanesPerChain;
+        const unsigned blocks = (unsigned)((threads + kThreads - 1) / kThreads);
+        state_update_kernel<T, kGate><<<blocks, kThreads, 0, stream>>>(p);
+    }
     return cudaGetLastError();
 }
 
