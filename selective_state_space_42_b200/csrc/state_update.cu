@@ -37,59 +37,110 @@ __device__ __forceinline__ float token_scalars(const StepParams &p, int64_t chai
     return dt;
 }
 
-// dstate == 16, state 16-byte aligned: vector path.
+// Four consecutive elements of B or C, widened to float (16-byte aligned for
+// float, 8-byte aligned for bf16).
+__device__ __forceinline__ float4 ld4_f32(const float *p) {
+    return __ldg(reinterpret_cast<const float4 *>(p));
+}
+__device__ __forceinline__ float4 ld4_f32(const __nv_bfloat16 *p) {
+    const uint2 r = __ldg(reinterpret_cast<const uint2 *>(p));
+    const float2 lo = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&r.x));
+    const float2 hi = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&r.y));
+    return make_float4(lo.x, lo.y, hi.x, hi.y);
+}
+
+// dstate == 16 with state, A, B, C aligned for vector accesses.
+//
+// A warp serves 32 consecutive chains base..base+31. Lane (j = lane/4,
+// q = lane%4) holds quarter q of the states of chains base + 8k + j,
+// k = 0..3, and owns the per-token scalars of chain base + 8q + j: it loads
+// that chain's x, delta and z (one 64-byte access per tensor per warp),
+// computes Δ and Δ·x once, and hands them to the three other lanes of its
+// quad that hold a quarter of that chain, by shuffle. After the quad
+// reduction of Σ_n C[n]·h[n] every lane of the quad has the sum, and the
+// owner writes the chain's y.
 template <typename T, bool kGate>
 __global__ void __launch_bounds__(kThreads)
 state_update_vec_kernel(const StepParams p) {
     const int lane = threadIdx.x & 31;
-    const int q = lane & 3;         // quarter of the chain's states
-    const int j = lane >> 2;        // chain within an 8-chain group
+    const int q = lane & 3;
+    const int j = lane >> 2;
+    const int quad0 = lane & ~3;
     const int64_t warp = ((int64_t)blockIdx.x * kThreads + threadIdx.x) >> 5;
     const int64_t total = p.batch * p.dim;
     const int64_t base = warp * kChainsPerWarp;
 
+    // state loads first, so that they are all in flight together
     float4 st[kChainsPerLane];
-    bool act[kChainsPerLane];
 #pragma unroll
     for (int k = 0; k < kChainsPerLane; ++k) {
         const int64_t chain = base + 8 * k + j;
-        act[k] = chain < total;
-        st[k] = act[k] ? *reinterpret_cast<const float4 *>(p.state + chain * kMaxN + 4 * q)
-                       : make_float4(0.f, 0.f, 0.f, 0.f);
+        st[k] = chain < total ? *reinterpret_cast<const float4 *>(p.state + chain * kMaxN + 4 * q)
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
     }
+
+    // (b, d) of chain base + j by one division, then of base + 8k + j by steps of 8
+    int64_t bk[kChainsPerLane], dk[kChainsPerLane];
+    {
+        int64_t b = (base + j) / p.dim;
+        int64_t d = base + j - b * p.dim;
+#pragma unroll
+        for (int k = 0; k < kChainsPerLane; ++k) {
+            bk[k] = b;
+            dk[k] = d;
+            d += 8;
+            while (d >= p.dim) {
+                d -= p.dim;
+                ++b;
+            }
+        }
+    }
+
+    // per-token scalars of the owned chain base + 8q + j
+    const int64_t own = base + 8 * q + j;
+    int64_t own_d = dk[0];
+#pragma unroll
+    for (int k = 1; k < kChainsPerLane; ++k) own_d = (q == k) ? dk[k] : own_d;
+    float dt_own = 0.f, u_own = 0.f, skip = 0.f, gate = 1.f;
+    if (own < total) {
+        float xv, zv;
+        dt_own = token_scalars<T, kGate>(p, own, own_d, xv, zv);
+        u_own = dt_own * xv;
+        skip = (p.Dskip ? p.Dskip[own_d] : 0.0f) * xv;
+        if (kGate) gate = silu_f32(zv);
+    }
+
     const T *Bp = static_cast<const T *>(p.B);
     const T *Cp = static_cast<const T *>(p.C);
+    float mine = 0.f;
 #pragma unroll
     for (int k = 0; k < kChainsPerLane; ++k) {
-        const int64_t chain = act[k] ? base + 8 * k + j : 0;
-        const int64_t b = chain / p.dim;
-        const int64_t d = chain - b * p.dim;
-        float xv = 0.f, zv = 0.f, dt = 0.f;
+        const int64_t chain = base + 8 * k + j;
+        const float dt = __shfl_sync(0xffffffffu, dt_own, quad0 | k);
+        const float u = __shfl_sync(0xffffffffu, u_own, quad0 | k);
         float partial = 0.0f;
-        if (act[k]) {
-            dt = token_scalars<T, kGate>(p, chain, d, xv, zv);
-            const float u = dt * xv;
-            const float4 a4 = *reinterpret_cast<const float4 *>(p.A + d * kMaxN + 4 * q);
-            const float av[4] = {a4.x, a4.y, a4.z, a4.w};
-            float h[4] = {st[k].x, st[k].y, st[k].z, st[k].w};
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int n = 4 * q + i;
-                const float a = ex2_approx(dt * av[i] * kLog2e);
-                h[i] = fmaf(a, h[i], u * ldg_f32(Bp + b * kMaxN + n));
-                partial = fmaf(ldg_f32(Cp + b * kMaxN + n), h[i], partial);
-            }
-            *reinterpret_cast<float4 *>(p.state + chain * kMaxN + 4 * q) =
-                make_float4(h[0], h[1], h[2], h[3]);
+        if (chain < total) {
+            const float4 a4 = __ldg(reinterpret_cast<const float4 *>(p.A + dk[k] * kMaxN + 4 * q));
+            const float4 b4 = ld4_f32(Bp + bk[k] * kMaxN + 4 * q);
+            const float4 c4 = ld4_f32(Cp + bk[k] * kMaxN + 4 * q);
+            const float dl = dt * kLog2e;
+            float4 h = st[k];
+            h.x = fmaf(ex2_approx(dl * a4.x), h.x, u * b4.x);
+            h.y = fmaf(ex2_approx(dl * a4.y), h.y, u * b4.y);
+            h.z = fmaf(ex2_approx(dl * a4.z), h.z, u * b4.z);
+            h.w = fmaf(ex2_approx(dl * a4.w), h.w, u * b4.w);
+            *reinterpret_cast<float4 *>(p.state + chain * kMaxN + 4 * q) = h;
+            partial = fmaf(c4.x, h.x, fmaf(c4.y, h.y, fmaf(c4.z, h.z, c4.w * h.w)));
         }
         // every lane takes part in the shuffles (inactive chains carry zeros)
         partial += __shfl_xor_sync(0xffffffffu, partial, 1);
         partial += __shfl_xor_sync(0xffffffffu, partial, 2);
-        if (act[k] && q == 0) {
-            float out = fmaf(p.Dskip ? p.Dskip[d] : 0.0f, xv, partial);
-            if (kGate) out *= silu_f32(zv);
-            static_cast<T *>(p.y)[chain] = from_f32<T>(out);
-        }
+        mine = (q == k) ? partial : mine;
+    }
+    if (own < total) {
+        float out = skip + mine;
+        if (kGate) out *= gate;
+        static_cast<T *>(p.y)[own] = from_f32<T>(out);
     }
 }
 
@@ -135,8 +186,11 @@ state_update_kernel(const StepParams p) {
 template <typename T, bool kGate>
 cudaError_t launch_gate(const StepParams &p, cudaStream_t stream) {
     const int64_t chains = p.batch * p.dim;
+    const uintptr_t bc_align = 4 * sizeof(T) - 1;
     const bool vec = p.dstate == kMaxN && (reinterpret_cast<uintptr_t>(p.state) & 15) == 0 &&
-                     (reinterpret_cast<uintptr_t>(p.A) & 15) == 0;
+                     (reinterpret_cast<uintptr_t>(p.A) & 15) == 0 &&
+                     (reinterpret_cast<uintptr_t>(p.B) & bc_align) == 0 &&
+                     (reinterpret_cast<uintptr_t>(p.C) & bc_align) == 0;
     if (vec) {
         const int64_t warps = (chains + kChainsPerWarp - 1) / kChainsPerWarp;
         const unsigned blocks = (unsigned)((warps * 32 + kThreads - 1) / kThreads);

@@ -1,0 +1,104 @@
+"""Run a fixed number of launches of one kernel on a named workload.
+
+Meant to sit under a profiler (one kernel, a few launches, nothing else on
+the device) and to give quick CUDA-event timings without one:
+
+    python -m selective_state_space_42_b200.profile_case scan mamba2p8b_layer --launches 2
+    python -m selective_state_space_42_b200.profile_case decode --launches 3
+
+``scan`` calls selscan_fwd on a scan workload; ``decode`` calls
+selscan_state_update on the decode workload. With ``--time`` it also prints
+the median CUDA-event time per launch, cold (a 512 MiB buffer is written
+between launches, which evicts L2) and back to back, as one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+
+import torch
+
+from . import selscan as ss
+from . import workloads as wl
+
+
+def _scan_case(name: str):
+    w = wl.WORKLOADS[name]
+    inp = wl.make_scan_inputs(w, device="cuda")
+    y = torch.empty_like(inp["x"])
+    fs = torch.empty(w.batch, w.dim, w.dstate, device="cuda") if w.final_state else None
+
+    def launch(_i: int) -> None:
+        ss.selscan_fwd(inp["x"], inp["delta"], inp["A"], inp["B"], inp["C"], inp["D"],
+                       inp["z"], inp["delta_bias"], softplus=w.softplus, y=y,
+                       final_state=fs)
+
+    return launch, w.algorithmic_bytes()
+
+
+def _decode_case():
+    w = wl.DECODE
+    state = wl.make_decode_state(w, device="cuda")
+    A, Dv, bias = wl.make_decode_params(w, device="cuda")
+    steps = [wl.make_decode_step(w, s, device="cuda") for s in range(8)]
+    y = torch.empty(w.batch, w.dim, device="cuda", dtype=wl.DTYPES[w.dtype])
+
+    def launch(i: int) -> None:
+        s = steps[i % len(steps)]
+        ss.selscan_state_update(state, s["x"], s["delta"], A, s["B"], s["C"], Dv, s["z"],
+                                bias, y=y)
+
+    return launch, w.algorithmic_bytes_per_step()
+
+
+def _median(v):
+    v = sorted(v)
+    return v[len(v) // 2]
+
+
+def main(argv=None) -> int:
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("kernel", choices=["scan", "decode"])
+    ap.add_argument("workload", nargs="?", default="mamba2p8b_layer",
+                    help="scan workload name (ignored for decode)")
+    ap.add_argument("--launches", type=int, default=2)
+    ap.add_argument("--time", action="store_true")
+    args = ap.parse_args(argv)
+
+    launch, nbytes = _scan_case(args.workload) if args.kernel == "scan" else _decode_case()
+    for i in range(args.launches):
+        launch(i)
+    torch.cuda.synchronize()
+    out = {"kernel": args.kernel, "launches": args.launches,
+           "workload": args.workload if args.kernel == "scan" else wl.DECODE.name,
+           "algorithmic_bytes": nbytes}
+    if args.time:
+        flush = torch.empty(512 << 20, dtype=torch.uint8, device="cuda")
+        cold = []
+        for i in range(20):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            launch(i)
+            e1.record()
+            torch.cuda.synchronize()
+            cold.append(e0.elapsed_time(e1))
+        n = 100
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for i in range(n):
+            launch(i)
+        e1.record()
+        torch.cuda.synchronize()
+        b2b = e0.elapsed_time(e1) / n
+        cold_ms = _median(cold)
+        out.update(cold_ms=cold_ms, cold_GBps=nbytes / cold_ms / 1e6, b2b_ms=b2b,
+                   b2b_GBps=nbytes / b2b / 1e6)
+    status = ss.selscan_device_status()
+    out["device_status"] = status
+    print(json.dumps(out), flush=True)
+    return 0 if status == 0 else 1
+
+
+if __name__ == "__main__":
+    raise SystemExit(main())

@@ -22,7 +22,8 @@ def _step(state, inp, params, softplus=True):
 
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
-@pytest.mark.parametrize("shape", [(1, 1, 1), (3, 37, 16), (5, 130, 7), (2, 64, 4)],
+@pytest.mark.parametrize("shape", [(1, 1, 1), (3, 37, 16), (5, 130, 7), (2, 64, 4),
+                                   (4, 3, 16), (7, 1, 16), (3, 9, 16)],
                          ids=str)
 @pytest.mark.parametrize("gate", [True, False])
 def test_small_steps_every_element(dtype, shape, gate):
@@ -50,6 +51,34 @@ def test_small_steps_every_element(dtype, shape, gate):
     # every element of every step; the rms floor is taken over the trajectory
     gh.compare(np.stack(ys), np.stack(yos), gh.RTOL[dtype], "y trajectory")
     gh.compare(np.stack(sts), np.stack(refs), gh.RTOL[dtype], "state trajectory")
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_unaligned_bc(dtype):
+    """B and C starting one element past an 8-byte (bf16) or 16-byte (f32)
+    boundary: the step must give the same values as the oracle (the vector
+    loads are not usable there)."""
+    batch, dim, N = 3, 70, 16
+    w = wl.DecodeWorkload("unaligned", batch, dim, N, 3, dtype, True, seed=77)
+    state = wl.make_decode_state(w).to(DEV)
+    A, Dv, bias = (t.to(DEV) for t in wl.make_decode_params(w))
+    ref = gh.to_np(state)
+    orc = oracle.default()
+    for s in range(w.steps):
+        inp = {k: (None if v is None else v.to(DEV)) for k, v in wl.make_decode_step(w, s).items()}
+        for key in ("B", "C"):
+            big = torch.empty(batch * N + 1, dtype=inp[key].dtype, device=DEV)
+            view = big[1:].view(batch, N)
+            view.copy_(inp[key])
+            inp[key] = view
+            assert view.data_ptr() % 8 != 0
+        y = _step(state, inp, (A, Dv, bias))
+        yo, ref = orc.state_update(ref, gh.to_np(inp["x"]), gh.to_np(inp["delta"]),
+                                   gh.to_np(A), gh.to_np(inp["B"]), gh.to_np(inp["C"]),
+                                   gh.to_np(Dv), gh.to_np(inp.get("z")), gh.to_np(bias))
+        torch.cuda.synchronize()
+        gh.compare(gh.to_np(y), yo, gh.RTOL[dtype], f"y step {s}")
+        gh.compare(gh.to_np(state), ref, gh.RTOL[dtype], f"state step {s}")
 
 
 def test_decode_workload_1000_steps_sampled():
