@@ -90,6 +90,10 @@ class Oracle:
             _i64, _i64, _i64]
         lib.oracle_compose.restype = None
         lib.oracle_compose.argtypes = [ctypes.c_double] * 4 + [_dp, _dp]
+        lib.oracle_selscan_bwd.restype = None
+        lib.oracle_selscan_bwd.argtypes = (
+            [_dp] * 8 + [ctypes.c_int] + [_dp] * 3 + [_dp] * 9
+            + [_i64, _i64, _i64, _i64, ctypes.c_int])
         lib.oracle_zoh_discretize.restype = None
         lib.oracle_zoh_discretize.argtypes = [ctypes.c_double, _dp, _dp, _dp,
                                               _dp, _i64]
@@ -146,6 +150,33 @@ class Oracle:
             int(bool(softplus)), int(bbar), _ptr(a["h0"]), _ptr(y), _ptr(hs),
             batch, L, dim, N, int(chunk), int(threads or default_threads()))
         return y, hs
+
+    def bwd(self, x, delta, A, B, C, D=None, z=None, delta_bias=None,
+            softplus=True, h0=None, dy=None, dfinal=None, threads=None):
+        """Gradient of the loss Σ dy·y + Σ dfinal·final_state with respect to
+        every input of ``fwd`` (input term Δ·B·x). Returns a dict with dx,
+        ddelta, dA, dB, dC, dD, dz (None without z), ddelta_bias and dh0
+        (None without h0), all float64."""
+        a, (batch, L, dim, N) = self._fwd_args(x, delta, A, B, C, D, z,
+                                               delta_bias, h0)
+        dy = _f64(dy, (batch, L, dim))
+        dfinal = _f64(dfinal, (batch, dim, N))
+        out = dict(
+            dx=np.empty((batch, L, dim)), ddelta=np.empty((batch, L, dim)),
+            dA=np.empty((dim, N)), dB=np.empty((batch, L, N)),
+            dC=np.empty((batch, L, N)), dD=np.empty((dim,)),
+            dz=np.empty((batch, L, dim)) if a["z"] is not None else None,
+            ddelta_bias=np.empty((dim,)),
+            dh0=np.empty((batch, dim, N)) if a["h0"] is not None else None)
+        self.lib.oracle_selscan_bwd(
+            _ptr(a["x"]), _ptr(a["delta"]), _ptr(a["A"]), _ptr(a["B"]),
+            _ptr(a["C"]), _ptr(a["D"]), _ptr(a["z"]), _ptr(a["delta_bias"]),
+            int(bool(softplus)), _ptr(a["h0"]), _ptr(dy), _ptr(dfinal),
+            _ptr(out["dx"]), _ptr(out["ddelta"]), _ptr(out["dA"]), _ptr(out["dB"]),
+            _ptr(out["dC"]), _ptr(out["dD"]), _ptr(out["dz"]),
+            _ptr(out["ddelta_bias"]), _ptr(out["dh0"]),
+            batch, L, dim, N, int(threads or default_threads()))
+        return out
 
     # -- single-token decode -------------------------------------------------
     def state_update(self, state, x, delta, A, B, C, D=None, z=None,

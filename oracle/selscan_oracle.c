@@ -46,6 +46,9 @@
 #include <math.h>
 #include <stdint.h>
 #include <stdlib.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
 
 #define ORACLE_BBAR_DELTA 0 /* B_bar = Δ·B   ([Johe] "SSM as RNN")        */
 #define ORACLE_BBAR_ZOH 1   /* B_bar = (exp(Δ·A) − 1)/A·B ([Guide] §1)    */
@@ -275,4 +278,152 @@ void oracle_zoh_discretize(double dt, const double *A, const double *B,
         A_bar[n] = exp(dt * A[n]);
         B_bar[n] = bbar_coeff(dt, A[n], ORACLE_BBAR_ZOH) * B[n];
     }
+}
+
+/* d silu(z)/dz = σ(z)·(1 + z·(1 − σ(z))). */
+static double silu_grad(double z)
+{
+    double sg = 1.0 / (1.0 + exp(-z));
+    return sg * (1.0 + z * (1.0 - sg));
+}
+
+/* d softplus(v)/dv = σ(v). */
+static double sigmoid(double v)
+{
+    return 1.0 / (1.0 + exp(-v));
+}
+
+/*
+ * Gradient of oracle_selscan_fwd (input term Δ·B·x) by reverse-mode
+ * differentiation of the recurrence: the loss is Σ dy·y + Σ dfinal·final_state
+ * for given dy [batch, L, D] and dfinal [batch, D, N] (null: 0).
+ *
+ * The backward pass with recomputation that [Infer] "Cena selekcji" names is
+ * the reverse sweep of the recurrence [Guide] §4 / [Johe] "SSM as RNN":
+ * with λ_t = ∂loss/∂h_t,
+ *   λ_{L−1} = ds_{L−1}·C_{L−1} + dfinal,   λ_t = ds_t·C_t + Abar_{t+1}·λ_{t+1},
+ * where ds_t = dy_t·silu(z_t) is the gradient of the pre-gate output
+ * s_t = Σ_n C_t[n]·h_t[n] + D·x_t. Each token then contributes
+ *   dB_t[n] += λ_t[n]·Δ_t·x_t          (summed over channels)
+ *   dC_t[n] += ds_t·h_t[n]             (summed over channels)
+ *   du_t     = Σ_n λ_t[n]·B_t[n]       (u_t = Δ_t·x_t)
+ *   dΔ_t     = Σ_n λ_t[n]·h_{t−1}[n]·Abar_t[n]·A[n] + du_t·x_t
+ *   dA[n]   += λ_t[n]·h_{t−1}[n]·Abar_t[n]·Δ_t
+ *   dx_t     = du_t·Δ_t + ds_t·D,   dD += ds_t·x_t,   dz_t = dy_t·s_t·silu'(z_t)
+ *   ddelta_t = dΔ_t·σ(delta_t + bias) (softplus on; dΔ_t otherwise),
+ *   dbias   += ddelta_t
+ * and dh0 = Abar_0·λ_0. The forward states h_t are kept per chain (this is
+ * the plain definition, not a memory-saving schedule).
+ *
+ * Outputs: dx, ddelta, dz [batch, L, D] (dz only when z is given); dB, dC
+ * [batch, L, N]; dA [D, N]; dDv, ddelta_bias [D]; dh0 [batch, D, N]
+ * (nullable). Every output is overwritten.
+ */
+void oracle_selscan_bwd(const double *x, const double *delta, const double *A,
+                        const double *B, const double *C, const double *Dv,
+                        const double *z, const double *delta_bias,
+                        int softplus_flag, const double *h0, const double *dy,
+                        const double *dfinal, double *dx, double *ddelta,
+                        double *dA, double *dB, double *dC, double *dDv,
+                        double *dz, double *ddelta_bias, double *dh0,
+                        int64_t batch, int64_t L, int64_t D, int64_t N,
+                        int nthreads)
+{
+    if (nthreads < 1)
+        nthreads = 1;
+    for (int64_t i = 0; i < D * N; ++i)
+        dA[i] = 0.0;
+    for (int64_t d = 0; d < D; ++d) {
+        dDv[d] = 0.0;
+        ddelta_bias[d] = 0.0;
+    }
+    for (int64_t i = 0; i < batch * L * N; ++i) {
+        dB[i] = 0.0;
+        dC[i] = 0.0;
+    }
+    /* dB and dC sum over channels: every thread accumulates its channels into
+     * a private [L, N] pair, added to the outputs in thread order. */
+    double *priv = (double *)calloc((size_t)(nthreads * 2 * L * N), sizeof(double));
+    for (int64_t b = 0; b < batch; ++b) {
+#pragma omp parallel num_threads(nthreads)
+        {
+            int tid = 0;
+#ifdef _OPENMP
+            tid = omp_get_thread_num();
+#endif
+            double *pB = priv + (size_t)tid * 2 * L * N, *pC = pB + L * N;
+            double *hs = (double *)malloc((size_t)((L + 1) * N) * sizeof(double));
+            double *dts = (double *)malloc((size_t)(L > 0 ? L : 1) * sizeof(double));
+            double *ss = (double *)malloc((size_t)(L > 0 ? L : 1) * sizeof(double));
+            double *lam = (double *)malloc((size_t)N * sizeof(double));
+#pragma omp for schedule(static)
+            for (int64_t d = 0; d < D; ++d) {
+                const double *Arow = A + d * N;
+                double dskip = Dv ? Dv[d] : 0.0;
+                /* forward, keeping h_{t} for every t (hs[t + 1]) */
+                for (int64_t n = 0; n < N; ++n)
+                    hs[n] = h0 ? h0[(b * D + d) * N + n] : 0.0;
+                for (int64_t t = 0; t < L; ++t) {
+                    int64_t i = (b * L + t) * D + d;
+                    int64_t j = (b * L + t) * N;
+                    double dt = step_size(delta[i], delta_bias, d, softplus_flag);
+                    double acc = 0.0;
+                    dts[t] = dt;
+                    for (int64_t n = 0; n < N; ++n) {
+                        double h = exp(dt * Arow[n]) * hs[t * N + n] + dt * B[j + n] * x[i];
+                        hs[(t + 1) * N + n] = h;
+                        acc += C[j + n] * h;
+                    }
+                    ss[t] = acc + dskip * x[i];
+                }
+                /* reverse sweep */
+                for (int64_t n = 0; n < N; ++n)
+                    lam[n] = dfinal ? dfinal[(b * D + d) * N + n] : 0.0;
+                for (int64_t t = L - 1; t >= 0; --t) {
+                    int64_t i = (b * L + t) * D + d;
+                    int64_t j = (b * L + t) * N;
+                    double dt = dts[t];
+                    double ds = z ? dy[i] * silu(z[i]) : dy[i];
+                    if (z)
+                        dz[i] = dy[i] * ss[t] * silu_grad(z[i]);
+                    dDv[d] += ds * x[i];
+                    double du = 0.0, ddt = 0.0;
+                    for (int64_t n = 0; n < N; ++n) {
+                        double h = hs[(t + 1) * N + n], hprev = hs[t * N + n];
+                        double a_bar = exp(dt * Arow[n]);
+                        lam[n] += ds * C[j + n]; /* λ_t */
+                        pC[t * N + n] += ds * h;
+                        pB[t * N + n] += lam[n] * dt * x[i];
+                        du += lam[n] * B[j + n];
+                        ddt += lam[n] * hprev * a_bar * Arow[n];
+                        dA[d * N + n] += lam[n] * hprev * a_bar * dt;
+                        lam[n] *= a_bar; /* Abar_t·λ_t, the part of λ_{t−1} from h_t */
+                    }
+                    ddt += du * x[i];
+                    dx[i] = du * dt + ds * dskip;
+                    double v = delta[i] + (delta_bias ? delta_bias[d] : 0.0);
+                    double dv = softplus_flag ? ddt * sigmoid(v) : ddt;
+                    ddelta[i] = dv;
+                    ddelta_bias[d] += dv;
+                }
+                if (dh0)
+                    for (int64_t n = 0; n < N; ++n)
+                        dh0[(b * D + d) * N + n] = lam[n];
+            }
+            free(hs);
+            free(dts);
+            free(ss);
+            free(lam);
+        }
+        for (int k = 0; k < nthreads; ++k) {
+            double *pB = priv + (size_t)k * 2 * L * N, *pC = pB + L * N;
+            for (int64_t i = 0; i < L * N; ++i) {
+                dB[b * L * N + i] += pB[i];
+                dC[b * L * N + i] += pC[i];
+                pB[i] = 0.0;
+                pC[i] = 0.0;
+            }
+        }
+    }
+    free(priv);
 }

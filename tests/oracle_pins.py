@@ -375,9 +375,129 @@ def pin_hand_worked(orc):
     assert _rel(hs[0, 0], [float(v) for v in h]) < 1e-15, "hand-worked state"
 
 
+# ---------------------------------------------------------------------------
+# Backward pass (gradient of the scan). The loss is Σ dy·y + Σ dfinal·h_{L−1};
+# the pins below check the oracle's reverse sweep against numerical
+# differentiation of the (separately pinned) forward, against exact
+# homogeneity identities of the recurrence, and against closed forms.
+
+_BWD_GRADS = {"x": "dx", "delta": "ddelta", "A": "dA", "B": "dB", "C": "dC",
+              "D": "dD", "z": "dz", "delta_bias": "ddelta_bias", "h0": "dh0"}
+
+
+def _bwd_case(seed, gate=True, with_h0=True, batch=2, L=5, D=3, N=4):
+    c = _rand_case(seed, batch=batch, L=L, D=D, N=N, gate=gate)
+    r = RNG(seed + 1000)
+    c["h0"] = r.standard_normal((batch, D, N)) if with_h0 else None
+    dy = r.standard_normal((batch, L, D))
+    dfinal = r.standard_normal((batch, D, N))
+    return c, dy, dfinal
+
+
+def _fwd_of(orc, c, softplus):
+    return orc.fwd(c["x"], c["delta"], c["A"], c["B"], c["C"], c["D"], c["z"],
+                   c["delta_bias"], softplus=softplus, h0=c["h0"], threads=1)
+
+
+def _bwd_of(orc, c, dy, dfinal, softplus):
+    return orc.bwd(c["x"], c["delta"], c["A"], c["B"], c["C"], c["D"], c["z"],
+                   c["delta_bias"], softplus=softplus, h0=c["h0"], dy=dy,
+                   dfinal=dfinal, threads=1)
+
+
+def pin_bwd_finite_differences(orc):
+    """Every gradient against central differences of the forward oracle,
+    element by element, with and without softplus, gate and initial state."""
+    for seed, softplus, gate, with_h0 in ((40, True, True, True),
+                                          (41, False, False, False)):
+        c, dy, dfinal = _bwd_case(seed, gate=gate, with_h0=with_h0)
+        if not softplus:  # Δ = delta + bias itself: keep it positive
+            c["delta"] = np.abs(c["delta"]) + 0.05
+            c["delta_bias"] = np.full_like(c["delta_bias"], 0.01)
+        g = _bwd_of(orc, c, dy, dfinal, softplus)
+
+        def loss(cc):
+            y, hs = _fwd_of(orc, cc, softplus)
+            return float(np.sum(dy * y) + np.sum(dfinal * hs))
+
+        for name, gname in _BWD_GRADS.items():
+            if c[name] is None:
+                assert g[gname] is None, f"{gname} returned without {name}"
+                continue
+            arr = c[name]
+            fd = np.zeros_like(arr)
+            for idx in np.ndindex(arr.shape):
+                e = 1e-6 * max(1.0, abs(arr[idx]))
+                cp = dict(c)
+                cp[name] = arr.copy()
+                cp[name][idx] += e
+                cm = dict(c)
+                cm[name] = arr.copy()
+                cm[name][idx] -= e
+                fd[idx] = (loss(cp) - loss(cm)) / (2 * e)
+            assert _rel(g[gname], fd) < 1e-6, f"{gname} vs finite differences"
+
+
+def pin_bwd_homogeneity(orc):
+    """Exact identities (no truncation error). Without the gate, y and h_{L−1}
+    are linear in (x, h0) jointly, and y − D·x and h_{L−1} are linear in
+    (B, h0) jointly and y − D·x in C; Euler's theorem for such maps gives
+        Σ dy·y + Σ dfinal·h_{L−1} = Σ dx·x + Σ dh0·h0,
+        Σ dy·(y − D·x) + Σ dfinal·h_{L−1} = Σ dB·B + Σ dh0·h0,
+        Σ dy·(y − D·x) = Σ dC·C (with dfinal = 0),   Σ dD·D = Σ dy·D·x."""
+    c, dy, dfinal = _bwd_case(50, gate=False, with_h0=True, L=9, D=4, N=5)
+    y, hs = _fwd_of(orc, c, True)
+    g = _bwd_of(orc, c, dy, dfinal, True)
+    dx_ = c["D"][None, None, :] * c["x"]
+    lhs1 = np.sum(dy * y) + np.sum(dfinal * hs)
+    rhs1 = np.sum(g["dx"] * c["x"]) + np.sum(g["dh0"] * c["h0"])
+    assert abs(lhs1 - rhs1) < 1e-12 * max(1.0, abs(lhs1)), "x/h0 homogeneity"
+    lhs2 = np.sum(dy * (y - dx_)) + np.sum(dfinal * hs)
+    rhs2 = np.sum(g["dB"] * c["B"]) + np.sum(g["dh0"] * c["h0"])
+    assert abs(lhs2 - rhs2) < 1e-12 * max(1.0, abs(lhs2)), "B/h0 homogeneity"
+    g0 = _bwd_of(orc, c, dy, np.zeros_like(dfinal), True)
+    lhs3 = np.sum(dy * (y - dx_))
+    assert abs(lhs3 - np.sum(g0["dC"] * c["C"])) < 1e-12 * max(1.0, abs(lhs3)), \
+        "C homogeneity"
+    lhs4 = np.sum(dy * dx_)
+    assert abs(lhs4 - np.sum(g0["dD"] * c["D"])) < 1e-12 * max(1.0, abs(lhs4)), \
+        "D homogeneity"
+
+
+def pin_bwd_single_token(orc):
+    """L = 1 from a zero state, no gate, softplus off: y = Σ_n C B Δ x + D x,
+    h = Δ x B, so with u = Δ·x
+        dx = dy (Σ C B Δ + D) + Δ Σ dfinal·B,   dΔ = x (dy Σ C B + Σ dfinal·B),
+        dB = (dy C + dfinal) Δ x (summed over channels),  dC = dy Δ x B
+        (summed over channels),  dA = 0,  dD = dy x."""
+    r = RNG(60)
+    D, N = 3, 4
+    x = r.standard_normal((1, 1, D))
+    dl = r.uniform(0.1, 0.9, (1, 1, D))
+    A = -r.uniform(0.5, 2.0, (D, N))
+    B = r.standard_normal((1, 1, N))
+    C = r.standard_normal((1, 1, N))
+    Dv = r.standard_normal(D)
+    dy = r.standard_normal((1, 1, D))
+    dfin = r.standard_normal((1, D, N))
+    g = orc.bwd(x, dl, A, B, C, Dv, None, None, softplus=False, dy=dy,
+                dfinal=dfin, threads=1)
+    cb = float(np.sum(C * B))
+    xv, dt, gy = x[0, 0], dl[0, 0], dy[0, 0]
+    fb = dfin[0] @ B[0, 0]                       # Σ_n dfinal[d, n]·B[n]
+    assert _rel(g["dx"][0, 0], gy * (cb * dt + Dv) + dt * fb) < 1e-14, "dx"
+    assert _rel(g["ddelta"][0, 0], xv * (gy * cb + fb)) < 1e-14, "ddelta"
+    dB = np.sum((gy[:, None] * C[0, 0][None, :] + dfin[0]) * (dt * xv)[:, None], axis=0)
+    assert _rel(g["dB"][0, 0], dB) < 1e-14, "dB"
+    assert _rel(g["dC"][0, 0], np.sum((gy * dt * xv)[:, None] * B[0, 0][None, :], axis=0)) < 1e-14, "dC"
+    assert np.all(g["dA"] == 0.0), "dA from a zero state"
+    assert _rel(g["dD"], gy * xv) < 1e-14, "dD"
+
+
 ALL_PINS = [
     pin_explicit_sum, pin_single_token, pin_lti_convolution, pin_zoh_matrix,
     pin_euler_vs_zoh, pin_linearity, pin_delta_to_zero, pin_chunked,
     pin_associativity, pin_geometric, pin_decay, pin_cross_entry,
     pin_decode_layout, pin_softplus_and_gate, pin_hand_worked,
+    pin_bwd_finite_differences, pin_bwd_homogeneity, pin_bwd_single_token,
 ]

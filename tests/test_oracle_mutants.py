@@ -43,6 +43,24 @@ MUTANTS = [
      "double dskip = Dv ? Dv[0] : 0.0;\n            for (int64_t t = 0; t < L; ++t)"),
     ("chunk_carry_dropped", "oracle_compose(P[c * N + n], H[c * N + n], 1.0,\n                                   hin[c * N + n],",
      "oracle_compose(P[c * N + n], H[c * N + n], 1.0,\n                                   0.0,"),
+    # backward pass
+    ("bwd_lambda_not_decayed", "lam[n] *= a_bar; /*", "lam[n] *= 1.0; /*"),
+    ("bwd_dA_without_dt", "dA[d * N + n] += lam[n] * hprev * a_bar * dt;",
+     "dA[d * N + n] += lam[n] * hprev * a_bar;"),
+    ("bwd_softplus_grad_dropped", "double dv = softplus_flag ? ddt * sigmoid(v) : ddt;",
+     "double dv = ddt;"),
+    ("bwd_h_instead_of_hprev", "ddt += lam[n] * hprev * a_bar * Arow[n];",
+     "ddt += lam[n] * h * a_bar * Arow[n];"),
+    ("bwd_dx_skip_dropped", "dx[i] = du * dt + ds * dskip;", "dx[i] = du * dt;"),
+    ("bwd_silu_grad_sign", "return sg * (1.0 + z * (1.0 - sg));",
+     "return sg * (1.0 - z * (1.0 - sg));"),
+    ("bwd_dB_without_x", "pB[t * N + n] += lam[n] * dt * x[i];",
+     "pB[t * N + n] += lam[n] * dt;"),
+    ("bwd_du_x_term_dropped", "    ddt += du * x[i];\n", "\n"),
+    ("bwd_dfinal_ignored", "lam[n] = dfinal ? dfinal[(b * D + d) * N + n] : 0.0;",
+     "lam[n] = 0.0;"),
+    ("bwd_gate_on_ds_dropped", "double ds = z ? dy[i] * silu(z[i]) : dy[i];",
+     "double ds = dy[i];"),
 ]
 
 
