@@ -182,6 +182,51 @@ SELSCAN_API int selscan_state_update(float *state, const void *x, const void *de
                          selscan_dtype_t dtype, selscan_stream_t stream);
 
 /*
+ * selscan_bwd -- gradient of selscan_fwd (the backward pass), with the
+ * forward states recomputed instead of stored ("Mamba: co potrafią modele
+ * przestrzeni stanów", "Cena selekcji": the backward pass recomputes the
+ * intermediate states).
+ *
+ * For the loss Σ dy·y + Σ dfinal_state·final_state of the selscan_fwd call
+ * with the same inputs, writes the loss's gradient with respect to each
+ * input. With λ_t = ∂loss/∂h_t, λ after the last token = dfinal_state and
+ * λ_t = ds_t·C_t + Abar_{t+1}·λ_{t+1}, ds_t = dy_t·silu(z_t):
+ *
+ *   x, delta, A, B, C, D, z, delta_bias, softplus_flag   as in selscan_fwd
+ *   dy            [batch, seqlen, dim]      dtype        required
+ *   dfinal_state  [batch, dim, dstate]      float32      NULL -> zero
+ *   dx, ddelta    [batch, seqlen, dim]      dtype        required outputs
+ *   dA            [dim, dstate]             float32      required output
+ *                                                        (sum over batch and tokens)
+ *   dB, dC        [batch, seqlen, dstate]   float32      required outputs
+ *                                                        (sums over channels)
+ *   dD            [dim]                     float32      NULL -> not written
+ *   dz            [batch, seqlen, dim]      dtype        required iff z != NULL
+ *   ddelta_bias   [dim]                     float32      NULL -> not written
+ *   batch <= 65535; other limits as in selscan_fwd.
+ *
+ * Every output is overwritten (not accumulated into); dB, dC, dA, dD and
+ * ddelta_bias are float32 whatever `dtype` is. Results are deterministic
+ * (fixed summation order, no atomics). Outputs must not overlap any input.
+ * Takes a stream-ordered device workspace (cudaMallocAsync / cudaFreeAsync
+ * on `stream`) of selscan_bwd_workspace_bytes() bytes: the state entering
+ * every 16-token tile of every chain, and per-32-channel partial sums of dB
+ * and dC.
+ */
+SELSCAN_API int selscan_bwd(const void *x, const void *delta, const float *A,
+                            const void *B, const void *C, const float *D, const void *z,
+                            const float *delta_bias, int softplus_flag, const void *dy,
+                            const float *dfinal_state, void *dx, void *ddelta, float *dA,
+                            float *dB, float *dC, float *dD, void *dz, float *ddelta_bias,
+                            int64_t batch, int64_t seqlen, int64_t dim, int64_t dstate,
+                            selscan_dtype_t dtype, selscan_stream_t stream);
+
+/* Host-only: device workspace bytes selscan_bwd takes for these sizes
+ * (0 for empty or invalid sizes). */
+SELSCAN_API int64_t selscan_bwd_workspace_bytes(int64_t batch, int64_t seqlen, int64_t dim,
+                                                int64_t dstate);
+
+/*
  * selscan_device_status -- the library's sticky device-side error word on
  * the current device (synchronous: waits for prior work). 0 means no device
  * wait has given up; otherwise the code of the first one that did (1: a

@@ -297,6 +297,52 @@ cudaError_t fwd_run(FwdPlan *plan, void *ws, cudaStream_t stream) {
 
 }  // namespace selscan
 
+namespace {
+
+struct BwdLayout {
+    size_t ckpt, part, pA, pD, pbias, total;
+};
+
+int64_t ceil_div64(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
+
+BwdLayout bwd_layout(int64_t batch, int64_t seqlen, int64_t dim) {
+    const int64_t K = ceil_div64(seqlen, selscan::bwd_tile_tokens());
+    const int64_t ct = ceil_div64(dim, selscan::bwd_tile_channels());
+    BwdLayout l;
+    size_t off = 0;
+    l.ckpt = off;
+    off = align256(off + (size_t)(batch * K * dim) * selscan::kMaxN * sizeof(float));
+    l.part = off;
+    off = align256(off + (size_t)(batch * ct * seqlen) * 2 * selscan::kMaxN * sizeof(float));
+    l.pA = off;
+    off = align256(off + (size_t)(batch * dim) * selscan::kMaxN * sizeof(float));
+    l.pD = off;
+    off = align256(off + (size_t)(batch * dim) * sizeof(float));
+    l.pbias = off;
+    off = align256(off + (size_t)(batch * dim) * sizeof(float));
+    l.total = off;
+    return l;
+}
+
+struct Span {
+    const void *p;
+    size_t n;
+};
+
+bool any_overlap(const Span *outs, int no, const Span *ins, int ni) {
+    for (int i = 0; i < no; ++i) {
+        for (int j = 0; j < ni; ++j)
+            if (overlaps(outs[i].p, outs[i].n, ins[j].p, ins[j].n)) return true;
+        for (int j = i + 1; j < no; ++j)
+            if (overlaps(outs[i].p, outs[i].n, outs[j].p, outs[j].n)) return true;
+    }
+    return false;
+}
+
+}  // namespace
+
 extern "C" {
 
 const char *selscan_status_string(int status) {
@@ -308,7 +354,7 @@ const char *selscan_status_string(int status) {
     case SELSCAN_ERR_MISALIGNED: return "a pointer is not aligned to its element size";
     case SELSCAN_ERR_DSTATE_UNSUPPORTED: return "dstate must be between 1 and 16";
     case SELSCAN_ERR_CUDA: return "a CUDA runtime call failed (see selscan_last_cuda_error)";
-    case SELSCAN_ERR_ALIAS: return "the output y overlaps an input";
+    case SELSCAN_ERR_ALIAS: return "an output overlaps an input";
     case SELSCAN_ERR_WORKSPACE:
         return "the sizes need more chunk workspace than the static scratch array holds";
     default: return "unknown status";
@@ -363,6 +409,92 @@ int selscan_fwd_plan(int64_t batch, int64_t seqlen, int64_t dim, int64_t dstate,
     if (launches) *launches = nl;
     if (workspace_bytes_out) *workspace_bytes_out = ws;
     return SELSCAN_OK;
+}
+
+int64_t selscan_bwd_workspace_bytes(int64_t batch, int64_t seqlen, int64_t dim,
+                                    int64_t dstate) {
+    if (batch <= 0 || seqlen <= 0 || dim <= 0 || dstate < 1 || dstate > SELSCAN_MAX_DSTATE)
+        return 0;
+    if (!mul_le(batch, seqlen, kMaxElems) || !mul_le(batch * seqlen, dim, kMaxElems))
+        return 0;
+    return (int64_t)bwd_layout(batch, seqlen, dim).total;
+}
+
+int selscan_bwd(const void *x, const void *delta, const float *A, const void *B, const void *C,
+                const float *D, const void *z, const float *delta_bias, int softplus_flag,
+                const void *dy, const float *dfinal_state, void *dx, void *ddelta, float *dA,
+                float *dB, float *dC, float *dD, void *dz, float *ddelta_bias, int64_t batch,
+                int64_t seqlen, int64_t dim, int64_t dstate, selscan_dtype_t dtype,
+                selscan_stream_t stream_) {
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    if (dtype != SELSCAN_F32 && dtype != SELSCAN_BF16) return SELSCAN_ERR_BAD_DTYPE;
+    if (batch < 0 || seqlen < 0 || dim < 0 || batch > 65535) return SELSCAN_ERR_BAD_DIM;
+    if (dstate < 1 || dstate > SELSCAN_MAX_DSTATE) return SELSCAN_ERR_DSTATE_UNSUPPORTED;
+    if (!mul_le(batch, seqlen, kMaxElems) || !mul_le(batch * seqlen, dim, kMaxElems) ||
+        !mul_le(batch, dim, kMaxElems))
+        return SELSCAN_ERR_BAD_DIM;
+    const bool has_tokens = batch * seqlen * dim > 0;
+    const bool has_bc = batch * seqlen > 0;
+    if (has_tokens && (!x || !delta || !dy || !dx || !ddelta || (z && !dz)))
+        return SELSCAN_ERR_NULL_ARG;
+    if (has_bc && (!B || !C || !dB || !dC)) return SELSCAN_ERR_NULL_ARG;
+    if (dim > 0 && (!A || !dA)) return SELSCAN_ERR_NULL_ARG;
+    const size_t es = dtype == SELSCAN_F32 ? 4 : 2;
+    if (misaligned(x, es) || misaligned(delta, es) || misaligned(z, es) ||
+        misaligned(B, es) || misaligned(C, es) || misaligned(dy, es) || misaligned(dx, es) ||
+        misaligned(ddelta, es) || misaligned(dz, es) || misaligned(A, 4) ||
+        misaligned(D, 4) || misaligned(delta_bias, 4) || misaligned(dfinal_state, 4) ||
+        misaligned(dA, 4) || misaligned(dB, 4) || misaligned(dC, 4) || misaligned(dD, 4) ||
+        misaligned(ddelta_bias, 4))
+        return SELSCAN_ERR_MISALIGNED;
+    const size_t nx = (size_t)(batch * seqlen * dim) * es;
+    const size_t nbc = (size_t)(batch * seqlen * dstate) * es;
+    const size_t nbcf = (size_t)(batch * seqlen * dstate) * 4;
+    const size_t na = (size_t)(dim * dstate) * 4, nd = (size_t)dim * 4;
+    const size_t ns = (size_t)(batch * dim * dstate) * 4;
+    const Span outs[] = {{dx, nx}, {ddelta, nx}, {dz, z ? nx : 0}, {dA, na}, {dB, nbcf},
+                         {dC, nbcf}, {dD, nd}, {ddelta_bias, nd}};
+    const Span ins[] = {{x, nx}, {delta, nx}, {z, nx}, {dy, nx}, {B, nbc}, {C, nbc},
+                        {A, na}, {D, nd}, {delta_bias, nd}, {dfinal_state, ns}};
+    if (any_overlap(outs, 8, ins, 10)) return SELSCAN_ERR_ALIAS;
+
+    if (!has_tokens) {
+        // no token reaches the loss through a channel: the float32 gradients are 0
+        cudaError_t e = cudaSuccess;
+        if (e == cudaSuccess && has_bc) e = cudaMemsetAsync(dB, 0, nbcf, stream);
+        if (e == cudaSuccess && has_bc) e = cudaMemsetAsync(dC, 0, nbcf, stream);
+        if (e == cudaSuccess && dim > 0) e = cudaMemsetAsync(dA, 0, na, stream);
+        if (e == cudaSuccess && dim > 0 && dD) e = cudaMemsetAsync(dD, 0, nd, stream);
+        if (e == cudaSuccess && dim > 0 && ddelta_bias)
+            e = cudaMemsetAsync(ddelta_bias, 0, nd, stream);
+        return e == cudaSuccess ? SELSCAN_OK : selscan::cuda_fail(e);
+    }
+
+    const BwdLayout l = bwd_layout(batch, seqlen, dim);
+    selscan::BwdParams p{};
+    p.x = x; p.delta = delta; p.z = z; p.B = B; p.C = C; p.dy = dy;
+    p.A = A; p.Dskip = D; p.delta_bias = delta_bias; p.dfinal = dfinal_state;
+    p.dx = dx; p.ddelta = ddelta; p.dz = dz;
+    p.dA = dA; p.dB = dB; p.dC = dC; p.dD = dD; p.ddelta_bias = ddelta_bias;
+    p.batch = batch; p.seqlen = seqlen; p.dim = dim; p.dstate = (int)dstate;
+    p.softplus = softplus_flag ? 1 : 0;
+    p.ktiles = (int)ceil_div64(seqlen, selscan::bwd_tile_tokens());
+    p.ctiles = (int)ceil_div64(dim, selscan::bwd_tile_channels());
+    if (!mul_le(p.ctiles, 1, INT32_MAX) || !mul_le(p.ktiles, 1, INT32_MAX))
+        return SELSCAN_ERR_BAD_DIM;
+    void *ws = nullptr;
+    cudaError_t e = cudaMallocAsync(&ws, l.total, stream);
+    if (e != cudaSuccess) return selscan::cuda_fail(e);
+    char *w = static_cast<char *>(ws);
+    p.ckpt = reinterpret_cast<float *>(w + l.ckpt);
+    p.part = reinterpret_cast<float *>(w + l.part);
+    p.pA = reinterpret_cast<float *>(w + l.pA);
+    p.pD = reinterpret_cast<float *>(w + l.pD);
+    p.pbias = reinterpret_cast<float *>(w + l.pbias);
+    e = selscan::launch_scan_bwd(p, dtype == SELSCAN_BF16, stream);
+    cudaError_t ef = cudaFreeAsync(ws, stream);
+    if (e == cudaSuccess) e = ef;
+    return e == cudaSuccess ? SELSCAN_OK : selscan::cuda_fail(e);
 }
 
 int selscan_device_status(int *status, int clear) {

@@ -66,6 +66,11 @@ __device__ __forceinline__ float silu_f32(float z) {
     return z * rcp_approx(1.0f + ex2_approx(-z * kLog2e));
 }
 
+// sigmoid(v) = 1 / (1 + e^-v); e^-v overflowing to +inf gives 0.
+__device__ __forceinline__ float sigmoid_f32(float v) {
+    return rcp_approx(1.0f + ex2_approx(-v * kLog2e));
+}
+
 // ---- launch parameters -------------------------------------------------------------
 struct ScanParams {
     const void *x, *delta, *z, *B, *C;
@@ -91,6 +96,25 @@ struct StepParams {
     int64_t batch, dim;
     int dstate;
     int softplus;
+};
+
+// Gradient of the scan (scan_bwd.cu).
+struct BwdParams {
+    const void *x, *delta, *z, *B, *C, *dy;
+    const float *A, *Dskip, *delta_bias, *dfinal;
+    void *dx, *ddelta, *dz;
+    float *dA, *dB, *dC, *dD, *ddelta_bias;  // outputs written by the reduction kernel
+    // workspace
+    float *ckpt;   // [batch][ktiles][dim][16]: state entering each token tile
+    float *part;   // [batch][ctiles][seqlen][32]: per channel tile, Σ over its channels of dB (0..15), dC (16..31)
+    float *pA;     // [batch][dim][16]: Σ over tokens of dA
+    float *pD;     // [batch][dim]
+    float *pbias;  // [batch][dim]
+    long long batch, seqlen, dim;
+    int dstate;
+    int softplus;
+    int ktiles;    // token tiles per sequence
+    int ctiles;    // channel tiles per batch row
 };
 
 // Persistent TMA-staged scan (scan_tma.cu).
@@ -128,6 +152,9 @@ cudaError_t launch_carry(const ScanParams &p, cudaStream_t stream);
 
 // Host-side launchers (one translation unit per kernel family).
 cudaError_t launch_scan(const ScanParams &p, bool bf16, cudaStream_t stream);
+cudaError_t launch_scan_bwd(const BwdParams &p, bool bf16, cudaStream_t stream);
+int bwd_tile_tokens();
+int bwd_tile_channels();
 cudaError_t launch_state_update(const StepParams &p, bool bf16, cudaStream_t stream);
 int scan_channels_per_cta();
 int scan_tile_tokens();

@@ -5,8 +5,10 @@ the device) and to give quick CUDA-event timings without one:
 
     python -m selective_state_space_42_b200.profile_case scan mamba2p8b_layer --launches 2
     python -m selective_state_space_42_b200.profile_case decode --launches 3
+    python -m selective_state_space_42_b200.profile_case bwd mamba2p8b_layer --launches 2
 
-``scan`` calls selscan_fwd on a scan workload; ``decode`` calls
+``scan`` calls selscan_fwd on a scan workload; ``bwd`` calls selscan_bwd on
+it (with a seeded dy and final-state gradient); ``decode`` calls
 selscan_state_update on the decode workload. With ``--time`` it also prints
 the median CUDA-event time per launch, cold (a 512 MiB buffer is written
 between launches, which evicts L2) and back to back, as one JSON line.
@@ -36,6 +38,22 @@ def _scan_case(name: str):
     return launch, w.algorithmic_bytes()
 
 
+def _bwd_case(name: str):
+    w = wl.WORKLOADS[name]
+    inp = wl.make_scan_inputs(w, device="cuda")
+    g = torch.Generator(device="cuda")
+    g.manual_seed(w.seed + 1000)
+    dy = torch.randn(w.batch, w.seqlen, w.dim, generator=g, device="cuda").to(inp["x"].dtype)
+    dfinal = torch.randn(w.batch, w.dim, w.dstate, generator=g, device="cuda")
+
+    def launch(_i: int) -> None:
+        ss.selscan_bwd(inp["x"], inp["delta"], inp["A"], inp["B"], inp["C"], inp["D"],
+                       inp["z"], inp["delta_bias"], softplus=w.softplus, dy=dy,
+                       dfinal_state=dfinal)
+
+    return launch, w.backward_algorithmic_bytes()
+
+
 def _decode_case():
     w = wl.DECODE
     state = wl.make_decode_state(w, device="cuda")
@@ -58,19 +76,24 @@ def _median(v):
 
 def main(argv=None) -> int:
     ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
-    ap.add_argument("kernel", choices=["scan", "decode"])
+    ap.add_argument("kernel", choices=["scan", "bwd", "decode"])
     ap.add_argument("workload", nargs="?", default="mamba2p8b_layer",
                     help="scan workload name (ignored for decode)")
     ap.add_argument("--launches", type=int, default=2)
     ap.add_argument("--time", action="store_true")
     args = ap.parse_args(argv)
 
-    launch, nbytes = _scan_case(args.workload) if args.kernel == "scan" else _decode_case()
+    if args.kernel == "scan":
+        launch, nbytes = _scan_case(args.workload)
+    elif args.kernel == "bwd":
+        launch, nbytes = _bwd_case(args.workload)
+    else:
+        launch, nbytes = _decode_case()
     for i in range(args.launches):
         launch(i)
     torch.cuda.synchronize()
     out = {"kernel": args.kernel, "launches": args.launches,
-           "workload": args.workload if args.kernel == "scan" else wl.DECODE.name,
+           "workload": wl.DECODE.name if args.kernel == "decode" else args.workload,
            "algorithmic_bytes": nbytes}
     if args.time:
         flush = torch.empty(512 << 20, dtype=torch.uint8, device="cuda")

@@ -43,6 +43,9 @@ SIGNATURES = {
                                    _vp, _i64, _i64, _i64, _i64, _int, _vp]),
     "selscan_fwd_plan": (_int, [_i64, _i64, _i64, _i64, ctypes.POINTER(_i64),
                                 ctypes.POINTER(_i64), ctypes.POINTER(_i64)]),
+    "selscan_bwd": (_int, [_vp] * 8 + [_int] + [_vp] * 10
+                    + [_i64, _i64, _i64, _i64, _int, _vp]),
+    "selscan_bwd_workspace_bytes": (_i64, [_i64, _i64, _i64, _i64]),
     "selscan_device_status": (_int, [ctypes.POINTER(_int), _int]),
     "selscan_status_string": (ctypes.c_char_p, [_int]),
     "selscan_last_cuda_error": (ctypes.c_char_p, []),
@@ -215,6 +218,57 @@ def _fwd(entry, x, delta, A, B, C, D, z, delta_bias, softplus, y, final_state,
     if return_final_state:
         return y, final_state
     return y
+
+
+def selscan_bwd(x, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=True,
+                dy=None, dfinal_state=None, stream=None):
+    """Gradient of ``selscan_fwd`` (C ABI ``selscan_bwd``) for the loss
+    Σ dy·y + Σ dfinal_state·final_state. Inputs as for ``selscan_fwd``; dy has
+    y's shape and dtype, dfinal_state is [batch, dim, dstate] float32 or None.
+    Returns a dict: dx, ddelta, dz (x's dtype; dz None without z), dA, dB, dC,
+    dD, ddelta_bias (float32)."""
+    torch = _torch()
+    if x.dim() != 3:
+        raise ValueError("x must be [batch, L, dim]")
+    batch, L, dim = x.shape
+    if A.dim() != 2 or A.shape[0] != dim:
+        raise ValueError("A must be [dim, dstate]")
+    N = A.shape[1]
+    dev, dt = x.device, x.dtype
+    code = _dtype_code(x)
+    f32 = torch.float32
+    out = dict(
+        dx=torch.empty_like(x), ddelta=torch.empty_like(x),
+        dz=torch.empty_like(x) if z is not None else None,
+        dA=torch.empty(dim, N, device=dev, dtype=f32),
+        dB=torch.empty(batch, L, N, device=dev, dtype=f32),
+        dC=torch.empty(batch, L, N, device=dev, dtype=f32),
+        dD=torch.empty(dim, device=dev, dtype=f32),
+        ddelta_bias=torch.empty(dim, device=dev, dtype=f32))
+    args = [
+        _ptr(x, "x", (batch, L, dim), dt, dev),
+        _ptr(delta, "delta", (batch, L, dim), dt, dev),
+        _ptr(A, "A", (dim, N), f32, dev),
+        _ptr(B, "B", (batch, L, N), dt, dev),
+        _ptr(C, "C", (batch, L, N), dt, dev),
+        _ptr(D, "D", (dim,), f32, dev, required=False),
+        _ptr(z, "z", (batch, L, dim), dt, dev, required=False),
+        _ptr(delta_bias, "delta_bias", (dim,), f32, dev, required=False),
+        int(bool(softplus)),
+        _ptr(dy, "dy", (batch, L, dim), dt, dev),
+        _ptr(dfinal_state, "dfinal_state", (batch, dim, N), f32, dev, required=False),
+        _ptr(out["dx"], "dx"), _ptr(out["ddelta"], "ddelta"), _ptr(out["dA"], "dA"),
+        _ptr(out["dB"], "dB"), _ptr(out["dC"], "dC"), _ptr(out["dD"], "dD"),
+        _ptr(out["dz"], "dz", required=False), _ptr(out["ddelta_bias"], "ddelta_bias"),
+        batch, L, dim, N, code, _stream_ptr(stream, dev),
+    ]
+    _check(load_library().selscan_bwd(*args))
+    return out
+
+
+def selscan_bwd_workspace_bytes(batch: int, seqlen: int, dim: int, dstate: int) -> int:
+    """Device workspace bytes ``selscan_bwd`` allocates for these sizes."""
+    return int(load_library().selscan_bwd_workspace_bytes(batch, seqlen, dim, dstate))
 
 
 def selscan_state_update(state, x, delta, A, B, C, D=None, z=None, delta_bias=None,

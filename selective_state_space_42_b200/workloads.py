@@ -57,6 +57,20 @@ class ScanWorkload:
         return (self.batch * self.seqlen * self.dim * per_bld
                 + self.batch * self.seqlen * per_bl + fixed)
 
+    def backward_algorithmic_bytes(self) -> int:
+        """Minimum HBM bytes of the gradient pass: x, delta, z, dy in and dx,
+        ddelta, dz out per (b, l, d); B and C in and dB, dC (float32) out per
+        (b, l); A, D, delta_bias and the final-state gradient in, dA, dD,
+        ddelta_bias out."""
+        es = 4 if self.dtype == "f32" else 2
+        gates = 2 if self.gate else 0  # z in, dz out
+        per_bld = (4 + 2 + gates) * es
+        per_bl = 2 * self.dstate * es + 2 * self.dstate * 4
+        fixed = 2 * (self.dim * self.dstate * 4 + 2 * self.dim * 4)
+        fixed += self.batch * self.dim * self.dstate * 4
+        return (self.batch * self.seqlen * self.dim * per_bld
+                + self.batch * self.seqlen * per_bl + fixed)
+
     def scaled(self, **kw) -> "ScanWorkload":
         return dataclasses.replace(self, **kw)
 

@@ -121,3 +121,47 @@ def test_binding_rejects_cpu_tensors(lib):
     with pytest.raises(ValueError):
         ss.selscan_fwd(x, x, torch.zeros(8, 16), torch.zeros(1, 4, 16),
                        torch.zeros(1, 4, 16))
+
+
+def bwd(lib, **kw):
+    names = ["x", "delta", "A", "B", "C", "D", "z", "delta_bias", "dy", "dfinal",
+             "dx", "ddelta", "dA", "dB", "dC", "dD", "dz", "ddelta_bias"]
+    a = {n: P + 4096 * i for i, n in enumerate(names)}
+    a.update(D=None, z=None, delta_bias=None, dfinal=None, dz=None, softplus=1,
+             batch=0, seqlen=8, dim=0, dstate=16, dtype=1, stream=None)
+    a.update(kw)
+    return lib.selscan_bwd(a["x"], a["delta"], a["A"], a["B"], a["C"], a["D"], a["z"],
+                           a["delta_bias"], a["softplus"], a["dy"], a["dfinal"], a["dx"],
+                           a["ddelta"], a["dA"], a["dB"], a["dC"], a["dD"], a["dz"],
+                           a["ddelta_bias"], a["batch"], a["seqlen"], a["dim"],
+                           a["dstate"], a["dtype"], a["stream"])
+
+
+def test_bwd_validation(lib):
+    """Every check runs before any CUDA call (no GPU here)."""
+    assert bwd(lib) == 0  # batch = 0 and dim = 0: no output has an element
+    assert bwd(lib, dtype=7) == -3
+    assert bwd(lib, batch=-1) == -2
+    assert bwd(lib, batch=70000, dim=4) == -2  # batch rows are a grid dimension
+    assert bwd(lib, dstate=0) == -5
+    full = dict(batch=1, dim=4)
+    assert bwd(lib, x=None, **full) == -1
+    assert bwd(lib, dy=None, **full) == -1
+    assert bwd(lib, dx=None, **full) == -1
+    assert bwd(lib, dB=None, **full) == -1
+    assert bwd(lib, A=None, **full) == -1
+    assert bwd(lib, dA=None, **full) == -1
+    assert bwd(lib, z=P + 4096 * 40, dz=None, **full) == -1  # dz required with z
+    assert bwd(lib, dx=P + 4096 * 10 + 1, **full) == -4
+    assert bwd(lib, dA=P + 4096 * 12 + 2, **full) == -4
+    assert bwd(lib, dx=P, **full) == -7  # dx == x
+    assert bwd(lib, dB=P + 4096 * 3 + 64, **full) == -7  # dB runs into B
+    assert bwd(lib, ddelta=P + 4096 * 10, **full) == -7  # two outputs overlap
+
+
+def test_bwd_workspace_bytes(lib):
+    assert lib.selscan_bwd_workspace_bytes(0, 8, 4, 16) == 0
+    assert lib.selscan_bwd_workspace_bytes(1, 8, 4, 17) == 0
+    # one 16-token tile, one 32-channel tile: checkpoints 4·16·4 B, partials
+    # 8·32·4 B, per-channel partials 4·(16 + 2)·4 B, each rounded up to 256 B
+    assert lib.selscan_bwd_workspace_bytes(1, 8, 4, 16) == 256 + 1024 + 256 + 256 + 256

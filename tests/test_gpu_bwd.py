@@ -1,0 +1,160 @@
+"""GPU parity of selscan_bwd (the gradient of the scan) against the float64
+oracle's reverse sweep, through the C ABI."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import selective_state_space_42_b200 as ss
+from selective_state_space_42_b200 import workloads as wl
+
+import gpu_helpers as gh
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+GRADS = ("dx", "ddelta", "dz", "dA", "dB", "dC", "dD", "ddelta_bias")
+
+
+def _inputs(batch, L, dim, N, dtype, gate, seed, structured=True, dfinal=True):
+    w = wl.ScanWorkload("bwd", batch, L, dim, N, dtype, gate=gate, seed=seed)
+    inp = wl.make_scan_inputs(w)
+    if not structured:
+        g = torch.Generator().manual_seed(seed + 1)
+        inp["A"] = -torch.rand(dim, N, generator=g) * 4 - 0.1
+    g = torch.Generator().manual_seed(seed + 2)
+    dy = torch.randn(batch, L, dim, generator=g).to(inp["x"].dtype)
+    df = torch.randn(batch, dim, N, generator=g) if dfinal else None
+    return inp, dy, df
+
+
+def _gpu_bwd(inp, dy, df, softplus=True):
+    d = {k: (None if v is None else v.to(DEV)) for k, v in inp.items()}
+    return ss.selscan_bwd(d["x"], d["delta"], d["A"], d["B"], d["C"], d["D"], d["z"],
+                          d["delta_bias"], softplus=softplus, dy=dy.to(DEV),
+                          dfinal_state=None if df is None else df.to(DEV))
+
+
+def _oracle_bwd(inp, dy, df, softplus=True, channels=None):
+    sel = slice(None) if channels is None else list(channels)
+
+    def bl(t):
+        return None if t is None else gh.to_np(t[:, :, sel])
+
+    def ch(t):
+        return None if t is None else gh.to_np(t[sel])
+
+    return oracle.default().bwd(
+        bl(inp["x"]), bl(inp["delta"]), ch(inp["A"]), gh.to_np(inp["B"]), gh.to_np(inp["C"]),
+        ch(inp["D"]), bl(inp["z"]), ch(inp["delta_bias"]), softplus=softplus, dy=bl(dy),
+        dfinal=None if df is None else gh.to_np(df[:, sel]))
+
+
+def _compare_all(g, o, dtype, what, names=GRADS):
+    rtol = gh.RTOL[dtype]
+    for k in names:
+        if o.get(k) is None:
+            assert g.get(k) is None, f"{what}: {k} should be absent"
+            continue
+        gh.compare(gh.to_np(g[k]), o[k], rtol, f"{what} {k}")
+
+
+SHAPES = [(1, 1, 1, 1), (2, 31, 33, 16), (1, 40, 64, 16), (3, 17, 5, 4), (2, 50, 70, 7),
+          (1, 300, 40, 16), (2, 16, 32, 16), (1, 257, 96, 8)]
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("shape", SHAPES, ids=str)
+@pytest.mark.parametrize("gate", [True, False])
+def test_small_every_element(dtype, shape, gate):
+    batch, L, dim, N = shape
+    inp, dy, df = _inputs(batch, L, dim, N, dtype, gate, seed=100 + L + dim)
+    g = _gpu_bwd(inp, dy, df)
+    torch.cuda.synchronize()
+    _compare_all(g, _oracle_bwd(inp, dy, df), dtype, f"{shape}")
+
+
+@pytest.mark.parametrize("structured", [True, False])
+@pytest.mark.parametrize("softplus", [True, False])
+def test_variants(structured, softplus):
+    inp, dy, df = _inputs(2, 100, 48, 16, "f32", True, seed=7, structured=structured,
+                          dfinal=not softplus)
+    if not softplus:  # Δ = delta + bias itself: keep it positive
+        inp["delta"] = inp["delta"].abs() + 0.05
+        inp["delta_bias"] = torch.full_like(inp["delta_bias"], 0.01)
+    g = _gpu_bwd(inp, dy, df, softplus=softplus)
+    torch.cuda.synchronize()
+    _compare_all(g, _oracle_bwd(inp, dy, df, softplus=softplus), "f32",
+                 f"structured={structured} softplus={softplus}")
+
+
+def test_medium_130m_shape():
+    """A Mamba-130M-shaped layer cut to 2 × 512 tokens × 1536 channels, every
+    element of every gradient."""
+    inp, dy, df = _inputs(2, 512, 1536, 16, "bf16", True, seed=11)
+    g = _gpu_bwd(inp, dy, df)
+    torch.cuda.synchronize()
+    _compare_all(g, _oracle_bwd(inp, dy, df), "bf16", "130m-shaped")
+
+
+def test_deterministic():
+    inp, dy, df = _inputs(2, 200, 100, 16, "bf16", True, seed=12)
+    g1 = _gpu_bwd(inp, dy, df)
+    g2 = _gpu_bwd(inp, dy, df)
+    torch.cuda.synchronize()
+    for k in GRADS:
+        assert torch.equal(g1[k], g2[k]), k
+
+
+def test_empty_and_degenerate():
+    # no tokens: float32 gradients are zero, token gradients empty
+    inp, dy, df = _inputs(2, 0, 8, 16, "bf16", True, seed=13)
+    g = _gpu_bwd(inp, dy, df)
+    torch.cuda.synchronize()
+    for k in ("dA", "dD", "ddelta_bias"):
+        assert torch.count_nonzero(g[k]) == 0, k
+    assert g["dx"].numel() == 0 and g["dB"].numel() == 0
+    # no channels: dB and dC are zero
+    w = wl.ScanWorkload("nodim", 2, 5, 0, 16, "bf16", gate=True, seed=14)
+    inp = wl.make_scan_inputs(w)
+    dy = torch.zeros(2, 5, 0, dtype=torch.bfloat16)
+    g = _gpu_bwd(inp, dy, None)
+    torch.cuda.synchronize()
+    assert g["dB"].shape == (2, 5, 16) and torch.count_nonzero(g["dB"]) == 0
+    assert torch.count_nonzero(g["dC"]) == 0
+
+
+def test_bench_shape_sampled_and_identities():
+    """The Mamba-2.8B-shaped layer (4 × 8192 × 5120, N = 16, bf16, gated):
+    per-channel gradients on a channel sample against the oracle on those
+    channels (channels are independent chains), and the channel sums dB, dC
+    through identities that hold at any size:
+        Σ dC·C = Σ dy·(y − D·x·silu(z)),   Σ dB·B = Σ dC·C + Σ dfinal·h_final
+    (h0 = 0; y and h_final from the GPU forward)."""
+    w = wl.WORKLOADS["mamba2p8b_layer"]
+    inp = wl.make_scan_inputs(w, device=DEV)
+    g = torch.Generator(device=DEV).manual_seed(99)
+    dy = torch.randn(w.batch, w.seqlen, w.dim, generator=g, device=DEV).to(torch.bfloat16)
+    df = torch.randn(w.batch, w.dim, w.dstate, generator=g, device=DEV)
+    grads = ss.selscan_bwd(inp["x"], inp["delta"], inp["A"], inp["B"], inp["C"], inp["D"],
+                           inp["z"], inp["delta_bias"], dy=dy, dfinal_state=df)
+    y, hf = ss.selscan_fwd(inp["x"], inp["delta"], inp["A"], inp["B"], inp["C"], inp["D"],
+                           inp["z"], inp["delta_bias"], return_final_state=True)
+    torch.cuda.synchronize()
+    chans = wl.channel_subset(w.dim, 64)
+    o = _oracle_bwd(inp, dy, df, channels=chans)
+    sel = list(chans)
+    for k in ("dx", "ddelta", "dz"):
+        gh.compare(gh.to_np(grads[k][:, :, sel]), o[k], gh.RTOL["bf16"], f"bench {k}")
+    for k in ("dA", "dD", "ddelta_bias"):
+        gh.compare(gh.to_np(grads[k][sel]), o[k], gh.RTOL["bf16"], f"bench {k}")
+    f64 = torch.float64
+    x, z = inp["x"].to(f64), inp["z"].to(f64)
+    ylin = y.to(f64) - inp["D"].to(f64) * x * (z * torch.sigmoid(z))
+    lhs_c = float((grads["dC"].to(f64) * inp["C"].to(f64)).sum())
+    rhs_c = float((dy.to(f64) * ylin).sum())
+    assert abs(lhs_c - rhs_c) <= 2e-2 * (abs(rhs_c) + float((dy.to(f64) * ylin).abs().sum()) / 1e3), \
+        (lhs_c, rhs_c)
+    lhs_b = float((grads["dB"].to(f64) * inp["B"].to(f64)).sum())
+    rhs_b = lhs_c + float((df.to(f64) * hf.to(f64)).sum())
+    assert abs(lhs_b - rhs_b) <= 1e-3 * (abs(rhs_b) + abs(lhs_c)), (lhs_b, rhs_b)
