@@ -67,8 +67,8 @@ enum {
     SELSCAN_ERR_DSTATE_UNSUPPORTED = -5, /* dstate outside 1..16 */
     SELSCAN_ERR_CUDA = -6,               /* a CUDA call failed */
     SELSCAN_ERR_ALIAS = -7,              /* y overlaps an input */
-    SELSCAN_ERR_WORKSPACE = -8           /* selscan_fwd_noalloc: the plan needs more
-                                            workspace than its static array holds */
+    SELSCAN_ERR_WORKSPACE = -8           /* the given or static workspace is too small
+                                            (selscan_fwd_noalloc, selscan_bwd_workspace) */
 };
 
 #define SELSCAN_MAX_DSTATE 16
@@ -210,7 +210,7 @@ SELSCAN_API int selscan_state_update(float *state, const void *x, const void *de
  * (fixed summation order, no atomics). Outputs must not overlap any input.
  * Takes a stream-ordered device workspace (cudaMallocAsync / cudaFreeAsync
  * on `stream`) of selscan_bwd_workspace_bytes() bytes: the state entering
- * every 16-token tile of every chain, and per-32-channel partial sums of dB
+ * every 8-token tile of every chain, and per-32-channel partial sums of dB
  * and dC.
  */
 SELSCAN_API int selscan_bwd(const void *x, const void *delta, const float *A,
@@ -225,6 +225,28 @@ SELSCAN_API int selscan_bwd(const void *x, const void *delta, const float *A,
  * (0 for empty or invalid sizes). */
 SELSCAN_API int64_t selscan_bwd_workspace_bytes(int64_t batch, int64_t seqlen, int64_t dim,
                                                 int64_t dstate);
+
+/*
+ * selscan_bwd_workspace -- selscan_bwd on a workspace the caller provides
+ * (e.g. from its own caching allocator) instead of one allocated on the
+ * stream: same arguments and results, plus
+ *   workspace        device buffer, 256-byte aligned, must not overlap any
+ *                    input or output; NULL only when no token is processed
+ *   workspace_bytes  its size: at least selscan_bwd_workspace_bytes() for
+ *                    these sizes, else SELSCAN_ERR_WORKSPACE
+ * Nothing is allocated. The workspace is free for reuse once the call's work
+ * on `stream` has completed; its contents are not meaningful afterwards.
+ */
+SELSCAN_API int selscan_bwd_workspace(const void *x, const void *delta, const float *A,
+                                      const void *B, const void *C, const float *D,
+                                      const void *z, const float *delta_bias,
+                                      int softplus_flag, const void *dy,
+                                      const float *dfinal_state, void *dx, void *ddelta,
+                                      float *dA, float *dB, float *dC, float *dD, void *dz,
+                                      float *ddelta_bias, int64_t batch, int64_t seqlen,
+                                      int64_t dim, int64_t dstate, selscan_dtype_t dtype,
+                                      void *workspace, int64_t workspace_bytes,
+                                      selscan_stream_t stream);
 
 /*
  * selscan_device_status -- the library's sticky device-side error word on

@@ -420,12 +420,19 @@ int64_t selscan_bwd_workspace_bytes(int64_t batch, int64_t seqlen, int64_t dim,
     return (int64_t)bwd_layout(batch, seqlen, dim).total;
 }
 
-int selscan_bwd(const void *x, const void *delta, const float *A, const void *B, const void *C,
-                const float *D, const void *z, const float *delta_bias, int softplus_flag,
-                const void *dy, const float *dfinal_state, void *dx, void *ddelta, float *dA,
-                float *dB, float *dC, float *dD, void *dz, float *ddelta_bias, int64_t batch,
-                int64_t seqlen, int64_t dim, int64_t dstate, selscan_dtype_t dtype,
-                selscan_stream_t stream_) {
+}  // extern "C"
+
+namespace {
+
+// Shared by selscan_bwd (workspace == NULL: allocated on the stream) and
+// selscan_bwd_workspace (the caller's workspace).
+int bwd_entry(const void *x, const void *delta, const float *A, const void *B, const void *C,
+              const float *D, const void *z, const float *delta_bias, int softplus_flag,
+              const void *dy, const float *dfinal_state, void *dx, void *ddelta, float *dA,
+              float *dB, float *dC, float *dD, void *dz, float *ddelta_bias, int64_t batch,
+              int64_t seqlen, int64_t dim, int64_t dstate, selscan_dtype_t dtype,
+              void *workspace, int64_t workspace_bytes, bool allocate,
+              selscan_stream_t stream_) {
     cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
     if (dtype != SELSCAN_F32 && dtype != SELSCAN_BF16) return SELSCAN_ERR_BAD_DTYPE;
     if (batch < 0 || seqlen < 0 || dim < 0 || batch > 65535) return SELSCAN_ERR_BAD_DIM;
@@ -445,7 +452,7 @@ int selscan_bwd(const void *x, const void *delta, const float *A, const void *B,
         misaligned(ddelta, es) || misaligned(dz, es) || misaligned(A, 4) ||
         misaligned(D, 4) || misaligned(delta_bias, 4) || misaligned(dfinal_state, 4) ||
         misaligned(dA, 4) || misaligned(dB, 4) || misaligned(dC, 4) || misaligned(dD, 4) ||
-        misaligned(ddelta_bias, 4))
+        misaligned(ddelta_bias, 4) || misaligned(workspace, 256))
         return SELSCAN_ERR_MISALIGNED;
     const size_t nx = (size_t)(batch * seqlen * dim) * es;
     const size_t nbc = (size_t)(batch * seqlen * dstate) * es;
@@ -471,6 +478,13 @@ int selscan_bwd(const void *x, const void *delta, const float *A, const void *B,
     }
 
     const BwdLayout l = bwd_layout(batch, seqlen, dim);
+    if (!allocate) {
+        if (!workspace) return SELSCAN_ERR_NULL_ARG;
+        if (workspace_bytes < (int64_t)l.total) return SELSCAN_ERR_WORKSPACE;
+        const Span wsp[] = {{workspace, l.total}};
+        if (any_overlap(wsp, 1, outs, 8) || any_overlap(wsp, 1, ins, 10))
+            return SELSCAN_ERR_ALIAS;
+    }
     selscan::BwdParams p{};
     p.x = x; p.delta = delta; p.z = z; p.B = B; p.C = C; p.dy = dy;
     p.A = A; p.Dskip = D; p.delta_bias = delta_bias; p.dfinal = dfinal_state;
@@ -482,9 +496,12 @@ int selscan_bwd(const void *x, const void *delta, const float *A, const void *B,
     p.ctiles = (int)ceil_div64(dim, selscan::bwd_tile_channels());
     if (!mul_le(p.ctiles, 1, INT32_MAX) || !mul_le(p.ktiles, 1, INT32_MAX))
         return SELSCAN_ERR_BAD_DIM;
-    void *ws = nullptr;
-    cudaError_t e = cudaMallocAsync(&ws, l.total, stream);
-    if (e != cudaSuccess) return selscan::cuda_fail(e);
+    void *ws = workspace;
+    cudaError_t e = cudaSuccess;
+    if (allocate) {
+        e = cudaMallocAsync(&ws, l.total, stream);
+        if (e != cudaSuccess) return selscan::cuda_fail(e);
+    }
     char *w = static_cast<char *>(ws);
     p.ckpt = reinterpret_cast<float *>(w + l.ckpt);
     p.part = reinterpret_cast<float *>(w + l.part);
@@ -492,9 +509,39 @@ int selscan_bwd(const void *x, const void *delta, const float *A, const void *B,
     p.pD = reinterpret_cast<float *>(w + l.pD);
     p.pbias = reinterpret_cast<float *>(w + l.pbias);
     e = selscan::launch_scan_bwd(p, dtype == SELSCAN_BF16, stream);
-    cudaError_t ef = cudaFreeAsync(ws, stream);
-    if (e == cudaSuccess) e = ef;
+    if (allocate) {
+        cudaError_t ef = cudaFreeAsync(ws, stream);
+        if (e == cudaSuccess) e = ef;
+    }
     return e == cudaSuccess ? SELSCAN_OK : selscan::cuda_fail(e);
+}
+
+}  // namespace
+
+extern "C" {
+
+int selscan_bwd(const void *x, const void *delta, const float *A, const void *B, const void *C,
+                const float *D, const void *z, const float *delta_bias, int softplus_flag,
+                const void *dy, const float *dfinal_state, void *dx, void *ddelta, float *dA,
+                float *dB, float *dC, float *dD, void *dz, float *ddelta_bias, int64_t batch,
+                int64_t seqlen, int64_t dim, int64_t dstate, selscan_dtype_t dtype,
+                selscan_stream_t stream) {
+    return bwd_entry(x, delta, A, B, C, D, z, delta_bias, softplus_flag, dy, dfinal_state, dx,
+                     ddelta, dA, dB, dC, dD, dz, ddelta_bias, batch, seqlen, dim, dstate, dtype,
+                     nullptr, 0, true, stream);
+}
+
+int selscan_bwd_workspace(const void *x, const void *delta, const float *A, const void *B,
+                          const void *C, const float *D, const void *z,
+                          const float *delta_bias, int softplus_flag, const void *dy,
+                          const float *dfinal_state, void *dx, void *ddelta, float *dA,
+                          float *dB, float *dC, float *dD, void *dz, float *ddelta_bias,
+                          int64_t batch, int64_t seqlen, int64_t dim, int64_t dstate,
+                          selscan_dtype_t dtype, void *workspace, int64_t workspace_bytes,
+                          selscan_stream_t stream) {
+    return bwd_entry(x, delta, A, B, C, D, z, delta_bias, softplus_flag, dy, dfinal_state, dx,
+                     ddelta, dA, dB, dC, dD, dz, ddelta_bias, batch, seqlen, dim, dstate, dtype,
+                     workspace, workspace_bytes, false, stream);
 }
 
 int selscan_device_status(int *status, int clear) {

@@ -16,369 +16,386 @@
 //   dD += ds_t·x_t,  dz_t = dy_t·s_t·silu'(z_t),  ddelta_t = dΔ_t·σ(delta_t + bias)
 // with u_t = Δ_t·x_t and s_t = Σ_n C_t[n]·h_t[n] + D·x_t.
 //
-// Organisation. A CTA owns 32 channels of one batch row for the whole
-// sequence (no inter-CTA dependency). Lanes work in quads: lane (chain j,
-// quarter q) holds states 4q..4q+3 of one chain. Tokens go in tiles of 16:
-//  1. forward sweep: every tile's entering state is stored as a checkpoint
-//     (float32, [batch][tiles][dim][16], 512 contiguous bytes per warp);
-//  2. reverse sweep over the tiles, last first: recompute the tile's 16
-//     states per lane from its checkpoint into registers, then walk the tile
-//     backwards carrying λ in registers.
-// Per-(token, channel) scalars (softplus, sigmoid, silu and its derivative,
-// the decay base) are computed once by an owner thread into shared memory;
-// the quad lanes read them. Channel sums of dB and dC are reduced within a
-// warp by a shuffle reduce-scatter (8 values per lane → 1), across the 4
-// warps in shared memory, and across channel tiles by a second kernel from a
-// per-tile partial buffer (deterministic, no atomics). dA, dD and ddelta_bias
-// are per-(batch row, channel) partials summed over batch rows the same way.
+// Organisation. One thread per (batch row, channel) chain holds its 16
+// states in registers, two per packed f32x2 instruction; a CTA is one warp of
+// 32 consecutive channels of one batch row and owns them for the whole
+// sequence (no inter-CTA dependency). Tokens go in tiles of 8:
+//  1. forward sweep: the state entering every tile is stored as a checkpoint
+//     (float32, [batch][tiles][dim][16]);
+//  2. reverse sweep over the tiles, last first: recompute the tile's states
+//     from its checkpoint into shared memory (with the per-token scalars:
+//     softplus, its derivative σ, silu(z) and its derivative, the decay base),
+//     then walk the tile backwards carrying λ in registers.
+// Global inputs of the next tile (x, delta, z, dy, B, C, the checkpoint) are
+// loaded into registers while the current tile is computed. The channel sums
+// of dB and dC are formed per token through shared memory (each lane writes
+// its 32 values, swizzled so that the writes and the column reads are free of
+// bank conflicts; eight lanes sum each group of four values over 8 channels,
+// two shuffles finish the warp sum) and written as one 128-byte row per token
+// to a per-channel-tile partial buffer, which a second kernel sums over the
+// channel tiles: deterministic, no atomics. dA, dD and ddelta_bias are
+// per-(batch row, channel) partials summed over batch rows the same way.
 #include "selscan_device.cuh"
 
 namespace selscan {
 namespace {
 
-constexpr int kSeg = 16;                 // tokens per tile (checkpoint interval)
-constexpr int kChains = 32;              // channels per CTA
-constexpr int kThreads = 4 * kChains;    // four lanes per channel
-constexpr int kWarps = kThreads / 32;
+constexpr int kSeg = 8;                  // tokens per tile (checkpoint interval)
+constexpr int kChains = 32;              // channels per CTA: one warp
 constexpr int kVals = 2 * kMaxN;         // dB and dC values per token
+constexpr int kPairs = kMaxN / 2;        // f32x2 registers per state vector
+
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+__device__ __forceinline__ float2 dup2(float v) { return make_float2(v, v); }
 
 struct BwdSmem {
-    float4 sc[kSeg][kChains];   // Δ, u = Δ·x, ds = dy·silu(z), r = 2^(Δ·A[d,0]·log2 e)
-    float4 so[kSeg][kChains];   // x, dy·silu'(z), σ(delta + bias), 0 (owner epilogue)
-    float Bs[kSeg][kMaxN];      // B and C of the tile, float32, zero beyond dstate
+    float Bs[kSeg][kMaxN];             // B and C of the tile, float32, zero beyond dstate
     float Cs[kSeg][kMaxN];
-    float s[kSeg][kChains];     // Σ_n C·h
-    float2 duq[kSeg][kChains];  // Σ_n λ·B, Σ_n λ·A·Abar·h_prev
-    float red[kWarps][kSeg][kVals];
+    float4 sc[kSeg][kChains];          // Δ, u = Δ·x, ds = dy·silu(z), r = 2^(Δ·A[d,0]·log2 e)
+    float4 so[kSeg][kChains];          // x, dy·silu'(z), σ(delta + bias), s = Σ C·h + D·x
+    float4 hs[kSeg + 1][4][kChains];   // hs[0]: entering state; hs[t + 1]: after token t
+    float4 red[kVals / 4][kChains];    // one token's dB (groups 0-3), dC (4-7), swizzled
 };
 
-// Decay factors Abar for the lane's four states at one token.
-// Structured A (A[d, n] = (n+1)·A[d, 0]): powers of r; otherwise one ex2 each.
-__device__ __forceinline__ void decay4(bool structured, int q, float dt, float r,
-                                       const float (&Av)[4], float (&a)[4]) {
-    if (structured) {
-        const float r2 = r * r, r4 = r2 * r2, r8 = r4 * r4;
-        const float base = q == 0 ? 1.0f : (q == 1 ? r4 : (q == 2 ? r8 : r8 * r4));
-        a[0] = base * r;
-        a[1] = a[0] * r;
-        a[2] = a[1] * r;
-        a[3] = a[2] * r;
-    } else {
-        const float dl = dt * kLog2e;
+// Raw per-token inputs of one tile for this lane's channel.
+template <typename T> struct Raw {
+    T x[kSeg], dl[kSeg], z[kSeg], dy[kSeg];
+};
+
+template <typename T, bool kGate, bool kBwd>
+__device__ __forceinline__ void load_raw(Raw<T> &r, const BwdParams &p, long long b,
+                                         long long t0, long long d, bool active) {
+    const T zero = from_f32<T>(0.0f);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) a[i] = ex2_approx(dl * Av[i]);
+    for (int t = 0; t < kSeg; ++t) {
+        const long long tok = t0 + t;
+        const bool ok = active && tok < p.seqlen;
+        const long long i = (b * p.seqlen + tok) * p.dim + d;
+        r.x[t] = ok ? __ldg(static_cast<const T *>(p.x) + i) : zero;
+        r.dl[t] = ok ? __ldg(static_cast<const T *>(p.delta) + i) : zero;
+        if (kBwd) {
+            r.dy[t] = ok ? __ldg(static_cast<const T *>(p.dy) + i) : zero;
+            if (kGate) r.z[t] = ok ? __ldg(static_cast<const T *>(p.z) + i) : zero;
+        }
     }
 }
 
+// Four B and four C elements of the tile for this lane: token lane / 4,
+// states 4·(lane % 4) .. + 3 (zero past the end or past dstate).
 template <typename T>
-__device__ __forceinline__ void load_bc(BwdSmem &S, const BwdParams &p, long long b,
-                                        long long t0, bool withC) {
-    const T *Bp = static_cast<const T *>(p.B);
-    const T *Cp = static_cast<const T *>(p.C);
-    for (int e = threadIdx.x; e < kSeg * kMaxN; e += kThreads) {
-        const int t = e / kMaxN, n = e % kMaxN;
-        const long long tok = t0 + t;
-        const bool ok = tok < p.seqlen && n < p.dstate;
-        const long long idx = (b * p.seqlen + tok) * p.dstate + n;
-        S.Bs[t][n] = ok ? ldg_f32(Bp + idx) : 0.0f;
-        if (withC) S.Cs[t][n] = ok ? ldg_f32(Cp + idx) : 0.0f;
-    }
-}
-
-// Owner step: per-(token, channel) scalars of tile t0 into shared memory.
-// Tokens past the end and channels past dim get Δ = u = ds = 0 and r = 1,
-// which leave every state and every gradient unchanged.
-template <typename T, bool kGate, bool kSoftplus, bool kBwd>
-__device__ __forceinline__ void owner_scalars(BwdSmem &S, const BwdParams &p, long long b,
-                                              long long t0, int oc, int ot, long long od,
-                                              float A0, float bias) {
-    const T *xp = static_cast<const T *>(p.x);
-    const T *dp = static_cast<const T *>(p.delta);
-#pragma unroll
-    for (int m = 0; m < kSeg / kWarps; ++m) {
-        const int t = ot + kWarps * m;
-        const long long tok = t0 + t;
-        float4 sc = make_float4(0.f, 0.f, 0.f, 1.f);
-        float4 so = make_float4(0.f, 0.f, 1.f, 0.f);
-        if (od < p.dim && tok < p.seqlen) {
-            const long long i = (b * p.seqlen + tok) * p.dim + od;
-            const float xv = ldg_f32(xp + i);
-            const float v = ldg_f32(dp + i) + bias;
-            const float dt = kSoftplus ? softplus_f32(v) : v;
-            sc.x = dt;
-            sc.y = dt * xv;
-            sc.w = ex2_approx(dt * A0 * kLog2e);
-            if (kBwd) {
-                const float dyv = ldg_f32(static_cast<const T *>(p.dy) + i);
-                if (kGate) {
-                    const float zv = ldg_f32(static_cast<const T *>(p.z) + i);
-                    const float sg = sigmoid_f32(zv);
-                    sc.z = dyv * zv * sg;
-                    so.y = dyv * sg * fmaf(zv, 1.0f - sg, 1.0f);
-                } else {
-                    sc.z = dyv;
-                }
-                so.x = xv;
-                so.z = kSoftplus ? sigmoid_f32(v) : 1.0f;
-            }
-        }
-        S.sc[t][oc] = sc;
-        if (kBwd) S.so[t][oc] = so;
-    }
-}
-
-constexpr int kHalf = kSeg / 2;
-
-// Shared-memory loads the compiler may neither merge with an earlier load of
-// the same address nor move across one another: each token's operands are
-// read when they are used, which keeps the per-token values of a half tile
-// from all being live at once.
-__device__ __forceinline__ float4 lds4(const void *ptr) {
-    float4 v;
-    const unsigned a = static_cast<unsigned>(__cvta_generic_to_shared(ptr));
-    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
-                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-                 : "r"(a));
-    return v;
-}
-
-// One token of the recurrence for the lane's four states.
-__device__ __forceinline__ void fwd_token(const BwdSmem &S, int t, int jc, int q, bool structured,
-                                          const float (&Av)[4], const float (&hin)[4],
-                                          float (&hout)[4]) {
-    const float4 sc = lds4(&S.sc[t][jc]);
-    const float4 b4 = lds4(&S.Bs[t][4 * q]);
-    float a[4];
-    decay4(structured, q, sc.x, sc.w, Av, a);
-    hout[0] = fmaf(a[0], hin[0], sc.y * b4.x);
-    hout[1] = fmaf(a[1], hin[1], sc.y * b4.y);
-    hout[2] = fmaf(a[2], hin[2], sc.y * b4.z);
-    hout[3] = fmaf(a[3], hin[3], sc.y * b4.w);
-}
-
-// States through tokens kBase .. kBase + kHalf − 1 of the tile, nothing kept.
-template <int kBase>
-__device__ __forceinline__ void advance(const BwdSmem &S, int jc, int q, bool structured,
-                                        const float (&Av)[4], float (&h)[4]) {
-#pragma unroll
-    for (int t = kBase; t < kBase + kHalf; ++t) {
-        float hn[4];
-        fwd_token(S, t, jc, q, structured, Av, h, hn);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) h[i] = hn[i];
-    }
-}
-
-// Tokens kBase .. kBase + kHalf − 1 of the tile: recompute their states from
-// h (the state entering token kBase) into registers, store Σ_n C·h for the
-// epilogue, then walk them backwards updating λ and the per-token gradients.
-template <int kBase>
-__device__ __forceinline__ void half_tile(BwdSmem &S, int jc, int q, int lane, int warp,
-                                          bool structured, const float (&Av)[4],
-                                          const float (&h)[4], float (&lam)[4],
-                                          float (&dAacc)[4]) {
-    float hs[kHalf + 1][4];  // hs[t + 1]: state after token kBase + t
-#pragma unroll
-    for (int i = 0; i < 4; ++i) hs[0][i] = h[i];
-#pragma unroll
-    for (int t = 0; t < kHalf; ++t) {
-        fwd_token(S, kBase + t, jc, q, structured, Av, hs[t], hs[t + 1]);
-        const float4 c4 = lds4(&S.Cs[kBase + t][4 * q]);
-        float sp = c4.x * hs[t + 1][0];
-        sp = fmaf(c4.y, hs[t + 1][1], sp);
-        sp = fmaf(c4.z, hs[t + 1][2], sp);
-        sp = fmaf(c4.w, hs[t + 1][3], sp);
-        sp += __shfl_xor_sync(0xffffffffu, sp, 1);
-        sp += __shfl_xor_sync(0xffffffffu, sp, 2);
-        if (q == 0) S.s[kBase + t][jc] = sp;
-    }
-    const int jw = lane >> 2;
-    const int b4bit = (lane >> 4) & 1, b3bit = (lane >> 3) & 1, b2bit = (lane >> 2) & 1;
-#pragma unroll
-    for (int t = kHalf - 1; t >= 0; --t) {
-        const int tt = kBase + t;
-        const float4 sc = lds4(&S.sc[tt][jc]);
-        const float4 b4 = lds4(&S.Bs[tt][4 * q]);
-        const float4 c4 = lds4(&S.Cs[tt][4 * q]);
-        const float bv[4] = {b4.x, b4.y, b4.z, b4.w};
-        const float cv[4] = {c4.x, c4.y, c4.z, c4.w};
-        float a[4];
-        decay4(structured, q, sc.x, sc.w, Av, a);
-        float vals[8];
-        float du = 0.f, qp = 0.f;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            lam[i] = fmaf(sc.z, cv[i], lam[i]);     // λ_t
-            const float hb = a[i] * hs[t][i];       // Abar_t·h_{t−1}
-            const float lh = lam[i] * hb;
-            du = fmaf(lam[i], bv[i], du);
-            qp = fmaf(lh, Av[i], qp);
-            dAacc[i] = fmaf(sc.x, lh, dAacc[i]);
-            vals[i] = lam[i] * sc.y;                // dB
-            vals[4 + i] = sc.z * hs[t + 1][i];      // dC
-            lam[i] *= a[i];                         // Abar_t·λ_t, carried to token t − 1
-        }
-        du += __shfl_xor_sync(0xffffffffu, du, 1);
-        du += __shfl_xor_sync(0xffffffffu, du, 2);
-        qp += __shfl_xor_sync(0xffffffffu, qp, 1);
-        qp += __shfl_xor_sync(0xffffffffu, qp, 2);
-        if (q == 0) S.duq[tt][jc] = make_float2(du, qp);
-        // reduce-scatter of the 8 values over the warp's 8 chains (lane bits
-        // 4, 3, 2): afterwards lane (jw, q) holds value jw summed over them
-        float w4[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const float keep = b4bit ? vals[4 + i] : vals[i];
-            const float send = b4bit ? vals[i] : vals[4 + i];
-            w4[i] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
-        }
-        float w2[2];
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {
-            const float keep = b3bit ? w4[2 + i] : w4[i];
-            const float send = b3bit ? w4[i] : w4[2 + i];
-            w2[i] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
-        }
-        const float keep = b2bit ? w2[1] : w2[0];
-        const float send = b2bit ? w2[0] : w2[1];
-        const float w1 = keep + __shfl_xor_sync(0xffffffffu, send, 4);
-        // value jw: 0..3 → dB[4q + jw], 4..7 → dC[4q + jw − 4]
-        const int v = jw < 4 ? 4 * q + jw : kMaxN + 4 * q + (jw - 4);
-        S.red[warp][tt][v] = w1;
-    }
-}
-
-template <typename T, bool kGate, bool kSoftplus>
-__global__ void __launch_bounds__(kThreads, 5) scan_bwd_kernel(const BwdParams p) {
-    __shared__ BwdSmem S;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int q = lane & 3;                 // quarter: states 4q..4q+3
-    const int jw = lane >> 2;               // chain within the warp
-    const int jc = warp * 8 + jw;           // chain within the CTA
-    const long long b = blockIdx.y;
-    const long long d0 = (long long)blockIdx.x * kChains;
-    const long long d = d0 + jc;
-    const bool active = d < p.dim;
-    const int oc = tid & 31, ot = tid >> 5;  // owner role: channel oc, tokens ot + 4m
-    const long long od = d0 + oc;
-    const int N = p.dstate;
-
-    // this lane's A values (0 for states past dstate) and the structure test
-    float Av[4];
-    bool ok = true;
-    const float A0 = active ? p.A[d * N] : 0.0f;
+__device__ __forceinline__ void load_bc(float (&bv)[4], float (&cv)[4], const BwdParams &p,
+                                        long long b, long long t0, int lane, bool withC) {
+    const int t = lane >> 2, n0 = 4 * (lane & 3);
+    const long long tok = t0 + t;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        const int n = 4 * q + i;
-        const bool has = active && n < N;
-        Av[i] = has ? p.A[d * N + n] : 0.0f;
-        if (has && Av[i] != (float)(n + 1) * A0) ok = false;
+        const bool ok = tok < p.seqlen && n0 + i < p.dstate;
+        const long long idx = (b * p.seqlen + tok) * p.dstate + n0 + i;
+        bv[i] = ok ? ldg_f32(static_cast<const T *>(p.B) + idx) : 0.0f;
+        cv[i] = (ok && withC) ? ldg_f32(static_cast<const T *>(p.C) + idx) : 0.0f;
     }
-    const bool structured = __all_sync(0xffffffffu, ok);
-    const float oA0 = od < p.dim ? p.A[od * N] : 0.0f;
-    const float obias = (od < p.dim && p.delta_bias) ? p.delta_bias[od] : 0.0f;
-    const float oD = (od < p.dim && p.Dskip) ? p.Dskip[od] : 0.0f;
+}
+
+__device__ __forceinline__ void store_bc(BwdSmem &S, const float (&bv)[4], const float (&cv)[4],
+                                         int lane) {
+    const int t = lane >> 2, n0 = 4 * (lane & 3);
+    *reinterpret_cast<float4 *>(&S.Bs[t][n0]) = make_float4(bv[0], bv[1], bv[2], bv[3]);
+    *reinterpret_cast<float4 *>(&S.Cs[t][n0]) = make_float4(cv[0], cv[1], cv[2], cv[3]);
+}
+
+// Abar for the 16 states at one token. Structured A: r^(n+1) by a power
+// ladder; otherwise 2^(Δ·A[n]·log2 e) per state (Al = A·log2 e).
+template <bool kStruct>
+__device__ __forceinline__ void decay16(float dt, float r, const float2 (&Al)[kPairs],
+                                        float2 (&a)[kPairs]) {
+    if (kStruct) {
+        const float r2 = r * r;
+        a[0] = make_float2(r, r2);
+        a[1] = mul2(a[0], dup2(r2));
+        const float2 q4 = dup2(a[1].y);
+        a[2] = mul2(a[0], q4);
+        a[3] = mul2(a[1], q4);
+        const float2 q8 = dup2(a[3].y);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) a[4 + j] = mul2(a[j], q8);
+    } else {
+#pragma unroll
+        for (int j = 0; j < kPairs; ++j)
+            a[j] = make_float2(ex2_approx(dt * Al[j].x), ex2_approx(dt * Al[j].y));
+    }
+}
+
+// States 4q .. 4q+3 of a shared-memory row as two f32x2 pairs.
+__device__ __forceinline__ void ld_quad(const float *base, int q, float2 &lo, float2 &hi) {
+    const float4 v = *reinterpret_cast<const float4 *>(base + 4 * q);
+    lo = make_float2(v.x, v.y);
+    hi = make_float2(v.z, v.w);
+}
+__device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
+
+template <typename T, bool kGate, bool kSoftplus, bool kStruct>
+__device__ __forceinline__ void bwd_body(BwdSmem &S, const BwdParams &p) {
+    const int lane = threadIdx.x;
+    const long long b = blockIdx.y;
+    const long long d = (long long)blockIdx.x * kChains + lane;
+    const bool active = d < p.dim;
+    const int N = p.dstate;
+    const long long dd = active ? d : 0;
+
+    // A as 2^(·) exponents (general A) and the structured-A decay base
+    float2 Al[kPairs];
+#pragma unroll
+    for (int j = 0; j < kPairs; ++j) {
+        const float a0 = (active && 2 * j < N) ? p.A[dd * N + 2 * j] : 0.0f;
+        const float a1 = (active && 2 * j + 1 < N) ? p.A[dd * N + 2 * j + 1] : 0.0f;
+        Al[j] = make_float2(a0 * kLog2e, a1 * kLog2e);
+    }
+    const float A0l = Al[0].x;
+    const float bias = (active && p.delta_bias) ? p.delta_bias[dd] : 0.0f;
+    const float Dv = (active && p.Dskip) ? p.Dskip[dd] : 0.0f;
     const int K = p.ktiles;
-    float4 *ck = reinterpret_cast<float4 *>(p.ckpt) + ((b * K) * p.dim + (active ? d : 0)) * 4 + q;
+    float4 *ck = reinterpret_cast<float4 *>(p.ckpt) + ((b * K) * p.dim + dd) * 4;
     const long long ck_stride = p.dim * 4;  // float4s between consecutive tiles
 
     // ---- 1. forward sweep: checkpoints ------------------------------------------
     {
-        float h[4] = {0.f, 0.f, 0.f, 0.f};
+        float2 h[kPairs];
+#pragma unroll
+        for (int j = 0; j < kPairs; ++j) h[j] = make_float2(0.f, 0.f);
+        Raw<T> cur, nxt;
+        float bv[4], cv[4];
+        load_raw<T, kGate, false>(cur, p, b, 0, dd, active);
+        load_bc<T>(bv, cv, p, b, 0, lane, false);
         for (int k = 0; k < K; ++k) {
             const long long t0 = (long long)k * kSeg;
-            if (active) ck[k * ck_stride] = make_float4(h[0], h[1], h[2], h[3]);
-            load_bc<T>(S, p, b, t0, false);
-            owner_scalars<T, kGate, kSoftplus, false>(S, p, b, t0, oc, ot, od, oA0, obias);
-            __syncthreads();
-            advance<0>(S, jc, q, structured, Av, h);
-            advance<kHalf>(S, jc, q, structured, Av, h);
-            __syncthreads();
+            if (active) {
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    ck[k * ck_stride + j] =
+                        make_float4(h[2 * j].x, h[2 * j].y, h[2 * j + 1].x, h[2 * j + 1].y);
+            }
+            __syncwarp();
+            store_bc(S, bv, cv, lane);
+            if (k + 1 < K) {
+                load_raw<T, kGate, false>(nxt, p, b, t0 + kSeg, dd, active);
+                load_bc<T>(bv, cv, p, b, t0 + kSeg, lane, false);
+            }
+            __syncwarp();
+#pragma unroll
+            for (int t = 0; t < kSeg; ++t) {
+                const float v = to_f32(cur.dl[t]) + bias;
+                const bool live = active && t0 + t < p.seqlen;
+                const float dt = live ? (kSoftplus ? softplus_f32(v) : v) : 0.0f;
+                const float2 u2 = dup2(dt * to_f32(cur.x[t]));
+                float2 a[kPairs];
+                decay16<kStruct>(dt, ex2_approx(dt * A0l), Al, a);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    float2 b0, b1;
+                    ld_quad(S.Bs[t], q, b0, b1);
+                    h[2 * q] = fma2(a[2 * q], h[2 * q], mul2(u2, b0));
+                    h[2 * q + 1] = fma2(a[2 * q + 1], h[2 * q + 1], mul2(u2, b1));
+                }
+            }
+            cur = nxt;
         }
     }
 
     // ---- 2. reverse sweep ---------------------------------------------------------
-    float lam[4], dAacc[4] = {0.f, 0.f, 0.f, 0.f};
+    float2 lam[kPairs], dA[kPairs];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const int n = 4 * q + i;
-        lam[i] = (active && n < N && p.dfinal) ? p.dfinal[(b * p.dim + d) * N + n] : 0.0f;
+    for (int j = 0; j < kPairs; ++j) {
+        const float l0 = (active && p.dfinal && 2 * j < N) ? p.dfinal[(b * p.dim + dd) * N + 2 * j] : 0.f;
+        const float l1 =
+            (active && p.dfinal && 2 * j + 1 < N) ? p.dfinal[(b * p.dim + dd) * N + 2 * j + 1] : 0.f;
+        lam[j] = make_float2(l0, l1);
+        dA[j] = make_float2(0.f, 0.f);
     }
     float accD = 0.f, accBias = 0.f;
+    const int kk = lane & 7, g = lane >> 3;  // reduction role: value group kk, channels 8g..8g+7
+    float *part = p.part + (b * p.ctiles + blockIdx.x) * p.seqlen * kVals;
+    Raw<T> cur, nxt;
+    float bv[4], cv[4];
+    float4 hc[4], hn[4];
+    {
+        const long long t0 = (long long)(K - 1) * kSeg;
+        load_raw<T, kGate, true>(cur, p, b, t0, dd, active);
+        load_bc<T>(bv, cv, p, b, t0, lane, true);
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            hc[j] = active ? ck[(K - 1) * ck_stride + j] : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
     for (int k = K - 1; k >= 0; --k) {
         const long long t0 = (long long)k * kSeg;
-        const float4 hc = active ? ck[k * ck_stride] : make_float4(0.f, 0.f, 0.f, 0.f);
-        load_bc<T>(S, p, b, t0, true);
-        owner_scalars<T, kGate, kSoftplus, true>(S, p, b, t0, oc, ot, od, oA0, obias);
-        __syncthreads();
-
-        // second half of the tile first, then the first half; each half
-        // recomputes its 8 states into registers from the checkpoint
-        float h[4] = {hc.x, hc.y, hc.z, hc.w};
-        advance<0>(S, jc, q, structured, Av, h);
-        half_tile<kHalf>(S, jc, q, lane, warp, structured, Av, h, lam, dAacc);
-        h[0] = hc.x;
-        h[1] = hc.y;
-        h[2] = hc.z;
-        h[3] = hc.w;
-        half_tile<0>(S, jc, q, lane, warp, structured, Av, h, lam, dAacc);
-        __syncthreads();
-
-        // owner epilogue: dx, ddelta, dz; dD and ddelta_bias partials
+        __syncwarp();
+        store_bc(S, bv, cv, lane);
+        if (k > 0) {
+            load_raw<T, kGate, true>(nxt, p, b, t0 - kSeg, dd, active);
+            load_bc<T>(bv, cv, p, b, t0 - kSeg, lane, true);
 #pragma unroll
-        for (int m = 0; m < kSeg / kWarps; ++m) {
-            const int t = ot + kWarps * m;
+            for (int j = 0; j < 4; ++j)
+                hn[j] = active ? ck[(k - 1) * ck_stride + j] : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        __syncwarp();
+
+        // recompute the tile's states and per-token scalars
+        float2 h[kPairs];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            h[2 * j] = make_float2(hc[j].x, hc[j].y);
+            h[2 * j + 1] = make_float2(hc[j].z, hc[j].w);
+            S.hs[0][j][lane] = hc[j];
+        }
+#pragma unroll
+        for (int t = 0; t < kSeg; ++t) {
+            const bool live = active && t0 + t < p.seqlen;
+            const float xv = to_f32(cur.x[t]);
+            const float v = to_f32(cur.dl[t]) + bias;
+            const float dt = live ? (kSoftplus ? softplus_f32(v) : v) : 0.0f;
+            const float u = dt * xv;
+            const float dyv = to_f32(cur.dy[t]);
+            float ds = dyv, dysz = 0.f;
+            if (kGate) {
+                const float zv = to_f32(cur.z[t]);
+                const float sgz = sigmoid_f32(zv);
+                ds = dyv * zv * sgz;
+                dysz = dyv * sgz * fmaf(zv, 1.0f - sgz, 1.0f);
+            }
+            const float sg = kSoftplus ? sigmoid_f32(v) : 1.0f;
+            const float r = ex2_approx(dt * A0l);
+            float2 a[kPairs];
+            decay16<kStruct>(dt, r, Al, a);
+            const float2 u2 = dup2(u);
+            float2 sacc = make_float2(0.f, 0.f);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                float2 b0, b1, c0, c1;
+                ld_quad(S.Bs[t], q, b0, b1);
+                ld_quad(S.Cs[t], q, c0, c1);
+                h[2 * q] = fma2(a[2 * q], h[2 * q], mul2(u2, b0));
+                h[2 * q + 1] = fma2(a[2 * q + 1], h[2 * q + 1], mul2(u2, b1));
+                sacc = fma2(c0, h[2 * q], sacc);
+                sacc = fma2(c1, h[2 * q + 1], sacc);
+            }
+            S.sc[t][lane] = make_float4(dt, u, ds, r);
+            S.so[t][lane] = make_float4(xv, dysz, sg, fmaf(Dv, xv, sacc.x + sacc.y));
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                S.hs[t + 1][j][lane] = make_float4(h[2 * j].x, h[2 * j].y, h[2 * j + 1].x, h[2 * j + 1].y);
+        }
+
+        // walk the tile backwards
+#pragma unroll 1
+        for (int t = kSeg - 1; t >= 0; --t) {
             const long long tok = t0 + t;
-            if (od < p.dim && tok < p.seqlen) {
-                const long long i = (b * p.seqlen + tok) * p.dim + od;
-                const float4 sc = S.sc[t][oc];
-                const float4 so = S.so[t][oc];
-                const float2 dq = S.duq[t][oc];
-                const float ddt = fmaf(dq.x, so.x, dq.y);
-                const float dv = ddt * so.z;
-                static_cast<T *>(p.dx)[i] = from_f32<T>(fmaf(dq.x, sc.x, sc.z * oD));
-                static_cast<T *>(p.ddelta)[i] = from_f32<T>(dv);
-                if (kGate) {
-                    const float s = fmaf(oD, so.x, S.s[t][oc]);
-                    static_cast<T *>(p.dz)[i] = from_f32<T>(s * so.y);
+            const float4 sc = S.sc[t][lane];
+            const float4 so = S.so[t][lane];
+            float2 a[kPairs];
+            decay16<kStruct>(sc.x, sc.w, Al, a);
+            const float2 ds2 = dup2(sc.z), u2 = dup2(sc.y), dt2 = dup2(sc.x);
+            float2 du2 = make_float2(0.f, 0.f), qp2 = make_float2(0.f, 0.f);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const float4 hq = S.hs[t + 1][j][lane];    // h_t
+                const float4 hp = S.hs[t][j][lane];        // h_{t−1}
+                const float2 hh[2] = {make_float2(hq.x, hq.y), make_float2(hq.z, hq.w)};
+                const float2 hprev[2] = {make_float2(hp.x, hp.y), make_float2(hp.z, hp.w)};
+                float dbv[4], dcv[4];
+                float2 bq[2], cq[2];
+                ld_quad(S.Bs[t], j, bq[0], bq[1]);
+                ld_quad(S.Cs[t], j, cq[0], cq[1]);
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const int jj = 2 * j + e;
+                    const float2 bb = bq[e];
+                    lam[jj] = fma2(ds2, cq[e], lam[jj]);                    // λ_t
+                    const float2 hb = mul2(a[jj], hprev[e]);                // Abar_t·h_{t−1}
+                    const float2 lh = mul2(lam[jj], hb);
+                    du2 = fma2(lam[jj], bb, du2);
+                    if (kStruct)
+                        qp2 = fma2(lh, make_float2((float)(2 * jj + 1), (float)(2 * jj + 2)), qp2);
+                    else
+                        qp2 = fma2(lh, Al[jj], qp2);
+                    dA[jj] = fma2(dt2, lh, dA[jj]);
+                    const float2 db = mul2(lam[jj], u2);
+                    const float2 dc = mul2(ds2, hh[e]);
+                    dbv[2 * e] = db.x;
+                    dbv[2 * e + 1] = db.y;
+                    dcv[2 * e] = dc.x;
+                    dcv[2 * e + 1] = dc.y;
+                    lam[jj] = mul2(lam[jj], a[jj]);                       // carried to token t − 1
                 }
+                S.red[j][lane ^ j] = make_float4(dbv[0], dbv[1], dbv[2], dbv[3]);
+                S.red[4 + j][lane ^ (4 + j)] = make_float4(dcv[0], dcv[1], dcv[2], dcv[3]);
+            }
+            const float du = du2.x + du2.y;
+            const float qsum = qp2.x + qp2.y;
+            // Σ_n λ·hb·A[n]: structured A[n] = (n+1)·A[0]; otherwise Al = A·log2 e
+            const float qp = kStruct ? qsum * A0l * kLn2 : qsum * kLn2;
+            if (active && tok < p.seqlen) {
+                const long long i = (b * p.seqlen + tok) * p.dim + d;
+                const float ddt = fmaf(du, so.x, qp);
+                const float dv = ddt * so.z;
+                static_cast<T *>(p.dx)[i] = from_f32<T>(fmaf(du, sc.x, sc.z * Dv));
+                static_cast<T *>(p.ddelta)[i] = from_f32<T>(dv);
+                if (kGate) static_cast<T *>(p.dz)[i] = from_f32<T>(so.w * so.y);
                 accD = fmaf(sc.z, so.x, accD);
                 accBias += dv;
             }
-        }
-        // this tile's channel sums of dB and dC
-        for (int e = tid; e < kSeg * kVals; e += kThreads) {
-            const int t = e / kVals, v = e % kVals;
-            const long long tok = t0 + t;
-            if (tok < p.seqlen) {
-                float sum = 0.f;
+            __syncwarp();
+            // channel sums of this token's 32 values
+            float2 alo = make_float2(0.f, 0.f), ahi = alo;
 #pragma unroll
-                for (int w = 0; w < kWarps; ++w) sum += S.red[w][t][v];
-                p.part[((b * p.ctiles + blockIdx.x) * p.seqlen + tok) * kVals + v] = sum;
+            for (int i = 0; i < 8; ++i) {
+                const float4 w = S.red[kk][(8 * g + i) ^ kk];
+                alo = add2(alo, make_float2(w.x, w.y));
+                ahi = add2(ahi, make_float2(w.z, w.w));
             }
+            float4 acc = make_float4(alo.x, alo.y, ahi.x, ahi.y);
+#pragma unroll
+            for (int m = 8; m <= 16; m <<= 1) {
+                acc.x += __shfl_xor_sync(0xffffffffu, acc.x, m);
+                acc.y += __shfl_xor_sync(0xffffffffu, acc.y, m);
+                acc.z += __shfl_xor_sync(0xffffffffu, acc.z, m);
+                acc.w += __shfl_xor_sync(0xffffffffu, acc.w, m);
+            }
+            const float mine = g == 0 ? acc.x : (g == 1 ? acc.y : (g == 2 ? acc.z : acc.w));
+            if (tok < p.seqlen) part[tok * kVals + 4 * kk + g] = mine;
+            __syncwarp();
         }
-        __syncthreads();
+        cur = nxt;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) hc[j] = hn[j];
     }
 
     // per-(batch row, channel) partials
     if (active) {
+        float4 *pa = reinterpret_cast<float4 *>(p.pA + (b * p.dim + d) * kMaxN);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) p.pA[(b * p.dim + d) * kMaxN + 4 * q + i] = dAacc[i];
+        for (int j = 0; j < 4; ++j)
+            pa[j] = make_float4(dA[2 * j].x, dA[2 * j].y, dA[2 * j + 1].x, dA[2 * j + 1].y);
+        p.pD[b * p.dim + d] = accD;
+        p.pbias[b * p.dim + d] = accBias;
     }
-    float *red = &S.red[0][0][0];
-    red[tid] = accD;
-    red[kThreads + tid] = accBias;
-    __syncthreads();
-    if (tid < kChains && od < p.dim) {
-        float sd = 0.f, sb = 0.f;
-#pragma unroll
-        for (int w = 0; w < kWarps; ++w) {
-            sd += red[w * 32 + tid];
-            sb += red[kThreads + w * 32 + tid];
-        }
-        p.pD[b * p.dim + od] = sd;
-        p.pbias[b * p.dim + od] = sb;
+}
+
+// A[d, n] == (n+1)·A[d, 0] for every state of every channel of the warp
+// selects the power-ladder decay (the A = −(1..N) initialisation).
+template <typename T, bool kGate, bool kSoftplus>
+__global__ void __launch_bounds__(kChains, 6) scan_bwd_kernel(const BwdParams p) {
+    __shared__ BwdSmem S;
+    const long long d = (long long)blockIdx.x * kChains + threadIdx.x;
+    bool ok = true;
+    if (d < p.dim) {
+        const float a0 = p.A[d * p.dstate];
+        for (int n = 1; n < p.dstate; ++n)
+            if (p.A[d * p.dstate + n] != (float)(n + 1) * a0) ok = false;
     }
+    if (__all_sync(0xffffffffu, ok))
+        bwd_body<T, kGate, kSoftplus, true>(S, p);
+    else
+        bwd_body<T, kGate, kSoftplus, false>(S, p);
 }
 
 // dB[b, t, n] and dC[b, t, n]: sums of the channel-tile partials.
@@ -425,9 +442,9 @@ template <typename T, bool kGate>
 cudaError_t launch_gate(const BwdParams &p, cudaStream_t stream) {
     const dim3 grid((unsigned)p.ctiles, (unsigned)p.batch);
     if (p.softplus)
-        scan_bwd_kernel<T, kGate, true><<<grid, kThreads, 0, stream>>>(p);
+        scan_bwd_kernel<T, kGate, true><<<grid, kChains, 0, stream>>>(p);
     else
-        scan_bwd_kernel<T, kGate, false><<<grid, kThreads, 0, stream>>>(p);
+        scan_bwd_kernel<T, kGate, false><<<grid, kChains, 0, stream>>>(p);
     return cudaGetLastError();
 }
 

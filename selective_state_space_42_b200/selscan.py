@@ -46,6 +46,8 @@ SIGNATURES = {
     "selscan_bwd": (_int, [_vp] * 8 + [_int] + [_vp] * 10
                     + [_i64, _i64, _i64, _i64, _int, _vp]),
     "selscan_bwd_workspace_bytes": (_i64, [_i64, _i64, _i64, _i64]),
+    "selscan_bwd_workspace": (_int, [_vp] * 8 + [_int] + [_vp] * 10
+                              + [_i64, _i64, _i64, _i64, _int, _vp, _i64, _vp]),
     "selscan_device_status": (_int, [ctypes.POINTER(_int), _int]),
     "selscan_status_string": (ctypes.c_char_p, [_int]),
     "selscan_last_cuda_error": (ctypes.c_char_p, []),
@@ -221,12 +223,16 @@ def _fwd(entry, x, delta, A, B, C, D, z, delta_bias, softplus, y, final_state,
 
 
 def selscan_bwd(x, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=True,
-                dy=None, dfinal_state=None, stream=None):
-    """Gradient of ``selscan_fwd`` (C ABI ``selscan_bwd``) for the loss
-    Σ dy·y + Σ dfinal_state·final_state. Inputs as for ``selscan_fwd``; dy has
-    y's shape and dtype, dfinal_state is [batch, dim, dstate] float32 or None.
-    Returns a dict: dx, ddelta, dz (x's dtype; dz None without z), dA, dB, dC,
-    dD, ddelta_bias (float32)."""
+                dy=None, dfinal_state=None, stream=None, allocate_in_library=False):
+    """Gradient of ``selscan_fwd`` for the loss Σ dy·y + Σ
+    dfinal_state·final_state. Inputs as for ``selscan_fwd``; dy has y's shape
+    and dtype, dfinal_state is [batch, dim, dstate] float32 or None. Returns a
+    dict: dx, ddelta, dz (x's dtype; dz None without z), dA, dB, dC, dD,
+    ddelta_bias (float32).
+
+    The workspace comes from torch's caching allocator (C ABI
+    ``selscan_bwd_workspace``); with ``allocate_in_library`` the library
+    allocates it on the stream instead (C ABI ``selscan_bwd``)."""
     torch = _torch()
     if x.dim() != 3:
         raise ValueError("x must be [batch, L, dim]")
@@ -260,9 +266,18 @@ def selscan_bwd(x, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=Tru
         _ptr(out["dx"], "dx"), _ptr(out["ddelta"], "ddelta"), _ptr(out["dA"], "dA"),
         _ptr(out["dB"], "dB"), _ptr(out["dC"], "dC"), _ptr(out["dD"], "dD"),
         _ptr(out["dz"], "dz", required=False), _ptr(out["ddelta_bias"], "ddelta_bias"),
-        batch, L, dim, N, code, _stream_ptr(stream, dev),
+        batch, L, dim, N, code,
     ]
-    _check(load_library().selscan_bwd(*args))
+    lib = load_library()
+    if allocate_in_library:
+        _check(lib.selscan_bwd(*args, _stream_ptr(stream, dev)))
+        return out
+    nbytes = int(lib.selscan_bwd_workspace_bytes(batch, L, dim, N))
+    ws = torch.empty(max(nbytes, 1), device=dev, dtype=torch.uint8)
+    if stream is not None and not isinstance(stream, int):
+        ws.record_stream(stream)  # keep it out of the cache until that stream is done
+    _check(lib.selscan_bwd_workspace(*args, ws.data_ptr() if nbytes else None, nbytes,
+                                     _stream_ptr(stream, dev)))
     return out
 
 

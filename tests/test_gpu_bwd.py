@@ -158,3 +158,35 @@ def test_bench_shape_sampled_and_identities():
     lhs_b = float((grads["dB"].to(f64) * inp["B"].to(f64)).sum())
     rhs_b = lhs_c + float((df.to(f64) * hf.to(f64)).sum())
     assert abs(lhs_b - rhs_b) <= 1e-3 * (abs(rhs_b) + abs(lhs_c)), (lhs_b, rhs_b)
+
+
+def test_library_allocated_workspace_matches():
+    """selscan_bwd (workspace allocated on the stream by the library) and
+    selscan_bwd_workspace (torch-allocated workspace) give identical results."""
+    inp, dy, df = _inputs(2, 77, 70, 16, "bf16", True, seed=15)
+    d = {k: (None if v is None else v.to(DEV)) for k, v in inp.items()}
+    args = (d["x"], d["delta"], d["A"], d["B"], d["C"], d["D"], d["z"], d["delta_bias"])
+    g1 = ss.selscan_bwd(*args, dy=dy.to(DEV), dfinal_state=df.to(DEV))
+    g2 = ss.selscan_bwd(*args, dy=dy.to(DEV), dfinal_state=df.to(DEV),
+                        allocate_in_library=True)
+    torch.cuda.synchronize()
+    for k in GRADS:
+        assert torch.equal(g1[k], g2[k]), k
+
+
+def test_workspace_too_small_is_rejected():
+    inp, dy, _ = _inputs(1, 20, 40, 16, "bf16", False, seed=16)
+    d = {k: (None if v is None else v.to(DEV)) for k, v in inp.items()}
+    lib = ss.load_library()
+    need = ss.selscan_bwd_workspace_bytes(1, 20, 40, 16)
+    ws = torch.empty(need, device=DEV, dtype=torch.uint8)
+    outs = [torch.empty_like(d["x"]), torch.empty_like(d["x"]),
+            torch.empty(40, 16, device=DEV), torch.empty(1, 20, 16, device=DEV),
+            torch.empty(1, 20, 16, device=DEV)]
+    st = lib.selscan_bwd_workspace(
+        d["x"].data_ptr(), d["delta"].data_ptr(), d["A"].data_ptr(), d["B"].data_ptr(),
+        d["C"].data_ptr(), None, None, None, 1, dy.to(DEV).data_ptr(), None,
+        outs[0].data_ptr(), outs[1].data_ptr(), outs[2].data_ptr(), outs[3].data_ptr(),
+        outs[4].data_ptr(), None, None, None, 1, 20, 40, 16, 1, ws.data_ptr(), need - 1,
+        None)
+    assert st == -8
