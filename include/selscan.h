@@ -108,6 +108,26 @@ SELSCAN_API int selscan_fwd(const void *x, const void *delta, const float *A,
                 int64_t dstate, selscan_dtype_t dtype, selscan_stream_t stream);
 
 /*
+ * selscan_fwd_from_state -- selscan_fwd starting from a given state instead
+ * of h = 0 before the first token: the state carried across blocks of a
+ * sequence ("Mamba и State Space Models: альтернатива Transformer",
+ * "Hardware-Aware Scan") handed in from outside, e.g. the final state of a
+ * previous call on the preceding tokens or a state advanced by
+ * selscan_state_update. Arguments as selscan_fwd, plus
+ *   initial_state [batch, dim, dstate]   float32   NULL -> zero (== selscan_fwd)
+ * initial_state may be the same buffer as final_state (the state is then
+ * advanced in place); any other overlap with an output is rejected. With
+ * seqlen == 0 the final state is a copy of the initial state.
+ */
+SELSCAN_API int selscan_fwd_from_state(const void *x, const void *delta, const float *A,
+                                       const void *B, const void *C, const float *D,
+                                       const void *z, const float *delta_bias,
+                                       int softplus_flag, const float *initial_state,
+                                       void *y, float *final_state, int64_t batch,
+                                       int64_t seqlen, int64_t dim, int64_t dstate,
+                                       selscan_dtype_t dtype, selscan_stream_t stream);
+
+/*
  * selscan_fwd_noalloc -- selscan_fwd without any device allocation.
  *
  * The pages have no counterpart of this call; it exists for callers that

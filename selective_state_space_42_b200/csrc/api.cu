@@ -177,7 +177,7 @@ void plan_for_sizes(int64_t batch, int64_t seqlen, int64_t dim, int64_t dstate, 
 // been cleared on stream).
 int fwd_setup(const void *x, const void *delta, const float *A, const void *B,
               const void *C, const float *D, const void *z, const float *delta_bias,
-              int softplus_flag, void *y, float *final_state, int64_t batch,
+              int softplus_flag, const float *h0, void *y, float *final_state, int64_t batch,
               int64_t seqlen, int64_t dim, int64_t dstate, int dtype,
               cudaStream_t stream, FwdPlan *plan, bool *done) {
     *done = false;
@@ -195,12 +195,16 @@ int fwd_setup(const void *x, const void *delta, const float *A, const void *B,
     if (misaligned(x, es) || misaligned(delta, es) || misaligned(z, es) ||
         misaligned(B, es) || misaligned(C, es) || misaligned(y, es) ||
         misaligned(A, 4) || misaligned(D, 4) || misaligned(delta_bias, 4) ||
-        misaligned(final_state, 4))
+        misaligned(final_state, 4) || misaligned(h0, 4))
         return SELSCAN_ERR_MISALIGNED;
     const size_t nx = (size_t)(batch * seqlen * dim) * es;
     const size_t nbc = (size_t)(batch * seqlen * dstate) * es;
+    const size_t ns = (size_t)(batch * dim * dstate) * sizeof(float);
     if (overlaps(y, nx, x, nx) || overlaps(y, nx, delta, nx) || overlaps(y, nx, z, nx) ||
-        overlaps(y, nx, B, nbc) || overlaps(y, nx, C, nbc))
+        overlaps(y, nx, B, nbc) || overlaps(y, nx, C, nbc) || overlaps(y, nx, h0, ns))
+        return SELSCAN_ERR_ALIAS;
+    // the final state may overwrite the initial state in place, but not partly
+    if (h0 && final_state && h0 != final_state && overlaps(h0, ns, final_state, ns))
         return SELSCAN_ERR_ALIAS;
 
     if (batch == 0 || dim == 0) {
@@ -209,10 +213,11 @@ int fwd_setup(const void *x, const void *delta, const float *A, const void *B,
     }
     if (seqlen == 0) {
         *done = true;
-        if (final_state) {
-            cudaError_t e = cudaMemsetAsync(final_state, 0,
-                                            (size_t)(batch * dim * dstate) * sizeof(float),
-                                            stream);
+        if (final_state && final_state != h0) {
+            // no token: the final state is the initial one
+            cudaError_t e = h0 ? cudaMemcpyAsync(final_state, h0, ns, cudaMemcpyDeviceToDevice,
+                                                 stream)
+                               : cudaMemsetAsync(final_state, 0, ns, stream);
             if (e != cudaSuccess) return cuda_fail(e);
         }
         return SELSCAN_OK;
@@ -228,14 +233,14 @@ int fwd_setup(const void *x, const void *delta, const float *A, const void *B,
     ScanParams &g = plan->gp;
     g.x = x; g.delta = delta; g.z = z; g.B = B; g.C = C;
     g.A = A; g.Dskip = D; g.delta_bias = delta_bias;
-    g.y = y; g.final_state = final_state;
+    g.y = y; g.final_state = final_state; g.h0 = h0;
     g.batch = batch; g.seqlen = seqlen; g.dim = dim; g.dstate = (int)dstate;
     g.softplus = softplus_flag ? 1 : 0;
     g.ws_P = g.ws_H = nullptr;
     if (plan->tma) {
         TmaScanParams &t = plan->tp;
         t.B = B; t.C = C; t.A = A; t.Dskip = D; t.delta_bias = delta_bias;
-        t.y = y; t.final_state = final_state;
+        t.y = y; t.final_state = final_state; t.h0 = h0;
         t.batch = batch; t.seqlen = seqlen; t.dim = dim; t.dstate = (int)dstate;
         t.softplus = g.softplus;
         const int64_t units = t.groups * t.nchunks;
@@ -366,15 +371,18 @@ const char *selscan_last_cuda_error(void) {
                                             : cudaGetErrorString(g_last_cuda_error);
 }
 
-int selscan_fwd(const void *x, const void *delta, const float *A, const void *B,
-                const void *C, const float *D, const void *z, const float *delta_bias,
-                int softplus_flag, void *y, float *final_state, int64_t batch,
-                int64_t seqlen, int64_t dim, int64_t dstate, selscan_dtype_t dtype,
-                selscan_stream_t stream_) {
+}  // extern "C"
+
+namespace {
+
+int fwd_entry(const void *x, const void *delta, const float *A, const void *B, const void *C,
+              const float *D, const void *z, const float *delta_bias, int softplus_flag,
+              const float *h0, void *y, float *final_state, int64_t batch, int64_t seqlen,
+              int64_t dim, int64_t dstate, selscan_dtype_t dtype, selscan_stream_t stream_) {
     cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
     selscan::FwdPlan plan;
     bool done = false;
-    const int st = selscan::fwd_setup(x, delta, A, B, C, D, z, delta_bias, softplus_flag,
+    const int st = selscan::fwd_setup(x, delta, A, B, C, D, z, delta_bias, softplus_flag, h0,
                                       y, final_state, batch, seqlen, dim, dstate, dtype,
                                       stream, &plan, &done);
     if (st != SELSCAN_OK || done) return st;
@@ -389,6 +397,29 @@ int selscan_fwd(const void *x, const void *delta, const float *A, const void *B,
         if (e == cudaSuccess) e = ef;
     }
     return e == cudaSuccess ? SELSCAN_OK : selscan::cuda_fail(e);
+}
+
+}  // namespace
+
+extern "C" {
+
+int selscan_fwd(const void *x, const void *delta, const float *A, const void *B,
+                const void *C, const float *D, const void *z, const float *delta_bias,
+                int softplus_flag, void *y, float *final_state, int64_t batch,
+                int64_t seqlen, int64_t dim, int64_t dstate, selscan_dtype_t dtype,
+                selscan_stream_t stream) {
+    return fwd_entry(x, delta, A, B, C, D, z, delta_bias, softplus_flag, nullptr, y,
+                     final_state, batch, seqlen, dim, dstate, dtype, stream);
+}
+
+int selscan_fwd_from_state(const void *x, const void *delta, const float *A, const void *B,
+                           const void *C, const float *D, const void *z,
+                           const float *delta_bias, int softplus_flag,
+                           const float *initial_state, void *y, float *final_state,
+                           int64_t batch, int64_t seqlen, int64_t dim, int64_t dstate,
+                           selscan_dtype_t dtype, selscan_stream_t stream) {
+    return fwd_entry(x, delta, A, B, C, D, z, delta_bias, softplus_flag, initial_state, y,
+                     final_state, batch, seqlen, dim, dstate, dtype, stream);
 }
 
 int selscan_fwd_plan(int64_t batch, int64_t seqlen, int64_t dim, int64_t dstate,

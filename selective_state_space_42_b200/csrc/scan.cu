@@ -163,6 +163,10 @@ scan_kernel(const ScanParams p) {
     if (kMode == kModeScan && p.nchunks > 1 && active) {
 #pragma unroll
         for (int n = 0; n < kMaxN; ++n) h[n] = p.ws_H[ws_row + n];  // carried-in state
+    } else if (kMode == kModeScan && p.h0 && active) {
+        const float *h0 = p.h0 + (b * p.dim + d) * p.dstate;
+#pragma unroll
+        for (int n = 0; n < kMaxN; ++n) h[n] = n < p.dstate ? h0[n] : 0.0f;
     } else {
 #pragma unroll
         for (int n = 0; n < kMaxN; ++n) h[n] = 0.0f;
@@ -220,7 +224,7 @@ __global__ void carry_kernel(const ScanParams p) {
     const int64_t bd = i / kMaxN;
     const int64_t d = bd % p.dim;
     const int64_t b = bd / p.dim;
-    float h = 0.0f;
+    float h = (p.h0 && n < p.dstate) ? p.h0[(b * p.dim + d) * p.dstate + n] : 0.0f;
     for (int c = 0; c < p.nchunks; ++c) {
         const size_t idx = (((size_t)b * p.nchunks + c) * p.dim + d) * kMaxN + n;
         if (c + 1 < p.nchunks) {

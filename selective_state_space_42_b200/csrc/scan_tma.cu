@@ -427,6 +427,10 @@ __device__ void consume(Shared<T> &S, const TmaScanParams &p, const CUtensorMap 
                         hs[4 * q] = v.x; hs[4 * q + 1] = v.y; hs[4 * q + 2] = v.z; hs[4 * q + 3] = v.w;
                     }
                 }
+            } else if (kMode == kModeSeq && p.h0 && active) {
+                const float *src = p.h0 + (inf.b * p.dim + d) * p.dstate;
+#pragma unroll
+                for (int n = 0; n < kMaxN; ++n) hs[n] = n < p.dstate ? src[n] : 0.0f;
             } else if (kMode == kModeRescan && p.nchunks > 1 && active) {
                 const float *src = p.ws_H + ((inf.b * p.nchunks + inf.chunk) * p.dim + d) * kMaxN;
 #pragma unroll

@@ -77,6 +77,7 @@ struct ScanParams {
     const float *A, *Dskip, *delta_bias;
     void *y;
     float *final_state;
+    const float *h0;     // state before the first token, [batch][dim][dstate] (NULL: zero)
     int64_t batch, seqlen, dim;
     int dstate;
     int softplus;
@@ -125,6 +126,7 @@ struct TmaScanParams {
     const float *A, *Dskip, *delta_bias;
     void *y;
     float *final_state;
+    const float *h0;      // state before the first token, [batch][dim][dstate] (NULL: zero)
     long long batch, seqlen, dim;
     int dstate;
     int softplus;
@@ -178,7 +180,7 @@ struct FwdPlan {
 
 int fwd_setup(const void *x, const void *delta, const float *A, const void *B,
               const void *C, const float *D, const void *z, const float *delta_bias,
-              int softplus_flag, void *y, float *final_state, int64_t batch,
+              int softplus_flag, const float *h0, void *y, float *final_state, int64_t batch,
               int64_t seqlen, int64_t dim, int64_t dstate, int dtype,
               cudaStream_t stream, FwdPlan *plan, bool *done);
 // Plans for the given sizes assuming 16-byte aligned tensors (selscan_fwd_plan).

@@ -39,6 +39,8 @@ SIGNATURES = {
                            _i64, _i64, _i64, _i64, _int, _vp]),
     "selscan_state_update": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                     _int, _vp, _i64, _i64, _i64, _int, _vp]),
+    "selscan_fwd_from_state": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _int, _vp,
+                                      _vp, _vp, _i64, _i64, _i64, _i64, _int, _vp]),
     "selscan_fwd_noalloc": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _int, _vp,
                                    _vp, _i64, _i64, _i64, _i64, _int, _vp]),
     "selscan_fwd_plan": (_int, [_i64, _i64, _i64, _i64, ctypes.POINTER(_i64),
@@ -165,12 +167,19 @@ def selscan_device_status(clear: bool = False) -> int:
 
 
 def selscan_fwd(x, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=True,
-                y=None, final_state=None, return_final_state=False, stream=None):
-    """Selective scan over whole sequences (C ABI ``selscan_fwd``).
+                y=None, final_state=None, return_final_state=False, stream=None,
+                initial_state=None):
+    """Selective scan over whole sequences (C ABI ``selscan_fwd``, or
+    ``selscan_fwd_from_state`` when ``initial_state`` is given).
 
     x, delta, z: [batch, L, dim]; B, C: [batch, L, dstate] (same dtype as x,
     float32 or bfloat16); A: [dim, dstate] float32; D, delta_bias: [dim]
-    float32. Returns y (allocated if not given) or (y, final_state)."""
+    float32; initial_state: [batch, dim, dstate] float32 (the state before the
+    first token; None: zero; may be the same tensor as final_state). Returns y
+    (allocated if not given) or (y, final_state)."""
+    if initial_state is not None:
+        return _fwd("selscan_fwd_from_state", x, delta, A, B, C, D, z, delta_bias, softplus,
+                    y, final_state, return_final_state, stream, initial_state=initial_state)
     return _fwd("selscan_fwd", x, delta, A, B, C, D, z, delta_bias, softplus, y,
                 final_state, return_final_state, stream)
 
@@ -187,7 +196,7 @@ def selscan_fwd_noalloc(x, delta, A, B, C, D=None, z=None, delta_bias=None,
 
 
 def _fwd(entry, x, delta, A, B, C, D, z, delta_bias, softplus, y, final_state,
-         return_final_state, stream):
+         return_final_state, stream, initial_state=None):
     torch = _torch()
     if x.dim() != 3:
         raise ValueError("x must be [batch, L, dim]")
@@ -212,6 +221,10 @@ def _fwd(entry, x, delta, A, B, C, D, z, delta_bias, softplus, y, final_state,
         _ptr(z, "z", (batch, L, dim), dt, dev, required=False),
         _ptr(delta_bias, "delta_bias", (dim,), f32, dev, required=False),
         int(bool(softplus)),
+    ]
+    if entry == "selscan_fwd_from_state":
+        args.append(_ptr(initial_state, "initial_state", (batch, dim, N), f32, dev))
+    args += [
         _ptr(y, "y", (batch, L, dim), dt, dev),
         _ptr(final_state, "final_state", (batch, dim, N), f32, dev, required=False),
         batch, L, dim, N, code, _stream_ptr(stream, dev),

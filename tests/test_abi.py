@@ -104,6 +104,23 @@ def test_fwd_validation(lib):
     assert fwd(lib, batch=1, y=P + 12288 - 2) == -7  # y runs into B
 
 
+def test_fwd_from_state_validation(lib):
+    def call(**kw):
+        a = dict(x=P, delta=P + 4096, A=P + 8192, B=P + 12288, C=P + 16384, D=None,
+                 z=None, delta_bias=None, softplus=1, h0=P + 32768, y=P + 65536,
+                 final_state=P + 32768, batch=0, seqlen=8, dim=4, dstate=16, dtype=1,
+                 stream=None)
+        a.update(kw)
+        return lib.selscan_fwd_from_state(
+            a["x"], a["delta"], a["A"], a["B"], a["C"], a["D"], a["z"], a["delta_bias"],
+            a["softplus"], a["h0"], a["y"], a["final_state"], a["batch"], a["seqlen"],
+            a["dim"], a["dstate"], a["dtype"], a["stream"])
+    assert call() == 0  # batch = 0; the state advanced in place is allowed
+    assert call(h0=P + 32770) == -4
+    assert call(batch=1, final_state=P + 32768 + 64) == -7  # partial overlap
+    assert call(batch=1, y=P + 32768) == -7  # y overlaps the initial state
+
+
 def test_state_update_validation(lib):
     assert step(lib) == 0
     assert step(lib, state=None) == 0  # batch = 0: empty
