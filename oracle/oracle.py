@@ -94,6 +94,9 @@ class Oracle:
         lib.oracle_selscan_bwd.argtypes = (
             [_dp] * 8 + [ctypes.c_int] + [_dp] * 3 + [_dp] * 9
             + [_i64, _i64, _i64, _i64, ctypes.c_int])
+        lib.oracle_causal_conv1d.restype = None
+        lib.oracle_causal_conv1d.argtypes = [_dp, _dp, _dp, _dp, _i64, _i64, _i64, _i64,
+                                             ctypes.c_int]
         lib.oracle_zoh_discretize.restype = None
         lib.oracle_zoh_discretize.argtypes = [ctypes.c_double, _dp, _dp, _dp,
                                               _dp, _i64]
@@ -176,6 +179,20 @@ class Oracle:
             _ptr(out["dC"]), _ptr(out["dD"]), _ptr(out["dz"]),
             _ptr(out["ddelta_bias"]), _ptr(out["dh0"]),
             batch, L, dim, N, int(threads or default_threads()))
+        return out
+
+    def causal_conv1d(self, x_in, w, cb=None, silu=True):
+        """Causal depthwise convolution (+ SiLU) in front of the scan:
+        x_in [batch, L, D], w [D, K], cb [D] or None -> [batch, L, D]."""
+        x_in = _f64(x_in)
+        batch, L, dim = x_in.shape
+        w = _f64(w)
+        if w.ndim != 2 or w.shape[0] != dim:
+            raise ValueError("w must be [D, K]")
+        cb = _f64(cb, (dim,))
+        out = np.empty_like(x_in)
+        self.lib.oracle_causal_conv1d(_ptr(x_in), _ptr(w), _ptr(cb), _ptr(out), batch, L,
+                                      dim, w.shape[1], int(bool(silu)))
         return out
 
     # -- single-token decode -------------------------------------------------

@@ -427,3 +427,32 @@ void oracle_selscan_bwd(const double *x, const double *delta, const double *A,
     }
     free(priv);
 }
+
+/*
+ * Causal depthwise convolution in front of the scan: the Conv1d with one
+ * filter per channel, kernel width K and K − 1 leading zeros of "Mamba и State
+ * Space Models: альтернатива Transformer" ("Mamba Block": groups = channels,
+ * padding d_conv − 1) and of "Mamba & State Space Models — Guide Complet" §7
+ * (kernel_size 4, keeping the first L outputs), followed by the SiLU of that
+ * page's block diagram (Conv1D → SiLU → SSM):
+ *   x[b, t, d] = silu( cb[d] + Σ_{k<K} w[d, k] · x_in[b, t − (K−1) + k, d] ),
+ * with x_in = 0 before the first token. Like torch's Conv1d this is a
+ * cross-correlation (w[d, K−1] multiplies the current token).
+ * x_in, x_out [batch, L, D]; w [D, K]; cb [D] (nullable: zero).
+ */
+void oracle_causal_conv1d(const double *x_in, const double *w, const double *cb,
+                          double *x_out, int64_t batch, int64_t L, int64_t D,
+                          int64_t K, int silu_flag)
+{
+    for (int64_t b = 0; b < batch; ++b)
+        for (int64_t t = 0; t < L; ++t)
+            for (int64_t d = 0; d < D; ++d) {
+                double acc = cb ? cb[d] : 0.0;
+                for (int64_t k = 0; k < K; ++k) {
+                    int64_t s = t - (K - 1) + k;
+                    if (s >= 0)
+                        acc += w[d * K + k] * x_in[(b * L + s) * D + d];
+                }
+                x_out[(b * L + t) * D + d] = silu_flag ? silu(acc) : acc;
+            }
+}

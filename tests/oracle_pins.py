@@ -494,10 +494,47 @@ def pin_bwd_single_token(orc):
     assert _rel(g["dD"], gy * xv) < 1e-14, "dD"
 
 
+# ---------------------------------------------------------------------------
+# Causal depthwise convolution in front of the scan.
+
+def pin_conv1d_library(orc):
+    """Each channel against numpy's full convolution with the reversed filter
+    (a cross-correlation with K − 1 leading zeros keeps the first L outputs),
+    plus the bias, then SiLU; widths 1 to 4."""
+    r = RNG(70)
+    for K in (1, 2, 3, 4):
+        x = r.standard_normal((2, 9, 3))
+        w = r.standard_normal((3, K))
+        cb = r.standard_normal(3)
+        got = orc.causal_conv1d(x, w, cb, silu=True)
+        ref = np.empty_like(x)
+        for b in range(2):
+            for d in range(3):
+                pre = np.convolve(x[b, :, d], w[d, ::-1])[:9] + cb[d]
+                ref[b, :, d] = pre * scipy.special.expit(pre)
+        assert _rel(got, ref) < 1e-13, f"conv width {K}"
+
+
+def pin_conv1d_impulse(orc):
+    """A unit impulse at token t0, no bias, no SiLU: the output from t0 on is
+    the filter read backwards (w[K−1] at t0, w[K−2] at t0 + 1, ...), zero
+    elsewhere, exactly; and the impulse's channel only."""
+    K, L, t0 = 4, 10, 3
+    w = np.array([[0.5, -1.0, 2.0, 3.0], [1.0, 1.0, 1.0, 1.0]])
+    x = np.zeros((1, L, 2))
+    x[0, t0, 0] = 1.0
+    got = orc.causal_conv1d(x, w, None, silu=False)
+    want = np.zeros((1, L, 2))
+    for j in range(K):
+        want[0, t0 + j, 0] = w[0, K - 1 - j]
+    assert np.array_equal(got, want), "impulse response"
+
+
 ALL_PINS = [
     pin_explicit_sum, pin_single_token, pin_lti_convolution, pin_zoh_matrix,
     pin_euler_vs_zoh, pin_linearity, pin_delta_to_zero, pin_chunked,
     pin_associativity, pin_geometric, pin_decay, pin_cross_entry,
     pin_decode_layout, pin_softplus_and_gate, pin_hand_worked,
     pin_bwd_finite_differences, pin_bwd_homogeneity, pin_bwd_single_token,
+    pin_conv1d_library, pin_conv1d_impulse,
 ]

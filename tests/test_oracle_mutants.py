@@ -59,6 +59,11 @@ MUTANTS = [
     ("bwd_du_x_term_dropped", "    ddt += du * x[i];\n", "\n"),
     ("bwd_dfinal_ignored", "lam[n] = dfinal ? dfinal[(b * D + d) * N + n] : 0.0;",
      "lam[n] = 0.0;"),
+    ("conv_tap_off_by_one", "int64_t s = t - (K - 1) + k;", "int64_t s = t - K + k;"),
+    ("conv_silu_skipped", "x_out[(b * L + t) * D + d] = silu_flag ? silu(acc) : acc;",
+     "x_out[(b * L + t) * D + d] = acc;"),
+    ("conv_bias_dropped", "double acc = cb ? cb[d] : 0.0;", "double acc = 0.0;"),
+    ("conv_filter_not_reversed", "acc += w[d * K + k] * x_in", "acc += w[d * K + (K - 1 - k)] * x_in"),
     ("bwd_gate_on_ds_dropped", "double ds = z ? dy[i] * silu(z[i]) : dy[i];",
      "double ds = dy[i];"),
 ]
