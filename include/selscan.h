@@ -128,6 +128,35 @@ SELSCAN_API int selscan_fwd_from_state(const void *x, const void *delta, const f
                                        selscan_dtype_t dtype, selscan_stream_t stream);
 
 /*
+ * selscan_fwd_conv -- the Mamba block's causal depthwise convolution and SiLU
+ * in front of the scan, fused into it ("Mamba и State Space Models:
+ * альтернатива Transformer", "Mamba Block": Conv1d with one filter per
+ * channel and d_conv − 1 leading zeros; "Mamba & State Space Models — Guide
+ * Complet" §7: kernel width 4, the first L outputs, Conv1D → SiLU → SSM).
+ * The scan's x is
+ *   x[b,t,d] = silu( conv_bias[d] + Σ_{k<K} conv_weight[d,k] · x_in[b, t−(K−1)+k, d] )
+ * (x_in = 0 before the first token of each sequence; a cross-correlation like
+ * torch's Conv1d), used both in Δ·B·x and in D·x; x itself is not written.
+ *   x_in          [batch, seqlen, dim]      dtype        required
+ *   conv_weight   [dim, conv_width]         float32      required
+ *   conv_bias     [dim]                     float32      NULL -> zero
+ *   conv_width    1 .. 4
+ *   conv_init     [batch, dim, 3]           float32      NULL -> zero: the x_in
+ *                 values of the 3 tokens before token 0, oldest first (with
+ *                 initial_state, continues a sequence exactly: pass the last 3
+ *                 x_in tokens of the preceding call)
+ * Other arguments as selscan_fwd_from_state (initial_state may be NULL).
+ */
+SELSCAN_API int selscan_fwd_conv(const void *x_in, const float *conv_weight,
+                                 const float *conv_bias, int conv_width,
+                                 const float *conv_init, const void *delta,
+                                 const float *A, const void *B, const void *C, const float *D,
+                                 const void *z, const float *delta_bias, int softplus_flag,
+                                 const float *initial_state, void *y, float *final_state,
+                                 int64_t batch, int64_t seqlen, int64_t dim, int64_t dstate,
+                                 selscan_dtype_t dtype, selscan_stream_t stream);
+
+/*
  * selscan_fwd_noalloc -- selscan_fwd without any device allocation.
  *
  * The pages have no counterpart of this call; it exists for callers that

@@ -177,7 +177,8 @@ void plan_for_sizes(int64_t batch, int64_t seqlen, int64_t dim, int64_t dstate, 
 // been cleared on stream).
 int fwd_setup(const void *x, const void *delta, const float *A, const void *B,
               const void *C, const float *D, const void *z, const float *delta_bias,
-              int softplus_flag, const float *h0, void *y, float *final_state, int64_t batch,
+              int softplus_flag, const float *h0, const float *conv_w, const float *conv_b,
+              const float *conv_init, int conv_width, void *y, float *final_state, int64_t batch,
               int64_t seqlen, int64_t dim, int64_t dstate, int dtype,
               cudaStream_t stream, FwdPlan *plan, bool *done) {
     *done = false;
@@ -187,6 +188,10 @@ int fwd_setup(const void *x, const void *delta, const float *A, const void *B,
     if (!mul_le(batch, seqlen, kMaxElems) || !mul_le(batch * seqlen, dim, kMaxElems) ||
         !mul_le(batch, dim, kMaxElems))
         return SELSCAN_ERR_BAD_DIM;
+    if (conv_width < 0 || conv_width > kMaxConv) return SELSCAN_ERR_BAD_DIM;
+    if (conv_width > 0 && dim > 0 && !conv_w) return SELSCAN_ERR_NULL_ARG;
+    if (misaligned(conv_w, 4) || misaligned(conv_b, 4) || misaligned(conv_init, 4))
+        return SELSCAN_ERR_MISALIGNED;
     // A tensor with zero elements may be passed as NULL.
     const bool has_tokens = batch * seqlen * dim > 0;
     if (has_tokens && (!x || !delta || !y || !B || !C)) return SELSCAN_ERR_NULL_ARG;
@@ -200,8 +205,10 @@ int fwd_setup(const void *x, const void *delta, const float *A, const void *B,
     const size_t nx = (size_t)(batch * seqlen * dim) * es;
     const size_t nbc = (size_t)(batch * seqlen * dstate) * es;
     const size_t ns = (size_t)(batch * dim * dstate) * sizeof(float);
+    const size_t nci = (size_t)(batch * dim) * (kMaxConv - 1) * sizeof(float);
     if (overlaps(y, nx, x, nx) || overlaps(y, nx, delta, nx) || overlaps(y, nx, z, nx) ||
-        overlaps(y, nx, B, nbc) || overlaps(y, nx, C, nbc) || overlaps(y, nx, h0, ns))
+        overlaps(y, nx, B, nbc) || overlaps(y, nx, C, nbc) || overlaps(y, nx, h0, ns) ||
+        (conv_width > 0 && overlaps(y, nx, conv_init, nci)))
         return SELSCAN_ERR_ALIAS;
     // the final state may overwrite the initial state in place, but not partly
     if (h0 && final_state && h0 != final_state && overlaps(h0, ns, final_state, ns))
@@ -234,6 +241,10 @@ int fwd_setup(const void *x, const void *delta, const float *A, const void *B,
     g.x = x; g.delta = delta; g.z = z; g.B = B; g.C = C;
     g.A = A; g.Dskip = D; g.delta_bias = delta_bias;
     g.y = y; g.final_state = final_state; g.h0 = h0;
+    g.conv_w = conv_width > 0 ? conv_w : nullptr;
+    g.conv_b = conv_width > 0 ? conv_b : nullptr;
+    g.conv_init = conv_width > 0 ? conv_init : nullptr;
+    g.conv_width = conv_width;
     g.batch = batch; g.seqlen = seqlen; g.dim = dim; g.dstate = (int)dstate;
     g.softplus = softplus_flag ? 1 : 0;
     g.ws_P = g.ws_H = nullptr;
@@ -241,6 +252,8 @@ int fwd_setup(const void *x, const void *delta, const float *A, const void *B,
         TmaScanParams &t = plan->tp;
         t.B = B; t.C = C; t.A = A; t.Dskip = D; t.delta_bias = delta_bias;
         t.y = y; t.final_state = final_state; t.h0 = h0;
+        t.conv_w = g.conv_w; t.conv_b = g.conv_b; t.conv_init = g.conv_init;
+        t.conv_width = conv_width;
         t.batch = batch; t.seqlen = seqlen; t.dim = dim; t.dstate = (int)dstate;
         t.softplus = g.softplus;
         const int64_t units = t.groups * t.nchunks;
@@ -377,14 +390,17 @@ namespace {
 
 int fwd_entry(const void *x, const void *delta, const float *A, const void *B, const void *C,
               const float *D, const void *z, const float *delta_bias, int softplus_flag,
-              const float *h0, void *y, float *final_state, int64_t batch, int64_t seqlen,
-              int64_t dim, int64_t dstate, selscan_dtype_t dtype, selscan_stream_t stream_) {
+              const float *h0, const float *conv_w, const float *conv_b,
+              const float *conv_init, int conv_width, void *y, float *final_state,
+              int64_t batch, int64_t seqlen, int64_t dim,
+              int64_t dstate, selscan_dtype_t dtype, selscan_stream_t stream_) {
     cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
     selscan::FwdPlan plan;
     bool done = false;
     const int st = selscan::fwd_setup(x, delta, A, B, C, D, z, delta_bias, softplus_flag, h0,
-                                      y, final_state, batch, seqlen, dim, dstate, dtype,
-                                      stream, &plan, &done);
+                                      conv_w, conv_b, conv_init, conv_width, y, final_state,
+                                      batch,
+                                      seqlen, dim, dstate, dtype, stream, &plan, &done);
     if (st != SELSCAN_OK || done) return st;
     void *ws = nullptr;
     if (plan.ws_bytes > 0) {
@@ -408,8 +424,9 @@ int selscan_fwd(const void *x, const void *delta, const float *A, const void *B,
                 int softplus_flag, void *y, float *final_state, int64_t batch,
                 int64_t seqlen, int64_t dim, int64_t dstate, selscan_dtype_t dtype,
                 selscan_stream_t stream) {
-    return fwd_entry(x, delta, A, B, C, D, z, delta_bias, softplus_flag, nullptr, y,
-                     final_state, batch, seqlen, dim, dstate, dtype, stream);
+    return fwd_entry(x, delta, A, B, C, D, z, delta_bias, softplus_flag, nullptr, nullptr,
+                     nullptr, nullptr, 0, y, final_state, batch, seqlen, dim, dstate, dtype,
+                     stream);
 }
 
 int selscan_fwd_from_state(const void *x, const void *delta, const float *A, const void *B,
@@ -418,8 +435,21 @@ int selscan_fwd_from_state(const void *x, const void *delta, const float *A, con
                            const float *initial_state, void *y, float *final_state,
                            int64_t batch, int64_t seqlen, int64_t dim, int64_t dstate,
                            selscan_dtype_t dtype, selscan_stream_t stream) {
-    return fwd_entry(x, delta, A, B, C, D, z, delta_bias, softplus_flag, initial_state, y,
-                     final_state, batch, seqlen, dim, dstate, dtype, stream);
+    return fwd_entry(x, delta, A, B, C, D, z, delta_bias, softplus_flag, initial_state,
+                     nullptr, nullptr, nullptr, 0, y, final_state, batch, seqlen, dim, dstate,
+                     dtype, stream);
+}
+
+int selscan_fwd_conv(const void *x_in, const float *conv_weight, const float *conv_bias,
+                     int conv_width, const float *conv_init, const void *delta, const float *A, const void *B,
+                     const void *C, const float *D, const void *z, const float *delta_bias,
+                     int softplus_flag, const float *initial_state, void *y,
+                     float *final_state, int64_t batch, int64_t seqlen, int64_t dim,
+                     int64_t dstate, selscan_dtype_t dtype, selscan_stream_t stream) {
+    if (conv_width < 1) return SELSCAN_ERR_BAD_DIM;
+    return fwd_entry(x_in, delta, A, B, C, D, z, delta_bias, softplus_flag, initial_state,
+                     conv_weight, conv_bias, conv_init, conv_width, y, final_state, batch,
+                     seqlen, dim, dstate, dtype, stream);
 }
 
 int selscan_fwd_plan(int64_t batch, int64_t seqlen, int64_t dim, int64_t dstate,

@@ -68,7 +68,9 @@ __device__ __forceinline__ void scan_tile(const ScanParams &p, int64_t b, int64_
                                           const float (*sC)[kMaxN],
                                           const float (&A2)[kMaxN], float dskip,
                                           float bias, float (&h)[kMaxN],
-                                          float &dt_sum) {
+                                          float &dt_sum, bool conv,
+                                          const float (&cw)[kMaxConv], float cb,
+                                          float (&xw)[kMaxConv - 1]) {
     const T *__restrict__ xp = static_cast<const T *>(p.x);
     const T *__restrict__ dp = static_cast<const T *>(p.delta);
     const T *__restrict__ zp = static_cast<const T *>(p.z);
@@ -89,6 +91,7 @@ __device__ __forceinline__ void scan_tile(const ScanParams &p, int64_t b, int64_
 #pragma unroll
         for (int k = 0; k < kU; ++k) {
             if (tt + k < nt) {
+                if (conv) xv[k] = conv_step(cw, cb, xw, xv[k]);
                 float dt = dv[k] + bias;
                 if (p.softplus) dt = softplus_f32(dt);
                 const float u = dt * xv[k];
@@ -173,6 +176,25 @@ scan_kernel(const ScanParams p) {
     }
     float dt_sum = 0.0f;
 
+    // causal conv: this channel's taps and the inputs of the kMaxConv − 1
+    // tokens before the chunk (zero before the sequence)
+    const bool conv = p.conv_width > 0;
+    float cw[kMaxConv] = {0.f, 0.f, 0.f, 0.f}, xw[kMaxConv - 1] = {0.f, 0.f, 0.f};
+    float cb = 0.0f;
+    if (conv && active) {
+        load_conv_taps(p.conv_w, p.conv_width, d, cw);
+        cb = p.conv_b ? p.conv_b[d] : 0.0f;
+        const T *xp = static_cast<const T *>(p.x);
+#pragma unroll
+        for (int k = 0; k < kMaxConv - 1; ++k) {
+            const int64_t t = t_begin - (kMaxConv - 1) + k;
+            if (t >= 0)
+                xw[k] = ldg_f32(xp + (b * p.seqlen + t) * p.dim + d);
+            else if (p.conv_init)
+                xw[k] = p.conv_init[(b * p.dim + d) * (kMaxConv - 1) + (t + kMaxConv - 1)];
+        }
+    }
+
     const T *Bp = static_cast<const T *>(p.B);
     const T *Cp = static_cast<const T *>(p.C);
     for (int64_t t0 = t_begin; t0 < t_end; t0 += kTileT) {
@@ -190,10 +212,10 @@ scan_kernel(const ScanParams p) {
         if (active) {
             if (structured)
                 scan_tile<T, kGate, kMode, true>(p, b, d, t0, nt, sB, sC, A2, dskip,
-                                                 bias, h, dt_sum);
+                                                 bias, h, dt_sum, conv, cw, cb, xw);
             else
                 scan_tile<T, kGate, kMode, false>(p, b, d, t0, nt, sB, sC, A2, dskip,
-                                                  bias, h, dt_sum);
+                                                  bias, h, dt_sum, conv, cw, cb, xw);
         }
     }
 

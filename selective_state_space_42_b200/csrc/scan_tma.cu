@@ -58,9 +58,13 @@ template <typename T> struct TileCfg;
 template <> struct TileCfg<__nv_bfloat16> { static constexpr int kTile = 32; };
 template <> struct TileCfg<float> { static constexpr int kTile = 16; };
 
+// Rows of x before a tile that the causal conv reads (the tile's tokens
+// start at row kHalo of the x buffer).
+constexpr int kHalo = kMaxConv - 1;
+
 template <typename T> struct alignas(128) Stage {
     static constexpr int kTile = TileCfg<T>::kTile;
-    T x[kTile][kChannels];
+    T x[kHalo + kTile][kChannels];  // with the conv: the kHalo tokens before the tile, then the tile
     T dl[kTile][kChannels];
     T z[kTile][kChannels];
     T Bs[kTile * kMaxN];  // TMA destination: the tile's B rows, dstate per row
@@ -143,7 +147,7 @@ __device__ __forceinline__ void convert_bc(Stage<T> &st, int nt, int dstate, int
 // converts its B/C kLag stages later, so it never waits on global memory
 // latency itself; the stage is handed to the consumers (32 arrivals on
 // `full`) after its conversion.
-template <typename T, bool kGate>
+template <typename T, bool kGate, bool kConv>
 __device__ void produce(Shared<T> &S, const TmaScanParams &p, const CUtensorMap *tm_x,
                         const CUtensorMap *tm_d, const CUtensorMap *tm_z,
                         const CUtensorMap *tm_b, const CUtensorMap *tm_c) {
@@ -158,7 +162,8 @@ __device__ void produce(Shared<T> &S, const TmaScanParams &p, const CUtensorMap 
         prefetch_tmap(tm_c);
     }
     constexpr uint32_t kTileBytes = kTile * kChannels * sizeof(T);
-    const uint32_t tx_bytes = (kGate ? 3u : 2u) * kTileBytes;
+    constexpr uint32_t kXBytes = (kConv ? kHalo + kTile : kTile) * kChannels * sizeof(T);
+    const uint32_t tx_bytes = (kGate ? 2u : 1u) * kTileBytes + kXBytes;
     const uint32_t bc_bytes = 2u * kTile * p.dstate * sizeof(T);
     int s = 0;                 // next stage to fill
     uint32_t phase = 0;
@@ -228,7 +233,14 @@ __device__ void produce(Shared<T> &S, const TmaScanParams &p, const CUtensorMap 
                 inf.flags = (j == 0 ? kFirst : 0) | (j == ntl - 1 ? kLast : 0);
                 const int c1 = (int)(b * p.seqlen + t0);
                 mbar_expect_tx(&S.full[s], tx_bytes);
-                tma_load_2d(&S.stage[s].x[0][0], tm_x, &S.full[s], tile * kChannels, c1);
+                // with the conv the box starts kHalo rows early (a negative row
+                // at the very start reads zeros; rows of the previous sequence
+                // are ignored by the consumers)
+                if (kConv)
+                    tma_load_2d(&S.stage[s].x[0][0], tm_x, &S.full[s], tile * kChannels,
+                                c1 - kHalo);
+                else
+                    tma_load_2d(&S.stage[s].x[kHalo][0], tm_x, &S.full[s], tile * kChannels, c1);
                 tma_load_2d(&S.stage[s].dl[0][0], tm_d, &S.full[s], tile * kChannels, c1);
                 if (kGate) tma_load_2d(&S.stage[s].z[0][0], tm_z, &S.full[s], tile * kChannels, c1);
                 mbar_arrive_expect_tx(&S.bc[s], bc_bytes);
@@ -259,11 +271,14 @@ __device__ __forceinline__ float softplus_fast(float v) {
 // valid tokens and y goes to this warp's shared-memory tile `ys` (written to
 // global memory by one TMA store per warp); otherwise tokens past nt leave
 // the state unchanged and y goes straight to global memory.
-template <typename T, bool kGate, int kMode, bool kStruct, bool kSoftplus, bool kFull>
+template <typename T, bool kGate, int kMode, bool kStruct, bool kSoftplus, bool kFull,
+          bool kConv>
 __device__ __forceinline__ void consume_tile(const Stage<T> &st, int nt, float2 (&h)[kMaxN / 2],
                                              const float (&A2)[kMaxN], float dskip, float bias,
                                              float &dt_sum, T *ys, T *yp, long long ybase,
-                                             long long ystride, bool active) {
+                                             long long ystride, bool active,
+                                             const float (&cw)[kMaxConv], float cb,
+                                             float (&xw)[kMaxConv - 1]) {
     constexpr int kTile = TileCfg<T>::kTile;
     constexpr bool kFastSp = sizeof(T) == 2;
     const int c = threadIdx.x;  // channel within the tile
@@ -276,7 +291,8 @@ __device__ __forceinline__ void consume_tile(const Stage<T> &st, int nt, float2 
 #pragma unroll
         for (int k = 0; k < kSub; ++k) {
             const int t = sub + k;
-            const float xv = to_f32(st.x[t][c]);
+            float xv = to_f32(st.x[kHalo + t][c]);
+            if (kConv) xv = conv_step(cw, cb, xw, xv);
             float dt = to_f32(st.dl[t][c]) + bias;
             if (kSoftplus) dt = kFastSp ? softplus_fast(dt) : softplus_f32(dt);
             if (!kFull) dt = t < nt ? dt : 0.0f;  // Abar = 1, no input: state unchanged
@@ -346,7 +362,7 @@ __device__ __forceinline__ void consume_tile(const Stage<T> &st, int nt, float2 
     }
 }
 
-template <typename T, bool kGate, int kMode, bool kSoftplus>
+template <typename T, bool kGate, int kMode, bool kSoftplus, bool kConv>
 __device__ void consume(Shared<T> &S, const TmaScanParams &p, const CUtensorMap *tm_y) {
     constexpr int kTile = TileCfg<T>::kTile;
     const int c = threadIdx.x;  // 0..127
@@ -364,6 +380,7 @@ __device__ void consume(Shared<T> &S, const TmaScanParams &p, const CUtensorMap 
     int cur_tile = -1;
     float A2[kMaxN];
     float dskip = 0.0f, bias = 0.0f;
+    float cw[kMaxConv] = {0.f, 0.f, 0.f, 0.f}, cb = 0.0f;  // conv taps of this channel
     bool structured = false;
     float2 h[kMaxN / 2];
 #pragma unroll
@@ -393,6 +410,10 @@ __device__ void consume(Shared<T> &S, const TmaScanParams &p, const CUtensorMap 
                     }
                     dskip = p.Dskip ? p.Dskip[d] : 0.0f;
                     bias = p.delta_bias ? p.delta_bias[d] : 0.0f;
+                    if (kConv) {
+                        load_conv_taps(p.conv_w, p.conv_width, d, cw);
+                        cb = p.conv_b ? p.conv_b[d] : 0.0f;
+                    }
                 } else {
 #pragma unroll
                     for (int n = 0; n < kMaxN; ++n) A2[n] = 0.0f;
@@ -441,6 +462,16 @@ __device__ void consume(Shared<T> &S, const TmaScanParams &p, const CUtensorMap 
         }
 
         const long long ybase = (inf.b * p.seqlen + inf.t0) * p.dim + d;
+        // conv window: the inputs of the kHalo tokens before the tile (zero
+        // before the sequence's first token)
+        float xw[kMaxConv - 1] = {0.f, 0.f, 0.f};
+        if (kConv && inf.t0 > 0) {
+#pragma unroll
+            for (int k = 0; k < kHalo; ++k) xw[k] = to_f32(S.stage[s].x[k][c]);
+        } else if (kConv && p.conv_init && active) {
+#pragma unroll
+            for (int k = 0; k < kHalo; ++k) xw[k] = p.conv_init[(inf.b * p.dim + d) * kHalo + k];
+        }
         if (inf.nt == kTile) {
             T *ys = S.ybuf[warp][kbuf];
             if (kMode != kModeAgg) {
@@ -449,11 +480,13 @@ __device__ void consume(Shared<T> &S, const TmaScanParams &p, const CUtensorMap 
                 __syncwarp();
             }
             if (structured)
-                consume_tile<T, kGate, kMode, true, kSoftplus, true>(
-                    S.stage[s], inf.nt, h, A2, dskip, bias, dt_sum, ys, yp, ybase, p.dim, active);
+                consume_tile<T, kGate, kMode, true, kSoftplus, true, kConv>(
+                    S.stage[s], inf.nt, h, A2, dskip, bias, dt_sum, ys, yp, ybase, p.dim, active,
+                    cw, cb, xw);
             else
-                consume_tile<T, kGate, kMode, false, kSoftplus, true>(
-                    S.stage[s], inf.nt, h, A2, dskip, bias, dt_sum, ys, yp, ybase, p.dim, active);
+                consume_tile<T, kGate, kMode, false, kSoftplus, true, kConv>(
+                    S.stage[s], inf.nt, h, A2, dskip, bias, dt_sum, ys, yp, ybase, p.dim, active,
+                    cw, cb, xw);
             if (kMode != kModeAgg) {
                 fence_proxy_async_smem();
                 __syncwarp();
@@ -466,13 +499,13 @@ __device__ void consume(Shared<T> &S, const TmaScanParams &p, const CUtensorMap 
             }
         } else {
             if (structured)
-                consume_tile<T, kGate, kMode, true, kSoftplus, false>(
+                consume_tile<T, kGate, kMode, true, kSoftplus, false, kConv>(
                     S.stage[s], inf.nt, h, A2, dskip, bias, dt_sum, nullptr, yp, ybase, p.dim,
-                    active);
+                    active, cw, cb, xw);
             else
-                consume_tile<T, kGate, kMode, false, kSoftplus, false>(
+                consume_tile<T, kGate, kMode, false, kSoftplus, false, kConv>(
                     S.stage[s], inf.nt, h, A2, dskip, bias, dt_sum, nullptr, yp, ybase, p.dim,
-                    active);
+                    active, cw, cb, xw);
         }
 
         if (inf.flags & kLast) {
@@ -520,7 +553,7 @@ __device__ void consume(Shared<T> &S, const TmaScanParams &p, const CUtensorMap 
     }
 }
 
-template <typename T, bool kGate, int kMode, bool kSoftplus>
+template <typename T, bool kGate, int kMode, bool kSoftplus, bool kConv>
 __global__ void __launch_bounds__(kBlock, 1)
 scan_tma_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_d,
                 const __grid_constant__ CUtensorMap tm_z, const __grid_constant__ CUtensorMap tm_b,
@@ -542,9 +575,9 @@ scan_tma_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
     }
     __syncthreads();
     if (threadIdx.x >= kChannels)
-        produce<T, kGate>(S, p, &tm_x, &tm_d, &tm_z, &tm_b, &tm_c);
+        produce<T, kGate, kConv>(S, p, &tm_x, &tm_d, &tm_z, &tm_b, &tm_c);
     else
-        consume<T, kGate, kMode, kSoftplus>(S, p, &tm_y);
+        consume<T, kGate, kMode, kSoftplus, kConv>(S, p, &tm_y);
 }
 
 // ---- host side -----------------------------------------------------------------------
@@ -565,14 +598,14 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 // box_cols × TileCfg<T>::kTile rows.
 template <typename T>
 bool make_map(CUtensorMap *m, const void *base, long long rows, long long cols,
-              int box_cols = kChannels) {
+              int box_cols = kChannels, int box_rows = TileCfg<T>::kTile) {
     auto fn = encode_fn();
     if (!fn) return false;
     const CUtensorMapDataType dt = sizeof(T) == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
                                                   : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
     cuuint64_t gdim[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
     cuuint64_t gstride[1] = {(cuuint64_t)(cols * sizeof(T))};
-    cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)TileCfg<T>::kTile};
+    cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
     cuuint32_t estride[2] = {1, 1};
     CUresult r = fn(m, dt, 2, const_cast<void *>(base), gdim, gstride, box, estride,
                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
@@ -591,13 +624,15 @@ int num_sms() {
     return sms;
 }
 
-template <typename T, bool kGate, int kMode, bool kSoftplus>
+template <typename T, bool kGate, int kMode, bool kSoftplus, bool kConv>
 cudaError_t launch_mode(const TmaScanParams &p, const void *x, const void *dl, const void *z,
                         cudaStream_t stream) {
     if (p.units <= 0) return cudaSuccess;
     CUtensorMap mx, md, mz, mb, mc, my;
     const long long rows = p.batch * p.seqlen;
-    if (!make_map<T>(&mx, x, rows, p.dim) || !make_map<T>(&md, dl, rows, p.dim) ||
+    const int x_rows = kConv ? kHalo + TileCfg<T>::kTile : TileCfg<T>::kTile;
+    if (!make_map<T>(&mx, x, rows, p.dim, kChannels, x_rows) ||
+        !make_map<T>(&md, dl, rows, p.dim) ||
         !make_map<T>(&mb, p.B, rows, p.dstate, p.dstate) ||
         !make_map<T>(&mc, p.C, rows, p.dstate, p.dstate) ||
         !make_map<T>(&my, p.y, rows, p.dim, 32))
@@ -608,7 +643,7 @@ cudaError_t launch_mode(const TmaScanParams &p, const void *x, const void *dl, c
         mz = md;
     }
     const size_t smem = sizeof(Shared<T>);
-    auto kern = scan_tma_kernel<T, kGate, kMode, kSoftplus>;
+    auto kern = scan_tma_kernel<T, kGate, kMode, kSoftplus, kConv>;
     // the shared-memory opt-in is set once per device for this instantiation
     static std::atomic<unsigned long long> configured{0};
     int dev = 0;
@@ -625,14 +660,21 @@ cudaError_t launch_mode(const TmaScanParams &p, const void *x, const void *dl, c
     return cudaGetLastError();
 }
 
+template <typename T, bool kGate, bool kSoftplus, bool kConv>
+cudaError_t launch_conv(const TmaScanParams &p, const void *x, const void *dl, const void *z,
+                        cudaStream_t stream) {
+    switch (p.mode) {
+    case kModeSeq: return launch_mode<T, kGate, kModeSeq, kSoftplus, kConv>(p, x, dl, z, stream);
+    case kModeAgg: return launch_mode<T, false, kModeAgg, kSoftplus, kConv>(p, x, dl, z, stream);
+    default: return launch_mode<T, kGate, kModeRescan, kSoftplus, kConv>(p, x, dl, z, stream);
+    }
+}
+
 template <typename T, bool kGate, bool kSoftplus>
 cudaError_t launch_sp(const TmaScanParams &p, const void *x, const void *dl, const void *z,
                       cudaStream_t stream) {
-    switch (p.mode) {
-    case kModeSeq: return launch_mode<T, kGate, kModeSeq, kSoftplus>(p, x, dl, z, stream);
-    case kModeAgg: return launch_mode<T, false, kModeAgg, kSoftplus>(p, x, dl, z, stream);
-    default: return launch_mode<T, kGate, kModeRescan, kSoftplus>(p, x, dl, z, stream);
-    }
+    return p.conv_width > 0 ? launch_conv<T, kGate, kSoftplus, true>(p, x, dl, z, stream)
+                            : launch_conv<T, kGate, kSoftplus, false>(p, x, dl, z, stream);
 }
 
 template <typename T, bool kGate>

@@ -10,6 +10,7 @@
 namespace selscan {
 
 constexpr int kMaxN = 16;           // largest supported d_state
+constexpr int kMaxConv = 4;         // widest causal conv in front of the scan
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
@@ -66,9 +67,32 @@ __device__ __forceinline__ float silu_f32(float z) {
     return z * rcp_approx(1.0f + ex2_approx(-z * kLog2e));
 }
 
+// Causal conv taps of one channel, right-aligned in four slots: slot 3
+// multiplies the current token, slot 3 − j the token j steps back; slots
+// before the filter's start are zero.
+__device__ __forceinline__ void load_conv_taps(const float *w, int width, long long d,
+                                               float (&cw)[kMaxConv]) {
+#pragma unroll
+    for (int k = 0; k < kMaxConv; ++k) {
+        const int j = k - (kMaxConv - width);  // filter index of slot k
+        cw[k] = j >= 0 ? w[d * width + j] : 0.0f;
+    }
+}
+
 // sigmoid(v) = 1 / (1 + e^-v); e^-v overflowing to +inf gives 0.
 __device__ __forceinline__ float sigmoid_f32(float v) {
     return rcp_approx(1.0f + ex2_approx(-v * kLog2e));
+}
+
+// One step of the causal conv + SiLU: xw holds the three previous inputs
+// (oldest first) and is shifted to include xi.
+__device__ __forceinline__ float conv_step(const float (&cw)[kMaxConv], float cb,
+                                           float (&xw)[kMaxConv - 1], float xi) {
+    const float pre = fmaf(cw[0], xw[0], fmaf(cw[1], xw[1], fmaf(cw[2], xw[2], fmaf(cw[3], xi, cb))));
+    xw[0] = xw[1];
+    xw[1] = xw[2];
+    xw[2] = xi;
+    return silu_f32(pre);
 }
 
 // ---- launch parameters -------------------------------------------------------------
@@ -78,6 +102,10 @@ struct ScanParams {
     void *y;
     float *final_state;
     const float *h0;     // state before the first token, [batch][dim][dstate] (NULL: zero)
+    const float *conv_w; // causal conv in front of the scan: [dim][conv_width] (NULL: none)
+    const float *conv_b; // [dim] (NULL: zero)
+    const float *conv_init;  // [batch][dim][kMaxConv − 1]: conv inputs before token 0 (NULL: zero)
+    int conv_width;      // 0 (no conv) or 1..kMaxConv
     int64_t batch, seqlen, dim;
     int dstate;
     int softplus;
@@ -127,6 +155,10 @@ struct TmaScanParams {
     void *y;
     float *final_state;
     const float *h0;      // state before the first token, [batch][dim][dstate] (NULL: zero)
+    const float *conv_w;  // causal conv in front of the scan: [dim][conv_width] (NULL: none)
+    const float *conv_b;  // [dim] (NULL: zero)
+    const float *conv_init;  // [batch][dim][kMaxConv − 1]: conv inputs before token 0 (NULL: zero)
+    int conv_width;       // 0 (no conv) or 1..kMaxConv
     long long batch, seqlen, dim;
     int dstate;
     int softplus;
@@ -180,7 +212,8 @@ struct FwdPlan {
 
 int fwd_setup(const void *x, const void *delta, const float *A, const void *B,
               const void *C, const float *D, const void *z, const float *delta_bias,
-              int softplus_flag, const float *h0, void *y, float *final_state, int64_t batch,
+              int softplus_flag, const float *h0, const float *conv_w, const float *conv_b,
+              const float *conv_init, int conv_width, void *y, float *final_state, int64_t batch,
               int64_t seqlen, int64_t dim, int64_t dstate, int dtype,
               cudaStream_t stream, FwdPlan *plan, bool *done);
 // Plans for the given sizes assuming 16-byte aligned tensors (selscan_fwd_plan).

@@ -41,6 +41,8 @@ SIGNATURES = {
                                     _int, _vp, _i64, _i64, _i64, _int, _vp]),
     "selscan_fwd_from_state": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _int, _vp,
                                       _vp, _vp, _i64, _i64, _i64, _i64, _int, _vp]),
+    "selscan_fwd_conv": (_int, [_vp, _vp, _vp, _int, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                _int, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _int, _vp]),
     "selscan_fwd_noalloc": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _int, _vp,
                                    _vp, _i64, _i64, _i64, _i64, _int, _vp]),
     "selscan_fwd_plan": (_int, [_i64, _i64, _i64, _i64, ctypes.POINTER(_i64),
@@ -168,15 +170,22 @@ def selscan_device_status(clear: bool = False) -> int:
 
 def selscan_fwd(x, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=True,
                 y=None, final_state=None, return_final_state=False, stream=None,
-                initial_state=None):
-    """Selective scan over whole sequences (C ABI ``selscan_fwd``, or
-    ``selscan_fwd_from_state`` when ``initial_state`` is given).
+                initial_state=None, conv_weight=None, conv_bias=None, conv_init=None):
+    """Selective scan over whole sequences (C ABI ``selscan_fwd``;
+    ``selscan_fwd_from_state`` when ``initial_state`` is given;
+    ``selscan_fwd_conv`` when ``conv_weight`` is given).
 
     x, delta, z: [batch, L, dim]; B, C: [batch, L, dstate] (same dtype as x,
     float32 or bfloat16); A: [dim, dstate] float32; D, delta_bias: [dim]
     float32; initial_state: [batch, dim, dstate] float32 (the state before the
-    first token; None: zero; may be the same tensor as final_state). Returns y
-    (allocated if not given) or (y, final_state)."""
+    first token; None: zero; may be the same tensor as final_state).
+    conv_weight [dim, K] (K ≤ 4), conv_bias [dim], conv_init [batch, dim, 3]
+    float32: x is then the input of the causal depthwise conv + SiLU in front
+    of the scan. Returns y (allocated if not given) or (y, final_state)."""
+    if conv_weight is not None:
+        return _fwd("selscan_fwd_conv", x, delta, A, B, C, D, z, delta_bias, softplus, y,
+                    final_state, return_final_state, stream, initial_state=initial_state,
+                    conv=(conv_weight, conv_bias, conv_init))
     if initial_state is not None:
         return _fwd("selscan_fwd_from_state", x, delta, A, B, C, D, z, delta_bias, softplus,
                     y, final_state, return_final_state, stream, initial_state=initial_state)
@@ -196,7 +205,7 @@ def selscan_fwd_noalloc(x, delta, A, B, C, D=None, z=None, delta_bias=None,
 
 
 def _fwd(entry, x, delta, A, B, C, D, z, delta_bias, softplus, y, final_state,
-         return_final_state, stream, initial_state=None):
+         return_final_state, stream, initial_state=None, conv=None):
     torch = _torch()
     if x.dim() != 3:
         raise ValueError("x must be [batch, L, dim]")
@@ -211,8 +220,16 @@ def _fwd(entry, x, delta, A, B, C, D, z, delta_bias, softplus, y, final_state,
     if final_state is None and return_final_state:
         final_state = torch.empty(batch, dim, N, device=dev, dtype=torch.float32)
     f32 = torch.float32
-    args = [
-        _ptr(x, "x", (batch, L, dim), dt, dev),
+    args = [_ptr(x, "x", (batch, L, dim), dt, dev)]
+    if entry == "selscan_fwd_conv":
+        cw, cbias, cinit = conv
+        if cw.dim() != 2 or cw.shape[0] != dim:
+            raise ValueError("conv_weight must be [dim, K]")
+        args += [_ptr(cw, "conv_weight", (dim, cw.shape[1]), f32, dev),
+                 _ptr(cbias, "conv_bias", (dim,), f32, dev, required=False),
+                 int(cw.shape[1]),
+                 _ptr(cinit, "conv_init", (batch, dim, 3), f32, dev, required=False)]
+    args += [
         _ptr(delta, "delta", (batch, L, dim), dt, dev),
         _ptr(A, "A", (dim, N), f32, dev),
         _ptr(B, "B", (batch, L, N), dt, dev),
@@ -224,6 +241,9 @@ def _fwd(entry, x, delta, A, B, C, D, z, delta_bias, softplus, y, final_state,
     ]
     if entry == "selscan_fwd_from_state":
         args.append(_ptr(initial_state, "initial_state", (batch, dim, N), f32, dev))
+    elif entry == "selscan_fwd_conv":
+        args.append(_ptr(initial_state, "initial_state", (batch, dim, N), f32, dev,
+                         required=False))
     args += [
         _ptr(y, "y", (batch, L, dim), dt, dev),
         _ptr(final_state, "final_state", (batch, dim, N), f32, dev, required=False),
