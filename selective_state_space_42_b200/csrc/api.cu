@@ -611,29 +611,40 @@ int selscan_device_status(int *status, int clear) {
     return e == cudaSuccess ? SELSCAN_OK : selscan::cuda_fail(e);
 }
 
-int selscan_state_update(float *state, const void *x, const void *delta, const float *A,
-                         const void *B, const void *C, const float *D, const void *z,
-                         const float *delta_bias, int softplus_flag, void *y,
-                         int64_t batch, int64_t dim, int64_t dstate, selscan_dtype_t dtype,
-                         selscan_stream_t stream_) {
+}  // extern "C"
+
+namespace {
+
+int step_entry(float *state, float *conv_state, const float *conv_w, const float *conv_b,
+               int conv_width, const void *x, const void *delta, const float *A,
+               const void *B, const void *C, const float *D, const void *z,
+               const float *delta_bias, int softplus_flag, void *y, int64_t batch, int64_t dim,
+               int64_t dstate, selscan_dtype_t dtype, selscan_stream_t stream_) {
     cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
     if (dtype != SELSCAN_F32 && dtype != SELSCAN_BF16) return SELSCAN_ERR_BAD_DTYPE;
     if (batch < 0 || dim < 0) return SELSCAN_ERR_BAD_DIM;
     if (dstate < 1 || dstate > SELSCAN_MAX_DSTATE) return SELSCAN_ERR_DSTATE_UNSUPPORTED;
+    if (conv_width < 0 || conv_width > selscan::kMaxConv) return SELSCAN_ERR_BAD_DIM;
     if (batch * dim > 0 && (!state || !x || !delta || !A || !B || !C || !y))
+        return SELSCAN_ERR_NULL_ARG;
+    if (batch * dim > 0 && conv_width > 0 && (!conv_state || !conv_w))
         return SELSCAN_ERR_NULL_ARG;
     if (!mul_le(batch, dim, kMaxElems / 64)) return SELSCAN_ERR_BAD_DIM;
     const size_t es = dtype == SELSCAN_F32 ? 4 : 2;
     if (misaligned(x, es) || misaligned(delta, es) || misaligned(z, es) ||
         misaligned(B, es) || misaligned(C, es) || misaligned(y, es) ||
         misaligned(state, 4) || misaligned(A, 4) || misaligned(D, 4) ||
-        misaligned(delta_bias, 4))
+        misaligned(delta_bias, 4) || misaligned(conv_state, 4) || misaligned(conv_w, 4) ||
+        misaligned(conv_b, 4))
         return SELSCAN_ERR_MISALIGNED;
     const size_t ny = (size_t)(batch * dim) * es;
     const size_t nbc = (size_t)(batch * dstate) * es;
     const size_t ns = (size_t)(batch * dim * dstate) * sizeof(float);
+    const size_t ncs = conv_width > 0 ? (size_t)(batch * dim) * 3 * sizeof(float) : 0;
     if (overlaps(y, ny, x, ny) || overlaps(y, ny, delta, ny) || overlaps(y, ny, z, ny) ||
-        overlaps(y, ny, B, nbc) || overlaps(y, ny, C, nbc) || overlaps(y, ny, state, ns))
+        overlaps(y, ny, B, nbc) || overlaps(y, ny, C, nbc) || overlaps(y, ny, state, ns) ||
+        overlaps(y, ny, conv_state, ncs) || overlaps(conv_state, ncs, state, ns) ||
+        overlaps(conv_state, ncs, x, ny))
         return SELSCAN_ERR_ALIAS;
     if (batch == 0 || dim == 0) return SELSCAN_OK;
     if (!mul_le(batch * dim, 4, (int64_t)INT32_MAX * 256)) return SELSCAN_ERR_BAD_DIM;
@@ -641,10 +652,39 @@ int selscan_state_update(float *state, const void *x, const void *delta, const f
     selscan::StepParams p{};
     p.state = state; p.x = x; p.delta = delta; p.z = z; p.B = B; p.C = C;
     p.A = A; p.Dskip = D; p.delta_bias = delta_bias; p.y = y;
+    p.conv_width = conv_width;
+    p.conv_state = conv_width > 0 ? conv_state : nullptr;
+    p.conv_w = conv_width > 0 ? conv_w : nullptr;
+    p.conv_b = conv_width > 0 ? conv_b : nullptr;
     p.batch = batch; p.dim = dim; p.dstate = (int)dstate;
     p.softplus = softplus_flag ? 1 : 0;
     cudaError_t e = selscan::launch_state_update(p, dtype == SELSCAN_BF16, stream);
     return e == cudaSuccess ? SELSCAN_OK : selscan::cuda_fail(e);
+}
+
+}  // namespace
+
+extern "C" {
+
+int selscan_state_update(float *state, const void *x, const void *delta, const float *A,
+                         const void *B, const void *C, const float *D, const void *z,
+                         const float *delta_bias, int softplus_flag, void *y,
+                         int64_t batch, int64_t dim, int64_t dstate, selscan_dtype_t dtype,
+                         selscan_stream_t stream) {
+    return step_entry(state, nullptr, nullptr, nullptr, 0, x, delta, A, B, C, D, z,
+                      delta_bias, softplus_flag, y, batch, dim, dstate, dtype, stream);
+}
+
+int selscan_state_update_conv(float *state, float *conv_state, const void *x_in,
+                              const float *conv_weight, const float *conv_bias, int conv_width,
+                              const void *delta, const float *A, const void *B, const void *C,
+                              const float *D, const void *z, const float *delta_bias,
+                              int softplus_flag, void *y, int64_t batch, int64_t dim,
+                              int64_t dstate, selscan_dtype_t dtype, selscan_stream_t stream) {
+    if (conv_width < 1) return SELSCAN_ERR_BAD_DIM;
+    return step_entry(state, conv_state, conv_weight, conv_bias, conv_width, x_in, delta, A,
+                      B, C, D, z, delta_bias, softplus_flag, y, batch, dim, dstate, dtype,
+                      stream);
 }
 
 }  // extern "C"

@@ -58,13 +58,22 @@ template <typename T> struct TileCfg;
 template <> struct TileCfg<__nv_bfloat16> { static constexpr int kTile = 32; };
 template <> struct TileCfg<float> { static constexpr int kTile = 16; };
 
-// Rows of x before a tile that the causal conv reads (the tile's tokens
-// start at row kHalo of the x buffer).
+// Rows of x before a tile that the causal conv reads.
 constexpr int kHalo = kMaxConv - 1;
 
-template <typename T> struct alignas(128) Stage {
+// The x rows of a stage: with the conv, the kHalo tokens before the tile
+// sit right before the tile's rows, so one TMA box fills both.
+template <typename T, bool kConv> struct XRows;
+template <typename T> struct XRows<T, false> {
+    T x[TileCfg<T>::kTile][kChannels];
+};
+template <typename T> struct XRows<T, true> {
+    T xh[kHalo][kChannels];
+    T x[TileCfg<T>::kTile][kChannels];
+};
+
+template <typename T, bool kConv> struct alignas(128) Stage : XRows<T, kConv> {
     static constexpr int kTile = TileCfg<T>::kTile;
-    T x[kHalo + kTile][kChannels];  // with the conv: the kHalo tokens before the tile, then the tile
     T dl[kTile][kChannels];
     T z[kTile][kChannels];
     T Bs[kTile * kMaxN];  // TMA destination: the tile's B rows, dstate per row
@@ -88,8 +97,8 @@ struct TileInfo {
 
 constexpr int kYBufs = 2;  // y staging tiles per consumer warp (TMA stores in flight)
 
-template <typename T> struct alignas(128) Shared {
-    Stage<T> stage[kStages];
+template <typename T, bool kConv> struct alignas(128) Shared {
+    Stage<T, kConv> stage[kStages];
     // per consumer warp: y of its 32 channels for one full tile, [kTile][32]
     alignas(128) T ybuf[kConsumerWarps][kYBufs][TileCfg<T>::kTile * 32];
     TileInfo info[kStages];
@@ -123,8 +132,8 @@ __device__ __forceinline__ void fail(const TmaScanParams &p, int *abort, int cod
 // per row) to float32 [kTile][16], zero for rows past nt and states past
 // dstate. Lane l handles float4 slots l, l + 32, ...: consecutive lanes write
 // consecutive 16-byte chunks.
-template <typename T>
-__device__ __forceinline__ void convert_bc(Stage<T> &st, int nt, int dstate, int lane) {
+template <typename T, bool kConv>
+__device__ __forceinline__ void convert_bc(Stage<T, kConv> &st, int nt, int dstate, int lane) {
     constexpr int kTile = TileCfg<T>::kTile;
     constexpr int kSlots = kTile * kMaxN / 4;
 #pragma unroll
@@ -148,7 +157,7 @@ __device__ __forceinline__ void convert_bc(Stage<T> &st, int nt, int dstate, int
 // latency itself; the stage is handed to the consumers (32 arrivals on
 // `full`) after its conversion.
 template <typename T, bool kGate, bool kConv>
-__device__ void produce(Shared<T> &S, const TmaScanParams &p, const CUtensorMap *tm_x,
+__device__ void produce(Shared<T, kConv> &S, const TmaScanParams &p, const CUtensorMap *tm_x,
                         const CUtensorMap *tm_d, const CUtensorMap *tm_z,
                         const CUtensorMap *tm_b, const CUtensorMap *tm_c) {
     constexpr int kTile = TileCfg<T>::kTile;
@@ -174,7 +183,7 @@ __device__ void produce(Shared<T> &S, const TmaScanParams &p, const CUtensorMap 
     // converts the oldest pending stage and hands it to the consumers
     auto convert_oldest = [&]() -> bool {
         if (!mbar_wait(&S.bc[cs], cphase, &S.abort, p.timeout_ns)) return false;
-        convert_bc<T>(S.stage[cs], S.info[cs].nt, p.dstate, lane);
+        convert_bc<T, kConv>(S.stage[cs], S.info[cs].nt, p.dstate, lane);
         __syncwarp();
         mbar_arrive(&S.full[cs]);
         if (++cs == kStages) {
@@ -236,11 +245,11 @@ __device__ void produce(Shared<T> &S, const TmaScanParams &p, const CUtensorMap 
                 // with the conv the box starts kHalo rows early (a negative row
                 // at the very start reads zeros; rows of the previous sequence
                 // are ignored by the consumers)
-                if (kConv)
-                    tma_load_2d(&S.stage[s].x[0][0], tm_x, &S.full[s], tile * kChannels,
+                if constexpr (kConv)
+                    tma_load_2d(&S.stage[s].xh[0][0], tm_x, &S.full[s], tile * kChannels,
                                 c1 - kHalo);
                 else
-                    tma_load_2d(&S.stage[s].x[kHalo][0], tm_x, &S.full[s], tile * kChannels, c1);
+                    tma_load_2d(&S.stage[s].x[0][0], tm_x, &S.full[s], tile * kChannels, c1);
                 tma_load_2d(&S.stage[s].dl[0][0], tm_d, &S.full[s], tile * kChannels, c1);
                 if (kGate) tma_load_2d(&S.stage[s].z[0][0], tm_z, &S.full[s], tile * kChannels, c1);
                 mbar_arrive_expect_tx(&S.bc[s], bc_bytes);
@@ -273,7 +282,8 @@ __device__ __forceinline__ float softplus_fast(float v) {
 // the state unchanged and y goes straight to global memory.
 template <typename T, bool kGate, int kMode, bool kStruct, bool kSoftplus, bool kFull,
           bool kConv>
-__device__ __forceinline__ void consume_tile(const Stage<T> &st, int nt, float2 (&h)[kMaxN / 2],
+__device__ __forceinline__ void consume_tile(const Stage<T, kConv> &st, int nt,
+                                             float2 (&h)[kMaxN / 2],
                                              const float (&A2)[kMaxN], float dskip, float bias,
                                              float &dt_sum, T *ys, T *yp, long long ybase,
                                              long long ystride, bool active,
@@ -291,7 +301,7 @@ __device__ __forceinline__ void consume_tile(const Stage<T> &st, int nt, float2 
 #pragma unroll
         for (int k = 0; k < kSub; ++k) {
             const int t = sub + k;
-            float xv = to_f32(st.x[kHalo + t][c]);
+            float xv = to_f32(st.x[t][c]);
             if (kConv) xv = conv_step(cw, cb, xw, xv);
             float dt = to_f32(st.dl[t][c]) + bias;
             if (kSoftplus) dt = kFastSp ? softplus_fast(dt) : softplus_f32(dt);
@@ -363,7 +373,7 @@ __device__ __forceinline__ void consume_tile(const Stage<T> &st, int nt, float2 
 }
 
 template <typename T, bool kGate, int kMode, bool kSoftplus, bool kConv>
-__device__ void consume(Shared<T> &S, const TmaScanParams &p, const CUtensorMap *tm_y) {
+__device__ void consume(Shared<T, kConv> &S, const TmaScanParams &p, const CUtensorMap *tm_y) {
     constexpr int kTile = TileCfg<T>::kTile;
     const int c = threadIdx.x;  // 0..127
     const int lane = c & 31;
@@ -465,12 +475,15 @@ __device__ void consume(Shared<T> &S, const TmaScanParams &p, const CUtensorMap 
         // conv window: the inputs of the kHalo tokens before the tile (zero
         // before the sequence's first token)
         float xw[kMaxConv - 1] = {0.f, 0.f, 0.f};
-        if (kConv && inf.t0 > 0) {
+        if constexpr (kConv) {
+            if (inf.t0 > 0) {
 #pragma unroll
-            for (int k = 0; k < kHalo; ++k) xw[k] = to_f32(S.stage[s].x[k][c]);
-        } else if (kConv && p.conv_init && active) {
+                for (int k = 0; k < kHalo; ++k) xw[k] = to_f32(S.stage[s].xh[k][c]);
+            } else if (p.conv_init && active) {
 #pragma unroll
-            for (int k = 0; k < kHalo; ++k) xw[k] = p.conv_init[(inf.b * p.dim + d) * kHalo + k];
+                for (int k = 0; k < kHalo; ++k)
+                    xw[k] = p.conv_init[(inf.b * p.dim + d) * kHalo + k];
+            }
         }
         if (inf.nt == kTile) {
             T *ys = S.ybuf[warp][kbuf];
@@ -563,7 +576,7 @@ scan_tma_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
     // to a shared-memory instruction (no generic addressing, no aliasing with
     // the global y stores).
     extern __shared__ __align__(1024) unsigned char smem_raw[];
-    Shared<T> &S = *reinterpret_cast<Shared<T> *>(smem_raw);
+    Shared<T, kConv> &S = *reinterpret_cast<Shared<T, kConv> *>(smem_raw);
     if (threadIdx.x == 0) {
         for (int i = 0; i < kStages; ++i) {
             mbar_init(&S.full[i], 32);              // producer lanes (+ TMA bytes)
@@ -642,7 +655,7 @@ cudaError_t launch_mode(const TmaScanParams &p, const void *x, const void *dl, c
     } else {
         mz = md;
     }
-    const size_t smem = sizeof(Shared<T>);
+    const size_t smem = sizeof(Shared<T, kConv>);
     auto kern = scan_tma_kernel<T, kGate, kMode, kSoftplus, kConv>;
     // the shared-memory opt-in is set once per device for this instantiation
     static std::atomic<unsigned long long> configured{0};

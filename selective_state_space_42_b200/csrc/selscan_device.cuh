@@ -122,6 +122,10 @@ struct StepParams {
     const void *x, *delta, *z, *B, *C;
     const float *A, *Dskip, *delta_bias;
     void *y;
+    float *conv_state;     // [batch][dim][kMaxConv − 1] conv inputs before the token (in-out)
+    const float *conv_w;   // [dim][conv_width] (conv_width > 0)
+    const float *conv_b;   // [dim] (NULL: zero)
+    int conv_width;        // 0: no conv
     int64_t batch, dim;
     int dstate;
     int softplus;

@@ -25,12 +25,29 @@ constexpr int kPerLane = kMaxN / kLanesPerChain;  // 4 states per lane
 constexpr int kChainsPerLane = 4;                 // chains per lane, 8 apart
 constexpr int kChainsPerWarp = 32 / kLanesPerChain * kChainsPerLane;  // 32
 
-template <typename T, bool kGate>
+// The causal conv + SiLU for one chain's token: reads the chain's window of
+// the previous inputs, writes it back shifted by the new input.
+template <typename T>
+__device__ __forceinline__ float conv_token(const StepParams &p, int64_t chain, int64_t d) {
+    const float xin = ldg_f32(static_cast<const T *>(p.x) + chain);
+    float cw[kMaxConv];
+    load_conv_taps(p.conv_w, p.conv_width, d, cw);
+    float *cs = p.conv_state + chain * (kMaxConv - 1);
+    float xw[kMaxConv - 1] = {cs[0], cs[1], cs[2]};
+    const float xv = conv_step(cw, p.conv_b ? p.conv_b[d] : 0.0f, xw, xin);
+#pragma unroll
+    for (int k = 0; k < kMaxConv - 1; ++k) cs[k] = xw[k];
+    return xv;
+}
+
+// x (after the conv, if any), z and Δ of one chain's token. With the conv,
+// conv_x is the conv output computed by the caller.
+template <typename T, bool kGate, bool kConv>
 __device__ __forceinline__ float token_scalars(const StepParams &p, int64_t chain, int64_t d,
-                                               float &xv, float &zv) {
+                                               float &xv, float &zv, float conv_x = 0.0f) {
     const T *xp = static_cast<const T *>(p.x);
     const T *dp = static_cast<const T *>(p.delta);
-    xv = ldg_f32(xp + chain);
+    xv = kConv ? conv_x : ldg_f32(xp + chain);
     zv = kGate ? ldg_f32(static_cast<const T *>(p.z) + chain) : 0.0f;
     float dt = ldg_f32(dp + chain) + (p.delta_bias ? p.delta_bias[d] : 0.0f);
     if (p.softplus) dt = softplus_f32(dt);
@@ -59,7 +76,7 @@ __device__ __forceinline__ float4 ld4_f32(const __nv_bfloat16 *p) {
 // quad that hold a quarter of that chain, by shuffle. After the quad
 // reduction of Σ_n C[n]·h[n] every lane of the quad has the sum, and the
 // owner writes the chain's y.
-template <typename T, bool kGate>
+template <typename T, bool kGate, bool kConv>
 __global__ void __launch_bounds__(kThreads)
 state_update_vec_kernel(const StepParams p) {
     const int lane = threadIdx.x & 31;
@@ -104,7 +121,8 @@ state_update_vec_kernel(const StepParams p) {
     float dt_own = 0.f, u_own = 0.f, skip = 0.f, gate = 1.f;
     if (own < total) {
         float xv, zv;
-        dt_own = token_scalars<T, kGate>(p, own, own_d, xv, zv);
+        const float xc = kConv ? conv_token<T>(p, own, own_d) : 0.0f;
+        dt_own = token_scalars<T, kGate, kConv>(p, own, own_d, xv, zv, xc);
         u_own = dt_own * xv;
         skip = (p.Dskip ? p.Dskip[own_d] : 0.0f) * xv;
         if (kGate) gate = silu_f32(zv);
@@ -145,7 +163,7 @@ state_update_vec_kernel(const StepParams p) {
 }
 
 // Any dstate ≤ 16: one quad of lanes per chain, scalar accesses.
-template <typename T, bool kGate>
+template <typename T, bool kGate, bool kConv>
 __global__ void __launch_bounds__(kThreads)
 state_update_kernel(const StepParams p) {
     const int64_t gid = (int64_t)blockIdx.x * kThreads + threadIdx.x;
@@ -159,8 +177,14 @@ state_update_kernel(const StepParams p) {
     const T *Cp = static_cast<const T *>(p.C);
 
     float partial = 0.0f, xv = 0.0f, zv = 0.0f;
+    // the conv window belongs to the chain: the quad's first lane advances it
+    float xc = 0.0f;
+    if (kConv) {
+        if (active && q == 0) xc = conv_token<T>(p, chain, d);
+        xc = __shfl_sync(0xffffffffu, xc, (threadIdx.x & 31) & ~3);
+    }
     if (active) {
-        const float dt = token_scalars<T, kGate>(p, chain, d, xv, zv);
+        const float dt = token_scalars<T, kGate, kConv>(p, chain, d, xv, zv, xc);
         const float u = dt * xv;
         float *st = p.state + chain * p.dstate + n0;
 #pragma unroll
@@ -183,8 +207,8 @@ state_update_kernel(const StepParams p) {
     }
 }
 
-template <typename T, bool kGate>
-cudaError_t launch_gate(const StepParams &p, cudaStream_t stream) {
+template <typename T, bool kGate, bool kConv>
+cudaError_t launch_conv(const StepParams &p, cudaStream_t stream) {
     const int64_t chains = p.batch * p.dim;
     const uintptr_t bc_align = 4 * sizeof(T) - 1;
     const bool vec = p.dstate == kMaxN && (reinterpret_cast<uintptr_t>(p.state) & 15) == 0 &&
@@ -194,13 +218,19 @@ cudaError_t launch_gate(const StepParams &p, cudaStream_t stream) {
     if (vec) {
         const int64_t warps = (chains + kChainsPerWarp - 1) / kChainsPerWarp;
         const unsigned blocks = (unsigned)((warps * 32 + kThreads - 1) / kThreads);
-        state_update_vec_kernel<T, kGate><<<blocks, kThreads, 0, stream>>>(p);
+        state_update_vec_kernel<T, kGate, kConv><<<blocks, kThreads, 0, stream>>>(p);
     } else {
         const int64_t threads = chains * kLanesPerChain;
         const unsigned blocks = (unsigned)((threads + kThreads - 1) / kThreads);
-        state_update_kernel<T, kGate><<<blocks, kThreads, 0, stream>>>(p);
+        state_update_kernel<T, kGate, kConv><<<blocks, kThreads, 0, stream>>>(p);
     }
     return cudaGetLastError();
+}
+
+template <typename T, bool kGate>
+cudaError_t launch_gate(const StepParams &p, cudaStream_t stream) {
+    return p.conv_width > 0 ? launch_conv<T, kGate, true>(p, stream)
+                            : launch_conv<T, kGate, false>(p, stream);
 }
 
 template <typename T>

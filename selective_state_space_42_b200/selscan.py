@@ -52,6 +52,9 @@ SIGNATURES = {
     "selscan_bwd_workspace_bytes": (_i64, [_i64, _i64, _i64, _i64]),
     "selscan_bwd_workspace": (_int, [_vp] * 8 + [_int] + [_vp] * 10
                               + [_i64, _i64, _i64, _i64, _int, _vp, _i64, _vp]),
+    "selscan_state_update_conv": (_int, [_vp, _vp, _vp, _vp, _vp, _int, _vp, _vp, _vp, _vp,
+                                         _vp, _vp, _vp, _int, _vp, _i64, _i64, _i64, _int,
+                                         _vp]),
     "selscan_device_status": (_int, [ctypes.POINTER(_int), _int]),
     "selscan_status_string": (ctypes.c_char_p, [_int]),
     "selscan_last_cuda_error": (ctypes.c_char_p, []),
@@ -320,11 +323,15 @@ def selscan_bwd_workspace_bytes(batch: int, seqlen: int, dim: int, dstate: int) 
 
 
 def selscan_state_update(state, x, delta, A, B, C, D=None, z=None, delta_bias=None,
-                         softplus=True, y=None, stream=None):
-    """One recurrent step in place on ``state`` (C ABI ``selscan_state_update``).
+                         softplus=True, y=None, stream=None, conv_state=None,
+                         conv_weight=None, conv_bias=None):
+    """One recurrent step in place on ``state`` (C ABI ``selscan_state_update``,
+    or ``selscan_state_update_conv`` when ``conv_weight`` is given).
 
     state: [batch, dim, dstate] float32 (updated); x, delta, z: [batch, dim];
-    B, C: [batch, dstate]. Returns y [batch, dim]."""
+    B, C: [batch, dstate]. With the conv: x is the conv input, conv_state
+    [batch, dim, 3] float32 holds the previous 3 inputs (updated), conv_weight
+    [dim, K], conv_bias [dim]. Returns y [batch, dim]."""
     torch = _torch()
     if state.dim() != 3:
         raise ValueError("state must be [batch, dim, dstate]")
@@ -334,9 +341,7 @@ def selscan_state_update(state, x, delta, A, B, C, D=None, z=None, delta_bias=No
     if y is None:
         y = torch.empty_like(x)
     f32 = torch.float32
-    args = [
-        _ptr(state, "state", (batch, dim, N), f32, dev),
-        _ptr(x, "x", (batch, dim), dt, dev),
+    tail = [
         _ptr(delta, "delta", (batch, dim), dt, dev),
         _ptr(A, "A", (dim, N), f32, dev),
         _ptr(B, "B", (batch, N), dt, dev),
@@ -348,5 +353,17 @@ def selscan_state_update(state, x, delta, A, B, C, D=None, z=None, delta_bias=No
         _ptr(y, "y", (batch, dim), dt, dev),
         batch, dim, N, code, _stream_ptr(stream, dev),
     ]
+    st = _ptr(state, "state", (batch, dim, N), f32, dev)
+    if conv_weight is not None:
+        if conv_weight.dim() != 2 or conv_weight.shape[0] != dim:
+            raise ValueError("conv_weight must be [dim, K]")
+        args = [st, _ptr(conv_state, "conv_state", (batch, dim, 3), f32, dev),
+                _ptr(x, "x", (batch, dim), dt, dev),
+                _ptr(conv_weight, "conv_weight", tuple(conv_weight.shape), f32, dev),
+                _ptr(conv_bias, "conv_bias", (dim,), f32, dev, required=False),
+                int(conv_weight.shape[1])] + tail
+        _check(load_library().selscan_state_update_conv(*args))
+        return y
+    args = [st, _ptr(x, "x", (batch, dim), dt, dev)] + tail
     _check(load_library().selscan_state_update(*args))
     return y

@@ -137,3 +137,67 @@ def test_conv_bench_shape_sampled():
     gh.compare(gh.to_np(y[:, :, list(chans)]), yo, gh.RTOL["bf16"], "bench conv y")
     gh.compare(gh.to_np(hf[:, list(chans)]), ho, gh.RTOL["bf16"], "bench conv state")
     assert ss.selscan_device_status() == 0
+
+
+@pytest.mark.parametrize("N", [16, 7])
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_decode_conv_trajectory(N, dtype):
+    """Decode steps with the conv in front: y, the SSM state and the conv
+    window after every step against the oracle's conv over the window and
+    the tokens, followed by its recurrent step."""
+    batch, dim, K, steps = 3, 70, 4, 12
+    w = wl.ScanWorkload("dconv", batch, steps, dim, N, dtype, gate=True, seed=4300 + N)
+    inp = wl.make_scan_inputs(w)
+    g = torch.Generator().manual_seed(4301 + N)
+    cw = torch.randn(dim, K, generator=g) * 0.5
+    cb = torch.randn(dim, generator=g) * 0.1
+    cs0 = torch.randn(batch, dim, 3, generator=g).to(inp["x"].dtype).float()
+    h0 = torch.randn(batch, dim, N, generator=g) * 0.1
+    if N != 16:
+        inp["A"] = -torch.rand(dim, N, generator=g) * 4 - 0.1
+    # oracle: conv over [window, tokens], then the recurrence step by step
+    orc = oracle.default()
+    n = gh.to_np
+    x_full = np.concatenate([np.transpose(n(cs0), (0, 2, 1)), n(inp["x"])], axis=1)
+    xc = orc.causal_conv1d(x_full, n(cw), n(cb), silu=True)[:, 3:]
+    ref = n(h0)
+    d = {k: (None if v is None else v.to(DEV)) for k, v in inp.items()}
+    state, cstate = h0.to(DEV).clone(), cs0.to(DEV).clone()
+    cwd, cbd = cw.to(DEV), cb.to(DEV)
+    for t in range(steps):
+        tok = {k: d[k][:, t].contiguous() for k in ("x", "delta", "z", "B", "C")}
+        y = ss.selscan_state_update(state, tok["x"], tok["delta"], d["A"], tok["B"], tok["C"],
+                                    d["D"], tok["z"], d["delta_bias"], conv_state=cstate,
+                                    conv_weight=cwd, conv_bias=cbd)
+        yo, ref = orc.state_update(ref, xc[:, t], n(inp["delta"][:, t]), n(inp["A"]),
+                                   n(inp["B"][:, t]), n(inp["C"][:, t]), n(inp["D"]),
+                                   n(inp["z"][:, t]), n(inp["delta_bias"]))
+        torch.cuda.synchronize()
+        gh.compare(gh.to_np(y), yo, gh.RTOL[dtype], f"step {t} y")
+        gh.compare(gh.to_np(state), ref, gh.RTOL[dtype], f"step {t} state")
+        want_cs = x_full[:, t + 1:t + 4].transpose(0, 2, 1)
+        assert np.array_equal(gh.to_np(cstate), want_cs), f"step {t} conv window"
+
+
+def test_prefill_then_decode_with_conv():
+    """selscan_fwd_conv over L tokens, then decode steps with the conv window
+    taken from the last 3 inputs, equal selscan_fwd_conv over all tokens."""
+    batch, dim, N, L, k = 2, 256, 16, 300, 6
+    inp, conv = _inputs(batch, L + k, dim, N, "f32", 4, seed=4400)
+    pre = {kk: (v[:, :L] if v is not None and v.dim() == 3 else v) for kk, v in inp.items()}
+    _, hf = _gpu(pre, conv)
+    state = hf.clone()
+    cstate = inp["x"][:, L - 3:L].float().permute(0, 2, 1).contiguous().to(DEV)
+    d = {kk: (None if v is None else v.to(DEV)) for kk, v in inp.items()}
+    ys = []
+    for t in range(L, L + k):
+        tok = {kk: d[kk][:, t].contiguous() for kk in ("x", "delta", "z", "B", "C")}
+        ys.append(ss.selscan_state_update(state, tok["x"], tok["delta"], d["A"], tok["B"],
+                                          tok["C"], d["D"], tok["z"], d["delta_bias"],
+                                          conv_state=cstate, conv_weight=conv["w"].to(DEV),
+                                          conv_bias=conv["b"].to(DEV)))
+    torch.cuda.synchronize()
+    yo, ho = _oracle(inp, conv)
+    got = np.stack([gh.to_np(v) for v in ys], axis=1)
+    gh.compare(got, yo[:, L:], gh.RTOL["f32"], "decode after prefill y")
+    gh.compare(gh.to_np(state), ho, gh.RTOL["f32"], "decode after prefill state")
