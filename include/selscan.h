@@ -156,6 +156,40 @@ SELSCAN_API int selscan_fwd_conv(const void *x_in, const float *conv_weight,
                                  int64_t batch, int64_t seqlen, int64_t dim, int64_t dstate,
                                  selscan_dtype_t dtype, selscan_stream_t stream);
 
+/* Input term of the discretisation. */
+enum {
+    SELSCAN_BBAR_DELTA = 0, /* Bbar·x = Δ·B·x ("SSM as RNN"; the default everywhere) */
+    SELSCAN_BBAR_ZOH = 1    /* Bbar·x = (exp(Δ·A) − 1)/A · B·x, zero-order hold ("Mamba &
+                               State Space Models — Guide Complet" §1 "Discrétisation",
+                               diagonal A; Δ·B·x where A = 0) */
+};
+
+/* Options of selscan_fwd_ex; a zero-initialised struct (or NULL) is
+ * selscan_fwd. Fields as in selscan_fwd_from_state and selscan_fwd_conv
+ * (conv_width 0: no conv). */
+typedef struct {
+    const float *initial_state; /* [batch, dim, dstate] or NULL */
+    const float *conv_weight;   /* [dim, conv_width] (conv_width > 0) */
+    const float *conv_bias;     /* [dim] or NULL */
+    const float *conv_init;     /* [batch, dim, 3] or NULL */
+    int conv_width;             /* 0 .. 4 */
+    int bbar_mode;              /* SELSCAN_BBAR_DELTA or SELSCAN_BBAR_ZOH */
+} selscan_fwd_options_t;
+
+/*
+ * selscan_fwd_ex -- selscan_fwd with every option: an initial state, the
+ * causal conv in front, and the input term. The zero-order-hold term runs on
+ * the generic (non-TMA) kernels, which also serve every shape the TMA kernel
+ * cannot take. options NULL: selscan_fwd. Unknown bbar_mode: SELSCAN_ERR_BAD_DIM.
+ */
+SELSCAN_API int selscan_fwd_ex(const void *x, const void *delta, const float *A,
+                               const void *B, const void *C, const float *D, const void *z,
+                               const float *delta_bias, int softplus_flag,
+                               const selscan_fwd_options_t *options, void *y,
+                               float *final_state, int64_t batch, int64_t seqlen,
+                               int64_t dim, int64_t dstate, selscan_dtype_t dtype,
+                               selscan_stream_t stream);
+
 /*
  * selscan_fwd_noalloc -- selscan_fwd without any device allocation.
  *
@@ -296,6 +330,47 @@ SELSCAN_API int selscan_bwd_workspace(const void *x, const void *delta, const fl
                                       int64_t dim, int64_t dstate, selscan_dtype_t dtype,
                                       void *workspace, int64_t workspace_bytes,
                                       selscan_stream_t stream);
+
+/*
+ * selscan_state_update_conv -- selscan_state_update with the causal conv +
+ * SiLU of selscan_fwd_conv in front, for decoding after a selscan_fwd_conv
+ * prefill: the token's x is silu(conv_bias + Σ_k conv_weight[d,k] · window),
+ * the window being the 3 previous inputs kept in conv_state followed by
+ * x_in; conv_state is then shifted to end with x_in.
+ *   conv_state    [batch, dim, 3]           float32      in-out: the x_in values
+ *                                                        of the 3 previous tokens,
+ *                                                        oldest first
+ *   x_in          [batch, dim]              dtype        required
+ *   conv_weight   [dim, conv_width], conv_bias [dim] (NULL -> zero), conv_width 1..4
+ * Other arguments as selscan_state_update. conv_state must not overlap any
+ * other argument.
+ */
+SELSCAN_API int selscan_state_update_conv(float *state, float *conv_state, const void *x_in,
+                                          const float *conv_weight, const float *conv_bias,
+                                          int conv_width, const void *delta, const float *A,
+                                          const void *B, const void *C, const float *D,
+                                          const void *z, const float *delta_bias,
+                                          int softplus_flag, void *y, int64_t batch,
+                                          int64_t dim, int64_t dstate, selscan_dtype_t dtype,
+                                          selscan_stream_t stream);
+
+/* Options of selscan_state_update_ex; zero-initialised (or NULL) is
+ * selscan_state_update. Fields as in selscan_state_update_conv. */
+typedef struct {
+    float *conv_state;          /* [batch, dim, 3], in-out (conv_width > 0) */
+    const float *conv_weight;   /* [dim, conv_width] */
+    const float *conv_bias;     /* [dim] or NULL */
+    int conv_width;             /* 0 .. 4 */
+    int bbar_mode;              /* SELSCAN_BBAR_DELTA or SELSCAN_BBAR_ZOH */
+} selscan_step_options_t;
+
+/* selscan_state_update with every option (conv window, input term). */
+SELSCAN_API int selscan_state_update_ex(float *state, const void *x, const void *delta,
+                                        const float *A, const void *B, const void *C,
+                                        const float *D, const void *z, const float *delta_bias,
+                                        int softplus_flag, const selscan_step_options_t *options,
+                                        void *y, int64_t batch, int64_t dim, int64_t dstate,
+                                        selscan_dtype_t dtype, selscan_stream_t stream);
 
 /*
  * selscan_device_status -- the library's sticky device-side error word on

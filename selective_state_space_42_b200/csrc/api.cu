@@ -178,7 +178,8 @@ void plan_for_sizes(int64_t batch, int64_t seqlen, int64_t dim, int64_t dstate, 
 int fwd_setup(const void *x, const void *delta, const float *A, const void *B,
               const void *C, const float *D, const void *z, const float *delta_bias,
               int softplus_flag, const float *h0, const float *conv_w, const float *conv_b,
-              const float *conv_init, int conv_width, void *y, float *final_state, int64_t batch,
+              const float *conv_init, int conv_width, int zoh, void *y, float *final_state,
+              int64_t batch,
               int64_t seqlen, int64_t dim, int64_t dstate, int dtype,
               cudaStream_t stream, FwdPlan *plan, bool *done) {
     *done = false;
@@ -232,7 +233,9 @@ int fwd_setup(const void *x, const void *delta, const float *A, const void *B,
 
     const bool aligned = !misaligned(x, 16) && !misaligned(delta, 16) && !misaligned(z, 16) &&
                          !misaligned(B, 16) && !misaligned(C, 16) && !misaligned(y, 16);
-    plan_for_sizes(batch, seqlen, dim, dstate, dtype, aligned, plan);
+    // the TMA kernel has no zero-order-hold input term: that mode takes the
+    // generic kernels
+    plan_for_sizes(batch, seqlen, dim, dstate, dtype, aligned && !zoh, plan);
     plan->x = x;
     plan->delta = delta;
     plan->z = z;
@@ -245,6 +248,7 @@ int fwd_setup(const void *x, const void *delta, const float *A, const void *B,
     g.conv_b = conv_width > 0 ? conv_b : nullptr;
     g.conv_init = conv_width > 0 ? conv_init : nullptr;
     g.conv_width = conv_width;
+    g.zoh = zoh ? 1 : 0;
     g.batch = batch; g.seqlen = seqlen; g.dim = dim; g.dstate = (int)dstate;
     g.softplus = softplus_flag ? 1 : 0;
     g.ws_P = g.ws_H = nullptr;
@@ -391,15 +395,15 @@ namespace {
 int fwd_entry(const void *x, const void *delta, const float *A, const void *B, const void *C,
               const float *D, const void *z, const float *delta_bias, int softplus_flag,
               const float *h0, const float *conv_w, const float *conv_b,
-              const float *conv_init, int conv_width, void *y, float *final_state,
+              const float *conv_init, int conv_width, int zoh, void *y, float *final_state,
               int64_t batch, int64_t seqlen, int64_t dim,
               int64_t dstate, selscan_dtype_t dtype, selscan_stream_t stream_) {
     cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
     selscan::FwdPlan plan;
     bool done = false;
     const int st = selscan::fwd_setup(x, delta, A, B, C, D, z, delta_bias, softplus_flag, h0,
-                                      conv_w, conv_b, conv_init, conv_width, y, final_state,
-                                      batch,
+                                      conv_w, conv_b, conv_init, conv_width, zoh, y,
+                                      final_state, batch,
                                       seqlen, dim, dstate, dtype, stream, &plan, &done);
     if (st != SELSCAN_OK || done) return st;
     void *ws = nullptr;
@@ -425,7 +429,7 @@ int selscan_fwd(const void *x, const void *delta, const float *A, const void *B,
                 int64_t seqlen, int64_t dim, int64_t dstate, selscan_dtype_t dtype,
                 selscan_stream_t stream) {
     return fwd_entry(x, delta, A, B, C, D, z, delta_bias, softplus_flag, nullptr, nullptr,
-                     nullptr, nullptr, 0, y, final_state, batch, seqlen, dim, dstate, dtype,
+                     nullptr, nullptr, 0, 0, y, final_state, batch, seqlen, dim, dstate, dtype,
                      stream);
 }
 
@@ -436,8 +440,8 @@ int selscan_fwd_from_state(const void *x, const void *delta, const float *A, con
                            int64_t batch, int64_t seqlen, int64_t dim, int64_t dstate,
                            selscan_dtype_t dtype, selscan_stream_t stream) {
     return fwd_entry(x, delta, A, B, C, D, z, delta_bias, softplus_flag, initial_state,
-                     nullptr, nullptr, nullptr, 0, y, final_state, batch, seqlen, dim, dstate,
-                     dtype, stream);
+                     nullptr, nullptr, nullptr, 0, 0, y, final_state, batch, seqlen, dim,
+                     dstate, dtype, stream);
 }
 
 int selscan_fwd_conv(const void *x_in, const float *conv_weight, const float *conv_bias,
@@ -448,8 +452,23 @@ int selscan_fwd_conv(const void *x_in, const float *conv_weight, const float *co
                      int64_t dstate, selscan_dtype_t dtype, selscan_stream_t stream) {
     if (conv_width < 1) return SELSCAN_ERR_BAD_DIM;
     return fwd_entry(x_in, delta, A, B, C, D, z, delta_bias, softplus_flag, initial_state,
-                     conv_weight, conv_bias, conv_init, conv_width, y, final_state, batch,
+                     conv_weight, conv_bias, conv_init, conv_width, 0, y, final_state, batch,
                      seqlen, dim, dstate, dtype, stream);
+}
+
+int selscan_fwd_ex(const void *x, const void *delta, const float *A, const void *B,
+                   const void *C, const float *D, const void *z, const float *delta_bias,
+                   int softplus_flag, const selscan_fwd_options_t *options, void *y,
+                   float *final_state, int64_t batch, int64_t seqlen, int64_t dim,
+                   int64_t dstate, selscan_dtype_t dtype, selscan_stream_t stream) {
+    selscan_fwd_options_t o{};
+    if (options) o = *options;
+    if (o.bbar_mode != SELSCAN_BBAR_DELTA && o.bbar_mode != SELSCAN_BBAR_ZOH)
+        return SELSCAN_ERR_BAD_DIM;
+    return fwd_entry(x, delta, A, B, C, D, z, delta_bias, softplus_flag, o.initial_state,
+                     o.conv_weight, o.conv_bias, o.conv_init, o.conv_width,
+                     o.bbar_mode == SELSCAN_BBAR_ZOH, y, final_state, batch, seqlen, dim,
+                     dstate, dtype, stream);
 }
 
 int selscan_fwd_plan(int64_t batch, int64_t seqlen, int64_t dim, int64_t dstate,
@@ -616,7 +635,7 @@ int selscan_device_status(int *status, int clear) {
 namespace {
 
 int step_entry(float *state, float *conv_state, const float *conv_w, const float *conv_b,
-               int conv_width, const void *x, const void *delta, const float *A,
+               int conv_width, int zoh, const void *x, const void *delta, const float *A,
                const void *B, const void *C, const float *D, const void *z,
                const float *delta_bias, int softplus_flag, void *y, int64_t batch, int64_t dim,
                int64_t dstate, selscan_dtype_t dtype, selscan_stream_t stream_) {
@@ -656,6 +675,7 @@ int step_entry(float *state, float *conv_state, const float *conv_w, const float
     p.conv_state = conv_width > 0 ? conv_state : nullptr;
     p.conv_w = conv_width > 0 ? conv_w : nullptr;
     p.conv_b = conv_width > 0 ? conv_b : nullptr;
+    p.zoh = zoh ? 1 : 0;
     p.batch = batch; p.dim = dim; p.dstate = (int)dstate;
     p.softplus = softplus_flag ? 1 : 0;
     cudaError_t e = selscan::launch_state_update(p, dtype == SELSCAN_BF16, stream);
@@ -671,7 +691,7 @@ int selscan_state_update(float *state, const void *x, const void *delta, const f
                          const float *delta_bias, int softplus_flag, void *y,
                          int64_t batch, int64_t dim, int64_t dstate, selscan_dtype_t dtype,
                          selscan_stream_t stream) {
-    return step_entry(state, nullptr, nullptr, nullptr, 0, x, delta, A, B, C, D, z,
+    return step_entry(state, nullptr, nullptr, nullptr, 0, 0, x, delta, A, B, C, D, z,
                       delta_bias, softplus_flag, y, batch, dim, dstate, dtype, stream);
 }
 
@@ -682,9 +702,24 @@ int selscan_state_update_conv(float *state, float *conv_state, const void *x_in,
                               int softplus_flag, void *y, int64_t batch, int64_t dim,
                               int64_t dstate, selscan_dtype_t dtype, selscan_stream_t stream) {
     if (conv_width < 1) return SELSCAN_ERR_BAD_DIM;
-    return step_entry(state, conv_state, conv_weight, conv_bias, conv_width, x_in, delta, A,
-                      B, C, D, z, delta_bias, softplus_flag, y, batch, dim, dstate, dtype,
+    return step_entry(state, conv_state, conv_weight, conv_bias, conv_width, 0, x_in, delta,
+                      A, B, C, D, z, delta_bias, softplus_flag, y, batch, dim, dstate, dtype,
                       stream);
+}
+
+int selscan_state_update_ex(float *state, const void *x, const void *delta, const float *A,
+                            const void *B, const void *C, const float *D, const void *z,
+                            const float *delta_bias, int softplus_flag,
+                            const selscan_step_options_t *options, void *y, int64_t batch,
+                            int64_t dim, int64_t dstate, selscan_dtype_t dtype,
+                            selscan_stream_t stream) {
+    selscan_step_options_t o{};
+    if (options) o = *options;
+    if (o.bbar_mode != SELSCAN_BBAR_DELTA && o.bbar_mode != SELSCAN_BBAR_ZOH)
+        return SELSCAN_ERR_BAD_DIM;
+    return step_entry(state, o.conv_state, o.conv_weight, o.conv_bias, o.conv_width,
+                      o.bbar_mode == SELSCAN_BBAR_ZOH, x, delta, A, B, C, D, z, delta_bias,
+                      softplus_flag, y, batch, dim, dstate, dtype, stream);
 }
 
 }  // extern "C"

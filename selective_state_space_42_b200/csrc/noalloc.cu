@@ -66,7 +66,7 @@ extern "C" int selscan_fwd_noalloc(const void *x, const void *delta, const float
     selscan::FwdPlan plan;
     bool done = false;
     const int st = selscan::fwd_setup(x, delta, A, B, C, D, z, delta_bias, softplus_flag,
-                                      nullptr, nullptr, nullptr, nullptr, 0, y, final_state, batch, seqlen, dim, dstate, dtype,
+                                      nullptr, nullptr, nullptr, nullptr, 0, 0, y, final_state, batch, seqlen, dim, dstate, dtype,
                                       stream, &plan, &done);
     if (st != SELSCAN_OK || done) return st;
     if (plan.ws_bytes > (size_t)SELSCAN_NOALLOC_WORKSPACE_BYTES) return SELSCAN_ERR_WORKSPACE;

@@ -97,7 +97,12 @@ __device__ __forceinline__ void scan_tile(const ScanParams &p, int64_t b, int64_
                 const float u = dt * xv[k];
                 float a[kMaxN];
                 discretize<kStruct>(dt, A2, a);
-                const float *Bt = sB[tt + k];
+                const float *Bt0 = sB[tt + k];
+                float Bz[kMaxN];  // B, times the ZOH factor in that mode
+#pragma unroll
+                for (int n = 0; n < kMaxN; ++n)
+                    Bz[n] = p.zoh ? Bt0[n] * zoh_factor(dt * A2[n] * kLn2, a[n]) : Bt0[n];
+                const float *Bt = Bz;
                 if (kMode == kModeAggregate) {
                     dt_sum += dt;
 #pragma unroll

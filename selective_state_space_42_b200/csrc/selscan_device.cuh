@@ -79,6 +79,15 @@ __device__ __forceinline__ void load_conv_taps(const float *w, int width, long l
     }
 }
 
+// Zero-order-hold input factor relative to Δ: (exp(z) − 1)/z with z = Δ·A,
+// given a = exp(z). Below |z| = 1/32 a four-term series (truncation under
+// z⁴/120 < 1e-8 relative); above, (a − 1)/z. The factor is 1 at z = 0, so
+// the ZOH input term Δ·B·x·factor reduces to the Δ·B·x term there.
+__device__ __forceinline__ float zoh_factor(float z, float a) {
+    const float series = fmaf(z, fmaf(z, fmaf(z, 1.0f / 24.0f, 1.0f / 6.0f), 0.5f), 1.0f);
+    return fabsf(z) < 0.03125f ? series : (a - 1.0f) / z;
+}
+
 // sigmoid(v) = 1 / (1 + e^-v); e^-v overflowing to +inf gives 0.
 __device__ __forceinline__ float sigmoid_f32(float v) {
     return rcp_approx(1.0f + ex2_approx(-v * kLog2e));
@@ -106,6 +115,7 @@ struct ScanParams {
     const float *conv_b; // [dim] (NULL: zero)
     const float *conv_init;  // [batch][dim][kMaxConv − 1]: conv inputs before token 0 (NULL: zero)
     int conv_width;      // 0 (no conv) or 1..kMaxConv
+    int zoh;             // input term: 0 Δ·B·x, 1 (exp(Δ·A) − 1)/A·B·x
     int64_t batch, seqlen, dim;
     int dstate;
     int softplus;
@@ -126,6 +136,7 @@ struct StepParams {
     const float *conv_w;   // [dim][conv_width] (conv_width > 0)
     const float *conv_b;   // [dim] (NULL: zero)
     int conv_width;        // 0: no conv
+    int zoh;               // input term: 0 Δ·B·x, 1 (exp(Δ·A) − 1)/A·B·x
     int64_t batch, dim;
     int dstate;
     int softplus;
@@ -217,7 +228,8 @@ struct FwdPlan {
 int fwd_setup(const void *x, const void *delta, const float *A, const void *B,
               const void *C, const float *D, const void *z, const float *delta_bias,
               int softplus_flag, const float *h0, const float *conv_w, const float *conv_b,
-              const float *conv_init, int conv_width, void *y, float *final_state, int64_t batch,
+              const float *conv_init, int conv_width, int zoh, void *y, float *final_state,
+              int64_t batch,
               int64_t seqlen, int64_t dim, int64_t dstate, int dtype,
               cudaStream_t stream, FwdPlan *plan, bool *done);
 // Plans for the given sizes assuming 16-byte aligned tensors (selscan_fwd_plan).

@@ -76,7 +76,7 @@ __device__ __forceinline__ float4 ld4_f32(const __nv_bfloat16 *p) {
 // quad that hold a quarter of that chain, by shuffle. After the quad
 // reduction of Σ_n C[n]·h[n] every lane of the quad has the sum, and the
 // owner writes the chain's y.
-template <typename T, bool kGate, bool kConv>
+template <typename T, bool kGate, bool kConv, bool kZoh>
 __global__ void __launch_bounds__(kThreads)
 state_update_vec_kernel(const StepParams p) {
     const int lane = threadIdx.x & 31;
@@ -143,10 +143,19 @@ state_update_vec_kernel(const StepParams p) {
             const float4 c4 = ld4_f32(Cp + bk[k] * kMaxN + 4 * q);
             const float dl = dt * kLog2e;
             float4 h = st[k];
-            h.x = fmaf(ex2_approx(dl * a4.x), h.x, u * b4.x);
-            h.y = fmaf(ex2_approx(dl * a4.y), h.y, u * b4.y);
-            h.z = fmaf(ex2_approx(dl * a4.z), h.z, u * b4.z);
-            h.w = fmaf(ex2_approx(dl * a4.w), h.w, u * b4.w);
+            const float e0 = ex2_approx(dl * a4.x), e1 = ex2_approx(dl * a4.y);
+            const float e2 = ex2_approx(dl * a4.z), e3 = ex2_approx(dl * a4.w);
+            float4 bz = b4;
+            if (kZoh) {
+                bz.x *= zoh_factor(dt * a4.x, e0);
+                bz.y *= zoh_factor(dt * a4.y, e1);
+                bz.z *= zoh_factor(dt * a4.z, e2);
+                bz.w *= zoh_factor(dt * a4.w, e3);
+            }
+            h.x = fmaf(e0, h.x, u * bz.x);
+            h.y = fmaf(e1, h.y, u * bz.y);
+            h.z = fmaf(e2, h.z, u * bz.z);
+            h.w = fmaf(e3, h.w, u * bz.w);
             *reinterpret_cast<float4 *>(p.state + chain * kMaxN + 4 * q) = h;
             partial = fmaf(c4.x, h.x, fmaf(c4.y, h.y, fmaf(c4.z, h.z, c4.w * h.w)));
         }
@@ -163,7 +172,7 @@ state_update_vec_kernel(const StepParams p) {
 }
 
 // Any dstate ≤ 16: one quad of lanes per chain, scalar accesses.
-template <typename T, bool kGate, bool kConv>
+template <typename T, bool kGate, bool kConv, bool kZoh>
 __global__ void __launch_bounds__(kThreads)
 state_update_kernel(const StepParams p) {
     const int64_t gid = (int64_t)blockIdx.x * kThreads + threadIdx.x;
@@ -191,8 +200,11 @@ state_update_kernel(const StepParams p) {
         for (int k = 0; k < kPerLane; ++k) {
             const int n = n0 + k;
             if (n < p.dstate) {
-                const float a = ex2_approx(dt * p.A[d * p.dstate + n] * kLog2e);
-                const float h = fmaf(a, st[k], u * ldg_f32(Bp + b * p.dstate + n));
+                const float an = p.A[d * p.dstate + n];
+                const float a = ex2_approx(dt * an * kLog2e);
+                float bn = ldg_f32(Bp + b * p.dstate + n);
+                if (kZoh) bn *= zoh_factor(dt * an, a);
+                const float h = fmaf(a, st[k], u * bn);
                 st[k] = h;
                 partial = fmaf(ldg_f32(Cp + b * p.dstate + n), h, partial);
             }
@@ -207,8 +219,8 @@ state_update_kernel(const StepParams p) {
     }
 }
 
-template <typename T, bool kGate, bool kConv>
-cudaError_t launch_conv(const StepParams &p, cudaStream_t stream) {
+template <typename T, bool kGate, bool kConv, bool kZoh>
+cudaError_t launch_zoh(const StepParams &p, cudaStream_t stream) {
     const int64_t chains = p.batch * p.dim;
     const uintptr_t bc_align = 4 * sizeof(T) - 1;
     const bool vec = p.dstate == kMaxN && (reinterpret_cast<uintptr_t>(p.state) & 15) == 0 &&
@@ -218,13 +230,19 @@ cudaError_t launch_conv(const StepParams &p, cudaStream_t stream) {
     if (vec) {
         const int64_t warps = (chains + kChainsPerWarp - 1) / kChainsPerWarp;
         const unsigned blocks = (unsigned)((warps * 32 + kThreads - 1) / kThreads);
-        state_update_vec_kernel<T, kGate, kConv><<<blocks, kThreads, 0, stream>>>(p);
+        state_update_vec_kernel<T, kGate, kConv, kZoh><<<blocks, kThreads, 0, stream>>>(p);
     } else {
         const int64_t threads = chains * kLanesPerChain;
         const unsigned blocks = (unsigned)((threads + kThreads - 1) / kThreads);
-        state_update_kernel<T, kGate, kConv><<<blocks, kThreads, 0, stream>>>(p);
+        state_update_kernel<T, kGate, kConv, kZoh><<<blocks, kThreads, 0, stream>>>(p);
     }
     return cudaGetLastError();
+}
+
+template <typename T, bool kGate, bool kConv>
+cudaError_t launch_conv(const StepParams &p, cudaStream_t stream) {
+    return p.zoh ? launch_zoh<T, kGate, kConv, true>(p, stream)
+                 : launch_zoh<T, kGate, kConv, false>(p, stream);
 }
 
 template <typename T, bool kGate>

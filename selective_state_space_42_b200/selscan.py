@@ -30,6 +30,23 @@ STATUS = {
 SELSCAN_NOALLOC_WORKSPACE_BYTES = 16 << 20
 
 _vp = ctypes.c_void_p
+
+
+class FwdOptions(ctypes.Structure):
+    """selscan_fwd_options_t (include/selscan.h)."""
+    _fields_ = [("initial_state", ctypes.c_void_p), ("conv_weight", ctypes.c_void_p),
+                ("conv_bias", ctypes.c_void_p), ("conv_init", ctypes.c_void_p),
+                ("conv_width", ctypes.c_int), ("bbar_mode", ctypes.c_int)]
+
+
+class StepOptions(ctypes.Structure):
+    """selscan_step_options_t (include/selscan.h)."""
+    _fields_ = [("conv_state", ctypes.c_void_p), ("conv_weight", ctypes.c_void_p),
+                ("conv_bias", ctypes.c_void_p), ("conv_width", ctypes.c_int),
+                ("bbar_mode", ctypes.c_int)]
+
+
+BBAR_MODES = {"delta": 0, "zoh": 1}
 _i64 = ctypes.c_int64
 _int = ctypes.c_int
 
@@ -55,6 +72,10 @@ SIGNATURES = {
     "selscan_state_update_conv": (_int, [_vp, _vp, _vp, _vp, _vp, _int, _vp, _vp, _vp, _vp,
                                          _vp, _vp, _vp, _int, _vp, _i64, _i64, _i64, _int,
                                          _vp]),
+    "selscan_fwd_ex": (_int, [_vp] * 8 + [_int, ctypes.POINTER(FwdOptions), _vp, _vp, _i64,
+                                          _i64, _i64, _i64, _int, _vp]),
+    "selscan_state_update_ex": (_int, [_vp] * 9 + [_int, ctypes.POINTER(StepOptions), _vp,
+                                                   _i64, _i64, _i64, _int, _vp]),
     "selscan_device_status": (_int, [ctypes.POINTER(_int), _int]),
     "selscan_status_string": (ctypes.c_char_p, [_int]),
     "selscan_last_cuda_error": (ctypes.c_char_p, []),
@@ -173,7 +194,8 @@ def selscan_device_status(clear: bool = False) -> int:
 
 def selscan_fwd(x, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=True,
                 y=None, final_state=None, return_final_state=False, stream=None,
-                initial_state=None, conv_weight=None, conv_bias=None, conv_init=None):
+                initial_state=None, conv_weight=None, conv_bias=None, conv_init=None,
+                bbar="delta"):
     """Selective scan over whole sequences (C ABI ``selscan_fwd``;
     ``selscan_fwd_from_state`` when ``initial_state`` is given;
     ``selscan_fwd_conv`` when ``conv_weight`` is given).
@@ -184,7 +206,12 @@ def selscan_fwd(x, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=Tru
     first token; None: zero; may be the same tensor as final_state).
     conv_weight [dim, K] (K ≤ 4), conv_bias [dim], conv_init [batch, dim, 3]
     float32: x is then the input of the causal depthwise conv + SiLU in front
-    of the scan. Returns y (allocated if not given) or (y, final_state)."""
+    of the scan. bbar: "delta" (Δ·B·x) or "zoh" (zero-order hold, C ABI
+    ``selscan_fwd_ex``). Returns y (allocated if not given) or (y, final_state)."""
+    if bbar != "delta":
+        return _fwd("selscan_fwd_ex", x, delta, A, B, C, D, z, delta_bias, softplus, y,
+                    final_state, return_final_state, stream, initial_state=initial_state,
+                    conv=(conv_weight, conv_bias, conv_init), bbar=bbar)
     if conv_weight is not None:
         return _fwd("selscan_fwd_conv", x, delta, A, B, C, D, z, delta_bias, softplus, y,
                     final_state, return_final_state, stream, initial_state=initial_state,
@@ -208,7 +235,7 @@ def selscan_fwd_noalloc(x, delta, A, B, C, D=None, z=None, delta_bias=None,
 
 
 def _fwd(entry, x, delta, A, B, C, D, z, delta_bias, softplus, y, final_state,
-         return_final_state, stream, initial_state=None, conv=None):
+         return_final_state, stream, initial_state=None, conv=None, bbar="delta"):
     torch = _torch()
     if x.dim() != 3:
         raise ValueError("x must be [batch, L, dim]")
@@ -242,6 +269,20 @@ def _fwd(entry, x, delta, A, B, C, D, z, delta_bias, softplus, y, final_state,
         _ptr(delta_bias, "delta_bias", (dim,), f32, dev, required=False),
         int(bool(softplus)),
     ]
+    keep = []  # objects the C call points into
+    if entry == "selscan_fwd_ex":
+        cw, cbias, cinit = conv
+        if bbar not in BBAR_MODES:
+            raise ValueError(f"bbar must be one of {list(BBAR_MODES)}")
+        opts = FwdOptions(
+            _ptr(initial_state, "initial_state", (batch, dim, N), f32, dev, required=False),
+            None if cw is None else _ptr(cw, "conv_weight", (dim, cw.shape[1]), f32, dev),
+            None if cw is None else _ptr(cbias, "conv_bias", (dim,), f32, dev, required=False),
+            None if cw is None else _ptr(cinit, "conv_init", (batch, dim, 3), f32, dev,
+                                         required=False),
+            0 if cw is None else int(cw.shape[1]), BBAR_MODES[bbar])
+        keep.append(opts)
+        args.append(ctypes.byref(opts))
     if entry == "selscan_fwd_from_state":
         args.append(_ptr(initial_state, "initial_state", (batch, dim, N), f32, dev))
     elif entry == "selscan_fwd_conv":
@@ -324,7 +365,7 @@ def selscan_bwd_workspace_bytes(batch: int, seqlen: int, dim: int, dstate: int) 
 
 def selscan_state_update(state, x, delta, A, B, C, D=None, z=None, delta_bias=None,
                          softplus=True, y=None, stream=None, conv_state=None,
-                         conv_weight=None, conv_bias=None):
+                         conv_weight=None, conv_bias=None, bbar="delta"):
     """One recurrent step in place on ``state`` (C ABI ``selscan_state_update``,
     or ``selscan_state_update_conv`` when ``conv_weight`` is given).
 
@@ -354,6 +395,20 @@ def selscan_state_update(state, x, delta, A, B, C, D=None, z=None, delta_bias=No
         batch, dim, N, code, _stream_ptr(stream, dev),
     ]
     st = _ptr(state, "state", (batch, dim, N), f32, dev)
+    if bbar != "delta":
+        if bbar not in BBAR_MODES:
+            raise ValueError(f"bbar must be one of {list(BBAR_MODES)}")
+        has_conv = conv_weight is not None
+        opts = StepOptions(
+            _ptr(conv_state, "conv_state", (batch, dim, 3), f32, dev) if has_conv else None,
+            _ptr(conv_weight, "conv_weight", tuple(conv_weight.shape), f32, dev)
+            if has_conv else None,
+            _ptr(conv_bias, "conv_bias", (dim,), f32, dev, required=False) if has_conv else None,
+            int(conv_weight.shape[1]) if has_conv else 0, BBAR_MODES[bbar])
+        args = [st, _ptr(x, "x", (batch, dim), dt, dev)] + tail[:8] + [ctypes.byref(opts)] \
+            + tail[8:]
+        _check(load_library().selscan_state_update_ex(*args))
+        return y
     if conv_weight is not None:
         if conv_weight.dim() != 2 or conv_weight.shape[0] != dim:
             raise ValueError("conv_weight must be [dim, K]")
