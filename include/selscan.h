@@ -64,14 +64,20 @@ enum {
     SELSCAN_ERR_BAD_DIM = -2,            /* a size is negative or too large */
     SELSCAN_ERR_BAD_DTYPE = -3,          /* dtype is not a selscan_dtype_t */
     SELSCAN_ERR_MISALIGNED = -4,         /* a pointer is not element-aligned */
-    SELSCAN_ERR_DSTATE_UNSUPPORTED = -5, /* dstate outside 1..16 */
+    SELSCAN_ERR_DSTATE_UNSUPPORTED = -5, /* dstate outside 1..SELSCAN_MAX_DSTATE
+                                            (1..SELSCAN_MAX_DSTATE_BWD for selscan_bwd) */
     SELSCAN_ERR_CUDA = -6,               /* a CUDA call failed */
     SELSCAN_ERR_ALIAS = -7,              /* y overlaps an input */
     SELSCAN_ERR_WORKSPACE = -8           /* the given or static workspace is too small
                                             (selscan_fwd_noalloc, selscan_bwd_workspace) */
 };
 
-#define SELSCAN_MAX_DSTATE 16
+/* Largest d_state of the forward and decode entry points. d_state ≤ 16 takes
+ * the TMA-staged and register-resident kernels; 17..256 take a kernel that
+ * splits each chain's states over 2-16 lanes (one pass, no chunking,
+ * batch ≤ 65535). The gradient (selscan_bwd) takes d_state ≤ 16. */
+#define SELSCAN_MAX_DSTATE 256
+#define SELSCAN_MAX_DSTATE_BWD 16
 
 /*
  * selscan_fwd -- selective scan over whole sequences (the forward pass).

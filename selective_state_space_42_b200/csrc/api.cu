@@ -165,10 +165,20 @@ void plan_for_sizes(int64_t batch, int64_t seqlen, int64_t dim, int64_t dstate, 
                           (dim * es) % 16 == 0 && (dstate * es) % 16 == 0 &&
                           batch * seqlen < ((int64_t)1 << 31) && dstate <= kMaxN;
     pl->bf16 = bf16;
-    if (eligible)
+    pl->wide = dstate > kMaxN;
+    if (pl->wide) {  // one pass of scan_wide.cu, no workspace
+        pl->tma = false;
+        pl->chunks = 1;
+        pl->launches = 1;
+        pl->ws_bytes = 0;
+        pl->ws_clear = 0;
+        pl->gp.nchunks = 1;
+        pl->gp.chunk_len = seqlen;
+    } else if (eligible) {
         plan_tma(batch, seqlen, dim, bf16, pl);
-    else
+    } else {
         plan_generic(batch, seqlen, dim, pl);
+    }
 }
 
 // Argument validation and launch plan shared by the selscan_fwd entry points.
@@ -190,6 +200,7 @@ int fwd_setup(const void *x, const void *delta, const float *A, const void *B,
         !mul_le(batch, dim, kMaxElems))
         return SELSCAN_ERR_BAD_DIM;
     if (conv_width < 0 || conv_width > kMaxConv) return SELSCAN_ERR_BAD_DIM;
+    if (dstate > kMaxN && batch > 65535) return SELSCAN_ERR_BAD_DIM;  // a grid dimension
     if (conv_width > 0 && dim > 0 && !conv_w) return SELSCAN_ERR_NULL_ARG;
     if (misaligned(conv_w, 4) || misaligned(conv_b, 4) || misaligned(conv_init, 4))
         return SELSCAN_ERR_MISALIGNED;
@@ -272,6 +283,7 @@ int fwd_setup(const void *x, const void *delta, const float *A, const void *B,
 }
 
 cudaError_t fwd_run(FwdPlan *plan, void *ws, cudaStream_t stream) {
+    if (plan->wide) return launch_scan_wide(plan->gp, plan->bf16, stream);
     if (!plan->tma) {
         ScanParams &g = plan->gp;
         if (g.nchunks > 1) {
@@ -493,7 +505,7 @@ int selscan_fwd_plan(int64_t batch, int64_t seqlen, int64_t dim, int64_t dstate,
 
 int64_t selscan_bwd_workspace_bytes(int64_t batch, int64_t seqlen, int64_t dim,
                                     int64_t dstate) {
-    if (batch <= 0 || seqlen <= 0 || dim <= 0 || dstate < 1 || dstate > SELSCAN_MAX_DSTATE)
+    if (batch <= 0 || seqlen <= 0 || dim <= 0 || dstate < 1 || dstate > selscan::kMaxN)
         return 0;
     if (!mul_le(batch, seqlen, kMaxElems) || !mul_le(batch * seqlen, dim, kMaxElems))
         return 0;
@@ -516,7 +528,7 @@ int bwd_entry(const void *x, const void *delta, const float *A, const void *B, c
     cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
     if (dtype != SELSCAN_F32 && dtype != SELSCAN_BF16) return SELSCAN_ERR_BAD_DTYPE;
     if (batch < 0 || seqlen < 0 || dim < 0 || batch > 65535) return SELSCAN_ERR_BAD_DIM;
-    if (dstate < 1 || dstate > SELSCAN_MAX_DSTATE) return SELSCAN_ERR_DSTATE_UNSUPPORTED;
+    if (dstate < 1 || dstate > selscan::kMaxN) return SELSCAN_ERR_DSTATE_UNSUPPORTED;
     if (!mul_le(batch, seqlen, kMaxElems) || !mul_le(batch * seqlen, dim, kMaxElems) ||
         !mul_le(batch, dim, kMaxElems))
         return SELSCAN_ERR_BAD_DIM;

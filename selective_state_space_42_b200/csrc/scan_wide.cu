@@ -1,0 +1,212 @@
+// scan_wide.cu -- the selective scan for d_state above 16 (up to 256).
+//
+// Pages: the same recurrence as scan.cu ("Mamba & State Space Models — Guide
+// Complet" §4, "Mamba и State Space Models: альтернатива Transformer", "SSM
+// as RNN"), at the larger state sizes the Guide's §5 ("Mamba-2") uses, where
+// A is a per-head scalar (A[d, n] constant across n) and d_state is 64 to 256.
+//
+// Work decomposition. A chain's states are split over kLanes = d_state / 16
+// (rounded up to a power of two) adjacent lanes of a warp, 16 states per lane
+// in registers. Every lane computes the chain's per-token scalars itself (the
+// loads of x, delta, z are broadcasts within the lane group), updates its 16
+// states and forms its part of Σ_n C[n]·h[n]; log2(kLanes) xor-shuffles finish
+// the sum and the group's first lane writes y. A CTA of 128 threads covers
+// 128 / kLanes consecutive channels of one batch row; B and C of a 16-token
+// tile are staged in shared memory as float32. One pass over the whole
+// sequence per CTA (no chunking). The exponent strategy follows scan.cu: with
+// A[d, n] == (n+1)·A[d, 0] on every channel of the CTA, Abar[n] = r^(n+1) is
+// a lane's base power r^(16·slice) times a ladder; otherwise one ex2 per
+// element. Optional: initial state, causal conv in front, ZOH input term.
+#include "selscan_device.cuh"
+
+namespace selscan {
+namespace {
+
+constexpr int kThreads = 128;
+constexpr int kTileT = 16;      // tokens per B/C tile
+constexpr int kMaxWide = 256;   // largest d_state of this kernel
+constexpr int kSlice = 16;      // states per lane
+
+template <typename T, bool kGate, int kLanes, bool kZoh>
+__global__ void __launch_bounds__(kThreads)
+scan_wide_kernel(const ScanParams p) {
+    constexpr int kWidth = kLanes * kSlice;  // padded d_state
+    constexpr int kChainsPerCta = kThreads / kLanes;
+    __shared__ float sB[kTileT][kWidth];
+    __shared__ float sC[kTileT][kWidth];
+    __shared__ float3 sX[kTileT][kChainsPerCta];  // x, delta, z of the tile per chain
+    const int tid = threadIdx.x;
+    const int slice = tid % kLanes;
+    const int64_t b = blockIdx.y;
+    const int64_t d = (int64_t)blockIdx.x * kChainsPerCta + tid / kLanes;
+    const bool active = d < p.dim;
+    const int N = p.dstate;
+    const int n0 = slice * kSlice;
+
+    float A2[kSlice];
+    bool structured = true, constant = true;
+    float a0 = 0.0f;
+    if (active) {
+        a0 = p.A[d * N];
+#pragma unroll
+        for (int i = 0; i < kSlice; ++i) {
+            const int n = n0 + i;
+            const float an = n < N ? p.A[d * N + n] : 0.0f;
+            A2[i] = an * kLog2e;
+            if (n < N) {
+                structured &= (an == (float)(n + 1) * a0);
+                constant &= (an == a0);
+            }
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < kSlice; ++i) A2[i] = 0.0f;
+    }
+    // decay strategy for the whole CTA: A[d, n] = A[d, 0] (a per-head scalar,
+    // one ex2 per token), A[d, n] = (n+1)·A[d, 0] (a power ladder), or general
+    constant = __syncthreads_and(constant);
+    structured = __syncthreads_and(structured);
+    const float dskip = (active && p.Dskip) ? p.Dskip[d] : 0.0f;
+    const float bias = (active && p.delta_bias) ? p.delta_bias[d] : 0.0f;
+
+    float h[kSlice];
+#pragma unroll
+    for (int i = 0; i < kSlice; ++i) {
+        const int n = n0 + i;
+        h[i] = (active && p.h0 && n < N) ? p.h0[(b * p.dim + d) * N + n] : 0.0f;
+    }
+
+    const bool conv = p.conv_width > 0;
+    float cw[kMaxConv] = {0.f, 0.f, 0.f, 0.f}, xw[kMaxConv - 1] = {0.f, 0.f, 0.f};
+    float cb = 0.0f;
+    if (conv && active) {
+        load_conv_taps(p.conv_w, p.conv_width, d, cw);
+        cb = p.conv_b ? p.conv_b[d] : 0.0f;
+        if (p.conv_init) {
+#pragma unroll
+            for (int k = 0; k < kMaxConv - 1; ++k)
+                xw[k] = p.conv_init[(b * p.dim + d) * (kMaxConv - 1) + k];
+        }
+    }
+
+    const T *xp = static_cast<const T *>(p.x);
+    const T *dp = static_cast<const T *>(p.delta);
+    const T *zp = static_cast<const T *>(p.z);
+    const T *Bp = static_cast<const T *>(p.B);
+    const T *Cp = static_cast<const T *>(p.C);
+    T *yp = static_cast<T *>(p.y);
+    for (int64_t t0 = 0; t0 < p.seqlen; t0 += kTileT) {
+        const int nt = (int)min((int64_t)kTileT, p.seqlen - t0);
+        __syncthreads();  // the previous tile is consumed
+        for (int e = tid; e < kTileT * kWidth; e += kThreads) {
+            const int t = e / kWidth, n = e % kWidth;
+            const bool in = t < nt && n < N;
+            const int64_t idx = (b * p.seqlen + t0 + t) * N + n;
+            sB[t][n] = in ? ldg_f32(Bp + idx) : 0.0f;
+            sC[t][n] = in ? ldg_f32(Cp + idx) : 0.0f;
+        }
+        // x, delta, z of the tile for the CTA's chains, staged once
+        for (int e = tid; e < kTileT * kChainsPerCta; e += kThreads) {
+            const int t = e / kChainsPerCta, cc = e % kChainsPerCta;
+            const int64_t dc = (int64_t)blockIdx.x * kChainsPerCta + cc;
+            const bool in = t < nt && dc < p.dim;
+            const int64_t i = (b * p.seqlen + t0 + t) * p.dim + dc;
+            sX[t][cc] = in ? make_float3(ldg_f32(xp + i), ldg_f32(dp + i),
+                                         kGate ? ldg_f32(zp + i) : 0.0f)
+                           : make_float3(0.f, 0.f, 0.f);
+        }
+        __syncthreads();
+        const int cc = tid / kLanes;
+#pragma unroll 1
+        for (int t = 0; t < nt; ++t) {
+            const float3 xdz = sX[t][cc];
+            float xv = xdz.x;
+            if (conv) xv = conv_step(cw, cb, xw, xv);
+            float dt = active ? xdz.y + bias : 0.0f;
+            if (p.softplus && active) dt = softplus_f32(dt);
+            const float u = dt * xv;
+            float a[kSlice];
+            if (constant) {
+                const float r = ex2_approx(dt * a0 * kLog2e);
+#pragma unroll
+                for (int k = 0; k < kSlice; ++k) a[k] = r;
+            } else if (structured) {
+                // r^(n0 + 1 + i) = r^n0 · r^(i + 1), the powers by a ladder of depth 4
+                const float r = ex2_approx(dt * a0 * kLog2e);
+                const float base = ex2_approx(dt * a0 * kLog2e * (float)n0);
+                float pw[kSlice];
+                pw[0] = r;
+                pw[1] = r * r;
+                pw[2] = pw[1] * r;
+                pw[3] = pw[1] * pw[1];
+#pragma unroll
+                for (int k = 4; k < 8; ++k) pw[k] = pw[k - 4] * pw[3];
+#pragma unroll
+                for (int k = 8; k < 16; ++k) pw[k] = pw[k - 8] * pw[7];
+#pragma unroll
+                for (int k = 0; k < kSlice; ++k) a[k] = base * pw[k];
+            } else {
+#pragma unroll
+                for (int k = 0; k < kSlice; ++k) a[k] = ex2_approx(dt * A2[k]);
+            }
+            float part0 = 0.0f, part1 = 0.0f;
+#pragma unroll
+            for (int k = 0; k < kSlice; k += 2) {
+                float b0 = sB[t][n0 + k], b1 = sB[t][n0 + k + 1];
+                if (kZoh) {
+                    b0 *= zoh_factor(dt * A2[k] * kLn2, a[k]);
+                    b1 *= zoh_factor(dt * A2[k + 1] * kLn2, a[k + 1]);
+                }
+                h[k] = fmaf(a[k], h[k], u * b0);
+                h[k + 1] = fmaf(a[k + 1], h[k + 1], u * b1);
+                part0 = fmaf(sC[t][n0 + k], h[k], part0);
+                part1 = fmaf(sC[t][n0 + k + 1], h[k + 1], part1);
+            }
+            float part = part0 + part1;
+#pragma unroll
+            for (int m = 1; m < kLanes; m <<= 1) part += __shfl_xor_sync(0xffffffffu, part, m);
+            if (active && slice == 0) {
+                float out = fmaf(dskip, xv, part);
+                if (kGate) out *= silu_f32(xdz.z);
+                yp[(b * p.seqlen + t0 + t) * p.dim + d] = from_f32<T>(out);
+            }
+        }
+    }
+    if (active && p.final_state) {
+#pragma unroll
+        for (int k = 0; k < kSlice; ++k)
+            if (n0 + k < N) p.final_state[(b * p.dim + d) * N + n0 + k] = h[k];
+    }
+}
+
+template <typename T, bool kGate, int kLanes>
+cudaError_t launch_lanes(const ScanParams &p, cudaStream_t stream) {
+    constexpr int kChainsPerCta = kThreads / kLanes;
+    const dim3 grid((unsigned)((p.dim + kChainsPerCta - 1) / kChainsPerCta), (unsigned)p.batch);
+    if (p.zoh)
+        scan_wide_kernel<T, kGate, kLanes, true><<<grid, kThreads, 0, stream>>>(p);
+    else
+        scan_wide_kernel<T, kGate, kLanes, false><<<grid, kThreads, 0, stream>>>(p);
+    return cudaGetLastError();
+}
+
+template <typename T, bool kGate>
+cudaError_t launch_gate(const ScanParams &p, cudaStream_t stream) {
+    if (p.dstate <= 32) return launch_lanes<T, kGate, 2>(p, stream);
+    if (p.dstate <= 64) return launch_lanes<T, kGate, 4>(p, stream);
+    if (p.dstate <= 128) return launch_lanes<T, kGate, 8>(p, stream);
+    return launch_lanes<T, kGate, 16>(p, stream);
+}
+
+}  // namespace
+
+int wide_max_dstate() { return kMaxWide; }
+
+cudaError_t launch_scan_wide(const ScanParams &p, bool bf16, cudaStream_t stream) {
+    if (bf16)
+        return p.z ? launch_gate<__nv_bfloat16, true>(p, stream)
+                   : launch_gate<__nv_bfloat16, false>(p, stream);
+    return p.z ? launch_gate<float, true>(p, stream) : launch_gate<float, false>(p, stream);
+}
+
+}  // namespace selscan

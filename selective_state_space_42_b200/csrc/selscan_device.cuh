@@ -202,6 +202,8 @@ cudaError_t launch_carry(const ScanParams &p, cudaStream_t stream);
 // Host-side launchers (one translation unit per kernel family).
 cudaError_t launch_scan(const ScanParams &p, bool bf16, cudaStream_t stream);
 cudaError_t launch_scan_bwd(const BwdParams &p, bool bf16, cudaStream_t stream);
+cudaError_t launch_scan_wide(const ScanParams &p, bool bf16, cudaStream_t stream);
+int wide_max_dstate();
 int bwd_tile_tokens();
 int bwd_tile_channels();
 cudaError_t launch_state_update(const StepParams &p, bool bf16, cudaStream_t stream);
@@ -219,6 +221,7 @@ struct FwdPlan {
     TmaScanParams tp{};   // TMA kernel
     const void *x = nullptr, *delta = nullptr, *z = nullptr;
     bool bf16 = false;
+    bool wide = false;    // d_state above kMaxN: scan_wide.cu
     int chunks = 1;       // sequence chunks
     int launches = 0;     // kernel launches
     size_t ws_bytes = 0;  // workspace bytes

@@ -21,7 +21,6 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kLanesPerChain = 4;
-constexpr int kPerLane = kMaxN / kLanesPerChain;  // 4 states per lane
 constexpr int kChainsPerLane = 4;                 // chains per lane, 8 apart
 constexpr int kChainsPerWarp = 32 / kLanesPerChain * kChainsPerLane;  // 32
 
@@ -171,7 +170,7 @@ state_update_vec_kernel(const StepParams p) {
     }
 }
 
-// Any dstate ≤ 16: one quad of lanes per chain, scalar accesses.
+// Any dstate: one quad of lanes per chain, lane q taking states q, q + 4, ...
 template <typename T, bool kGate, bool kConv, bool kZoh>
 __global__ void __launch_bounds__(kThreads)
 state_update_kernel(const StepParams p) {
@@ -181,7 +180,6 @@ state_update_kernel(const StepParams p) {
     const bool active = chain < p.batch * p.dim;
     const int64_t b = active ? chain / p.dim : 0;
     const int64_t d = active ? chain % p.dim : 0;
-    const int n0 = q * kPerLane;
     const T *Bp = static_cast<const T *>(p.B);
     const T *Cp = static_cast<const T *>(p.C);
 
@@ -195,19 +193,17 @@ state_update_kernel(const StepParams p) {
     if (active) {
         const float dt = token_scalars<T, kGate, kConv>(p, chain, d, xv, zv, xc);
         const float u = dt * xv;
-        float *st = p.state + chain * p.dstate + n0;
-#pragma unroll
-        for (int k = 0; k < kPerLane; ++k) {
-            const int n = n0 + k;
-            if (n < p.dstate) {
-                const float an = p.A[d * p.dstate + n];
-                const float a = ex2_approx(dt * an * kLog2e);
-                float bn = ldg_f32(Bp + b * p.dstate + n);
-                if (kZoh) bn *= zoh_factor(dt * an, a);
-                const float h = fmaf(a, st[k], u * bn);
-                st[k] = h;
-                partial = fmaf(ldg_f32(Cp + b * p.dstate + n), h, partial);
-            }
+        float *st = p.state + chain * p.dstate;
+        // lane q takes states q, q + 4, q + 8, ... (any d_state)
+#pragma unroll 4
+        for (int n = q; n < p.dstate; n += kLanesPerChain) {
+            const float an = p.A[d * p.dstate + n];
+            const float a = ex2_approx(dt * an * kLog2e);
+            float bn = ldg_f32(Bp + b * p.dstate + n);
+            if (kZoh) bn *= zoh_factor(dt * an, a);
+            const float h = fmaf(a, st[n], u * bn);
+            st[n] = h;
+            partial = fmaf(ldg_f32(Cp + b * p.dstate + n), h, partial);
         }
     }
     partial += __shfl_xor_sync(0xffffffffu, partial, 1);

@@ -96,7 +96,9 @@ def test_fwd_validation(lib):
     assert fwd(lib, seqlen=-5) == -2
     assert fwd(lib, batch=1 << 30, seqlen=1 << 30, dim=1 << 30) == -2
     assert fwd(lib, dstate=0) == -5
-    assert fwd(lib, dstate=17) == -5
+    assert fwd(lib, dstate=257) == -5
+    assert fwd(lib, dstate=17) == 0  # batch = 0: nothing to do
+    assert fwd(lib, batch=70000, dstate=32) == -2  # wide kernel: batch rows are a grid dimension
     assert fwd(lib, x=P + 1) == -4  # bf16 needs 2-byte alignment
     assert fwd(lib, x=P + 2, dtype=0) == -4  # fp32 needs 4-byte alignment
     assert fwd(lib, A=P + 2) == -4
@@ -127,7 +129,7 @@ def test_state_update_validation(lib):
     assert step(lib, batch=1, state=None) == -1
     assert step(lib, dtype=-1) == -3
     assert step(lib, dim=-1) == -2
-    assert step(lib, dstate=20) == -5
+    assert step(lib, dstate=257) == -5
     assert step(lib, state=P + 2) == -4
     assert step(lib, batch=1, y=P + 131072) == -7  # y overlaps the state
 
@@ -161,6 +163,7 @@ def test_bwd_validation(lib):
     assert bwd(lib, batch=-1) == -2
     assert bwd(lib, batch=70000, dim=4) == -2  # batch rows are a grid dimension
     assert bwd(lib, dstate=0) == -5
+    assert bwd(lib, dstate=17) == -5  # the gradient takes d_state <= 16
     full = dict(batch=1, dim=4)
     assert bwd(lib, x=None, **full) == -1
     assert bwd(lib, dy=None, **full) == -1

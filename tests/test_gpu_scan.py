@@ -143,8 +143,8 @@ def test_empty_and_degenerate():
 
 def test_errors_raise():
     x = torch.zeros(1, 4, 8, device=DEV, dtype=torch.bfloat16)
-    A = -torch.ones(8, 17, device=DEV)
-    BC = torch.zeros(1, 4, 17, device=DEV, dtype=torch.bfloat16)
+    A = -torch.ones(8, 257, device=DEV)
+    BC = torch.zeros(1, 4, 257, device=DEV, dtype=torch.bfloat16)
     with pytest.raises(ss.SelscanError) as e:
         ss.selscan_fwd(x, x, A, BC, BC)
     assert e.value.status == -5
