@@ -391,6 +391,44 @@ def main():
     h2d = sum(host[k].numel() * host[k].element_size() for k in names)
     d2h = y_h.numel() * y_h.element_size() + fs_h.numel() * fs_h.element_size()
 
+    # the decode step (one token in place on the [256, 5120, 16] state):
+    # back to back, and after an L2-evicting write; not part of the metric
+    dw = wl.DECODE
+    dstate_t = wl.make_decode_state(dw, device=dev)
+    dA, dDv, dbias = wl.make_decode_params(dw, device=dev)
+    dsteps = [wl.make_decode_step(dw, s, device=dev) for s in range(4)]
+
+    def decode(i):
+        t = dsteps[i % len(dsteps)]
+        ss.selscan_state_update(dstate_t, t["x"], t["delta"], dA, t["B"], t["C"], dDv, t["z"],
+                                dbias, stream=stream)
+
+    for i in range(5):
+        decode(i)
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    cold = []
+    for i in range(10):
+        flush.zero_()
+        c0 = torch.cuda.Event(enable_timing=True)
+        c1 = torch.cuda.Event(enable_timing=True)
+        c0.record(stream)
+        decode(i)
+        c1.record(stream)
+        torch.cuda.synchronize(dev)
+        cold.append(c0.elapsed_time(c1))
+    del flush
+    d0 = torch.cuda.Event(enable_timing=True)
+    d1 = torch.cuda.Event(enable_timing=True)
+    n_dec = 200
+    d0.record(stream)
+    for i in range(n_dec):
+        decode(i)
+    d1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    dec_ms = max_over_ranks(d0.elapsed_time(d1) / n_dec, dist if world > 1 else None, dev)
+    dec_cold = max_over_ranks(sorted(cold)[len(cold) // 2], dist if world > 1 else None, dev)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = oracle_cpu_baseline(inp, w, args.cpu_seconds)
@@ -422,6 +460,12 @@ def main():
         "e2e": {"value": job_rate(w.elements, world, args.e2e_steps, e2e_ms),
                 "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": e2e_ms / args.e2e_steps},
+        "decode_step": {
+            "workload": dw.name, "bytes_per_step": dw.algorithmic_bytes_per_step(),
+            "us_back_to_back": dec_ms * 1e3, "us_after_l2_flush": dec_cold * 1e3,
+            "GBps_back_to_back": dw.algorithmic_bytes_per_step() / dec_ms / 1e6,
+            "frac_back_to_back": dw.algorithmic_bytes_per_step() / dec_ms / 1e6 / peak,
+            "kernel": "state_update_vec_kernel<bf16, gate>"},
         "gpu_launches": args.steps * plan["launches"],
         "plan": plan,
         "cpu_baseline": cpu,

@@ -185,3 +185,21 @@ def test_bwd_workspace_bytes(lib):
     # one 16-token tile, one 32-channel tile: checkpoints 4·16·4 B, partials
     # 8·32·4 B, per-channel partials 4·(16 + 2)·4 B, each rounded up to 256 B
     assert lib.selscan_bwd_workspace_bytes(1, 8, 4, 16) == 256 + 1024 + 256 + 256 + 256
+
+
+def test_plans_of_the_workloads(lib):
+    """The host planner (no GPU: the SM count falls back to 148) picks one
+    pass for the Mamba-2.8B layer, the chunked plan for the 1M-token
+    sequence and the wide kernel (one launch, no workspace) above d_state 16."""
+    from selective_state_space_42_b200 import workloads as wl  # noqa: F401
+    p = ss.selscan_fwd_plan(4, 8192, 5120, 16)
+    assert p["launches"] == 1 and p["chunks"] == 8
+    p = ss.selscan_fwd_plan(1, 1 << 20, 2048, 16)
+    assert p["launches"] == 3 and p["chunks"] > 1 and p["workspace_bytes"] > 0
+    p = ss.selscan_fwd_plan(2, 4096, 2048, 128)
+    assert p == {"chunks": 1, "launches": 1, "workspace_bytes": 0}
+    w = wl.WORKLOADS["mamba130m_layer"]
+    p = ss.selscan_fwd_plan(w.batch, w.seqlen, w.dim, w.dstate)
+    assert p["launches"] == 1 and p["chunks"] == 2  # 96 groups: enough for one pass
+    p = ss.selscan_fwd_plan(1, 8192, 1536, 16)  # 12 groups: chunked
+    assert p["launches"] == 3
