@@ -338,6 +338,29 @@ SELSCAN_API int selscan_bwd_workspace(const void *x, const void *delta, const fl
                                       selscan_stream_t stream);
 
 /*
+ * selscan_bwd_from_state -- the gradient of selscan_fwd_from_state: as
+ * selscan_bwd_workspace, plus
+ *   initial_state   [batch, dim, dstate]  float32  the forward's initial state
+ *                                                  (NULL: zero)
+ *   dinitial_state  [batch, dim, dstate]  float32  output: the loss's gradient
+ *                                                  with respect to it (NULL: not
+ *                                                  written); λ carried past the
+ *                                                  first token, Abar_0·λ_0
+ * workspace NULL: allocated on the stream as selscan_bwd does.
+ */
+SELSCAN_API int selscan_bwd_from_state(const void *x, const void *delta, const float *A,
+                                       const void *B, const void *C, const float *D,
+                                       const void *z, const float *delta_bias,
+                                       int softplus_flag, const float *initial_state,
+                                       const void *dy, const float *dfinal_state, void *dx,
+                                       void *ddelta, float *dA, float *dB, float *dC,
+                                       float *dD, void *dz, float *ddelta_bias,
+                                       float *dinitial_state, int64_t batch, int64_t seqlen,
+                                       int64_t dim, int64_t dstate, selscan_dtype_t dtype,
+                                       void *workspace, int64_t workspace_bytes,
+                                       selscan_stream_t stream);
+
+/*
  * selscan_state_update_conv -- selscan_state_update with the causal conv +
  * SiLU of selscan_fwd_conv in front, for decoding after a selscan_fwd_conv
  * prefill: the token's x is silu(conv_bias + Σ_k conv_weight[d,k] · window),

@@ -523,7 +523,8 @@ int bwd_entry(const void *x, const void *delta, const float *A, const void *B, c
               const void *dy, const float *dfinal_state, void *dx, void *ddelta, float *dA,
               float *dB, float *dC, float *dD, void *dz, float *ddelta_bias, int64_t batch,
               int64_t seqlen, int64_t dim, int64_t dstate, selscan_dtype_t dtype,
-              void *workspace, int64_t workspace_bytes, bool allocate,
+              const float *h0, float *dh0, void *workspace, int64_t workspace_bytes,
+              bool allocate,
               selscan_stream_t stream_) {
     cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
     if (dtype != SELSCAN_F32 && dtype != SELSCAN_BF16) return SELSCAN_ERR_BAD_DTYPE;
@@ -544,7 +545,8 @@ int bwd_entry(const void *x, const void *delta, const float *A, const void *B, c
         misaligned(ddelta, es) || misaligned(dz, es) || misaligned(A, 4) ||
         misaligned(D, 4) || misaligned(delta_bias, 4) || misaligned(dfinal_state, 4) ||
         misaligned(dA, 4) || misaligned(dB, 4) || misaligned(dC, 4) || misaligned(dD, 4) ||
-        misaligned(ddelta_bias, 4) || misaligned(workspace, 256))
+        misaligned(ddelta_bias, 4) || misaligned(workspace, 256) || misaligned(h0, 4) ||
+        misaligned(dh0, 4))
         return SELSCAN_ERR_MISALIGNED;
     const size_t nx = (size_t)(batch * seqlen * dim) * es;
     const size_t nbc = (size_t)(batch * seqlen * dstate) * es;
@@ -552,10 +554,10 @@ int bwd_entry(const void *x, const void *delta, const float *A, const void *B, c
     const size_t na = (size_t)(dim * dstate) * 4, nd = (size_t)dim * 4;
     const size_t ns = (size_t)(batch * dim * dstate) * 4;
     const Span outs[] = {{dx, nx}, {ddelta, nx}, {dz, z ? nx : 0}, {dA, na}, {dB, nbcf},
-                         {dC, nbcf}, {dD, nd}, {ddelta_bias, nd}};
+                         {dC, nbcf}, {dD, nd}, {ddelta_bias, nd}, {dh0, ns}};
     const Span ins[] = {{x, nx}, {delta, nx}, {z, nx}, {dy, nx}, {B, nbc}, {C, nbc},
-                        {A, na}, {D, nd}, {delta_bias, nd}, {dfinal_state, ns}};
-    if (any_overlap(outs, 8, ins, 10)) return SELSCAN_ERR_ALIAS;
+                        {A, na}, {D, nd}, {delta_bias, nd}, {dfinal_state, ns}, {h0, ns}};
+    if (any_overlap(outs, 9, ins, 11)) return SELSCAN_ERR_ALIAS;
 
     if (!has_tokens) {
         // no token reaches the loss through a channel: the float32 gradients are 0
@@ -566,6 +568,11 @@ int bwd_entry(const void *x, const void *delta, const float *A, const void *B, c
         if (e == cudaSuccess && dim > 0 && dD) e = cudaMemsetAsync(dD, 0, nd, stream);
         if (e == cudaSuccess && dim > 0 && ddelta_bias)
             e = cudaMemsetAsync(ddelta_bias, 0, nd, stream);
+        // no token: the final state is the initial one
+        if (e == cudaSuccess && dh0 && ns > 0)
+            e = dfinal_state ? cudaMemcpyAsync(dh0, dfinal_state, ns, cudaMemcpyDeviceToDevice,
+                                               stream)
+                             : cudaMemsetAsync(dh0, 0, ns, stream);
         return e == cudaSuccess ? SELSCAN_OK : selscan::cuda_fail(e);
     }
 
@@ -574,12 +581,13 @@ int bwd_entry(const void *x, const void *delta, const float *A, const void *B, c
         if (!workspace) return SELSCAN_ERR_NULL_ARG;
         if (workspace_bytes < (int64_t)l.total) return SELSCAN_ERR_WORKSPACE;
         const Span wsp[] = {{workspace, l.total}};
-        if (any_overlap(wsp, 1, outs, 8) || any_overlap(wsp, 1, ins, 10))
+        if (any_overlap(wsp, 1, outs, 9) || any_overlap(wsp, 1, ins, 11))
             return SELSCAN_ERR_ALIAS;
     }
     selscan::BwdParams p{};
     p.x = x; p.delta = delta; p.z = z; p.B = B; p.C = C; p.dy = dy;
     p.A = A; p.Dskip = D; p.delta_bias = delta_bias; p.dfinal = dfinal_state;
+    p.h0 = h0; p.dh0 = dh0;
     p.dx = dx; p.ddelta = ddelta; p.dz = dz;
     p.dA = dA; p.dB = dB; p.dC = dC; p.dD = dD; p.ddelta_bias = ddelta_bias;
     p.batch = batch; p.seqlen = seqlen; p.dim = dim; p.dstate = (int)dstate;
@@ -620,7 +628,7 @@ int selscan_bwd(const void *x, const void *delta, const float *A, const void *B,
                 selscan_stream_t stream) {
     return bwd_entry(x, delta, A, B, C, D, z, delta_bias, softplus_flag, dy, dfinal_state, dx,
                      ddelta, dA, dB, dC, dD, dz, ddelta_bias, batch, seqlen, dim, dstate, dtype,
-                     nullptr, 0, true, stream);
+                     nullptr, nullptr, nullptr, 0, true, stream);
 }
 
 int selscan_bwd_workspace(const void *x, const void *delta, const float *A, const void *B,
@@ -633,7 +641,22 @@ int selscan_bwd_workspace(const void *x, const void *delta, const float *A, cons
                           selscan_stream_t stream) {
     return bwd_entry(x, delta, A, B, C, D, z, delta_bias, softplus_flag, dy, dfinal_state, dx,
                      ddelta, dA, dB, dC, dD, dz, ddelta_bias, batch, seqlen, dim, dstate, dtype,
-                     workspace, workspace_bytes, false, stream);
+                     nullptr, nullptr, workspace, workspace_bytes, false, stream);
+}
+
+int selscan_bwd_from_state(const void *x, const void *delta, const float *A, const void *B,
+                           const void *C, const float *D, const void *z,
+                           const float *delta_bias, int softplus_flag,
+                           const float *initial_state, const void *dy,
+                           const float *dfinal_state, void *dx, void *ddelta, float *dA,
+                           float *dB, float *dC, float *dD, void *dz, float *ddelta_bias,
+                           float *dinitial_state, int64_t batch, int64_t seqlen, int64_t dim,
+                           int64_t dstate, selscan_dtype_t dtype, void *workspace,
+                           int64_t workspace_bytes, selscan_stream_t stream) {
+    return bwd_entry(x, delta, A, B, C, D, z, delta_bias, softplus_flag, dy, dfinal_state, dx,
+                     ddelta, dA, dB, dC, dD, dz, ddelta_bias, batch, seqlen, dim, dstate, dtype,
+                     initial_state, dinitial_state, workspace, workspace_bytes,
+                     workspace == nullptr, stream);
 }
 
 int selscan_device_status(int *status, int clear) {

@@ -162,7 +162,11 @@ __device__ __forceinline__ void bwd_body(BwdSmem &S, const BwdParams &p) {
     {
         float2 h[kPairs];
 #pragma unroll
-        for (int j = 0; j < kPairs; ++j) h[j] = make_float2(0.f, 0.f);
+        for (int j = 0; j < kPairs; ++j) {
+            const float *h0 = p.h0 + (b * p.dim + dd) * N;
+            h[j] = make_float2((active && p.h0 && 2 * j < N) ? h0[2 * j] : 0.f,
+                               (active && p.h0 && 2 * j + 1 < N) ? h0[2 * j + 1] : 0.f);
+        }
         Raw<T> cur, nxt;
         float bv[4], cv[4];
         load_raw<T, kGate, false>(cur, p, b, 0, dd, active);
@@ -369,6 +373,15 @@ __device__ __forceinline__ void bwd_body(BwdSmem &S, const BwdParams &p) {
         for (int j = 0; j < 4; ++j) hc[j] = hn[j];
     }
 
+    // the initial state's gradient: λ carried past the first token
+    if (active && p.dh0) {
+        float *dh0 = p.dh0 + (b * p.dim + d) * N;
+#pragma unroll
+        for (int j = 0; j < kPairs; ++j) {
+            if (2 * j < N) dh0[2 * j] = lam[j].x;
+            if (2 * j + 1 < N) dh0[2 * j + 1] = lam[j].y;
+        }
+    }
     // per-(batch row, channel) partials
     if (active) {
         float4 *pa = reinterpret_cast<float4 *>(p.pA + (b * p.dim + d) * kMaxN);

@@ -146,6 +146,8 @@ struct StepParams {
 struct BwdParams {
     const void *x, *delta, *z, *B, *C, *dy;
     const float *A, *Dskip, *delta_bias, *dfinal;
+    const float *h0;  // state before the first token (NULL: zero)
+    float *dh0;       // its gradient (NULL: not written)
     void *dx, *ddelta, *dz;
     float *dA, *dB, *dC, *dD, *ddelta_bias;  // outputs written by the reduction kernel
     // workspace

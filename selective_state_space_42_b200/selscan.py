@@ -68,6 +68,8 @@ SIGNATURES = {
     "selscan_bwd": (_int, [_vp] * 8 + [_int] + [_vp] * 10
                     + [_i64, _i64, _i64, _i64, _int, _vp]),
     "selscan_bwd_workspace_bytes": (_i64, [_i64, _i64, _i64, _i64]),
+    "selscan_bwd_from_state": (_int, [_vp] * 8 + [_int] + [_vp] * 12
+                               + [_i64, _i64, _i64, _i64, _int, _vp, _i64, _vp]),
     "selscan_bwd_workspace": (_int, [_vp] * 8 + [_int] + [_vp] * 10
                               + [_i64, _i64, _i64, _i64, _int, _vp, _i64, _vp]),
     "selscan_state_update_conv": (_int, [_vp, _vp, _vp, _vp, _vp, _int, _vp, _vp, _vp, _vp,
@@ -301,7 +303,8 @@ def _fwd(entry, x, delta, A, B, C, D, z, delta_bias, softplus, y, final_state,
 
 
 def selscan_bwd(x, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=True,
-                dy=None, dfinal_state=None, stream=None, allocate_in_library=False):
+                dy=None, dfinal_state=None, stream=None, allocate_in_library=False,
+                initial_state=None):
     """Gradient of ``selscan_fwd`` for the loss Σ dy·y + Σ
     dfinal_state·final_state. Inputs as for ``selscan_fwd``; dy has y's shape
     and dtype, dfinal_state is [batch, dim, dstate] float32 or None. Returns a
@@ -310,7 +313,9 @@ def selscan_bwd(x, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=Tru
 
     The workspace comes from torch's caching allocator (C ABI
     ``selscan_bwd_workspace``); with ``allocate_in_library`` the library
-    allocates it on the stream instead (C ABI ``selscan_bwd``)."""
+    allocates it on the stream instead (C ABI ``selscan_bwd``). With
+    ``initial_state`` (the forward's, [batch, dim, dstate] float32) the dict
+    also holds its gradient ``dh0`` (C ABI ``selscan_bwd_from_state``)."""
     torch = _torch()
     if x.dim() != 3:
         raise ValueError("x must be [batch, L, dim]")
@@ -347,6 +352,17 @@ def selscan_bwd(x, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=Tru
         batch, L, dim, N, code,
     ]
     lib = load_library()
+    if initial_state is not None:
+        out["dh0"] = torch.empty(batch, dim, N, device=dev, dtype=f32)
+        nbytes = int(lib.selscan_bwd_workspace_bytes(batch, L, dim, N))
+        ws = torch.empty(max(nbytes, 1), device=dev, dtype=torch.uint8)
+        if stream is not None and not isinstance(stream, int):
+            ws.record_stream(stream)
+        fargs = args[:9] + [_ptr(initial_state, "initial_state", (batch, dim, N), f32, dev)] \
+            + args[9:19] + [_ptr(out["dh0"], "dh0")] + args[19:] \
+            + [ws.data_ptr() if nbytes else None, nbytes, _stream_ptr(stream, dev)]
+        _check(lib.selscan_bwd_from_state(*fargs))
+        return out
     if allocate_in_library:
         _check(lib.selscan_bwd(*args, _stream_ptr(stream, dev)))
         return out

@@ -190,3 +190,22 @@ def test_workspace_too_small_is_rejected():
         outs[4].data_ptr(), None, None, None, 1, 20, 40, 16, 1, ws.data_ptr(), need - 1,
         None)
     assert st == -8
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_initial_state_gradient(dtype):
+    """The gradient of the scan started from a given state: every gradient,
+    the initial state's included, against the oracle."""
+    inp, dy, df = _inputs(2, 90, 70, 16, dtype, True, seed=17)
+    g = torch.Generator().manual_seed(18)
+    h0 = torch.randn(2, 70, 16, generator=g)
+    d = {k: (None if v is None else v.to(DEV)) for k, v in inp.items()}
+    got = ss.selscan_bwd(d["x"], d["delta"], d["A"], d["B"], d["C"], d["D"], d["z"],
+                         d["delta_bias"], dy=dy.to(DEV), dfinal_state=df.to(DEV),
+                         initial_state=h0.to(DEV))
+    torch.cuda.synchronize()
+    n = gh.to_np
+    o = oracle.default().bwd(n(inp["x"]), n(inp["delta"]), n(inp["A"]), n(inp["B"]),
+                             n(inp["C"]), n(inp["D"]), n(inp["z"]), n(inp["delta_bias"]),
+                             h0=n(h0), dy=n(dy), dfinal=n(df))
+    _compare_all(got, o, dtype, "from state", names=GRADS + ("dh0",))
