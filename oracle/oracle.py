@@ -97,6 +97,9 @@ class Oracle:
         lib.oracle_causal_conv1d.restype = None
         lib.oracle_causal_conv1d.argtypes = [_dp, _dp, _dp, _dp, _i64, _i64, _i64, _i64,
                                              ctypes.c_int]
+        lib.oracle_causal_conv1d_bwd.restype = None
+        lib.oracle_causal_conv1d_bwd.argtypes = [_dp] * 7 + [_i64, _i64, _i64, _i64,
+                                                             ctypes.c_int]
         lib.oracle_zoh_discretize.restype = None
         lib.oracle_zoh_discretize.argtypes = [ctypes.c_double, _dp, _dp, _dp,
                                               _dp, _i64]
@@ -194,6 +197,23 @@ class Oracle:
         self.lib.oracle_causal_conv1d(_ptr(x_in), _ptr(w), _ptr(cb), _ptr(out), batch, L,
                                       dim, w.shape[1], int(bool(silu)))
         return out
+
+    def causal_conv1d_bwd(self, x_in, w, cb, dxc, silu=True):
+        """Gradient of ``causal_conv1d`` for the loss Σ dxc·x: returns
+        (dx_in, dw, dcb) as float64 arrays (dcb None without a bias)."""
+        x_in = _f64(x_in)
+        batch, L, dim = x_in.shape
+        w = _f64(w)
+        K = w.shape[1]
+        cb = _f64(cb, (dim,))
+        dxc = _f64(dxc, x_in.shape)
+        dx = np.empty_like(x_in)
+        dw = np.empty_like(w)
+        dcb = np.empty(dim) if cb is not None else None
+        self.lib.oracle_causal_conv1d_bwd(_ptr(x_in), _ptr(w), _ptr(cb), _ptr(dxc), _ptr(dx),
+                                          _ptr(dw), _ptr(dcb), batch, L, dim, K,
+                                          int(bool(silu)))
+        return dx, dw, dcb
 
     # -- single-token decode -------------------------------------------------
     def state_update(self, state, x, delta, A, B, C, D=None, z=None,

@@ -456,3 +456,62 @@ void oracle_causal_conv1d(const double *x_in, const double *w, const double *cb,
                 x_out[(b * L + t) * D + d] = silu_flag ? silu(acc) : acc;
             }
 }
+
+/*
+ * Gradient of oracle_causal_conv1d for the loss Σ dxc·x (x the conv output):
+ * with pre = cb + Σ_k w[k]·x_in[t − (K−1) + k] and dpre = dxc·silu'(pre)
+ * (dxc itself when silu_flag is 0),
+ *   dx_in[s]  = Σ_k w[d, k] · dpre[s + (K−1) − k]   (tokens past the end: 0)
+ *   dw[d, k]  = Σ_{b,t} dpre[b, t, d] · x_in[b, t − (K−1) + k, d]
+ *   dcb[d]    = Σ_{b,t} dpre[b, t, d].
+ * dx_in [batch, L, D]; dw [D, K]; dcb [D] (nullable). Outputs overwritten.
+ */
+void oracle_causal_conv1d_bwd(const double *x_in, const double *w, const double *cb,
+                              const double *dxc, double *dx_in, double *dw, double *dcb,
+                              int64_t batch, int64_t L, int64_t D, int64_t K,
+                              int silu_flag)
+{
+    double *dpre = (double *)malloc((size_t)(batch * L * D > 0 ? batch * L * D : 1) *
+                                    sizeof(double));
+    for (int64_t b = 0; b < batch; ++b)
+        for (int64_t t = 0; t < L; ++t)
+            for (int64_t d = 0; d < D; ++d) {
+                double pre = cb ? cb[d] : 0.0;
+                for (int64_t k = 0; k < K; ++k) {
+                    int64_t s = t - (K - 1) + k;
+                    if (s >= 0)
+                        pre += w[d * K + k] * x_in[(b * L + s) * D + d];
+                }
+                int64_t i = (b * L + t) * D + d;
+                dpre[i] = silu_flag ? dxc[i] * silu_grad(pre) : dxc[i];
+            }
+    for (int64_t i = 0; i < D * K; ++i)
+        dw[i] = 0.0;
+    if (dcb)
+        for (int64_t d = 0; d < D; ++d)
+            dcb[d] = 0.0;
+    for (int64_t b = 0; b < batch; ++b)
+        for (int64_t s = 0; s < L; ++s)
+            for (int64_t d = 0; d < D; ++d) {
+                double acc = 0.0;
+                for (int64_t k = 0; k < K; ++k) {
+                    int64_t t = s + (K - 1) - k; /* the output token x_in[s] feeds via w[k] */
+                    if (t < L)
+                        acc += w[d * K + k] * dpre[(b * L + t) * D + d];
+                }
+                dx_in[(b * L + s) * D + d] = acc;
+            }
+    for (int64_t b = 0; b < batch; ++b)
+        for (int64_t t = 0; t < L; ++t)
+            for (int64_t d = 0; d < D; ++d) {
+                double g = dpre[(b * L + t) * D + d];
+                if (dcb)
+                    dcb[d] += g;
+                for (int64_t k = 0; k < K; ++k) {
+                    int64_t s = t - (K - 1) + k;
+                    if (s >= 0)
+                        dw[d * K + k] += g * x_in[(b * L + s) * D + d];
+                }
+            }
+    free(dpre);
+}

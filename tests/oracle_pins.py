@@ -530,11 +530,40 @@ def pin_conv1d_impulse(orc):
     assert np.array_equal(got, want), "impulse response"
 
 
+def pin_conv1d_bwd_finite_differences(orc):
+    """The conv gradient against central differences of the (pinned) conv,
+    for every input, weight and bias element, widths 1 and 4, with and
+    without SiLU."""
+    r = RNG(80)
+    for K, silu in ((4, True), (1, False), (3, True)):
+        x = r.standard_normal((2, 6, 3))
+        w = r.standard_normal((3, K))
+        cb = r.standard_normal(3)
+        dxc = r.standard_normal((2, 6, 3))
+        dx, dw, dcb = orc.causal_conv1d_bwd(x, w, cb, dxc, silu=silu)
+
+        def loss(xx, ww, bb):
+            return float(np.sum(dxc * orc.causal_conv1d(xx, ww, bb, silu=silu)))
+
+        for arr, got, which in ((x, dx, 0), (w, dw, 1), (cb, dcb, 2)):
+            fd = np.zeros_like(arr)
+            for idx in np.ndindex(arr.shape):
+                e = 1e-6 * max(1.0, abs(arr[idx]))
+                ap, am = arr.copy(), arr.copy()
+                ap[idx] += e
+                am[idx] -= e
+                args_p = [x, w, cb]
+                args_m = [x, w, cb]
+                args_p[which], args_m[which] = ap, am
+                fd[idx] = (loss(*args_p) - loss(*args_m)) / (2 * e)
+            assert _rel(got, fd) < 1e-6, f"conv gradient {which} K={K}"
+
+
 ALL_PINS = [
     pin_explicit_sum, pin_single_token, pin_lti_convolution, pin_zoh_matrix,
     pin_euler_vs_zoh, pin_linearity, pin_delta_to_zero, pin_chunked,
     pin_associativity, pin_geometric, pin_decay, pin_cross_entry,
     pin_decode_layout, pin_softplus_and_gate, pin_hand_worked,
     pin_bwd_finite_differences, pin_bwd_homogeneity, pin_bwd_single_token,
-    pin_conv1d_library, pin_conv1d_impulse,
+    pin_conv1d_library, pin_conv1d_impulse, pin_conv1d_bwd_finite_differences,
 ]

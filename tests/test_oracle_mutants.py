@@ -64,6 +64,11 @@ MUTANTS = [
      "x_out[(b * L + t) * D + d] = acc;"),
     ("conv_bias_dropped", "double acc = cb ? cb[d] : 0.0;", "double acc = 0.0;"),
     ("conv_filter_not_reversed", "acc += w[d * K + k] * x_in", "acc += w[d * K + (K - 1 - k)] * x_in"),
+    ("conv_bwd_taps_not_transposed",
+     "int64_t t = s + (K - 1) - k; /* the output token x_in[s] feeds via w[k] */",
+     "int64_t t = s + k; /* the output token x_in[s] feeds via w[k] */"),
+    ("conv_bwd_silu_grad_dropped", "dpre[i] = silu_flag ? dxc[i] * silu_grad(pre) : dxc[i];",
+     "dpre[i] = dxc[i];"),
     ("bwd_gate_on_ds_dropped", "double ds = z ? dy[i] * silu(z[i]) : dy[i];",
      "double ds = dy[i];"),
 ]
