@@ -361,6 +361,36 @@ SELSCAN_API int selscan_bwd_from_state(const void *x, const void *delta, const f
                                        selscan_stream_t stream);
 
 /*
+ * selscan_bwd_conv -- the gradient of selscan_fwd_conv (conv_init NULL: the
+ * conv sees zeros before token 0): as selscan_bwd_from_state with x_in, the
+ * conv arguments, and
+ *   dx_in          [batch, seqlen, dim]  dtype    output: gradient w.r.t. x_in
+ *                                                 (through the conv and SiLU)
+ *   dconv_weight   [dim, conv_width]     float32  output
+ *   dconv_bias     [dim]                 float32  output (NULL: not written)
+ * The workspace (NULL: allocated on the stream) needs
+ * selscan_bwd_conv_workspace_bytes() bytes: besides the scan gradient's it
+ * holds the conv output's gradient (float32 [batch, seqlen, dim]) and conv
+ * partial sums. The conv output is recomputed, never stored.
+ */
+SELSCAN_API int selscan_bwd_conv(const void *x_in, const float *conv_weight,
+                                 const float *conv_bias, int conv_width, const void *delta,
+                                 const float *A, const void *B, const void *C, const float *D,
+                                 const void *z, const float *delta_bias, int softplus_flag,
+                                 const float *initial_state, const void *dy,
+                                 const float *dfinal_state, void *dx_in, void *ddelta,
+                                 float *dA, float *dB, float *dC, float *dD, void *dz,
+                                 float *ddelta_bias, float *dinitial_state,
+                                 float *dconv_weight, float *dconv_bias, int64_t batch,
+                                 int64_t seqlen, int64_t dim, int64_t dstate,
+                                 selscan_dtype_t dtype, void *workspace,
+                                 int64_t workspace_bytes, selscan_stream_t stream);
+
+/* Host-only: workspace bytes selscan_bwd_conv takes (0 for empty or invalid sizes). */
+SELSCAN_API int64_t selscan_bwd_conv_workspace_bytes(int64_t batch, int64_t seqlen,
+                                                     int64_t dim, int64_t dstate);
+
+/*
  * selscan_state_update_conv -- selscan_state_update with the causal conv +
  * SiLU of selscan_fwd_conv in front, for decoding after a selscan_fwd_conv
  * prefill: the token's x is silu(conv_bias + Σ_k conv_weight[d,k] · window),

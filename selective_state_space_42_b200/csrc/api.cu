@@ -334,14 +334,14 @@ cudaError_t fwd_run(FwdPlan *plan, void *ws, cudaStream_t stream) {
 namespace {
 
 struct BwdLayout {
-    size_t ckpt, part, pA, pD, pbias, total;
+    size_t ckpt, part, pA, pD, pbias, dxc, pconv, total;
 };
 
 int64_t ceil_div64(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
 
-BwdLayout bwd_layout(int64_t batch, int64_t seqlen, int64_t dim) {
+BwdLayout bwd_layout(int64_t batch, int64_t seqlen, int64_t dim, bool conv = false) {
     const int64_t K = ceil_div64(seqlen, selscan::bwd_tile_tokens());
     const int64_t ct = ceil_div64(dim, selscan::bwd_tile_channels());
     BwdLayout l;
@@ -356,6 +356,15 @@ BwdLayout bwd_layout(int64_t batch, int64_t seqlen, int64_t dim) {
     off = align256(off + (size_t)(batch * dim) * sizeof(float));
     l.pbias = off;
     off = align256(off + (size_t)(batch * dim) * sizeof(float));
+    l.dxc = l.pconv = off;
+    if (conv) {  // the conv output's gradient and the conv-gradient partials
+        const int64_t ctt = ceil_div64(seqlen, selscan::bwd_conv_tile_tokens());
+        l.dxc = off;
+        off = align256(off + (size_t)(batch * seqlen * dim) * sizeof(float));
+        l.pconv = off;
+        off = align256(off + (size_t)(batch * ctt * dim) * (selscan::kMaxConv + 1) *
+                                 sizeof(float));
+    }
     l.total = off;
     return l;
 }
@@ -523,7 +532,8 @@ int bwd_entry(const void *x, const void *delta, const float *A, const void *B, c
               const void *dy, const float *dfinal_state, void *dx, void *ddelta, float *dA,
               float *dB, float *dC, float *dD, void *dz, float *ddelta_bias, int64_t batch,
               int64_t seqlen, int64_t dim, int64_t dstate, selscan_dtype_t dtype,
-              const float *h0, float *dh0, void *workspace, int64_t workspace_bytes,
+              const float *h0, float *dh0, const float *conv_w,
+              const float *conv_b, int conv_width, float *dconv_w, float *dconv_b, void *workspace, int64_t workspace_bytes,
               bool allocate,
               selscan_stream_t stream_) {
     cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
@@ -546,18 +556,24 @@ int bwd_entry(const void *x, const void *delta, const float *A, const void *B, c
         misaligned(D, 4) || misaligned(delta_bias, 4) || misaligned(dfinal_state, 4) ||
         misaligned(dA, 4) || misaligned(dB, 4) || misaligned(dC, 4) || misaligned(dD, 4) ||
         misaligned(ddelta_bias, 4) || misaligned(workspace, 256) || misaligned(h0, 4) ||
-        misaligned(dh0, 4))
+        misaligned(dh0, 4) || misaligned(conv_w, 4) || misaligned(conv_b, 4) ||
+        misaligned(dconv_w, 4) || misaligned(dconv_b, 4))
         return SELSCAN_ERR_MISALIGNED;
+    if (conv_width < 0 || conv_width > selscan::kMaxConv) return SELSCAN_ERR_BAD_DIM;
+    if (conv_width > 0 && dim > 0 && (!conv_w || !dconv_w)) return SELSCAN_ERR_NULL_ARG;
     const size_t nx = (size_t)(batch * seqlen * dim) * es;
     const size_t nbc = (size_t)(batch * seqlen * dstate) * es;
     const size_t nbcf = (size_t)(batch * seqlen * dstate) * 4;
     const size_t na = (size_t)(dim * dstate) * 4, nd = (size_t)dim * 4;
     const size_t ns = (size_t)(batch * dim * dstate) * 4;
+    const size_t ncw = (size_t)(dim * conv_width) * 4;
     const Span outs[] = {{dx, nx}, {ddelta, nx}, {dz, z ? nx : 0}, {dA, na}, {dB, nbcf},
-                         {dC, nbcf}, {dD, nd}, {ddelta_bias, nd}, {dh0, ns}};
+                         {dC, nbcf}, {dD, nd}, {ddelta_bias, nd}, {dh0, ns},
+                         {dconv_w, ncw}, {dconv_b, conv_width > 0 ? nd : 0}};
     const Span ins[] = {{x, nx}, {delta, nx}, {z, nx}, {dy, nx}, {B, nbc}, {C, nbc},
-                        {A, na}, {D, nd}, {delta_bias, nd}, {dfinal_state, ns}, {h0, ns}};
-    if (any_overlap(outs, 9, ins, 11)) return SELSCAN_ERR_ALIAS;
+                        {A, na}, {D, nd}, {delta_bias, nd}, {dfinal_state, ns}, {h0, ns},
+                        {conv_w, ncw}, {conv_b, conv_width > 0 ? nd : 0}};
+    if (any_overlap(outs, 11, ins, 13)) return SELSCAN_ERR_ALIAS;
 
     if (!has_tokens) {
         // no token reaches the loss through a channel: the float32 gradients are 0
@@ -569,6 +585,10 @@ int bwd_entry(const void *x, const void *delta, const float *A, const void *B, c
         if (e == cudaSuccess && dim > 0 && ddelta_bias)
             e = cudaMemsetAsync(ddelta_bias, 0, nd, stream);
         // no token: the final state is the initial one
+        if (e == cudaSuccess && conv_width > 0 && dim > 0)
+            e = cudaMemsetAsync(dconv_w, 0, ncw, stream);
+        if (e == cudaSuccess && conv_width > 0 && dconv_b && dim > 0)
+            e = cudaMemsetAsync(dconv_b, 0, nd, stream);
         if (e == cudaSuccess && dh0 && ns > 0)
             e = dfinal_state ? cudaMemcpyAsync(dh0, dfinal_state, ns, cudaMemcpyDeviceToDevice,
                                                stream)
@@ -576,18 +596,24 @@ int bwd_entry(const void *x, const void *delta, const float *A, const void *B, c
         return e == cudaSuccess ? SELSCAN_OK : selscan::cuda_fail(e);
     }
 
-    const BwdLayout l = bwd_layout(batch, seqlen, dim);
+    const BwdLayout l = bwd_layout(batch, seqlen, dim, conv_width > 0);
     if (!allocate) {
         if (!workspace) return SELSCAN_ERR_NULL_ARG;
         if (workspace_bytes < (int64_t)l.total) return SELSCAN_ERR_WORKSPACE;
         const Span wsp[] = {{workspace, l.total}};
-        if (any_overlap(wsp, 1, outs, 9) || any_overlap(wsp, 1, ins, 11))
+        if (any_overlap(wsp, 1, outs, 11) || any_overlap(wsp, 1, ins, 13))
             return SELSCAN_ERR_ALIAS;
     }
     selscan::BwdParams p{};
     p.x = x; p.delta = delta; p.z = z; p.B = B; p.C = C; p.dy = dy;
     p.A = A; p.Dskip = D; p.delta_bias = delta_bias; p.dfinal = dfinal_state;
     p.h0 = h0; p.dh0 = dh0;
+    p.conv_width = conv_width;
+    p.conv_w = conv_width > 0 ? conv_w : nullptr;
+    p.conv_b = conv_width > 0 ? conv_b : nullptr;
+    p.dconv_w = conv_width > 0 ? dconv_w : nullptr;
+    p.dconv_b = conv_width > 0 ? dconv_b : nullptr;
+    p.conv_tiles = (int)ceil_div64(seqlen, selscan::bwd_conv_tile_tokens());
     p.dx = dx; p.ddelta = ddelta; p.dz = dz;
     p.dA = dA; p.dB = dB; p.dC = dC; p.dD = dD; p.ddelta_bias = ddelta_bias;
     p.batch = batch; p.seqlen = seqlen; p.dim = dim; p.dstate = (int)dstate;
@@ -608,6 +634,8 @@ int bwd_entry(const void *x, const void *delta, const float *A, const void *B, c
     p.pA = reinterpret_cast<float *>(w + l.pA);
     p.pD = reinterpret_cast<float *>(w + l.pD);
     p.pbias = reinterpret_cast<float *>(w + l.pbias);
+    p.dxc = conv_width > 0 ? reinterpret_cast<float *>(w + l.dxc) : nullptr;
+    p.pconv = conv_width > 0 ? reinterpret_cast<float *>(w + l.pconv) : nullptr;
     e = selscan::launch_scan_bwd(p, dtype == SELSCAN_BF16, stream);
     if (allocate) {
         cudaError_t ef = cudaFreeAsync(ws, stream);
@@ -628,7 +656,8 @@ int selscan_bwd(const void *x, const void *delta, const float *A, const void *B,
                 selscan_stream_t stream) {
     return bwd_entry(x, delta, A, B, C, D, z, delta_bias, softplus_flag, dy, dfinal_state, dx,
                      ddelta, dA, dB, dC, dD, dz, ddelta_bias, batch, seqlen, dim, dstate, dtype,
-                     nullptr, nullptr, nullptr, 0, true, stream);
+                     nullptr, nullptr, nullptr, nullptr, 0, nullptr, nullptr, nullptr, 0, true,
+                     stream);
 }
 
 int selscan_bwd_workspace(const void *x, const void *delta, const float *A, const void *B,
@@ -641,7 +670,8 @@ int selscan_bwd_workspace(const void *x, const void *delta, const float *A, cons
                           selscan_stream_t stream) {
     return bwd_entry(x, delta, A, B, C, D, z, delta_bias, softplus_flag, dy, dfinal_state, dx,
                      ddelta, dA, dB, dC, dD, dz, ddelta_bias, batch, seqlen, dim, dstate, dtype,
-                     nullptr, nullptr, workspace, workspace_bytes, false, stream);
+                     nullptr, nullptr, nullptr, nullptr, 0, nullptr, nullptr, workspace,
+                     workspace_bytes, false, stream);
 }
 
 int selscan_bwd_from_state(const void *x, const void *delta, const float *A, const void *B,
@@ -655,8 +685,35 @@ int selscan_bwd_from_state(const void *x, const void *delta, const float *A, con
                            int64_t workspace_bytes, selscan_stream_t stream) {
     return bwd_entry(x, delta, A, B, C, D, z, delta_bias, softplus_flag, dy, dfinal_state, dx,
                      ddelta, dA, dB, dC, dD, dz, ddelta_bias, batch, seqlen, dim, dstate, dtype,
-                     initial_state, dinitial_state, workspace, workspace_bytes,
+                     initial_state, dinitial_state, nullptr, nullptr, 0, nullptr, nullptr,
+                     workspace, workspace_bytes, workspace == nullptr, stream);
+}
+
+int selscan_bwd_conv(const void *x_in, const float *conv_weight, const float *conv_bias,
+                     int conv_width, const void *delta, const float *A, const void *B,
+                     const void *C, const float *D, const void *z, const float *delta_bias,
+                     int softplus_flag, const float *initial_state, const void *dy,
+                     const float *dfinal_state, void *dx_in, void *ddelta, float *dA,
+                     float *dB, float *dC, float *dD, void *dz, float *ddelta_bias,
+                     float *dinitial_state, float *dconv_weight, float *dconv_bias,
+                     int64_t batch, int64_t seqlen, int64_t dim, int64_t dstate,
+                     selscan_dtype_t dtype, void *workspace, int64_t workspace_bytes,
+                     selscan_stream_t stream) {
+    if (conv_width < 1) return SELSCAN_ERR_BAD_DIM;
+    return bwd_entry(x_in, delta, A, B, C, D, z, delta_bias, softplus_flag, dy, dfinal_state,
+                     dx_in, ddelta, dA, dB, dC, dD, dz, ddelta_bias, batch, seqlen, dim, dstate,
+                     dtype, initial_state, dinitial_state, conv_weight, conv_bias, conv_width,
+                     dconv_weight, dconv_bias, workspace, workspace_bytes,
                      workspace == nullptr, stream);
+}
+
+int64_t selscan_bwd_conv_workspace_bytes(int64_t batch, int64_t seqlen, int64_t dim,
+                                         int64_t dstate) {
+    if (batch <= 0 || seqlen <= 0 || dim <= 0 || dstate < 1 || dstate > selscan::kMaxN)
+        return 0;
+    if (!mul_le(batch, seqlen, kMaxElems) || !mul_le(batch * seqlen, dim, kMaxElems))
+        return 0;
+    return (int64_t)bwd_layout(batch, seqlen, dim, true).total;
 }
 
 int selscan_device_status(int *status, int clear) {

@@ -61,12 +61,22 @@ struct BwdSmem {
 // Raw per-token inputs of one tile for this lane's channel.
 template <typename T> struct Raw {
     T x[kSeg], dl[kSeg], z[kSeg], dy[kSeg];
+    T xh[kMaxConv - 1];  // conv: the inputs of the kMaxConv − 1 tokens before the tile
 };
 
-template <typename T, bool kGate, bool kBwd>
+template <typename T, bool kGate, bool kBwd, bool kConv = false>
 __device__ __forceinline__ void load_raw(Raw<T> &r, const BwdParams &p, long long b,
                                          long long t0, long long d, bool active) {
     const T zero = from_f32<T>(0.0f);
+    if (kConv) {
+#pragma unroll
+        for (int k = 0; k < kMaxConv - 1; ++k) {
+            const long long tok = t0 - (kMaxConv - 1) + k;
+            const bool ok = active && tok >= 0 && tok < p.seqlen;
+            r.xh[k] = ok ? __ldg(static_cast<const T *>(p.x) + (b * p.seqlen + tok) * p.dim + d)
+                         : zero;
+        }
+    }
 #pragma unroll
     for (int t = 0; t < kSeg; ++t) {
         const long long tok = t0 + t;
@@ -134,7 +144,7 @@ __device__ __forceinline__ void ld_quad(const float *base, int q, float2 &lo, fl
 }
 __device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
 
-template <typename T, bool kGate, bool kSoftplus, bool kStruct>
+template <typename T, bool kGate, bool kSoftplus, bool kStruct, bool kConv>
 __device__ __forceinline__ void bwd_body(BwdSmem &S, const BwdParams &p) {
     const int lane = threadIdx.x;
     const long long b = blockIdx.y;
@@ -155,6 +165,12 @@ __device__ __forceinline__ void bwd_body(BwdSmem &S, const BwdParams &p) {
     const float bias = (active && p.delta_bias) ? p.delta_bias[dd] : 0.0f;
     const float Dv = (active && p.Dskip) ? p.Dskip[dd] : 0.0f;
     const int K = p.ktiles;
+    // conv taps of this channel (the conv output is the scan's x)
+    float cw[kMaxConv] = {0.f, 0.f, 0.f, 0.f}, cbias = 0.0f;
+    if (kConv && active) {
+        load_conv_taps(p.conv_w, p.conv_width, dd, cw);
+        cbias = p.conv_b ? p.conv_b[dd] : 0.0f;
+    }
     float4 *ck = reinterpret_cast<float4 *>(p.ckpt) + ((b * K) * p.dim + dd) * 4;
     const long long ck_stride = p.dim * 4;  // float4s between consecutive tiles
 
@@ -171,6 +187,7 @@ __device__ __forceinline__ void bwd_body(BwdSmem &S, const BwdParams &p) {
         float bv[4], cv[4];
         load_raw<T, kGate, false>(cur, p, b, 0, dd, active);
         load_bc<T>(bv, cv, p, b, 0, lane, false);
+        float xw[kMaxConv - 1] = {0.f, 0.f, 0.f};  // conv window, zero before token 0
         for (int k = 0; k < K; ++k) {
             const long long t0 = (long long)k * kSeg;
             if (active) {
@@ -191,7 +208,9 @@ __device__ __forceinline__ void bwd_body(BwdSmem &S, const BwdParams &p) {
                 const float v = to_f32(cur.dl[t]) + bias;
                 const bool live = active && t0 + t < p.seqlen;
                 const float dt = live ? (kSoftplus ? softplus_f32(v) : v) : 0.0f;
-                const float2 u2 = dup2(dt * to_f32(cur.x[t]));
+                float xv = to_f32(cur.x[t]);
+                if (kConv) xv = conv_step(cw, cbias, xw, xv);
+                const float2 u2 = dup2(dt * xv);
                 float2 a[kPairs];
                 decay16<kStruct>(dt, ex2_approx(dt * A0l), Al, a);
 #pragma unroll
@@ -224,7 +243,7 @@ __device__ __forceinline__ void bwd_body(BwdSmem &S, const BwdParams &p) {
     float4 hc[4], hn[4];
     {
         const long long t0 = (long long)(K - 1) * kSeg;
-        load_raw<T, kGate, true>(cur, p, b, t0, dd, active);
+        load_raw<T, kGate, true, kConv>(cur, p, b, t0, dd, active);
         load_bc<T>(bv, cv, p, b, t0, lane, true);
 #pragma unroll
         for (int j = 0; j < 4; ++j)
@@ -235,7 +254,7 @@ __device__ __forceinline__ void bwd_body(BwdSmem &S, const BwdParams &p) {
         __syncwarp();
         store_bc(S, bv, cv, lane);
         if (k > 0) {
-            load_raw<T, kGate, true>(nxt, p, b, t0 - kSeg, dd, active);
+            load_raw<T, kGate, true, kConv>(nxt, p, b, t0 - kSeg, dd, active);
             load_bc<T>(bv, cv, p, b, t0 - kSeg, lane, true);
 #pragma unroll
             for (int j = 0; j < 4; ++j)
@@ -244,6 +263,9 @@ __device__ __forceinline__ void bwd_body(BwdSmem &S, const BwdParams &p) {
         __syncwarp();
 
         // recompute the tile's states and per-token scalars
+        float xw[kMaxConv - 1];
+#pragma unroll
+        for (int k = 0; k < kMaxConv - 1; ++k) xw[k] = kConv ? to_f32(cur.xh[k]) : 0.0f;
         float2 h[kPairs];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
@@ -254,7 +276,8 @@ __device__ __forceinline__ void bwd_body(BwdSmem &S, const BwdParams &p) {
 #pragma unroll
         for (int t = 0; t < kSeg; ++t) {
             const bool live = active && t0 + t < p.seqlen;
-            const float xv = to_f32(cur.x[t]);
+            float xv = to_f32(cur.x[t]);
+            if (kConv) xv = conv_step(cw, cbias, xw, xv);
             const float v = to_f32(cur.dl[t]) + bias;
             const float dt = live ? (kSoftplus ? softplus_f32(v) : v) : 0.0f;
             const float u = dt * xv;
@@ -341,7 +364,11 @@ __device__ __forceinline__ void bwd_body(BwdSmem &S, const BwdParams &p) {
                 const long long i = (b * p.seqlen + tok) * p.dim + d;
                 const float ddt = fmaf(du, so.x, qp);
                 const float dv = ddt * so.z;
-                static_cast<T *>(p.dx)[i] = from_f32<T>(fmaf(du, sc.x, sc.z * Dv));
+                const float dxv = fmaf(du, sc.x, sc.z * Dv);
+                if (kConv)
+                    p.dxc[i] = dxv;  // the conv's input gradient comes from conv_bwd_kernel
+                else
+                    static_cast<T *>(p.dx)[i] = from_f32<T>(dxv);
                 static_cast<T *>(p.ddelta)[i] = from_f32<T>(dv);
                 if (kGate) static_cast<T *>(p.dz)[i] = from_f32<T>(so.w * so.y);
                 accD = fmaf(sc.z, so.x, accD);
@@ -395,7 +422,7 @@ __device__ __forceinline__ void bwd_body(BwdSmem &S, const BwdParams &p) {
 
 // A[d, n] == (n+1)·A[d, 0] for every state of every channel of the warp
 // selects the power-ladder decay (the A = −(1..N) initialisation).
-template <typename T, bool kGate, bool kSoftplus>
+template <typename T, bool kGate, bool kSoftplus, bool kConv>
 __global__ void __launch_bounds__(kChains, 6) scan_bwd_kernel(const BwdParams p) {
     __shared__ BwdSmem S;
     const long long d = (long long)blockIdx.x * kChains + threadIdx.x;
@@ -406,9 +433,9 @@ __global__ void __launch_bounds__(kChains, 6) scan_bwd_kernel(const BwdParams p)
             if (p.A[d * p.dstate + n] != (float)(n + 1) * a0) ok = false;
     }
     if (__all_sync(0xffffffffu, ok))
-        bwd_body<T, kGate, kSoftplus, true>(S, p);
+        bwd_body<T, kGate, kSoftplus, true, kConv>(S, p);
     else
-        bwd_body<T, kGate, kSoftplus, false>(S, p);
+        bwd_body<T, kGate, kSoftplus, false, kConv>(S, p);
 }
 
 // dB[b, t, n] and dC[b, t, n]: sums of the channel-tile partials.
@@ -451,13 +478,111 @@ __global__ void bwd_reduce_params_kernel(const BwdParams p) {
     }
 }
 
-template <typename T, bool kGate>
-cudaError_t launch_gate(const BwdParams &p, cudaStream_t stream) {
+// Gradient of the causal conv + SiLU in front of the scan, from the
+// gradient of its output (dxc, written by scan_bwd_kernel): with
+// pre[t] = cb + Σ_k cw[k]·x_in[t − 3 + k] (taps right-aligned in 4 slots) and
+// dpre[t] = dxc[t]·silu'(pre[t]),
+//   dx_in[s] = Σ_k cw[k]·dpre[s + 3 − k],  dw[k] += dpre[t]·x_in[t − 3 + k],
+//   db += dpre[t].
+// A thread walks one channel over kConvTile tokens (3 more at the end for
+// the dx_in of its last tokens), sliding windows of x_in and dpre in
+// registers; dw and db go to a per-(batch row, token tile) partial buffer.
+constexpr int kConvTile = 512;
+constexpr int kConvThreads = 128;
+
+template <typename T>
+__global__ void __launch_bounds__(kConvThreads) conv_bwd_kernel(const BwdParams p) {
+    const long long d = (long long)blockIdx.x * kConvThreads + threadIdx.x;
+    const int tile = blockIdx.y;
+    const long long b = blockIdx.z;
+    if (d >= p.dim) return;
+    const long long ta = (long long)tile * kConvTile;
+    const long long tb = min(ta + kConvTile, p.seqlen);
+    float cw[kMaxConv];
+    load_conv_taps(p.conv_w, p.conv_width, d, cw);
+    const float cb = p.conv_b ? p.conv_b[d] : 0.0f;
+    const T *xp = static_cast<const T *>(p.x);
+    const long long row = b * p.seqlen;
+    float xw[kMaxConv - 1];
+#pragma unroll
+    for (int k = 0; k < kMaxConv - 1; ++k) {
+        const long long t = ta - (kMaxConv - 1) + k;
+        xw[k] = t >= 0 ? ldg_f32(xp + (row + t) * p.dim + d) : 0.0f;
+    }
+    float dq[kMaxConv] = {0.f, 0.f, 0.f, 0.f};  // dpre of the last 4 tokens, oldest first
+    float dw[kMaxConv] = {0.f, 0.f, 0.f, 0.f}, db = 0.0f;
+    T *dxp = static_cast<T *>(p.dx);
+    for (long long t = ta; t < tb + (kMaxConv - 1); ++t) {
+        float g = 0.0f;
+        if (t < p.seqlen) {
+            const long long i = (row + t) * p.dim + d;
+            const float xi = ldg_f32(xp + i);
+            const float pre =
+                fmaf(cw[0], xw[0], fmaf(cw[1], xw[1], fmaf(cw[2], xw[2], fmaf(cw[3], xi, cb))));
+            const float sg = sigmoid_f32(pre);
+            g = p.dxc[i] * sg * fmaf(pre, 1.0f - sg, 1.0f);
+            if (t < tb) {
+                dw[0] = fmaf(g, xw[0], dw[0]);
+                dw[1] = fmaf(g, xw[1], dw[1]);
+                dw[2] = fmaf(g, xw[2], dw[2]);
+                dw[3] = fmaf(g, xi, dw[3]);
+                db += g;
+            }
+            xw[0] = xw[1];
+            xw[1] = xw[2];
+            xw[2] = xi;
+        }
+        dq[0] = dq[1];
+        dq[1] = dq[2];
+        dq[2] = dq[3];
+        dq[3] = g;
+        const long long s = t - (kMaxConv - 1);
+        if (s >= ta && s < tb)
+            dxp[(row + s) * p.dim + d] = from_f32<T>(
+                fmaf(cw[3], dq[0], fmaf(cw[2], dq[1], fmaf(cw[1], dq[2], cw[0] * dq[3]))));
+    }
+    float *pc = p.pconv + ((b * p.conv_tiles + tile) * p.dim + d) * (kMaxConv + 1);
+#pragma unroll
+    for (int k = 0; k < kMaxConv; ++k) pc[k] = dw[k];
+    pc[kMaxConv] = db;
+}
+
+// dconv_w[d, j] and dconv_b[d]: sums of the partials over batch rows and tiles.
+__global__ void conv_reduce_kernel(const BwdParams p) {
+    const long long d = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (d >= p.dim) return;
+    float acc[kMaxConv + 1] = {0.f, 0.f, 0.f, 0.f, 0.f};
+    for (long long r = 0; r < p.batch * p.conv_tiles; ++r) {
+        const float *pc = p.pconv + (r * p.dim + d) * (kMaxConv + 1);
+#pragma unroll
+        for (int k = 0; k <= kMaxConv; ++k) acc[k] += pc[k];
+    }
+    for (int j = 0; j < p.conv_width; ++j)
+        p.dconv_w[d * p.conv_width + j] = acc[j + kMaxConv - p.conv_width];
+    if (p.dconv_b) p.dconv_b[d] = acc[kMaxConv];
+}
+
+template <typename T, bool kGate, bool kConv>
+cudaError_t launch_conv(const BwdParams &p, cudaStream_t stream) {
     const dim3 grid((unsigned)p.ctiles, (unsigned)p.batch);
     if (p.softplus)
-        scan_bwd_kernel<T, kGate, true><<<grid, kChains, 0, stream>>>(p);
+        scan_bwd_kernel<T, kGate, true, kConv><<<grid, kChains, 0, stream>>>(p);
     else
-        scan_bwd_kernel<T, kGate, false><<<grid, kChains, 0, stream>>>(p);
+        scan_bwd_kernel<T, kGate, false, kConv><<<grid, kChains, 0, stream>>>(p);
+    return cudaGetLastError();
+}
+
+template <typename T, bool kGate>
+cudaError_t launch_gate(const BwdParams &p, cudaStream_t stream) {
+    cudaError_t e = p.conv_width > 0 ? launch_conv<T, kGate, true>(p, stream)
+                                     : launch_conv<T, kGate, false>(p, stream);
+    if (e != cudaSuccess || p.conv_width == 0) return e;
+    const dim3 grid((unsigned)((p.dim + kConvThreads - 1) / kConvThreads),
+                    (unsigned)p.conv_tiles, (unsigned)p.batch);
+    conv_bwd_kernel<T><<<grid, kConvThreads, 0, stream>>>(p);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    conv_reduce_kernel<<<(unsigned)((p.dim + 255) / 256), 256, 0, stream>>>(p);
     return cudaGetLastError();
 }
 
@@ -465,6 +590,7 @@ cudaError_t launch_gate(const BwdParams &p, cudaStream_t stream) {
 
 int bwd_tile_tokens() { return kSeg; }
 int bwd_tile_channels() { return kChains; }
+int bwd_conv_tile_tokens() { return kConvTile; }
 
 cudaError_t launch_scan_bwd(const BwdParams &p, bool bf16, cudaStream_t stream) {
     cudaError_t e;

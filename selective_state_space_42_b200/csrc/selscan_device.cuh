@@ -148,6 +148,12 @@ struct BwdParams {
     const float *A, *Dskip, *delta_bias, *dfinal;
     const float *h0;  // state before the first token (NULL: zero)
     float *dh0;       // its gradient (NULL: not written)
+    const float *conv_w, *conv_b;  // causal conv in front (conv_width > 0)
+    int conv_width;
+    float *dxc;       // with the conv: gradient of the conv output, [batch][seqlen][dim]
+    float *dconv_w, *dconv_b;      // conv gradients (outputs; dconv_b nullable)
+    float *pconv;     // [batch][conv tiles][dim][kMaxConv + 1] conv-gradient partials
+    int conv_tiles;   // token tiles of the conv-gradient kernel
     void *dx, *ddelta, *dz;
     float *dA, *dB, *dC, *dD, *ddelta_bias;  // outputs written by the reduction kernel
     // workspace
@@ -208,6 +214,7 @@ cudaError_t launch_scan_wide(const ScanParams &p, bool bf16, cudaStream_t stream
 int wide_max_dstate();
 int bwd_tile_tokens();
 int bwd_tile_channels();
+int bwd_conv_tile_tokens();
 cudaError_t launch_state_update(const StepParams &p, bool bf16, cudaStream_t stream);
 int scan_channels_per_cta();
 int scan_tile_tokens();

@@ -68,6 +68,9 @@ SIGNATURES = {
     "selscan_bwd": (_int, [_vp] * 8 + [_int] + [_vp] * 10
                     + [_i64, _i64, _i64, _i64, _int, _vp]),
     "selscan_bwd_workspace_bytes": (_i64, [_i64, _i64, _i64, _i64]),
+    "selscan_bwd_conv": (_int, [_vp, _vp, _vp, _int] + [_vp] * 7 + [_int] + [_vp] * 14
+                         + [_i64, _i64, _i64, _i64, _int, _vp, _i64, _vp]),
+    "selscan_bwd_conv_workspace_bytes": (_i64, [_i64, _i64, _i64, _i64]),
     "selscan_bwd_from_state": (_int, [_vp] * 8 + [_int] + [_vp] * 12
                                + [_i64, _i64, _i64, _i64, _int, _vp, _i64, _vp]),
     "selscan_bwd_workspace": (_int, [_vp] * 8 + [_int] + [_vp] * 10
@@ -304,7 +307,7 @@ def _fwd(entry, x, delta, A, B, C, D, z, delta_bias, softplus, y, final_state,
 
 def selscan_bwd(x, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=True,
                 dy=None, dfinal_state=None, stream=None, allocate_in_library=False,
-                initial_state=None):
+                initial_state=None, conv_weight=None, conv_bias=None):
     """Gradient of ``selscan_fwd`` for the loss Σ dy·y + Σ
     dfinal_state·final_state. Inputs as for ``selscan_fwd``; dy has y's shape
     and dtype, dfinal_state is [batch, dim, dstate] float32 or None. Returns a
@@ -315,7 +318,11 @@ def selscan_bwd(x, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=Tru
     ``selscan_bwd_workspace``); with ``allocate_in_library`` the library
     allocates it on the stream instead (C ABI ``selscan_bwd``). With
     ``initial_state`` (the forward's, [batch, dim, dstate] float32) the dict
-    also holds its gradient ``dh0`` (C ABI ``selscan_bwd_from_state``)."""
+    also holds its gradient ``dh0`` (C ABI ``selscan_bwd_from_state``). With
+    ``conv_weight`` [dim, K] (and ``conv_bias``), x is the input of the causal
+    conv + SiLU in front of the scan (C ABI ``selscan_bwd_conv``): dx is then
+    the gradient w.r.t. that input, and the dict also holds ``dconv_weight``
+    and ``dconv_bias``."""
     torch = _torch()
     if x.dim() != 3:
         raise ValueError("x must be [batch, L, dim]")
@@ -352,6 +359,32 @@ def selscan_bwd(x, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=Tru
         batch, L, dim, N, code,
     ]
     lib = load_library()
+    if conv_weight is not None:
+        if conv_weight.dim() != 2 or conv_weight.shape[0] != dim:
+            raise ValueError("conv_weight must be [dim, K]")
+        K = int(conv_weight.shape[1])
+        if initial_state is not None:
+            out["dh0"] = torch.empty(batch, dim, N, device=dev, dtype=f32)
+        out["dconv_weight"] = torch.empty(dim, K, device=dev, dtype=f32)
+        out["dconv_bias"] = torch.empty(dim, device=dev, dtype=f32) if conv_bias is not None \
+            else None
+        nbytes = int(lib.selscan_bwd_conv_workspace_bytes(batch, L, dim, N))
+        ws = torch.empty(max(nbytes, 1), device=dev, dtype=torch.uint8)
+        if stream is not None and not isinstance(stream, int):
+            ws.record_stream(stream)
+        cargs = ([args[0], _ptr(conv_weight, "conv_weight", (dim, K), f32, dev),
+                  _ptr(conv_bias, "conv_bias", (dim,), f32, dev, required=False), K]
+                 + args[1:9]
+                 + [_ptr(initial_state, "initial_state", (batch, dim, N), f32, dev,
+                         required=False)]
+                 + args[9:19]
+                 + [_ptr(out.get("dh0"), "dh0", required=False),
+                    _ptr(out["dconv_weight"], "dconv_weight"),
+                    _ptr(out["dconv_bias"], "dconv_bias", required=False)]
+                 + args[19:]
+                 + [ws.data_ptr() if nbytes else None, nbytes, _stream_ptr(stream, dev)])
+        _check(lib.selscan_bwd_conv(*cargs))
+        return out
     if initial_state is not None:
         out["dh0"] = torch.empty(batch, dim, N, device=dev, dtype=f32)
         nbytes = int(lib.selscan_bwd_workspace_bytes(batch, L, dim, N))

@@ -209,3 +209,33 @@ def test_initial_state_gradient(dtype):
                              n(inp["C"]), n(inp["D"]), n(inp["z"]), n(inp["delta_bias"]),
                              h0=n(h0), dy=n(dy), dfinal=n(df))
     _compare_all(got, o, dtype, "from state", names=GRADS + ("dh0",))
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("K", [4, 2])
+@pytest.mark.parametrize("shape", [(2, 90, 70), (1, 1100, 40)], ids=str)
+def test_conv_gradient(dtype, K, shape):
+    """The gradient through the causal conv + SiLU in front of the scan
+    (selscan_bwd_conv) against the oracle's scan gradient at the conv output
+    followed by its conv gradient."""
+    batch, L, dim = shape
+    inp, dy, df = _inputs(batch, L, dim, 16, dtype, True, seed=19 + K)
+    g = torch.Generator().manual_seed(20 + K)
+    cw = torch.randn(dim, K, generator=g) * 0.5
+    cb = torch.randn(dim, generator=g) * 0.1
+    h0 = torch.randn(batch, dim, 16, generator=g)
+    d = {k: (None if v is None else v.to(DEV)) for k, v in inp.items()}
+    got = ss.selscan_bwd(d["x"], d["delta"], d["A"], d["B"], d["C"], d["D"], d["z"],
+                         d["delta_bias"], dy=dy.to(DEV), dfinal_state=df.to(DEV),
+                         initial_state=h0.to(DEV), conv_weight=cw.to(DEV),
+                         conv_bias=cb.to(DEV))
+    torch.cuda.synchronize()
+    n = gh.to_np
+    orc = oracle.default()
+    xc = orc.causal_conv1d(n(inp["x"]), n(cw), n(cb))
+    o = orc.bwd(xc, n(inp["delta"]), n(inp["A"]), n(inp["B"]), n(inp["C"]), n(inp["D"]),
+                n(inp["z"]), n(inp["delta_bias"]), h0=n(h0), dy=n(dy), dfinal=n(df))
+    dx_in, dw, dcb = orc.causal_conv1d_bwd(n(inp["x"]), n(cw), n(cb), o["dx"])
+    o.update(dx=dx_in, dconv_weight=dw, dconv_bias=dcb)
+    _compare_all(got, o, dtype, f"conv K={K}",
+                 names=GRADS + ("dh0", "dconv_weight", "dconv_bias"))
