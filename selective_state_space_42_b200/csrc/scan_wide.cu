@@ -32,8 +32,11 @@ __global__ void __launch_bounds__(kThreads)
 scan_wide_kernel(const ScanParams p) {
     constexpr int kWidth = kLanes * kSlice;  // padded d_state
     constexpr int kChainsPerCta = kThreads / kLanes;
-    __shared__ float sB[kTileT][kWidth];
-    __shared__ float sC[kTileT][kWidth];
+    // B and C rows as [slice][16 + 4 pad]: a lane reads its 16 states as four
+    // 16-byte loads, and the pad puts the 8 slices of a row on distinct banks
+    constexpr int kRow = kSlice + 4;
+    __shared__ __align__(16) float sB[kTileT][kLanes][kRow];
+    __shared__ __align__(16) float sC[kTileT][kLanes][kRow];
     __shared__ float3 sX[kTileT][kChainsPerCta];  // x, delta, z of the tile per chain
     const int tid = threadIdx.x;
     const int slice = tid % kLanes;
@@ -95,29 +98,54 @@ scan_wide_kernel(const ScanParams p) {
     const T *Bp = static_cast<const T *>(p.B);
     const T *Cp = static_cast<const T *>(p.C);
     T *yp = static_cast<T *>(p.y);
+    // The next tile's B, C, x, delta, z are loaded into registers while the
+    // current one is computed, then staged into shared memory.
+    constexpr int kBCPer = kTileT * kWidth / kThreads;          // B (and C) values per thread
+    constexpr int kXPer = kTileT * kChainsPerCta / kThreads;    // (x, delta, z) per thread
+    float pb[kBCPer], pc[kBCPer];
+    float3 px[kXPer];
+    auto fetch = [&](int64_t t0) {
+#pragma unroll
+        for (int i = 0; i < kBCPer; ++i) {
+            const int e = tid + i * kThreads;
+            const int t = e / kWidth, n = e % kWidth;
+            const bool in = t0 + t < p.seqlen && n < N;
+            const int64_t idx = (b * p.seqlen + t0 + t) * N + n;
+            pb[i] = in ? ldg_f32(Bp + idx) : 0.0f;
+            pc[i] = in ? ldg_f32(Cp + idx) : 0.0f;
+        }
+#pragma unroll
+        for (int i = 0; i < kXPer; ++i) {
+            const int e = tid + i * kThreads;
+            const int t = e / kChainsPerCta, cc = e % kChainsPerCta;
+            const int64_t dc = (int64_t)blockIdx.x * kChainsPerCta + cc;
+            const bool in = t0 + t < p.seqlen && dc < p.dim;
+            const int64_t i2 = (b * p.seqlen + t0 + t) * p.dim + dc;
+            px[i] = in ? make_float3(ldg_f32(xp + i2), ldg_f32(dp + i2),
+                                     kGate ? ldg_f32(zp + i2) : 0.0f)
+                       : make_float3(0.f, 0.f, 0.f);
+        }
+    };
+    fetch(0);
     for (int64_t t0 = 0; t0 < p.seqlen; t0 += kTileT) {
         const int nt = (int)min((int64_t)kTileT, p.seqlen - t0);
         __syncthreads();  // the previous tile is consumed
-        for (int e = tid; e < kTileT * kWidth; e += kThreads) {
+#pragma unroll
+        for (int i = 0; i < kBCPer; ++i) {
+            const int e = tid + i * kThreads;
             const int t = e / kWidth, n = e % kWidth;
-            const bool in = t < nt && n < N;
-            const int64_t idx = (b * p.seqlen + t0 + t) * N + n;
-            sB[t][n] = in ? ldg_f32(Bp + idx) : 0.0f;
-            sC[t][n] = in ? ldg_f32(Cp + idx) : 0.0f;
+            sB[t][n / kSlice][n % kSlice] = pb[i];
+            sC[t][n / kSlice][n % kSlice] = pc[i];
         }
-        // x, delta, z of the tile for the CTA's chains, staged once
-        for (int e = tid; e < kTileT * kChainsPerCta; e += kThreads) {
-            const int t = e / kChainsPerCta, cc = e % kChainsPerCta;
-            const int64_t dc = (int64_t)blockIdx.x * kChainsPerCta + cc;
-            const bool in = t < nt && dc < p.dim;
-            const int64_t i = (b * p.seqlen + t0 + t) * p.dim + dc;
-            sX[t][cc] = in ? make_float3(ldg_f32(xp + i), ldg_f32(dp + i),
-                                         kGate ? ldg_f32(zp + i) : 0.0f)
-                           : make_float3(0.f, 0.f, 0.f);
+#pragma unroll
+        for (int i = 0; i < kXPer; ++i) {
+            const int e = tid + i * kThreads;
+            sX[e / kChainsPerCta][e % kChainsPerCta] = px[i];
         }
+        if (t0 + kTileT < p.seqlen) fetch(t0 + kTileT);
         __syncthreads();
         const int cc = tid / kLanes;
-#pragma unroll 1
+#pragma unroll 2
         for (int t = 0; t < nt; ++t) {
             const float3 xdz = sX[t][cc];
             float xv = xdz.x;
@@ -150,17 +178,23 @@ scan_wide_kernel(const ScanParams p) {
                 for (int k = 0; k < kSlice; ++k) a[k] = ex2_approx(dt * A2[k]);
             }
             float part0 = 0.0f, part1 = 0.0f;
+            const float4 *B4 = reinterpret_cast<const float4 *>(&sB[t][slice][0]);
+            const float4 *C4 = reinterpret_cast<const float4 *>(&sC[t][slice][0]);
 #pragma unroll
-            for (int k = 0; k < kSlice; k += 2) {
-                float b0 = sB[t][n0 + k], b1 = sB[t][n0 + k + 1];
-                if (kZoh) {
-                    b0 *= zoh_factor(dt * A2[k] * kLn2, a[k]);
-                    b1 *= zoh_factor(dt * A2[k + 1] * kLn2, a[k + 1]);
+            for (int q = 0; q < kSlice / 4; ++q) {
+                const float4 bq = B4[q], cq = C4[q];
+                float bv[4] = {bq.x, bq.y, bq.z, bq.w};
+                const float cv[4] = {cq.x, cq.y, cq.z, cq.w};
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int k = 4 * q + i;
+                    if (kZoh) bv[i] *= zoh_factor(dt * A2[k] * kLn2, a[k]);
+                    h[k] = fmaf(a[k], h[k], u * bv[i]);
+                    if (i & 1)
+                        part1 = fmaf(cv[i], h[k], part1);
+                    else
+                        part0 = fmaf(cv[i], h[k], part0);
                 }
-                h[k] = fmaf(a[k], h[k], u * b0);
-                h[k + 1] = fmaf(a[k + 1], h[k + 1], u * b1);
-                part0 = fmaf(sC[t][n0 + k], h[k], part0);
-                part1 = fmaf(sC[t][n0 + k + 1], h[k + 1], part1);
             }
             float part = part0 + part1;
 #pragma unroll
