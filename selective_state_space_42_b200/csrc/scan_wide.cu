@@ -38,6 +38,11 @@ scan_wide_kernel(const ScanParams p) {
     __shared__ __align__(16) float sB[kTileT][kLanes][kRow];
     __shared__ __align__(16) float sC[kTileT][kLanes][kRow];
     __shared__ float3 sX[kTileT][kChainsPerCta];  // x, delta, z of the tile per chain
+    // without the conv, each (token, chain)'s scalars are computed once, by
+    // one thread, before the lanes of the chain read them: Δ, Δ·x, the decay
+    // base r = 2^(Δ·A[d,0]·log2 e), silu(z); and D·x·silu(z)
+    __shared__ float4 sS[kTileT][kChainsPerCta];
+    __shared__ float sY[kTileT][kChainsPerCta];
     const int tid = threadIdx.x;
     const int slice = tid % kLanes;
     const int64_t b = blockIdx.y;
@@ -144,23 +149,53 @@ scan_wide_kernel(const ScanParams p) {
         }
         if (t0 + kTileT < p.seqlen) fetch(t0 + kTileT);
         __syncthreads();
+        if (!conv) {
+#pragma unroll
+            for (int i = 0; i < kXPer; ++i) {
+                const int e = tid + i * kThreads;
+                const int t = e / kChainsPerCta, c2 = e % kChainsPerCta;
+                const int64_t dc = (int64_t)blockIdx.x * kChainsPerCta + c2;
+                float4 sc = make_float4(0.f, 0.f, 1.f, 1.f);
+                float dxg = 0.0f;
+                if (dc < p.dim && t < nt) {
+                    const float3 xdz = sX[t][c2];
+                    float v = xdz.y + (p.delta_bias ? p.delta_bias[dc] : 0.0f);
+                    if (p.softplus) v = softplus_f32(v);
+                    const float g = kGate ? silu_f32(xdz.z) : 1.0f;
+                    sc = make_float4(v, v * xdz.x, ex2_approx(v * p.A[dc * N] * kLog2e), g);
+                    dxg = (p.Dskip ? p.Dskip[dc] : 0.0f) * xdz.x * g;
+                }
+                sS[t][c2] = sc;
+                sY[t][c2] = dxg;
+            }
+            __syncthreads();
+        }
         const int cc = tid / kLanes;
 #pragma unroll 2
         for (int t = 0; t < nt; ++t) {
-            const float3 xdz = sX[t][cc];
-            float xv = xdz.x;
-            if (conv) xv = conv_step(cw, cb, xw, xv);
-            float dt = active ? xdz.y + bias : 0.0f;
-            if (p.softplus && active) dt = softplus_f32(dt);
-            const float u = dt * xv;
+            float xv, dt, u, r, gate;
+            if (conv) {
+                const float3 xdz = sX[t][cc];
+                xv = conv_step(cw, cb, xw, xdz.x);
+                dt = active ? xdz.y + bias : 0.0f;
+                if (p.softplus && active) dt = softplus_f32(dt);
+                u = dt * xv;
+                r = ex2_approx(dt * a0 * kLog2e);
+                gate = kGate ? silu_f32(xdz.z) : 1.0f;
+            } else {
+                const float4 sc = sS[t][cc];
+                xv = 0.0f;
+                dt = sc.x;
+                u = sc.y;
+                r = sc.z;
+                gate = sc.w;
+            }
             float a[kSlice];
             if (constant) {
-                const float r = ex2_approx(dt * a0 * kLog2e);
 #pragma unroll
                 for (int k = 0; k < kSlice; ++k) a[k] = r;
             } else if (structured) {
                 // r^(n0 + 1 + i) = r^n0 · r^(i + 1), the powers by a ladder of depth 4
-                const float r = ex2_approx(dt * a0 * kLog2e);
                 const float base = ex2_approx(dt * a0 * kLog2e * (float)n0);
                 float pw[kSlice];
                 pw[0] = r;
@@ -200,8 +235,8 @@ scan_wide_kernel(const ScanParams p) {
 #pragma unroll
             for (int m = 1; m < kLanes; m <<= 1) part += __shfl_xor_sync(0xffffffffu, part, m);
             if (active && slice == 0) {
-                float out = fmaf(dskip, xv, part);
-                if (kGate) out *= silu_f32(xdz.z);
+                const float out = conv ? fmaf(dskip, xv, part) * gate
+                                       : fmaf(part, gate, sY[t][cc]);
                 yp[(b * p.seqlen + t0 + t) * p.dim + d] = from_f32<T>(out);
             }
         }
