@@ -432,6 +432,37 @@ SELSCAN_API int selscan_state_update_ex(float *state, const void *x, const void 
                                         selscan_dtype_t dtype, selscan_stream_t stream);
 
 /*
+ * selscan_ssd_fwd -- the scan with one scalar A per head, computed in the
+ * chunked matrix form of "Mamba & State Space Models — Guide Complet" §5
+ * ("SSD — State Space Dual": y = (L ◦ S)·u, a causal mask times a structured
+ * semiseparable matrix). Channel d = h·headdim + p of head h:
+ *   Δ_t = softplus(dt[b,t,h] + dt_bias[h]) (or no softplus),
+ *   h_t[n] = exp(Δ_t·A[h])·h_{t−1}[n] + Δ_t·B[b,t,n]·x[b,t,d],
+ *   y[b,t,d] = (Σ_n C[b,t,n]·h_t[n] + D[h]·x[b,t,d])·silu(z[b,t,d]),
+ * i.e. selscan_fwd_from_state with delta, delta_bias, A and D broadcast from
+ * the heads to their channels.
+ *   x, z          [batch, seqlen, nheads·headdim]   dtype   (z NULL -> no gate)
+ *   dt            [batch, seqlen, nheads]           dtype
+ *   A, D, dt_bias [nheads]                          float32 (D, dt_bias nullable)
+ *   B, C          [batch, seqlen, dstate]           dtype   (one group)
+ *   initial_state, final_state [batch, nheads·headdim, dstate] float32, nullable
+ *   headdim 1..64, dstate 1..128, batch and nheads ≤ 65535.
+ * Chunks of 64 tokens; workspace (NULL: allocated on the stream) of
+ * selscan_ssd_workspace_bytes() bytes.
+ */
+SELSCAN_API int selscan_ssd_fwd(const void *x, const void *dt, const float *A, const void *B,
+                                const void *C, const float *D, const void *z,
+                                const float *dt_bias, int softplus_flag,
+                                const float *initial_state, void *y, float *final_state,
+                                int64_t batch, int64_t seqlen, int64_t nheads, int64_t headdim,
+                                int64_t dstate, selscan_dtype_t dtype, void *workspace,
+                                int64_t workspace_bytes, selscan_stream_t stream);
+
+/* Host-only: workspace bytes selscan_ssd_fwd takes (0 for empty or invalid sizes). */
+SELSCAN_API int64_t selscan_ssd_workspace_bytes(int64_t batch, int64_t seqlen, int64_t nheads,
+                                                int64_t headdim, int64_t dstate);
+
+/*
  * selscan_device_status -- the library's sticky device-side error word on
  * the current device (synchronous: waits for prior work). 0 means no device
  * wait has given up; otherwise the code of the first one that did (1: a

@@ -11,9 +11,9 @@ from .selscan import (LIB_PATH, SELSCAN_BF16, SELSCAN_F32, SELSCAN_MAX_DSTATE,
                       selscan_device_status, selscan_fwd, selscan_fwd_noalloc,
                       selscan_fwd_plan,
                       selscan_last_cuda_error,
-                      selscan_state_update, selscan_status_string)
+                      selscan_ssd_fwd, selscan_state_update, selscan_status_string)
 
-__all__ = ["selscan_bwd", "selscan_bwd_workspace_bytes", "selscan_device_status", "selscan_fwd", "selscan_fwd_noalloc", "selscan_fwd_plan", "selscan_state_update", "selscan_status_string",
+__all__ = ["selscan_bwd", "selscan_bwd_workspace_bytes", "selscan_device_status", "selscan_fwd", "selscan_fwd_noalloc", "selscan_fwd_plan", "selscan_state_update", "selscan_ssd_fwd", "selscan_status_string",
            "selscan_last_cuda_error", "load_library", "SelscanError",
            "SelscanUnavailable", "LIB_PATH", "SELSCAN_F32", "SELSCAN_BF16",
            "SELSCAN_MAX_DSTATE", "SELSCAN_NOALLOC_WORKSPACE_BYTES"]

@@ -17,8 +17,8 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB_PATH = os.path.join(HERE, "libselscan.so")
-SOURCES = ["api.cu", "scan.cu", "scan_tma.cu", "scan_wide.cu", "scan_bwd.cu", "state_update.cu",
-           "noalloc.cu"]
+SOURCES = ["api.cu", "scan.cu", "scan_tma.cu", "scan_wide.cu", "scan_bwd.cu", "ssd.cu",
+           "state_update.cu", "noalloc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

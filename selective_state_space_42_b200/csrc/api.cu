@@ -716,6 +716,117 @@ int64_t selscan_bwd_conv_workspace_bytes(int64_t batch, int64_t seqlen, int64_t 
     return (int64_t)bwd_layout(batch, seqlen, dim, true).total;
 }
 
+}  // extern "C"
+
+namespace {
+
+struct SsdLayout {
+    size_t ypart, cstate, decay, sin, total;
+};
+
+SsdLayout ssd_layout(int64_t batch, int64_t seqlen, int64_t nheads, int64_t headdim) {
+    const int64_t nc = ceil_div64(seqlen, selscan::ssd_chunk_tokens());
+    const size_t per = (size_t)selscan::ssd_max_dstate() * selscan::ssd_max_headdim();
+    SsdLayout l;
+    size_t off = 0;
+    l.ypart = off;
+    off = align256(off + (size_t)(batch * seqlen * nheads * headdim) * sizeof(float));
+    l.cstate = off;
+    off = align256(off + (size_t)(batch * nheads * nc) * per * sizeof(float));
+    l.decay = off;
+    off = align256(off + (size_t)(batch * nheads * nc) * sizeof(float));
+    l.sin = off;
+    off = align256(off + (size_t)(batch * nheads * nc) * per * sizeof(float));
+    l.total = off;
+    return l;
+}
+
+}  // namespace
+
+extern "C" {
+
+int64_t selscan_ssd_workspace_bytes(int64_t batch, int64_t seqlen, int64_t nheads,
+                                    int64_t headdim, int64_t dstate) {
+    if (batch <= 0 || seqlen <= 0 || nheads <= 0 || headdim <= 0 ||
+        headdim > selscan::ssd_max_headdim() || dstate < 1 || dstate > selscan::ssd_max_dstate())
+        return 0;
+    if (!mul_le(batch, seqlen, kMaxElems) || !mul_le(batch * seqlen, nheads * headdim, kMaxElems))
+        return 0;
+    return (int64_t)ssd_layout(batch, seqlen, nheads, headdim).total;
+}
+
+int selscan_ssd_fwd(const void *x, const void *dt, const float *A, const void *B, const void *C,
+                    const float *D, const void *z, const float *dt_bias, int softplus_flag,
+                    const float *initial_state, void *y, float *final_state, int64_t batch,
+                    int64_t seqlen, int64_t nheads, int64_t headdim, int64_t dstate,
+                    selscan_dtype_t dtype, void *workspace, int64_t workspace_bytes,
+                    selscan_stream_t stream_) {
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    if (dtype != SELSCAN_F32 && dtype != SELSCAN_BF16) return SELSCAN_ERR_BAD_DTYPE;
+    if (batch < 0 || seqlen < 0 || nheads < 0 || batch > 65535 || nheads > 65535 ||
+        headdim < 1 || headdim > selscan::ssd_max_headdim())
+        return SELSCAN_ERR_BAD_DIM;
+    if (dstate < 1 || dstate > selscan::ssd_max_dstate()) return SELSCAN_ERR_DSTATE_UNSUPPORTED;
+    const int64_t dim = nheads * headdim;
+    if (!mul_le(batch, seqlen, kMaxElems) || !mul_le(batch * seqlen, dim, kMaxElems) ||
+        !mul_le(batch, dim * dstate, kMaxElems))
+        return SELSCAN_ERR_BAD_DIM;
+    const bool has_tokens = batch * seqlen * dim > 0;
+    if (has_tokens && (!x || !dt || !A || !B || !C || !y)) return SELSCAN_ERR_NULL_ARG;
+    const size_t es = dtype == SELSCAN_F32 ? 4 : 2;
+    if (misaligned(x, es) || misaligned(dt, es) || misaligned(z, es) || misaligned(B, es) ||
+        misaligned(C, es) || misaligned(y, es) || misaligned(A, 4) || misaligned(D, 4) ||
+        misaligned(dt_bias, 4) || misaligned(initial_state, 4) || misaligned(final_state, 4) ||
+        misaligned(workspace, 256))
+        return SELSCAN_ERR_MISALIGNED;
+    const size_t nx = (size_t)(batch * seqlen * dim) * es;
+    const size_t ndt = (size_t)(batch * seqlen * nheads) * es;
+    const size_t nbc = (size_t)(batch * seqlen * dstate) * es;
+    const size_t ns = (size_t)(batch * dim * dstate) * sizeof(float);
+    const Span outs[] = {{y, nx}, {final_state, ns}};
+    const Span ins[] = {{x, nx}, {dt, ndt}, {z, nx}, {B, nbc}, {C, nbc}, {initial_state, ns}};
+    if (any_overlap(outs, 2, ins, 6)) return SELSCAN_ERR_ALIAS;
+    if (!has_tokens) {
+        if (final_state && batch * dim > 0) {
+            cudaError_t e = initial_state
+                                ? cudaMemcpyAsync(final_state, initial_state, ns,
+                                                  cudaMemcpyDeviceToDevice, stream)
+                                : cudaMemsetAsync(final_state, 0, ns, stream);
+            if (e != cudaSuccess) return selscan::cuda_fail(e);
+        }
+        return SELSCAN_OK;
+    }
+    const SsdLayout l = ssd_layout(batch, seqlen, nheads, headdim);
+    void *ws = workspace;
+    if (ws) {
+        if (workspace_bytes < (int64_t)l.total) return SELSCAN_ERR_WORKSPACE;
+        const Span wsp[] = {{ws, l.total}};
+        if (any_overlap(wsp, 1, outs, 2) || any_overlap(wsp, 1, ins, 6)) return SELSCAN_ERR_ALIAS;
+    } else {
+        cudaError_t e = cudaMallocAsync(&ws, l.total, stream);
+        if (e != cudaSuccess) return selscan::cuda_fail(e);
+    }
+    char *w = static_cast<char *>(ws);
+    selscan::SsdParams p{};
+    p.x = x; p.dt = dt; p.z = z; p.B = B; p.C = C;
+    p.A = A; p.Dskip = D; p.dt_bias = dt_bias; p.h0 = initial_state;
+    p.y = y; p.final_state = final_state;
+    p.ypart = reinterpret_cast<float *>(w + l.ypart);
+    p.chunk_state = reinterpret_cast<float *>(w + l.cstate);
+    p.chunk_decay = reinterpret_cast<float *>(w + l.decay);
+    p.state_in = reinterpret_cast<float *>(w + l.sin);
+    p.batch = batch; p.seqlen = seqlen;
+    p.nheads = (int)nheads; p.headdim = (int)headdim; p.dstate = (int)dstate;
+    p.nchunks = (int)ceil_div64(seqlen, selscan::ssd_chunk_tokens());
+    p.softplus = softplus_flag ? 1 : 0;
+    cudaError_t e = selscan::launch_ssd(p, dtype == SELSCAN_BF16, stream);
+    if (!workspace) {
+        cudaError_t ef = cudaFreeAsync(ws, stream);
+        if (e == cudaSuccess) e = ef;
+    }
+    return e == cudaSuccess ? SELSCAN_OK : selscan::cuda_fail(e);
+}
+
 int selscan_device_status(int *status, int clear) {
     if (!status) return SELSCAN_ERR_NULL_ARG;
     cudaError_t e = selscan::read_device_status(status, clear != 0);

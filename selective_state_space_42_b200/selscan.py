@@ -82,6 +82,9 @@ SIGNATURES = {
                                           _i64, _i64, _i64, _int, _vp]),
     "selscan_state_update_ex": (_int, [_vp] * 9 + [_int, ctypes.POINTER(StepOptions), _vp,
                                                    _i64, _i64, _i64, _int, _vp]),
+    "selscan_ssd_fwd": (_int, [_vp] * 8 + [_int, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64,
+                                          _int, _vp, _i64, _vp]),
+    "selscan_ssd_workspace_bytes": (_i64, [_i64, _i64, _i64, _i64, _i64]),
     "selscan_device_status": (_int, [ctypes.POINTER(_int), _int]),
     "selscan_status_string": (ctypes.c_char_p, [_int]),
     "selscan_last_cuda_error": (ctypes.c_char_p, []),
@@ -406,6 +409,57 @@ def selscan_bwd(x, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=Tru
     _check(lib.selscan_bwd_workspace(*args, ws.data_ptr() if nbytes else None, nbytes,
                                      _stream_ptr(stream, dev)))
     return out
+
+
+def selscan_ssd_fwd(x, dt, A, B, C, D=None, z=None, dt_bias=None, softplus=True,
+                    initial_state=None, y=None, final_state=None, return_final_state=False,
+                    stream=None):
+    """The scan with one scalar A per head in chunked matrix form (C ABI
+    ``selscan_ssd_fwd``). x, z: [batch, L, nheads·headdim]; dt: [batch, L,
+    nheads]; A, D, dt_bias: [nheads] float32; B, C: [batch, L, dstate];
+    initial_state / final_state: [batch, nheads·headdim, dstate] float32.
+    Returns y (or (y, final_state))."""
+    torch = _torch()
+    if x.dim() != 3 or dt.dim() != 3:
+        raise ValueError("x must be [batch, L, dim] and dt [batch, L, nheads]")
+    batch, L, dim = x.shape
+    nheads = dt.shape[2]
+    if nheads == 0 or dim % nheads:
+        raise ValueError("dim must be a multiple of nheads")
+    headdim = dim // nheads
+    N = B.shape[2]
+    dev, dtp = x.device, x.dtype
+    code = _dtype_code(x)
+    f32 = torch.float32
+    if y is None:
+        y = torch.empty_like(x)
+    if final_state is None and return_final_state:
+        final_state = torch.empty(batch, dim, N, device=dev, dtype=f32)
+    lib = load_library()
+    nbytes = int(lib.selscan_ssd_workspace_bytes(batch, L, nheads, headdim, N))
+    ws = torch.empty(max(nbytes, 1), device=dev, dtype=torch.uint8)
+    if stream is not None and not isinstance(stream, int):
+        ws.record_stream(stream)
+    args = [
+        _ptr(x, "x", (batch, L, dim), dtp, dev),
+        _ptr(dt, "dt", (batch, L, nheads), dtp, dev),
+        _ptr(A, "A", (nheads,), f32, dev),
+        _ptr(B, "B", (batch, L, N), dtp, dev),
+        _ptr(C, "C", (batch, L, N), dtp, dev),
+        _ptr(D, "D", (nheads,), f32, dev, required=False),
+        _ptr(z, "z", (batch, L, dim), dtp, dev, required=False),
+        _ptr(dt_bias, "dt_bias", (nheads,), f32, dev, required=False),
+        int(bool(softplus)),
+        _ptr(initial_state, "initial_state", (batch, dim, N), f32, dev, required=False),
+        _ptr(y, "y", (batch, L, dim), dtp, dev),
+        _ptr(final_state, "final_state", (batch, dim, N), f32, dev, required=False),
+        batch, L, nheads, headdim, N, code, ws.data_ptr() if nbytes else None, nbytes,
+        _stream_ptr(stream, dev),
+    ]
+    _check(lib.selscan_ssd_fwd(*args))
+    if return_final_state:
+        return y, final_state
+    return y
 
 
 def selscan_bwd_workspace_bytes(batch: int, seqlen: int, dim: int, dstate: int) -> int:

@@ -1,0 +1,103 @@
+"""GPU parity of selscan_ssd_fwd (the scan with one scalar A per head, in
+chunked matrix form) against the oracle's scan with the heads' Δ, A, D and
+bias broadcast to their channels."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import selective_state_space_42_b200 as ss
+from selective_state_space_42_b200 import workloads as wl
+
+import gpu_helpers as gh
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def _inputs(batch, L, H, P, N, dtype, seed, gate=True):
+    g = torch.Generator().manual_seed(seed)
+    dt_ = wl.DTYPES[dtype]
+    D = H * P
+    inp = dict(
+        x=torch.randn(batch, L, D, generator=g).to(dt_),
+        dt=(0.5 * torch.randn(batch, L, H, generator=g)).to(dt_),
+        z=torch.randn(batch, L, D, generator=g).to(dt_) if gate else None,
+        B=torch.randn(batch, L, N, generator=g).to(dt_),
+        C=torch.randn(batch, L, N, generator=g).to(dt_),
+        A=-(torch.rand(H, generator=g) * 3.5 + 0.5),
+        Dh=1.0 + 0.1 * torch.randn(H, generator=g),
+        dt_bias=torch.log(torch.expm1(1e-3 + (1e-1 - 1e-3) * torch.rand(H, generator=g,
+                                                                         dtype=torch.float64))
+                          ).float(),
+    )
+    return inp
+
+
+def _oracle(inp, P, h0=None):
+    n = gh.to_np
+    H = inp["A"].shape[0]
+    N = inp["B"].shape[2]
+    rep = lambda v: np.repeat(n(v), P, axis=-1)  # noqa: E731  heads -> channels
+    A_full = np.repeat(n(inp["A"])[:, None], P, axis=0).repeat(N, axis=1)
+    return oracle.default().fwd(n(inp["x"]), rep(inp["dt"]), A_full, n(inp["B"]), n(inp["C"]),
+                                rep(inp["Dh"]), None if inp["z"] is None else n(inp["z"]),
+                                rep(inp["dt_bias"]), h0=None if h0 is None else n(h0))
+
+
+def _gpu(inp, h0=None):
+    d = {k: (None if v is None else v.to(DEV)) for k, v in inp.items()}
+    return ss.selscan_ssd_fwd(d["x"], d["dt"], d["A"], d["B"], d["C"], D=d["Dh"], z=d["z"],
+                              dt_bias=d["dt_bias"], initial_state=h0,
+                              return_final_state=True)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("shape", [(1, 1, 1, 1, 1), (2, 100, 3, 64, 16), (1, 200, 2, 64, 128),
+                                   (2, 65, 4, 32, 64), (1, 1000, 2, 64, 64),
+                                   (1, 130, 5, 7, 33)], ids=str)
+def test_ssd_matches_scan(dtype, shape):
+    batch, L, H, P, N = shape
+    inp = _inputs(batch, L, H, P, N, dtype, seed=7000 + L + H + N)
+    y, hf = _gpu(inp)
+    torch.cuda.synchronize()
+    yo, ho = _oracle(inp, P)
+    gh.compare(gh.to_np(y), yo, gh.RTOL[dtype], f"{shape} y")
+    gh.compare(gh.to_np(hf), ho, gh.RTOL[dtype], f"{shape} final state")
+
+
+def test_ssd_initial_state_and_no_gate():
+    inp = _inputs(2, 300, 3, 64, 64, "f32", seed=7100, gate=False)
+    g = torch.Generator().manual_seed(7101)
+    h0 = torch.randn(2, 3 * 64, 64, generator=g)
+    y, hf = _gpu(inp, h0.to(DEV))
+    torch.cuda.synchronize()
+    yo, ho = _oracle(inp, 64, h0)
+    gh.compare(gh.to_np(y), yo, gh.RTOL["f32"], "h0 y")
+    gh.compare(gh.to_np(hf), ho, gh.RTOL["f32"], "h0 final state")
+
+
+def test_ssd_equals_wide_scan_on_a_head_layer():
+    """A Mamba-2-sized layer (2 × 2048 tokens, 32 heads of 64, d_state 128):
+    the chunked form against the recurrence of the wide-state scan kernel
+    with the same inputs broadcast to channels, and a channel sample against
+    the oracle."""
+    inp = _inputs(2, 2048, 32, 64, 128, "bf16", seed=7200)
+    y, hf = _gpu(inp)
+    d = {k: (None if v is None else v.to(DEV)) for k, v in inp.items()}
+    rep = lambda v: v.repeat_interleave(64, dim=-1).contiguous()  # noqa: E731
+    A_full = d["A"].repeat_interleave(64)[:, None].repeat(1, 128).contiguous()
+    yw, hw = ss.selscan_fwd(d["x"], rep(d["dt"]), A_full, d["B"], d["C"], rep(d["Dh"]), d["z"],
+                            rep(d["dt_bias"]), return_final_state=True)
+    torch.cuda.synchronize()
+    gh.compare(gh.to_np(y), gh.to_np(yw), 2e-2, "ssd vs recurrence y")
+    gh.compare(gh.to_np(hf), gh.to_np(hw), 2e-2, "ssd vs recurrence state")
+    chans = list(wl.channel_subset(2048, 64))
+    n = gh.to_np
+    heads = [c // 64 for c in chans]
+    A_s = np.repeat(n(inp["A"])[heads][:, None], 128, axis=1)
+    yo, ho = oracle.default().fwd(n(inp["x"][:, :, chans]), n(inp["dt"][:, :, heads]), A_s,
+                                  n(inp["B"]), n(inp["C"]), n(inp["Dh"])[heads],
+                                  n(inp["z"][:, :, chans]), n(inp["dt_bias"])[heads])
+    gh.compare(gh.to_np(y[:, :, chans]), yo, gh.RTOL["bf16"], "ssd layer y")
+    gh.compare(gh.to_np(hf[:, chans]), ho, gh.RTOL["bf16"], "ssd layer state")
