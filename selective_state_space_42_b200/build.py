@@ -17,7 +17,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB_PATH = os.path.join(HERE, "libselscan.so")
-SOURCES = ["api.cu", "scan.cu", "scan_tma.cu", "scan_wide.cu", "scan_bwd.cu", "ssd.cu",
+SOURCES = ["api.cu", "scan.cu", "scan_tma.cu", "scan_wide.cu", "scan_bwd.cu", "ssd.cu", "ssd_tc.cu",
            "state_update.cu", "noalloc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

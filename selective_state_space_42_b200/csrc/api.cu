@@ -819,6 +819,12 @@ int selscan_ssd_fwd(const void *x, const void *dt, const float *A, const void *B
     p.nheads = (int)nheads; p.headdim = (int)headdim; p.dstate = (int)dstate;
     p.nchunks = (int)ceil_div64(seqlen, selscan::ssd_chunk_tokens());
     p.softplus = softplus_flag ? 1 : 0;
+    p.vec_x = (headdim % 8 == 0) && !misaligned(x, 16) && !misaligned(y, 16) && !misaligned(z, 16);
+    p.vec_bc = (dstate % 8 == 0) && !misaligned(B, 16) && !misaligned(C, 16);
+    {
+        cudaError_t es = selscan::device_status_address(&p.status);
+        if (es != cudaSuccess) return selscan::cuda_fail(es);
+    }
     cudaError_t e = selscan::launch_ssd(p, dtype == SELSCAN_BF16, stream);
     if (!workspace) {
         cudaError_t ef = cudaFreeAsync(ws, stream);

@@ -699,6 +699,10 @@ cudaError_t launch_gate(const TmaScanParams &p, const void *x, const void *dl, c
 
 }  // namespace
 
+cudaError_t device_status_address(int **p) {
+    return cudaGetSymbolAddress(reinterpret_cast<void **>(p), g_device_status);
+}
+
 cudaError_t read_device_status(int *out, bool clear) {
     cudaError_t e = cudaMemcpyFromSymbol(out, g_device_status, sizeof(int));
     if (e == cudaSuccess && clear) {

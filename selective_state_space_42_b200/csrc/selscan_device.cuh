@@ -184,8 +184,17 @@ struct SsdParams {
     long long batch, seqlen;
     int nheads, headdim, dstate, nchunks;
     int softplus;
+    int vec_x;                       // x, z, y rows allow 16-byte accesses (tensor-core path)
+    int vec_bc;                      // B, C rows allow 16-byte accesses (tensor-core path)
+    int *status;                     // the library's device error word
 };
 cudaError_t launch_ssd(const SsdParams &p, bool bf16, cudaStream_t stream);
+// Tensor-core form for bfloat16 I/O (ssd_tc.cu): 128-token chunks.
+bool ssd_tc_supported(int headdim, int dstate);
+int ssd_tc_chunk_tokens();
+cudaError_t launch_ssd_tc_state(const SsdParams &p, cudaStream_t stream);
+cudaError_t launch_ssd_tc_out(const SsdParams &p, cudaStream_t stream);
+cudaError_t device_status_address(int **p);
 int ssd_chunk_tokens();
 int ssd_max_headdim();
 int ssd_max_dstate();

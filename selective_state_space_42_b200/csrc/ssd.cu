@@ -278,37 +278,40 @@ __global__ void __launch_bounds__(kThr) ssd_out_kernel(const SsdParams p) {
     }
 }
 
-template <typename T>
-cudaError_t launch_typed(const SsdParams &p, cudaStream_t stream) {
+cudaError_t launch_state(const SsdParams &p, cudaStream_t stream) {
+    const long long nst = (long long)p.batch * p.nheads * kNS * kP;
+    ssd_state_kernel<<<(unsigned)((nst + 255) / 256), 256, 0, stream>>>(p);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_f32(const SsdParams &p, cudaStream_t stream) {
     const size_t smem = sizeof(SsdSmem);
     static bool configured[64] = {false};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev >= 0 && dev < 64 && !configured[dev]) {
-        e = cudaFuncSetAttribute(ssd_chunk_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)smem);
+        e = cudaFuncSetAttribute(ssd_chunk_kernel<float>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(ssd_out_kernel<T, true>,
+            e = cudaFuncSetAttribute(ssd_out_kernel<float, true>,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(ssd_out_kernel<T, false>,
+            e = cudaFuncSetAttribute(ssd_out_kernel<float, false>,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
         configured[dev] = true;
     }
     const dim3 grid((unsigned)p.nchunks, (unsigned)p.nheads, (unsigned)p.batch);
-    ssd_chunk_kernel<T><<<grid, kThr, smem, stream>>>(p);
+    ssd_chunk_kernel<float><<<grid, kThr, smem, stream>>>(p);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    const long long nst = (long long)p.batch * p.nheads * kNS * kP;
-    ssd_state_kernel<<<(unsigned)((nst + 255) / 256), 256, 0, stream>>>(p);
-    e = cudaGetLastError();
+    e = launch_state(p, stream);
     if (e != cudaSuccess) return e;
     if (p.z)
-        ssd_out_kernel<T, true><<<grid, kThr, smem, stream>>>(p);
+        ssd_out_kernel<float, true><<<grid, kThr, smem, stream>>>(p);
     else
-        ssd_out_kernel<T, false><<<grid, kThr, smem, stream>>>(p);
+        ssd_out_kernel<float, false><<<grid, kThr, smem, stream>>>(p);
     return cudaGetLastError();
 }
 
@@ -318,8 +321,23 @@ int ssd_chunk_tokens() { return kQ; }
 int ssd_max_headdim() { return kP; }
 int ssd_max_dstate() { return kNS; }
 
-cudaError_t launch_ssd(const SsdParams &p, bool bf16, cudaStream_t stream) {
-    return bf16 ? launch_typed<__nv_bfloat16>(p, stream) : launch_typed<float>(p, stream);
+// float32 I/O: the float32 chunk kernels above with 64-token chunks.
+// bfloat16 I/O: the tensor-core chunk kernels (ssd_tc.cu) with 128-token
+// chunks; the element-wise carry between chunks is the same kernel.
+cudaError_t launch_ssd(const SsdParams &p_in, bool bf16, cudaStream_t stream) {
+    SsdParams p = p_in;
+    if (!bf16) {
+        p.nchunks = (int)((p.seqlen + kQ - 1) / kQ);
+        return launch_f32(p, stream);
+    }
+    if (!ssd_tc_supported(p.headdim, p.dstate)) return cudaErrorInvalidValue;
+    const int q = ssd_tc_chunk_tokens();
+    p.nchunks = (int)((p.seqlen + q - 1) / q);
+    cudaError_t e = launch_ssd_tc_state(p, stream);
+    if (e != cudaSuccess) return e;
+    e = launch_state(p, stream);
+    if (e != cudaSuccess) return e;
+    return launch_ssd_tc_out(p, stream);
 }
 
 }  // namespace selscan
