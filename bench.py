@@ -86,6 +86,16 @@ def peaks():
         return 6650.0, "fallback"
 
 
+def tensor_peak() -> float:
+    """Dense bf16 TFLOP/s for a kernel timed alone (the measured burst figure,
+    else the pool's earlier measurement)."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops"])
+    except Exception:
+        return 1590.0
+
+
 # ---- clocks sampled during the timed region -----------------------------------
 class ClockSampler:
     FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,"
@@ -429,6 +439,45 @@ def main():
     dec_ms = max_over_ranks(d0.elapsed_time(d1) / n_dec, dist if world > 1 else None, dev)
     dec_cold = max_over_ranks(sorted(cold)[len(cold) // 2], dist if world > 1 else None, dev)
 
+    # the Mamba-2-shaped SSD layer (one scalar A per head, chunked form on the
+    # tensor cores): back to back, and after an L2-evicting write; not part
+    # of the metric
+    sw = wl.SSD
+    sinp = wl.make_ssd_inputs(sw, device=dev)
+    sy = torch.empty_like(sinp["x"])
+    sfs = torch.empty(sw.batch, sw.dim, sw.dstate, device=dev)
+
+    def ssd_call():
+        ss.selscan_ssd_fwd(sinp["x"], sinp["dt"], sinp["A"], sinp["B"], sinp["C"], D=sinp["D"],
+                           z=sinp["z"], dt_bias=sinp["dt_bias"], y=sy, final_state=sfs,
+                           stream=stream)
+
+    for _ in range(5):
+        ssd_call()
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    scold = []
+    for _ in range(10):
+        flush.zero_()
+        c0 = torch.cuda.Event(enable_timing=True)
+        c1 = torch.cuda.Event(enable_timing=True)
+        c0.record(stream)
+        ssd_call()
+        c1.record(stream)
+        torch.cuda.synchronize(dev)
+        scold.append(c0.elapsed_time(c1))
+    del flush
+    s0 = torch.cuda.Event(enable_timing=True)
+    s1 = torch.cuda.Event(enable_timing=True)
+    n_ssd = 50
+    s0.record(stream)
+    for _ in range(n_ssd):
+        ssd_call()
+    s1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    ssd_ms = max_over_ranks(s0.elapsed_time(s1) / n_ssd, dist if world > 1 else None, dev)
+    ssd_cold = max_over_ranks(sorted(scold)[len(scold) // 2], dist if world > 1 else None, dev)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = oracle_cpu_baseline(inp, w, args.cpu_seconds)
@@ -466,6 +515,15 @@ def main():
             "GBps_back_to_back": dw.algorithmic_bytes_per_step() / dec_ms / 1e6,
             "frac_back_to_back": dw.algorithmic_bytes_per_step() / dec_ms / 1e6 / peak,
             "kernel": "state_update_vec_kernel<bf16, gate>"},
+        "ssd_layer": {
+            "workload": sw.name, "bytes_per_call": sw.algorithmic_bytes(),
+            "flops_per_call": sw.algorithmic_flops(),
+            "us_back_to_back": ssd_ms * 1e3, "us_after_l2_flush": ssd_cold * 1e3,
+            "GBps_back_to_back": sw.algorithmic_bytes() / ssd_ms / 1e6,
+            "TFLOPs_back_to_back": sw.algorithmic_flops() / ssd_ms / 1e9,
+            "frac_hbm_back_to_back": sw.algorithmic_bytes() / ssd_ms / 1e6 / peak,
+            "frac_tensor_back_to_back": sw.algorithmic_flops() / ssd_ms / 1e9 / tensor_peak(),
+            "kernels": ["ssd_tc_state_kernel", "ssd_tc_carry_kernel", "ssd_tc_out_kernel<gate>"]},
         "gpu_launches": args.steps * plan["launches"],
         "plan": plan,
         "cpu_baseline": cpu,

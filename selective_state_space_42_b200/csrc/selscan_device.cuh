@@ -193,6 +193,7 @@ cudaError_t launch_ssd(const SsdParams &p, bool bf16, cudaStream_t stream);
 bool ssd_tc_supported(int headdim, int dstate);
 int ssd_tc_chunk_tokens();
 cudaError_t launch_ssd_tc_state(const SsdParams &p, cudaStream_t stream);
+cudaError_t launch_ssd_tc_carry(const SsdParams &p, cudaStream_t stream);
 cudaError_t launch_ssd_tc_out(const SsdParams &p, cudaStream_t stream);
 cudaError_t device_status_address(int **p);
 int ssd_chunk_tokens();

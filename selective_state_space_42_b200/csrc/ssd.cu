@@ -335,7 +335,7 @@ cudaError_t launch_ssd(const SsdParams &p_in, bool bf16, cudaStream_t stream) {
     p.nchunks = (int)((p.seqlen + q - 1) / q);
     cudaError_t e = launch_ssd_tc_state(p, stream);
     if (e != cudaSuccess) return e;
-    e = launch_state(p, stream);
+    e = launch_ssd_tc_carry(p, stream);
     if (e != cudaSuccess) return e;
     return launch_ssd_tc_out(p, stream);
 }

@@ -10,10 +10,12 @@
 //   chunk output            y  = M·X + diag(exp(Acum_i))·C·h_in + D·x,
 //                           M  = (C·Bᵀ) ◦ [j ≤ i]·exp(Acum_i − Acum_j)·Δ_j        (Q×Q)
 // and h_in, the state entering each chunk, comes from the element-wise carry
-// h_c = exp(Acum_end,c)·h_{c−1} + S_c (ssd.cu). Two kernels here:
+// h_c = exp(Acum_end,c)·h_{c−1} + S_c. Three kernels:
 //   ssd_tc_state_kernel  S for one (chunk, head, batch row): MMAs of
 //                        M=128 (state n) × N=64 (head channel p) × K=2×128
 //                        (token; w ◦ X as a bfloat16 high/low pair)
+//   ssd_tc_carry_kernel  the element-wise carry over chunks, writing each h_in
+//                        in the output kernel's operand layout
 //   ssd_tc_out_kernel    G = C·Bᵀ (128×128, K = d_state) and C·h_in (128×64) on
 //                        the tensor cores (h_in as a bfloat16 high/low pair),
 //                        M built from G by the 128 threads
@@ -22,8 +24,9 @@
 //                        M_hi + M_lo, then M·X (128×64, K = 2×128) and the
 //                        epilogue y = M·X + exp(Acum_i)·C·h_in + D·x, gated
 //                        by silu(z).
-// Operands are bfloat16 in shared memory, written by the threads (no TMA: the
-// Δ-dependent scalings are applied while staging) in the interleaved layout
+// Operands are bfloat16 in shared memory, copied in (cp.async rows, one bulk
+// copy for h_in) or written by the threads where a Δ-dependent scaling is
+// applied while staging, in the interleaved layout
 // the MMA reads without swizzling: 8×8 core matrices of 128 contiguous bytes,
 // eight rows of 16 bytes along the tile's contiguous dimension. Accumulators
 // are float32 in tensor memory; one elected thread issues every MMA and a
@@ -31,13 +34,14 @@
 #include "selscan_device.cuh"
 #include "tma_util.cuh"
 
+#include <cstddef>
+
 namespace selscan {
 namespace {
 
 constexpr int kQ = 128;   // tokens per chunk (= MMA M, one tensor-memory lane per token)
 constexpr int kPp = 64;   // head dimension, zero-padded
 constexpr int kNp = 128;  // d_state, zero-padded
-constexpr int kThr = 128;
 constexpr uint64_t kWaitNs = 2000000000ull;  // bounded MMA-completion wait (2 s)
 constexpr int kStatusMmaWait = 4;             // device error code: an MMA wait gave up
 
@@ -171,29 +175,82 @@ __device__ __forceinline__ void st_smem16(void *base, uint32_t off, const uint4 
     *reinterpret_cast<uint4 *>(static_cast<char *>(base) + off) = v;
 }
 
-// Δ_t for this thread's token t (zero past the sequence end) and the
-// inclusive prefix sums of Δ·A over the chunk into acum[].
-__device__ __forceinline__ float chunk_delta(const SsdParams &p, long long b, int h,
-                                             long long t0, int nq, float *acum, float *wsum) {
+// 16-byte asynchronous global -> shared copy; src_bytes 0 writes zeros.
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
+                 "r"(src_bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+    asm volatile("cp.async.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+    asm volatile("cp.async.wait_all;" ::: "memory");
+}
+
+// Contiguous global -> shared bulk copy (16-byte aligned, size a multiple of
+// 16) completing on an mbarrier's transaction count.
+__device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes,
+                                          uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        ::"r"(smem_addr(dst)), "l"(src), "r"(bytes), "r"(smem_addr(bar))
+        : "memory");
+}
+
+// Column chunks [k_lo, k_hi) (8 columns each) of row r of an interleaved tile
+// from a global row of ncols bfloat16 (zero past ncols, or everywhere when
+// !live): asynchronous 16-byte copies where the row allows them (vec:
+// 16-byte aligned rows, ncols a multiple of 8), else loads and stores through
+// registers. `safe` is any valid global address, named by the zero-filling
+// copies.
+template <int kCols>
+__device__ __forceinline__ void stage_row(bf16 *tile, int r, int k_lo, int k_hi, const bf16 *row,
+                                          const bf16 *safe, bool live, int ncols, bool vec) {
+    if (vec) {
+        const uint32_t base = smem_addr(tile);
+#pragma unroll 4
+        for (int k8 = k_lo; k8 < k_hi; ++k8) {
+            const bool in = live && 8 * k8 < ncols;
+            cp_async16(base + core_off<kCols>(r, 8 * k8), in ? row + 8 * k8 : safe, in ? 16u : 0u);
+        }
+    } else {
+#pragma unroll 2
+        for (int k8 = k_lo; k8 < k_hi; ++k8)
+            st_smem16(tile, core_off<kCols>(r, 8 * k8),
+                      live ? ld8(row, 8 * k8, ncols, false) : make_uint4(0, 0, 0, 0));
+    }
+}
+
+// Δ_t of the chunk's tokens t (zero past the sequence end) into dt[], and the
+// inclusive prefix sums of Δ·A over the chunk, times log2(e), into acum2[]
+// (so exp(Acum_i − Acum_j) = 2^(acum2_i − acum2_j)). Threads 0..kQ−1 compute;
+// every thread of the block takes part in the two barriers.
+__device__ __forceinline__ void chunk_delta(const SsdParams &p, long long b, int h, long long t0,
+                                            int nq, float *dt, float *acum2, float *wsum) {
     const int t = threadIdx.x, lane = t & 31, w = t >> 5;
-    float d = 0.0f;
-    if (t < nq) {
-        d = ldg_f32(static_cast<const bf16 *>(p.dt) + (b * p.seqlen + t0 + t) * p.nheads + h) +
-            (p.dt_bias ? p.dt_bias[h] : 0.0f);
-        if (p.softplus) d = softplus_f32(d);
-    }
-    float s = d * p.A[h];
+    float d = 0.0f, s = 0.0f;
+    if (t < kQ) {
+        if (t < nq) {
+            d = ldg_f32(static_cast<const bf16 *>(p.dt) + (b * p.seqlen + t0 + t) * p.nheads + h) +
+                (p.dt_bias ? p.dt_bias[h] : 0.0f);
+            if (p.softplus) d = softplus_f32(d);
+        }
+        s = d * p.A[h] * kLog2e;
 #pragma unroll
-    for (int m = 1; m < 32; m <<= 1) {
-        const float o = __shfl_up_sync(0xffffffffu, s, m);
-        if (lane >= m) s += o;
+        for (int m = 1; m < 32; m <<= 1) {
+            const float o = __shfl_up_sync(0xffffffffu, s, m);
+            if (lane >= m) s += o;
+        }
+        if (lane == 31) wsum[w] = s;
     }
-    if (lane == 31) wsum[w] = s;
     __syncthreads();
-    for (int k = 0; k < w; ++k) s += wsum[k];
-    acum[t] = s;
+    if (t < kQ) {
+        for (int k = 0; k < w; ++k) s += wsum[k];
+        acum2[t] = s;
+        dt[t] = d;
+    }
     __syncthreads();
-    return d;
 }
 
 __device__ __forceinline__ bool wait_mma(uint64_t *bar, uint32_t parity, int *status) {
@@ -203,61 +260,70 @@ __device__ __forceinline__ bool wait_mma(uint64_t *bar, uint32_t parity, int *st
 }
 
 // ---- chunk states -----------------------------------------------------------------
+// 256 threads: thread t works on row r = t mod 128 (token j while staging,
+// state n = tensor-memory lane n in the epilogue) and column half t / 128.
+constexpr int kThrTc = 256;
+
 struct TcStateSmem {
     bf16 Bt[kQ * kNp];  // rows token j, columns state n
     bf16 Xw[kQ * kPp];  // rows token j, columns channel p: w_j·x, bfloat16 high part
     bf16 Xl[kQ * kPp];  // the low part, w_j·x − high
-    float acum[kQ];
+    float acum2[kQ];
+    float dt[kQ];
     float wsum[4];
     uint64_t bar;
     uint32_t tmem;
 };
 
-__global__ void __launch_bounds__(kThr) ssd_tc_state_kernel(const SsdParams p) {
+__global__ void __launch_bounds__(kThrTc) ssd_tc_state_kernel(const SsdParams p) {
     extern __shared__ __align__(128) unsigned char smem_raw[];
     TcStateSmem &S = *reinterpret_cast<TcStateSmem *>(smem_raw);
     const int c = blockIdx.x, h = blockIdx.y;
     const long long b = blockIdx.z;
     const long long t0 = (long long)c * kQ;
     const int nq = (int)min((long long)kQ, p.seqlen - t0);
-    const int t = threadIdx.x, warp = t >> 5;
+    const int t = threadIdx.x, warp = t >> 5, r = t & (kQ - 1), hh = t / kQ;
     const int N = p.dstate, P = p.headdim;
     const long long D = (long long)p.nheads * P;
+    const bool live = r < nq;
+    const long long row = b * p.seqlen + t0 + r;
 
     if (warp == 0) tmem_alloc(&S.tmem, 64);
     if (t == 0) {
         mbar_init(&S.bar, 1);
         fence_barrier_init();
     }
-    const float d = chunk_delta(p, b, h, t0, nq, S.acum, S.wsum);
-    const float aend = S.acum[kQ - 1];
-    const float w = __expf(aend - S.acum[t]) * d;  // 0 past the sequence end (Δ = 0)
-
-    // row j = t of B (states) and of w ◦ X (channels)
+    // row j = r of B: this thread's half of the states, asynchronously
+    stage_row<kNp>(S.Bt, r, hh * (kNp / 16), (hh + 1) * (kNp / 16),
+                   static_cast<const bf16 *>(p.B) + row * N, static_cast<const bf16 *>(p.B), live,
+                   N, p.vec_bc);
+    cp_async_commit();
+    uint4 xr[kPp / 16];
     {
-        const bool live = t < nq;
-        const bf16 *brow = static_cast<const bf16 *>(p.B) + (b * p.seqlen + t0 + t) * N;
-#pragma unroll 4
-        for (int k8 = 0; k8 < kNp / 8; ++k8) {
-            const uint4 v = live ? ld8(brow, 8 * k8, N, p.vec_bc) : make_uint4(0, 0, 0, 0);
-            st_smem16(S.Bt, core_off<kNp>(t, 8 * k8), v);
-        }
-        const bf16 *xrow = static_cast<const bf16 *>(p.x) + (b * p.seqlen + t0 + t) * D +
-                           (long long)h * P;
+        const bf16 *xrow = static_cast<const bf16 *>(p.x) + row * D + (long long)h * P;
 #pragma unroll
-        for (int k8 = 0; k8 < kPp / 8; ++k8) {
-            uint4 hi = make_uint4(0, 0, 0, 0), lo = hi;
-            if (live) {
-                float f[8];
-                unpack8(ld8(xrow, 8 * k8, P, p.vec_x), f);
+        for (int k = 0; k < kPp / 16; ++k)
+            xr[k] = live ? ld8(xrow, 8 * (hh * (kPp / 16) + k), P, p.vec_x) : make_uint4(0, 0, 0, 0);
+    }
+    chunk_delta(p, b, h, t0, nq, S.dt, S.acum2, S.wsum);
+    const float aend2 = S.acum2[kQ - 1];
+    // w_j ◦ x_j as a bfloat16 pair (0 past the sequence end: Δ = 0)
+    {
+        const float w = ex2_approx(aend2 - S.acum2[r]) * S.dt[r];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) f[e] *= w;
-                split8(f, hi, lo);
-            }
-            st_smem16(S.Xw, core_off<kPp>(t, 8 * k8), hi);
-            st_smem16(S.Xl, core_off<kPp>(t, 8 * k8), lo);
+        for (int k = 0; k < kPp / 16; ++k) {
+            float f[8];
+            unpack8(xr[k], f);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) f[e] *= w;
+            uint4 hi, lo;
+            split8(f, hi, lo);
+            const uint32_t off = core_off<kPp>(r, 8 * (hh * (kPp / 16) + k));
+            st_smem16(S.Xw, off, hi);
+            st_smem16(S.Xl, off, lo);
         }
     }
+    cp_async_wait_all();
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
@@ -286,22 +352,64 @@ __global__ void __launch_bounds__(kThr) ssd_tc_state_kernel(const SsdParams p) {
     const bool ok = __syncthreads_and(wait_mma(&S.bar, 0, p.status));
     tc_fence_after();
     if (ok) {
-        // lane t holds state row n = t: S[n][0..63]
-        float *dst = p.chunk_state + (((b * p.nheads + h) * p.nchunks + c) * 128 + t) * 64;
+        // lane r holds state row n = r: this thread stores S[n][32·hh .. 32·hh + 31]
+        float *dst = p.chunk_state + (((b * p.nheads + h) * p.nchunks + c) * 128 + r) * 64 + 32 * hh;
+        float v[32];
+        tmem_ld32(tmem + ((uint32_t)((warp & 3) * 32) << 16) + 32 * hh, v);
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-            float v[32];
-            tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + 32 * half, v);
-#pragma unroll
-            for (int k = 0; k < 32; k += 4)
-                *reinterpret_cast<float4 *>(dst + 32 * half + k) =
-                    make_float4(v[k], v[k + 1], v[k + 2], v[k + 3]);
-        }
-        if (t == 0) p.chunk_decay[(b * p.nheads + h) * p.nchunks + c] = __expf(aend);
+        for (int k = 0; k < 32; k += 4)
+            *reinterpret_cast<float4 *>(dst + k) = make_float4(v[k], v[k + 1], v[k + 2], v[k + 3]);
+        if (t == 0) p.chunk_decay[(b * p.nheads + h) * p.nchunks + c] = ex2_approx(aend2);
     }
     tc_fence_before();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tmem, 64);
+}
+
+// ---- states entering the chunks ----------------------------------------------------
+// h_in for every chunk, h_c = exp(Acum_end,c)·h_{c−1} + S_c from h_{−1} = h0
+// (or zero), written per chunk as the bfloat16 pair (high, low) in the
+// interleaved operand layout the output kernel's MMA reads: one 32 KB block
+// per (batch row, head, chunk) = high tile [state n][channel p] then low
+// tile. One thread per (batch row, head, state n, group of 8 channels).
+__global__ void ssd_tc_carry_kernel(const SsdParams p) {
+    const long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    const long long per = (long long)kNp * (kPp / 8);
+    if (e >= (long long)p.batch * p.nheads * per) return;
+    const long long bh = e / per;
+    const int n = (int)((e % per) / (kPp / 8)), pg = (int)(e % (kPp / 8));
+    const long long b = bh / p.nheads;
+    const int h = (int)(bh % p.nheads);
+    const int N = p.dstate, P = p.headdim;
+    float st[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        const int pp = 8 * pg + k;
+        st[k] = (p.h0 && n < N && pp < P)
+                    ? p.h0[((b * p.nheads + h) * (long long)P + pp) * N + n] : 0.0f;
+    }
+    const uint32_t off = core_off<kPp>(n, 8 * pg);
+    for (int c = 0; c < p.nchunks; ++c) {
+        char *blk = reinterpret_cast<char *>(p.state_in) + (bh * p.nchunks + c) * 32768ll;
+        uint4 hi, lo;
+        split8(st, hi, lo);
+        *reinterpret_cast<uint4 *>(blk + off) = hi;
+        *reinterpret_cast<uint4 *>(blk + 16384 + off) = lo;
+        const float dec = p.chunk_decay[bh * p.nchunks + c];
+        const float *cs = p.chunk_state + ((bh * p.nchunks + c) * 128 + n) * 64 + 8 * pg;
+        const float4 u = *reinterpret_cast<const float4 *>(cs);
+        const float4 v = *reinterpret_cast<const float4 *>(cs + 4);
+        const float s8[8] = {u.x, u.y, u.z, u.w, v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int k = 0; k < 8; ++k) st[k] = fmaf(dec, st[k], s8[k]);
+    }
+    if (p.final_state && n < N) {
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const int pp = 8 * pg + k;
+            if (pp < P) p.final_state[((b * p.nheads + h) * (long long)P + pp) * N + n] = st[k];
+        }
+    }
 }
 
 // ---- chunk outputs ----------------------------------------------------------------
@@ -310,72 +418,67 @@ struct TcOutSmem {
     bf16 BM[kQ * kNp];  // B (rows token j, columns n), then M_hi (rows i, columns j)
     bf16 HX[kNp * kPp]; // h_in high part (rows state n, columns channel p), then X
                         // (rows token j, columns p)
-    bf16 Hl[kNp * kPp]; // h_in low part
-    float acum[kQ];
+    bf16 Hl[kNp * kPp]; // h_in low part, then z (rows token i, columns p)
+    float acum2[kQ];
     float dt[kQ];
     float wsum[4];
-    uint64_t bar[2];
+    uint64_t bar[3];    // first MMAs, second MMAs, h_in bulk copy
     uint32_t tmem;
 };
 static_assert(kQ == kNp, "M reuses the B tile");
+static_assert(offsetof(TcOutSmem, Hl) == offsetof(TcOutSmem, HX) + 2 * kNp * kPp,
+              "h_in's two tiles are one contiguous copy");
 
 // Tensor-memory columns of the accumulators.
 constexpr uint32_t kColG = 0, kColYd = 128, kColYo = 192;
 
+// 256 threads: thread t works on token row r = t mod 128 (tensor-memory lane
+// r) and column half hh = t / 128 of every tile, of M and of y.
 template <bool kGate>
-__global__ void __launch_bounds__(kThr) ssd_tc_out_kernel(const SsdParams p) {
+__global__ void __launch_bounds__(kThrTc) ssd_tc_out_kernel(const SsdParams p) {
     extern __shared__ __align__(128) unsigned char smem_raw[];
     TcOutSmem &S = *reinterpret_cast<TcOutSmem *>(smem_raw);
     const int c = blockIdx.x, h = blockIdx.y;
     const long long b = blockIdx.z;
     const long long t0 = (long long)c * kQ;
     const int nq = (int)min((long long)kQ, p.seqlen - t0);
-    const int t = threadIdx.x, warp = t >> 5;
+    const int t = threadIdx.x, warp = t >> 5, r = t & (kQ - 1), hh = t / kQ;
     const int N = p.dstate, P = p.headdim;
     const long long D = (long long)p.nheads * P;
+    const bool live = r < nq;
+    const long long row = b * p.seqlen + t0 + r;
+    const long long bh = b * p.nheads + h;
+    const uint32_t lane_q = (uint32_t)((warp & 3) * 32) << 16;  // this warp's 32 lanes
 
     if (warp == 0) tmem_alloc(&S.tmem, 256);
     if (t == 0) {
         mbar_init(&S.bar[0], 1);
         mbar_init(&S.bar[1], 1);
+        mbar_init(&S.bar[2], 1);
         fence_barrier_init();
+        // h_in's (high, low) block for this chunk, already in operand layout
+        mbar_arrive_expect_tx(&S.bar[2], 32768);
+        bulk_load(S.HX, reinterpret_cast<const char *>(p.state_in) + (bh * p.nchunks + c) * 32768ll,
+                  32768, &S.bar[2]);
     }
-    S.dt[t] = chunk_delta(p, b, h, t0, nq, S.acum, S.wsum);
-
+    // this thread's halves of rows i = j = r of C and B (asynchronous
+    // copies), and of x row r into registers
+    stage_row<kNp>(S.C, r, hh * (kNp / 16), (hh + 1) * (kNp / 16),
+                   static_cast<const bf16 *>(p.C) + row * N, static_cast<const bf16 *>(p.C), live,
+                   N, p.vec_bc);
+    stage_row<kNp>(S.BM, r, hh * (kNp / 16), (hh + 1) * (kNp / 16),
+                   static_cast<const bf16 *>(p.B) + row * N, static_cast<const bf16 *>(p.B), live,
+                   N, p.vec_bc);
+    cp_async_commit();
+    uint4 xr[kPp / 16];
     {
-        const bool live = t < nq;
-        const long long row = b * p.seqlen + t0 + t;
-        const bf16 *crow = static_cast<const bf16 *>(p.C) + row * N;
-        const bf16 *brow = static_cast<const bf16 *>(p.B) + row * N;
-#pragma unroll 4
-        for (int k8 = 0; k8 < kNp / 8; ++k8) {
-            const uint4 z4 = make_uint4(0, 0, 0, 0);
-            st_smem16(S.C, core_off<kNp>(t, 8 * k8), live ? ld8(crow, 8 * k8, N, p.vec_bc) : z4);
-            st_smem16(S.BM, core_off<kNp>(t, 8 * k8), live ? ld8(brow, 8 * k8, N, p.vec_bc) : z4);
-        }
-        // h_in row n = t (float32, zero for n ≥ d_state and p ≥ headdim) as a
-        // bfloat16 pair: the carried state can dominate y early in a chunk
-        const float *hrow = p.state_in + (((b * p.nheads + h) * p.nchunks + c) * 128 + t) * 64;
+        const bf16 *xrow = static_cast<const bf16 *>(p.x) + row * D + (long long)h * P;
 #pragma unroll
-        for (int k8 = 0; k8 < kPp / 8; ++k8) {
-            const float4 u = __ldg(reinterpret_cast<const float4 *>(hrow + 8 * k8));
-            const float4 v = __ldg(reinterpret_cast<const float4 *>(hrow + 8 * k8 + 4));
-            const float f[8] = {u.x, u.y, u.z, u.w, v.x, v.y, v.z, v.w};
-            uint4 hi, lo;
-            split8(f, hi, lo);
-            st_smem16(S.HX, core_off<kPp>(t, 8 * k8), hi);
-            st_smem16(S.Hl, core_off<kPp>(t, 8 * k8), lo);
-        }
+        for (int k = 0; k < kPp / 16; ++k)
+            xr[k] = live ? ld8(xrow, 8 * (hh * (kPp / 16) + k), P, p.vec_x) : make_uint4(0, 0, 0, 0);
     }
-    // x row j = t, held in registers until h_in's tile is free
-    uint4 xr[kPp / 8];
-    {
-        const bf16 *xrow = static_cast<const bf16 *>(p.x) + (b * p.seqlen + t0 + t) * D +
-                           (long long)h * P;
-#pragma unroll
-        for (int k8 = 0; k8 < kPp / 8; ++k8)
-            xr[k8] = t < nq ? ld8(xrow, 8 * k8, P, p.vec_x) : make_uint4(0, 0, 0, 0);
-    }
+    chunk_delta(p, b, h, t0, nq, S.dt, S.acum2, S.wsum);
+    cp_async_wait_all();
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
@@ -384,61 +487,68 @@ __global__ void __launch_bounds__(kThr) ssd_tc_out_kernel(const SsdParams p) {
     const int ksteps_n = (N + 15) / 16;  // K = d_state in steps of 16 (zero-padded)
     constexpr uint32_t kRowN = (kNp / 8) * 128, kRowP = (kPp / 8) * 128;
 
+    bool ok = true;
     if (t == 0) {
+        ok = wait_mma(&S.bar[2], 0, p.status);  // h_in landed
+        tc_fence_after();
         // G = C·Bᵀ: A = C (M = token i, K = n, K-major), B = B (N = token j, K = n, K-major)
         // C·h_in:  A = C, B = h_in (N = channel p contiguous, K = n: M/N-major)
         const uint32_t c0 = smem_addr(S.C), b0 = smem_addr(S.BM);
-        const uint32_t hh = smem_addr(S.HX), hl = smem_addr(S.Hl);
-        for (int k = 0; k < ksteps_n; ++k) {
+        const uint32_t hh0 = smem_addr(S.HX), hl0 = smem_addr(S.Hl);
+        for (int k = 0; ok && k < ksteps_n; ++k) {
             const uint64_t a = umma_desc(c0 + k * 256, 128, kRowN);
             umma_bf16(tmem + kColG, a, umma_desc(b0 + k * 256, 128, kRowN),
                       idesc_bf16(128, 128, 0, 0), k > 0);
-            umma_bf16(tmem + kColYo, a, umma_desc(hh + k * 2 * kRowP, kRowP, 128),
+            umma_bf16(tmem + kColYo, a, umma_desc(hh0 + k * 2 * kRowP, kRowP, 128),
                       idesc_bf16(128, kPp, 0, 1), k > 0);
-            umma_bf16(tmem + kColYo, a, umma_desc(hl + k * 2 * kRowP, kRowP, 128),
+            umma_bf16(tmem + kColYo, a, umma_desc(hl0 + k * 2 * kRowP, kRowP, 128),
                       idesc_bf16(128, kPp, 0, 1), 1);
         }
         umma_commit(&S.bar[0]);
     }
-    bool ok = __syncthreads_and(wait_mma(&S.bar[0], 0, p.status));
+    ok = __syncthreads_and(ok && wait_mma(&S.bar[0], 0, p.status));
     tc_fence_after();
 
-    // M row i = t from G row i: (C_i·B_j)·exp(Acum_i − Acum_j)·Δ_j for j ≤ i,
-    // stored as two bfloat16 parts M = M_hi + M_lo (M_hi into the B tile, M_lo
-    // into the C tile: both are free once the first MMAs are done). Single
-    // products M_ij·x_j can be far larger than y_i, so one bfloat16 rounding
-    // of M would cost more than the output's own rounding; the pair keeps
-    // about 16 significant bits.
+    // z row r (this thread's half) into h_in's low tile (its MMAs are done)
+    if (kGate) {
+        stage_row<kPp>(S.Hl, r, hh * (kPp / 16), (hh + 1) * (kPp / 16),
+                       static_cast<const bf16 *>(p.z) + row * D + (long long)h * P,
+                       static_cast<const bf16 *>(p.z), live, P, p.vec_x);
+        cp_async_commit();
+    }
+    // M row i = r, columns j in this thread's half, from G row i:
+    // (C_i·B_j)·exp(Acum_i − Acum_j)·Δ_j for j ≤ i, stored as two bfloat16
+    // parts M = M_hi + M_lo (M_hi into the B tile, M_lo into the C tile: both
+    // are free once the first MMAs are done). Single products M_ij·x_j can be
+    // far larger than y_i, so one bfloat16 rounding of M would cost more than
+    // the output's own rounding; the pair keeps about 16 significant bits.
     if (ok) {
-        const float ai = S.acum[t];
-        const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+        const float ai = S.acum2[r];
 #pragma unroll 1
-        for (int cb = 0; cb < kQ / 32; ++cb) {
+        for (int cb = 2 * hh; cb < 2 * hh + 2; ++cb) {
             float g[32];
-            tmem_ld32(lane_base + kColG + 32 * cb, g);
+            tmem_ld32(tmem + lane_q + kColG + 32 * cb, g);
 #pragma unroll
             for (int k8 = 0; k8 < 4; ++k8) {
-                float m[8], r[8];
+                float m[8];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
                     const int j = 32 * cb + 8 * k8 + e;
-                    m[e] = (j <= t && t < nq) ? g[8 * k8 + e] * __expf(ai - S.acum[j]) * S.dt[j]
-                                              : 0.0f;
-                    r[e] = m[e] - __bfloat162float(__float2bfloat16_rn(m[e]));
+                    m[e] = (j <= r && live) ? g[8 * k8 + e] * ex2_approx(ai - S.acum2[j]) * S.dt[j]
+                                            : 0.0f;
                 }
-                const uint32_t off = core_off<kQ>(t, 32 * cb + 8 * k8);
-                st_smem16(S.BM, off,
-                          make_uint4(pack_bf16x2(m[0], m[1]), pack_bf16x2(m[2], m[3]),
-                                     pack_bf16x2(m[4], m[5]), pack_bf16x2(m[6], m[7])));
-                st_smem16(S.C, off,
-                          make_uint4(pack_bf16x2(r[0], r[1]), pack_bf16x2(r[2], r[3]),
-                                     pack_bf16x2(r[4], r[5]), pack_bf16x2(r[6], r[7])));
+                uint4 hi, lo;
+                split8(m, hi, lo);
+                const uint32_t off = core_off<kQ>(r, 32 * cb + 8 * k8);
+                st_smem16(S.BM, off, hi);
+                st_smem16(S.C, off, lo);
             }
         }
     }
-    // X row j = t into the h_in tile (its MMAs are done)
+    // X row j = r (this thread's half) into h_in's high tile
 #pragma unroll
-    for (int k8 = 0; k8 < kPp / 8; ++k8) st_smem16(S.HX, core_off<kPp>(t, 8 * k8), xr[k8]);
+    for (int k = 0; k < kPp / 16; ++k)
+        st_smem16(S.HX, core_off<kPp>(r, 8 * (hh * (kPp / 16) + k)), xr[k]);
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
@@ -458,52 +568,42 @@ __global__ void __launch_bounds__(kThr) ssd_tc_out_kernel(const SsdParams p) {
                       umma_desc(x0 + k * 2 * kRowP, kRowP, 128), idesc_bf16(128, kPp, 0, 1), 1);
         umma_commit(&S.bar[1]);
     }
+    if (kGate) cp_async_wait_all();  // this thread's part of z row r
     ok = __syncthreads_and(ok && wait_mma(&S.bar[1], 0, p.status));
     tc_fence_after();
 
     // every lane loads its accumulator rows (tcgen05.ld is warp-wide); rows
-    // past the sequence end store nothing
-    if (ok) {
-        const bool live = t < nq;
-        const long long row = b * p.seqlen + t0 + t;
-        const bf16 *xrow = static_cast<const bf16 *>(p.x) + row * D + (long long)h * P;
-        const bf16 *zrow = kGate ? static_cast<const bf16 *>(p.z) + row * D + (long long)h * P
-                                 : nullptr;
+    // past the sequence end store nothing. x and z come from shared memory.
+    if (ok && 32 * hh < P) {
         bf16 *yrow = static_cast<bf16 *>(p.y) + row * D + (long long)h * P;
-        const float dec = __expf(S.acum[t]);
+        const float dec = ex2_approx(S.acum2[r]);
         const float dsk = p.Dskip ? p.Dskip[h] : 0.0f;
-        const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
-#pragma unroll 1
-        for (int half = 0; half < 2; ++half) {
-            if (32 * half >= P) break;
-            float yd[32], yo[32];
-            tmem_ld32(lane_base + kColYd + 32 * half, yd);
-            tmem_ld32(lane_base + kColYo + 32 * half, yo);
+        float yd[32], yo[32];
+        tmem_ld32(tmem + lane_q + kColYd + 32 * hh, yd);
+        tmem_ld32(tmem + lane_q + kColYo + 32 * hh, yo);
 #pragma unroll
-            for (int k8 = 0; k8 < 4; ++k8) {
-                const int c0 = 32 * half + 8 * k8;
-                if (c0 >= P) break;
-                float xv[8] = {}, zv[8] = {}, o[8];
-                if (live) {
-                    unpack8(ld8(xrow, c0, P, p.vec_x), xv);
-                    if (kGate) unpack8(ld8(zrow, c0, P, p.vec_x), zv);
-                }
+        for (int k8 = 0; k8 < 4; ++k8) {
+            const int c0 = 32 * hh + 8 * k8;
+            if (c0 >= P || !live) break;
+            const uint32_t off = core_off<kPp>(r, c0);
+            float xv[8], zv[8], o[8];
+            unpack8(*reinterpret_cast<const uint4 *>(reinterpret_cast<const char *>(S.HX) + off), xv);
+            if (kGate)
+                unpack8(*reinterpret_cast<const uint4 *>(reinterpret_cast<const char *>(S.Hl) + off), zv);
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    float v = fmaf(dec, yo[8 * k8 + e], yd[8 * k8 + e]) + dsk * xv[e];
-                    if (kGate) v *= silu_f32(zv[e]);
-                    o[e] = v;
-                }
-                if (!live) continue;
-                if (p.vec_x && c0 + 8 <= P) {
-                    *reinterpret_cast<uint4 *>(yrow + c0) =
-                        make_uint4(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]),
-                                   pack_bf16x2(o[4], o[5]), pack_bf16x2(o[6], o[7]));
-                } else {
+            for (int e = 0; e < 8; ++e) {
+                float v = fmaf(dec, yo[8 * k8 + e], yd[8 * k8 + e]) + dsk * xv[e];
+                if (kGate) v *= silu_f32(zv[e]);
+                o[e] = v;
+            }
+            if (p.vec_x && c0 + 8 <= P) {
+                *reinterpret_cast<uint4 *>(yrow + c0) =
+                    make_uint4(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]),
+                               pack_bf16x2(o[4], o[5]), pack_bf16x2(o[6], o[7]));
+            } else {
 #pragma unroll
-                    for (int e = 0; e < 8; ++e)
-                        if (c0 + e < P) yrow[c0 + e] = __float2bfloat16_rn(o[e]);
-                }
+                for (int e = 0; e < 8; ++e)
+                    if (c0 + e < P) yrow[c0 + e] = __float2bfloat16_rn(o[e]);
             }
         }
     }
@@ -536,7 +636,13 @@ cudaError_t launch_ssd_tc_state(const SsdParams &p, cudaStream_t stream) {
         configured[dev] = true;
     }
     const dim3 grid((unsigned)p.nchunks, (unsigned)p.nheads, (unsigned)p.batch);
-    ssd_tc_state_kernel<<<grid, kThr, sizeof(TcStateSmem), stream>>>(p);
+    ssd_tc_state_kernel<<<grid, kThrTc, sizeof(TcStateSmem), stream>>>(p);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_ssd_tc_carry(const SsdParams &p, cudaStream_t stream) {
+    const long long n = (long long)p.batch * p.nheads * kNp * (kPp / 8);
+    ssd_tc_carry_kernel<<<(unsigned)((n + 255) / 256), 256, 0, stream>>>(p);
     return cudaGetLastError();
 }
 
@@ -553,9 +659,9 @@ cudaError_t launch_ssd_tc_out(const SsdParams &p, cudaStream_t stream) {
     }
     const dim3 grid((unsigned)p.nchunks, (unsigned)p.nheads, (unsigned)p.batch);
     if (p.z)
-        ssd_tc_out_kernel<true><<<grid, kThr, sizeof(TcOutSmem), stream>>>(p);
+        ssd_tc_out_kernel<true><<<grid, kThrTc, sizeof(TcOutSmem), stream>>>(p);
     else
-        ssd_tc_out_kernel<false><<<grid, kThr, sizeof(TcOutSmem), stream>>>(p);
+        ssd_tc_out_kernel<false><<<grid, kThrTc, sizeof(TcOutSmem), stream>>>(p);
     return cudaGetLastError();
 }
 

@@ -6,10 +6,12 @@ the device) and to give quick CUDA-event timings without one:
     python -m selective_state_space_42_b200.profile_case scan mamba2p8b_layer --launches 2
     python -m selective_state_space_42_b200.profile_case decode --launches 3
     python -m selective_state_space_42_b200.profile_case bwd mamba2p8b_layer --launches 2
+    python -m selective_state_space_42_b200.profile_case ssd --launches 3
 
 ``scan`` calls selscan_fwd on a scan workload; ``bwd`` calls selscan_bwd on
 it (with a seeded dy and final-state gradient); ``decode`` calls
-selscan_state_update on the decode workload. With ``--time`` it also prints
+selscan_state_update on the decode workload; ``ssd`` calls selscan_ssd_fwd
+on the Mamba-2-shaped head workload. With ``--time`` it also prints
 the median CUDA-event time per launch, cold (a 512 MiB buffer is written
 between launches, which evicts L2) and back to back, as one JSON line.
 """
@@ -69,6 +71,19 @@ def _decode_case():
     return launch, w.algorithmic_bytes_per_step()
 
 
+def _ssd_case():
+    w = wl.SSD
+    inp = wl.make_ssd_inputs(w, device="cuda")
+    y = torch.empty_like(inp["x"])
+    fs = torch.empty(w.batch, w.dim, w.dstate, device="cuda")
+
+    def launch(_i: int) -> None:
+        ss.selscan_ssd_fwd(inp["x"], inp["dt"], inp["A"], inp["B"], inp["C"], D=inp["D"],
+                           z=inp["z"], dt_bias=inp["dt_bias"], y=y, final_state=fs)
+
+    return launch, w.algorithmic_bytes()
+
+
 def _median(v):
     v = sorted(v)
     return v[len(v) // 2]
@@ -76,7 +91,7 @@ def _median(v):
 
 def main(argv=None) -> int:
     ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
-    ap.add_argument("kernel", choices=["scan", "bwd", "decode"])
+    ap.add_argument("kernel", choices=["scan", "bwd", "decode", "ssd"])
     ap.add_argument("workload", nargs="?", default="mamba2p8b_layer",
                     help="scan workload name (ignored for decode)")
     ap.add_argument("--launches", type=int, default=2)
@@ -87,13 +102,16 @@ def main(argv=None) -> int:
         launch, nbytes = _scan_case(args.workload)
     elif args.kernel == "bwd":
         launch, nbytes = _bwd_case(args.workload)
+    elif args.kernel == "ssd":
+        launch, nbytes = _ssd_case()
     else:
         launch, nbytes = _decode_case()
     for i in range(args.launches):
         launch(i)
     torch.cuda.synchronize()
     out = {"kernel": args.kernel, "launches": args.launches,
-           "workload": wl.DECODE.name if args.kernel == "decode" else args.workload,
+           "workload": {"decode": wl.DECODE.name, "ssd": wl.SSD.name}.get(args.kernel,
+                                                                          args.workload),
            "algorithmic_bytes": nbytes}
     if args.time:
         flush = torch.empty(512 << 20, dtype=torch.uint8, device="cuda")

@@ -98,6 +98,47 @@ class DecodeWorkload:
         return self.batch * self.dim * self.dstate
 
 
+@dataclasses.dataclass(frozen=True)
+class SsdWorkload:
+    """One scalar A per head (the Mamba-2 form): x, z, y [batch, L, nheads·headdim],
+    dt [batch, L, nheads], B, C [batch, L, dstate]."""
+    name: str
+    batch: int
+    seqlen: int
+    nheads: int
+    headdim: int
+    dstate: int
+    dtype: str
+    gate: bool
+    seed: int
+
+    @property
+    def dim(self) -> int:
+        return self.nheads * self.headdim
+
+    def algorithmic_bytes(self) -> int:
+        """x, z in and y out per (b, l, d); dt per (b, l, head); B and C per
+        (b, l); the float32 final state; A, D, dt_bias per head."""
+        es = 4 if self.dtype == "f32" else 2
+        bl = self.batch * self.seqlen
+        return (bl * self.dim * (3 if self.gate else 2) * es + bl * self.nheads * es
+                + 2 * bl * self.dstate * es + self.batch * self.dim * self.dstate * 4
+                + 3 * self.nheads * 4)
+
+    def algorithmic_flops(self, chunk: int = 128) -> int:
+        """Multiply-adds ×2 of the chunked form at `chunk` tokens per chunk, per
+        head: C·Bᵀ (q×q×N), M·X (q×q×P), C·h_in (q×N×P), Bᵀ·(w∘X) (N×q×P)."""
+        total = 0
+        for c0 in range(0, self.seqlen, chunk):
+            q = min(chunk, self.seqlen - c0)
+            total += 2 * (q * q * self.dstate + q * q * self.headdim
+                          + 2 * q * self.dstate * self.headdim)
+        return total * self.batch * self.nheads
+
+
+SSD = SsdWorkload("mamba2_ssd_layer", 2, 4096, 32, 64, 128, "bf16", gate=True, seed=5)
+
+
 WORKLOADS: Dict[str, ScanWorkload] = {
     # tiny fp32 scan, no gate, D = 1
     "tiny_f32": ScanWorkload("tiny_f32", 1, 256, 64, 16, "f32", gate=False,
@@ -157,6 +198,28 @@ def make_scan_inputs(w: ScanWorkload, device="cpu") -> Dict[str, torch.Tensor]:
     out["C"] = _randn(bshp, g, device).to(dt)
     out["A"], out["D"], out["delta_bias"] = param_tensors(
         w.dim, w.dstate, g, device, w.skip_ones)
+    return out
+
+
+def make_ssd_inputs(w: SsdWorkload, device="cpu") -> Dict[str, torch.Tensor]:
+    """Inputs of one selscan_ssd_fwd call from one generator seeded with
+    ``w.seed``: x, z, B, C ~ N(0, 1); dt ~ 0.5·N(0, 1) (softplus applied in
+    the kernel); per head A ~ −U[0.5, 4], D = 1 + 0.1·N(0, 1) and dt_bias =
+    log(expm1(U[1e-3, 1e-1]))."""
+    dt = DTYPES[w.dtype]
+    g = _gen(w.seed, device)
+    shp = (w.batch, w.seqlen, w.dim)
+    bshp = (w.batch, w.seqlen, w.dstate)
+    out = {}
+    out["x"] = _randn(shp, g, device).to(dt)
+    out["dt"] = _randn((w.batch, w.seqlen, w.nheads), g, device, 0.5).to(dt)
+    out["z"] = _randn(shp, g, device).to(dt) if w.gate else None
+    out["B"] = _randn(bshp, g, device).to(dt)
+    out["C"] = _randn(bshp, g, device).to(dt)
+    out["A"] = -(torch.rand(w.nheads, generator=g, device=device) * 3.5 + 0.5)
+    out["D"] = _randn((w.nheads,), g, device, 0.1).add_(1.0)
+    u = torch.rand(w.nheads, generator=g, device=device, dtype=torch.float64)
+    out["dt_bias"] = torch.log(torch.expm1(1e-3 + (1e-1 - 1e-3) * u)).to(torch.float32)
     return out
 
 
