@@ -389,19 +389,34 @@ __global__ void ssd_tc_carry_kernel(const SsdParams p) {
                     ? p.h0[((b * p.nheads + h) * (long long)P + pp) * N + n] : 0.0f;
     }
     const uint32_t off = core_off<kPp>(n, 8 * pg);
-    for (int c = 0; c < p.nchunks; ++c) {
-        char *blk = reinterpret_cast<char *>(p.state_in) + (bh * p.nchunks + c) * 32768ll;
-        uint4 hi, lo;
-        split8(st, hi, lo);
-        *reinterpret_cast<uint4 *>(blk + off) = hi;
-        *reinterpret_cast<uint4 *>(blk + 16384 + off) = lo;
-        const float dec = p.chunk_decay[bh * p.nchunks + c];
-        const float *cs = p.chunk_state + ((bh * p.nchunks + c) * 128 + n) * 64 + 8 * pg;
-        const float4 u = *reinterpret_cast<const float4 *>(cs);
-        const float4 v = *reinterpret_cast<const float4 *>(cs + 4);
-        const float s8[8] = {u.x, u.y, u.z, u.w, v.x, v.y, v.z, v.w};
+    char *blk0 = reinterpret_cast<char *>(p.state_in) + bh * p.nchunks * 32768ll;
+    const float *cs0 = p.chunk_state + (bh * p.nchunks * 128 + n) * 64 + 8 * pg;
+    const float *dec0 = p.chunk_decay + bh * p.nchunks;
+    // groups of kAhead chunks: every load of a group is issued before the
+    // group's dependent updates, so the chain waits once per group
+    constexpr int kAhead = 4;
+    for (int c0 = 0; c0 < p.nchunks; c0 += kAhead) {
+        float4 u[kAhead], v[kAhead];
+        float dec[kAhead];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) st[k] = fmaf(dec, st[k], s8[k]);
+        for (int k = 0; k < kAhead; ++k) {
+            const int c = min(c0 + k, p.nchunks - 1);
+            u[k] = __ldg(reinterpret_cast<const float4 *>(cs0 + (long long)c * 128 * 64));
+            v[k] = __ldg(reinterpret_cast<const float4 *>(cs0 + (long long)c * 128 * 64 + 4));
+            dec[k] = __ldg(dec0 + c);
+        }
+#pragma unroll
+        for (int k = 0; k < kAhead; ++k) {
+            if (c0 + k >= p.nchunks) break;
+            uint4 hi, lo;
+            split8(st, hi, lo);
+            char *blk = blk0 + (long long)(c0 + k) * 32768;
+            *reinterpret_cast<uint4 *>(blk + off) = hi;
+            *reinterpret_cast<uint4 *>(blk + 16384 + off) = lo;
+            const float s8[8] = {u[k].x, u[k].y, u[k].z, u[k].w, v[k].x, v[k].y, v[k].z, v[k].w};
+#pragma unroll
+            for (int e = 0; e < 8; ++e) st[e] = fmaf(dec[k], st[e], s8[e]);
+        }
     }
     if (p.final_state && n < N) {
 #pragma unroll
