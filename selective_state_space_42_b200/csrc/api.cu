@@ -9,6 +9,7 @@
 
 #include "selscan.h"
 #include "selscan_device.cuh"
+#include "ssd_params.cuh"
 
 namespace {
 

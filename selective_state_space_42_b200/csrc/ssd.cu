@@ -23,7 +23,7 @@
 // The products are FP32 (register-blocked 4×4 per thread from shared memory);
 // chunks are independent, so the whole sequence runs in parallel except for
 // the element-wise carry.
-#include "selscan_device.cuh"
+#include "ssd_params.cuh"
 
 namespace selscan {
 namespace {

@@ -31,7 +31,7 @@
 // eight rows of 16 bytes along the tile's contiguous dimension. Accumulators
 // are float32 in tensor memory; one elected thread issues every MMA and a
 // tcgen05.commit to an mbarrier tells the CTA they are done.
-#include "selscan_device.cuh"
+#include "ssd_params.cuh"
 #include "tma_util.cuh"
 
 #include <cstddef>
