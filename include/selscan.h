@@ -447,8 +447,14 @@ SELSCAN_API int selscan_state_update_ex(float *state, const void *x, const void 
  *   B, C          [batch, seqlen, dstate]           dtype   (one group)
  *   initial_state, final_state [batch, nheads·headdim, dstate] float32, nullable
  *   headdim 1..64, dstate 1..128, batch and nheads ≤ 65535.
- * Chunks of 64 tokens; workspace (NULL: allocated on the stream) of
- * selscan_ssd_workspace_bytes() bytes.
+ * float32 I/O: 64-token chunks, products in float32 on the CUDA cores.
+ * bfloat16 I/O: 128-token chunks on the tensor cores (tcgen05, float32
+ * accumulators); the operands that are not inputs (the masked decay matrix
+ * M, w ◦ x for the chunk states, the carried state h_in) are split into
+ * bfloat16 high/low pairs, so the products keep about 16 significant bits.
+ * Workspace (NULL: allocated on the stream) of selscan_ssd_workspace_bytes()
+ * bytes; the caller owns every buffer. No output may overlap an input
+ * (SELSCAN_ERR_ALIAS). Asynchronous like selscan_fwd.
  */
 SELSCAN_API int selscan_ssd_fwd(const void *x, const void *dt, const float *A, const void *B,
                                 const void *C, const float *D, const void *z,
@@ -467,7 +473,8 @@ SELSCAN_API int64_t selscan_ssd_workspace_bytes(int64_t batch, int64_t seqlen, i
  * the current device (synchronous: waits for prior work). 0 means no device
  * wait has given up; otherwise the code of the first one that did (1: a
  * sequence chunk waited too long for its predecessor's state; 2, 3: a
- * pipeline stage waited too long). Every device-side wait in the library is
+ * pipeline stage waited too long; 4: a tensor-core MMA or its operand copy
+ * of selscan_ssd_fwd did not complete in time). Every device-side wait in the library is
  * bounded (2 s); a wait that gives up records its code here and the kernel
  * returns instead of hanging, leaving its outputs undefined. `clear` nonzero
  * resets the word to 0 after reading it.
