@@ -203,3 +203,51 @@ def test_plans_of_the_workloads(lib):
     assert p["launches"] == 1 and p["chunks"] == 2  # 96 groups: enough for one pass
     p = ss.selscan_fwd_plan(1, 8192, 1536, 16)  # 12 groups: chunked
     assert p["launches"] == 3
+
+
+def ssd(lib, **kw):
+    names = ["x", "dt", "A", "B", "C", "D", "z", "dt_bias", "h0", "y", "final"]
+    a = {n: P + 4096 * i for i, n in enumerate(names)}
+    a.update(D=None, z=None, dt_bias=None, h0=None, final=None, softplus=1, batch=0,
+             seqlen=8, nheads=2, headdim=4, dstate=16, dtype=1, ws=None, wsb=0, stream=None)
+    a.update(kw)
+    return lib.selscan_ssd_fwd(a["x"], a["dt"], a["A"], a["B"], a["C"], a["D"], a["z"],
+                               a["dt_bias"], a["softplus"], a["h0"], a["y"], a["final"],
+                               a["batch"], a["seqlen"], a["nheads"], a["headdim"],
+                               a["dstate"], a["dtype"], a["ws"], a["wsb"], a["stream"])
+
+
+def test_ssd_validation(lib):
+    """Every check of selscan_ssd_fwd runs before any CUDA call (no GPU here)."""
+    assert ssd(lib) == 0  # batch = 0: no output has an element
+    assert ssd(lib, dtype=7) == -3
+    assert ssd(lib, batch=-1) == -2
+    assert ssd(lib, seqlen=-1) == -2
+    assert ssd(lib, headdim=0) == -2
+    assert ssd(lib, headdim=65) == -2  # one head's channels fit one 64-wide tile
+    assert ssd(lib, nheads=70000) == -2  # heads are a grid dimension
+    assert ssd(lib, dstate=0) == -5
+    assert ssd(lib, dstate=129) == -5  # d_state fits one 128-wide tile
+    full = dict(batch=1)
+    for name in ("x", "dt", "A", "B", "C", "y"):
+        assert ssd(lib, **{name: None}, **full) == -1, name
+    assert ssd(lib, x=P + 1, **full) == -4  # bf16 element alignment
+    assert ssd(lib, A=P + 4096 * 2 + 2, **full) == -4
+    assert ssd(lib, ws=P + 4096 * 64 + 16, wsb=1 << 20, **full) == -4  # 256-byte workspace
+    assert ssd(lib, y=P, **full) == -7  # y == x
+    assert ssd(lib, final=P + 4096 * 3, **full) == -7  # the final state runs into B
+    assert ssd(lib, ws=P + 4096 * 64, wsb=16, **full) == -8  # too small
+    need = lib.selscan_ssd_workspace_bytes(1, 8, 2, 4, 16)
+    assert ssd(lib, ws=P + 4096 * 3, wsb=need, **full) == -7  # workspace runs into B
+
+
+def test_ssd_workspace_bytes(lib):
+    assert lib.selscan_ssd_workspace_bytes(0, 8, 2, 4, 16) == 0
+    assert lib.selscan_ssd_workspace_bytes(1, 8, 2, 65, 16) == 0
+    assert lib.selscan_ssd_workspace_bytes(1, 8, 2, 4, 129) == 0
+    # one 64-token chunk, 2 heads: partial output 8·8·4 B; chunk states and
+    # carried states 2·128·64·4 B each; decays 2·4 B; each rounded up to 256 B
+    assert lib.selscan_ssd_workspace_bytes(1, 8, 2, 4, 16) == 256 + 65536 + 256 + 65536
+    # the tensor-core path (128-token chunks) fits in the float32 path's layout
+    assert (lib.selscan_ssd_workspace_bytes(2, 1000, 4, 64, 128)
+            >= 2 * 4 * 8 * 32768 * 2)

@@ -101,3 +101,85 @@ def test_ssd_equals_wide_scan_on_a_head_layer():
                                   n(inp["z"][:, :, chans]), n(inp["dt_bias"])[heads])
     gh.compare(gh.to_np(y[:, :, chans]), yo, gh.RTOL["bf16"], "ssd layer y")
     gh.compare(gh.to_np(hf[:, chans]), ho, gh.RTOL["bf16"], "ssd layer state")
+
+
+def _misaligned(t):
+    """A copy of t whose data starts one element past a 16-byte boundary."""
+    buf = torch.empty(t.numel() + 8, dtype=t.dtype, device=t.device)
+    out = buf[1:1 + t.numel()].view(t.shape)
+    out.copy_(t)
+    return out
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_ssd_options(dtype):
+    """Initial state without the gate, softplus off (positive Δ), no D and no
+    dt_bias, on 3 chunks of the bf16 path (2 of 64 + 1 of the f32 path)."""
+    inp = _inputs(2, 300, 3, 64, 128, dtype, seed=7300, gate=False)
+    g = torch.Generator().manual_seed(7301)
+    h0 = torch.randn(2, 3 * 64, 128, generator=g) * 0.3
+    y, hf = _gpu(inp, h0.to(DEV))
+    torch.cuda.synchronize()
+    yo, ho = _oracle(inp, 64, h0)
+    gh.compare(gh.to_np(y), yo, gh.RTOL[dtype], "h0 no gate y")
+    gh.compare(gh.to_np(hf), ho, gh.RTOL[dtype], "h0 no gate final state")
+
+    inp2 = dict(inp)
+    inp2["dt"] = (inp["dt"].float().abs() * 0.2 + 0.01).to(inp["dt"].dtype)
+    inp2["Dh"] = torch.zeros_like(inp["Dh"])
+    inp2["dt_bias"] = torch.zeros_like(inp["dt_bias"])
+    d = {k: (None if v is None else v.to(DEV)) for k, v in inp2.items()}
+    y2, h2 = ss.selscan_ssd_fwd(d["x"], d["dt"], d["A"], d["B"], d["C"], softplus=False,
+                                return_final_state=True)
+    torch.cuda.synchronize()
+    n = gh.to_np
+    A_full = np.repeat(n(inp2["A"])[:, None], 64, axis=0).repeat(128, axis=1)
+    yo2, ho2 = oracle.default().fwd(n(inp2["x"]), np.repeat(n(inp2["dt"]), 64, axis=-1),
+                                    A_full, n(inp2["B"]), n(inp2["C"]), None, None, None,
+                                    softplus=False)
+    gh.compare(gh.to_np(y2), yo2, gh.RTOL[dtype], "no softplus, D, bias y")
+    gh.compare(gh.to_np(h2), ho2, gh.RTOL[dtype], "no softplus, D, bias final state")
+
+
+@pytest.mark.parametrize("L", [127, 128, 129, 256, 257])
+def test_ssd_chunk_edges(L):
+    """Sequence lengths at the 128-token chunk edges of the tensor-core path
+    (and 64-token edges of the float32 one)."""
+    for dtype in ("bf16", "f32"):
+        inp = _inputs(1, L, 2, 64, 64, dtype, seed=7400 + L)
+        y, hf = _gpu(inp)
+        torch.cuda.synchronize()
+        yo, ho = _oracle(inp, 64)
+        gh.compare(gh.to_np(y), yo, gh.RTOL[dtype], f"L={L} {dtype} y")
+        gh.compare(gh.to_np(hf), ho, gh.RTOL[dtype], f"L={L} {dtype} final state")
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_ssd_misaligned_rows(dtype):
+    """x, z, y, B and C one element off a 16-byte boundary: the element-wise
+    staging and store paths instead of the 16-byte copies."""
+    inp = _inputs(2, 150, 2, 64, 32, dtype, seed=7500)
+    d = {k: (None if v is None else v.to(DEV)) for k, v in inp.items()}
+    for k in ("x", "z", "B", "C"):
+        d[k] = _misaligned(d[k])
+    y = _misaligned(torch.zeros_like(d["x"]))
+    _, hf = ss.selscan_ssd_fwd(d["x"], d["dt"], d["A"], d["B"], d["C"], D=d["Dh"], z=d["z"],
+                               dt_bias=d["dt_bias"], y=y, return_final_state=True)
+    torch.cuda.synchronize()
+    yo, ho = _oracle(inp, 64)
+    gh.compare(gh.to_np(y), yo, gh.RTOL[dtype], "misaligned y")
+    gh.compare(gh.to_np(hf), ho, gh.RTOL[dtype], "misaligned final state")
+
+
+def test_ssd_rejects_unsupported_sizes():
+    x = torch.zeros(1, 4, 2 * 65, device=DEV, dtype=torch.bfloat16)
+    dt = torch.zeros(1, 4, 2, device=DEV, dtype=torch.bfloat16)
+    A = -torch.ones(2, device=DEV)
+    B = torch.zeros(1, 4, 16, device=DEV, dtype=torch.bfloat16)
+    with pytest.raises(ss.SelscanError):
+        ss.selscan_ssd_fwd(x, dt, A, B, B)  # headdim 65
+    x = torch.zeros(1, 4, 2 * 64, device=DEV, dtype=torch.bfloat16)
+    B = torch.zeros(1, 4, 129, device=DEV, dtype=torch.bfloat16)
+    with pytest.raises(ss.SelscanError):
+        ss.selscan_ssd_fwd(x, dt, A, B, B)  # d_state 129
+    assert ss.selscan_device_status() == 0
