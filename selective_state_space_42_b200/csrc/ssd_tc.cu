@@ -135,15 +135,22 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return *reinterpret_cast<const uint32_t *>(&v);
 }
 
-// Eight floats as bfloat16 pairs v = hi + lo: hi = bf16(v), lo = bf16(v − hi).
+// Eight floats as bfloat16 pairs v = hi + lo: hi is v with its low 16 bits
+// cleared (bfloat16 truncation, integer operations only) and lo = bf16(v − hi)
+// rounded to nearest (v − hi is exact in float32), so |v − hi − lo| ≤
+// 2⁻⁹·|v − hi| < 2⁻¹⁶·|v| without bias. One packed conversion per two
+// elements: the conversions share the MUFU's issue rate.
 __device__ __forceinline__ void split8(const float (&v)[8], uint4 &hi, uint4 &lo) {
-    float r[8];
+    uint32_t h[4], l[4];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) r[e] = v[e] - __bfloat162float(__float2bfloat16_rn(v[e]));
-    hi = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
-                    pack_bf16x2(v[6], v[7]));
-    lo = make_uint4(pack_bf16x2(r[0], r[1]), pack_bf16x2(r[2], r[3]), pack_bf16x2(r[4], r[5]),
-                    pack_bf16x2(r[6], r[7]));
+    for (int k = 0; k < 4; ++k) {
+        const uint32_t a = __float_as_uint(v[2 * k]) & 0xFFFF0000u;
+        const uint32_t b = __float_as_uint(v[2 * k + 1]) & 0xFFFF0000u;
+        h[k] = (a >> 16) | b;
+        l[k] = pack_bf16x2(v[2 * k] - __uint_as_float(a), v[2 * k + 1] - __uint_as_float(b));
+    }
+    hi = make_uint4(h[0], h[1], h[2], h[3]);
+    lo = make_uint4(l[0], l[1], l[2], l[3]);
 }
 
 __device__ __forceinline__ void unpack8(const uint4 &u, float (&f)[8]) {
@@ -198,36 +205,66 @@ __device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t b
         : "memory");
 }
 
-// Column chunks [k_lo, k_hi) (8 columns each) of row r of an interleaved tile
-// from a global row of ncols bfloat16 (zero past ncols, or everywhere when
-// !live): asynchronous 16-byte copies where the row allows them (vec:
-// 16-byte aligned rows, ncols a multiple of 8), else loads and stores through
-// registers. `safe` is any valid global address, named by the zero-filling
-// copies.
+constexpr int kThrTc = 256;  // threads of the two MMA kernels
+
+// Work item k of this thread in a cooperative pass over a kQ-row tile with
+// kCols columns: lane l of warp w takes row 8·g + l mod 8 and 8-column chunk
+// 4·c + l / 8 of item (g, c) = w + 8·k, so that one warp instruction touches
+// 8 row segments of 64 contiguous bytes in global memory and 4 whole core
+// matrices (512 contiguous bytes) of the tile.
 template <int kCols>
-__device__ __forceinline__ void stage_row(bf16 *tile, int r, int k_lo, int k_hi, const bf16 *row,
-                                          const bf16 *safe, bool live, int ncols, bool vec) {
-    if (vec) {
-        const uint32_t base = smem_addr(tile);
-#pragma unroll 4
-        for (int k8 = k_lo; k8 < k_hi; ++k8) {
-            const bool in = live && 8 * k8 < ncols;
-            cp_async16(base + core_off<kCols>(r, 8 * k8), in ? row + 8 * k8 : safe, in ? 16u : 0u);
-        }
-    } else {
-#pragma unroll 2
-        for (int k8 = k_lo; k8 < k_hi; ++k8)
-            st_smem16(tile, core_off<kCols>(r, 8 * k8),
-                      live ? ld8(row, 8 * k8, ncols, false) : make_uint4(0, 0, 0, 0));
+__device__ __forceinline__ void tile_item(int k, int &row, int &chunk) {
+    constexpr int kQuads = kCols / 32;
+    const int it = (int)(threadIdx.x >> 5) + (kThrTc / 32) * k;
+    row = 8 * (it / kQuads) + (int)(threadIdx.x & 7);
+    chunk = 4 * (it % kQuads) + (int)((threadIdx.x & 31) >> 3);
+}
+template <int kCols> constexpr int tile_items() { return (kQ / 8) * (kCols / 32) / (kThrTc / 32); }
+
+// The whole tile from global rows base + row·stride (ncols valid bfloat16
+// columns; rows ≥ nrows and columns ≥ ncols zero): asynchronous 16-byte
+// copies where the rows allow them (vec: 16-byte aligned rows, ncols a
+// multiple of 8), else loads and stores through registers. All threads.
+template <int kCols>
+__device__ __forceinline__ void stage_tile(bf16 *tile, const bf16 *base, long long stride,
+                                           int nrows, int ncols, bool vec) {
+    const uint32_t sbase = smem_addr(tile);
+#pragma unroll
+    for (int k = 0; k < tile_items<kCols>(); ++k) {
+        int row, chunk;
+        tile_item<kCols>(k, row, chunk);
+        const bool in = row < nrows && 8 * chunk < ncols;
+        const uint32_t off = core_off<kCols>(row, 8 * chunk);
+        if (vec)
+            cp_async16(sbase + off, in ? base + row * stride + 8 * chunk : base, in ? 16u : 0u);
+        else
+            st_smem16(tile, off, in ? ld8(base + row * stride, 8 * chunk, ncols, false)
+                                    : make_uint4(0, 0, 0, 0));
+    }
+}
+
+// This thread's items of such a tile into registers (zero outside).
+template <int kCols>
+__device__ __forceinline__ void load_tile_regs(uint4 (&v)[tile_items<kCols>()], const bf16 *base,
+                                               long long stride, int nrows, int ncols, bool vec) {
+#pragma unroll
+    for (int k = 0; k < tile_items<kCols>(); ++k) {
+        int row, chunk;
+        tile_item<kCols>(k, row, chunk);
+        v[k] = row < nrows ? ld8(base + row * stride, 8 * chunk, ncols, vec)
+                           : make_uint4(0, 0, 0, 0);
     }
 }
 
 // Δ_t of the chunk's tokens t (zero past the sequence end) into dt[], and the
 // inclusive prefix sums of Δ·A over the chunk, times log2(e), into acum2[]
-// (so exp(Acum_i − Acum_j) = 2^(acum2_i − acum2_j)). Threads 0..kQ−1 compute;
-// every thread of the block takes part in the two barriers.
+// (so exp(Acum_i − Acum_j) = 2^(acum2_i − acum2_j)). With F given, also
+// F[t] = 2^(−acum2_t)·Δ_t and the per-warp maxima of |acum2| in wmax[4].
+// Threads 0..kQ−1 compute; every thread of the block takes part in the two
+// barriers.
 __device__ __forceinline__ void chunk_delta(const SsdParams &p, long long b, int h, long long t0,
-                                            int nq, float *dt, float *acum2, float *wsum) {
+                                            int nq, float *dt, float *acum2, float *wsum,
+                                            float *F = nullptr, float *wmax = nullptr) {
     const int t = threadIdx.x, lane = t & 31, w = t >> 5;
     float d = 0.0f, s = 0.0f;
     if (t < kQ) {
@@ -249,9 +286,21 @@ __device__ __forceinline__ void chunk_delta(const SsdParams &p, long long b, int
         for (int k = 0; k < w; ++k) s += wsum[k];
         acum2[t] = s;
         dt[t] = d;
+        if (F) {
+            F[t] = ex2_approx(-s) * d;  // used only when every |acum2| ≤ kFactorMax
+            float m = fabsf(s);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+            if (lane == 0) wmax[w] = m;
+        }
     }
     __syncthreads();
 }
+
+// Largest |acum2| of a chunk for which 2^(acum2_i − acum2_j) may be taken as
+// 2^acum2_i · 2^(−acum2_j): both factors stay normal float32 numbers and
+// 2^(−acum2_j)·Δ_j stays finite for Δ_j < 2^27.
+constexpr float kFactorMax = 100.0f;
 
 __device__ __forceinline__ bool wait_mma(uint64_t *bar, uint32_t parity, int *status) {
     if (mbar_wait(bar, parity, &kNoAbortTc, kWaitNs)) return true;
@@ -260,9 +309,8 @@ __device__ __forceinline__ bool wait_mma(uint64_t *bar, uint32_t parity, int *st
 }
 
 // ---- chunk states -----------------------------------------------------------------
-// 256 threads: thread t works on row r = t mod 128 (token j while staging,
-// state n = tensor-memory lane n in the epilogue) and column half t / 128.
-constexpr int kThrTc = 256;
+// 256 threads; in the epilogue thread t reads state row n = t mod 128
+// (tensor-memory lane n), column half t / 128.
 
 struct TcStateSmem {
     bf16 Bt[kQ * kNp];  // rows token j, columns state n
@@ -285,43 +333,36 @@ __global__ void __launch_bounds__(kThrTc) ssd_tc_state_kernel(const SsdParams p)
     const int t = threadIdx.x, warp = t >> 5, r = t & (kQ - 1), hh = t / kQ;
     const int N = p.dstate, P = p.headdim;
     const long long D = (long long)p.nheads * P;
-    const bool live = r < nq;
-    const long long row = b * p.seqlen + t0 + r;
 
     if (warp == 0) tmem_alloc(&S.tmem, 64);
     if (t == 0) {
         mbar_init(&S.bar, 1);
         fence_barrier_init();
     }
-    // row j = r of B: this thread's half of the states, asynchronously
-    stage_row<kNp>(S.Bt, r, hh * (kNp / 16), (hh + 1) * (kNp / 16),
-                   static_cast<const bf16 *>(p.B) + row * N, static_cast<const bf16 *>(p.B), live,
-                   N, p.vec_bc);
+    // the chunk's B rows (asynchronously) and x rows (into registers)
+    const long long row0 = b * p.seqlen + t0;
+    stage_tile<kNp>(S.Bt, static_cast<const bf16 *>(p.B) + row0 * N, N, nq, N, p.vec_bc);
     cp_async_commit();
-    uint4 xr[kPp / 16];
-    {
-        const bf16 *xrow = static_cast<const bf16 *>(p.x) + row * D + (long long)h * P;
-#pragma unroll
-        for (int k = 0; k < kPp / 16; ++k)
-            xr[k] = live ? ld8(xrow, 8 * (hh * (kPp / 16) + k), P, p.vec_x) : make_uint4(0, 0, 0, 0);
-    }
+    uint4 xr[tile_items<kPp>()];
+    load_tile_regs<kPp>(xr, static_cast<const bf16 *>(p.x) + row0 * D + (long long)h * P, D, nq,
+                        P, p.vec_x);
     chunk_delta(p, b, h, t0, nq, S.dt, S.acum2, S.wsum);
     const float aend2 = S.acum2[kQ - 1];
     // w_j ◦ x_j as a bfloat16 pair (0 past the sequence end: Δ = 0)
-    {
-        const float w = ex2_approx(aend2 - S.acum2[r]) * S.dt[r];
 #pragma unroll
-        for (int k = 0; k < kPp / 16; ++k) {
-            float f[8];
-            unpack8(xr[k], f);
+    for (int k = 0; k < tile_items<kPp>(); ++k) {
+        int j, chunk;
+        tile_item<kPp>(k, j, chunk);
+        const float w = ex2_approx(aend2 - S.acum2[j]) * S.dt[j];
+        float f[8];
+        unpack8(xr[k], f);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) f[e] *= w;
-            uint4 hi, lo;
-            split8(f, hi, lo);
-            const uint32_t off = core_off<kPp>(r, 8 * (hh * (kPp / 16) + k));
-            st_smem16(S.Xw, off, hi);
-            st_smem16(S.Xl, off, lo);
-        }
+        for (int e = 0; e < 8; ++e) f[e] *= w;
+        uint4 hi, lo;
+        split8(f, hi, lo);
+        const uint32_t off = core_off<kPp>(j, 8 * chunk);
+        st_smem16(S.Xw, off, hi);
+        st_smem16(S.Xl, off, lo);
     }
     cp_async_wait_all();
     fence_proxy_async_smem();
@@ -436,7 +477,9 @@ struct TcOutSmem {
     bf16 Hl[kNp * kPp]; // h_in low part, then z (rows token i, columns p)
     float acum2[kQ];
     float dt[kQ];
+    float F[kQ];        // 2^(−acum2_j)·Δ_j
     float wsum[4];
+    float wmax[4];
     uint64_t bar[3];    // first MMAs, second MMAs, h_in bulk copy
     uint32_t tmem;
 };
@@ -476,23 +519,16 @@ __global__ void __launch_bounds__(kThrTc) ssd_tc_out_kernel(const SsdParams p) {
         bulk_load(S.HX, reinterpret_cast<const char *>(p.state_in) + (bh * p.nchunks + c) * 32768ll,
                   32768, &S.bar[2]);
     }
-    // this thread's halves of rows i = j = r of C and B (asynchronous
-    // copies), and of x row r into registers
-    stage_row<kNp>(S.C, r, hh * (kNp / 16), (hh + 1) * (kNp / 16),
-                   static_cast<const bf16 *>(p.C) + row * N, static_cast<const bf16 *>(p.C), live,
-                   N, p.vec_bc);
-    stage_row<kNp>(S.BM, r, hh * (kNp / 16), (hh + 1) * (kNp / 16),
-                   static_cast<const bf16 *>(p.B) + row * N, static_cast<const bf16 *>(p.B), live,
-                   N, p.vec_bc);
+    // the chunk's C and B rows (asynchronous copies) and x rows (into
+    // registers, until h_in's tile is free)
+    const long long row0 = b * p.seqlen + t0;
+    stage_tile<kNp>(S.C, static_cast<const bf16 *>(p.C) + row0 * N, N, nq, N, p.vec_bc);
+    stage_tile<kNp>(S.BM, static_cast<const bf16 *>(p.B) + row0 * N, N, nq, N, p.vec_bc);
     cp_async_commit();
-    uint4 xr[kPp / 16];
-    {
-        const bf16 *xrow = static_cast<const bf16 *>(p.x) + row * D + (long long)h * P;
-#pragma unroll
-        for (int k = 0; k < kPp / 16; ++k)
-            xr[k] = live ? ld8(xrow, 8 * (hh * (kPp / 16) + k), P, p.vec_x) : make_uint4(0, 0, 0, 0);
-    }
-    chunk_delta(p, b, h, t0, nq, S.dt, S.acum2, S.wsum);
+    uint4 xr[tile_items<kPp>()];
+    load_tile_regs<kPp>(xr, static_cast<const bf16 *>(p.x) + row0 * D + (long long)h * P, D, nq,
+                        P, p.vec_x);
+    chunk_delta(p, b, h, t0, nq, S.dt, S.acum2, S.wsum, S.F, S.wmax);
     cp_async_wait_all();
     fence_proxy_async_smem();
     tc_fence_before();
@@ -524,11 +560,10 @@ __global__ void __launch_bounds__(kThrTc) ssd_tc_out_kernel(const SsdParams p) {
     ok = __syncthreads_and(ok && wait_mma(&S.bar[0], 0, p.status));
     tc_fence_after();
 
-    // z row r (this thread's half) into h_in's low tile (its MMAs are done)
+    // the chunk's z rows into h_in's low tile (its MMAs are done)
     if (kGate) {
-        stage_row<kPp>(S.Hl, r, hh * (kPp / 16), (hh + 1) * (kPp / 16),
-                       static_cast<const bf16 *>(p.z) + row * D + (long long)h * P,
-                       static_cast<const bf16 *>(p.z), live, P, p.vec_x);
+        stage_tile<kPp>(S.Hl, static_cast<const bf16 *>(p.z) + row0 * D + (long long)h * P, D, nq,
+                        P, p.vec_x);
         cp_async_commit();
     }
     // M row i = r, columns j in this thread's half, from G row i:
@@ -537,20 +572,46 @@ __global__ void __launch_bounds__(kThrTc) ssd_tc_out_kernel(const SsdParams p) {
     // are free once the first MMAs are done). Single products M_ij·x_j can be
     // far larger than y_i, so one bfloat16 rounding of M would cost more than
     // the output's own rounding; the pair keeps about 16 significant bits.
+    // Column blocks above the diagonal for all of a warp's 32 rows are zero
+    // (no tensor-memory read); the decay is 2^acum2_i · F_j when the chunk's
+    // prefix sums allow it (no MUFU per element), else 2^(acum2_i − acum2_j).
     if (ok) {
+        const int q = warp & 3;  // this warp's rows are 32q .. 32q + 31
         const float ai = S.acum2[r];
+        const bool factored = fmaxf(fmaxf(S.wmax[0], S.wmax[1]), fmaxf(S.wmax[2], S.wmax[3])) <=
+                              kFactorMax;
+        const float ei = ex2_approx(ai);
 #pragma unroll 1
         for (int cb = 2 * hh; cb < 2 * hh + 2; ++cb) {
+            if (cb > q) {
+                const uint4 z4 = make_uint4(0, 0, 0, 0);
+#pragma unroll
+                for (int k8 = 0; k8 < 4; ++k8) {
+                    const uint32_t off = core_off<kQ>(r, 32 * cb + 8 * k8);
+                    st_smem16(S.BM, off, z4);
+                    st_smem16(S.C, off, z4);
+                }
+                continue;
+            }
             float g[32];
             tmem_ld32(tmem + lane_q + kColG + 32 * cb, g);
 #pragma unroll
             for (int k8 = 0; k8 < 4; ++k8) {
                 float m[8];
+                if (factored) {
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const int j = 32 * cb + 8 * k8 + e;
-                    m[e] = (j <= r && live) ? g[8 * k8 + e] * ex2_approx(ai - S.acum2[j]) * S.dt[j]
-                                            : 0.0f;
+                    for (int e = 0; e < 8; ++e) {
+                        const int j = 32 * cb + 8 * k8 + e;
+                        m[e] = (j <= r && live) ? g[8 * k8 + e] * ei * S.F[j] : 0.0f;
+                    }
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const int j = 32 * cb + 8 * k8 + e;
+                        m[e] = (j <= r && live)
+                                   ? g[8 * k8 + e] * ex2_approx(ai - S.acum2[j]) * S.dt[j]
+                                   : 0.0f;
+                    }
                 }
                 uint4 hi, lo;
                 split8(m, hi, lo);
@@ -560,10 +621,13 @@ __global__ void __launch_bounds__(kThrTc) ssd_tc_out_kernel(const SsdParams p) {
             }
         }
     }
-    // X row j = r (this thread's half) into h_in's high tile
+    // the x rows into h_in's high tile
 #pragma unroll
-    for (int k = 0; k < kPp / 16; ++k)
-        st_smem16(S.HX, core_off<kPp>(r, 8 * (hh * (kPp / 16) + k)), xr[k]);
+    for (int k = 0; k < tile_items<kPp>(); ++k) {
+        int j, chunk;
+        tile_item<kPp>(k, j, chunk);
+        st_smem16(S.HX, core_off<kPp>(j, 8 * chunk), xr[k]);
+    }
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
@@ -583,7 +647,7 @@ __global__ void __launch_bounds__(kThrTc) ssd_tc_out_kernel(const SsdParams p) {
                       umma_desc(x0 + k * 2 * kRowP, kRowP, 128), idesc_bf16(128, kPp, 0, 1), 1);
         umma_commit(&S.bar[1]);
     }
-    if (kGate) cp_async_wait_all();  // this thread's part of z row r
+    if (kGate) cp_async_wait_all();  // this thread's z copies (the barrier below publishes them)
     ok = __syncthreads_and(ok && wait_mma(&S.bar[1], 0, p.status));
     tc_fence_after();
 
