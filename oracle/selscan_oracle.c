@@ -30,7 +30,7 @@
  *             blocks of the sequence.
  *          "Mamba Block": output gated by silu(gate).
  *
- * Readings where the pages are garbled or silent (each listed in the design doc):
+ * Readings where the pages are garbled or silent:
  *  - The input term on the hot path is B_bar·x = Δ·B·x (the delta-scaled B of
  *    [Johe] "SSM as RNN"), with the x that page's ssm_step drops restored.
  *    The ZOH coefficient (exp(Δ·A) − 1)/A of [Guide] §1 is kept as a second
