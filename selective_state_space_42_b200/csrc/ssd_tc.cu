@@ -256,23 +256,30 @@ __device__ __forceinline__ void load_tile_regs(uint4 (&v)[tile_items<kCols>()], 
     }
 }
 
-// Δ_t of the chunk's tokens t (zero past the sequence end) into dt[], and the
+// Δ_t of the chunk's tokens t (zero past the sequence end; from chunk_dt_raw)
+// into dt[], and the
 // inclusive prefix sums of Δ·A over the chunk, times log2(e), into acum2[]
 // (so exp(Acum_i − Acum_j) = 2^(acum2_i − acum2_j)). With F given, also
 // F[t] = 2^(−acum2_t)·Δ_t and the per-warp maxima of |acum2| in wmax[4].
 // Threads 0..kQ−1 compute; every thread of the block takes part in the two
 // barriers.
-__device__ __forceinline__ void chunk_delta(const SsdParams &p, long long b, int h, long long t0,
-                                            int nq, float *dt, float *acum2, float *wsum,
-                                            float *F = nullptr, float *wmax = nullptr) {
+// dt + dt_bias of this thread's token (threads 0..kQ−1 of a chunk with nq
+// tokens; 0 otherwise): issued early, consumed by chunk_delta.
+__device__ __forceinline__ float chunk_dt_raw(const SsdParams &p, long long b, int h, long long t0,
+                                              int nq) {
+    const int t = threadIdx.x;
+    if (t >= kQ || t >= nq) return 0.0f;
+    return ldg_f32(static_cast<const bf16 *>(p.dt) + (b * p.seqlen + t0 + t) * p.nheads + h) +
+           (p.dt_bias ? p.dt_bias[h] : 0.0f);
+}
+
+__device__ __forceinline__ void chunk_delta(const SsdParams &p, int h, int nq, float raw, float *dt,
+                                            float *acum2, float *wsum, float *F = nullptr,
+                                            float *wmax = nullptr) {
     const int t = threadIdx.x, lane = t & 31, w = t >> 5;
     float d = 0.0f, s = 0.0f;
     if (t < kQ) {
-        if (t < nq) {
-            d = ldg_f32(static_cast<const bf16 *>(p.dt) + (b * p.seqlen + t0 + t) * p.nheads + h) +
-                (p.dt_bias ? p.dt_bias[h] : 0.0f);
-            if (p.softplus) d = softplus_f32(d);
-        }
+        if (t < nq) d = p.softplus ? softplus_f32(raw) : raw;
         s = d * p.A[h] * kLog2e;
 #pragma unroll
         for (int m = 1; m < 32; m <<= 1) {
@@ -346,7 +353,7 @@ __global__ void __launch_bounds__(kThrTc) ssd_tc_state_kernel(const SsdParams p)
     uint4 xr[tile_items<kPp>()];
     load_tile_regs<kPp>(xr, static_cast<const bf16 *>(p.x) + row0 * D + (long long)h * P, D, nq,
                         P, p.vec_x);
-    chunk_delta(p, b, h, t0, nq, S.dt, S.acum2, S.wsum);
+    chunk_delta(p, h, nq, chunk_dt_raw(p, b, h, t0, nq), S.dt, S.acum2, S.wsum);
     const float aend2 = S.acum2[kQ - 1];
     // w_j ◦ x_j as a bfloat16 pair (0 past the sequence end: Δ = 0)
 #pragma unroll
@@ -528,7 +535,7 @@ __global__ void __launch_bounds__(kThrTc) ssd_tc_out_kernel(const SsdParams p) {
     uint4 xr[tile_items<kPp>()];
     load_tile_regs<kPp>(xr, static_cast<const bf16 *>(p.x) + row0 * D + (long long)h * P, D, nq,
                         P, p.vec_x);
-    chunk_delta(p, b, h, t0, nq, S.dt, S.acum2, S.wsum, S.F, S.wmax);
+    const float dt_raw = chunk_dt_raw(p, b, h, t0, nq);
     cp_async_wait_all();
     fence_proxy_async_smem();
     tc_fence_before();
@@ -537,25 +544,31 @@ __global__ void __launch_bounds__(kThrTc) ssd_tc_out_kernel(const SsdParams p) {
     const uint32_t tmem = S.tmem;
     const int ksteps_n = (N + 15) / 16;  // K = d_state in steps of 16 (zero-padded)
     constexpr uint32_t kRowN = (kNp / 8) * 128, kRowP = (kPp / 8) * 128;
+    const uint32_t c0 = smem_addr(S.C), b0 = smem_addr(S.BM);
+
+    // G = C·Bᵀ as soon as B and C are in: A = C (M = token i, K = n,
+    // K-major), B = B (N = token j, K = n, K-major); the Δ prefix sums below
+    // run while it executes
+    if (t == 0)
+        for (int k = 0; k < ksteps_n; ++k)
+            umma_bf16(tmem + kColG, umma_desc(c0 + k * 256, 128, kRowN),
+                      umma_desc(b0 + k * 256, 128, kRowN), idesc_bf16(128, 128, 0, 0), k > 0);
+    chunk_delta(p, h, nq, dt_raw, S.dt, S.acum2, S.wsum, S.F, S.wmax);
 
     bool ok = true;
     if (t == 0) {
         ok = wait_mma(&S.bar[2], 0, p.status);  // h_in landed
         tc_fence_after();
-        // G = C·Bᵀ: A = C (M = token i, K = n, K-major), B = B (N = token j, K = n, K-major)
-        // C·h_in:  A = C, B = h_in (N = channel p contiguous, K = n: M/N-major)
-        const uint32_t c0 = smem_addr(S.C), b0 = smem_addr(S.BM);
+        // C·h_in: A = C, B = h_in (N = channel p contiguous, K = n: M/N-major)
         const uint32_t hh0 = smem_addr(S.HX), hl0 = smem_addr(S.Hl);
         for (int k = 0; ok && k < ksteps_n; ++k) {
             const uint64_t a = umma_desc(c0 + k * 256, 128, kRowN);
-            umma_bf16(tmem + kColG, a, umma_desc(b0 + k * 256, 128, kRowN),
-                      idesc_bf16(128, 128, 0, 0), k > 0);
             umma_bf16(tmem + kColYo, a, umma_desc(hh0 + k * 2 * kRowP, kRowP, 128),
                       idesc_bf16(128, kPp, 0, 1), k > 0);
             umma_bf16(tmem + kColYo, a, umma_desc(hl0 + k * 2 * kRowP, kRowP, 128),
                       idesc_bf16(128, kPp, 0, 1), 1);
         }
-        umma_commit(&S.bar[0]);
+        umma_commit(&S.bar[0]);  // tracks the G and C·h_in MMAs
     }
     ok = __syncthreads_and(ok && wait_mma(&S.bar[0], 0, p.status));
     tc_fence_after();
