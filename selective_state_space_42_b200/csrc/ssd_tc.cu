@@ -11,9 +11,10 @@
 //                           M  = (C·Bᵀ) ◦ [j ≤ i]·exp(Acum_i − Acum_j)·Δ_j        (Q×Q)
 // and h_in, the state entering each chunk, comes from the element-wise carry
 // h_c = exp(Acum_end,c)·h_{c−1} + S_c. Three kernels:
-//   ssd_tc_state_kernel  S for one (chunk, head, batch row): MMAs of
-//                        M=128 (state n) × N=64 (head channel p) × K=2×128
-//                        (token; w ◦ X as a bfloat16 high/low pair)
+//   ssd_tc_state_kernel  S for one (chunk, group of heads, batch row): B staged
+//                        once, per head MMAs of M=128 (state n) × N=64 (head
+//                        channel p) × K=2×128 (token; w ◦ X as a bfloat16
+//                        high/low pair)
 //   ssd_tc_carry_kernel  the element-wise carry over chunks, writing each h_in
 //                        in the output kernel's operand layout
 //   ssd_tc_out_kernel    G = C·Bᵀ (128×128, K = d_state) and C·h_in (128×64) on
@@ -34,6 +35,7 @@
 #include "ssd_params.cuh"
 #include "tma_util.cuh"
 
+#include <algorithm>
 #include <cstddef>
 
 namespace selscan {
@@ -316,24 +318,30 @@ __device__ __forceinline__ bool wait_mma(uint64_t *bar, uint32_t parity, int *st
 }
 
 // ---- chunk states -----------------------------------------------------------------
+// One CTA per (chunk, group of heads, batch row): B is staged once and used by
+// every head of the group; per head the w ◦ x operand pair and the
+// accumulator alternate between two buffers, so that the MMAs of head k run
+// while head k − 1's result is stored and head k + 1's x is in flight.
 // 256 threads; in the epilogue thread t reads state row n = t mod 128
 // (tensor-memory lane n), column half t / 128.
 
 struct TcStateSmem {
-    bf16 Bt[kQ * kNp];  // rows token j, columns state n
-    bf16 Xw[kQ * kPp];  // rows token j, columns channel p: w_j·x, bfloat16 high part
-    bf16 Xl[kQ * kPp];  // the low part, w_j·x − high
+    bf16 Bt[kQ * kNp];     // rows token j, columns state n
+    bf16 Xw[2][kQ * kPp];  // rows token j, columns channel p: w_j·x, bfloat16 high part
+    bf16 Xl[2][kQ * kPp];  // the low part, w_j·x − high
     float acum2[kQ];
     float dt[kQ];
     float wsum[4];
-    uint64_t bar;
+    uint64_t bar[2];
     uint32_t tmem;
 };
 
 __global__ void __launch_bounds__(kThrTc) ssd_tc_state_kernel(const SsdParams p) {
     extern __shared__ __align__(128) unsigned char smem_raw[];
     TcStateSmem &S = *reinterpret_cast<TcStateSmem *>(smem_raw);
-    const int c = blockIdx.x, h = blockIdx.y;
+    const int c = blockIdx.x;
+    const int h_first = blockIdx.y * p.heads_per_cta;
+    const int nh = min(p.heads_per_cta, p.nheads - h_first);
     const long long b = blockIdx.z;
     const long long t0 = (long long)c * kQ;
     const int nq = (int)min((long long)kQ, p.seqlen - t0);
@@ -341,77 +349,104 @@ __global__ void __launch_bounds__(kThrTc) ssd_tc_state_kernel(const SsdParams p)
     const int N = p.dstate, P = p.headdim;
     const long long D = (long long)p.nheads * P;
 
-    if (warp == 0) tmem_alloc(&S.tmem, 64);
+    if (warp == 0) tmem_alloc(&S.tmem, 128);
     if (t == 0) {
-        mbar_init(&S.bar, 1);
+        mbar_init(&S.bar[0], 1);
+        mbar_init(&S.bar[1], 1);
         fence_barrier_init();
     }
-    // the chunk's B rows (asynchronously) and x rows (into registers)
+    // the chunk's B rows (asynchronously), the first head's x rows (registers)
     const long long row0 = b * p.seqlen + t0;
     stage_tile<kNp>(S.Bt, static_cast<const bf16 *>(p.B) + row0 * N, N, nq, N, p.vec_bc);
     cp_async_commit();
+    const bf16 *xbase = static_cast<const bf16 *>(p.x) + row0 * D;
     uint4 xr[tile_items<kPp>()];
-    load_tile_regs<kPp>(xr, static_cast<const bf16 *>(p.x) + row0 * D + (long long)h * P, D, nq,
-                        P, p.vec_x);
-    chunk_delta(p, h, nq, chunk_dt_raw(p, b, h, t0, nq), S.dt, S.acum2, S.wsum);
-    const float aend2 = S.acum2[kQ - 1];
-    // w_j ◦ x_j as a bfloat16 pair (0 past the sequence end: Δ = 0)
-#pragma unroll
-    for (int k = 0; k < tile_items<kPp>(); ++k) {
-        int j, chunk;
-        tile_item<kPp>(k, j, chunk);
-        const float w = ex2_approx(aend2 - S.acum2[j]) * S.dt[j];
-        float f[8];
-        unpack8(xr[k], f);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) f[e] *= w;
-        uint4 hi, lo;
-        split8(f, hi, lo);
-        const uint32_t off = core_off<kPp>(j, 8 * chunk);
-        st_smem16(S.Xw, off, hi);
-        st_smem16(S.Xl, off, lo);
-    }
-    cp_async_wait_all();
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = S.tmem;
+    load_tile_regs<kPp>(xr, xbase + (long long)h_first * P, D, nq, P, p.vec_x);
+    float dt_raw = chunk_dt_raw(p, b, h_first, t0, nq);
+    uint32_t tmem = 0;
+    bool ok = true;
+    float aend_prev = 0.0f;  // Acum_end·log2(e) of the previous head
+    constexpr uint32_t kRowB = (kNp / 8) * 128, kRowX = (kPp / 8) * 128;
 
-    if (t == 0) {
-        // A = Bᵀ: M = state n (contiguous), K = token j  -> M/N-major; core
-        // matrices along n 128 bytes apart, along j (kNp/8)·128 bytes apart.
-        // B = w ◦ X (high, then low part): N = channel p (contiguous), K =
-        // token j -> M/N-major. The pair keeps the chunk state to about 16
-        // significant bits: it is carried over the whole sequence.
-        const uint32_t a0 = smem_addr(S.Bt), bh = smem_addr(S.Xw), bl = smem_addr(S.Xl);
-        constexpr uint32_t kRowB = (kNp / 8) * 128, kRowX = (kPp / 8) * 128;
-        constexpr uint32_t id = idesc_bf16(128, kPp, 1, 1);
+    for (int k = 0; k <= nh; ++k) {
+        float aend2 = 0.0f;
+        if (k < nh) {
+            const int h = h_first + k;
+            chunk_delta(p, h, nq, dt_raw, S.dt, S.acum2, S.wsum);
+            aend2 = S.acum2[kQ - 1];
+            // w_j ◦ x_j as a bfloat16 pair (0 past the sequence end: Δ = 0)
+            bf16 *xw = S.Xw[k & 1], *xl = S.Xl[k & 1];
 #pragma unroll
-        for (int k = 0; k < kQ / 16; ++k)
-            umma_bf16(tmem, umma_desc(a0 + k * 2 * kRowB, kRowB, 128),
-                      umma_desc(bh + k * 2 * kRowX, kRowX, 128), id, k > 0);
+            for (int i = 0; i < tile_items<kPp>(); ++i) {
+                int j, chunk;
+                tile_item<kPp>(i, j, chunk);
+                const float w = ex2_approx(aend2 - S.acum2[j]) * S.dt[j];
+                float f[8];
+                unpack8(xr[i], f);
 #pragma unroll
-        for (int k = 0; k < kQ / 16; ++k)
-            umma_bf16(tmem, umma_desc(a0 + k * 2 * kRowB, kRowB, 128),
-                      umma_desc(bl + k * 2 * kRowX, kRowX, 128), id, 1);
-        umma_commit(&S.bar);
+                for (int e = 0; e < 8; ++e) f[e] *= w;
+                uint4 hi, lo;
+                split8(f, hi, lo);
+                const uint32_t off = core_off<kPp>(j, 8 * chunk);
+                st_smem16(xw, off, hi);
+                st_smem16(xl, off, lo);
+            }
+            if (k + 1 < nh) {  // the next head's x and dt, in flight from here
+                load_tile_regs<kPp>(xr, xbase + (long long)(h + 1) * P, D, nq, P, p.vec_x);
+                dt_raw = chunk_dt_raw(p, b, h + 1, t0, nq);
+            }
+            if (k == 0) cp_async_wait_all();
+            fence_proxy_async_smem();
+            tc_fence_before();
+            __syncthreads();
+            tc_fence_after();
+            if (k == 0) tmem = S.tmem;
+            if (t == 0 && ok) {
+                // A = Bᵀ: M = state n (contiguous), K = token j  -> M/N-major;
+                // core matrices along n 128 bytes apart, along j (kNp/8)·128
+                // bytes apart. B = w ◦ X (high, then low part): N = channel p
+                // (contiguous), K = token j -> M/N-major. The pair keeps the
+                // chunk state to about 16 significant bits: it is carried over
+                // the whole sequence.
+                const uint32_t a0 = smem_addr(S.Bt), bh = smem_addr(xw), bl = smem_addr(xl);
+                const uint32_t d = tmem + 64u * (uint32_t)(k & 1);
+                constexpr uint32_t id = idesc_bf16(128, kPp, 1, 1);
+#pragma unroll
+                for (int q = 0; q < kQ / 16; ++q)
+                    umma_bf16(d, umma_desc(a0 + q * 2 * kRowB, kRowB, 128),
+                              umma_desc(bh + q * 2 * kRowX, kRowX, 128), id, q > 0);
+#pragma unroll
+                for (int q = 0; q < kQ / 16; ++q)
+                    umma_bf16(d, umma_desc(a0 + q * 2 * kRowB, kRowB, 128),
+                              umma_desc(bl + q * 2 * kRowX, kRowX, 128), id, 1);
+                umma_commit(&S.bar[k & 1]);
+            }
+        }
+        if (k > 0) {  // the previous head's state, while this head's MMAs run
+            const int kk = k - 1, h = h_first + kk;
+            ok = __syncthreads_and(ok && wait_mma(&S.bar[kk & 1], (kk >> 1) & 1, p.status));
+            tc_fence_after();
+            if (ok) {
+                // lane r holds state row n = r: this thread stores S[n][32·hh .. 32·hh + 31]
+                float *dst = p.chunk_state +
+                             (((b * p.nheads + h) * p.nchunks + c) * 128 + r) * 64 + 32 * hh;
+                float v[32];
+                tmem_ld32(tmem + ((uint32_t)((warp & 3) * 32) << 16) + 64u * (uint32_t)(kk & 1) +
+                              32 * hh,
+                          v);
+#pragma unroll
+                for (int q = 0; q < 32; q += 4)
+                    *reinterpret_cast<float4 *>(dst + q) =
+                        make_float4(v[q], v[q + 1], v[q + 2], v[q + 3]);
+                if (t == 0)
+                    p.chunk_decay[(b * p.nheads + h) * p.nchunks + c] = ex2_approx(aend_prev);
+            }
+            tc_fence_before();
+        }
+        aend_prev = aend2;
     }
-    const bool ok = __syncthreads_and(wait_mma(&S.bar, 0, p.status));
-    tc_fence_after();
-    if (ok) {
-        // lane r holds state row n = r: this thread stores S[n][32·hh .. 32·hh + 31]
-        float *dst = p.chunk_state + (((b * p.nheads + h) * p.nchunks + c) * 128 + r) * 64 + 32 * hh;
-        float v[32];
-        tmem_ld32(tmem + ((uint32_t)((warp & 3) * 32) << 16) + 32 * hh, v);
-#pragma unroll
-        for (int k = 0; k < 32; k += 4)
-            *reinterpret_cast<float4 *>(dst + k) = make_float4(v[k], v[k + 1], v[k + 2], v[k + 3]);
-        if (t == 0) p.chunk_decay[(b * p.nheads + h) * p.nchunks + c] = ex2_approx(aend2);
-    }
-    tc_fence_before();
     __syncthreads();
-    if (warp == 0) tmem_dealloc(tmem, 64);
+    if (warp == 0) tmem_dealloc(tmem, 128);
 }
 
 // ---- states entering the chunks ----------------------------------------------------
@@ -727,8 +762,15 @@ cudaError_t launch_ssd_tc_state(const SsdParams &p, cudaStream_t stream) {
         if (e != cudaSuccess) return e;
         configured[dev] = true;
     }
-    const dim3 grid((unsigned)p.nchunks, (unsigned)p.nheads, (unsigned)p.batch);
-    ssd_tc_state_kernel<<<grid, kThrTc, sizeof(TcStateSmem), stream>>>(p);
+    // heads per CTA: as many as keep about two waves of CTAs on 148 SMs (two
+    // CTAs each), at most 8
+    SsdParams q = p;
+    const long long items = (long long)p.nchunks * p.nheads * p.batch;
+    q.heads_per_cta = (int)std::min<long long>(8, std::max<long long>(1, items / (2 * 2 * 148)));
+    const dim3 grid((unsigned)p.nchunks,
+                    (unsigned)((p.nheads + q.heads_per_cta - 1) / q.heads_per_cta),
+                    (unsigned)p.batch);
+    ssd_tc_state_kernel<<<grid, kThrTc, sizeof(TcStateSmem), stream>>>(q);
     return cudaGetLastError();
 }
 
