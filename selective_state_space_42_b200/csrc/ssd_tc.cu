@@ -475,19 +475,23 @@ __global__ void ssd_tc_carry_kernel(const SsdParams p) {
     char *blk0 = reinterpret_cast<char *>(p.state_in) + bh * p.nchunks * 32768ll;
     const float *cs0 = p.chunk_state + (bh * p.nchunks * 128 + n) * 64 + 8 * pg;
     const float *dec0 = p.chunk_decay + bh * p.nchunks;
-    // groups of kAhead chunks: every load of a group is issued before the
-    // group's dependent updates, so the chain waits once per group
+    // groups of kAhead chunks in two alternating register sets: the loads of
+    // the next group are in flight while the current group's dependent
+    // updates run (loads past the last chunk re-read it and are not used)
     constexpr int kAhead = 4;
-    for (int c0 = 0; c0 < p.nchunks; c0 += kAhead) {
-        float4 u[kAhead], v[kAhead];
-        float dec[kAhead];
+    float4 ua[kAhead], va[kAhead], ub[kAhead], vb[kAhead];
+    float da[kAhead], db[kAhead];
+    auto load = [&](float4 (&u)[kAhead], float4 (&v)[kAhead], float (&d)[kAhead], int c0) {
 #pragma unroll
         for (int k = 0; k < kAhead; ++k) {
             const int c = min(c0 + k, p.nchunks - 1);
             u[k] = __ldg(reinterpret_cast<const float4 *>(cs0 + (long long)c * 128 * 64));
             v[k] = __ldg(reinterpret_cast<const float4 *>(cs0 + (long long)c * 128 * 64 + 4));
-            dec[k] = __ldg(dec0 + c);
+            d[k] = __ldg(dec0 + c);
         }
+    };
+    auto update = [&](const float4 (&u)[kAhead], const float4 (&v)[kAhead],
+                      const float (&d)[kAhead], int c0) {
 #pragma unroll
         for (int k = 0; k < kAhead; ++k) {
             if (c0 + k >= p.nchunks) break;
@@ -498,8 +502,15 @@ __global__ void ssd_tc_carry_kernel(const SsdParams p) {
             *reinterpret_cast<uint4 *>(blk + 16384 + off) = lo;
             const float s8[8] = {u[k].x, u[k].y, u[k].z, u[k].w, v[k].x, v[k].y, v[k].z, v[k].w};
 #pragma unroll
-            for (int e = 0; e < 8; ++e) st[e] = fmaf(dec[k], st[e], s8[e]);
+            for (int e = 0; e < 8; ++e) st[e] = fmaf(d[k], st[e], s8[e]);
         }
+    };
+    load(ua, va, da, 0);
+    for (int c0 = 0; c0 < p.nchunks; c0 += 2 * kAhead) {
+        load(ub, vb, db, c0 + kAhead);
+        update(ua, va, da, c0);
+        load(ua, va, da, c0 + 2 * kAhead);
+        update(ub, vb, db, c0 + kAhead);
     }
     if (p.final_state && n < N) {
 #pragma unroll
