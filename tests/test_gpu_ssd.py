@@ -183,3 +183,22 @@ def test_ssd_rejects_unsupported_sizes():
     with pytest.raises(ss.SelscanError):
         ss.selscan_ssd_fwd(x, dt, A, B, B)  # d_state 129
     assert ss.selscan_device_status() == 0
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_ssd_matches_matrix_form(dtype):
+    """Against the semiseparable matrix form written out in float64 (the
+    dense (L ◦ S)·diag(Δ)·x per head), with an initial state, 2 batch rows
+    and 3 chunks of the tensor-core path."""
+    from oracle import ssd_matrix
+    inp = _inputs(2, 300, 3, 64, 128, dtype, seed=7600)
+    g = torch.Generator().manual_seed(7601)
+    h0 = torch.randn(2, 3 * 64, 128, generator=g) * 0.3
+    y, hf = _gpu(inp, h0.to(DEV))
+    torch.cuda.synchronize()
+    n = gh.to_np
+    yo, ho = ssd_matrix.ssd_matrix_form(n(inp["x"]), n(inp["dt"]), n(inp["A"]), n(inp["B"]),
+                                        n(inp["C"]), n(inp["Dh"]), n(inp["z"]),
+                                        n(inp["dt_bias"]), h0=n(h0))
+    gh.compare(gh.to_np(y), yo, gh.RTOL[dtype], "matrix form y")
+    gh.compare(gh.to_np(hf), ho, gh.RTOL[dtype], "matrix form final state")

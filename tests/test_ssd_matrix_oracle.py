@@ -1,0 +1,109 @@
+"""The matrix (semiseparable) form of the scalar-A-per-head scan, written out
+in float64 numpy, against the recurrence oracle, closed forms and the mask's
+structure (CPU only). Source: "Mamba & State Space Models — Guide Complet"
+§5 "Mamba-2" / "SSD — State Space Dual"."""
+import numpy as np
+import pytest
+
+from oracle import ssd_matrix
+
+
+def _case(seed, batch=2, T=37, H=3, P=4, N=5, gate=True, h0=True):
+    r = np.random.default_rng(seed)
+    c = dict(
+        x=r.standard_normal((batch, T, H * P)),
+        dt=0.5 * r.standard_normal((batch, T, H)),
+        A=-(r.random(H) * 3.5 + 0.5),
+        B=r.standard_normal((batch, T, N)),
+        C=r.standard_normal((batch, T, N)),
+        D=1.0 + 0.1 * r.standard_normal(H),
+        z=r.standard_normal((batch, T, H * P)) if gate else None,
+        dt_bias=np.log(np.expm1(1e-3 + (1e-1 - 1e-3) * r.random(H))),
+        h0=0.3 * r.standard_normal((batch, H * P, N)) if h0 else None,
+    )
+    return c
+
+
+def _scan(orc, c, P, softplus=True):
+    """The recurrence oracle with the heads' parameters repeated over their
+    channels."""
+    N = c["B"].shape[2]
+    rep = lambda v: None if v is None else np.repeat(v, P, axis=-1)  # noqa: E731
+    A_full = np.repeat(c["A"][:, None], P, axis=0).repeat(N, axis=1)
+    return orc.fwd(c["x"], rep(c["dt"]), A_full, c["B"], c["C"], rep(c["D"]), c["z"],
+                   rep(c["dt_bias"]), softplus=softplus, h0=c["h0"])
+
+
+def _close(a, b, tol=1e-11):
+    scale = max(float(np.max(np.abs(b))), 1e-300)
+    assert float(np.max(np.abs(a - b))) <= tol * scale, float(np.max(np.abs(a - b))) / scale
+
+
+@pytest.mark.parametrize("gate,h0,softplus", [(True, True, True), (False, False, True),
+                                              (True, False, False)])
+def test_matrix_form_equals_recurrence(orc, gate, h0, softplus):
+    c = _case(9100 + 2 * gate + h0, gate=gate, h0=h0)
+    if not softplus:  # positive Δ without the softplus
+        c["dt"] = np.abs(c["dt"]) * 0.2 + 0.01
+        c["dt_bias"] = np.zeros_like(c["dt_bias"])
+    y, hf = ssd_matrix.ssd_matrix_form(c["x"], c["dt"], c["A"], c["B"], c["C"], c["D"], c["z"],
+                                       c["dt_bias"], softplus=softplus, h0=c["h0"])
+    yo, ho = _scan(orc, c, 4, softplus=softplus)
+    _close(y, yo)
+    _close(hf, ho)
+
+
+def test_single_token_closed_form():
+    """T = 1: y = ((C·B)·Δ + D)·x + exp(Δ·A)·C·h0, gated; final = exp(Δ·A)·h0 + Δ·B ⊗ x."""
+    c = _case(9200, batch=1, T=1, H=2, P=3, N=4)
+    y, hf = ssd_matrix.ssd_matrix_form(c["x"], c["dt"], c["A"], c["B"], c["C"], c["D"], c["z"],
+                                       c["dt_bias"], h0=c["h0"])
+    for h in range(2):
+        delta = np.logaddexp(0.0, c["dt"][0, 0, h] + c["dt_bias"][h])
+        a = np.exp(delta * c["A"][h])
+        cb = float(c["C"][0, 0] @ c["B"][0, 0])
+        for p in range(3):
+            d = h * 3 + p
+            xv, zv = c["x"][0, 0, d], c["z"][0, 0, d]
+            h0v = c["h0"][0, d]
+            want = (cb * delta * xv + c["D"][h] * xv + a * float(c["C"][0, 0] @ h0v))
+            want *= zv / (1.0 + np.exp(-zv))
+            assert abs(y[0, 0, d] - want) <= 1e-13 * max(1.0, abs(want))
+            np.testing.assert_allclose(hf[0, d], a * h0v + delta * c["B"][0, 0] * xv,
+                                       rtol=1e-13, atol=1e-15)
+
+
+def test_mask_is_semiseparable():
+    """Every block of the mask strictly below the diagonal has rank 1:
+    L[i, j] = exp(Acum_i)·exp(−Acum_j) (the structure [Guide] §5 names)."""
+    r = np.random.default_rng(9300)
+    L = ssd_matrix.decay_mask(0.5 * r.standard_normal(40), -1.3, dt_bias=-2.0)
+    for i0 in range(1, 40, 7):
+        for j0 in range(0, i0, 5):
+            block = L[i0:, :j0 + 1]
+            s = np.linalg.svd(block, compute_uv=False)
+            assert s[1] <= 1e-12 * s[0] if s.size > 1 else True
+
+
+def test_a_shifted_mask_is_caught(orc):
+    """A plausible slip — the decay taken from Acum_{j−1} instead of Acum_j —
+    changes the result well beyond the pin's tolerance."""
+    c = _case(9400)
+    yo, _ = _scan(orc, c, 4)
+    x, dt, A, B, C = c["x"], c["dt"], c["A"], c["B"], c["C"]
+    batch, T, dim = x.shape
+    H, P = 3, 4
+    y = np.zeros_like(yo)
+    for b in range(batch):
+        S = C[b] @ B[b].T
+        for h in range(H):
+            delta = np.logaddexp(0.0, dt[b, :, h] + c["dt_bias"][h])
+            acum = np.cumsum(delta * A[h])
+            prev = np.concatenate([[0.0], acum[:-1]])  # the slip
+            L = np.tril(np.exp(acum[:, None] - prev[None, :]))
+            xh = x[b, :, h * P:(h + 1) * P]
+            yh = ((L * S) * delta[None, :]) @ xh + c["D"][h] * xh
+            yh = yh + np.exp(acum)[:, None] * (C[b] @ c["h0"][b, h * P:(h + 1) * P, :].T)
+            zh = c["z"][b, :, h * P:(h + 1) * P]
+            y[b, :, h * P:(h + 1) * P] = yh * zh / (1.0 + np.exp(-zh))
+    assert float(np.max(np.abs(y - yo))) > 1e-3 * float(np.max(np.abs(yo)))
