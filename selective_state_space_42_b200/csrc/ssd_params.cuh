@@ -26,6 +26,7 @@ struct SsdParams {
     int vec_bc;                      // B, C rows allow 16-byte accesses (tensor-core path)
     int *status;                     // the library's device error word
     int heads_per_cta;               // set by the launcher of the tensor-core state kernel
+    int tma_bc;                      // tensor-core kernels: B and C tiles by TMA (set by the launchers)
 };
 // float32 I/O: the float32 chunk kernels; bfloat16 I/O: the tensor-core kernels.
 cudaError_t launch_ssd(const SsdParams &p, bool bf16, cudaStream_t stream);

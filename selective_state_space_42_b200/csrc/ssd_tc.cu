@@ -32,6 +32,9 @@
 // eight rows of 16 bytes along the tile's contiguous dimension. Accumulators
 // are float32 in tensor memory; one elected thread issues every MMA and a
 // tcgen05.commit to an mbarrier tells the CTA they are done.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include "ssd_params.cuh"
 #include "tma_util.cuh"
 
@@ -64,6 +67,37 @@ __device__ __forceinline__ uint32_t core_off(int r, int c) {
 __device__ __forceinline__ uint64_t umma_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
     return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
            ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46);
+}
+
+// The same for the 128-byte swizzled layout (layout type 2): 8-row atoms of
+// 128-byte rows whose 16-byte chunks are permuted by the row index, as a
+// 128B-swizzled TMA load writes them. K-major: the start advances by 32
+// bytes per K step of 16 inside a 64-column slab; the stride byte offset is
+// the distance between 8-row atoms (1024 bytes). M/N-major: leading byte
+// offset = distance between 64-element slabs, stride byte offset = between
+// 8-row atoms along K.
+__device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+    return umma_desc(saddr, lbo, sbo) | (2ull << 61);
+}
+
+// 3-D tiled TMA load (coordinates innermost first) completing on an mbarrier.
+__device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, uint64_t *bar,
+                                            int32_t c0, int32_t c1, int32_t c2) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_addr(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_addr(bar)), "r"(c0), "r"(c1), "r"(c2)
+        : "memory");
+}
+
+// The B or C tile of a chunk by TMA: two 64-column slabs of 128 token rows,
+// 128-byte swizzled; rows past the sequence and columns past d_state (the
+// whole second slab when d_state ≤ 64) are zero-filled by the copy.
+constexpr uint32_t kBcTileBytes = 2u * kQ * 64 * 2;
+__device__ __forceinline__ void tma_bc_tile(bf16 *tile, const CUtensorMap *map, uint64_t *bar,
+                                            int t0, int b) {
+    tma_load_3d(tile, map, bar, 0, t0, b);
+    tma_load_3d(tile + kQ * 64, map, bar, 64, t0, b);
 }
 
 // Instruction descriptor of kind::f16: bfloat16 A and B, float32 D, shape
@@ -333,12 +367,16 @@ struct TcStateSmem {
     float dt[kQ];
     float wsum[4];
     uint64_t bar[2];
+    uint64_t bar_b;       // the B tile's TMA
     uint32_t tmem;
 };
 
-__global__ void __launch_bounds__(kThrTc) ssd_tc_state_kernel(const SsdParams p) {
+__global__ void __launch_bounds__(kThrTc)
+ssd_tc_state_kernel(const SsdParams p, const __grid_constant__ CUtensorMap tm_b) {
     extern __shared__ __align__(128) unsigned char smem_raw[];
-    TcStateSmem &S = *reinterpret_cast<TcStateSmem *>(smem_raw);
+    // 1024-byte aligned: the 128-byte swizzle pattern is taken from address bits 7..9
+    TcStateSmem &S = *reinterpret_cast<TcStateSmem *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     const int c = blockIdx.x;
     const int h_first = blockIdx.y * p.heads_per_cta;
     const int nh = min(p.heads_per_cta, p.nheads - h_first);
@@ -353,12 +391,20 @@ __global__ void __launch_bounds__(kThrTc) ssd_tc_state_kernel(const SsdParams p)
     if (t == 0) {
         mbar_init(&S.bar[0], 1);
         mbar_init(&S.bar[1], 1);
+        mbar_init(&S.bar_b, 1);
         fence_barrier_init();
+        if (p.tma_bc) {  // the chunk's B rows by TMA (128-byte swizzled slabs)
+            mbar_arrive_expect_tx(&S.bar_b, kBcTileBytes);
+            tma_bc_tile(S.Bt, &tm_b, &S.bar_b, (int)t0, (int)b);
+        }
     }
-    // the chunk's B rows (asynchronously), the first head's x rows (registers)
+    // else the chunk's B rows by asynchronous copies (interleaved layout);
+    // the first head's x rows into registers
     const long long row0 = b * p.seqlen + t0;
-    stage_tile<kNp>(S.Bt, static_cast<const bf16 *>(p.B) + row0 * N, N, nq, N, p.vec_bc);
-    cp_async_commit();
+    if (!p.tma_bc) {
+        stage_tile<kNp>(S.Bt, static_cast<const bf16 *>(p.B) + row0 * N, N, nq, N, p.vec_bc);
+        cp_async_commit();
+    }
     const bf16 *xbase = static_cast<const bf16 *>(p.x) + row0 * D;
     uint4 xr[tile_items<kPp>()];
     load_tile_regs<kPp>(xr, xbase + (long long)h_first * P, D, nq, P, p.vec_x);
@@ -395,30 +441,38 @@ __global__ void __launch_bounds__(kThrTc) ssd_tc_state_kernel(const SsdParams p)
                 load_tile_regs<kPp>(xr, xbase + (long long)(h + 1) * P, D, nq, P, p.vec_x);
                 dt_raw = chunk_dt_raw(p, b, h + 1, t0, nq);
             }
-            if (k == 0) cp_async_wait_all();
+            if (k == 0 && !p.tma_bc) cp_async_wait_all();
             fence_proxy_async_smem();
             tc_fence_before();
             __syncthreads();
             tc_fence_after();
             if (k == 0) tmem = S.tmem;
+            if (t == 0 && k == 0 && p.tma_bc) {
+                ok = wait_mma(&S.bar_b, 0, p.status);  // B landed
+                tc_fence_after();
+            }
             if (t == 0 && ok) {
-                // A = Bᵀ: M = state n (contiguous), K = token j  -> M/N-major;
-                // core matrices along n 128 bytes apart, along j (kNp/8)·128
-                // bytes apart. B = w ◦ X (high, then low part): N = channel p
-                // (contiguous), K = token j -> M/N-major. The pair keeps the
-                // chunk state to about 16 significant bits: it is carried over
-                // the whole sequence.
+                // A = Bᵀ: M = state n (contiguous), K = token j -> M/N-major.
+                // TMA tile: 64-state slabs 16 KB apart, 8-token atoms 1024
+                // bytes apart; interleaved tile: core matrices along n 128
+                // bytes apart, along j (kNp/8)·128 bytes apart.
+                // B = w ◦ X (high, then low part): N = channel p (contiguous),
+                // K = token j -> M/N-major. The pair keeps the chunk state to
+                // about 16 significant bits: it is carried over the whole
+                // sequence.
                 const uint32_t a0 = smem_addr(S.Bt), bh = smem_addr(xw), bl = smem_addr(xl);
                 const uint32_t d = tmem + 64u * (uint32_t)(k & 1);
                 constexpr uint32_t id = idesc_bf16(128, kPp, 1, 1);
+                auto adesc = [&](int q) {
+                    return p.tma_bc ? umma_desc_sw128(a0 + q * 2048, kQ * 64 * 2, 1024)
+                                    : umma_desc(a0 + q * 2 * kRowB, kRowB, 128);
+                };
 #pragma unroll
                 for (int q = 0; q < kQ / 16; ++q)
-                    umma_bf16(d, umma_desc(a0 + q * 2 * kRowB, kRowB, 128),
-                              umma_desc(bh + q * 2 * kRowX, kRowX, 128), id, q > 0);
+                    umma_bf16(d, adesc(q), umma_desc(bh + q * 2 * kRowX, kRowX, 128), id, q > 0);
 #pragma unroll
                 for (int q = 0; q < kQ / 16; ++q)
-                    umma_bf16(d, umma_desc(a0 + q * 2 * kRowB, kRowB, 128),
-                              umma_desc(bl + q * 2 * kRowX, kRowX, 128), id, 1);
+                    umma_bf16(d, adesc(q), umma_desc(bl + q * 2 * kRowX, kRowX, 128), id, 1);
                 umma_commit(&S.bar[k & 1]);
             }
         }
@@ -533,7 +587,7 @@ struct TcOutSmem {
     float F[kQ];        // 2^(−acum2_j)·Δ_j
     float wsum[4];
     float wmax[4];
-    uint64_t bar[3];    // first MMAs, second MMAs, h_in bulk copy
+    uint64_t bar[4];    // first MMAs, second MMAs, h_in bulk copy, B and C TMA
     uint32_t tmem;
 };
 static_assert(kQ == kNp, "M reuses the B tile");
@@ -546,9 +600,13 @@ constexpr uint32_t kColG = 0, kColYd = 128, kColYo = 192;
 // 256 threads: thread t works on token row r = t mod 128 (tensor-memory lane
 // r) and column half hh = t / 128 of every tile, of M and of y.
 template <bool kGate>
-__global__ void __launch_bounds__(kThrTc) ssd_tc_out_kernel(const SsdParams p) {
+__global__ void __launch_bounds__(kThrTc)
+ssd_tc_out_kernel(const SsdParams p, const __grid_constant__ CUtensorMap tm_b,
+                  const __grid_constant__ CUtensorMap tm_c) {
     extern __shared__ __align__(128) unsigned char smem_raw[];
-    TcOutSmem &S = *reinterpret_cast<TcOutSmem *>(smem_raw);
+    // 1024-byte aligned: the 128-byte swizzle pattern is taken from address bits 7..9
+    TcOutSmem &S = *reinterpret_cast<TcOutSmem *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     const int c = blockIdx.x, h = blockIdx.y;
     const long long b = blockIdx.z;
     const long long t0 = (long long)c * kQ;
@@ -566,7 +624,13 @@ __global__ void __launch_bounds__(kThrTc) ssd_tc_out_kernel(const SsdParams p) {
         mbar_init(&S.bar[0], 1);
         mbar_init(&S.bar[1], 1);
         mbar_init(&S.bar[2], 1);
+        mbar_init(&S.bar[3], 1);
         fence_barrier_init();
+        if (p.tma_bc) {  // the chunk's C and B rows by TMA (128-byte swizzled slabs)
+            mbar_arrive_expect_tx(&S.bar[3], 2 * kBcTileBytes);
+            tma_bc_tile(S.C, &tm_c, &S.bar[3], (int)t0, (int)b);
+            tma_bc_tile(S.BM, &tm_b, &S.bar[3], (int)t0, (int)b);
+        }
         // h_in's (high, low) block for this chunk, already in operand layout
         mbar_arrive_expect_tx(&S.bar[2], 32768);
         bulk_load(S.HX, reinterpret_cast<const char *>(p.state_in) + (bh * p.nchunks + c) * 32768ll,
@@ -575,14 +639,16 @@ __global__ void __launch_bounds__(kThrTc) ssd_tc_out_kernel(const SsdParams p) {
     // the chunk's C and B rows (asynchronous copies) and x rows (into
     // registers, until h_in's tile is free)
     const long long row0 = b * p.seqlen + t0;
-    stage_tile<kNp>(S.C, static_cast<const bf16 *>(p.C) + row0 * N, N, nq, N, p.vec_bc);
-    stage_tile<kNp>(S.BM, static_cast<const bf16 *>(p.B) + row0 * N, N, nq, N, p.vec_bc);
-    cp_async_commit();
+    if (!p.tma_bc) {
+        stage_tile<kNp>(S.C, static_cast<const bf16 *>(p.C) + row0 * N, N, nq, N, p.vec_bc);
+        stage_tile<kNp>(S.BM, static_cast<const bf16 *>(p.B) + row0 * N, N, nq, N, p.vec_bc);
+        cp_async_commit();
+    }
     uint4 xr[tile_items<kPp>()];
     load_tile_regs<kPp>(xr, static_cast<const bf16 *>(p.x) + row0 * D + (long long)h * P, D, nq,
                         P, p.vec_x);
     const float dt_raw = chunk_dt_raw(p, b, h, t0, nq);
-    cp_async_wait_all();
+    if (!p.tma_bc) cp_async_wait_all();
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
@@ -591,24 +657,37 @@ __global__ void __launch_bounds__(kThrTc) ssd_tc_out_kernel(const SsdParams p) {
     const int ksteps_n = (N + 15) / 16;  // K = d_state in steps of 16 (zero-padded)
     constexpr uint32_t kRowN = (kNp / 8) * 128, kRowP = (kPp / 8) * 128;
     const uint32_t c0 = smem_addr(S.C), b0 = smem_addr(S.BM);
+    // K-major operand descriptors of the C and B tiles for K step k (16
+    // states): 128-byte swizzled TMA slabs (32 bytes per step inside a
+    // 64-column slab of 16 KB, 8-row atoms 1024 bytes apart), or the
+    // interleaved layout (core matrices 128 bytes apart along K, 8-row
+    // groups (kNp/8)·128 bytes apart)
+    auto kdesc = [&](uint32_t base, int k) {
+        return p.tma_bc ? umma_desc_sw128(base + (k >> 2) * (kQ * 64 * 2) + (k & 3) * 32, 16, 1024)
+                        : umma_desc(base + k * 256, 128, kRowN);
+    };
 
     // G = C·Bᵀ as soon as B and C are in: A = C (M = token i, K = n,
     // K-major), B = B (N = token j, K = n, K-major); the Δ prefix sums below
     // run while it executes
-    if (t == 0)
-        for (int k = 0; k < ksteps_n; ++k)
-            umma_bf16(tmem + kColG, umma_desc(c0 + k * 256, 128, kRowN),
-                      umma_desc(b0 + k * 256, 128, kRowN), idesc_bf16(128, 128, 0, 0), k > 0);
-    chunk_delta(p, h, nq, dt_raw, S.dt, S.acum2, S.wsum, S.F, S.wmax);
-
     bool ok = true;
     if (t == 0) {
-        ok = wait_mma(&S.bar[2], 0, p.status);  // h_in landed
+        if (p.tma_bc) {
+            ok = wait_mma(&S.bar[3], 0, p.status);  // B and C landed
+            tc_fence_after();
+        }
+        for (int k = 0; ok && k < ksteps_n; ++k)
+            umma_bf16(tmem + kColG, kdesc(c0, k), kdesc(b0, k), idesc_bf16(128, 128, 0, 0), k > 0);
+    }
+    chunk_delta(p, h, nq, dt_raw, S.dt, S.acum2, S.wsum, S.F, S.wmax);
+
+    if (t == 0) {
+        ok = ok && wait_mma(&S.bar[2], 0, p.status);  // h_in landed
         tc_fence_after();
         // C·h_in: A = C, B = h_in (N = channel p contiguous, K = n: M/N-major)
         const uint32_t hh0 = smem_addr(S.HX), hl0 = smem_addr(S.Hl);
         for (int k = 0; ok && k < ksteps_n; ++k) {
-            const uint64_t a = umma_desc(c0 + k * 256, 128, kRowN);
+            const uint64_t a = kdesc(c0, k);
             umma_bf16(tmem + kColYo, a, umma_desc(hh0 + k * 2 * kRowP, kRowP, 128),
                       idesc_bf16(128, kPp, 0, 1), k > 0);
             umma_bf16(tmem + kColYo, a, umma_desc(hl0 + k * 2 * kRowP, kRowP, 128),
@@ -750,6 +829,35 @@ __global__ void __launch_bounds__(kThrTc) ssd_tc_out_kernel(const SsdParams p) {
     if (warp == 0) tmem_dealloc(tmem, 256);
 }
 
+// cuTensorMapEncodeTiled from the driver (through the runtime's entry-point
+// query, so the library links against the runtime only).
+PFN_cuTensorMapEncodeTiled_v12000 tma_encode() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        cudaDriverEntryPointQueryResult q;
+        void *ptr = nullptr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    }
+    return fn;
+}
+
+// A [batch][seqlen][dstate] bfloat16 tensor (B or C) as a 3-D map with
+// 64-column × 128-token boxes, 128-byte swizzle, zero fill outside.
+bool make_bc_map(CUtensorMap *m, const void *base, long long batch, long long seqlen, int dstate) {
+    auto fn = tma_encode();
+    if (!fn) return false;
+    cuuint64_t gdim[3] = {(cuuint64_t)dstate, (cuuint64_t)seqlen, (cuuint64_t)batch};
+    cuuint64_t gstride[2] = {(cuuint64_t)dstate * 2, (cuuint64_t)(seqlen * dstate * 2)};
+    cuuint32_t box[3] = {64, (cuuint32_t)kQ, 1};
+    cuuint32_t estride[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), gdim, gstride, box,
+              estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <typename K>
 cudaError_t set_smem(K kernel, size_t bytes) {
     return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
@@ -769,7 +877,7 @@ cudaError_t launch_ssd_tc_state(const SsdParams &p, cudaStream_t stream) {
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev >= 0 && dev < 64 && !configured[dev]) {
-        e = set_smem(ssd_tc_state_kernel, sizeof(TcStateSmem));
+        e = set_smem(ssd_tc_state_kernel, sizeof(TcStateSmem) + 1024);
         if (e != cudaSuccess) return e;
         configured[dev] = true;
     }
@@ -781,7 +889,9 @@ cudaError_t launch_ssd_tc_state(const SsdParams &p, cudaStream_t stream) {
     const dim3 grid((unsigned)p.nchunks,
                     (unsigned)((p.nheads + q.heads_per_cta - 1) / q.heads_per_cta),
                     (unsigned)p.batch);
-    ssd_tc_state_kernel<<<grid, kThrTc, sizeof(TcStateSmem), stream>>>(q);
+    CUtensorMap mb{};
+    q.tma_bc = p.vec_bc && make_bc_map(&mb, p.B, p.batch, p.seqlen, p.dstate) ? 1 : 0;
+    ssd_tc_state_kernel<<<grid, kThrTc, sizeof(TcStateSmem) + 1024, stream>>>(q, mb);
     return cudaGetLastError();
 }
 
@@ -797,16 +907,21 @@ cudaError_t launch_ssd_tc_out(const SsdParams &p, cudaStream_t stream) {
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev >= 0 && dev < 64 && !configured[dev]) {
-        e = set_smem(ssd_tc_out_kernel<true>, sizeof(TcOutSmem));
-        if (e == cudaSuccess) e = set_smem(ssd_tc_out_kernel<false>, sizeof(TcOutSmem));
+        e = set_smem(ssd_tc_out_kernel<true>, sizeof(TcOutSmem) + 1024);
+        if (e == cudaSuccess) e = set_smem(ssd_tc_out_kernel<false>, sizeof(TcOutSmem) + 1024);
         if (e != cudaSuccess) return e;
         configured[dev] = true;
     }
     const dim3 grid((unsigned)p.nchunks, (unsigned)p.nheads, (unsigned)p.batch);
+    SsdParams q = p;
+    CUtensorMap mb{}, mc{};
+    q.tma_bc = p.vec_bc && make_bc_map(&mb, p.B, p.batch, p.seqlen, p.dstate) &&
+                       make_bc_map(&mc, p.C, p.batch, p.seqlen, p.dstate)
+                   ? 1 : 0;
     if (p.z)
-        ssd_tc_out_kernel<true><<<grid, kThrTc, sizeof(TcOutSmem), stream>>>(p);
+        ssd_tc_out_kernel<true><<<grid, kThrTc, sizeof(TcOutSmem) + 1024, stream>>>(q, mb, mc);
     else
-        ssd_tc_out_kernel<false><<<grid, kThrTc, sizeof(TcOutSmem), stream>>>(p);
+        ssd_tc_out_kernel<false><<<grid, kThrTc, sizeof(TcOutSmem) + 1024, stream>>>(q, mb, mc);
     return cudaGetLastError();
 }
 
