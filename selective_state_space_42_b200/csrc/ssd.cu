@@ -22,7 +22,9 @@
 //                     times silu(z).
 // The products are FP32 (register-blocked 4×4 per thread from shared memory);
 // chunks are independent, so the whole sequence runs in parallel except for
-// the element-wise carry.
+// the element-wise carry. These kernels serve float32 I/O (64-token chunks);
+// bfloat16 I/O goes to the tensor-core kernels of ssd_tc.cu (launch_ssd
+// below chooses).
 #include "ssd_params.cuh"
 
 namespace selscan {

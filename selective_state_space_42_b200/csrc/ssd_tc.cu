@@ -19,18 +19,19 @@
 //                        in the output kernel's operand layout
 //   ssd_tc_out_kernel    G = C·Bᵀ (128×128, K = d_state) and C·h_in (128×64) on
 //                        the tensor cores (h_in as a bfloat16 high/low pair),
-//                        M built from G by the 128 threads
-//                        (thread i = token i = tensor-memory lane i) and
+//                        M built from G by the 256 threads (token row i =
+//                        tensor-memory lane i, two threads per row) and
 //                        written back to shared memory as a bfloat16 pair
 //                        M_hi + M_lo, then M·X (128×64, K = 2×128) and the
 //                        epilogue y = M·X + exp(Acum_i)·C·h_in + D·x, gated
 //                        by silu(z).
-// Operands are bfloat16 in shared memory, copied in (cp.async rows, one bulk
-// copy for h_in) or written by the threads where a Δ-dependent scaling is
-// applied while staging, in the interleaved layout
-// the MMA reads without swizzling: 8×8 core matrices of 128 contiguous bytes,
-// eight rows of 16 bytes along the tile's contiguous dimension. Accumulators
-// are float32 in tensor memory; one elected thread issues every MMA and a
+// Operands are bfloat16 in shared memory: B and C by TMA into 128-byte
+// swizzled slabs (or, where the rows do not allow TMA, by cp.async), h_in by
+// one bulk copy, and the operands that carry a Δ-dependent scaling written
+// by the threads; the last three in the interleaved layout the MMA reads
+// without swizzling (8×8 core matrices of 128 contiguous bytes, eight rows
+// of 16 bytes along the tile's contiguous dimension). Accumulators are
+// float32 in tensor memory; one elected thread issues every MMA and a
 // tcgen05.commit to an mbarrier tells the CTA they are done.
 #include <cuda.h>
 #include <cudaTypedefs.h>
