@@ -92,7 +92,7 @@ class Oracle:
         lib.oracle_compose.argtypes = [ctypes.c_double] * 4 + [_dp, _dp]
         lib.oracle_selscan_bwd.restype = None
         lib.oracle_selscan_bwd.argtypes = (
-            [_dp] * 8 + [ctypes.c_int] + [_dp] * 3 + [_dp] * 9
+            [_dp] * 8 + [ctypes.c_int, ctypes.c_int] + [_dp] * 3 + [_dp] * 9
             + [_i64, _i64, _i64, _i64, ctypes.c_int])
         lib.oracle_causal_conv1d.restype = None
         lib.oracle_causal_conv1d.argtypes = [_dp, _dp, _dp, _dp, _i64, _i64, _i64, _i64,
@@ -158,9 +158,10 @@ class Oracle:
         return y, hs
 
     def bwd(self, x, delta, A, B, C, D=None, z=None, delta_bias=None,
-            softplus=True, h0=None, dy=None, dfinal=None, threads=None):
+            softplus=True, h0=None, dy=None, dfinal=None, threads=None, bbar=BBAR_DELTA):
         """Gradient of the loss Σ dy·y + Σ dfinal·final_state with respect to
-        every input of ``fwd`` (input term Δ·B·x). Returns a dict with dx,
+        every input of ``fwd`` (input term Δ·B·x, or the ZOH term with
+        ``bbar=BBAR_ZOH``). Returns a dict with dx,
         ddelta, dA, dB, dC, dD, dz (None without z), ddelta_bias and dh0
         (None without h0), all float64."""
         a, (batch, L, dim, N) = self._fwd_args(x, delta, A, B, C, D, z,
@@ -177,7 +178,7 @@ class Oracle:
         self.lib.oracle_selscan_bwd(
             _ptr(a["x"]), _ptr(a["delta"]), _ptr(a["A"]), _ptr(a["B"]),
             _ptr(a["C"]), _ptr(a["D"]), _ptr(a["z"]), _ptr(a["delta_bias"]),
-            int(bool(softplus)), _ptr(a["h0"]), _ptr(dy), _ptr(dfinal),
+            int(bool(softplus)), int(bbar), _ptr(a["h0"]), _ptr(dy), _ptr(dfinal),
             _ptr(out["dx"]), _ptr(out["ddelta"]), _ptr(out["dA"]), _ptr(out["dB"]),
             _ptr(out["dC"]), _ptr(out["dD"]), _ptr(out["dz"]),
             _ptr(out["ddelta_bias"]), _ptr(out["dh0"]),

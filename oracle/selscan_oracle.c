@@ -83,6 +83,22 @@ static double bbar_coeff(double dt, double a, int bbar_mode)
     return dt;
 }
 
+/* The ZOH coefficient c = (exp(Δ·a) − 1)/a of [Guide] §1 and its partial
+ * derivatives: ∂c/∂Δ = exp(Δ·a) (for every a, including the limit a → 0),
+ * ∂c/∂a = (z·exp(z) − (exp(z) − 1))/a² = Δ²·(z·exp(z) − expm1(z))/z² with
+ * z = Δ·a, whose z → 0 limit is Δ²/2 (the series 1/2 + z/3 + z²/8 below
+ * |z| = 1e-4). */
+static void zoh_coeff_grads(double dt, double a, double *c, double *c_dt, double *c_a)
+{
+    double z = dt * a;
+    *c = a == 0.0 ? dt : expm1(z) / a;
+    *c_dt = exp(z);
+    if (fabs(z) < 1e-4)
+        *c_a = dt * dt * (0.5 + z / 3.0 + z * z / 8.0);
+    else
+        *c_a = dt * dt * (z * exp(z) - expm1(z)) / (z * z);
+}
+
 /*
  * One token of one channel: the discrete recurrence of [Guide] §1/§4 with the
  * selective (per-token) Δ, B, C. Updates h[0..N) in place and returns the
@@ -312,8 +328,13 @@ static double sigmoid(double v)
  *   dx_t     = du_t·Δ_t + ds_t·D,   dD += ds_t·x_t,   dz_t = dy_t·s_t·silu'(z_t)
  *   ddelta_t = dΔ_t·σ(delta_t + bias) (softplus on; dΔ_t otherwise),
  *   dbias   += ddelta_t
- * and dh0 = Abar_0·λ_0. The forward states h_t are kept per chain (this is
- * the plain definition, not a memory-saving schedule).
+ * and dh0 = Abar_0·λ_0. With the ZOH input term (bbar_mode = 1) the input
+ * of token t is c_t[n]·B_t[n]·x_t with c = (exp(Δ·A[n]) − 1)/A[n] instead of
+ * Δ·B_t[n]·x_t; then dB_t[n] += λ_t[n]·c_t[n]·x_t, dx_t = Σ_n λ_t[n]·c_t[n]·
+ * B_t[n] + ds_t·D, the input part of dΔ_t is Σ_n λ_t[n]·(∂c/∂Δ)·B_t[n]·x_t
+ * and dA[n] gains λ_t[n]·(∂c/∂A)·B_t[n]·x_t (zoh_coeff_grads). The forward
+ * states h_t are kept per chain (this is the plain definition, not a
+ * memory-saving schedule).
  *
  * Outputs: dx, ddelta, dz [batch, L, D] (dz only when z is given); dB, dC
  * [batch, L, N]; dA [D, N]; dDv, ddelta_bias [D]; dh0 [batch, D, N]
@@ -322,7 +343,7 @@ static double sigmoid(double v)
 void oracle_selscan_bwd(const double *x, const double *delta, const double *A,
                         const double *B, const double *C, const double *Dv,
                         const double *z, const double *delta_bias,
-                        int softplus_flag, const double *h0, const double *dy,
+                        int softplus_flag, int bbar_mode, const double *h0, const double *dy,
                         const double *dfinal, double *dx, double *ddelta,
                         double *dA, double *dB, double *dC, double *dDv,
                         double *dz, double *ddelta_bias, double *dh0,
@@ -370,7 +391,8 @@ void oracle_selscan_bwd(const double *x, const double *delta, const double *A,
                     double acc = 0.0;
                     dts[t] = dt;
                     for (int64_t n = 0; n < N; ++n) {
-                        double h = exp(dt * Arow[n]) * hs[t * N + n] + dt * B[j + n] * x[i];
+                        double h = exp(dt * Arow[n]) * hs[t * N + n] +
+                                   bbar_coeff(dt, Arow[n], bbar_mode) * B[j + n] * x[i];
                         hs[(t + 1) * N + n] = h;
                         acc += C[j + n] * h;
                     }
@@ -388,19 +410,38 @@ void oracle_selscan_bwd(const double *x, const double *delta, const double *A,
                         dz[i] = dy[i] * ss[t] * silu_grad(z[i]);
                     dDv[d] += ds * x[i];
                     double du = 0.0, ddt = 0.0;
-                    for (int64_t n = 0; n < N; ++n) {
-                        double h = hs[(t + 1) * N + n], hprev = hs[t * N + n];
-                        double a_bar = exp(dt * Arow[n]);
-                        lam[n] += ds * C[j + n]; /* λ_t */
-                        pC[t * N + n] += ds * h;
-                        pB[t * N + n] += lam[n] * dt * x[i];
-                        du += lam[n] * B[j + n];
-                        ddt += lam[n] * hprev * a_bar * Arow[n];
-                        dA[d * N + n] += lam[n] * hprev * a_bar * dt;
-                        lam[n] *= a_bar; /* Abar_t·λ_t, the part of λ_{t−1} from h_t */
+                    if (bbar_mode == ORACLE_BBAR_ZOH) {
+                        for (int64_t n = 0; n < N; ++n) {
+                            double h = hs[(t + 1) * N + n], hprev = hs[t * N + n];
+                            double a_bar = exp(dt * Arow[n]);
+                            double c, c_dt, c_a;
+                            zoh_coeff_grads(dt, Arow[n], &c, &c_dt, &c_a);
+                            lam[n] += ds * C[j + n]; /* λ_t */
+                            pC[t * N + n] += ds * h;
+                            pB[t * N + n] += lam[n] * c * x[i];
+                            du += lam[n] * c * B[j + n]; /* here: dx without the D term */
+                            ddt += lam[n] * hprev * a_bar * Arow[n] +
+                                   lam[n] * c_dt * B[j + n] * x[i];
+                            dA[d * N + n] += lam[n] * hprev * a_bar * dt +
+                                             lam[n] * c_a * B[j + n] * x[i];
+                            lam[n] *= a_bar;
+                        }
+                        dx[i] = du + ds * dskip;
+                    } else {
+                        for (int64_t n = 0; n < N; ++n) {
+                            double h = hs[(t + 1) * N + n], hprev = hs[t * N + n];
+                            double a_bar = exp(dt * Arow[n]);
+                            lam[n] += ds * C[j + n]; /* λ_t */
+                            pC[t * N + n] += ds * h;
+                            pB[t * N + n] += lam[n] * dt * x[i];
+                            du += lam[n] * B[j + n];
+                            ddt += lam[n] * hprev * a_bar * Arow[n];
+                            dA[d * N + n] += lam[n] * hprev * a_bar * dt;
+                            lam[n] *= a_bar; /* Abar_t·λ_t, the part of λ_{t−1} from h_t */
+                        }
+                        ddt += du * x[i];
+                        dx[i] = du * dt + ds * dskip;
                     }
-                    ddt += du * x[i];
-                    dx[i] = du * dt + ds * dskip;
                     double v = delta[i] + (delta_bias ? delta_bias[d] : 0.0);
                     double dv = softplus_flag ? ddt * sigmoid(v) : ddt;
                     ddelta[i] = dv;

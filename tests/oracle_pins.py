@@ -438,6 +438,40 @@ def pin_bwd_finite_differences(orc):
             assert _rel(g[gname], fd) < 1e-6, f"{gname} vs finite differences"
 
 
+def pin_bwd_zoh_finite_differences(orc):
+    """The gradient with the ZOH input term c·B·x, c = (exp(Δ·A) − 1)/A
+    ([Guide] §1), against central differences of the forward oracle in the
+    same mode, element by element; one A entry is 0 (the c → Δ limit)."""
+    c, dy, dfinal = _bwd_case(45, gate=True, with_h0=True)
+    c["A"] = c["A"].copy()
+    c["A"][0, 1] = 0.0
+    g = orc.bwd(c["x"], c["delta"], c["A"], c["B"], c["C"], c["D"], c["z"], c["delta_bias"],
+                h0=c["h0"], dy=dy, dfinal=dfinal, threads=1, bbar=1)
+
+    def loss(cc):
+        y, hs = orc.fwd(cc["x"], cc["delta"], cc["A"], cc["B"], cc["C"], cc["D"], cc["z"],
+                        cc["delta_bias"], h0=cc["h0"], threads=1, bbar=1)
+        return float(np.sum(dy * y) + np.sum(dfinal * hs))
+
+    for name, gname in _BWD_GRADS.items():
+        arr = c[name]
+        fd = np.zeros_like(arr)
+        for idx in np.ndindex(arr.shape):
+            e = 1e-6 * max(1.0, abs(arr[idx]))
+            cp = dict(c)
+            cp[name] = arr.copy()
+            cp[name][idx] += e
+            cm = dict(c)
+            cm[name] = arr.copy()
+            cm[name][idx] -= e
+            fd[idx] = (loss(cp) - loss(cm)) / (2 * e)
+        assert _rel(g[gname], fd) < 1e-6, f"ZOH {gname} vs finite differences"
+    # the input-term gradients differ from the Euler ones (the pin has teeth)
+    ge = orc.bwd(c["x"], c["delta"], c["A"], c["B"], c["C"], c["D"], c["z"], c["delta_bias"],
+                 h0=c["h0"], dy=dy, dfinal=dfinal, threads=1)
+    assert _rel(g["dA"], ge["dA"]) > 1e-3 and _rel(g["dx"], ge["dx"]) > 1e-4
+
+
 def pin_bwd_homogeneity(orc):
     """Exact identities (no truncation error). Without the gate, y and h_{L−1}
     are linear in (x, h0) jointly, and y − D·x and h_{L−1} are linear in
@@ -564,6 +598,7 @@ ALL_PINS = [
     pin_euler_vs_zoh, pin_linearity, pin_delta_to_zero, pin_chunked,
     pin_associativity, pin_geometric, pin_decay, pin_cross_entry,
     pin_decode_layout, pin_softplus_and_gate, pin_hand_worked,
-    pin_bwd_finite_differences, pin_bwd_homogeneity, pin_bwd_single_token,
+    pin_bwd_finite_differences, pin_bwd_zoh_finite_differences, pin_bwd_homogeneity,
+    pin_bwd_single_token,
     pin_conv1d_library, pin_conv1d_impulse, pin_conv1d_bwd_finite_differences,
 ]

@@ -71,6 +71,14 @@ MUTANTS = [
      "dpre[i] = dxc[i];"),
     ("bwd_gate_on_ds_dropped", "double ds = z ? dy[i] * silu(z[i]) : dy[i];",
      "double ds = dy[i];"),
+    ("zoh_grad_dA_term_dropped",
+     "dA[d * N + n] += lam[n] * hprev * a_bar * dt +\n"
+     "                                             lam[n] * c_a * B[j + n] * x[i];",
+     "dA[d * N + n] += lam[n] * hprev * a_bar * dt;"),
+    ("zoh_grad_ddelta_uses_c", "lam[n] * c_dt * B[j + n] * x[i];",
+     "lam[n] * c * B[j + n] * x[i];"),
+    ("zoh_grad_limit_wrong", "*c_a = dt * dt * (0.5 + z / 3.0 + z * z / 8.0);",
+     "*c_a = dt * dt * (1.0 + z / 3.0 + z * z / 8.0);"),
 ]
 
 
