@@ -386,6 +386,39 @@ SELSCAN_API int selscan_bwd_conv(const void *x_in, const float *conv_weight,
                                  selscan_dtype_t dtype, void *workspace,
                                  int64_t workspace_bytes, selscan_stream_t stream);
 
+/* Options of selscan_bwd_ex; zero-initialised (or NULL) is selscan_bwd. */
+typedef struct {
+    const float *initial_state;  /* [batch, dim, dstate] or NULL (the forward's) */
+    float *dinitial_state;       /* [batch, dim, dstate] or NULL: its gradient */
+    const float *conv_weight;    /* [dim, conv_width] (conv_width > 0): x is then the
+                                    conv's input and dx its gradient */
+    const float *conv_bias;      /* [dim] or NULL */
+    int conv_width;              /* 0 .. 4 */
+    float *dconv_weight;         /* [dim, conv_width] (conv_width > 0) */
+    float *dconv_bias;           /* [dim] or NULL */
+    int bbar_mode;               /* SELSCAN_BBAR_DELTA or SELSCAN_BBAR_ZOH */
+} selscan_bwd_options_t;
+
+/*
+ * selscan_bwd_ex -- the gradient of selscan_fwd_ex with every option of the
+ * forward that has one: initial state, the conv front end, and the input
+ * term. With SELSCAN_BBAR_ZOH the forward input is c·B·x with
+ * c = (exp(Δ·A[d,n]) − 1)/A[d,n] ("Mamba & State Space Models — Guide
+ * Complet" §1, zero-order hold); its gradient uses ∂c/∂Δ = exp(Δ·A) and
+ * ∂c/∂A = Δ²·f'(Δ·A), f(z) = (e^z − 1)/z. Arguments as selscan_bwd plus
+ * the options; workspace NULL -> allocated on the stream, else at least
+ * selscan_bwd_conv_workspace_bytes() (conv) or selscan_bwd_workspace_bytes()
+ * bytes. Unknown bbar_mode or a negative conv_width: SELSCAN_ERR_BAD_DIM.
+ */
+SELSCAN_API int selscan_bwd_ex(const void *x, const void *delta, const float *A, const void *B,
+                               const void *C, const float *D, const void *z,
+                               const float *delta_bias, int softplus_flag, const void *dy,
+                               const float *dfinal_state, const selscan_bwd_options_t *options,
+                               void *dx, void *ddelta, float *dA, float *dB, float *dC, float *dD,
+                               void *dz, float *ddelta_bias, int64_t batch, int64_t seqlen,
+                               int64_t dim, int64_t dstate, selscan_dtype_t dtype,
+                               void *workspace, int64_t workspace_bytes, selscan_stream_t stream);
+
 /* Host-only: workspace bytes selscan_bwd_conv takes (0 for empty or invalid sizes). */
 SELSCAN_API int64_t selscan_bwd_conv_workspace_bytes(int64_t batch, int64_t seqlen,
                                                      int64_t dim, int64_t dstate);

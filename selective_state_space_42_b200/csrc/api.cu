@@ -536,7 +536,7 @@ int bwd_entry(const void *x, const void *delta, const float *A, const void *B, c
               const float *h0, float *dh0, const float *conv_w,
               const float *conv_b, int conv_width, float *dconv_w, float *dconv_b, void *workspace, int64_t workspace_bytes,
               bool allocate,
-              selscan_stream_t stream_) {
+              selscan_stream_t stream_, int zoh = 0) {
     cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
     if (dtype != SELSCAN_F32 && dtype != SELSCAN_BF16) return SELSCAN_ERR_BAD_DTYPE;
     if (batch < 0 || seqlen < 0 || dim < 0 || batch > 65535) return SELSCAN_ERR_BAD_DIM;
@@ -619,6 +619,7 @@ int bwd_entry(const void *x, const void *delta, const float *A, const void *B, c
     p.dA = dA; p.dB = dB; p.dC = dC; p.dD = dD; p.ddelta_bias = ddelta_bias;
     p.batch = batch; p.seqlen = seqlen; p.dim = dim; p.dstate = (int)dstate;
     p.softplus = softplus_flag ? 1 : 0;
+    p.zoh = zoh ? 1 : 0;
     p.ktiles = (int)ceil_div64(seqlen, selscan::bwd_tile_tokens());
     p.ctiles = (int)ceil_div64(dim, selscan::bwd_tile_channels());
     if (!mul_le(p.ctiles, 1, INT32_MAX) || !mul_le(p.ktiles, 1, INT32_MAX))
@@ -706,6 +707,25 @@ int selscan_bwd_conv(const void *x_in, const float *conv_weight, const float *co
                      dtype, initial_state, dinitial_state, conv_weight, conv_bias, conv_width,
                      dconv_weight, dconv_bias, workspace, workspace_bytes,
                      workspace == nullptr, stream);
+}
+
+int selscan_bwd_ex(const void *x, const void *delta, const float *A, const void *B,
+                   const void *C, const float *D, const void *z, const float *delta_bias,
+                   int softplus_flag, const void *dy, const float *dfinal_state,
+                   const selscan_bwd_options_t *options, void *dx, void *ddelta, float *dA,
+                   float *dB, float *dC, float *dD, void *dz, float *ddelta_bias, int64_t batch,
+                   int64_t seqlen, int64_t dim, int64_t dstate, selscan_dtype_t dtype,
+                   void *workspace, int64_t workspace_bytes, selscan_stream_t stream) {
+    selscan_bwd_options_t o{};
+    if (options) o = *options;
+    if (o.bbar_mode != SELSCAN_BBAR_DELTA && o.bbar_mode != SELSCAN_BBAR_ZOH)
+        return SELSCAN_ERR_BAD_DIM;
+    if (o.conv_width < 0) return SELSCAN_ERR_BAD_DIM;
+    return bwd_entry(x, delta, A, B, C, D, z, delta_bias, softplus_flag, dy, dfinal_state, dx,
+                     ddelta, dA, dB, dC, dD, dz, ddelta_bias, batch, seqlen, dim, dstate, dtype,
+                     o.initial_state, o.dinitial_state, o.conv_weight, o.conv_bias,
+                     o.conv_width, o.dconv_weight, o.dconv_bias, workspace, workspace_bytes,
+                     workspace == nullptr, stream, o.bbar_mode == SELSCAN_BBAR_ZOH);
 }
 
 int64_t selscan_bwd_conv_workspace_bytes(int64_t batch, int64_t seqlen, int64_t dim,

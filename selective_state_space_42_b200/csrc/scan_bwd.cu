@@ -136,6 +136,29 @@ __device__ __forceinline__ void decay16(float dt, float r, const float2 (&Al)[kP
     }
 }
 
+// Derivative of the ZOH factor f(z) = (e^z − 1)/z given a = e^z:
+// f'(z) = (a·(z − 1) + 1)/z²; below |z| = 1/2 the series Σ_m (m + 1)·z^m /
+// (m + 2)! to m = 7 (the next term is under 1e-8 of the sum), above the
+// closed form (no cancellation there: a·(z − 1) + 1 ≥ 0.17).
+__device__ __forceinline__ float zoh_factor_deriv(float z, float a) {
+    float s = fmaf(z, 1.0f / 45360.0f, 1.0f / 5760.0f);
+    s = fmaf(z, s, 1.0f / 840.0f);
+    s = fmaf(z, s, 1.0f / 144.0f);
+    s = fmaf(z, s, 1.0f / 30.0f);
+    s = fmaf(z, s, 1.0f / 8.0f);
+    s = fmaf(z, s, 1.0f / 3.0f);
+    s = fmaf(z, s, 0.5f);
+    return fabsf(z) < 0.5f ? s : fmaf(a, z - 1.0f, 1.0f) / (z * z);
+}
+
+// z = Δ·A[n] (natural units) of states 2j, 2j + 1: structured A[n] =
+// (n + 1)·A[0]; otherwise Al = A·log2 e.
+template <bool kStruct>
+__device__ __forceinline__ float2 zoh_z(float dt, int j, float A0n, const float2 (&Al)[kPairs]) {
+    return kStruct ? make_float2(dt * A0n * (float)(2 * j + 1), dt * A0n * (float)(2 * j + 2))
+                   : make_float2(dt * Al[j].x * kLn2, dt * Al[j].y * kLn2);
+}
+
 // States 4q .. 4q+3 of a shared-memory row as two f32x2 pairs.
 __device__ __forceinline__ void ld_quad(const float *base, int q, float2 &lo, float2 &hi) {
     const float4 v = *reinterpret_cast<const float4 *>(base + 4 * q);
@@ -144,7 +167,7 @@ __device__ __forceinline__ void ld_quad(const float *base, int q, float2 &lo, fl
 }
 __device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
 
-template <typename T, bool kGate, bool kSoftplus, bool kStruct, bool kConv>
+template <typename T, bool kGate, bool kSoftplus, bool kStruct, bool kConv, bool kZoh>
 __device__ __forceinline__ void bwd_body(BwdSmem &S, const BwdParams &p) {
     const int lane = threadIdx.x;
     const long long b = blockIdx.y;
@@ -162,6 +185,7 @@ __device__ __forceinline__ void bwd_body(BwdSmem &S, const BwdParams &p) {
         Al[j] = make_float2(a0 * kLog2e, a1 * kLog2e);
     }
     const float A0l = Al[0].x;
+    const float A0n = A0l * kLn2;  // A[0] itself (natural units)
     const float bias = (active && p.delta_bias) ? p.delta_bias[dd] : 0.0f;
     const float Dv = (active && p.Dskip) ? p.Dskip[dd] : 0.0f;
     const int K = p.ktiles;
@@ -217,6 +241,14 @@ __device__ __forceinline__ void bwd_body(BwdSmem &S, const BwdParams &p) {
                 for (int q = 0; q < 4; ++q) {
                     float2 b0, b1;
                     ld_quad(S.Bs[t], q, b0, b1);
+                    if (kZoh) {  // B·(e^z − 1)/z per state
+                        const float2 z0 = zoh_z<kStruct>(dt, 2 * q, A0n, Al);
+                        const float2 z1 = zoh_z<kStruct>(dt, 2 * q + 1, A0n, Al);
+                        b0 = mul2(b0, make_float2(zoh_factor(z0.x, a[2 * q].x),
+                                                  zoh_factor(z0.y, a[2 * q].y)));
+                        b1 = mul2(b1, make_float2(zoh_factor(z1.x, a[2 * q + 1].x),
+                                                  zoh_factor(z1.y, a[2 * q + 1].y)));
+                    }
                     h[2 * q] = fma2(a[2 * q], h[2 * q], mul2(u2, b0));
                     h[2 * q + 1] = fma2(a[2 * q + 1], h[2 * q + 1], mul2(u2, b1));
                 }
@@ -300,6 +332,14 @@ __device__ __forceinline__ void bwd_body(BwdSmem &S, const BwdParams &p) {
                 float2 b0, b1, c0, c1;
                 ld_quad(S.Bs[t], q, b0, b1);
                 ld_quad(S.Cs[t], q, c0, c1);
+                if (kZoh) {
+                    const float2 z0 = zoh_z<kStruct>(dt, 2 * q, A0n, Al);
+                    const float2 z1 = zoh_z<kStruct>(dt, 2 * q + 1, A0n, Al);
+                    b0 = mul2(b0, make_float2(zoh_factor(z0.x, a[2 * q].x),
+                                              zoh_factor(z0.y, a[2 * q].y)));
+                    b1 = mul2(b1, make_float2(zoh_factor(z1.x, a[2 * q + 1].x),
+                                              zoh_factor(z1.y, a[2 * q + 1].y)));
+                }
                 h[2 * q] = fma2(a[2 * q], h[2 * q], mul2(u2, b0));
                 h[2 * q + 1] = fma2(a[2 * q + 1], h[2 * q + 1], mul2(u2, b1));
                 sacc = fma2(c0, h[2 * q], sacc);
@@ -321,7 +361,9 @@ __device__ __forceinline__ void bwd_body(BwdSmem &S, const BwdParams &p) {
             float2 a[kPairs];
             decay16<kStruct>(sc.x, sc.w, Al, a);
             const float2 ds2 = dup2(sc.z), u2 = dup2(sc.y), dt2 = dup2(sc.x);
-            float2 du2 = make_float2(0.f, 0.f), qp2 = make_float2(0.f, 0.f);
+            // du2: Σ λ·c'·B over states for dx (c' = 1, or the ZOH factor f);
+            // dd2: Σ λ·∂(c'Δ)/∂Δ·B for dΔ (ZOH: a; Δ·B·x: the same sum as du2)
+            float2 du2 = make_float2(0.f, 0.f), dd2 = du2, qp2 = du2;
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 const float4 hq = S.hs[t + 1][j][lane];    // h_t
@@ -339,13 +381,25 @@ __device__ __forceinline__ void bwd_body(BwdSmem &S, const BwdParams &p) {
                     lam[jj] = fma2(ds2, cq[e], lam[jj]);                    // λ_t
                     const float2 hb = mul2(a[jj], hprev[e]);                // Abar_t·h_{t−1}
                     const float2 lh = mul2(lam[jj], hb);
-                    du2 = fma2(lam[jj], bb, du2);
+                    float2 lf = lam[jj];                                    // λ·f (ZOH) or λ
+                    if (kZoh) {
+                        const float2 zz = zoh_z<kStruct>(sc.x, jj, A0n, Al);
+                        const float2 f = make_float2(zoh_factor(zz.x, a[jj].x),
+                                                     zoh_factor(zz.y, a[jj].y));
+                        const float2 fp = make_float2(zoh_factor_deriv(zz.x, a[jj].x),
+                                                      zoh_factor_deriv(zz.y, a[jj].y));
+                        lf = mul2(lam[jj], f);
+                        dd2 = fma2(mul2(lam[jj], a[jj]), bb, dd2);
+                        // ∂c/∂A = Δ²·f'(z): dA += λ·f'·Δ·u·B
+                        dA[jj] = fma2(mul2(lam[jj], fp), mul2(mul2(dt2, u2), bb), dA[jj]);
+                    }
+                    du2 = fma2(lf, bb, du2);
                     if (kStruct)
                         qp2 = fma2(lh, make_float2((float)(2 * jj + 1), (float)(2 * jj + 2)), qp2);
                     else
                         qp2 = fma2(lh, Al[jj], qp2);
                     dA[jj] = fma2(dt2, lh, dA[jj]);
-                    const float2 db = mul2(lam[jj], u2);
+                    const float2 db = mul2(lf, u2);
                     const float2 dc = mul2(ds2, hh[e]);
                     dbv[2 * e] = db.x;
                     dbv[2 * e + 1] = db.y;
@@ -357,12 +411,13 @@ __device__ __forceinline__ void bwd_body(BwdSmem &S, const BwdParams &p) {
                 S.red[4 + j][lane ^ (4 + j)] = make_float4(dcv[0], dcv[1], dcv[2], dcv[3]);
             }
             const float du = du2.x + du2.y;
+            const float dd = kZoh ? dd2.x + dd2.y : du;
             const float qsum = qp2.x + qp2.y;
             // Σ_n λ·hb·A[n]: structured A[n] = (n+1)·A[0]; otherwise Al = A·log2 e
             const float qp = kStruct ? qsum * A0l * kLn2 : qsum * kLn2;
             if (active && tok < p.seqlen) {
                 const long long i = (b * p.seqlen + tok) * p.dim + d;
-                const float ddt = fmaf(du, so.x, qp);
+                const float ddt = fmaf(dd, so.x, qp);
                 const float dv = ddt * so.z;
                 const float dxv = fmaf(du, sc.x, sc.z * Dv);
                 if (kConv)
@@ -422,7 +477,7 @@ __device__ __forceinline__ void bwd_body(BwdSmem &S, const BwdParams &p) {
 
 // A[d, n] == (n+1)·A[d, 0] for every state of every channel of the warp
 // selects the power-ladder decay (the A = −(1..N) initialisation).
-template <typename T, bool kGate, bool kSoftplus, bool kConv>
+template <typename T, bool kGate, bool kSoftplus, bool kConv, bool kZoh>
 __global__ void __launch_bounds__(kChains, 6) scan_bwd_kernel(const BwdParams p) {
     __shared__ BwdSmem S;
     const long long d = (long long)blockIdx.x * kChains + threadIdx.x;
@@ -433,9 +488,9 @@ __global__ void __launch_bounds__(kChains, 6) scan_bwd_kernel(const BwdParams p)
             if (p.A[d * p.dstate + n] != (float)(n + 1) * a0) ok = false;
     }
     if (__all_sync(0xffffffffu, ok))
-        bwd_body<T, kGate, kSoftplus, true, kConv>(S, p);
+        bwd_body<T, kGate, kSoftplus, true, kConv, kZoh>(S, p);
     else
-        bwd_body<T, kGate, kSoftplus, false, kConv>(S, p);
+        bwd_body<T, kGate, kSoftplus, false, kConv, kZoh>(S, p);
 }
 
 // dB[b, t, n] and dC[b, t, n]: sums of the channel-tile partials.
@@ -562,14 +617,20 @@ __global__ void conv_reduce_kernel(const BwdParams p) {
     if (p.dconv_b) p.dconv_b[d] = acc[kMaxConv];
 }
 
-template <typename T, bool kGate, bool kConv>
-cudaError_t launch_conv(const BwdParams &p, cudaStream_t stream) {
+template <typename T, bool kGate, bool kConv, bool kZoh>
+cudaError_t launch_zoh(const BwdParams &p, cudaStream_t stream) {
     const dim3 grid((unsigned)p.ctiles, (unsigned)p.batch);
     if (p.softplus)
-        scan_bwd_kernel<T, kGate, true, kConv><<<grid, kChains, 0, stream>>>(p);
+        scan_bwd_kernel<T, kGate, true, kConv, kZoh><<<grid, kChains, 0, stream>>>(p);
     else
-        scan_bwd_kernel<T, kGate, false, kConv><<<grid, kChains, 0, stream>>>(p);
+        scan_bwd_kernel<T, kGate, false, kConv, kZoh><<<grid, kChains, 0, stream>>>(p);
     return cudaGetLastError();
+}
+
+template <typename T, bool kGate, bool kConv>
+cudaError_t launch_conv(const BwdParams &p, cudaStream_t stream) {
+    return p.zoh ? launch_zoh<T, kGate, kConv, true>(p, stream)
+                 : launch_zoh<T, kGate, kConv, false>(p, stream);
 }
 
 template <typename T, bool kGate>

@@ -165,6 +165,7 @@ struct BwdParams {
     long long batch, seqlen, dim;
     int dstate;
     int softplus;
+    int zoh;       // input term (exp(Δ·A) − 1)/A·B·x instead of Δ·B·x
     int ktiles;    // token tiles per sequence
     int ctiles;    // channel tiles per batch row
 };

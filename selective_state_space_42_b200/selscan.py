@@ -47,6 +47,14 @@ class StepOptions(ctypes.Structure):
                 ("bbar_mode", ctypes.c_int)]
 
 
+class BwdOptions(ctypes.Structure):
+    """selscan_bwd_options_t (include/selscan.h)."""
+    _fields_ = [("initial_state", ctypes.c_void_p), ("dinitial_state", ctypes.c_void_p),
+                ("conv_weight", ctypes.c_void_p), ("conv_bias", ctypes.c_void_p),
+                ("conv_width", ctypes.c_int), ("dconv_weight", ctypes.c_void_p),
+                ("dconv_bias", ctypes.c_void_p), ("bbar_mode", ctypes.c_int)]
+
+
 BBAR_MODES = {"delta": 0, "zoh": 1}
 _i64 = ctypes.c_int64
 _int = ctypes.c_int
@@ -71,6 +79,8 @@ SIGNATURES = {
     "selscan_bwd_conv": (_int, [_vp, _vp, _vp, _int] + [_vp] * 7 + [_int] + [_vp] * 14
                          + [_i64, _i64, _i64, _i64, _int, _vp, _i64, _vp]),
     "selscan_bwd_conv_workspace_bytes": (_i64, [_i64, _i64, _i64, _i64]),
+    "selscan_bwd_ex": (_int, [_vp] * 8 + [_int, _vp, _vp, ctypes.POINTER(BwdOptions)]
+                       + [_vp] * 8 + [_i64, _i64, _i64, _i64, _int, _vp, _i64, _vp]),
     "selscan_bwd_from_state": (_int, [_vp] * 8 + [_int] + [_vp] * 12
                                + [_i64, _i64, _i64, _i64, _int, _vp, _i64, _vp]),
     "selscan_bwd_workspace": (_int, [_vp] * 8 + [_int] + [_vp] * 10
@@ -310,7 +320,7 @@ def _fwd(entry, x, delta, A, B, C, D, z, delta_bias, softplus, y, final_state,
 
 def selscan_bwd(x, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=True,
                 dy=None, dfinal_state=None, stream=None, allocate_in_library=False,
-                initial_state=None, conv_weight=None, conv_bias=None):
+                initial_state=None, conv_weight=None, conv_bias=None, bbar="delta"):
     """Gradient of ``selscan_fwd`` for the loss Σ dy·y + Σ
     dfinal_state·final_state. Inputs as for ``selscan_fwd``; dy has y's shape
     and dtype, dfinal_state is [batch, dim, dstate] float32 or None. Returns a
@@ -325,7 +335,8 @@ def selscan_bwd(x, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=Tru
     ``conv_weight`` [dim, K] (and ``conv_bias``), x is the input of the causal
     conv + SiLU in front of the scan (C ABI ``selscan_bwd_conv``): dx is then
     the gradient w.r.t. that input, and the dict also holds ``dconv_weight``
-    and ``dconv_bias``."""
+    and ``dconv_bias``. ``bbar="zoh"`` differentiates the forward's ZOH input
+    term (C ABI ``selscan_bwd_ex``, which takes all of these options)."""
     torch = _torch()
     if x.dim() != 3:
         raise ValueError("x must be [batch, L, dim]")
@@ -362,6 +373,35 @@ def selscan_bwd(x, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=Tru
         batch, L, dim, N, code,
     ]
     lib = load_library()
+    if bbar not in BBAR_MODES:
+        raise ValueError(f"bbar must be one of {sorted(BBAR_MODES)}")
+    if bbar != "delta":
+        K = 0
+        if conv_weight is not None:
+            if conv_weight.dim() != 2 or conv_weight.shape[0] != dim:
+                raise ValueError("conv_weight must be [dim, K]")
+            K = int(conv_weight.shape[1])
+            out["dconv_weight"] = torch.empty(dim, K, device=dev, dtype=f32)
+            out["dconv_bias"] = (torch.empty(dim, device=dev, dtype=f32)
+                                 if conv_bias is not None else None)
+        if initial_state is not None:
+            out["dh0"] = torch.empty(batch, dim, N, device=dev, dtype=f32)
+        opts = BwdOptions(
+            _ptr(initial_state, "initial_state", (batch, dim, N), f32, dev, required=False),
+            _ptr(out.get("dh0"), "dh0", required=False),
+            _ptr(conv_weight, "conv_weight", (dim, K), f32, dev, required=False),
+            _ptr(conv_bias, "conv_bias", (dim,), f32, dev, required=False), K,
+            _ptr(out.get("dconv_weight"), "dconv_weight", required=False),
+            _ptr(out.get("dconv_bias"), "dconv_bias", required=False), BBAR_MODES[bbar])
+        nbytes = int(lib.selscan_bwd_conv_workspace_bytes(batch, L, dim, N) if K
+                     else lib.selscan_bwd_workspace_bytes(batch, L, dim, N))
+        ws = torch.empty(max(nbytes, 1), device=dev, dtype=torch.uint8)
+        if stream is not None and not isinstance(stream, int):
+            ws.record_stream(stream)
+        eargs = args[:11] + [ctypes.byref(opts)] + args[11:] \
+            + [ws.data_ptr() if nbytes else None, nbytes, _stream_ptr(stream, dev)]
+        _check(lib.selscan_bwd_ex(*eargs))
+        return out
     if conv_weight is not None:
         if conv_weight.dim() != 2 or conv_weight.shape[0] != dim:
             raise ValueError("conv_weight must be [dim, K]")

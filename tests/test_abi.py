@@ -251,3 +251,32 @@ def test_ssd_workspace_bytes(lib):
     # the tensor-core path (128-token chunks) fits in the float32 path's layout
     assert (lib.selscan_ssd_workspace_bytes(2, 1000, 4, 64, 128)
             >= 2 * 4 * 8 * 32768 * 2)
+
+
+_BwdOpts = ss.selscan.BwdOptions  # selscan_bwd_options_t
+
+
+def test_bwd_ex_validation(lib):
+    """selscan_bwd_ex: the options are checked before anything runs; with
+    batch = 0 and dim = 0 nothing has an element (status 0)."""
+    names = ["x", "delta", "A", "B", "C", "D", "z", "delta_bias", "dy", "dfinal",
+             "dx", "ddelta", "dA", "dB", "dC", "dD", "dz", "ddelta_bias"]
+    a = {n: P + 4096 * i for i, n in enumerate(names)}
+    a.update(D=None, z=None, delta_bias=None, dfinal=None, dz=None)
+
+    def call(opts, **kw):
+        b = dict(a, batch=0, dim=0, dstate=16)
+        b.update(kw)
+        return ss.selscan.load_library().selscan_bwd_ex(
+            b["x"], b["delta"], b["A"], b["B"], b["C"], b["D"], b["z"], b["delta_bias"], 1,
+            b["dy"], b["dfinal"], ctypes.byref(opts) if opts is not None else None, b["dx"],
+            b["ddelta"], b["dA"], b["dB"], b["dC"], b["dD"], b["dz"], b["ddelta_bias"],
+            b["batch"], 8, b["dim"], b["dstate"], 1, None, 0, None)
+
+    assert call(None) == 0
+    assert call(_BwdOpts(bbar_mode=1)) == 0
+    assert call(_BwdOpts(bbar_mode=2)) == -2
+    assert call(_BwdOpts(conv_width=-1)) == -2
+    assert call(_BwdOpts(conv_width=5)) == -2
+    assert call(_BwdOpts(bbar_mode=1), dstate=17) == -5  # the gradient takes d_state <= 16
+    assert call(_BwdOpts(bbar_mode=1), batch=1, dim=4, x=None) == -1

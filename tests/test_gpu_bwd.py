@@ -239,3 +239,52 @@ def test_conv_gradient(dtype, K, shape):
     o.update(dx=dx_in, dconv_weight=dw, dconv_bias=dcb)
     _compare_all(got, o, dtype, f"conv K={K}",
                  names=GRADS + ("dh0", "dconv_weight", "dconv_bias"))
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("structured", [True, False])
+@pytest.mark.parametrize("shape", [(2, 37, 40, 16), (1, 130, 33, 7)], ids=str)
+def test_zoh_gradient(dtype, structured, shape):
+    """The gradient of the ZOH input term (C ABI selscan_bwd_ex) against the
+    oracle's, every element; one A entry of 0 exercises the c → Δ limit."""
+    batch, L, dim, N = shape
+    inp, dy, df = _inputs(batch, L, dim, N, dtype, True, seed=900 + L, structured=structured)
+    if not structured:
+        inp["A"][3, 1] = 0.0
+    d = {k: (None if v is None else v.to(DEV)) for k, v in inp.items()}
+    g = ss.selscan_bwd(d["x"], d["delta"], d["A"], d["B"], d["C"], d["D"], d["z"],
+                       d["delta_bias"], dy=dy.to(DEV), dfinal_state=df.to(DEV), bbar="zoh")
+    torch.cuda.synchronize()
+    n = gh.to_np
+    o = oracle.default().bwd(n(inp["x"]), n(inp["delta"]), n(inp["A"]), n(inp["B"]),
+                             n(inp["C"]), n(inp["D"]), n(inp["z"]), n(inp["delta_bias"]),
+                             dy=n(dy), dfinal=n(df), bbar=oracle.BBAR_ZOH)
+    _compare_all(g, o, dtype, f"zoh {shape}")
+
+
+def test_zoh_gradient_with_state_and_conv():
+    """ZOH together with the initial state and the conv front end."""
+    inp, dy, df = _inputs(2, 45, 24, 16, "f32", True, seed=950, structured=False)
+    g0 = torch.Generator().manual_seed(951)
+    h0 = torch.randn(2, 24, 16, generator=g0) * 0.3
+    cw = torch.randn(24, 4, generator=g0) * 0.5
+    cb = torch.randn(24, generator=g0) * 0.1
+    d = {k: (None if v is None else v.to(DEV)) for k, v in inp.items()}
+    g = ss.selscan_bwd(d["x"], d["delta"], d["A"], d["B"], d["C"], d["D"], d["z"],
+                       d["delta_bias"], dy=dy.to(DEV), dfinal_state=df.to(DEV),
+                       initial_state=h0.to(DEV), conv_weight=cw.to(DEV), conv_bias=cb.to(DEV),
+                       bbar="zoh")
+    torch.cuda.synchronize()
+    n = gh.to_np
+    orc = oracle.default()
+    xc = orc.causal_conv1d(n(inp["x"]), n(cw), n(cb))
+    o = orc.bwd(xc, n(inp["delta"]), n(inp["A"]), n(inp["B"]), n(inp["C"]), n(inp["D"]),
+                n(inp["z"]), n(inp["delta_bias"]), h0=n(h0), dy=n(dy), dfinal=n(df),
+                bbar=oracle.BBAR_ZOH)
+    for k in ("ddelta", "dz", "dA", "dB", "dC", "dD", "ddelta_bias", "dh0"):
+        gh.compare(gh.to_np(g[k]), o[k], gh.RTOL["f32"], f"zoh+conv {k}")
+    # dx is w.r.t. the conv's input: the oracle's conv backward of the scan's dx
+    dxin, dw, dcb = orc.causal_conv1d_bwd(n(inp["x"]), n(cw), n(cb), o["dx"])
+    gh.compare(gh.to_np(g["dx"]), dxin, gh.RTOL["f32"], "zoh+conv dx_in")
+    gh.compare(gh.to_np(g["dconv_weight"]), dw, gh.RTOL["f32"], "zoh+conv dconv_weight")
+    gh.compare(gh.to_np(g["dconv_bias"]), dcb, gh.RTOL["f32"], "zoh+conv dconv_bias")
