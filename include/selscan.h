@@ -75,9 +75,9 @@ enum {
 /* Largest d_state of the forward and decode entry points. d_state ≤ 16 takes
  * the TMA-staged and register-resident kernels; 17..256 take a kernel that
  * splits each chain's states over 2-16 lanes (one pass, no chunking,
- * batch ≤ 65535). The gradient (selscan_bwd) takes d_state ≤ 16. */
+ * batch ≤ 65535). The gradient (selscan_bwd) takes d_state ≤ 256 as well. */
 #define SELSCAN_MAX_DSTATE 256
-#define SELSCAN_MAX_DSTATE_BWD 16
+#define SELSCAN_MAX_DSTATE_BWD 256
 
 /*
  * selscan_fwd -- selective scan over whole sequences (the forward pass).
@@ -292,7 +292,8 @@ SELSCAN_API int selscan_state_update(float *state, const void *x, const void *de
  *   dD            [dim]                     float32      NULL -> not written
  *   dz            [batch, seqlen, dim]      dtype        required iff z != NULL
  *   ddelta_bias   [dim]                     float32      NULL -> not written
- *   batch <= 65535; other limits as in selscan_fwd.
+ *   batch <= 65535, dstate 1..SELSCAN_MAX_DSTATE_BWD; other limits as in
+ *   selscan_fwd.
  *
  * Every output is overwritten (not accumulated into); dB, dC, dA, dD and
  * ddelta_bias are float32 whatever `dtype` is. Results are deterministic
@@ -300,7 +301,9 @@ SELSCAN_API int selscan_state_update(float *state, const void *x, const void *de
  * Takes a stream-ordered device workspace (cudaMallocAsync / cudaFreeAsync
  * on `stream`) of selscan_bwd_workspace_bytes() bytes: the state entering
  * every 8-token tile of every chain, and per-32-channel partial sums of dB
- * and dC.
+ * and dC. Above 16 states the chains are walked once per group of 16
+ * states, and the workspace adds three float32 [batch, seqlen, dim] arrays
+ * that carry the per-token sums over the groups.
  */
 SELSCAN_API int selscan_bwd(const void *x, const void *delta, const float *A,
                             const void *B, const void *C, const float *D, const void *z,

@@ -10,6 +10,7 @@
 #include "selscan.h"
 #include "selscan_device.cuh"
 #include "ssd_params.cuh"
+#include "bwd_params.cuh"
 
 namespace {
 
@@ -335,24 +336,29 @@ cudaError_t fwd_run(FwdPlan *plan, void *ws, cudaStream_t stream) {
 namespace {
 
 struct BwdLayout {
-    size_t ckpt, part, pA, pD, pbias, dxc, pconv, total;
+    size_t ckpt, part, pA, pD, pbias, dxc, pconv, acc, total;
 };
+
+// 16-state groups the gradient walks per chain
+int64_t bwd_groups(int64_t dstate) { return (dstate + 15) / 16; }
 
 int64_t ceil_div64(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
 
-BwdLayout bwd_layout(int64_t batch, int64_t seqlen, int64_t dim, bool conv = false) {
+BwdLayout bwd_layout(int64_t batch, int64_t seqlen, int64_t dim, int64_t dstate,
+                     bool conv = false) {
     const int64_t K = ceil_div64(seqlen, selscan::bwd_tile_tokens());
     const int64_t ct = ceil_div64(dim, selscan::bwd_tile_channels());
+    const int64_t G = bwd_groups(dstate);
     BwdLayout l;
     size_t off = 0;
-    l.ckpt = off;
+    l.ckpt = off;  // one group's checkpoints at a time
     off = align256(off + (size_t)(batch * K * dim) * selscan::kMaxN * sizeof(float));
     l.part = off;
-    off = align256(off + (size_t)(batch * ct * seqlen) * 2 * selscan::kMaxN * sizeof(float));
+    off = align256(off + (size_t)(G * batch * ct * seqlen) * 2 * selscan::kMaxN * sizeof(float));
     l.pA = off;
-    off = align256(off + (size_t)(batch * dim) * selscan::kMaxN * sizeof(float));
+    off = align256(off + (size_t)(G * batch * dim) * selscan::kMaxN * sizeof(float));
     l.pD = off;
     off = align256(off + (size_t)(batch * dim) * sizeof(float));
     l.pbias = off;
@@ -366,6 +372,8 @@ BwdLayout bwd_layout(int64_t batch, int64_t seqlen, int64_t dim, bool conv = fal
         off = align256(off + (size_t)(batch * ctt * dim) * (selscan::kMaxConv + 1) *
                                  sizeof(float));
     }
+    l.acc = off;
+    if (G > 1) off = align256(off + 3 * (size_t)(batch * seqlen * dim) * sizeof(float));
     l.total = off;
     return l;
 }
@@ -515,11 +523,11 @@ int selscan_fwd_plan(int64_t batch, int64_t seqlen, int64_t dim, int64_t dstate,
 
 int64_t selscan_bwd_workspace_bytes(int64_t batch, int64_t seqlen, int64_t dim,
                                     int64_t dstate) {
-    if (batch <= 0 || seqlen <= 0 || dim <= 0 || dstate < 1 || dstate > selscan::kMaxN)
+    if (batch <= 0 || seqlen <= 0 || dim <= 0 || dstate < 1 || dstate > SELSCAN_MAX_DSTATE_BWD)
         return 0;
     if (!mul_le(batch, seqlen, kMaxElems) || !mul_le(batch * seqlen, dim, kMaxElems))
         return 0;
-    return (int64_t)bwd_layout(batch, seqlen, dim).total;
+    return (int64_t)bwd_layout(batch, seqlen, dim, dstate).total;
 }
 
 }  // extern "C"
@@ -540,7 +548,7 @@ int bwd_entry(const void *x, const void *delta, const float *A, const void *B, c
     cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
     if (dtype != SELSCAN_F32 && dtype != SELSCAN_BF16) return SELSCAN_ERR_BAD_DTYPE;
     if (batch < 0 || seqlen < 0 || dim < 0 || batch > 65535) return SELSCAN_ERR_BAD_DIM;
-    if (dstate < 1 || dstate > selscan::kMaxN) return SELSCAN_ERR_DSTATE_UNSUPPORTED;
+    if (dstate < 1 || dstate > SELSCAN_MAX_DSTATE_BWD) return SELSCAN_ERR_DSTATE_UNSUPPORTED;
     if (!mul_le(batch, seqlen, kMaxElems) || !mul_le(batch * seqlen, dim, kMaxElems) ||
         !mul_le(batch, dim, kMaxElems))
         return SELSCAN_ERR_BAD_DIM;
@@ -597,7 +605,7 @@ int bwd_entry(const void *x, const void *delta, const float *A, const void *B, c
         return e == cudaSuccess ? SELSCAN_OK : selscan::cuda_fail(e);
     }
 
-    const BwdLayout l = bwd_layout(batch, seqlen, dim, conv_width > 0);
+    const BwdLayout l = bwd_layout(batch, seqlen, dim, dstate, conv_width > 0);
     if (!allocate) {
         if (!workspace) return SELSCAN_ERR_NULL_ARG;
         if (workspace_bytes < (int64_t)l.total) return SELSCAN_ERR_WORKSPACE;
@@ -636,6 +644,8 @@ int bwd_entry(const void *x, const void *delta, const float *A, const void *B, c
     p.pA = reinterpret_cast<float *>(w + l.pA);
     p.pD = reinterpret_cast<float *>(w + l.pD);
     p.pbias = reinterpret_cast<float *>(w + l.pbias);
+    p.groups = (int)bwd_groups(dstate);
+    p.acc = p.groups > 1 ? reinterpret_cast<float *>(w + l.acc) : nullptr;
     p.dxc = conv_width > 0 ? reinterpret_cast<float *>(w + l.dxc) : nullptr;
     p.pconv = conv_width > 0 ? reinterpret_cast<float *>(w + l.pconv) : nullptr;
     e = selscan::launch_scan_bwd(p, dtype == SELSCAN_BF16, stream);
@@ -730,11 +740,11 @@ int selscan_bwd_ex(const void *x, const void *delta, const float *A, const void 
 
 int64_t selscan_bwd_conv_workspace_bytes(int64_t batch, int64_t seqlen, int64_t dim,
                                          int64_t dstate) {
-    if (batch <= 0 || seqlen <= 0 || dim <= 0 || dstate < 1 || dstate > selscan::kMaxN)
+    if (batch <= 0 || seqlen <= 0 || dim <= 0 || dstate < 1 || dstate > SELSCAN_MAX_DSTATE_BWD)
         return 0;
     if (!mul_le(batch, seqlen, kMaxElems) || !mul_le(batch * seqlen, dim, kMaxElems))
         return 0;
-    return (int64_t)bwd_layout(batch, seqlen, dim, true).total;
+    return (int64_t)bwd_layout(batch, seqlen, dim, dstate, true).total;
 }
 
 }  // extern "C"

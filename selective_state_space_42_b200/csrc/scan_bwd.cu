@@ -35,7 +35,7 @@
 // to a per-channel-tile partial buffer, which a second kernel sums over the
 // channel tiles: deterministic, no atomics. dA, dD and ddelta_bias are
 // per-(batch row, channel) partials summed over batch rows the same way.
-#include "selscan_device.cuh"
+#include "bwd_params.cuh"
 
 namespace selscan {
 namespace {
@@ -92,11 +92,12 @@ __device__ __forceinline__ void load_raw(Raw<T> &r, const BwdParams &p, long lon
 }
 
 // Four B and four C elements of the tile for this lane: token lane / 4,
-// states 4·(lane % 4) .. + 3 (zero past the end or past dstate).
+// states ng + 4·(lane % 4) .. + 3 of the 16-state group starting at ng (zero
+// past the end or past dstate).
 template <typename T>
 __device__ __forceinline__ void load_bc(float (&bv)[4], float (&cv)[4], const BwdParams &p,
-                                        long long b, long long t0, int lane, bool withC) {
-    const int t = lane >> 2, n0 = 4 * (lane & 3);
+                                        long long b, long long t0, int lane, bool withC, int ng) {
+    const int t = lane >> 2, n0 = ng + 4 * (lane & 3);
     const long long tok = t0 + t;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -167,21 +168,27 @@ __device__ __forceinline__ void ld_quad(const float *base, int q, float2 &lo, fl
 }
 __device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
 
+// One pass over the chains' sequence for the 16-state group g (states
+// ng = 16·g .. ng + 15). With one group the per-token outputs are written
+// directly; with several, groups before the last add their parts of dΔ, dx
+// and the pre-gate output into p.acc and the last group finishes them.
 template <typename T, bool kGate, bool kSoftplus, bool kStruct, bool kConv, bool kZoh>
-__device__ __forceinline__ void bwd_body(BwdSmem &S, const BwdParams &p) {
+__device__ __forceinline__ void bwd_body(BwdSmem &S, const BwdParams &p, int g) {
     const int lane = threadIdx.x;
     const long long b = blockIdx.y;
     const long long d = (long long)blockIdx.x * kChains + lane;
     const bool active = d < p.dim;
     const int N = p.dstate;
+    const int ng = 16 * g;                  // first state of the group
+    const bool last = g + 1 == p.groups;
     const long long dd = active ? d : 0;
 
     // A as 2^(·) exponents (general A) and the structured-A decay base
     float2 Al[kPairs];
 #pragma unroll
     for (int j = 0; j < kPairs; ++j) {
-        const float a0 = (active && 2 * j < N) ? p.A[dd * N + 2 * j] : 0.0f;
-        const float a1 = (active && 2 * j + 1 < N) ? p.A[dd * N + 2 * j + 1] : 0.0f;
+        const float a0 = (active && ng + 2 * j < N) ? p.A[dd * N + ng + 2 * j] : 0.0f;
+        const float a1 = (active && ng + 2 * j + 1 < N) ? p.A[dd * N + ng + 2 * j + 1] : 0.0f;
         Al[j] = make_float2(a0 * kLog2e, a1 * kLog2e);
     }
     const float A0l = Al[0].x;
@@ -203,14 +210,14 @@ __device__ __forceinline__ void bwd_body(BwdSmem &S, const BwdParams &p) {
         float2 h[kPairs];
 #pragma unroll
         for (int j = 0; j < kPairs; ++j) {
-            const float *h0 = p.h0 + (b * p.dim + dd) * N;
-            h[j] = make_float2((active && p.h0 && 2 * j < N) ? h0[2 * j] : 0.f,
-                               (active && p.h0 && 2 * j + 1 < N) ? h0[2 * j + 1] : 0.f);
+            const float *h0 = p.h0 + (b * p.dim + dd) * N + ng;
+            h[j] = make_float2((active && p.h0 && ng + 2 * j < N) ? h0[2 * j] : 0.f,
+                               (active && p.h0 && ng + 2 * j + 1 < N) ? h0[2 * j + 1] : 0.f);
         }
         Raw<T> cur, nxt;
         float bv[4], cv[4];
         load_raw<T, kGate, false>(cur, p, b, 0, dd, active);
-        load_bc<T>(bv, cv, p, b, 0, lane, false);
+        load_bc<T>(bv, cv, p, b, 0, lane, false, ng);
         float xw[kMaxConv - 1] = {0.f, 0.f, 0.f};  // conv window, zero before token 0
         for (int k = 0; k < K; ++k) {
             const long long t0 = (long long)k * kSeg;
@@ -224,7 +231,7 @@ __device__ __forceinline__ void bwd_body(BwdSmem &S, const BwdParams &p) {
             store_bc(S, bv, cv, lane);
             if (k + 1 < K) {
                 load_raw<T, kGate, false>(nxt, p, b, t0 + kSeg, dd, active);
-                load_bc<T>(bv, cv, p, b, t0 + kSeg, lane, false);
+                load_bc<T>(bv, cv, p, b, t0 + kSeg, lane, false, ng);
             }
             __syncwarp();
 #pragma unroll
@@ -261,22 +268,24 @@ __device__ __forceinline__ void bwd_body(BwdSmem &S, const BwdParams &p) {
     float2 lam[kPairs], dA[kPairs];
 #pragma unroll
     for (int j = 0; j < kPairs; ++j) {
-        const float l0 = (active && p.dfinal && 2 * j < N) ? p.dfinal[(b * p.dim + dd) * N + 2 * j] : 0.f;
+        const float l0 = (active && p.dfinal && ng + 2 * j < N)
+                             ? p.dfinal[(b * p.dim + dd) * N + ng + 2 * j] : 0.f;
         const float l1 =
-            (active && p.dfinal && 2 * j + 1 < N) ? p.dfinal[(b * p.dim + dd) * N + 2 * j + 1] : 0.f;
+            (active && p.dfinal && ng + 2 * j + 1 < N) ? p.dfinal[(b * p.dim + dd) * N + ng + 2 * j + 1] : 0.f;
         lam[j] = make_float2(l0, l1);
         dA[j] = make_float2(0.f, 0.f);
     }
     float accD = 0.f, accBias = 0.f;
-    const int kk = lane & 7, g = lane >> 3;  // reduction role: value group kk, channels 8g..8g+7
-    float *part = p.part + (b * p.ctiles + blockIdx.x) * p.seqlen * kVals;
+    const int kk = lane & 7, cg = lane >> 3;  // reduction role: value group kk, channels 8cg..8cg+7
+    float *part = p.part + ((long long)g * p.batch * p.ctiles + b * p.ctiles + blockIdx.x) *
+                               p.seqlen * kVals;
     Raw<T> cur, nxt;
     float bv[4], cv[4];
     float4 hc[4], hn[4];
     {
         const long long t0 = (long long)(K - 1) * kSeg;
         load_raw<T, kGate, true, kConv>(cur, p, b, t0, dd, active);
-        load_bc<T>(bv, cv, p, b, t0, lane, true);
+        load_bc<T>(bv, cv, p, b, t0, lane, true, ng);
 #pragma unroll
         for (int j = 0; j < 4; ++j)
             hc[j] = active ? ck[(K - 1) * ck_stride + j] : make_float4(0.f, 0.f, 0.f, 0.f);
@@ -287,7 +296,7 @@ __device__ __forceinline__ void bwd_body(BwdSmem &S, const BwdParams &p) {
         store_bc(S, bv, cv, lane);
         if (k > 0) {
             load_raw<T, kGate, true, kConv>(nxt, p, b, t0 - kSeg, dd, active);
-            load_bc<T>(bv, cv, p, b, t0 - kSeg, lane, true);
+            load_bc<T>(bv, cv, p, b, t0 - kSeg, lane, true, ng);
 #pragma unroll
             for (int j = 0; j < 4; ++j)
                 hn[j] = active ? ck[(k - 1) * ck_stride + j] : make_float4(0.f, 0.f, 0.f, 0.f);
@@ -346,7 +355,9 @@ __device__ __forceinline__ void bwd_body(BwdSmem &S, const BwdParams &p) {
                 sacc = fma2(c1, h[2 * q + 1], sacc);
             }
             S.sc[t][lane] = make_float4(dt, u, ds, r);
-            S.so[t][lane] = make_float4(xv, dysz, sg, fmaf(Dv, xv, sacc.x + sacc.y));
+            // s = Σ_n C·h + D·x: the D term once, with the first group
+            S.so[t][lane] = make_float4(xv, dysz, sg,
+                                        fmaf(g == 0 ? Dv : 0.0f, xv, sacc.x + sacc.y));
 #pragma unroll
             for (int j = 0; j < 4; ++j)
                 S.hs[t + 1][j][lane] = make_float4(h[2 * j].x, h[2 * j].y, h[2 * j + 1].x, h[2 * j + 1].y);
@@ -417,24 +428,40 @@ __device__ __forceinline__ void bwd_body(BwdSmem &S, const BwdParams &p) {
             const float qp = kStruct ? qsum * A0l * kLn2 : qsum * kLn2;
             if (active && tok < p.seqlen) {
                 const long long i = (b * p.seqlen + tok) * p.dim + d;
-                const float ddt = fmaf(dd, so.x, qp);
-                const float dv = ddt * so.z;
-                const float dxv = fmaf(du, sc.x, sc.z * Dv);
-                if (kConv)
-                    p.dxc[i] = dxv;  // the conv's input gradient comes from conv_bwd_kernel
-                else
-                    static_cast<T *>(p.dx)[i] = from_f32<T>(dxv);
-                static_cast<T *>(p.ddelta)[i] = from_f32<T>(dv);
-                if (kGate) static_cast<T *>(p.dz)[i] = from_f32<T>(so.w * so.y);
-                accD = fmaf(sc.z, so.x, accD);
-                accBias += dv;
+                float ddt = fmaf(dd, so.x, qp);
+                float dxv = fmaf(du, sc.x, g == 0 ? sc.z * Dv : 0.0f);
+                float sv = so.w;
+                if (p.groups > 1) {  // the sums over the state groups, in group order
+                    const long long n3 = p.batch * p.seqlen * p.dim;
+                    if (g > 0) {
+                        ddt += p.acc[i];
+                        dxv += p.acc[n3 + i];
+                        sv += p.acc[2 * n3 + i];
+                    }
+                    if (!last) {
+                        p.acc[i] = ddt;
+                        p.acc[n3 + i] = dxv;
+                        p.acc[2 * n3 + i] = sv;
+                    }
+                }
+                if (last) {
+                    const float dv = ddt * so.z;
+                    if (kConv)
+                        p.dxc[i] = dxv;  // the conv's input gradient comes from conv_bwd_kernel
+                    else
+                        static_cast<T *>(p.dx)[i] = from_f32<T>(dxv);
+                    static_cast<T *>(p.ddelta)[i] = from_f32<T>(dv);
+                    if (kGate) static_cast<T *>(p.dz)[i] = from_f32<T>(sv * so.y);
+                    accD = fmaf(sc.z, so.x, accD);
+                    accBias += dv;
+                }
             }
             __syncwarp();
             // channel sums of this token's 32 values
             float2 alo = make_float2(0.f, 0.f), ahi = alo;
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
-                const float4 w = S.red[kk][(8 * g + i) ^ kk];
+                const float4 w = S.red[kk][(8 * cg + i) ^ kk];
                 alo = add2(alo, make_float2(w.x, w.y));
                 ahi = add2(ahi, make_float2(w.z, w.w));
             }
@@ -446,8 +473,8 @@ __device__ __forceinline__ void bwd_body(BwdSmem &S, const BwdParams &p) {
                 acc.z += __shfl_xor_sync(0xffffffffu, acc.z, m);
                 acc.w += __shfl_xor_sync(0xffffffffu, acc.w, m);
             }
-            const float mine = g == 0 ? acc.x : (g == 1 ? acc.y : (g == 2 ? acc.z : acc.w));
-            if (tok < p.seqlen) part[tok * kVals + 4 * kk + g] = mine;
+            const float mine = cg == 0 ? acc.x : (cg == 1 ? acc.y : (cg == 2 ? acc.z : acc.w));
+            if (tok < p.seqlen) part[tok * kVals + 4 * kk + cg] = mine;
             __syncwarp();
         }
         cur = nxt;
@@ -457,21 +484,24 @@ __device__ __forceinline__ void bwd_body(BwdSmem &S, const BwdParams &p) {
 
     // the initial state's gradient: λ carried past the first token
     if (active && p.dh0) {
-        float *dh0 = p.dh0 + (b * p.dim + d) * N;
+        float *dh0 = p.dh0 + (b * p.dim + d) * N + ng;
 #pragma unroll
         for (int j = 0; j < kPairs; ++j) {
-            if (2 * j < N) dh0[2 * j] = lam[j].x;
-            if (2 * j + 1 < N) dh0[2 * j + 1] = lam[j].y;
+            if (ng + 2 * j < N) dh0[2 * j] = lam[j].x;
+            if (ng + 2 * j + 1 < N) dh0[2 * j + 1] = lam[j].y;
         }
     }
     // per-(batch row, channel) partials
     if (active) {
-        float4 *pa = reinterpret_cast<float4 *>(p.pA + (b * p.dim + d) * kMaxN);
+        float4 *pa = reinterpret_cast<float4 *>(p.pA + ((long long)g * p.batch * p.dim +
+                                                         b * p.dim + d) * kMaxN);
 #pragma unroll
         for (int j = 0; j < 4; ++j)
             pa[j] = make_float4(dA[2 * j].x, dA[2 * j].y, dA[2 * j + 1].x, dA[2 * j + 1].y);
-        p.pD[b * p.dim + d] = accD;
-        p.pbias[b * p.dim + d] = accBias;
+        if (last) {
+            p.pD[b * p.dim + d] = accD;
+            p.pbias[b * p.dim + d] = accBias;
+        }
     }
 }
 
@@ -481,32 +511,40 @@ template <typename T, bool kGate, bool kSoftplus, bool kConv, bool kZoh>
 __global__ void __launch_bounds__(kChains, 6) scan_bwd_kernel(const BwdParams p) {
     __shared__ BwdSmem S;
     const long long d = (long long)blockIdx.x * kChains + threadIdx.x;
-    bool ok = true;
-    if (d < p.dim) {
+    bool ok = p.groups == 1;  // the power ladder covers states 1..16 of one group
+    if (ok && d < p.dim) {
         const float a0 = p.A[d * p.dstate];
         for (int n = 1; n < p.dstate; ++n)
             if (p.A[d * p.dstate + n] != (float)(n + 1) * a0) ok = false;
     }
-    if (__all_sync(0xffffffffu, ok))
-        bwd_body<T, kGate, kSoftplus, true, kConv, kZoh>(S, p);
-    else
-        bwd_body<T, kGate, kSoftplus, false, kConv, kZoh>(S, p);
+    if (__all_sync(0xffffffffu, ok)) {
+        bwd_body<T, kGate, kSoftplus, true, kConv, kZoh>(S, p, 0);
+    } else {
+        for (int g = 0; g < p.groups; ++g) {
+            bwd_body<T, kGate, kSoftplus, false, kConv, kZoh>(S, p, g);
+            __syncwarp();
+        }
+    }
 }
 
-// dB[b, t, n] and dC[b, t, n]: sums of the channel-tile partials.
+// dB[b, t, n] and dC[b, t, n]: sums of the channel-tile partials (one
+// thread per (batch row, token, value, state group)).
 __global__ void bwd_reduce_bc_kernel(const BwdParams p) {
     const long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-    const long long total = p.batch * p.seqlen * kVals;
-    if (e >= total) return;
-    const long long b = e / (p.seqlen * kVals);
-    const long long rest = e - b * p.seqlen * kVals;  // tok * 32 + v
+    const long long per = p.batch * p.seqlen * kVals;
+    if (e >= per * p.groups) return;
+    const int g = (int)(e / per);
+    const long long eg = e - g * per;
+    const long long b = eg / (p.seqlen * kVals);
+    const long long rest = eg - b * p.seqlen * kVals;  // tok * 32 + v
     const int v = (int)(rest % kVals);
     const long long tok = rest / kVals;
-    const float *src = p.part + (b * p.ctiles) * p.seqlen * kVals + rest;
+    const int n = 16 * g + v % kMaxN;
+    if (n >= p.dstate) return;
+    const float *src = p.part + ((long long)g * p.batch * p.ctiles + b * p.ctiles) * p.seqlen * kVals +
+                       rest;
     float sum = 0.f;
     for (int c = 0; c < p.ctiles; ++c) sum += src[(long long)c * p.seqlen * kVals];
-    const int n = v % kMaxN;
-    if (n >= p.dstate) return;
     float *dst = v < kMaxN ? p.dB : p.dC;
     dst[(b * p.seqlen + tok) * p.dstate + n] = sum;
 }
@@ -514,12 +552,14 @@ __global__ void bwd_reduce_bc_kernel(const BwdParams p) {
 // dA[d, n], dD[d], ddelta_bias[d]: sums over batch rows.
 __global__ void bwd_reduce_params_kernel(const BwdParams p) {
     const long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-    if (e >= p.dim * kMaxN) return;
-    const long long d = e / kMaxN;
-    const int n = (int)(e % kMaxN);
+    const int width = kMaxN * p.groups;
+    if (e >= p.dim * width) return;
+    const long long d = e / width;
+    const int n = (int)(e % width);
     if (n < p.dstate) {
+        const float *src = p.pA + (long long)(n / kMaxN) * p.batch * p.dim * kMaxN + n % kMaxN;
         float s = 0.f;
-        for (long long b = 0; b < p.batch; ++b) s += p.pA[(b * p.dim + d) * kMaxN + n];
+        for (long long b = 0; b < p.batch; ++b) s += src[(b * p.dim + d) * kMaxN];
         p.dA[d * p.dstate + n] = s;
     }
     if (n == 0) {
@@ -661,11 +701,11 @@ cudaError_t launch_scan_bwd(const BwdParams &p, bool bf16, cudaStream_t stream) 
     else
         e = p.z ? launch_gate<float, true>(p, stream) : launch_gate<float, false>(p, stream);
     if (e != cudaSuccess) return e;
-    const long long nbc = p.batch * p.seqlen * kVals;
+    const long long nbc = p.batch * p.seqlen * kVals * p.groups;
     bwd_reduce_bc_kernel<<<(unsigned)((nbc + 255) / 256), 256, 0, stream>>>(p);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    const long long npar = p.dim * kMaxN;
+    const long long npar = p.dim * kMaxN * p.groups;
     bwd_reduce_params_kernel<<<(unsigned)((npar + 255) / 256), 256, 0, stream>>>(p);
     return cudaGetLastError();
 }

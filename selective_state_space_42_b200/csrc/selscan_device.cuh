@@ -142,33 +142,6 @@ struct StepParams {
     int softplus;
 };
 
-// Gradient of the scan (scan_bwd.cu).
-struct BwdParams {
-    const void *x, *delta, *z, *B, *C, *dy;
-    const float *A, *Dskip, *delta_bias, *dfinal;
-    const float *h0;  // state before the first token (NULL: zero)
-    float *dh0;       // its gradient (NULL: not written)
-    const float *conv_w, *conv_b;  // causal conv in front (conv_width > 0)
-    int conv_width;
-    float *dxc;       // with the conv: gradient of the conv output, [batch][seqlen][dim]
-    float *dconv_w, *dconv_b;      // conv gradients (outputs; dconv_b nullable)
-    float *pconv;     // [batch][conv tiles][dim][kMaxConv + 1] conv-gradient partials
-    int conv_tiles;   // token tiles of the conv-gradient kernel
-    void *dx, *ddelta, *dz;
-    float *dA, *dB, *dC, *dD, *ddelta_bias;  // outputs written by the reduction kernel
-    // workspace
-    float *ckpt;   // [batch][ktiles][dim][16]: state entering each token tile
-    float *part;   // [batch][ctiles][seqlen][32]: per channel tile, Σ over its channels of dB (0..15), dC (16..31)
-    float *pA;     // [batch][dim][16]: Σ over tokens of dA
-    float *pD;     // [batch][dim]
-    float *pbias;  // [batch][dim]
-    long long batch, seqlen, dim;
-    int dstate;
-    int softplus;
-    int zoh;       // input term (exp(Δ·A) − 1)/A·B·x instead of Δ·B·x
-    int ktiles;    // token tiles per sequence
-    int ctiles;    // channel tiles per batch row
-};
 
 // The library's device error word (defined with the TMA scan).
 cudaError_t device_status_address(int **p);
@@ -213,12 +186,8 @@ cudaError_t launch_carry(const ScanParams &p, cudaStream_t stream);
 
 // Host-side launchers (one translation unit per kernel family).
 cudaError_t launch_scan(const ScanParams &p, bool bf16, cudaStream_t stream);
-cudaError_t launch_scan_bwd(const BwdParams &p, bool bf16, cudaStream_t stream);
 cudaError_t launch_scan_wide(const ScanParams &p, bool bf16, cudaStream_t stream);
 int wide_max_dstate();
-int bwd_tile_tokens();
-int bwd_tile_channels();
-int bwd_conv_tile_tokens();
 cudaError_t launch_state_update(const StepParams &p, bool bf16, cudaStream_t stream);
 int scan_channels_per_cta();
 int scan_tile_tokens();

@@ -163,7 +163,7 @@ def test_bwd_validation(lib):
     assert bwd(lib, batch=-1) == -2
     assert bwd(lib, batch=70000, dim=4) == -2  # batch rows are a grid dimension
     assert bwd(lib, dstate=0) == -5
-    assert bwd(lib, dstate=17) == -5  # the gradient takes d_state <= 16
+    assert bwd(lib, dstate=257) == -5  # the gradient takes d_state <= 256
     full = dict(batch=1, dim=4)
     assert bwd(lib, x=None, **full) == -1
     assert bwd(lib, dy=None, **full) == -1
@@ -181,10 +181,13 @@ def test_bwd_validation(lib):
 
 def test_bwd_workspace_bytes(lib):
     assert lib.selscan_bwd_workspace_bytes(0, 8, 4, 16) == 0
-    assert lib.selscan_bwd_workspace_bytes(1, 8, 4, 17) == 0
+    assert lib.selscan_bwd_workspace_bytes(1, 8, 4, 257) == 0
     # one 16-token tile, one 32-channel tile: checkpoints 4·16·4 B, partials
     # 8·32·4 B, per-channel partials 4·(16 + 2)·4 B, each rounded up to 256 B
     assert lib.selscan_bwd_workspace_bytes(1, 8, 4, 16) == 256 + 1024 + 256 + 256 + 256
+    # 17 states: two 16-state groups, so the dB/dC and dA partials double and
+    # three float32 [1, 8, 4] arrays carry the per-token sums over the groups
+    assert lib.selscan_bwd_workspace_bytes(1, 8, 4, 17) == 256 + 2048 + 512 + 256 + 256 + 512
 
 
 def test_plans_of_the_workloads(lib):
@@ -278,5 +281,5 @@ def test_bwd_ex_validation(lib):
     assert call(_BwdOpts(bbar_mode=2)) == -2
     assert call(_BwdOpts(conv_width=-1)) == -2
     assert call(_BwdOpts(conv_width=5)) == -2
-    assert call(_BwdOpts(bbar_mode=1), dstate=17) == -5  # the gradient takes d_state <= 16
+    assert call(_BwdOpts(bbar_mode=1), dstate=257) == -5  # the gradient takes d_state <= 256
     assert call(_BwdOpts(bbar_mode=1), batch=1, dim=4, x=None) == -1

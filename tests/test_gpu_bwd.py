@@ -288,3 +288,73 @@ def test_zoh_gradient_with_state_and_conv():
     gh.compare(gh.to_np(g["dx"]), dxin, gh.RTOL["f32"], "zoh+conv dx_in")
     gh.compare(gh.to_np(g["dconv_weight"]), dw, gh.RTOL["f32"], "zoh+conv dconv_weight")
     gh.compare(gh.to_np(g["dconv_bias"]), dcb, gh.RTOL["f32"], "zoh+conv dconv_bias")
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("N", [17, 32, 64, 100, 256])
+@pytest.mark.parametrize("structured", [True, False])
+def test_wide_state_gradient(dtype, N, structured):
+    """d_state above 16: the chains are walked once per group of 16 states and
+    the per-token sums over the groups carried in float32; every element
+    against the oracle (which takes any d_state)."""
+    inp, dy, df = _inputs(2, 37, 40, N, dtype, True, seed=1100 + N, structured=structured)
+    g = _gpu_bwd(inp, dy, df)
+    torch.cuda.synchronize()
+    _compare_all(g, _oracle_bwd(inp, dy, df), dtype, f"N={N}")
+
+
+def test_wide_state_gradient_with_options():
+    """d_state 48 with the initial state, the conv front end and the ZOH term."""
+    N = 48
+    inp, dy, df = _inputs(2, 45, 24, N, "f32", True, seed=1200, structured=False)
+    g0 = torch.Generator().manual_seed(1201)
+    h0 = torch.randn(2, 24, N, generator=g0) * 0.3
+    cw = torch.randn(24, 4, generator=g0) * 0.5
+    cb = torch.randn(24, generator=g0) * 0.1
+    d = {k: (None if v is None else v.to(DEV)) for k, v in inp.items()}
+    n = gh.to_np
+    orc = oracle.default()
+    xc = orc.causal_conv1d(n(inp["x"]), n(cw), n(cb))
+    for bbar, mode in (("delta", oracle.BBAR_DELTA), ("zoh", oracle.BBAR_ZOH)):
+        g = ss.selscan_bwd(d["x"], d["delta"], d["A"], d["B"], d["C"], d["D"], d["z"],
+                           d["delta_bias"], dy=dy.to(DEV), dfinal_state=df.to(DEV),
+                           initial_state=h0.to(DEV), conv_weight=cw.to(DEV),
+                           conv_bias=cb.to(DEV), bbar=bbar)
+        torch.cuda.synchronize()
+        o = orc.bwd(xc, n(inp["delta"]), n(inp["A"]), n(inp["B"]), n(inp["C"]), n(inp["D"]),
+                    n(inp["z"]), n(inp["delta_bias"]), h0=n(h0), dy=n(dy), dfinal=n(df),
+                    bbar=mode)
+        for k in ("ddelta", "dz", "dA", "dB", "dC", "dD", "ddelta_bias", "dh0"):
+            gh.compare(gh.to_np(g[k]), o[k], gh.RTOL["f32"], f"N={N} {bbar} {k}")
+        dxin, dw, dcb = orc.causal_conv1d_bwd(n(inp["x"]), n(cw), n(cb), o["dx"])
+        gh.compare(gh.to_np(g["dx"]), dxin, gh.RTOL["f32"], f"N={N} {bbar} dx_in")
+        gh.compare(gh.to_np(g["dconv_weight"]), dw, gh.RTOL["f32"], f"N={N} {bbar} dconv_weight")
+        gh.compare(gh.to_np(g["dconv_bias"]), dcb, gh.RTOL["f32"], f"N={N} {bbar} dconv_bias")
+
+
+def test_wide_state_gradient_layer_sampled():
+    """A Mamba-2-sized layer (2 × 2048 tokens, 2048 channels, d_state 128):
+    the gradient of a channel sample against the oracle on those channels
+    (the channels are independent), and dC, a sum over all channels, by the
+    identity Σ dC·C = Σ dy·(y − D·x·silu(z)) (y − D·x·silu(z) is linear and
+    homogeneous in C; no final-state gradient)."""
+    w = wl.ScanWorkload("wide_bwd", 2, 2048, 2048, 128, "bf16", gate=True, seed=1300)
+    inp = wl.make_scan_inputs(w)
+    g0 = torch.Generator().manual_seed(1301)
+    dy = torch.randn(2, 2048, 2048, generator=g0).to(torch.bfloat16)
+    g = _gpu_bwd(inp, dy, None)
+    torch.cuda.synchronize()
+    chans = list(wl.channel_subset(2048, 64))
+    o = _oracle_bwd(inp, dy, None, channels=chans)
+    for k in ("dx", "ddelta", "dz"):
+        gh.compare(gh.to_np(g[k][:, :, chans]), o[k], gh.RTOL["bf16"], f"layer {k}")
+    for k in ("dA", "dD", "ddelta_bias"):
+        gh.compare(gh.to_np(g[k][chans]), o[k], gh.RTOL["bf16"], f"layer {k}")
+    d = {k: (None if v is None else v.to(DEV)) for k, v in inp.items()}
+    y = ss.selscan_fwd(d["x"], d["delta"], d["A"], d["B"], d["C"], d["D"], d["z"],
+                       d["delta_bias"])
+    zz = d["z"].double()
+    rest = y.double() - d["D"].double() * d["x"].double() * zz * torch.sigmoid(zz)
+    rhs = float((dy.to(DEV).double() * rest).sum())
+    lhs = float((g["dC"].double() * d["C"].double()).sum())
+    assert abs(lhs - rhs) <= 2e-2 * abs(rhs), (lhs, rhs)
