@@ -353,8 +353,8 @@ BwdLayout bwd_layout(int64_t batch, int64_t seqlen, int64_t dim, int64_t dstate,
     const int64_t G = bwd_groups(dstate);
     BwdLayout l;
     size_t off = 0;
-    l.ckpt = off;  // one group's checkpoints at a time
-    off = align256(off + (size_t)(batch * K * dim) * selscan::kMaxN * sizeof(float));
+    l.ckpt = off;  // every group's checkpoints (the groups run side by side)
+    off = align256(off + (size_t)(G * batch * K * dim) * selscan::kMaxN * sizeof(float));
     l.part = off;
     off = align256(off + (size_t)(G * batch * ct * seqlen) * 2 * selscan::kMaxN * sizeof(float));
     l.pA = off;
@@ -373,7 +373,7 @@ BwdLayout bwd_layout(int64_t batch, int64_t seqlen, int64_t dim, int64_t dstate,
                                  sizeof(float));
     }
     l.acc = off;
-    if (G > 1) off = align256(off + 3 * (size_t)(batch * seqlen * dim) * sizeof(float));
+    if (G > 1) off = align256(off + 3 * (size_t)(G * batch * seqlen * dim) * sizeof(float));
     l.total = off;
     return l;
 }

@@ -21,19 +21,19 @@ struct BwdParams {
     void *dx, *ddelta, *dz;
     float *dA, *dB, *dC, *dD, *ddelta_bias;  // outputs written by the reduction kernel
     // workspace
-    float *ckpt;   // [batch][ktiles][dim][16]: state of one 16-state group entering each token tile
+    float *ckpt;   // [groups][batch][ktiles][dim][16]: state of each 16-state group entering each token tile
     float *part;   // [groups][batch][ctiles][seqlen][32]: per channel tile, Σ over its channels
                    // of dB (0..15), dC (16..31) of the group's states
     float *pA;     // [groups][batch][dim][16]: Σ over tokens of dA
-    float *acc;    // groups > 1: [3][batch][seqlen][dim] float32 sums over the groups done so
-                   // far of dΔ (before the softplus derivative), dx and the pre-gate output
+    float *acc;    // groups > 1: [groups][3][batch][seqlen][dim] float32: each group's part of
+                   // dΔ (before the softplus derivative), dx and the pre-gate output
     float *pD;     // [batch][dim]
     float *pbias;  // [batch][dim]
     long long batch, seqlen, dim;
     int dstate;
     int softplus;
     int zoh;       // input term (exp(Δ·A) − 1)/A·B·x instead of Δ·B·x
-    int groups;    // ⌈dstate / 16⌉: 16-state groups, walked one after another per chain
+    int groups;    // ⌈dstate / 16⌉: 16-state groups, one grid plane each
     int ktiles;    // token tiles per sequence
     int ctiles;    // channel tiles per batch row
 };

@@ -170,8 +170,9 @@ __device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a
 
 // One pass over the chains' sequence for the 16-state group g (states
 // ng = 16·g .. ng + 15). With one group the per-token outputs are written
-// directly; with several, groups before the last add their parts of dΔ, dx
-// and the pre-gate output into p.acc and the last group finishes them.
+// directly; with several, every group writes its parts of dΔ, dx and the
+// pre-gate output to its own slice of p.acc, and bwd_groups_finish_kernel
+// sums them.
 template <typename T, bool kGate, bool kSoftplus, bool kStruct, bool kConv, bool kZoh>
 __device__ __forceinline__ void bwd_body(BwdSmem &S, const BwdParams &p, int g) {
     const int lane = threadIdx.x;
@@ -180,7 +181,6 @@ __device__ __forceinline__ void bwd_body(BwdSmem &S, const BwdParams &p, int g) 
     const bool active = d < p.dim;
     const int N = p.dstate;
     const int ng = 16 * g;                  // first state of the group
-    const bool last = g + 1 == p.groups;
     const long long dd = active ? d : 0;
 
     // A as 2^(·) exponents (general A) and the structured-A decay base
@@ -202,7 +202,8 @@ __device__ __forceinline__ void bwd_body(BwdSmem &S, const BwdParams &p, int g) 
         load_conv_taps(p.conv_w, p.conv_width, dd, cw);
         cbias = p.conv_b ? p.conv_b[dd] : 0.0f;
     }
-    float4 *ck = reinterpret_cast<float4 *>(p.ckpt) + ((b * K) * p.dim + dd) * 4;
+    float4 *ck = reinterpret_cast<float4 *>(p.ckpt) +
+                 ((((long long)g * p.batch + b) * K) * p.dim + dd) * 4;  // this group's region
     const long long ck_stride = p.dim * 4;  // float4s between consecutive tiles
 
     // ---- 1. forward sweep: checkpoints ------------------------------------------
@@ -431,20 +432,14 @@ __device__ __forceinline__ void bwd_body(BwdSmem &S, const BwdParams &p, int g) 
                 float ddt = fmaf(dd, so.x, qp);
                 float dxv = fmaf(du, sc.x, g == 0 ? sc.z * Dv : 0.0f);
                 float sv = so.w;
-                if (p.groups > 1) {  // the sums over the state groups, in group order
+                if (p.groups > 1) {  // this group's parts, summed by the finish kernel
                     const long long n3 = p.batch * p.seqlen * p.dim;
-                    if (g > 0) {
-                        ddt += p.acc[i];
-                        dxv += p.acc[n3 + i];
-                        sv += p.acc[2 * n3 + i];
-                    }
-                    if (!last) {
-                        p.acc[i] = ddt;
-                        p.acc[n3 + i] = dxv;
-                        p.acc[2 * n3 + i] = sv;
-                    }
-                }
-                if (last) {
+                    float *a = p.acc + (long long)g * 3 * n3;
+                    a[i] = ddt;
+                    a[n3 + i] = dxv;
+                    a[2 * n3 + i] = sv;
+                    if (g == 0) accD = fmaf(sc.z, so.x, accD);
+                } else {
                     const float dv = ddt * so.z;
                     if (kConv)
                         p.dxc[i] = dxv;  // the conv's input gradient comes from conv_bwd_kernel
@@ -498,10 +493,8 @@ __device__ __forceinline__ void bwd_body(BwdSmem &S, const BwdParams &p, int g) 
 #pragma unroll
         for (int j = 0; j < 4; ++j)
             pa[j] = make_float4(dA[2 * j].x, dA[2 * j].y, dA[2 * j + 1].x, dA[2 * j + 1].y);
-        if (last) {
-            p.pD[b * p.dim + d] = accD;
-            p.pbias[b * p.dim + d] = accBias;
-        }
+        if (g == 0) p.pD[b * p.dim + d] = accD;
+        if (p.groups == 1) p.pbias[b * p.dim + d] = accBias;  // else: the finish kernel
     }
 }
 
@@ -517,14 +510,50 @@ __global__ void __launch_bounds__(kChains, 6) scan_bwd_kernel(const BwdParams p)
         for (int n = 1; n < p.dstate; ++n)
             if (p.A[d * p.dstate + n] != (float)(n + 1) * a0) ok = false;
     }
-    if (__all_sync(0xffffffffu, ok)) {
+    if (__all_sync(0xffffffffu, ok))
         bwd_body<T, kGate, kSoftplus, true, kConv, kZoh>(S, p, 0);
-    } else {
+    else
+        bwd_body<T, kGate, kSoftplus, false, kConv, kZoh>(S, p, (int)blockIdx.z);
+}
+
+// Above 16 states: the per-token sums over the state groups, in group order
+// (deterministic), and what follows from them — dx (or the conv output's
+// gradient), ddelta = dΔ·σ(delta + bias), dz = dy·s·silu'(z) — plus the
+// per-(batch row, channel) sum of ddelta. One thread per (batch row,
+// channel) walks the tokens; consecutive threads take consecutive channels.
+template <typename T, bool kGate, bool kConv>
+__global__ void bwd_groups_finish_kernel(const BwdParams p) {
+    const long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (e >= p.batch * p.dim) return;
+    const long long b = e / p.dim, d = e - b * p.dim;
+    const long long n3 = p.batch * p.seqlen * p.dim;
+    const float bias = p.delta_bias ? p.delta_bias[d] : 0.0f;
+    float sb = 0.0f;
+    for (long long t = 0; t < p.seqlen; ++t) {
+        const long long i = (b * p.seqlen + t) * p.dim + d;
+        float ddt = 0.f, dxv = 0.f, sv = 0.f;
         for (int g = 0; g < p.groups; ++g) {
-            bwd_body<T, kGate, kSoftplus, false, kConv, kZoh>(S, p, g);
-            __syncwarp();
+            const float *a = p.acc + (long long)g * 3 * n3;
+            ddt += a[i];
+            dxv += a[n3 + i];
+            sv += a[2 * n3 + i];
         }
+        const float v = ldg_f32(static_cast<const T *>(p.delta) + i) + bias;
+        const float dv = p.softplus ? ddt * sigmoid_f32(v) : ddt;
+        if (kConv)
+            p.dxc[i] = dxv;
+        else
+            static_cast<T *>(p.dx)[i] = from_f32<T>(dxv);
+        static_cast<T *>(p.ddelta)[i] = from_f32<T>(dv);
+        if (kGate) {
+            const float zv = ldg_f32(static_cast<const T *>(p.z) + i);
+            const float dyv = ldg_f32(static_cast<const T *>(p.dy) + i);
+            const float sgz = sigmoid_f32(zv);
+            static_cast<T *>(p.dz)[i] = from_f32<T>(sv * (dyv * sgz * fmaf(zv, 1.0f - sgz, 1.0f)));
+        }
+        sb += dv;
     }
+    p.pbias[b * p.dim + d] = sb;
 }
 
 // dB[b, t, n] and dC[b, t, n]: sums of the channel-tile partials (one
@@ -659,7 +688,7 @@ __global__ void conv_reduce_kernel(const BwdParams p) {
 
 template <typename T, bool kGate, bool kConv, bool kZoh>
 cudaError_t launch_zoh(const BwdParams &p, cudaStream_t stream) {
-    const dim3 grid((unsigned)p.ctiles, (unsigned)p.batch);
+    const dim3 grid((unsigned)p.ctiles, (unsigned)p.batch, (unsigned)p.groups);
     if (p.softplus)
         scan_bwd_kernel<T, kGate, true, kConv, kZoh><<<grid, kChains, 0, stream>>>(p);
     else
@@ -669,8 +698,12 @@ cudaError_t launch_zoh(const BwdParams &p, cudaStream_t stream) {
 
 template <typename T, bool kGate, bool kConv>
 cudaError_t launch_conv(const BwdParams &p, cudaStream_t stream) {
-    return p.zoh ? launch_zoh<T, kGate, kConv, true>(p, stream)
-                 : launch_zoh<T, kGate, kConv, false>(p, stream);
+    cudaError_t e = p.zoh ? launch_zoh<T, kGate, kConv, true>(p, stream)
+                          : launch_zoh<T, kGate, kConv, false>(p, stream);
+    if (e != cudaSuccess || p.groups == 1) return e;
+    const long long n = p.batch * p.dim;
+    bwd_groups_finish_kernel<T, kGate, kConv><<<(unsigned)((n + 127) / 128), 128, 0, stream>>>(p);
+    return cudaGetLastError();
 }
 
 template <typename T, bool kGate>

@@ -185,9 +185,10 @@ def test_bwd_workspace_bytes(lib):
     # one 16-token tile, one 32-channel tile: checkpoints 4·16·4 B, partials
     # 8·32·4 B, per-channel partials 4·(16 + 2)·4 B, each rounded up to 256 B
     assert lib.selscan_bwd_workspace_bytes(1, 8, 4, 16) == 256 + 1024 + 256 + 256 + 256
-    # 17 states: two 16-state groups, so the dB/dC and dA partials double and
-    # three float32 [1, 8, 4] arrays carry the per-token sums over the groups
-    assert lib.selscan_bwd_workspace_bytes(1, 8, 4, 17) == 256 + 2048 + 512 + 256 + 256 + 512
+    # 17 states: two 16-state groups side by side, so the checkpoints and the
+    # dB/dC and dA partials double, and each group writes three float32
+    # [1, 8, 4] per-token arrays for the finishing sum
+    assert lib.selscan_bwd_workspace_bytes(1, 8, 4, 17) == 512 + 2048 + 512 + 256 + 256 + 768
 
 
 def test_plans_of_the_workloads(lib):
