@@ -301,9 +301,10 @@ SELSCAN_API int selscan_state_update(float *state, const void *x, const void *de
  * Takes a stream-ordered device workspace (cudaMallocAsync / cudaFreeAsync
  * on `stream`) of selscan_bwd_workspace_bytes() bytes: the state entering
  * every 8-token tile of every chain, and per-32-channel partial sums of dB
- * and dC. Above 16 states the chains are walked once per group of 16
- * states, and the workspace adds three float32 [batch, seqlen, dim] arrays
- * that carry the per-token sums over the groups.
+ * and dC. Above 16 states the states go in groups of 16 computed side by
+ * side; the workspace then holds every group's checkpoints and partials and
+ * three float32 [batch, seqlen, dim] arrays per group, summed in group
+ * order.
  */
 SELSCAN_API int selscan_bwd(const void *x, const void *delta, const float *A,
                             const void *B, const void *C, const float *D, const void *z,
