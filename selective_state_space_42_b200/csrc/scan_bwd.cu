@@ -35,6 +35,14 @@
 // to a per-channel-tile partial buffer, which a second kernel sums over the
 // channel tiles: deterministic, no atomics. dA, dD and ddelta_bias are
 // per-(batch row, channel) partials summed over batch rows the same way.
+//
+// Above 16 states the states go in groups of 16, one grid plane per group,
+// each the pass above on its states. The recurrence, λ and the per-state
+// gradients separate by state; the per-token sums over n (dx, dΔ and the
+// pre-gate output s, which dz needs) are written per group and summed in
+// group order by bwd_groups_finish_kernel, which also applies σ and silu'.
+// The ZOH input term (p.zoh) scales B by f(Δ·A[n]) = (e^z − 1)/z in the
+// recomputed forward and takes f and f' into dB, dx, dΔ and dA.
 #include "bwd_params.cuh"
 
 namespace selscan {
