@@ -18,7 +18,7 @@ LIB_PATH = os.path.join(HERE, "libselscan.so")
 SELSCAN_F32 = 0
 SELSCAN_BF16 = 1
 SELSCAN_MAX_DSTATE = 256
-SELSCAN_MAX_DSTATE_BWD = 16
+SELSCAN_MAX_DSTATE_BWD = 256
 
 STATUS = {
     0: "SELSCAN_OK", -1: "SELSCAN_ERR_NULL_ARG", -2: "SELSCAN_ERR_BAD_DIM",

@@ -284,3 +284,14 @@ def test_bwd_ex_validation(lib):
     assert call(_BwdOpts(conv_width=5)) == -2
     assert call(_BwdOpts(bbar_mode=1), dstate=257) == -5  # the gradient takes d_state <= 256
     assert call(_BwdOpts(bbar_mode=1), batch=1, dim=4, x=None) == -1
+
+
+def test_binding_constants_match_the_header():
+    """The binding's copies of the header's limits and status codes."""
+    text = open(os.path.join(ROOT, "include", "selscan.h")).read()
+    defines = dict(re.findall(r"#define\s+(SELSCAN_\w+)\s+(\d+)", text))
+    for name in ("SELSCAN_MAX_DSTATE", "SELSCAN_MAX_DSTATE_BWD"):
+        assert int(defines[name]) == getattr(ss.selscan, name), name
+    codes = dict((n, int(v)) for n, v in re.findall(r"(SELSCAN_(?:OK|ERR_\w+))\s*=\s*(-?\d+)", text))
+    for code, name in ss.selscan.STATUS.items():
+        assert codes[name] == code, name
