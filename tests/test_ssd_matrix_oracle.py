@@ -4,6 +4,7 @@ structure (CPU only). Source: "Mamba & State Space Models — Guide Complet"
 §5 "Mamba-2" / "SSD — State Space Dual"."""
 import numpy as np
 import pytest
+from hypothesis import given, settings, strategies as st
 
 from oracle import ssd_matrix
 
@@ -107,3 +108,23 @@ def test_a_shifted_mask_is_caught(orc):
             zh = c["z"][b, :, h * P:(h + 1) * P]
             y[b, :, h * P:(h + 1) * P] = yh * zh / (1.0 + np.exp(-zh))
     assert float(np.max(np.abs(y - yo))) > 1e-3 * float(np.max(np.abs(yo)))
+
+
+
+@settings(max_examples=40, deadline=None)
+@given(batch=st.integers(1, 2), T=st.integers(1, 24), H=st.integers(1, 3), P=st.integers(1, 4),
+       N=st.integers(1, 6), seed=st.integers(0, 10_000), gate=st.booleans(), h0=st.booleans(),
+       softplus=st.booleans())
+def test_matrix_form_equals_recurrence_any_shape(orc, batch, T, H, P, N, seed, gate, h0, softplus):
+    """The dense semiseparable form and the recurrence agree to float64
+    rounding on every small shape, with or without gate, initial state and
+    softplus."""
+    c = _case(seed, batch=batch, T=T, H=H, P=P, N=N, gate=gate, h0=h0)
+    if not softplus:
+        c["dt"] = np.abs(c["dt"]) * 0.2 + 0.01
+        c["dt_bias"] = np.zeros_like(c["dt_bias"])
+    y, hf = ssd_matrix.ssd_matrix_form(c["x"], c["dt"], c["A"], c["B"], c["C"], c["D"], c["z"],
+                                       c["dt_bias"], softplus=softplus, h0=c["h0"])
+    yo, ho = _scan(orc, c, P, softplus=softplus)
+    _close(y, yo)
+    _close(hf, ho)
