@@ -438,6 +438,32 @@ def pin_bwd_finite_differences(orc):
             assert _rel(g[gname], fd) < 1e-6, f"{gname} vs finite differences"
 
 
+def pin_bwd_wide_state_finite_differences(orc):
+    """The gradient at d_state 20 (more states than one 16-state group of the
+    CUDA gradient) against central differences of the forward oracle, element
+    by element, with gate and initial state."""
+    c, dy, dfinal = _bwd_case(47, gate=True, with_h0=True, batch=1, L=4, D=2, N=20)
+    g = _bwd_of(orc, c, dy, dfinal, True)
+
+    def loss(cc):
+        y, hs = _fwd_of(orc, cc, True)
+        return float(np.sum(dy * y) + np.sum(dfinal * hs))
+
+    for name, gname in _BWD_GRADS.items():
+        arr = c[name]
+        fd = np.zeros_like(arr)
+        for idx in np.ndindex(arr.shape):
+            e = 1e-6 * max(1.0, abs(arr[idx]))
+            cp = dict(c)
+            cp[name] = arr.copy()
+            cp[name][idx] += e
+            cm = dict(c)
+            cm[name] = arr.copy()
+            cm[name][idx] -= e
+            fd[idx] = (loss(cp) - loss(cm)) / (2 * e)
+        assert _rel(g[gname], fd) < 1e-6, f"N=20 {gname} vs finite differences"
+
+
 def pin_bwd_zoh_finite_differences(orc):
     """The gradient with the ZOH input term c·B·x, c = (exp(Δ·A) − 1)/A
     ([Guide] §1), against central differences of the forward oracle in the
@@ -598,7 +624,8 @@ ALL_PINS = [
     pin_euler_vs_zoh, pin_linearity, pin_delta_to_zero, pin_chunked,
     pin_associativity, pin_geometric, pin_decay, pin_cross_entry,
     pin_decode_layout, pin_softplus_and_gate, pin_hand_worked,
-    pin_bwd_finite_differences, pin_bwd_zoh_finite_differences, pin_bwd_homogeneity,
+    pin_bwd_finite_differences, pin_bwd_wide_state_finite_differences,
+    pin_bwd_zoh_finite_differences, pin_bwd_homogeneity,
     pin_bwd_single_token,
     pin_conv1d_library, pin_conv1d_impulse, pin_conv1d_bwd_finite_differences,
 ]
