@@ -23,7 +23,7 @@ it is pinned against the recurrence oracle in the tests.
 """
 from __future__ import annotations
 
-from typing import Optional, Tuple
+from typing import Tuple
 
 import numpy as np
 

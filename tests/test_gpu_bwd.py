@@ -1,6 +1,5 @@
 """GPU parity of selscan_bwd (the gradient of the scan) against the float64
 oracle's reverse sweep, through the C ABI."""
-import numpy as np
 import pytest
 import torch
 

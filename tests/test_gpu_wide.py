@@ -1,7 +1,6 @@
 """GPU parity of the scan and the decode step for d_state 17..256 (the
 wide-state kernel: each chain's states split over several lanes) against the
 oracle, which takes any d_state."""
-import numpy as np
 import pytest
 import torch
 
