@@ -1,6 +1,7 @@
 """The float64 oracle against closed forms, invariants, library routines and
 brute force (CPU only)."""
 import pytest
+from hypothesis import given, settings, strategies as st
 
 import oracle_pins
 
@@ -37,3 +38,29 @@ def test_bwd_threads_agree(orc):
         assert np.array_equal(g1[k], g8[k]), k
     for k in ("dB", "dC"):
         assert np.allclose(g1[k], g8[k], rtol=1e-13, atol=1e-13), k
+
+
+
+@settings(max_examples=60, deadline=None)
+@given(batch=st.integers(1, 2), L=st.integers(1, 9), D=st.integers(1, 4), N=st.integers(1, 7),
+       seed=st.integers(0, 10_000), gate=st.booleans(), softplus=st.booleans(),
+       zoh=st.booleans(), chunk=st.integers(1, 12))
+def test_recurrence_equals_unrolled_sum_any_shape(orc, batch, L, D, N, seed, gate, softplus,
+                                                  zoh, chunk):
+    """On every tiny shape the C recurrence equals the unrolled closed sum
+    (one exponential of a sum of Δ per term, no running product), and the
+    chunk-aggregate / carry / rescan form equals the plain scan for any chunk
+    length, shorter or longer than the sequence."""
+    import numpy as np
+    c = oracle_pins._rand_case(seed, batch=batch, L=L, D=D, N=N, gate=gate)
+    if not softplus:
+        c["delta"] = np.abs(c["delta"]) + 0.05
+        c["delta_bias"] = np.zeros_like(c["delta_bias"])
+    args = (c["x"], c["delta"], c["A"], c["B"], c["C"], c["D"], c["z"], c["delta_bias"])
+    y, hs = orc.fwd(*args, softplus=softplus, bbar=int(zoh), threads=1)
+    ye, he = oracle_pins.explicit_sum_fwd(c, softplus=softplus, zoh=zoh)
+    assert oracle_pins._rel(y, ye) < 1e-12
+    assert oracle_pins._rel(hs, he) < 1e-12
+    yc, hc = orc.fwd_chunked(*args, softplus=softplus, bbar=int(zoh), chunk=chunk, threads=1)
+    assert oracle_pins._rel(yc, y) < 1e-12
+    assert oracle_pins._rel(hc, hs) < 1e-12
