@@ -64,3 +64,43 @@ def test_recurrence_equals_unrolled_sum_any_shape(orc, batch, L, D, N, seed, gat
     yc, hc = orc.fwd_chunked(*args, softplus=softplus, bbar=int(zoh), chunk=chunk, threads=1)
     assert oracle_pins._rel(yc, y) < 1e-12
     assert oracle_pins._rel(hc, hs) < 1e-12
+
+
+@settings(max_examples=40, deadline=None)
+@given(batch=st.integers(1, 2), L=st.integers(1, 8), D=st.integers(1, 3), N=st.integers(1, 20),
+       seed=st.integers(0, 10_000), gate=st.booleans(), softplus=st.booleans(),
+       zoh=st.booleans(), with_h0=st.booleans())
+def test_gradient_directional_derivative_any_shape(orc, batch, L, D, N, seed, gate, softplus,
+                                                   zoh, with_h0):
+    """For the loss Σ dy·y + Σ dfinal·h_last, the reverse sweep's gradients
+    dotted with a random direction v through every input at once equal the
+    central difference of the forward oracle along v, on every tiny shape."""
+    import numpy as np
+    c, dy, dfinal = oracle_pins._bwd_case(seed, gate=gate, with_h0=with_h0, batch=batch, L=L,
+                                          D=D, N=N)
+    if not softplus:
+        c["delta"] = np.abs(c["delta"]) + 0.05
+        c["delta_bias"] = np.full_like(c["delta_bias"], 0.01)
+    names = [k for k in oracle_pins._BWD_GRADS if c[k] is not None]
+    r = np.random.default_rng(seed + 77)
+    v = {k: r.standard_normal(c[k].shape) for k in names}
+
+    def inputs(cc):
+        return (cc["x"], cc["delta"], cc["A"], cc["B"], cc["C"], cc["D"], cc["z"],
+                cc["delta_bias"])
+
+    def loss(eps):
+        cc = dict(c)
+        for k in names:
+            cc[k] = c[k] + eps * v[k]
+        y, hs = orc.fwd(*inputs(cc), softplus=softplus, bbar=int(zoh), h0=cc["h0"], threads=1)
+        return float(np.sum(dy * y) + np.sum(dfinal * hs))
+
+    g = orc.bwd(*inputs(c), softplus=softplus, bbar=int(zoh), h0=c["h0"], dy=dy,
+                dfinal=dfinal, threads=1)
+    terms = [g[oracle_pins._BWD_GRADS[k]] * v[k] for k in names]
+    want = sum(float(np.sum(t)) for t in terms)
+    scale = sum(float(np.sum(np.abs(t))) for t in terms)
+    eps = 1e-6
+    fd = (loss(eps) - loss(-eps)) / (2 * eps)
+    assert abs(fd - want) <= 1e-6 * max(scale, 1e-12), (fd, want, scale)
