@@ -27,10 +27,16 @@ RNG = np.random.default_rng
 
 
 def _rel(a, b):
+    """Max |a − b| over max |b|; infinite when either side holds a NaN or an
+    infinity, so that a non-finite result never passes a bound."""
     a = np.asarray(a, dtype=np.float64)
     b = np.asarray(b, dtype=np.float64)
-    scale = max(float(np.max(np.abs(b))) if b.size else 0.0, 1e-300)
-    return float(np.max(np.abs(a - b))) / scale if a.size else 0.0
+    if not a.size:
+        return 0.0
+    if not (np.isfinite(a).all() and np.isfinite(b).all()):
+        return math.inf
+    scale = max(float(np.max(np.abs(b))), 1e-300)
+    return float(np.max(np.abs(a - b))) / scale
 
 
 def _rand_case(seed, batch=2, L=7, D=3, N=4, gate=True):
