@@ -1,8 +1,11 @@
 """Host-side logic of bench.py on CPU: the parsing of the clock samples taken
 during the timed region, the check that ties the recorded DRAM traffic to the
-kernel sources it was captured from, and the default launch arguments."""
+kernel sources it was captured from, the default launch arguments, and the
+reference arm (the float64 oracle timed on the host cores, rank 0 only)."""
+import json
 import os
 import shutil
+import subprocess
 import sys
 
 import pytest
@@ -125,3 +128,38 @@ def test_default_launch_is_one_gpu_with_enough_warmup(monkeypatch):
 def test_job_rate_counts_every_rank():
     # 2 ranks x 10 steps x 1e9 elements in 4 ms (the slowest rank)
     assert bench.job_rate(10**9, 2, 10, 4.0) == pytest.approx(5e12)
+
+
+def _run_bench(extra_env, *argv):
+    env = dict(os.environ)
+    env.update(extra_env)
+    root = os.path.dirname(os.path.abspath(bench.__file__))
+    out = subprocess.run([sys.executable, os.path.join(root, "bench.py"), *argv], env=env,
+                         capture_output=True, text=True, timeout=300, cwd=root)
+    assert out.returncode == 0, out.stderr[-2000:]
+    return [json.loads(ln) for ln in out.stdout.splitlines() if ln.startswith("{")]
+
+
+def test_reference_arm_prints_one_line_in_the_contract():
+    """--impl reference times the float64 oracle on the host cores and prints
+    one JSON line with the metric, unit and config of the GPU arm."""
+    lines = _run_bench({"RANK": "0", "OMP_NUM_THREADS": "2"}, "--impl", "reference",
+                       "--workload", "tiny_f32", "--steps", "2", "--warmup", "1",
+                       "--cpu-seconds", "0.05")
+    assert len(lines) == 1
+    j = lines[0]
+    assert j["impl"] == "reference" and j["metric"] == bench.METRIC and j["unit"] == bench.UNIT
+    assert j["steps"] == 2 and j["warmup"] == 1 and j["higher_is_better"] is True
+    assert j["value"] > 0 and j["ms_per_step"] > 0 and j["dtype"] == "f64"
+    assert j["config"]["workload"] == "tiny_f32"
+    cb = j["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["value"] == j["value"] and cb["cores"] >= 1
+    assert "tiny_f32" in cb["sample"]
+    assert j["e2e"] == {"value": j["value"], "unit": bench.UNIT, "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}
+
+
+def test_reference_arm_runs_on_rank_zero_only():
+    lines = _run_bench({"RANK": "1", "WORLD_SIZE": "2"}, "--impl", "reference",
+                       "--workload", "tiny_f32", "--steps", "2", "--warmup", "1")
+    assert lines == []
