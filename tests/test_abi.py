@@ -295,3 +295,210 @@ def test_binding_constants_match_the_header():
     codes = dict((n, int(v)) for n, v in re.findall(r"(SELSCAN_(?:OK|ERR_\w+))\s*=\s*(-?\d+)", text))
     for code, name in ss.selscan.STATUS.items():
         assert codes[name] == code, name
+
+
+def _ptrs(names, spacing=4096):
+    return {n: P + spacing * i for i, n in enumerate(names)}
+
+
+def test_fwd_conv_validation(lib):
+    """selscan_fwd_conv: conv width 1..4, the weight required, alignment, and
+    y kept clear of the conv's carried inputs."""
+    def call(**kw):
+        a = _ptrs(["x_in", "cw", "cb", "ci", "delta", "A", "B", "C", "h0", "y", "final"])
+        a.update(cb=None, ci=None, h0=None, final=None, width=4, batch=0, dim=4)
+        a.update(kw)
+        return lib.selscan_fwd_conv(a["x_in"], a["cw"], a["cb"], a["width"], a["ci"],
+                                    a["delta"], a["A"], a["B"], a["C"], None, None, None, 1,
+                                    a["h0"], a["y"], a["final"], a["batch"], 8, a["dim"], 16,
+                                    1, None)
+    assert call() == 0  # batch = 0
+    assert call(width=0) == -2
+    assert call(width=5) == -2
+    assert call(width=-1) == -2
+    assert call(batch=1, cw=None) == -1
+    assert call(cw=P + 4096 + 2) == -4
+    assert call(ci=P + 4096 * 3 + 2) == -4
+    assert call(batch=1, ci=P + 4096 * 9 + 32) == -7  # y runs into conv_init
+
+
+def test_fwd_ex_validation(lib):
+    Opts = ss.selscan.FwdOptions
+
+    def call(opts, **kw):
+        a = _ptrs(["x", "delta", "A", "B", "C", "y", "h0", "cw", "ci"])
+        a.update(batch=0, dim=4, dstate=16)
+        a.update(kw)
+        return lib.selscan_fwd_ex(a["x"], a["delta"], a["A"], a["B"], a["C"], None, None,
+                                  None, 1, ctypes.byref(opts) if opts is not None else None,
+                                  a["y"], None, a["batch"], 8, a["dim"], a["dstate"], 1, None)
+    assert call(None) == 0
+    assert call(Opts(bbar_mode=1)) == 0
+    assert call(Opts(bbar_mode=2)) == -2
+    assert call(Opts(bbar_mode=-1)) == -2
+    assert call(Opts(conv_width=5)) == -2
+    assert call(Opts(conv_width=4), batch=1) == -1  # no conv weight
+    assert call(Opts(initial_state=P + 4096 * 6 + 2)) == -4
+    assert call(Opts(conv_width=4, conv_weight=P + 4096 * 7, conv_init=P + 4096 * 5),
+                batch=1) == -7  # y == conv_init
+    assert call(Opts(bbar_mode=1), dstate=257) == -5
+
+
+def test_fwd_noalloc_validation(lib):
+    """The same checks as selscan_fwd, and sizes whose chunked plan needs more
+    than the fixed array are refused before anything runs."""
+    def call(spacing=4096, **kw):
+        a = _ptrs(["x", "delta", "A", "B", "C", "y"], spacing)
+        a.update(batch=0, seqlen=8, dim=4, dstate=16, dtype=1)
+        a.update(kw)
+        return lib.selscan_fwd_noalloc(a["x"], a["delta"], a["A"], a["B"], a["C"], None,
+                                       None, None, 1, a["y"], None, a["batch"], a["seqlen"],
+                                       a["dim"], a["dstate"], a["dtype"], None)
+    assert call() == 0
+    assert call(dtype=7) == -3
+    assert call(batch=-1) == -2
+    assert call(dstate=0) == -5
+    assert call(batch=1, x=None) == -1
+    assert call(x=P + 1) == -4
+    assert call(batch=1, y=P) == -7
+    need = ss.selscan_fwd_plan(1, 1 << 20, 2048, 16)["workspace_bytes"]
+    assert need > ss.SELSCAN_NOALLOC_WORKSPACE_BYTES
+    # 4 GiB tensors: the fake addresses sit 8 GiB apart so that none overlap
+    assert call(spacing=8 << 30, batch=1, seqlen=1 << 20, dim=2048) == -8
+
+
+def _bwd_names():
+    return ["x", "delta", "A", "B", "C", "D", "z", "delta_bias", "dy", "dfinal", "dx",
+            "ddelta", "dA", "dB", "dC", "dD", "dz", "ddelta_bias", "h0", "dh0", "cw", "cb",
+            "dcw", "dcb", "ws"]
+
+
+def _bwd_ptrs(**kw):
+    a = _ptrs(_bwd_names())
+    a.update(D=None, z=None, delta_bias=None, dfinal=None, dz=None, h0=None, dh0=None,
+             cb=None, dcb=None, batch=0, dim=0, dstate=16, wsb=0)
+    a.update(kw)
+    return a
+
+
+def test_bwd_workspace_validation(lib):
+    """selscan_bwd_workspace takes the caller's buffer: required when a token
+    is processed, 256-byte aligned, large enough, and clear of every tensor."""
+    def call(**kw):
+        a = _bwd_ptrs(**kw)
+        return lib.selscan_bwd_workspace(
+            a["x"], a["delta"], a["A"], a["B"], a["C"], a["D"], a["z"], a["delta_bias"], 1,
+            a["dy"], a["dfinal"], a["dx"], a["ddelta"], a["dA"], a["dB"], a["dC"], a["dD"],
+            a["dz"], a["ddelta_bias"], a["batch"], 8, a["dim"], a["dstate"], 1, a["ws"],
+            a["wsb"], None)
+    need = lib.selscan_bwd_workspace_bytes(1, 8, 4, 16)
+    ws = P + (1 << 24)  # far from every tensor
+    assert call(ws=None) == 0  # nothing processed: no workspace needed
+    full = dict(batch=1, dim=4)
+    assert call(ws=None, wsb=need, **full) == -1
+    assert call(ws=ws + 16, wsb=need, **full) == -4  # 256-byte alignment
+    assert call(ws=ws, wsb=need - 1, **full) == -8
+    assert call(ws=P + 4096 * 3, wsb=need, **full) == -7  # runs into B
+    assert call(ws=P + 4096 * 13, wsb=need, **full) == -7  # runs into dB
+
+
+def test_bwd_from_state_validation(lib):
+    def call(**kw):
+        a = _bwd_ptrs(**kw)
+        return lib.selscan_bwd_from_state(
+            a["x"], a["delta"], a["A"], a["B"], a["C"], a["D"], a["z"], a["delta_bias"], 1,
+            a["h0"], a["dy"], a["dfinal"], a["dx"], a["ddelta"], a["dA"], a["dB"], a["dC"],
+            a["dD"], a["dz"], a["ddelta_bias"], a["dh0"], a["batch"], 8, a["dim"],
+            a["dstate"], 1, None, 0, None)
+    h0, dh0 = P + 4096 * 18, P + 4096 * 19
+    assert call(h0=h0, dh0=dh0) == 0  # batch = 0, dim = 0
+    assert call(h0=h0, dh0=dh0 + 2) == -4
+    assert call(h0=h0 + 2) == -4
+    full = dict(batch=1, dim=4)
+    assert call(h0=h0, dh0=h0, **full) == -7  # the gradient over its own input
+    assert call(h0=P + 4096 * 10, **full) == -7  # the initial state runs into dx
+    assert call(dfinal=P + 4096 * 9, dh0=P + 4096 * 9 + 64, **full) == -7
+    assert call(dstate=257) == -5
+
+
+def test_bwd_conv_validation(lib):
+    def call(**kw):
+        a = _bwd_ptrs(**kw)
+        a.setdefault("width", 4)
+        return lib.selscan_bwd_conv(
+            a["x"], a["cw"], a["cb"], a["width"], a["delta"], a["A"], a["B"], a["C"], a["D"],
+            a["z"], a["delta_bias"], 1, a["h0"], a["dy"], a["dfinal"], a["dx"], a["ddelta"],
+            a["dA"], a["dB"], a["dC"], a["dD"], a["dz"], a["ddelta_bias"], a["dh0"], a["dcw"],
+            a["dcb"], a["batch"], 8, a["dim"], a["dstate"], 1, None, 0, None)
+    assert call() == 0
+    assert call(width=0) == -2
+    assert call(width=5) == -2
+    full = dict(batch=1, dim=4)
+    assert call(cw=None, **full) == -1
+    assert call(dcw=None, **full) == -1
+    assert call(dcw=P + 4096 * 22 + 2) == -4
+    assert call(dcw=P + 4096 * 20, **full) == -7  # dconv_weight over conv_weight
+    assert call(dcb=P + 4096 * 10, **full) == -7  # two outputs overlap
+
+
+def test_bwd_conv_workspace_bytes(lib):
+    f = lib.selscan_bwd_conv_workspace_bytes
+    assert f(0, 8, 4, 16) == 0 and f(1, 0, 4, 16) == 0 and f(1, 8, 0, 16) == 0
+    assert f(1, 8, 4, 0) == 0 and f(1, 8, 4, 257) == 0
+    for shape in ((1, 8, 4, 16), (2, 300, 70, 16), (1, 100, 40, 40)):
+        plain = lib.selscan_bwd_workspace_bytes(*shape)
+        # besides the scan gradient's workspace: the conv output's float32 gradient
+        assert f(*shape) >= plain + shape[0] * shape[1] * shape[2] * 4
+
+
+def _step_ptrs(**kw):
+    a = _ptrs(["state", "cs", "x", "cw", "cb", "delta", "A", "B", "C", "y"])
+    a.update(cb=None, batch=0, dim=4, dstate=16, width=4)
+    a.update(kw)
+    return a
+
+
+def test_state_update_conv_validation(lib):
+    def call(**kw):
+        a = _step_ptrs(**kw)
+        return lib.selscan_state_update_conv(
+            a["state"], a["cs"], a["x"], a["cw"], a["cb"], a["width"], a["delta"], a["A"],
+            a["B"], a["C"], None, None, None, 1, a["y"], a["batch"], a["dim"], a["dstate"], 1,
+            None)
+    assert call() == 0
+    assert call(width=0) == -2
+    assert call(width=5) == -2
+    assert call(batch=1, cs=None) == -1
+    assert call(batch=1, cw=None) == -1
+    assert call(cs=P + 4096 + 2) == -4
+    assert call(batch=1, cs=P + 32) == -7  # conv_state runs into the state
+    assert call(batch=1, cs=P + 4096 * 2) == -7  # conv_state over x_in
+    assert call(batch=1, y=P + 4096) == -7  # y over conv_state
+
+
+def test_state_update_ex_validation(lib):
+    Opts = ss.selscan.StepOptions
+
+    def call(opts, **kw):
+        a = _step_ptrs(**kw)
+        return lib.selscan_state_update_ex(
+            a["state"], a["x"], a["delta"], a["A"], a["B"], a["C"], None, None, None, 1,
+            ctypes.byref(opts) if opts is not None else None, a["y"], a["batch"], a["dim"],
+            a["dstate"], 1, None)
+    assert call(None) == 0
+    assert call(Opts(bbar_mode=1)) == 0
+    assert call(Opts(bbar_mode=2)) == -2
+    assert call(Opts(conv_width=5)) == -2
+    assert call(Opts(conv_width=4), batch=1) == -1  # no conv_state, no weight
+    assert call(Opts(bbar_mode=1), dstate=257) == -5
+
+
+def test_device_status_without_a_gpu(lib):
+    assert lib.selscan_device_status(None, 0) == -1
+    assert isinstance(ss.selscan_last_cuda_error(), str)
+    torch = pytest.importorskip("torch")
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is visible: the status read succeeds there")
+    st = ctypes.c_int(7)
+    assert lib.selscan_device_status(ctypes.byref(st), 0) == -6  # no device: a CUDA error
+    assert ss.selscan_last_cuda_error() != "no error"
