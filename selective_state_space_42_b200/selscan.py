@@ -126,7 +126,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
             f"selective_state_space_42_b200.build` (nvcc, sm_100a)")
     try:
         lib = ctypes.CDLL(path)
-    except OSError as e:  # pragma: no cover
+    except OSError as e:
         raise SelscanUnavailable(f"cannot load {path}: {e}") from e
     for name, (res, args) in SIGNATURES.items():
         fn = getattr(lib, name)

@@ -502,3 +502,14 @@ def test_device_status_without_a_gpu(lib):
     st = ctypes.c_int(7)
     assert lib.selscan_device_status(ctypes.byref(st), 0) == -6  # no device: a CUDA error
     assert ss.selscan_last_cuda_error() != "no error"
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    """Without the built library the binding raises: there is no fallback."""
+    monkeypatch.setattr(ss.selscan, "_lib", None)
+    with pytest.raises(ss.SelscanUnavailable, match="missing"):
+        ss.selscan.load_library(str(tmp_path / "libselscan.so"))
+    bad = tmp_path / "not_a_library.so"
+    bad.write_bytes(b"not an ELF file")
+    with pytest.raises(ss.SelscanUnavailable, match="cannot load"):
+        ss.selscan.load_library(str(bad))
