@@ -64,7 +64,7 @@ class ScanWorkload:
         ddelta_bias out."""
         es = 4 if self.dtype == "f32" else 2
         gates = 2 if self.gate else 0  # z in, dz out
-        per_bld = (4 + 2 + gates) * es
+        per_bld = (3 + 2 + gates) * es  # x, delta, dy in; dx, ddelta out
         per_bl = 2 * self.dstate * es + 2 * self.dstate * 4
         fixed = 2 * (self.dim * self.dstate * 4 + 2 * self.dim * 4)
         fixed += self.batch * self.dim * self.dstate * 4
