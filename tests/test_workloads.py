@@ -119,3 +119,4 @@ def test_bench_workload_byte_counts():
     assert wl.WORKLOADS["mamba130m_layer"].backward_algorithmic_bytes() == 356_474_880
     assert wl.DECODE.algorithmic_bytes_per_step() == 178_642_944
     assert wl.SSD.algorithmic_bytes() == 107_479_424
+    assert wl.SSD.algorithmic_flops() == 21_474_836_480  # 2·32 heads·32 chunks·10.5 MFLOP
