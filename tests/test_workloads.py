@@ -74,6 +74,7 @@ def test_ssd_flops_count_each_chunk_product_once():
     q×q×P, C·h_in q×N×P and Bᵀ·(w∘X) N×q×P; a ragged last chunk counts
     its own length."""
     w = wl.SsdWorkload("t", 1, 200, 1, 8, 16, "bf16", gate=False, seed=3)
+
     def per_chunk(q, N=16, P=8):
         return 2 * (q * q * N + q * q * P + q * N * P + N * q * P)
     assert w.algorithmic_flops(128) == per_chunk(128) + per_chunk(72)
@@ -93,7 +94,7 @@ def test_generators_are_deterministic_and_seeded():
 
 def test_generators_draw_the_stated_distributions():
     """A[d, n] = −(n+1); softplus(delta_bias) in [1e-3, 1e-1]; x, z, B, C
-    standard normal and delta 0.5·N(0, 1) (moments over 256k draws); SSD
+    standard normal and delta 0.5·N(0, 1) (moments of each tensor); SSD
     heads' A in −[0.5, 4]."""
     w = wl.ScanWorkload("t", 2, 512, 256, 16, "f32", gate=True, seed=5)
     i = wl.make_scan_inputs(w)
