@@ -513,3 +513,24 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     bad.write_bytes(b"not an ELF file")
     with pytest.raises(ss.SelscanUnavailable, match="cannot load"):
         ss.selscan.load_library(str(bad))
+
+
+def test_product_and_oracle_share_no_code():
+    """The package and its CUDA sources never import, include or load the
+    oracle, and the oracle references none of the CUDA sources: the two sides
+    of every parity test are independent."""
+    pkg = os.path.join(ROOT, "selective_state_space_42_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if not f.endswith((".py", ".cu", ".cuh", ".h", ".cc", ".cpp")):
+                continue
+            text = open(os.path.join(dirpath, f), encoding="utf-8").read()
+            assert not re.search(r"^\s*(import|from)\s+oracle\b", text, re.M), f
+            assert not re.search(r'#include\s+["<][^">]*oracle', text), f
+            assert "selscan_oracle" not in text, f
+    for f in os.listdir(os.path.join(ROOT, "oracle")):
+        if f.endswith((".py", ".c", ".h")):
+            text = open(os.path.join(ROOT, "oracle", f), encoding="utf-8").read()
+            assert not re.search(r"^\s*(import|from)\s+selective_state_space_42_b200\b",
+                                 text, re.M), f
+            assert not re.search(r'#include\s+["<][^">]*(selscan\.h|\.cuh)', text), f
