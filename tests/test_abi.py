@@ -7,6 +7,7 @@ import os
 import re
 
 import pytest
+from hypothesis import given, settings, strategies as st
 
 import selective_state_space_42_b200 as ss
 from selective_state_space_42_b200 import build as ssbuild
@@ -534,3 +535,35 @@ def test_product_and_oracle_share_no_code():
             assert not re.search(r"^\s*(import|from)\s+selective_state_space_42_b200\b",
                                  text, re.M), f
             assert not re.search(r'#include\s+["<][^">]*(selscan\.h|\.cuh)', text), f
+
+
+
+@settings(max_examples=300, deadline=None)
+@given(batch=st.integers(1, 16), seqlen=st.integers(1, 16384), dim=st.integers(1, 4096),
+       dstate=st.integers(1, 256))
+def test_plan_invariants_any_size(lib, batch, seqlen, dim, dstate):
+    """The host planner (no GPU: 148 SMs assumed) on random sizes, with bf16
+    tensors on 16-byte boundaries. It always makes one launch or three; the
+    wide kernel (d_state above 16) runs in one pass with no workspace; a
+    chunked plan has two or more chunks of at least 256 tokens and holds P and
+    H for every chunk; TMA-eligible shapes with at least 60% as many
+    (row, 128-channel) groups as SMs take the one-pass plan."""
+    p = ss.selscan_fwd_plan(batch, seqlen, dim, dstate)
+    assert p["launches"] in (1, 3) and p["chunks"] >= 1
+    if dstate > 16:
+        assert p == {"chunks": 1, "launches": 1, "workspace_bytes": 0}
+        return
+    if p["launches"] == 3:
+        assert 2 <= p["chunks"] <= max(1, seqlen // 256)
+        assert p["workspace_bytes"] >= 2 * batch * p["chunks"] * dim * 16 * 4
+    eligible = dim >= 128 and (dim * 2) % 16 == 0 and (dstate * 2) % 16 == 0
+    groups = batch * -(-dim // 128)
+    if eligible and groups * 5 >= 148 * 3:
+        assert p["launches"] == 1
+        # the one pass keeps each group's 128 chains' states between chunks
+        assert p["workspace_bytes"] >= groups * 128 * 16 * 4
+
+
+def test_plan_of_empty_sizes(lib):
+    for shape in ((0, 8, 4, 16), (2, 0, 4, 16), (2, 8, 0, 16)):
+        assert ss.selscan_fwd_plan(*shape) == {"chunks": 0, "launches": 0, "workspace_bytes": 0}
