@@ -567,3 +567,36 @@ def test_plan_invariants_any_size(lib, batch, seqlen, dim, dstate):
 def test_plan_of_empty_sizes(lib):
     for shape in ((0, 8, 4, 16), (2, 0, 4, 16), (2, 8, 0, 16)):
         assert ss.selscan_fwd_plan(*shape) == {"chunks": 0, "launches": 0, "workspace_bytes": 0}
+
+
+@settings(max_examples=200, deadline=None)
+@given(b=st.integers(1, 8), l=st.integers(1, 5000), d=st.integers(1, 3000),
+       n=st.integers(1, 256), grow=st.sampled_from(["b", "l", "d", "n"]),
+       by=st.integers(1, 300))
+def test_gradient_workspace_grows_with_every_size(lib, b, l, d, n, grow, by):
+    """More batch rows, tokens, channels or states never need less gradient
+    workspace, and it always holds the float32 checkpoints: 16 states per
+    chain and 16-state group every 8 tokens."""
+    size = dict(b=b, l=l, d=d, n=n)
+    bigger = dict(size)
+    bigger[grow] = min(bigger[grow] + by, 256) if grow == "n" else bigger[grow] + by
+    for f in (lib.selscan_bwd_workspace_bytes, lib.selscan_bwd_conv_workspace_bytes):
+        small = f(size["b"], size["l"], size["d"], size["n"])
+        large = f(bigger["b"], bigger["l"], bigger["d"], bigger["n"])
+        assert 0 < small <= large
+        groups = -(-n // 16)
+        assert small >= groups * b * -(-l // 8) * d * 16 * 4
+
+
+@settings(max_examples=200, deadline=None)
+@given(b=st.integers(1, 4), l=st.integers(1, 5000), h=st.integers(1, 64),
+       p=st.integers(1, 64), n=st.integers(1, 128),
+       grow=st.sampled_from(["b", "l", "h", "p", "n"]), by=st.integers(1, 64))
+def test_ssd_workspace_grows_with_every_size(lib, b, l, h, p, n, grow, by):
+    size = dict(b=b, l=l, h=h, p=p, n=n)
+    cap = {"p": 64, "n": 128}
+    bigger = dict(size)
+    bigger[grow] = min(bigger[grow] + by, cap.get(grow, 1 << 30))
+    small = lib.selscan_ssd_workspace_bytes(*size.values())
+    large = lib.selscan_ssd_workspace_bytes(*bigger.values())
+    assert 0 < small <= large
