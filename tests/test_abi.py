@@ -600,3 +600,26 @@ def test_ssd_workspace_grows_with_every_size(lib, b, l, h, p, n, grow, by):
     small = lib.selscan_ssd_workspace_bytes(*size.values())
     large = lib.selscan_ssd_workspace_bytes(*bigger.values())
     assert 0 < small <= large
+
+
+def test_binding_error_mapping(lib):
+    """A nonzero status becomes SelscanError carrying the status and the
+    library's text; a CUDA failure appends the CUDA error text."""
+    torch = pytest.importorskip("torch")
+    ss.selscan._check(0)
+    for code, name in ss.selscan.STATUS.items():
+        if code == 0:
+            continue
+        with pytest.raises(ss.SelscanError) as e:
+            ss.selscan._check(code)
+        assert e.value.status == code and name in str(e.value)
+        assert ss.selscan_status_string(code) in str(e.value)
+    with pytest.raises(ss.SelscanError, match=re.escape(ss.selscan_last_cuda_error())):
+        ss.selscan._check(-6)
+    assert ss.selscan._dtype_code(torch.zeros(1)) == ss.SELSCAN_F32
+    assert ss.selscan._dtype_code(torch.zeros(1, dtype=torch.bfloat16)) == ss.SELSCAN_BF16
+    with pytest.raises(TypeError):
+        ss.selscan._dtype_code(torch.zeros(1, dtype=torch.float16))
+    with pytest.raises(ValueError, match="required"):
+        ss.selscan._ptr(None, "x")
+    assert ss.selscan._ptr(None, "z", required=False) is None
