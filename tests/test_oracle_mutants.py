@@ -79,6 +79,10 @@ MUTANTS = [
      "lam[n] * c * B[j + n] * x[i];"),
     ("zoh_grad_limit_wrong", "*c_a = dt * dt * (0.5 + z / 3.0 + z * z / 8.0);",
      "*c_a = dt * dt * (1.0 + z / 3.0 + z * z / 8.0);"),
+    ("bwd_dh0_missing_first_decay", "lam[n] *= a_bar; /* Abar_t",
+     "if (t > 0) lam[n] *= a_bar; /* Abar_t"),
+    ("bwd_dC_uses_previous_state", "pC[t * N + n] += ds * h;", "pC[t * N + n] += ds * hprev;"),
+    ("bwd_bias_grad_without_softplus", "ddelta_bias[d] += dv;", "ddelta_bias[d] += ddt;"),
 ]
 
 
