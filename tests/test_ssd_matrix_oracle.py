@@ -86,29 +86,59 @@ def test_mask_is_semiseparable():
             assert s[1] <= 1e-12 * s[0] if s.size > 1 else True
 
 
-def test_a_shifted_mask_is_caught(orc):
-    """A plausible slip — the decay taken from Acum_{j−1} instead of Acum_j —
-    changes the result well beyond the pin's tolerance."""
-    c = _case(9400)
-    yo, _ = _scan(orc, c, 4)
+def _slipped_matrix_form(c, slip):
+    """The matrix form with one plausible slip planted (test-local copy):
+    'shifted_mask' takes the decay from Acum_{j-1}; 'S_transposed' forms
+    B·Cᵀ instead of C·Bᵀ; 'delta_on_rows' scales the rows of L ◦ S by Δ
+    instead of its columns; 'state_without_delta' drops Δ_j from the final
+    state's sum."""
     x, dt, A, B, C = c["x"], c["dt"], c["A"], c["B"], c["C"]
     batch, T, dim = x.shape
-    H, P = 3, 4
-    y = np.zeros_like(yo)
+    H = dt.shape[2]
+    P = dim // H
+    y = np.zeros_like(x)
+    final = np.zeros((batch, dim, B.shape[2]))
     for b in range(batch):
-        S = C[b] @ B[b].T
+        S = (B[b] @ C[b].T) if slip == "S_transposed" else (C[b] @ B[b].T)
         for h in range(H):
             delta = np.logaddexp(0.0, dt[b, :, h] + c["dt_bias"][h])
             acum = np.cumsum(delta * A[h])
-            prev = np.concatenate([[0.0], acum[:-1]])  # the slip
+            prev = np.concatenate([[0.0], acum[:-1]]) if slip == "shifted_mask" else acum
             L = np.tril(np.exp(acum[:, None] - prev[None, :]))
+            M = L * S
+            M = M * (delta[:, None] if slip == "delta_on_rows" else delta[None, :])
             xh = x[b, :, h * P:(h + 1) * P]
-            yh = ((L * S) * delta[None, :]) @ xh + c["D"][h] * xh
-            yh = yh + np.exp(acum)[:, None] * (C[b] @ c["h0"][b, h * P:(h + 1) * P, :].T)
+            h0h = c["h0"][b, h * P:(h + 1) * P, :].T
+            yh = M @ xh + c["D"][h] * xh + np.exp(acum)[:, None] * (C[b] @ h0h)
             zh = c["z"][b, :, h * P:(h + 1) * P]
             y[b, :, h * P:(h + 1) * P] = yh * zh / (1.0 + np.exp(-zh))
-    assert float(np.max(np.abs(y - yo))) > 1e-3 * float(np.max(np.abs(yo)))
+            w = np.exp(acum[-1] - acum) * (1.0 if slip == "state_without_delta" else delta)
+            final[b, h * P:(h + 1) * P, :] = ((w[:, None] * B[b]).T @ xh
+                                              + np.exp(acum[-1]) * h0h).T
+    return y, final
 
+
+@pytest.mark.parametrize("slip", ["shifted_mask", "S_transposed", "delta_on_rows",
+                                  "state_without_delta"])
+def test_a_planted_slip_is_caught(orc, slip):
+    """Each plausible slip in the matrix form misses the recurrence oracle by
+    far more than the pin's tolerance, in y or in the final state."""
+    c = _case(9400)
+    yo, ho = _scan(orc, c, 4)
+    y, hf = _slipped_matrix_form(c, slip)
+    err = max(float(np.max(np.abs(y - yo))) / float(np.max(np.abs(yo))),
+              float(np.max(np.abs(hf - ho))) / float(np.max(np.abs(ho))))
+    assert err > 1e-3, (slip, err)
+
+
+def test_the_slip_free_copy_matches(orc):
+    """The test-local copy without a slip equals the recurrence: the slips
+    above are the only difference."""
+    c = _case(9400)
+    yo, ho = _scan(orc, c, 4)
+    y, hf = _slipped_matrix_form(c, None)
+    _close(y, yo)
+    _close(hf, ho)
 
 
 @settings(max_examples=40, deadline=None)
