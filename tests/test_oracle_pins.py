@@ -104,3 +104,24 @@ def test_gradient_directional_derivative_any_shape(orc, batch, L, D, N, seed, ga
     eps = 1e-6
     fd = (loss(eps) - loss(-eps)) / (2 * eps)
     assert abs(fd - want) <= 1e-6 * max(scale, 1e-12), (fd, want, scale)
+
+
+@settings(max_examples=60, deadline=None)
+@given(batch=st.integers(1, 2), L=st.integers(1, 12), D=st.integers(1, 4), K=st.integers(1, 4),
+       seed=st.integers(0, 10_000), bias=st.booleans(), silu=st.booleans())
+def test_conv1d_equals_library_convolution_any_shape(orc, batch, L, D, K, seed, bias, silu):
+    """The causal conv against numpy's full convolution with the reversed
+    filter on every small shape, sequences shorter than the filter included."""
+    import numpy as np
+    import scipy.special
+    r = np.random.default_rng(seed)
+    x = r.standard_normal((batch, L, D))
+    w = r.standard_normal((D, K))
+    cb = r.standard_normal(D) if bias else None
+    got = orc.causal_conv1d(x, w, cb, silu=silu)
+    ref = np.empty_like(x)
+    for b in range(batch):
+        for d in range(D):
+            pre = np.convolve(x[b, :, d], w[d, ::-1])[:L] + (cb[d] if bias else 0.0)
+            ref[b, :, d] = pre * scipy.special.expit(pre) if silu else pre
+    assert oracle_pins._rel(got, ref) < 1e-13
