@@ -5,6 +5,8 @@ import ctypes
 import glob
 import os
 import re
+import shutil
+import subprocess
 
 import pytest
 from hypothesis import given, settings, strategies as st
@@ -623,3 +625,47 @@ def test_binding_error_mapping(lib):
     with pytest.raises(ValueError, match="required"):
         ss.selscan._ptr(None, "x")
     assert ss.selscan._ptr(None, "z", required=False) is None
+
+
+C_CLIENT = r"""
+#include <stdio.h>
+#include <string.h>
+#include "selscan.h"
+
+int main(void) {
+    int64_t chunks = -1, launches = -1, ws = -1;
+    int st = selscan_fwd_plan(4, 8192, 5120, 16, &chunks, &launches, &ws);
+    printf("%d %lld %lld %lld\n", st, (long long)chunks, (long long)launches, (long long)ws);
+    printf("%lld\n", (long long)selscan_bwd_workspace_bytes(1, 8, 4, 16));
+    printf("%s\n", selscan_status_string(SELSCAN_ERR_ALIAS));
+    /* batch = 0, dim = 0: validated, nothing to do, no CUDA call */
+    printf("%d\n", selscan_fwd(0, 0, 0, 0, 0, 0, 0, 0, 1, 0, 0, 0, 8, 0, 16, SELSCAN_BF16, 0));
+    /* dim = 4 without A: rejected before any CUDA call */
+    printf("%d\n", selscan_fwd(0, 0, 0, 0, 0, 0, 0, 0, 1, 0, 0, 0, 8, 4, 16, SELSCAN_BF16, 0));
+    return 0;
+}
+"""
+
+
+def test_plain_c_client_links_and_calls(lib, tmp_path):
+    """The header compiles as pedantic C99 and a C program links against
+    libselscan and calls its host-only entry points: the ABI needs neither
+    Python nor C++."""
+    if shutil.which("gcc") is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "client.c"
+    src.write_text(C_CLIENT)
+    exe = tmp_path / "client"
+    libdir = os.path.dirname(ss.LIB_PATH)
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror",
+                    "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe),
+                    "-L", libdir, "-lselscan", "-Wl,-rpath," + libdir],
+                   check=True, capture_output=True, text=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True,
+                         timeout=60).stdout.split("\n")
+    st, chunks, launches, ws = (int(v) for v in out[0].split())
+    assert (st, chunks, launches) == (0, 8, 1) and ws > 0
+    assert int(out[1]) == lib.selscan_bwd_workspace_bytes(1, 8, 4, 16)
+    assert out[2] == ss.selscan_status_string(-7)
+    assert int(out[3]) == 0
+    assert int(out[4]) == -1  # SELSCAN_ERR_NULL_ARG
