@@ -185,6 +185,57 @@ class Oracle:
             batch, L, dim, N, int(threads or default_threads()))
         return out
 
+    # -- one scalar A per head ("Mamba & State Space Models — Guide Complet" §5
+    #    "Mamba-2": the state matrix is a scalar times the identity per head) --
+    @staticmethod
+    def _heads(x, dt, A, B):
+        x = _f64(x)
+        dt = _f64(dt)
+        if x.ndim != 3 or dt.ndim != 3 or dt.shape[:2] != x.shape[:2]:
+            raise ValueError("x must be [batch, L, H·P] and dt [batch, L, H]")
+        H = dt.shape[2]
+        if H < 1 or x.shape[2] % H:
+            raise ValueError("the channel count must be a multiple of the head count")
+        N = np.asarray(B).shape[2]
+        return x, dt, H, x.shape[2] // H, N
+
+    def ssd_fwd(self, x, dt, A, B, C, D=None, z=None, dt_bias=None, softplus=True,
+                h0=None, threads=None):
+        """The scan with one scalar A per head: channel d = h·P + p of head h
+        takes Δ from dt[..., h] + dt_bias[h], decay exp(Δ·A[h]) on every
+        state, and skip D[h]; B and C are shared by all heads. x, z
+        [batch, L, H·P]; dt [batch, L, H]; A, D, dt_bias [H]; B, C
+        [batch, L, N]; h0 [batch, H·P, N]. It is the selective scan with each
+        head's parameters repeated over its P channels (and A over the N
+        states). Returns (y, final_state)."""
+        x, dt, H, P, N = self._heads(x, dt, A, B)
+        rep = (lambda v: None if v is None else np.repeat(_f64(v), P, axis=-1))  # noqa: E731
+        A_ch = np.repeat(_f64(A, (H,))[:, None], P, axis=0) * np.ones((1, N))
+        return self.fwd(x, rep(dt), A_ch, B, C, rep(D), z, rep(dt_bias), softplus=softplus,
+                        h0=h0, threads=threads)
+
+    def ssd_bwd(self, x, dt, A, B, C, D=None, z=None, dt_bias=None, softplus=True,
+                h0=None, dy=None, dfinal=None, threads=None):
+        """Gradient of Σ dy·y + Σ dfinal·final_state for ``ssd_fwd``. A head's
+        Δ, A, D and Δ-bias reach the loss through each of its channels (and
+        A through each state), so their gradients are the per-channel
+        gradients of the selective scan summed over those channels and
+        states; x, z, B, C and h0 enter unchanged. Returns dx, ddt, dA, dB,
+        dC, dD, dz (None without z), ddt_bias and dh0 (None without h0)."""
+        x, dt, H, P, N = self._heads(x, dt, A, B)
+        rep = (lambda v: None if v is None else np.repeat(_f64(v), P, axis=-1))  # noqa: E731
+        A_ch = np.repeat(_f64(A, (H,))[:, None], P, axis=0) * np.ones((1, N))
+        g = self.bwd(x, rep(dt), A_ch, B, C, rep(D), z, rep(dt_bias), softplus=softplus,
+                     h0=h0, dy=dy, dfinal=dfinal, threads=threads)
+
+        def per_head(v):  # [..., H·P] -> [..., H], summed over each head's channels
+            return v.reshape(*v.shape[:-1], H, P).sum(axis=-1)
+
+        return dict(dx=g["dx"], ddt=per_head(g["ddelta"]),
+                    dA=g["dA"].reshape(H, P, N).sum(axis=(1, 2)), dB=g["dB"], dC=g["dC"],
+                    dD=per_head(g["dD"]), dz=g["dz"], ddt_bias=per_head(g["ddelta_bias"]),
+                    dh0=g["dh0"])
+
     def causal_conv1d(self, x_in, w, cb=None, silu=True):
         """Causal depthwise convolution (+ SiLU) in front of the scan:
         x_in [batch, L, D], w [D, K], cb [D] or None -> [batch, L, D]."""

@@ -158,3 +158,102 @@ def test_matrix_form_equals_recurrence_any_shape(orc, batch, T, H, P, N, seed, g
     yo, ho = _scan(orc, c, P, softplus=softplus)
     _close(y, yo)
     _close(hf, ho)
+
+
+# --------------------------------------------------------------------------- #
+# The oracle's scalar-A-per-head entry points against the matrix form, which
+# shares no code with the C recurrence they are built on.
+
+_SSD_GRADS = {"x": "dx", "dt": "ddt", "A": "dA", "B": "dB", "C": "dC", "D": "dD",
+              "z": "dz", "dt_bias": "ddt_bias", "h0": "dh0"}
+
+
+def _matrix(c, softplus=True):
+    return ssd_matrix.ssd_matrix_form(c["x"], c["dt"], c["A"], c["B"], c["C"], c["D"], c["z"],
+                                      c["dt_bias"], softplus=softplus, h0=c["h0"])
+
+
+def _positive_dt(c):
+    c["dt"] = np.abs(c["dt"]) * 0.2 + 0.01
+    c["dt_bias"] = np.full_like(c["dt_bias"], 0.01)
+    return c
+
+
+@pytest.mark.parametrize("gate,h0,softplus", [(True, True, True), (False, False, False)])
+def test_ssd_fwd_method_equals_matrix_form(orc, gate, h0, softplus):
+    c = _case(9500 + gate, gate=gate, h0=h0)
+    if not softplus:
+        _positive_dt(c)
+    y, hf = orc.ssd_fwd(c["x"], c["dt"], c["A"], c["B"], c["C"], c["D"], c["z"], c["dt_bias"],
+                        softplus=softplus, h0=c["h0"], threads=1)
+    ym, hm = _matrix(c, softplus)
+    _close(y, ym)
+    _close(hf, hm)
+
+
+@pytest.mark.parametrize("gate,h0,softplus", [(True, True, True), (False, False, False)])
+def test_ssd_gradient_finite_differences(orc, gate, h0, softplus):
+    """Every element of every gradient of the head form against central
+    differences of the matrix form's loss Σ dy·y + Σ dfinal·h_last."""
+    c = _case(9600 + gate, batch=1, T=6, H=2, P=2, N=3, gate=gate, h0=h0)
+    if not softplus:
+        _positive_dt(c)
+    r = np.random.default_rng(9601)
+    dy = r.standard_normal(c["x"].shape)
+    dfinal = r.standard_normal((1, 4, 3))
+    g = orc.ssd_bwd(c["x"], c["dt"], c["A"], c["B"], c["C"], c["D"], c["z"], c["dt_bias"],
+                    softplus=softplus, h0=c["h0"], dy=dy, dfinal=dfinal, threads=1)
+
+    def loss(cc):
+        y, hf = _matrix(cc, softplus)
+        return float(np.sum(dy * y) + np.sum(dfinal * hf))
+
+    for name, gname in _SSD_GRADS.items():
+        if c[name] is None:
+            assert g[gname] is None, gname
+            continue
+        arr = c[name]
+        fd = np.zeros_like(arr)
+        for idx in np.ndindex(arr.shape):
+            e = 1e-6 * max(1.0, abs(arr[idx]))
+            cp, cm = dict(c), dict(c)
+            cp[name] = arr.copy()
+            cp[name][idx] += e
+            cm[name] = arr.copy()
+            cm[name][idx] -= e
+            fd[idx] = (loss(cp) - loss(cm)) / (2 * e)
+        scale = max(float(np.max(np.abs(fd))), 1e-12)
+        assert float(np.max(np.abs(g[gname] - fd))) <= 1e-6 * scale, gname
+
+
+@settings(max_examples=40, deadline=None)
+@given(batch=st.integers(1, 2), T=st.integers(1, 12), H=st.integers(1, 3), P=st.integers(1, 3),
+       N=st.integers(1, 5), seed=st.integers(0, 10_000), gate=st.booleans(), h0=st.booleans(),
+       softplus=st.booleans())
+def test_ssd_gradient_directional_derivative_any_shape(orc, batch, T, H, P, N, seed, gate, h0,
+                                                       softplus):
+    """The head form's gradients dotted with a random direction through
+    every input equal the central difference of the matrix form along it."""
+    c = _case(seed, batch=batch, T=T, H=H, P=P, N=N, gate=gate, h0=h0)
+    if not softplus:
+        _positive_dt(c)
+    r = np.random.default_rng(seed + 3)
+    dy = r.standard_normal(c["x"].shape)
+    dfinal = r.standard_normal((batch, H * P, N))
+    names = [k for k in _SSD_GRADS if c[k] is not None]
+    v = {k: r.standard_normal(np.shape(c[k])) for k in names}
+    g = orc.ssd_bwd(c["x"], c["dt"], c["A"], c["B"], c["C"], c["D"], c["z"], c["dt_bias"],
+                    softplus=softplus, h0=c["h0"], dy=dy, dfinal=dfinal, threads=1)
+
+    def loss(eps):
+        cc = dict(c)
+        for k in names:
+            cc[k] = c[k] + eps * v[k]
+        y, hf = _matrix(cc, softplus)
+        return float(np.sum(dy * y) + np.sum(dfinal * hf))
+
+    terms = [g[_SSD_GRADS[k]] * v[k] for k in names]
+    want = sum(float(np.sum(t)) for t in terms)
+    scale = sum(float(np.sum(np.abs(t))) for t in terms)
+    fd = (loss(1e-6) - loss(-1e-6)) / 2e-6
+    assert abs(fd - want) <= 1e-6 * max(scale, 1e-12), (fd, want, scale)
