@@ -1,5 +1,6 @@
 """Writes tests/golden/oracle_small.json: small seeded inputs (from the input
-generator module) and the float64 oracle's outputs on them.
+generator module) and the float64 oracle's outputs on them: y, the final
+state, and the gradient for a seeded dy.
 
 Run from the repository root:  python tests/golden/make_golden.py
 Only the oracle computes the stored expected values; nothing here calls the
@@ -9,6 +10,8 @@ a regression fixture of the pinned oracle, not a value from the pages.
 import json
 import os
 import sys
+
+import numpy as np
 
 ROOT = os.path.dirname(os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
 sys.path.insert(0, ROOT)
@@ -37,11 +40,19 @@ def main():
         y, hs = orc.fwd(*(None if inp[k] is None else inp[k].double().numpy()
                           for k in ("x", "delta", "A", "B", "C", "D", "z",
                                     "delta_bias")), softplus=True, threads=1)
+        # the gradient for a seeded dy (an input of the fixture, stored with it)
+        dy = np.random.default_rng(w.seed).standard_normal(y.shape)
+        g = orc.bwd(*(None if inp[k] is None else inp[k].double().numpy()
+                      for k in ("x", "delta", "A", "B", "C", "D", "z", "delta_bias")),
+                    softplus=True, dy=dy, threads=1)
         out["cases"].append({
             "name": w.name, "batch": w.batch, "seqlen": w.seqlen, "dim": w.dim,
             "dstate": w.dstate, "dtype": w.dtype, "gate": w.gate,
             "inputs": {k: _lst(inp[k]) for k in inp},
             "y": y.flatten().tolist(), "final_state": hs.flatten().tolist(),
+            "dy": dy.flatten().tolist(),
+            "grads": {k: (None if v is None else v.flatten().tolist())
+                      for k, v in g.items() if k != "dh0"},
         })
     path = os.path.join(os.path.dirname(os.path.abspath(__file__)),
                         "oracle_small.json")

@@ -29,3 +29,21 @@ def test_oracle_matches_golden(orc):
                        inp["D"], inp["z"], inp["delta_bias"], threads=1)
         assert np.array_equal(y, y_ref), case["name"]
         assert np.array_equal(h, h_ref), case["name"]
+
+
+def test_oracle_gradient_matches_golden(orc):
+    """The gradient for the stored dy: the reverse sweep of the oracle has not
+    drifted (its channel sums may round in another order across thread
+    counts, hence a relative bound of 1e-13 rather than bit equality)."""
+    for case in load_golden():
+        inp, y_ref, _ = golden_arrays(case)
+        dy = np.asarray(case["dy"]).reshape(y_ref.shape)
+        g = orc.bwd(inp["x"], inp["delta"], inp["A"], inp["B"], inp["C"], inp["D"], inp["z"],
+                    inp["delta_bias"], dy=dy, threads=1)
+        for k, ref in case["grads"].items():
+            if ref is None:
+                assert g[k] is None, (case["name"], k)
+                continue
+            ref = np.asarray(ref).reshape(g[k].shape)
+            scale = max(float(np.max(np.abs(ref))), 1e-300)
+            assert float(np.max(np.abs(g[k] - ref))) <= 1e-13 * scale, (case["name"], k)
