@@ -125,3 +125,27 @@ def test_conv1d_equals_library_convolution_any_shape(orc, batch, L, D, K, seed, 
             pre = np.convolve(x[b, :, d], w[d, ::-1])[:L] + (cb[d] if bias else 0.0)
             ref[b, :, d] = pre * scipy.special.expit(pre) if silu else pre
     assert oracle_pins._rel(got, ref) < 1e-13
+
+
+@settings(max_examples=50, deadline=None)
+@given(batch=st.integers(1, 2), L=st.integers(1, 8), D=st.integers(1, 4), N=st.integers(1, 7),
+       seed=st.integers(0, 10_000), gate=st.booleans(), softplus=st.booleans())
+def test_decode_steps_equal_the_scan_any_shape(orc, batch, L, D, N, seed, gate, softplus):
+    """Recurrent inference token by token from an initial state gives the
+    whole-sequence scan from that state: the same y at every token and the
+    same final state, on every small shape."""
+    import numpy as np
+    c = oracle_pins._rand_case(seed, batch=batch, L=L, D=D, N=N, gate=gate)
+    if not softplus:
+        c["delta"] = np.abs(c["delta"]) + 0.05
+        c["delta_bias"] = np.zeros_like(c["delta_bias"])
+    h0 = np.random.default_rng(seed + 9).standard_normal((batch, D, N))
+    y, hs = orc.fwd(c["x"], c["delta"], c["A"], c["B"], c["C"], c["D"], c["z"],
+                    c["delta_bias"], softplus=softplus, h0=h0, threads=1)
+    st_ = h0
+    for t in range(L):
+        yt, st_ = orc.state_update(st_, c["x"][:, t], c["delta"][:, t], c["A"], c["B"][:, t],
+                                   c["C"][:, t], c["D"], None if c["z"] is None else c["z"][:, t],
+                                   c["delta_bias"], softplus=softplus)
+        assert oracle_pins._rel(yt, y[:, t]) < 1e-13
+    assert oracle_pins._rel(st_, hs) < 1e-13
