@@ -163,3 +163,19 @@ def test_reference_arm_runs_on_rank_zero_only():
     lines = _run_bench({"RANK": "1", "WORLD_SIZE": "2"}, "--impl", "reference",
                        "--workload", "tiny_f32", "--steps", "2", "--warmup", "1")
     assert lines == []
+
+
+def test_cpu_sample_size_is_bounded():
+    """The oracle's CPU-baseline sample: at least one channel, never more than
+    the workload has, and a whole number of rounds of the host's threads when
+    it is at least one round, so no thread idles in the timed pass."""
+    from selective_state_space_42_b200 import workloads as wl
+    w = wl.WORKLOADS["mamba2p8b_layer"]
+    per_ch = w.seqlen * w.dstate
+    for rate in (1e3, 1e6, 3e8, 1e9, 1e15):
+        for seconds in (0.01, 10.0):
+            for cores in (1, 8, 48):
+                n = bench._sample_channels(w, rate, seconds, cores)
+                assert 1 <= n <= w.dim
+                if cores <= int(rate * seconds / per_ch) < w.dim:
+                    assert n % cores == 0

@@ -6,6 +6,7 @@ import math
 
 import pytest
 import torch
+from hypothesis import given, settings, strategies as st
 
 from selective_state_space_42_b200 import workloads as wl
 
@@ -121,3 +122,23 @@ def test_bench_workload_byte_counts():
     assert wl.DECODE.algorithmic_bytes_per_step() == 178_642_944
     assert wl.SSD.algorithmic_bytes() == 107_479_424
     assert wl.SSD.algorithmic_flops() == 21_474_836_480  # 2·32 heads·32 chunks·10.5 MFLOP
+
+
+@settings(max_examples=200, deadline=None)
+@given(dim=st.integers(1, 10_000), stride=st.integers(1, 512))
+def test_channel_subset_covers_the_edges(dim, stride):
+    """The channels the full-size parity tests sample: sorted, distinct, in
+    range, always the first, second and last channel, and every stride-th."""
+    s = list(wl.channel_subset(dim, stride))
+    assert s == sorted(set(s)) and all(0 <= c < dim for c in s)
+    assert {0, min(1, dim - 1), dim - 1} <= set(s)
+    assert set(range(0, dim, stride)) <= set(s)
+
+
+def test_ragged_shapes_span_tiles_with_tails():
+    """The small parity shapes include lengths and widths that are not
+    multiples of the kernels' 32-token and 32/128-channel tiles."""
+    shapes = wl.ragged_shapes()
+    assert shapes
+    assert any(s[1] % 32 for s in shapes) and any(s[2] % 32 for s in shapes)
+    assert any(s[1] > 32 for s in shapes) and any(s[2] > 128 for s in shapes)
