@@ -211,9 +211,12 @@ SELSCAN_API int selscan_fwd_ex(const void *x, const void *delta, const float *A,
  * library until the process exits; sizes whose workspace (selscan_fwd_plan)
  * exceeds it are rejected with SELSCAN_ERR_WORKSPACE before anything runs.
  * This call never calls cudaMalloc, cudaMallocAsync or cudaFree.
- *  - The first call on a device that needs the workspace looks up the
- *    array's device address (cudaGetSymbolAddress, once per device, with that
- *    device current); make that first call before any stream capture.
+ *  - Every call that needs the workspace looks up the array's device address
+ *    on the current device (cudaGetSymbolAddress); nothing is cached, so a
+ *    device reset or a re-created primary context, after which the array may
+ *    sit at a new address, is picked up by the next call. The first such
+ *    call on a device also loads the library's device code there; make it
+ *    before any stream capture.
  *  - All calls on a device share the one array, and it keeps the contents
  *    of the last call. Calls that overlap on the GPU (e.g. on two streams
  *    without ordering between them) race on it and give wrong results; order

@@ -11,13 +11,15 @@
 // which every GPU that loads the library holds until the process exits.
 //
 // Host code must not use the array's name as a device address: in host code
-// it names a host-side stand-in. The device address is looked up once per
-// device with cudaGetSymbolAddress (with that device current), checked, cached
-// and passed to the kernels as a plain pointer.
+// it names a host-side stand-in. Every call that needs the workspace looks the
+// device address up with cudaGetSymbolAddress (on the current device, which is
+// the one the call runs on), checks the result and passes it to the kernels as
+// a plain pointer. Nothing is cached: after a device reset, or after the
+// primary context is released and created again, the library's module is
+// loaded again and the array may sit at a new address, which a kept pointer
+// would miss.
 #include <cuda_runtime.h>
 #include <stdint.h>
-
-#include <mutex>
 
 #include "selscan.h"
 #include "selscan_device.cuh"
@@ -32,24 +34,14 @@ constexpr size_t kScratchFloats = (size_t)SELSCAN_NOALLOC_WORKSPACE_BYTES / size
 // It keeps the last call's contents.
 static __device__ __align__(256) float g_scratch[kScratchFloats];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_mutex;
-float *g_scratch_ptr[kMaxDevices] = {nullptr};
-
-// Device address of g_scratch on the current device (looked up on first use).
+// Device address of g_scratch in the current context (looked up afresh on
+// every call, see above).
 cudaError_t scratch_address(float **out) {
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+    void *ptr = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&ptr, g_scratch);
     if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-    std::lock_guard<std::mutex> lock(g_mutex);
-    if (g_scratch_ptr[dev] == nullptr) {
-        void *ptr = nullptr;
-        e = cudaGetSymbolAddress(&ptr, g_scratch);
-        if (e != cudaSuccess) return e;
-        g_scratch_ptr[dev] = static_cast<float *>(ptr);
-    }
-    *out = g_scratch_ptr[dev];
+    if (ptr == nullptr) return cudaErrorInvalidSymbol;
+    *out = static_cast<float *>(ptr);
     return cudaSuccess;
 }
 

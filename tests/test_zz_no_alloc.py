@@ -2,8 +2,14 @@
 device memory while they run (their device memory belongs to another
 allocator, an allocation could stall a latency-critical loop, or stream-ordered
 memory pools are unavailable). Its chunk workspace is a fixed array inside the
-library instead of a stream-ordered allocation; its results must match
-selscan_fwd's.
+library instead of a stream-ordered allocation. It runs the same plan and the
+same kernels as selscan_fwd on the same inputs, so its results must be
+bit-identical to selscan_fwd's.
+
+The array is laid out three ways, one per plan, and each is exercised here:
+the one-pass TMA plan (tickets, hand-over flags and handed-over states), the
+chunked TMA plan (tickets, chunk aggregates and carried states) and the
+generic kernels' chunked plan (aggregates and states only).
 
 This file is collected last on purpose, so that a run stopping at the first
 failure has already run every other test.
@@ -18,9 +24,22 @@ import gpu_helpers as gh
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
+F32 = 4
 
-# a shape whose launch plan is chunked, so the fixed workspace is used
-SHAPE = wl.ScanWorkload("noalloc", 2, 3000, 384, 16, "bf16", gate=True, seed=11)
+# (workload, expected plan); selscan_fwd_plan reports the plan of 16-byte
+# aligned bf16 tensors, and the fp32 shape below takes the same generic plan
+# (dim < 128 rules out the TMA kernel for either dtype).
+CASES = {
+    # one pass, 1024-token units handed from chunk to chunk: 2 units per group
+    "tma_one_pass": wl.ScanWorkload("noalloc_seq", 4, 2048, 5120, 16, "bf16", gate=True,
+                                    seed=21),
+    # few groups: aggregates -> carry -> rescan
+    "tma_chunked": wl.ScanWorkload("noalloc_chunked", 2, 3000, 384, 16, "bf16", gate=True,
+                                   seed=11),
+    # generic kernels (fp32, 96 channels): aggregates -> carry -> rescan
+    "generic_chunked": wl.ScanWorkload("noalloc_generic", 1, 4096, 96, 16, "f32", gate=True,
+                                       seed=31),
+}
 
 
 def _cuda_inputs(w):
@@ -28,12 +47,26 @@ def _cuda_inputs(w):
             for k, v in wl.make_scan_inputs(w).items()}
 
 
-def test_noalloc_matches_selscan_fwd_on_two_calls_in_a_row():
-    w = SHAPE
+def _check_plan(name, w):
     plan = ss.selscan_fwd_plan(w.batch, w.seqlen, w.dim, w.dstate)
-    assert plan["chunks"] > 1
     assert 0 < plan["workspace_bytes"] <= ss.SELSCAN_NOALLOC_WORKSPACE_BYTES
-    for seed in (11, 12):  # the second call finds the first call's workspace contents
+    if name == "tma_one_pass":
+        assert plan["launches"] == 1 and plan["chunks"] == 2
+    elif name == "tma_chunked":
+        assert plan["launches"] == 3 and plan["chunks"] > 1
+        # 256 bytes of counters, then P and H: [batch][chunks][dim][16] each
+        assert plan["workspace_bytes"] == 256 + 2 * w.batch * plan["chunks"] * w.dim * 16 * F32
+    else:
+        assert plan["launches"] == 3 and plan["chunks"] > 1
+        # no counters: P and H only
+        assert plan["workspace_bytes"] == 2 * w.batch * plan["chunks"] * w.dim * 16 * F32
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_noalloc_matches_selscan_fwd_on_two_calls_in_a_row(name):
+    w = CASES[name]
+    _check_plan(name, w)
+    for seed in (w.seed, w.seed + 1):  # the second call finds the first call's contents
         inp = _cuda_inputs(w.scaled(seed=seed))
         args = (inp["x"], inp["delta"], inp["A"], inp["B"], inp["C"], inp["D"],
                 inp["z"], inp["delta_bias"])
@@ -42,9 +75,9 @@ def test_noalloc_matches_selscan_fwd_on_two_calls_in_a_row():
         h = torch.empty(w.batch, w.dim, w.dstate, device=DEV, dtype=torch.float32)
         ss.selscan_fwd_noalloc(*args, softplus=True, y=y, final_state=h)
         torch.cuda.synchronize()
-        gh.compare(gh.to_np(y), gh.to_np(y_ref), gh.RTOL["bf16"], f"noalloc y (seed {seed})")
-        gh.compare(gh.to_np(h), gh.to_np(h_ref), gh.RTOL["bf16"],
-                   f"noalloc final state (seed {seed})")
+        assert torch.equal(y, y_ref), f"{name}: noalloc y differs (seed {seed})"
+        assert torch.equal(h, h_ref), f"{name}: noalloc final state differs (seed {seed})"
+    assert ss.selscan_device_status() == 0
 
 
 def test_noalloc_rejects_sizes_beyond_its_workspace():
