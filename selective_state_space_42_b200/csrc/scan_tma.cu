@@ -361,6 +361,36 @@ struct Run {
     float dt_sum;           // Σ Δ / ln 2 over the unit (agg; this lane's tokens)
 };
 
+// Byte offsets of this lane's owned tokens within a sub-tile starting at row
+// 0: the row of a token in sub-tile `sub` adds sub·128 (x, delta, z) or
+// sub·(row bytes) (y staging), which leaves the swizzle pattern unchanged
+// because sub is a multiple of 8.
+struct Offs {
+    int x[kOwn], t[kOwn], y[kOwn];
+    int xw[kHalo];  // the three x rows before the first owned token (conv)
+};
+
+template <typename T, bool kConv>
+__device__ __forceinline__ Offs lane_offsets(int c, int hsub, int cl) {
+    constexpr int kTile = TileCfg<T>::kTile;
+    constexpr int kXRows = Rows<T, kConv>::kX;
+    constexpr int kXOff = Rows<T, kConv>::kXOff;
+    constexpr unsigned kMask = TileCfg<T>::kYSwizzleMask;
+    Offs o;
+#pragma unroll
+    for (int j = 0; j < kOwn; ++j) {
+        const int r = hsub + j;
+        o.x[j] = swz_offset<T>(kXRows, r + kXOff, c);
+        o.t[j] = swz_offset<T>(kTile, r, c);
+        const int off = r * (kWarpChannels * (int)sizeof(T)) + cl * (int)sizeof(T);
+        o.y[j] = off ^ (int)(((off >> 7) & kMask) << 4);
+    }
+#pragma unroll
+    for (int k = 0; k < kHalo; ++k)
+        o.xw[k] = kConv ? swz_offset<T>(kXRows, hsub - kHalo + k + kXOff, c) : 0;
+    return o;
+}
+
 // The decay factors of one token for this lane's 8 states, from the ladder
 // base c1 = (u_{t−1}/u_t)·r and r: pairs (r^(1+o), r^(3+o)), (r^(5+o), …), …
 // times u_{t−1}/u_t, o = 1 on the upper lane.
@@ -375,180 +405,239 @@ __device__ __forceinline__ void ladder(float c1, float r, bool odd, float2 (&a)[
     a[3] = mul2(a[1], make_float2(s4, s4));
 }
 
-// One ring stage for this lane. kFull: the stage holds kTile valid tokens and
-// y goes to this warp's shared-memory tile `ys` (written to global memory by
-// one TMA store per warp); otherwise tokens from nt on are not processed and
-// y goes straight to global memory.
+// Per-token scalars of the 4 tokens this lane owns in one sub-tile.
+struct Scal {
+    float uu[kOwn];  // structured: u = Δ/ln 2 · x, kept off zero; else Δ/ln 2 · x
+    float rr[kOwn];  // structured: r / u (times the previous token's u after link_prev); else Δ/ln 2
+    float r1[kOwn];  // structured: r = 2^(Δ/ln 2 · A[d, 0])
+    float dx[kOwn];  // D·x
+    float zg[kOwn];  // silu(z), or 1 without a gate
+};
+
 template <typename T, bool kGate, int kMode, bool kStruct, bool kSoftplus, bool kFull,
           bool kConv>
-__device__ __forceinline__ void consume_tile(const Stage<T, kConv> &st, int nt, Run &run,
-                                             const Chain &ch, bool seq_start,
-                                             const float *conv_init, T *ys, T *yp,
-                                             long long ybase, long long ystride, bool active) {
-    constexpr int kTile = TileCfg<T>::kTile;
-    constexpr int kXRows = Rows<T, kConv>::kX;
-    constexpr int kXOff = Rows<T, kConv>::kXOff;
+__device__ __forceinline__ void token_scalars(const Stage<T, kConv> &st, int sub, int nt,
+                                              const Chain &ch, const Offs &o, bool seq_start,
+                                              const float *conv_init, bool active, Run &run,
+                                              Scal &S) {
     constexpr bool kFast = sizeof(T) == 2;  // MUFU softplus and tanh silu for bf16 I/O
-    const int lane = threadIdx.x & 31;
-    const bool odd = lane >= 16;
-    const int cl = lane & 15;
-    const int c = (threadIdx.x >> 5) * kWarpChannels + cl;  // channel within the tile
-    const int hsub = odd ? kOwn : 0;                         // first owned token of a sub-tile
-    const int own_src = cl;                                  // owner of tokens 0-3: lower lane
-#pragma unroll 1
-    for (int sub = 0; sub < kTile; sub += kSub) {
-        if (!kFull && sub >= nt) break;
-        // ---- per-token scalars of the 4 tokens this lane owns -------------------
-        // structured: u, r/u (times the previous u below), r; else u, Δ/ln 2
-        float uu[kOwn], rr[kOwn], r1[kOwn], dx[kOwn];
-        float xw[kHalo] = {0.f, 0.f, 0.f};
-        if constexpr (kConv) {
-            const int t0 = sub + hsub;
-            if (seq_start && t0 == 0) {
-                if (conv_init && active) {
+    const int hsub = (threadIdx.x & 16) ? kOwn : 0;  // first owned token of a sub-tile
+    const unsigned char *xs = st.x + sub * 128;
+    const unsigned char *ds = st.dl + sub * 128;
+    const unsigned char *zs = st.z + sub * 128;
+    float xw[kHalo] = {0.f, 0.f, 0.f};
+    if constexpr (kConv) {
+        if (seq_start && sub + hsub == 0) {
+            if (conv_init && active) {
 #pragma unroll
-                    for (int k = 0; k < kHalo; ++k) xw[k] = conv_init[k];
-                }
-            } else {
-#pragma unroll
-                for (int k = 0; k < kHalo; ++k)
-                    xw[k] = lds_f32<T>(st.x + swz_offset<T>(kXRows, t0 - kHalo + k + kXOff, c));
-            }
-        }
-#pragma unroll
-        for (int j = 0; j < kOwn; ++j) {
-            const int t = sub + hsub + j;
-            float xv = lds_f32<T>(st.x + swz_offset<T>(kXRows, t + kXOff, c));
-            if (kConv) xv = conv_step(ch.cw, ch.cb, xw, xv);
-            const float dv = lds_f32<T>(st.dl + swz_offset<T>(kTile, t, c));
-            float dtl;  // Δ / ln 2
-            if (kSoftplus)
-                dtl = kFast ? softplus_log2_fast(fmaf(dv, kLog2e, ch.biasl))
-                            : softplus_f32(dv + ch.bias) * kLog2e;
-            else
-                dtl = (dv + ch.bias) * kLog2e;
-            if (!kFull) dtl = t < nt ? dtl : 0.0f;
-            if (kStruct) {
-                const float u = fmaf(dtl, xv, signed_tiny(xv));
-                const float r = ex2_approx(dtl * ch.A0);
-                uu[j] = u;
-                rr[j] = r * rcp_approx(u);
-                r1[j] = r;
-            } else {
-                uu[j] = dtl * xv;
-                rr[j] = dtl;
-            }
-            if (kMode == kModeAgg) {
-                run.dt_sum += dtl;
-                dx[j] = 0.0f;
-            } else {
-                dx[j] = ch.dskip * xv;
-            }
-        }
-        // silu(z) after the loop above frees its registers
-        float zg[kOwn];
-#pragma unroll
-        for (int j = 0; j < kOwn; ++j) {
-            const int t = sub + hsub + j;
-            if (kMode != kModeAgg && kGate) {
-                const float zv = lds_f32<T>(st.z + swz_offset<T>(kTile, t, c));
-                zg[j] = kFast ? silu_tanh(zv) : silu_f32(zv);
-            } else {
-                zg[j] = 1.0f;
-            }
-        }
-        // ---- hand the scalars to the other lane ---------------------------------
-        float P0[kSub], P1[kSub];  // structured: ladder base and r; else Δ/ln 2 and u
-        if (kStruct) {
-            // u of the token before each lane's first owned token: for the
-            // lower lane the upper lane's last token of the previous sub-tile
-            const float send = odd ? run.ulast : uu[kOwn - 1];
-            const float prev = __shfl_xor_sync(0xffffffffu, send, 16);
-            run.ulast = uu[kOwn - 1];
-            rr[0] *= prev;
-#pragma unroll
-            for (int j = 1; j < kOwn; ++j) rr[j] *= uu[j - 1];
-#pragma unroll
-            for (int k = 0; k < kSub; ++k) {
-                P0[k] = __shfl_sync(0xffffffffu, rr[k % kOwn], own_src + 16 * (k / kOwn));
-                P1[k] = __shfl_sync(0xffffffffu, r1[k % kOwn], own_src + 16 * (k / kOwn));
+                for (int k = 0; k < kHalo; ++k) xw[k] = conv_init[k];
             }
         } else {
 #pragma unroll
-            for (int k = 0; k < kSub; ++k) {
-                P0[k] = __shfl_sync(0xffffffffu, rr[k % kOwn], own_src + 16 * (k / kOwn));
-                P1[k] = __shfl_sync(0xffffffffu, uu[k % kOwn], own_src + 16 * (k / kOwn));
-            }
+            for (int k = 0; k < kHalo; ++k) xw[k] = lds_f32<T>(xs + o.xw[k]);
         }
-        // ---- recurrence over the 8 tokens, this lane's 8 states -------------------
-        float part[kSub];
+    }
 #pragma unroll
-        for (int k = 0; k < kSub; ++k) part[k] = 0.0f;
-#pragma unroll
-        for (int k = 0; k < kSub; ++k) {
-            const int t = sub + k;
-            if (!kFull && t >= nt) break;
-            const float4 *B4 = reinterpret_cast<const float4 *>(&st.B[t][odd ? kHalf : 0]);
-            float2 a[kHalf / 2];
-            if (kStruct) {
-                ladder(P0[k], P1[k], odd, a);
-                const float4 b0 = B4[0], b1 = B4[1];
-                run.h[0] = fma2(a[0], run.h[0], make_float2(b0.x, b0.y));
-                run.h[1] = fma2(a[1], run.h[1], make_float2(b0.z, b0.w));
-                run.h[2] = fma2(a[2], run.h[2], make_float2(b1.x, b1.y));
-                run.h[3] = fma2(a[3], run.h[3], make_float2(b1.z, b1.w));
-            } else {
-#pragma unroll
-                for (int q = 0; q < kHalf / 2; ++q)
-                    a[q] = make_float2(ex2_approx(P0[k] * ch.An[2 * q]),
-                                       ex2_approx(P0[k] * ch.An[2 * q + 1]));
-                const float2 u2 = make_float2(P1[k], P1[k]);
-                const float4 b0 = B4[0], b1 = B4[1];
-                run.h[0] = fma2(a[0], run.h[0], mul2(u2, make_float2(b0.x, b0.y)));
-                run.h[1] = fma2(a[1], run.h[1], mul2(u2, make_float2(b0.z, b0.w)));
-                run.h[2] = fma2(a[2], run.h[2], mul2(u2, make_float2(b1.x, b1.y)));
-                run.h[3] = fma2(a[3], run.h[3], mul2(u2, make_float2(b1.z, b1.w)));
-            }
-            if (kMode != kModeAgg) {
-                const float4 *C4 = reinterpret_cast<const float4 *>(&st.C[t][odd ? kHalf : 0]);
-                const float4 c0 = C4[0], c1 = C4[1];
-                float2 y0 = mul2(make_float2(c0.x, c0.y), run.h[0]);
-                float2 y1 = mul2(make_float2(c0.z, c0.w), run.h[1]);
-                y0 = fma2(make_float2(c1.x, c1.y), run.h[2], y0);
-                y1 = fma2(make_float2(c1.z, c1.w), run.h[3], y1);
-                const float2 yv = add2(y0, y1);
-                part[k] = yv.x + yv.y;
-            }
-        }
-        // u of the tile's last processed token, for a state handed out of the unit
+    for (int j = 0; j < kOwn; ++j) {
+        const int t = sub + hsub + j;
+        float xv = lds_f32<T>(xs + o.x[j]);
+        if (kConv) xv = conv_step(ch.cw, ch.cb, xw, xv);
+        const float dv = lds_f32<T>(ds + o.t[j]);
+        float dtl;  // Δ / ln 2
+        if (kSoftplus)
+            dtl = kFast ? softplus_log2_fast(fmaf(dv, kLog2e, ch.biasl))
+                        : softplus_f32(dv + ch.bias) * kLog2e;
+        else
+            dtl = (dv + ch.bias) * kLog2e;
+        if (!kFull) dtl = t < nt ? dtl : 0.0f;
         if (kStruct) {
-            const int tl = (kFull ? kSub : min(nt - sub, kSub)) - 1;
-            if (kFull || sub + kSub >= nt) {
-                float us = uu[0];
-#pragma unroll
-                for (int j = 1; j < kOwn; ++j) us = (tl % kOwn) == j ? uu[j] : us;
-                run.uend = __shfl_sync(0xffffffffu, us, own_src + 16 * (tl / kOwn));
-            }
+            const float u = fmaf(dtl, xv, signed_tiny(xv));
+            const float r = ex2_approx(dtl * ch.A0);
+            S.uu[j] = u;
+            S.rr[j] = r * rcp_approx(u);
+            S.r1[j] = r;
+        } else {
+            S.uu[j] = dtl * xv;
+            S.rr[j] = dtl;
         }
-        // ---- the two partial sums meet at the owner lane, which writes y -----------
-        if (kMode != kModeAgg) {
+        if (kMode == kModeAgg) {
+            run.dt_sum += dtl;
+            S.dx[j] = 0.0f;
+        } else {
+            S.dx[j] = ch.dskip * xv;
+        }
+    }
 #pragma unroll
-            for (int j = 0; j < kOwn; ++j) {
-                const float snd = odd ? part[j] : part[kOwn + j];
-                const float rcv = __shfl_xor_sync(0xffffffffu, snd, 16);
-                const float tot = (odd ? part[kOwn + j] : part[j]) + rcv;
-                const float yv = kStruct ? fmaf(uu[j], tot, dx[j]) * zg[j] : (tot + dx[j]) * zg[j];
-                const int t = sub + hsub + j;
-                const T out = from_f32<T>(yv);
-                if (kFull) {
-                    const int off = t * (kWarpChannels * (int)sizeof(T)) + cl * (int)sizeof(T);
-                    const unsigned mask = TileCfg<T>::kYSwizzleMask;
-                    *reinterpret_cast<T *>(reinterpret_cast<unsigned char *>(ys) +
-                                           (off ^ (((off >> 7) & mask) << 4))) = out;
-                } else if (active && t < nt) {
-                    yp[ybase + (long long)t * ystride] = out;
-                }
+    for (int j = 0; j < kOwn; ++j) {
+        if (kMode != kModeAgg && kGate) {
+            const float zv = lds_f32<T>(zs + o.t[j]);
+            S.zg[j] = kFast ? silu_tanh(zv) : silu_f32(zv);
+        } else {
+            S.zg[j] = 1.0f;
+        }
+    }
+}
+
+// Structured form: multiplies each owned token's r/u by the u of the token
+// before it. For the first owned token that u lives on the other lane: for
+// the lower lane the upper lane's last token of the previous sub-tile
+// (`ulast`, updated here), for the upper lane the lower lane's token 3.
+__device__ __forceinline__ void link_prev(Scal &S, bool odd, float &ulast) {
+    const float send = odd ? ulast : S.uu[kOwn - 1];
+    const float prev = __shfl_xor_sync(0xffffffffu, send, 16);
+    ulast = S.uu[kOwn - 1];
+    S.rr[0] *= prev;
+#pragma unroll
+    for (int j = 1; j < kOwn; ++j) S.rr[j] *= S.uu[j - 1];
+}
+
+// Hands every token's two scalars from its owner lane to both lanes:
+// structured: the ladder base and r; else Δ/ln 2 and u.
+template <bool kStruct>
+__device__ __forceinline__ void broadcast(const Scal &S, float (&P0)[kSub], float (&P1)[kSub]) {
+    const int cl = threadIdx.x & 15;
+#pragma unroll
+    for (int k = 0; k < kSub; ++k) {
+        P0[k] = __shfl_sync(0xffffffffu, S.rr[k % kOwn], cl + 16 * (k / kOwn));
+        P1[k] = __shfl_sync(0xffffffffu, kStruct ? S.r1[k % kOwn] : S.uu[k % kOwn],
+                            cl + 16 * (k / kOwn));
+    }
+}
+
+// Advances this lane's 8 states over the sub-tile's tokens (up to nt) and
+// forms its partial sums Σ C·h per token.
+template <typename T, int kMode, bool kStruct, bool kFull, bool kConv>
+__device__ __forceinline__ void recurrence(const Stage<T, kConv> &st, int sub, int nt,
+                                           const float (&P0)[kSub], const float (&P1)[kSub],
+                                           const Chain &ch, Run &run, float (&part)[kSub]) {
+    const bool odd = threadIdx.x & 16;
+#pragma unroll
+    for (int k = 0; k < kSub; ++k) part[k] = 0.0f;
+#pragma unroll
+    for (int k = 0; k < kSub; ++k) {
+        const int t = sub + k;
+        if (!kFull && t >= nt) break;
+        const float4 *B4 = reinterpret_cast<const float4 *>(&st.B[t][odd ? kHalf : 0]);
+        float2 a[kHalf / 2];
+        if (kStruct) {
+            ladder(P0[k], P1[k], odd, a);
+            const float4 b0 = B4[0], b1 = B4[1];
+            run.h[0] = fma2(a[0], run.h[0], make_float2(b0.x, b0.y));
+            run.h[1] = fma2(a[1], run.h[1], make_float2(b0.z, b0.w));
+            run.h[2] = fma2(a[2], run.h[2], make_float2(b1.x, b1.y));
+            run.h[3] = fma2(a[3], run.h[3], make_float2(b1.z, b1.w));
+        } else {
+#pragma unroll
+            for (int q = 0; q < kHalf / 2; ++q)
+                a[q] = make_float2(ex2_approx(P0[k] * ch.An[2 * q]),
+                                   ex2_approx(P0[k] * ch.An[2 * q + 1]));
+            const float2 u2 = make_float2(P1[k], P1[k]);
+            const float4 b0 = B4[0], b1 = B4[1];
+            run.h[0] = fma2(a[0], run.h[0], mul2(u2, make_float2(b0.x, b0.y)));
+            run.h[1] = fma2(a[1], run.h[1], mul2(u2, make_float2(b0.z, b0.w)));
+            run.h[2] = fma2(a[2], run.h[2], mul2(u2, make_float2(b1.x, b1.y)));
+            run.h[3] = fma2(a[3], run.h[3], mul2(u2, make_float2(b1.z, b1.w)));
+        }
+        if (kMode != kModeAgg) {
+            const float4 *C4 = reinterpret_cast<const float4 *>(&st.C[t][odd ? kHalf : 0]);
+            const float4 c0 = C4[0], c1 = C4[1];
+            float2 y0 = mul2(make_float2(c0.x, c0.y), run.h[0]);
+            float2 y1 = mul2(make_float2(c0.z, c0.w), run.h[1]);
+            y0 = fma2(make_float2(c1.x, c1.y), run.h[2], y0);
+            y1 = fma2(make_float2(c1.z, c1.w), run.h[3], y1);
+            const float2 yv = add2(y0, y1);
+            part[k] = yv.x + yv.y;
+        }
+    }
+}
+
+// The two partial sums of each owned token meet at the owner lane, which
+// writes y: to the warp's staging tile (kFull) or to global memory.
+template <typename T, bool kStruct, bool kFull>
+__device__ __forceinline__ void write_y(const Scal &S, const float (&part)[kSub], int sub,
+                                        int nt, const Offs &o, T *ys, T *yp, long long ybase,
+                                        long long ystride, bool active) {
+    const bool odd = threadIdx.x & 16;
+    const int hsub = odd ? kOwn : 0;
+#pragma unroll
+    for (int j = 0; j < kOwn; ++j) {
+        const float snd = odd ? part[j] : part[kOwn + j];
+        const float rcv = __shfl_xor_sync(0xffffffffu, snd, 16);
+        const float tot = (odd ? part[kOwn + j] : part[j]) + rcv;
+        const float yv = kStruct ? fmaf(S.uu[j], tot, S.dx[j]) * S.zg[j]
+                                 : (tot + S.dx[j]) * S.zg[j];
+        const int t = sub + hsub + j;
+        const T out = from_f32<T>(yv);
+        if (kFull) {
+            *reinterpret_cast<T *>(reinterpret_cast<unsigned char *>(ys) +
+                                   sub * (kWarpChannels * (int)sizeof(T)) + o.y[j]) = out;
+        } else if (active && t < nt) {
+            yp[ybase + (long long)t * ystride] = out;
+        }
+    }
+}
+
+// One ring stage for this lane. kFull: the stage holds kTile valid tokens and
+// y goes to this warp's shared-memory tile `ys` (written to global memory by
+// one TMA store per warp); the sub-tiles are software-pipelined (the scalars
+// of sub-tile s + 1 are formed while sub-tile s runs its recurrence).
+// Otherwise tokens from nt on are not processed and y goes straight to global
+// memory.
+template <typename T, bool kGate, int kMode, bool kStruct, bool kSoftplus, bool kFull,
+          bool kConv>
+__device__ __forceinline__ void consume_tile(const Stage<T, kConv> &st, int nt, Run &run,
+                                             const Chain &ch, const Offs &o, bool seq_start,
+                                             const float *conv_init, T *ys, T *yp,
+                                             long long ybase, long long ystride, bool active) {
+    constexpr int kTile = TileCfg<T>::kTile;
+    const bool odd = threadIdx.x & 16;
+    if constexpr (kFull) {
+        Scal S;
+        token_scalars<T, kGate, kMode, kStruct, kSoftplus, true, kConv>(
+            st, 0, nt, ch, o, seq_start, conv_init, active, run, S);
+        if (kStruct) link_prev(S, odd, run.ulast);
+#pragma unroll 1
+        for (int sub = 0; sub < kTile - kSub; sub += kSub) {
+            float P0[kSub], P1[kSub], part[kSub];
+            broadcast<kStruct>(S, P0, P1);
+            Scal N;
+            token_scalars<T, kGate, kMode, kStruct, kSoftplus, true, kConv>(
+                st, sub + kSub, nt, ch, o, seq_start, conv_init, active, run, N);
+            if (kStruct) link_prev(N, odd, run.ulast);
+            recurrence<T, kMode, kStruct, true, kConv>(st, sub, nt, P0, P1, ch, run, part);
+            if (kMode != kModeAgg)
+                write_y<T, kStruct, true>(S, part, sub, nt, o, ys, yp, ybase, ystride, active);
+            S = N;
+        }
+        float P0[kSub], P1[kSub], part[kSub];
+        broadcast<kStruct>(S, P0, P1);
+        recurrence<T, kMode, kStruct, true, kConv>(st, kTile - kSub, nt, P0, P1, ch, run, part);
+        if (kMode != kModeAgg)
+            write_y<T, kStruct, true>(S, part, kTile - kSub, nt, o, ys, yp, ybase, ystride,
+                                      active);
+    } else {
+#pragma unroll 1
+        for (int sub = 0; sub < nt; sub += kSub) {
+            Scal S;
+            token_scalars<T, kGate, kMode, kStruct, kSoftplus, false, kConv>(
+                st, sub, nt, ch, o, seq_start, conv_init, active, run, S);
+            if (kStruct) link_prev(S, odd, run.ulast);
+            float P0[kSub], P1[kSub], part[kSub];
+            broadcast<kStruct>(S, P0, P1);
+            recurrence<T, kMode, kStruct, false, kConv>(st, sub, nt, P0, P1, ch, run, part);
+            // u of the sequence's last token (a partial tile ends the
+            // sequence), for the state handed out of the unit
+            if (kStruct && sub + kSub >= nt) {
+                const int tl = nt - sub - 1;
+                const int hsub = odd ? kOwn : 0;
+                float us = S.uu[0];  // this lane's u of its last owned token before nt
+#pragma unroll
+                for (int j = 1; j < kOwn; ++j)
+                    if (sub + hsub + j < nt) us = S.uu[j];
+                run.uend = __shfl_sync(0xffffffffu, us, (threadIdx.x & 15) + 16 * (tl / kOwn));
             }
+            if (kMode != kModeAgg)
+                write_y<T, kStruct, false>(S, part, sub, nt, o, ys, yp, ybase, ystride, active);
         }
     }
 }
@@ -572,6 +661,7 @@ __device__ void consume(Shared<T, kConv> &S, const TmaScanParams &p, const CUten
     uint32_t phase = 0;
     int cur_tile = -1;
     Chain ch;
+    const Offs offs = lane_offsets<T, kConv>(c, odd ? kOwn : 0, lane & 15);
     bool structured = false;
     Run run;
 #pragma unroll
@@ -680,10 +770,10 @@ __device__ void consume(Shared<T, kConv> &S, const TmaScanParams &p, const CUten
             }
             if (structured)
                 consume_tile<T, kGate, kMode, true, kSoftplus, true, kConv>(
-                    S.stage[s], inf.nt, run, ch, seq_start, cinit, ys, yp, ybase, p.dim, active);
+                    S.stage[s], inf.nt, run, ch, offs, seq_start, cinit, ys, yp, ybase, p.dim, active);
             else
                 consume_tile<T, kGate, kMode, false, kSoftplus, true, kConv>(
-                    S.stage[s], inf.nt, run, ch, seq_start, cinit, ys, yp, ybase, p.dim, active);
+                    S.stage[s], inf.nt, run, ch, offs, seq_start, cinit, ys, yp, ybase, p.dim, active);
             if (kMode != kModeAgg) {
                 fence_proxy_async_smem();
                 __syncwarp();
@@ -697,18 +787,21 @@ __device__ void consume(Shared<T, kConv> &S, const TmaScanParams &p, const CUten
         } else {
             if (structured)
                 consume_tile<T, kGate, kMode, true, kSoftplus, false, kConv>(
-                    S.stage[s], inf.nt, run, ch, seq_start, cinit, nullptr, yp, ybase, p.dim,
+                    S.stage[s], inf.nt, run, ch, offs, seq_start, cinit, nullptr, yp, ybase, p.dim,
                     active);
             else
                 consume_tile<T, kGate, kMode, false, kSoftplus, false, kConv>(
-                    S.stage[s], inf.nt, run, ch, seq_start, cinit, nullptr, yp, ybase, p.dim,
+                    S.stage[s], inf.nt, run, ch, offs, seq_start, cinit, nullptr, yp, ybase, p.dim,
                     active);
         }
 
         if (inf.flags & kLast) {
             const bool last_chunk = inf.chunk == p.nchunks - 1;
             // the unit's final state, this lane's 8 states
-            const float sc = kLn2 * (structured ? run.uend : 1.0f);
+            // u of the unit's last token: the upper lane's latest u after a full
+            // tile, else recorded by the partial tile
+            const float ul = __shfl_sync(0xffffffffu, run.ulast, (lane & 15) + 16);
+            const float sc = kLn2 * (structured ? (inf.nt == kTile ? ul : run.uend) : 1.0f);
             float hf[kHalf];
 #pragma unroll
             for (int q = 0; q < kHalf / 2; ++q) {
