@@ -71,20 +71,29 @@ constexpr int kConsumers = 32 * kConsumerWarps;
 constexpr int kBlock = kConsumers + 32;         // + producer warp
 constexpr int kMaxConsumerWarps = 8;            // flags per group in the workspace
 #ifndef SELSCAN_TMA_STAGES
-#define SELSCAN_TMA_STAGES 4
+#define SELSCAN_TMA_STAGES 3
 #endif
 constexpr int kStages = SELSCAN_TMA_STAGES;
 constexpr int kSub = 8;    // tokens per sub-tile (4 per lane of a pair)
 constexpr int kOwn = kSub / 2;
 constexpr int kHalf = kMaxN / 2;  // states per lane
 
+#ifndef SELSCAN_TMA_TILE_BF16
+#define SELSCAN_TMA_TILE_BF16 64
+#endif
+#ifndef SELSCAN_TMA_TILE_F32
+#define SELSCAN_TMA_TILE_F32 32
+#endif
+#ifndef SELSCAN_TMA_LAG
+#define SELSCAN_TMA_LAG 1
+#endif
 template <typename T> struct TileCfg;
 template <> struct TileCfg<__nv_bfloat16> {
-    static constexpr int kTile = 32;
+    static constexpr int kTile = SELSCAN_TMA_TILE_BF16;
     static constexpr unsigned kYSwizzleMask = 1;  // 32-byte rows: 32-byte swizzle
 };
 template <> struct TileCfg<float> {
-    static constexpr int kTile = 16;
+    static constexpr int kTile = SELSCAN_TMA_TILE_F32;
     static constexpr unsigned kYSwizzleMask = 3;  // 64-byte rows: 64-byte swizzle
 };
 
@@ -138,7 +147,6 @@ template <typename T> __device__ __forceinline__ float lds_f32(const unsigned ch
 // for two lanes of work).
 __device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
 __device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
-__device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
 
 enum : int { kFirst = 1, kLast = 2, kEnd = 4 };
 
@@ -220,7 +228,7 @@ __device__ void produce(Shared<T, kConv> &S, const TmaScanParams &p, const CUten
                         const CUtensorMap *tm_d, const CUtensorMap *tm_z,
                         const CUtensorMap *tm_b, const CUtensorMap *tm_c) {
     constexpr int kTile = TileCfg<T>::kTile;
-    constexpr int kLag = kStages > 2 ? 2 : 1;
+    constexpr int kLag = SELSCAN_TMA_LAG < kStages ? SELSCAN_TMA_LAG : kStages - 1;
     constexpr int kNB = n_boxes<T>();
     constexpr int kBoxCh = box_channels<T>();
     constexpr int kXRows = Rows<T, kConv>::kX;
@@ -513,6 +521,13 @@ __device__ __forceinline__ void recurrence(const Stage<T, kConv> &st, int sub, i
     const bool odd = threadIdx.x & 16;
 #pragma unroll
     for (int k = 0; k < kSub; ++k) part[k] = 0.0f;
+    // the decay ladders of all 8 tokens first: they do not depend on the
+    // states, so their multiply chains overlap the state updates below
+    float2 lad[kSub][kHalf / 2];
+    if (kStruct) {
+#pragma unroll
+        for (int k = 0; k < kSub; ++k) ladder(P0[k], P1[k], odd, lad[k]);
+    }
 #pragma unroll
     for (int k = 0; k < kSub; ++k) {
         const int t = sub + k;
@@ -520,7 +535,8 @@ __device__ __forceinline__ void recurrence(const Stage<T, kConv> &st, int sub, i
         const float4 *B4 = reinterpret_cast<const float4 *>(&st.B[t][odd ? kHalf : 0]);
         float2 a[kHalf / 2];
         if (kStruct) {
-            ladder(P0[k], P1[k], odd, a);
+#pragma unroll
+            for (int q = 0; q < kHalf / 2; ++q) a[q] = lad[k][q];
             const float4 b0 = B4[0], b1 = B4[1];
             run.h[0] = fma2(a[0], run.h[0], make_float2(b0.x, b0.y));
             run.h[1] = fma2(a[1], run.h[1], make_float2(b0.z, b0.w));
@@ -541,11 +557,10 @@ __device__ __forceinline__ void recurrence(const Stage<T, kConv> &st, int sub, i
         if (kMode != kModeAgg) {
             const float4 *C4 = reinterpret_cast<const float4 *>(&st.C[t][odd ? kHalf : 0]);
             const float4 c0 = C4[0], c1 = C4[1];
-            float2 y0 = mul2(make_float2(c0.x, c0.y), run.h[0]);
-            float2 y1 = mul2(make_float2(c0.z, c0.w), run.h[1]);
-            y0 = fma2(make_float2(c1.x, c1.y), run.h[2], y0);
-            y1 = fma2(make_float2(c1.z, c1.w), run.h[3], y1);
-            const float2 yv = add2(y0, y1);
+            float2 yv = mul2(make_float2(c0.x, c0.y), run.h[0]);
+            yv = fma2(make_float2(c0.z, c0.w), run.h[1], yv);
+            yv = fma2(make_float2(c1.x, c1.y), run.h[2], yv);
+            yv = fma2(make_float2(c1.z, c1.w), run.h[3], yv);
             part[k] = yv.x + yv.y;
         }
     }
