@@ -148,6 +148,42 @@ template <typename T> __device__ __forceinline__ float lds_f32(const unsigned ch
 __device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
 __device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
 
+// 2^e for a pair of exponents e <= 0 on the FMA pipe, for bf16 I/O (the
+// MUFU's ex2 takes the other states of a lane, so that the two pipes share
+// the exps of the general-A decay). Cody–Waite style range reduction: e =
+// n + f with n = round(e) (by adding 1.5·2^23, which leaves n in the low
+// mantissa bits) and f in [-1/2, 1/2]; 2^f by a degree-4 polynomial with the
+// smallest maximum relative error on that interval (Remez exchange, fitted
+// by fit_exp2_poly.py next to this file: 2.7e-6 with float32 coefficients
+// and Horner evaluation); 2^n by adding n to the exponent field. e is
+// clamped at -126 so that the exponent field cannot wrap (2^-126 underflows
+// the states' contribution just the same).
+__device__ __forceinline__ float2 exp2_poly2(float2 e) {
+    constexpr float kC0 = 0.9999992847442627f, kC1 = 0.6931217908859253f,
+                    kC2 = 0.240247443318367f, kC3 = 0.05591785907745361f,
+                    kC4 = 0.009570102207362652f;
+    constexpr float kRound = 12582912.0f;  // 1.5·2^23
+    e = make_float2(fmaxf(e.x, -126.0f), fmaxf(e.y, -126.0f));
+    const float2 t = __fadd2_rn(e, make_float2(kRound, kRound));
+    const float2 n = __fadd2_rn(t, make_float2(-kRound, -kRound));
+    const float2 f = __ffma2_rn(n, make_float2(-1.0f, -1.0f), e);
+    float2 p = __ffma2_rn(make_float2(kC4, kC4), f, make_float2(kC3, kC3));
+    p = __ffma2_rn(p, f, make_float2(kC2, kC2));
+    p = __ffma2_rn(p, f, make_float2(kC1, kC1));
+    p = __ffma2_rn(p, f, make_float2(kC0, kC0));
+    return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23)),
+                       __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
+}
+
+#ifndef SELSCAN_POLY_PAIRS
+#define SELSCAN_POLY_PAIRS 1
+#endif
+// How many of a lane's 4 state pairs take their general-A decay from
+// exp2_poly2 (bf16 I/O): the last ones, whose states (n = 12..15 with A in
+// the usual increasing order) forget fastest, so the polynomial's error
+// accumulates over the fewest tokens; the rest use the MUFU.
+template <typename T> constexpr int poly_pairs() { return sizeof(T) == 2 ? SELSCAN_POLY_PAIRS : 0; }
+
 enum : int { kFirst = 1, kLast = 2, kEnd = 4 };
 
 struct TileInfo {
@@ -544,9 +580,13 @@ __device__ __forceinline__ void recurrence(const Stage<T, kConv> &st, int sub, i
             run.h[3] = fma2(a[3], run.h[3], make_float2(b1.z, b1.w));
         } else {
 #pragma unroll
-            for (int q = 0; q < kHalf / 2; ++q)
-                a[q] = make_float2(ex2_approx(P0[k] * ch.An[2 * q]),
-                                   ex2_approx(P0[k] * ch.An[2 * q + 1]));
+            for (int q = 0; q < kHalf / 2; ++q) {
+                const float2 e = mul2(make_float2(P0[k], P0[k]),
+                                      make_float2(ch.An[2 * q], ch.An[2 * q + 1]));
+                a[q] = q >= kHalf / 2 - poly_pairs<T>()
+                           ? exp2_poly2(e)
+                           : make_float2(ex2_approx(e.x), ex2_approx(e.y));
+            }
             const float2 u2 = make_float2(P1[k], P1[k]);
             const float4 b0 = B4[0], b1 = B4[1];
             run.h[0] = fma2(a[0], run.h[0], mul2(u2, make_float2(b0.x, b0.y)));

@@ -38,6 +38,10 @@ class ScanWorkload:
     skip_ones: bool = False  # D = 1.0 instead of 1 + 0.1·N(0,1)
     softplus: bool = True
     final_state: bool = True
+    # A[d, n]: "ladder" −(n+1); "exp_log" −exp(log(n+1)) evaluated in float32
+    # (the pages' A = −exp(A_log) with A_log = log(1..N)), which is −(n+1)
+    # only up to rounding
+    a_init: str = "ladder"
 
     @property
     def elements(self) -> int:
@@ -153,6 +157,9 @@ WORKLOADS: Dict[str, ScanWorkload] = {
     "long_1m": ScanWorkload("long_1m", 1, 1 << 20, 2048, 16, "bf16",
                             gate=True, seed=3),
 }
+# the 2.8B layer with the pages' A = −exp(A_log) parametrisation
+WORKLOADS["mamba2p8b_layer_expA"] = WORKLOADS["mamba2p8b_layer"].scaled(
+    name="mamba2p8b_layer_expA", a_init="exp_log")
 
 DECODE = DecodeWorkload("decode_b256", 256, 5120, 16, 1000, "bf16", gate=True,
                         seed=4)
@@ -169,10 +176,22 @@ def _randn(shape, g, device, scale=1.0) -> torch.Tensor:
     return t.mul_(scale) if scale != 1.0 else t
 
 
-def param_tensors(dim: int, dstate: int, g, device, skip_ones: bool):
+def a_matrix(dim: int, dstate: int, a_init: str = "ladder", device="cpu") -> torch.Tensor:
+    """A [dim, dstate]: −(n+1), or −exp(log(n+1)) evaluated in float32 on the
+    CPU (so that every device sees the same values)."""
+    n1 = torch.arange(1, dstate + 1, dtype=torch.float32)
+    if a_init == "exp_log":
+        row = -torch.exp(torch.log(n1))
+    elif a_init == "ladder":
+        row = -n1
+    else:
+        raise ValueError(a_init)
+    return row.repeat(dim, 1).contiguous().to(device)
+
+
+def param_tensors(dim: int, dstate: int, g, device, skip_ones: bool, a_init: str = "ladder"):
     """A, D (skip) and delta_bias for `dim` channels."""
-    A = -torch.arange(1, dstate + 1, dtype=torch.float32, device=device)
-    A = A.repeat(dim, 1).contiguous()
+    A = a_matrix(dim, dstate, a_init, device)
     u = torch.rand(dim, generator=g, device=device, dtype=torch.float64)
     u = 1e-3 + (1e-1 - 1e-3) * u
     delta_bias = torch.log(torch.expm1(u)).to(torch.float32)
@@ -197,7 +216,7 @@ def make_scan_inputs(w: ScanWorkload, device="cpu") -> Dict[str, torch.Tensor]:
     out["B"] = _randn(bshp, g, device).to(dt)
     out["C"] = _randn(bshp, g, device).to(dt)
     out["A"], out["D"], out["delta_bias"] = param_tensors(
-        w.dim, w.dstate, g, device, w.skip_ones)
+        w.dim, w.dstate, g, device, w.skip_ones, w.a_init)
     return out
 
 

@@ -187,6 +187,30 @@ def test_mamba2p8b_layer_sampled():
     _full_size_sampled("mamba2p8b_layer", 160)
 
 
+def test_mamba2p8b_layer_expA_sampled():
+    """The benchmark's workload with the pages' A = −exp(log(1..16)) in float32,
+    which misses the exact-ladder test and takes the general decay (one exp
+    per state, part of them on the FMA pipe)."""
+    _full_size_sampled("mamba2p8b_layer_expA", 160)
+
+
+@pytest.mark.parametrize("a_init", ["exp_log", "random"])
+def test_general_A_final_state_tight(a_init):
+    """General A with bf16 I/O: y is rounded to bf16, but the float32 final
+    state carries the error of the decay factors themselves (MUFU ex2 and the
+    degree-4 polynomial, 2.7e-6), so it is held to 1e-3."""
+    w = wl.ScanWorkload("genA", 2, 2048, 256, 16, "bf16", gate=True, seed=41,
+                        a_init="exp_log")
+    inp = _cuda(wl.make_scan_inputs(w))
+    if a_init == "random":
+        inp["A"] = _random_A(w.dim, w.dstate, 42).to(DEV)
+    y, hs = gh.gpu_fwd(inp)
+    torch.cuda.synchronize()
+    yo, ho = gh.oracle_fwd(inp)
+    gh.compare(gh.to_np(y), yo, gh.RTOL["bf16"], "general A y")
+    gh.compare(gh.to_np(hs), ho, 1e-3, "general A final_state")
+
+
 def test_mamba2p8b_layer_chunked_sampled():
     _full_size_sampled("mamba2p8b_layer", 512, chunks=4, batches=[0, 3])
 
