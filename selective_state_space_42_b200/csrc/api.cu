@@ -130,6 +130,12 @@ void plan_tma(int64_t batch, int64_t seqlen, int64_t dim, bool bf16, selscan::Fw
     t.timeout_ns = 2000000000ull;
     const int64_t tmo = env_int("SELSCAN_TIMEOUT_MS");
     if (tmo > 0) t.timeout_ns = (unsigned long long)tmo * 1000000ull;
+    // Test hook (off unless set): the one-pass plan's units of this chunk do
+    // not publish their completion flag, so their successors' bounded waits
+    // run out; the fault-handling test uses it together with a short
+    // SELSCAN_TIMEOUT_MS.
+    const char *skip = getenv("SELSCAN_TEST_SKIP_RELEASE");
+    t.skip_release_chunk = (skip && *skip) ? atoi(skip) : -1;
     pl->tma = true;
     pl->chunks = (int)nchunks;
     pl->launches = seq ? 1 : 3;
@@ -246,9 +252,7 @@ int fwd_setup(const void *x, const void *delta, const float *A, const void *B,
 
     const bool aligned = !misaligned(x, 16) && !misaligned(delta, 16) && !misaligned(z, 16) &&
                          !misaligned(B, 16) && !misaligned(C, 16) && !misaligned(y, 16);
-    // the TMA kernel has no zero-order-hold input term: that mode takes the
-    // generic kernels
-    plan_for_sizes(batch, seqlen, dim, dstate, dtype, aligned && !zoh, plan);
+    plan_for_sizes(batch, seqlen, dim, dstate, dtype, aligned, plan);
     plan->x = x;
     plan->delta = delta;
     plan->z = z;
@@ -271,6 +275,7 @@ int fwd_setup(const void *x, const void *delta, const float *A, const void *B,
         t.y = y; t.final_state = final_state; t.h0 = h0;
         t.conv_w = g.conv_w; t.conv_b = g.conv_b; t.conv_init = g.conv_init;
         t.conv_width = conv_width;
+        t.zoh = zoh ? 1 : 0;
         t.batch = batch; t.seqlen = seqlen; t.dim = dim; t.dstate = (int)dstate;
         t.softplus = g.softplus;
         const int64_t units = t.groups * t.nchunks;

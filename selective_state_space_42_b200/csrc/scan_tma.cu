@@ -175,6 +175,21 @@ __device__ __forceinline__ float2 exp2_poly2(float2 e) {
                        __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
 }
 
+// Zero-order-hold input factor (exp(z) − 1)/z of a pair, z = Δ·A (here
+// e·ln 2 with e the log2 exponent), given a = exp(z): below |z| = 1/32 the
+// series 1 + z/2 + z²/6 + z³/24 (truncation under z⁴/120 < 1e-8 relative),
+// above (a − 1)/z with the MUFU reciprocal.
+__device__ __forceinline__ float2 zoh_factor2(float2 e, float2 a) {
+    const float2 z = __fmul2_rn(e, make_float2(kLn2, kLn2));
+    float2 sr = __ffma2_rn(z, make_float2(1.0f / 24.0f, 1.0f / 24.0f),
+                           make_float2(1.0f / 6.0f, 1.0f / 6.0f));
+    sr = __ffma2_rn(z, sr, make_float2(0.5f, 0.5f));
+    sr = __ffma2_rn(z, sr, make_float2(1.0f, 1.0f));
+    const float2 am1 = __fadd2_rn(a, make_float2(-1.0f, -1.0f));
+    return make_float2(fabsf(z.x) < 0.03125f ? sr.x : am1.x * rcp_approx(z.x),
+                       fabsf(z.y) < 0.03125f ? sr.y : am1.y * rcp_approx(z.y));
+}
+
 #ifndef SELSCAN_POLY_PAIRS
 #define SELSCAN_POLY_PAIRS 1
 #endif
@@ -550,7 +565,7 @@ __device__ __forceinline__ void broadcast(const Scal &S, float (&P0)[kSub], floa
 
 // Advances this lane's 8 states over the sub-tile's tokens (up to nt) and
 // forms its partial sums Σ C·h per token.
-template <typename T, int kMode, bool kStruct, bool kFull, bool kConv>
+template <typename T, int kMode, bool kStruct, bool kFull, bool kConv, bool kZoh>
 __device__ __forceinline__ void recurrence(const Stage<T, kConv> &st, int sub, int nt,
                                            const float (&P0)[kSub], const float (&P1)[kSub],
                                            const Chain &ch, Run &run, float (&part)[kSub]) {
@@ -579,20 +594,27 @@ __device__ __forceinline__ void recurrence(const Stage<T, kConv> &st, int sub, i
             run.h[2] = fma2(a[2], run.h[2], make_float2(b1.x, b1.y));
             run.h[3] = fma2(a[3], run.h[3], make_float2(b1.z, b1.w));
         } else {
+            float2 e[kHalf / 2];
 #pragma unroll
             for (int q = 0; q < kHalf / 2; ++q) {
-                const float2 e = mul2(make_float2(P0[k], P0[k]),
-                                      make_float2(ch.An[2 * q], ch.An[2 * q + 1]));
+                e[q] = mul2(make_float2(P0[k], P0[k]),
+                            make_float2(ch.An[2 * q], ch.An[2 * q + 1]));
                 a[q] = q >= kHalf / 2 - poly_pairs<T>()
-                           ? exp2_poly2(e)
-                           : make_float2(ex2_approx(e.x), ex2_approx(e.y));
+                           ? exp2_poly2(e[q])
+                           : make_float2(ex2_approx(e[q].x), ex2_approx(e[q].y));
             }
             const float2 u2 = make_float2(P1[k], P1[k]);
             const float4 b0 = B4[0], b1 = B4[1];
-            run.h[0] = fma2(a[0], run.h[0], mul2(u2, make_float2(b0.x, b0.y)));
-            run.h[1] = fma2(a[1], run.h[1], mul2(u2, make_float2(b0.z, b0.w)));
-            run.h[2] = fma2(a[2], run.h[2], mul2(u2, make_float2(b1.x, b1.y)));
-            run.h[3] = fma2(a[3], run.h[3], mul2(u2, make_float2(b1.z, b1.w)));
+            float2 bu[kHalf / 2] = {mul2(u2, make_float2(b0.x, b0.y)),
+                                    mul2(u2, make_float2(b0.z, b0.w)),
+                                    mul2(u2, make_float2(b1.x, b1.y)),
+                                    mul2(u2, make_float2(b1.z, b1.w))};
+            if (kZoh) {
+#pragma unroll
+                for (int q = 0; q < kHalf / 2; ++q) bu[q] = mul2(bu[q], zoh_factor2(e[q], a[q]));
+            }
+#pragma unroll
+            for (int q = 0; q < kHalf / 2; ++q) run.h[q] = fma2(a[q], run.h[q], bu[q]);
         }
         if (kMode != kModeAgg) {
             const float4 *C4 = reinterpret_cast<const float4 *>(&st.C[t][odd ? kHalf : 0]);
@@ -639,7 +661,7 @@ __device__ __forceinline__ void write_y(const Scal &S, const float (&part)[kSub]
 // Otherwise tokens from nt on are not processed and y goes straight to global
 // memory.
 template <typename T, bool kGate, int kMode, bool kStruct, bool kSoftplus, bool kFull,
-          bool kConv>
+          bool kConv, bool kZoh>
 __device__ __forceinline__ void consume_tile(const Stage<T, kConv> &st, int nt, Run &run,
                                              const Chain &ch, const Offs &o, bool seq_start,
                                              const float *conv_init, T *ys, T *yp,
@@ -659,14 +681,14 @@ __device__ __forceinline__ void consume_tile(const Stage<T, kConv> &st, int nt, 
             token_scalars<T, kGate, kMode, kStruct, kSoftplus, true, kConv>(
                 st, sub + kSub, nt, ch, o, seq_start, conv_init, active, run, N);
             if (kStruct) link_prev(N, odd, run.ulast);
-            recurrence<T, kMode, kStruct, true, kConv>(st, sub, nt, P0, P1, ch, run, part);
+            recurrence<T, kMode, kStruct, true, kConv, kZoh>(st, sub, nt, P0, P1, ch, run, part);
             if (kMode != kModeAgg)
                 write_y<T, kStruct, true>(S, part, sub, nt, o, ys, yp, ybase, ystride, active);
             S = N;
         }
         float P0[kSub], P1[kSub], part[kSub];
         broadcast<kStruct>(S, P0, P1);
-        recurrence<T, kMode, kStruct, true, kConv>(st, kTile - kSub, nt, P0, P1, ch, run, part);
+        recurrence<T, kMode, kStruct, true, kConv, kZoh>(st, kTile - kSub, nt, P0, P1, ch, run, part);
         if (kMode != kModeAgg)
             write_y<T, kStruct, true>(S, part, kTile - kSub, nt, o, ys, yp, ybase, ystride,
                                       active);
@@ -679,7 +701,7 @@ __device__ __forceinline__ void consume_tile(const Stage<T, kConv> &st, int nt, 
             if (kStruct) link_prev(S, odd, run.ulast);
             float P0[kSub], P1[kSub], part[kSub];
             broadcast<kStruct>(S, P0, P1);
-            recurrence<T, kMode, kStruct, false, kConv>(st, sub, nt, P0, P1, ch, run, part);
+            recurrence<T, kMode, kStruct, false, kConv, kZoh>(st, sub, nt, P0, P1, ch, run, part);
             // u of the sequence's last token (a partial tile ends the
             // sequence), for the state handed out of the unit
             if (kStruct && sub + kSub >= nt) {
@@ -697,7 +719,7 @@ __device__ __forceinline__ void consume_tile(const Stage<T, kConv> &st, int nt, 
     }
 }
 
-template <typename T, bool kGate, int kMode, bool kSoftplus, bool kConv>
+template <typename T, bool kGate, int kMode, bool kSoftplus, bool kConv, bool kZoh>
 __device__ void consume(Shared<T, kConv> &S, const TmaScanParams &p, const CUtensorMap *tm_y) {
     constexpr int kTile = TileCfg<T>::kTile;
     const int tid = threadIdx.x;  // 0..255
@@ -823,11 +845,11 @@ __device__ void consume(Shared<T, kConv> &S, const TmaScanParams &p, const CUten
                 if (lane == 0) bulk_wait_read<kYBufs - 1>();
                 __syncwarp();
             }
-            if (structured)
-                consume_tile<T, kGate, kMode, true, kSoftplus, true, kConv>(
+            if (!kZoh && structured)
+                consume_tile<T, kGate, kMode, true, kSoftplus, true, kConv, false>(
                     S.stage[s], inf.nt, run, ch, offs, seq_start, cinit, ys, yp, ybase, p.dim, active);
             else
-                consume_tile<T, kGate, kMode, false, kSoftplus, true, kConv>(
+                consume_tile<T, kGate, kMode, false, kSoftplus, true, kConv, kZoh>(
                     S.stage[s], inf.nt, run, ch, offs, seq_start, cinit, ys, yp, ybase, p.dim, active);
             if (kMode != kModeAgg) {
                 fence_proxy_async_smem();
@@ -840,12 +862,12 @@ __device__ void consume(Shared<T, kConv> &S, const TmaScanParams &p, const CUten
                 kbuf ^= 1;
             }
         } else {
-            if (structured)
-                consume_tile<T, kGate, kMode, true, kSoftplus, false, kConv>(
+            if (!kZoh && structured)
+                consume_tile<T, kGate, kMode, true, kSoftplus, false, kConv, false>(
                     S.stage[s], inf.nt, run, ch, offs, seq_start, cinit, nullptr, yp, ybase, p.dim,
                     active);
             else
-                consume_tile<T, kGate, kMode, false, kSoftplus, false, kConv>(
+                consume_tile<T, kGate, kMode, false, kSoftplus, false, kConv, kZoh>(
                     S.stage[s], inf.nt, run, ch, offs, seq_start, cinit, nullptr, yp, ybase, p.dim,
                     active);
         }
@@ -856,7 +878,7 @@ __device__ void consume(Shared<T, kConv> &S, const TmaScanParams &p, const CUten
             // u of the unit's last token: the upper lane's latest u after a full
             // tile, else recorded by the partial tile
             const float ul = __shfl_sync(0xffffffffu, run.ulast, (lane & 15) + 16);
-            const float sc = kLn2 * (structured ? (inf.nt == kTile ? ul : run.uend) : 1.0f);
+            const float sc = kLn2 * ((!kZoh && structured) ? (inf.nt == kTile ? ul : run.uend) : 1.0f);
             float hf[kHalf];
 #pragma unroll
             for (int q = 0; q < kHalf / 2; ++q) {
@@ -891,7 +913,7 @@ __device__ void consume(Shared<T, kConv> &S, const TmaScanParams &p, const CUten
                 }
                 __threadfence();
                 __syncwarp();
-                if (lane == 0)
+                if (lane == 0 && inf.chunk != p.skip_release_chunk)
                     st_release_gpu(p.flags + g * kMaxConsumerWarps + warp, inf.chunk + 1);
             }
         }
@@ -908,7 +930,7 @@ template <typename T, bool kConv> constexpr size_t smem_bytes() {
     return sizeof(Shared<T, kConv>) + 1024;  // + room to align the base to 1024 bytes
 }
 
-template <typename T, bool kGate, int kMode, bool kSoftplus, bool kConv>
+template <typename T, bool kGate, int kMode, bool kSoftplus, bool kConv, bool kZoh>
 __global__ void __launch_bounds__(kBlock, 1)
 scan_tma_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_d,
                 const __grid_constant__ CUtensorMap tm_z, const __grid_constant__ CUtensorMap tm_b,
@@ -933,7 +955,7 @@ scan_tma_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
     if (threadIdx.x >= kConsumers)
         produce<T, kGate, kConv>(S, p, &tm_x, &tm_d, &tm_z, &tm_b, &tm_c);
     else
-        consume<T, kGate, kMode, kSoftplus, kConv>(S, p, &tm_y);
+        consume<T, kGate, kMode, kSoftplus, kConv, kZoh>(S, p, &tm_y);
 }
 
 // ---- host side -----------------------------------------------------------------------
@@ -979,7 +1001,7 @@ int num_sms() {
     return sms;
 }
 
-template <typename T, bool kGate, int kMode, bool kSoftplus, bool kConv>
+template <typename T, bool kGate, int kMode, bool kSoftplus, bool kConv, bool kZoh>
 cudaError_t launch_mode(const TmaScanParams &p, const void *x, const void *dl, const void *z,
                         cudaStream_t stream) {
     if (p.units <= 0) return cudaSuccess;
@@ -1003,7 +1025,7 @@ cudaError_t launch_mode(const TmaScanParams &p, const void *x, const void *dl, c
         mz = md;
     }
     const size_t smem = smem_bytes<T, kConv>();
-    auto kern = scan_tma_kernel<T, kGate, kMode, kSoftplus, kConv>;
+    auto kern = scan_tma_kernel<T, kGate, kMode, kSoftplus, kConv, kZoh>;
     // the shared-memory opt-in is set once per device for this instantiation
     static std::atomic<unsigned long long> configured{0};
     int dev = 0;
@@ -1020,21 +1042,31 @@ cudaError_t launch_mode(const TmaScanParams &p, const void *x, const void *dl, c
     return cudaGetLastError();
 }
 
-template <typename T, bool kGate, bool kSoftplus, bool kConv>
+template <typename T, bool kGate, bool kSoftplus, bool kConv, bool kZoh>
 cudaError_t launch_conv(const TmaScanParams &p, const void *x, const void *dl, const void *z,
                         cudaStream_t stream) {
     switch (p.mode) {
-    case kModeSeq: return launch_mode<T, kGate, kModeSeq, kSoftplus, kConv>(p, x, dl, z, stream);
-    case kModeAgg: return launch_mode<T, false, kModeAgg, kSoftplus, kConv>(p, x, dl, z, stream);
-    default: return launch_mode<T, kGate, kModeRescan, kSoftplus, kConv>(p, x, dl, z, stream);
+    case kModeSeq:
+        return launch_mode<T, kGate, kModeSeq, kSoftplus, kConv, kZoh>(p, x, dl, z, stream);
+    case kModeAgg:
+        return launch_mode<T, false, kModeAgg, kSoftplus, kConv, kZoh>(p, x, dl, z, stream);
+    default:
+        return launch_mode<T, kGate, kModeRescan, kSoftplus, kConv, kZoh>(p, x, dl, z, stream);
     }
+}
+
+template <typename T, bool kGate, bool kSoftplus, bool kZoh>
+cudaError_t launch_zoh(const TmaScanParams &p, const void *x, const void *dl, const void *z,
+                       cudaStream_t stream) {
+    return p.conv_width > 0 ? launch_conv<T, kGate, kSoftplus, true, kZoh>(p, x, dl, z, stream)
+                            : launch_conv<T, kGate, kSoftplus, false, kZoh>(p, x, dl, z, stream);
 }
 
 template <typename T, bool kGate, bool kSoftplus>
 cudaError_t launch_sp(const TmaScanParams &p, const void *x, const void *dl, const void *z,
                       cudaStream_t stream) {
-    return p.conv_width > 0 ? launch_conv<T, kGate, kSoftplus, true>(p, x, dl, z, stream)
-                            : launch_conv<T, kGate, kSoftplus, false>(p, x, dl, z, stream);
+    return p.zoh ? launch_zoh<T, kGate, kSoftplus, true>(p, x, dl, z, stream)
+                 : launch_zoh<T, kGate, kSoftplus, false>(p, x, dl, z, stream);
 }
 
 template <typename T, bool kGate>

@@ -173,6 +173,7 @@ struct TmaScanParams {
     const float *conv_b;  // [dim] (NULL: zero)
     const float *conv_init;  // [batch][dim][kMaxConv − 1]: conv inputs before token 0 (NULL: zero)
     int conv_width;       // 0 (no conv) or 1..kMaxConv
+    int zoh;              // input term: 0 Δ·B·x, 1 (exp(Δ·A) − 1)/A·B·x
     long long batch, seqlen, dim;
     int dstate;
     int softplus;
@@ -189,6 +190,8 @@ struct TmaScanParams {
     float *ws_state;      // kModeSeq: [groups][128][16] state handed between units
     float *ws_P, *ws_H;   // chunked: [batch][nchunks][dim][16]
     unsigned long long timeout_ns;  // bound on every device-side wait
+    int skip_release_chunk;  // fault-injection hook for tests: the kSeq units of this
+                             // chunk publish no completion flag (-1: none)
 };
 
 cudaError_t launch_scan_tma(const TmaScanParams &p, bool bf16, const void *x, const void *dl,

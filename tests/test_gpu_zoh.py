@@ -108,3 +108,23 @@ def test_zoh_decode_steps(N):
         torch.cuda.synchronize()
         gh.compare(gh.to_np(y), yo[:, 0], gh.RTOL["f32"], f"step {t} y")
         gh.compare(gh.to_np(sd), ho, gh.RTOL["f32"], f"step {t} state")
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("plan", ["seq_unit64", "chunked3"])
+@pytest.mark.parametrize("A_kind", ["structured", "random", "with_zeros"])
+def test_zoh_tma_plans(dtype, plan, A_kind):
+    """The ZOH term on the TMA-staged kernel (dim a multiple of 128, aligned
+    rows): the one-pass plan with state hand-off and the chunked plan, over
+    several tiles and a ragged tail."""
+    env = {"seq_unit64": dict(SELSCAN_PATH="seq", SELSCAN_UNIT="64", SELSCAN_CHUNKS=None),
+           "chunked3": dict(SELSCAN_PATH="chunked", SELSCAN_UNIT=None, SELSCAN_CHUNKS="3")}[plan]
+    inp = _inputs(2, 1000, 384, 16, dtype, 5200, A_kind)
+    d = {k: (None if v is None else v.to(DEV)) for k, v in inp.items()}
+    with gh.env(**env):
+        y, hf = ss.selscan_fwd(d["x"], d["delta"], d["A"], d["B"], d["C"], d["D"], d["z"],
+                               d["delta_bias"], bbar="zoh", return_final_state=True)
+        torch.cuda.synchronize()
+    yo, ho = _oracle(inp)
+    gh.compare(gh.to_np(y), yo, gh.RTOL[dtype], f"{plan} {A_kind} y")
+    gh.compare(gh.to_np(hf), ho, gh.RTOL[dtype], f"{plan} {A_kind} final state")
