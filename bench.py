@@ -188,41 +188,53 @@ def _sample_channels(w, rate, seconds, cores, rows=1):
     return max(1, min(w.dim, n))
 
 
+def oracle_sample(w, inp, target_s, cores):
+    """The one sample definition shared by `cpu_baseline` and the reference
+    arm: the workload's batch rows in order, all of their tokens; channels
+    0..n-1 of row 0 when one row takes longer than target_s seconds on
+    `cores` threads, else whole rows, repeated when the whole workload is
+    shorter. Sized from a short probe. Returns (oracle args, passes,
+    elements per pass, description)."""
+    import oracle
+    orc = oracle.default()
+    probe = max(cores, 8)
+    t = time.perf_counter()
+    orc.fwd(*_oracle_args(inp, (0,), probe), softplus=True, threads=cores)
+    rate = probe * w.seqlen * w.dstate / max(time.perf_counter() - t, 1e-9)
+    row_s = w.dim * w.seqlen * w.dstate / rate
+    if row_s >= target_s:
+        rows, nch, reps = 1, _sample_channels(w, rate, target_s, cores), 1
+        what = f"batch row 0, channels 0..{nch - 1} of {w.dim}"
+    else:
+        rows, nch = min(w.batch, max(1, int(target_s / row_s))), w.dim
+        reps = max(1, int(round(target_s / (rows * row_s)))) if rows == w.batch else 1
+        what = (f"batch rows 0..{rows - 1} of {w.batch}, all {w.dim} channels"
+                + (f", {reps} passes" if reps > 1 else ""))
+    desc = (f"{w.name}: {what}, all {w.seqlen} tokens, d_state {w.dstate}; "
+            f"float64 oracle, OpenMP over channels")
+    return (_oracle_args(inp, tuple(range(rows)), nch), reps,
+            rows * nch * w.seqlen * w.dstate, desc)
+
+
 def oracle_cpu_baseline(inp, w, target_s):
-    """The oracle, as it stands, on a sample of the workload sized to take
-    about target_s seconds of the host's cores: a channel subset of every
-    batch row, or the whole workload repeated when one pass is shorter.
-    Returns the cpu_baseline object (scan elements per second)."""
+    """The oracle, as it stands, timed on the host cores on the shared sample
+    (oracle_sample) of the workload; scan elements per second."""
     import oracle
     orc = oracle.default()
     cores = oracle.default_threads()
-    rows = tuple(range(w.batch))
-    probe = max(cores, 8)
-    t = time.perf_counter()
-    orc.fwd(*_oracle_args(inp, rows, probe), softplus=True, threads=cores)
-    rate = w.batch * probe * w.seqlen * w.dstate / max(time.perf_counter() - t, 1e-9)
-    nch = _sample_channels(w, rate, target_s, cores, rows=w.batch)
-    reps = 1
-    if nch == w.dim:
-        one = w.elements / rate
-        reps = max(1, int(round(target_s / max(one, 1e-9))))
-    args = _oracle_args(inp, rows, nch)
+    args, reps, per_pass, desc = oracle_sample(w, inp, target_s, cores)
     t = time.perf_counter()
     for _ in range(reps):
         orc.fwd(*args, softplus=True, threads=cores)
     dt = time.perf_counter() - t
-    el = reps * w.batch * nch * w.seqlen * w.dstate
-    what = (f"the whole workload x{reps}" if nch == w.dim else
-            f"channels 0..{nch - 1} of {w.dim}")
+    el = reps * per_pass
     return {"value": el / dt, "unit": UNIT, "cores": cores, "kind": "oracle",
-            "sample": (f"{w.name}: all {w.batch} batch rows, {what}, all {w.seqlen} tokens, "
-                       f"d_state {w.dstate}: {el:.3e} scan elements in {dt:.2f} s "
-                       f"(float64, OpenMP over channels)")}
+            "sample": f"{desc}: {el:.3e} scan elements in {dt:.2f} s"}
 
 
 def run_reference(args):
-    """--impl reference: the oracle timed on the host cores; each step is a
-    bounded sample (batch row 0, a channel subset) of the workload."""
+    """--impl reference: the oracle timed on the host cores; each step is the
+    same bounded sample as the GPU arm's cpu_baseline (oracle_sample)."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
@@ -230,27 +242,20 @@ def run_reference(args):
     from selective_state_space_42_b200 import workloads as wl
     w = wl.WORKLOADS[args.workload]
     cores = oracle.default_threads()
-    sub = w.scaled(batch=1, dim=min(w.dim, 4 * max(cores, 8) * 8))
-    inp = wl.make_scan_inputs(sub, device="cpu")
+    inp = wl.make_scan_inputs(w, device="cpu")
     orc = oracle.default()
     per_step_s = min(args.cpu_seconds, 150.0 / max(args.steps + args.warmup, 1))
-    probe = max(cores, 8)
-    t = time.perf_counter()
-    orc.fwd(*_oracle_args(inp, (0,), probe), softplus=True, threads=cores)
-    rate = probe * w.seqlen * w.dstate / max(time.perf_counter() - t, 1e-9)
-    nch = min(_sample_channels(w, rate, per_step_s, cores), sub.dim)
-    a = _oracle_args(inp, (0,), nch)
+    a, reps, per_pass, desc = oracle_sample(w, inp, per_step_s, cores)
     times = []
     for i in range(args.warmup + args.steps):
         t = time.perf_counter()
-        orc.fwd(*a, softplus=True, threads=cores)
+        for _ in range(reps):
+            orc.fwd(*a, softplus=True, threads=cores)
         if i >= args.warmup:
             times.append(time.perf_counter() - t)
     total = sum(times)
-    elems = len(times) * nch * w.seqlen * w.dstate
+    elems = len(times) * reps * per_pass
     value = elems / total
-    sample = (f"{w.name}: per step batch row 0, channels 0..{nch - 1}, all {w.seqlen} "
-              f"tokens, d_state {w.dstate}; float64 oracle, OpenMP over channels")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
@@ -258,7 +263,7 @@ def run_reference(args):
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": config_block(w, 1),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores,
-                         "kind": "oracle", "sample": sample},
+                         "kind": "oracle", "sample": desc},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -304,6 +309,122 @@ def smi_id(torch, dev, local):
         return f"{p.pci_domain_id:08X}:{p.pci_bus_id:02X}:{p.pci_device_id:02X}.0"
     except AttributeError:
         return str(local)
+
+
+def time_calls(torch, stream, fn, n, flush=None):
+    """CUDA-event time of one call in ms: the mean of n back-to-back calls,
+    and (with `flush`, a buffer larger than L2 written before each call) the
+    median of 10 calls each after an L2-evicting write."""
+    for _ in range(3):
+        fn()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(n):
+        fn()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    b2b = e0.elapsed_time(e1) / n
+    if flush is None:
+        return b2b, None
+    cold = []
+    for _ in range(10):
+        flush.zero_()
+        c0 = torch.cuda.Event(enable_timing=True)
+        c1 = torch.cuda.Event(enable_timing=True)
+        c0.record(stream)
+        fn()
+        c1.record(stream)
+        torch.cuda.synchronize()
+        cold.append(c0.elapsed_time(c1))
+    return b2b, sorted(cold)[len(cold) // 2]
+
+
+def extra_legs(args, torch, ss, wl, dev, stream, peak, over_ranks):
+    """Other workloads of the path, timed the same way (not part of the
+    headline metric): the other scan shapes, the general-A and ZOH variants
+    of the headline shape, the decode step and the SSD layer."""
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    out = {}
+
+    def scan_leg(name, n, bbar="delta", ref_ms=None):
+        w = wl.WORKLOADS[name]
+        inp = wl.make_scan_inputs(w, device=dev)
+        y = torch.empty_like(inp["x"])
+        fs = torch.empty(w.batch, w.dim, w.dstate, device=dev, dtype=torch.float32)
+
+        def call():
+            ss.selscan_fwd(inp["x"], inp["delta"], inp["A"], inp["B"], inp["C"], inp["D"],
+                           inp["z"], inp["delta_bias"], softplus=True, y=y, final_state=fs,
+                           stream=stream, bbar=bbar)
+        b2b, cold = time_calls(torch, stream, call, n, flush)
+        b2b, cold = over_ranks(b2b), over_ranks(cold)
+        nb = w.algorithmic_bytes()
+        leg = {"workload": name, "bytes_per_call": nb, "elements_per_call": w.elements,
+               "us_back_to_back": b2b * 1e3, "us_after_l2_flush": cold * 1e3,
+               "elems_per_s": w.elements / (b2b / 1e3),
+               "GBps_back_to_back": nb / b2b / 1e6, "frac_back_to_back": nb / b2b / 1e6 / peak,
+               "plan": ss.selscan_fwd_plan(w.batch, w.seqlen, w.dim, w.dstate)}
+        if ref_ms is not None:
+            leg["time_vs_headline_shape"] = b2b / ref_ms
+        del inp, y, fs
+        return leg, b2b
+
+    out["mamba130m_layer"], _ = scan_leg("mamba130m_layer", 200)
+    out["long_1m"], _ = scan_leg("long_1m", 5)
+    ref = args.headline_ms
+    out["general_A"], _ = scan_leg("mamba2p8b_layer_expA", 100, ref_ms=ref)
+    out["general_A"]["A"] = "-exp(log(n+1)) in float32 (not bit-exactly (n+1)*A[d,0]: general decay)"
+    out["zoh"], _ = scan_leg("mamba2p8b_layer", 50, bbar="zoh", ref_ms=ref)
+    out["zoh"]["input_term"] = "(exp(delta*A)-1)/A*B*x"
+
+    # the decode step (one token in place on the [256, 5120, 16] state); the
+    # after-flush time is the headline: back to back the 84 MB state stays in L2
+    dw = wl.DECODE
+    dstate_t = wl.make_decode_state(dw, device=dev)
+    dA, dDv, dbias = wl.make_decode_params(dw, device=dev)
+    dsteps = [wl.make_decode_step(dw, s, device=dev) for s in range(4)]
+    k = [0]
+
+    def decode():
+        t = dsteps[k[0] % len(dsteps)]
+        k[0] += 1
+        ss.selscan_state_update(dstate_t, t["x"], t["delta"], dA, t["B"], t["C"], dDv, t["z"],
+                                dbias, stream=stream)
+    b2b, cold = time_calls(torch, stream, decode, 200, flush)
+    b2b, cold = over_ranks(b2b), over_ranks(cold)
+    nb = dw.algorithmic_bytes_per_step()
+    out["decode_step"] = {
+        "workload": dw.name, "bytes_per_step": nb,
+        "us": cold * 1e3, "GBps": nb / cold / 1e6, "frac": nb / cold / 1e6 / peak,
+        "timing": "after an L2-evicting write",
+        "us_back_to_back": b2b * 1e3, "GBps_back_to_back": nb / b2b / 1e6,
+        "kernel": "state_update_vec_kernel<bf16, gate>"}
+
+    # the Mamba-2-shaped SSD layer (one scalar A per head, chunked form on
+    # the tensor cores)
+    sw = wl.SSD
+    sinp = wl.make_ssd_inputs(sw, device=dev)
+    sy = torch.empty_like(sinp["x"])
+    sfs = torch.empty(sw.batch, sw.dim, sw.dstate, device=dev)
+
+    def ssd_call():
+        ss.selscan_ssd_fwd(sinp["x"], sinp["dt"], sinp["A"], sinp["B"], sinp["C"], D=sinp["D"],
+                           z=sinp["z"], dt_bias=sinp["dt_bias"], y=sy, final_state=sfs,
+                           stream=stream)
+    b2b, cold = time_calls(torch, stream, ssd_call, 50, flush)
+    b2b, cold = over_ranks(b2b), over_ranks(cold)
+    out["ssd_layer"] = {
+        "workload": sw.name, "bytes_per_call": sw.algorithmic_bytes(),
+        "flops_per_call": sw.algorithmic_flops(),
+        "us_back_to_back": b2b * 1e3, "us_after_l2_flush": cold * 1e3,
+        "GBps_back_to_back": sw.algorithmic_bytes() / b2b / 1e6,
+        "TFLOPs_back_to_back": sw.algorithmic_flops() / b2b / 1e9,
+        "frac_hbm_back_to_back": sw.algorithmic_bytes() / b2b / 1e6 / peak,
+        "frac_tensor_back_to_back": sw.algorithmic_flops() / b2b / 1e9 / tensor_peak()}
+    del flush
+    return out
 
 
 def main():
@@ -368,6 +489,7 @@ def main():
     ms = ev0.elapsed_time(ev1)
     clocks = sampler.stop() if sampler else None
     ms = max_over_ranks(ms, dist if world > 1 else None, dev)
+    args.headline_ms = ms / args.steps
 
     # end to end through the public call: pinned host inputs -> device ->
     # selscan_fwd -> y and final state back to pinned host memory, every step
@@ -401,82 +523,9 @@ def main():
     h2d = sum(host[k].numel() * host[k].element_size() for k in names)
     d2h = y_h.numel() * y_h.element_size() + fs_h.numel() * fs_h.element_size()
 
-    # the decode step (one token in place on the [256, 5120, 16] state):
-    # back to back, and after an L2-evicting write; not part of the metric
-    dw = wl.DECODE
-    dstate_t = wl.make_decode_state(dw, device=dev)
-    dA, dDv, dbias = wl.make_decode_params(dw, device=dev)
-    dsteps = [wl.make_decode_step(dw, s, device=dev) for s in range(4)]
-
-    def decode(i):
-        t = dsteps[i % len(dsteps)]
-        ss.selscan_state_update(dstate_t, t["x"], t["delta"], dA, t["B"], t["C"], dDv, t["z"],
-                                dbias, stream=stream)
-
-    for i in range(5):
-        decode(i)
-    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
-    cold = []
-    for i in range(10):
-        flush.zero_()
-        c0 = torch.cuda.Event(enable_timing=True)
-        c1 = torch.cuda.Event(enable_timing=True)
-        c0.record(stream)
-        decode(i)
-        c1.record(stream)
-        torch.cuda.synchronize(dev)
-        cold.append(c0.elapsed_time(c1))
-    del flush
-    d0 = torch.cuda.Event(enable_timing=True)
-    d1 = torch.cuda.Event(enable_timing=True)
-    n_dec = 200
-    d0.record(stream)
-    for i in range(n_dec):
-        decode(i)
-    d1.record(stream)
-    torch.cuda.synchronize(dev)
-    barrier()
-    dec_ms = max_over_ranks(d0.elapsed_time(d1) / n_dec, dist if world > 1 else None, dev)
-    dec_cold = max_over_ranks(sorted(cold)[len(cold) // 2], dist if world > 1 else None, dev)
-
-    # the Mamba-2-shaped SSD layer (one scalar A per head, chunked form on the
-    # tensor cores): back to back, and after an L2-evicting write; not part
-    # of the metric
-    sw = wl.SSD
-    sinp = wl.make_ssd_inputs(sw, device=dev)
-    sy = torch.empty_like(sinp["x"])
-    sfs = torch.empty(sw.batch, sw.dim, sw.dstate, device=dev)
-
-    def ssd_call():
-        ss.selscan_ssd_fwd(sinp["x"], sinp["dt"], sinp["A"], sinp["B"], sinp["C"], D=sinp["D"],
-                           z=sinp["z"], dt_bias=sinp["dt_bias"], y=sy, final_state=sfs,
-                           stream=stream)
-
-    for _ in range(5):
-        ssd_call()
-    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
-    scold = []
-    for _ in range(10):
-        flush.zero_()
-        c0 = torch.cuda.Event(enable_timing=True)
-        c1 = torch.cuda.Event(enable_timing=True)
-        c0.record(stream)
-        ssd_call()
-        c1.record(stream)
-        torch.cuda.synchronize(dev)
-        scold.append(c0.elapsed_time(c1))
-    del flush
-    s0 = torch.cuda.Event(enable_timing=True)
-    s1 = torch.cuda.Event(enable_timing=True)
-    n_ssd = 50
-    s0.record(stream)
-    for _ in range(n_ssd):
-        ssd_call()
-    s1.record(stream)
-    torch.cuda.synchronize(dev)
-    barrier()
-    ssd_ms = max_over_ranks(s0.elapsed_time(s1) / n_ssd, dist if world > 1 else None, dev)
-    ssd_cold = max_over_ranks(sorted(scold)[len(scold) // 2], dist if world > 1 else None, dev)
+    peak, peak_kind = peaks()
+    legs = extra_legs(args, torch, ss, wl, dev, stream, peak,
+                      lambda v: max_over_ranks(v, dist if world > 1 else None, dev))
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -492,7 +541,6 @@ def main():
     per_launch_s = ms / 1e3 / args.steps
     alg_bytes = w.algorithmic_bytes()
     achieved = alg_bytes / per_launch_s / 1e9
-    peak, peak_kind = peaks()
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup,
@@ -504,26 +552,12 @@ def main():
                      "frac": achieved / peak, "peak_kind": peak_kind,
                      "frac_of_8TBps": achieved / 8000.0,
                      "algorithmic_bytes_per_launch": alg_bytes,
-                     "kernel": "scan_tma_kernel<bf16, gate, seq>",
+                     "kernel": "scan_tma_kernel<bf16, gate, seq, softplus> (two lanes per chain)",
                      "traffic": profiled_traffic()},
         "e2e": {"value": job_rate(w.elements, world, args.e2e_steps, e2e_ms),
                 "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": e2e_ms / args.e2e_steps},
-        "decode_step": {
-            "workload": dw.name, "bytes_per_step": dw.algorithmic_bytes_per_step(),
-            "us_back_to_back": dec_ms * 1e3, "us_after_l2_flush": dec_cold * 1e3,
-            "GBps_back_to_back": dw.algorithmic_bytes_per_step() / dec_ms / 1e6,
-            "frac_back_to_back": dw.algorithmic_bytes_per_step() / dec_ms / 1e6 / peak,
-            "kernel": "state_update_vec_kernel<bf16, gate>"},
-        "ssd_layer": {
-            "workload": sw.name, "bytes_per_call": sw.algorithmic_bytes(),
-            "flops_per_call": sw.algorithmic_flops(),
-            "us_back_to_back": ssd_ms * 1e3, "us_after_l2_flush": ssd_cold * 1e3,
-            "GBps_back_to_back": sw.algorithmic_bytes() / ssd_ms / 1e6,
-            "TFLOPs_back_to_back": sw.algorithmic_flops() / ssd_ms / 1e9,
-            "frac_hbm_back_to_back": sw.algorithmic_bytes() / ssd_ms / 1e6 / peak,
-            "frac_tensor_back_to_back": sw.algorithmic_flops() / ssd_ms / 1e9 / tensor_peak(),
-            "kernels": ["ssd_tc_state_kernel", "ssd_tc_carry_kernel", "ssd_tc_out_kernel<gate>"]},
+        **legs,
         "gpu_launches": args.steps * plan["launches"],
         "plan": plan,
         "cpu_baseline": cpu,

@@ -179,3 +179,23 @@ def test_cpu_sample_size_is_bounded():
                 assert 1 <= n <= w.dim
                 if cores <= int(rate * seconds / per_ch) < w.dim:
                     assert n % cores == 0
+
+
+def test_cpu_baseline_and_reference_share_one_sample():
+    """cpu_baseline and the reference arm draw their sample from the same
+    definition: a channel subset of batch row 0 for a short budget, whole
+    rows (and repeated passes) for a long one; the elements it reports match
+    the arrays it hands to the oracle."""
+    from selective_state_space_42_b200 import workloads as wl
+    w = wl.ScanWorkload("sample", 3, 64, 96, 16, "f32", gate=True, seed=3)
+    inp = wl.make_scan_inputs(w)
+    short = bench.oracle_sample(w, inp, 1e-9, 2)
+    args, reps, per_pass, desc = short
+    assert reps == 1 and args[0].shape[0] == 1 and args[0].shape[2] < w.dim
+    assert per_pass == args[0].shape[0] * args[0].shape[2] * w.seqlen * w.dstate
+    assert "batch row 0, channels 0.." in desc
+    args, reps, per_pass, desc = bench.oracle_sample(w, inp, 1e3, 2)
+    assert args[0].shape == (w.batch, w.seqlen, w.dim) and reps >= 1
+    assert per_pass == w.elements
+    cb = bench.oracle_cpu_baseline(inp, w, 1e-9)
+    assert cb["kind"] == "oracle" and cb["value"] > 0 and "channels 0.." in cb["sample"]
