@@ -130,8 +130,8 @@ def test_channel_slices_properties():
             assert sl[0][0] == 0 and sl[-1][1] == dim
             assert all(a[1] == b[0] for a, b in zip(sl, sl[1:]))
             assert all(d0 % 128 == 0 or d0 == dim for d0, _ in sl)
-            widths = [d1 - d0 for d0, d1 in sl]
-            assert max(widths) - min(widths) <= 128
+            tiles = [-(-(d1 - d0) // 128) for d0, d1 in sl]
+            assert max(tiles) - min(tiles) <= 1  # balanced in whole tiles
 
 
 def test_two_ranks_gloo():
