@@ -21,7 +21,7 @@ CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB_PATH = os.path.join(HERE, "libselscan.so")
 OBJ_DIR = os.path.join(HERE, "_build")
-SOURCES = ["api.cu", "scan.cu", "scan_tma.cu", "scan_wide.cu", "scan_bwd.cu", "ssd.cu", "ssd_tc.cu",
+SOURCES = ["api.cu", "scan.cu", "scan_tma.cu", "scan_wide.cu", "scan_bwd.cu", "scan_bwd2.cu", "ssd.cu", "ssd_tc.cu",
            "state_update.cu", "noalloc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

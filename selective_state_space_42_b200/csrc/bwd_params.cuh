@@ -39,6 +39,9 @@ struct BwdParams {
 };
 
 cudaError_t launch_scan_bwd(const BwdParams &p, bool bf16, cudaStream_t stream);
+// Two lanes per chain (scan_bwd2.cu): one 16-state group, no conv, Δ·B·x input.
+bool bwd_pairs_supported(const BwdParams &p);
+cudaError_t launch_scan_bwd_pairs(const BwdParams &p, bool bf16, cudaStream_t stream);
 int bwd_tile_tokens();
 int bwd_tile_channels();
 int bwd_conv_tile_tokens();

@@ -736,7 +736,9 @@ int bwd_conv_tile_tokens() { return kConvTile; }
 
 cudaError_t launch_scan_bwd(const BwdParams &p, bool bf16, cudaStream_t stream) {
     cudaError_t e;
-    if (bf16)
+    if (bwd_pairs_supported(p))
+        e = launch_scan_bwd_pairs(p, bf16, stream);
+    else if (bf16)
         e = p.z ? launch_gate<__nv_bfloat16, true>(p, stream)
                 : launch_gate<__nv_bfloat16, false>(p, stream);
     else

@@ -6,6 +6,7 @@ the device) and to give quick CUDA-event timings without one:
     python -m selective_state_space_42_b200.profile_case scan mamba2p8b_layer --launches 2
     python -m selective_state_space_42_b200.profile_case decode --launches 3
     python -m selective_state_space_42_b200.profile_case bwd mamba2p8b_layer --launches 2
+    python -m selective_state_space_42_b200.profile_case bwd mamba2p8b_layer --seqlen 1024
     python -m selective_state_space_42_b200.profile_case ssd --launches 3
 
 ``scan`` calls selscan_fwd on a scan workload; ``bwd`` calls selscan_bwd on
@@ -18,6 +19,7 @@ between launches, which evicts L2) and back to back, as one JSON line.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 
 import torch
@@ -26,8 +28,13 @@ from . import selscan as ss
 from . import workloads as wl
 
 
-def _scan_case(name: str):
+def _workload(name: str, seqlen: int | None):
     w = wl.WORKLOADS[name]
+    return w if seqlen is None else dataclasses.replace(w, seqlen=seqlen)
+
+
+def _scan_case(name: str, seqlen: int | None = None):
+    w = _workload(name, seqlen)
     inp = wl.make_scan_inputs(w, device="cuda")
     y = torch.empty_like(inp["x"])
     fs = torch.empty(w.batch, w.dim, w.dstate, device="cuda") if w.final_state else None
@@ -40,8 +47,8 @@ def _scan_case(name: str):
     return launch, w.algorithmic_bytes()
 
 
-def _bwd_case(name: str):
-    w = wl.WORKLOADS[name]
+def _bwd_case(name: str, seqlen: int | None = None):
+    w = _workload(name, seqlen)
     inp = wl.make_scan_inputs(w, device="cuda")
     g = torch.Generator(device="cuda")
     g.manual_seed(w.seed + 1000)
@@ -96,12 +103,14 @@ def main(argv=None) -> int:
                     help="scan workload name (ignored for decode)")
     ap.add_argument("--launches", type=int, default=2)
     ap.add_argument("--time", action="store_true")
+    ap.add_argument("--seqlen", type=int, default=None,
+                    help="scan and bwd: the workload cut (or grown) to this many tokens")
     args = ap.parse_args(argv)
 
     if args.kernel == "scan":
-        launch, nbytes = _scan_case(args.workload)
+        launch, nbytes = _scan_case(args.workload, args.seqlen)
     elif args.kernel == "bwd":
-        launch, nbytes = _bwd_case(args.workload)
+        launch, nbytes = _bwd_case(args.workload, args.seqlen)
     elif args.kernel == "ssd":
         launch, nbytes = _ssd_case()
     else:
@@ -112,7 +121,7 @@ def main(argv=None) -> int:
     out = {"kernel": args.kernel, "launches": args.launches,
            "workload": {"decode": wl.DECODE.name, "ssd": wl.SSD.name}.get(args.kernel,
                                                                           args.workload),
-           "algorithmic_bytes": nbytes}
+           "seqlen": args.seqlen, "algorithmic_bytes": nbytes}
     if args.time:
         flush = torch.empty(512 << 20, dtype=torch.uint8, device="cuda")
         cold = []
