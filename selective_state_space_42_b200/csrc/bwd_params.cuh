@@ -23,7 +23,9 @@ struct BwdParams {
     // workspace
     float *ckpt;   // [groups][batch][ktiles][dim][16]: state of each 16-state group entering each token tile
     float *part;   // [groups][batch][ctiles][seqlen][32]: per channel tile, Σ over its channels
-                   // of dB (0..15), dC (16..31) of the group's states
+                   // of dB (0..15), dC (16..31) of the group's states; with part_lane_order
+                   // value 16·c + n (c = 1 for dC) sits at 4·(4c + 2·(n & 1) + n / 8) + (n / 2) % 4
+    int part_lane_order;  // set by launch_scan_bwd for the kernel it runs
     float *pA;     // [groups][batch][dim][16]: Σ over tokens of dA
     float *acc;    // groups > 1: [groups][3][batch][seqlen][dim] float32: each group's part of
                    // dΔ (before the softplus derivative), dx and the pre-gate output
@@ -40,7 +42,7 @@ struct BwdParams {
 
 cudaError_t launch_scan_bwd(const BwdParams &p, bool bf16, cudaStream_t stream);
 // Two lanes per chain (scan_bwd2.cu): one 16-state group, no conv, Δ·B·x input.
-bool bwd_pairs_supported(const BwdParams &p);
+bool bwd_pairs_supported(const BwdParams &p, bool bf16);
 cudaError_t launch_scan_bwd_pairs(const BwdParams &p, bool bf16, cudaStream_t stream);
 int bwd_tile_tokens();
 int bwd_tile_channels();

@@ -578,8 +578,10 @@ __global__ void bwd_reduce_bc_kernel(const BwdParams p) {
     const long long tok = rest / kVals;
     const int n = 16 * g + v % kMaxN;
     if (n >= p.dstate) return;
+    const int m = v % kMaxN;
+    const int pv = p.part_lane_order ? 4 * (4 * (v / kMaxN) + 2 * (m & 1) + m / 8) + (m / 2) % 4 : v;
     const float *src = p.part + ((long long)g * p.batch * p.ctiles + b * p.ctiles) * p.seqlen * kVals +
-                       rest;
+                       tok * kVals + pv;
     float sum = 0.f;
     for (int c = 0; c < p.ctiles; ++c) sum += src[(long long)c * p.seqlen * kVals];
     float *dst = v < kMaxN ? p.dB : p.dC;
@@ -734,9 +736,11 @@ int bwd_tile_tokens() { return kSeg; }
 int bwd_tile_channels() { return kChains; }
 int bwd_conv_tile_tokens() { return kConvTile; }
 
-cudaError_t launch_scan_bwd(const BwdParams &p, bool bf16, cudaStream_t stream) {
+cudaError_t launch_scan_bwd(const BwdParams &params, bool bf16, cudaStream_t stream) {
     cudaError_t e;
-    if (bwd_pairs_supported(p))
+    BwdParams p = params;
+    p.part_lane_order = bwd_pairs_supported(p, bf16) ? 1 : 0;
+    if (p.part_lane_order)
         e = launch_scan_bwd_pairs(p, bf16, stream);
     else if (bf16)
         e = p.z ? launch_gate<__nv_bfloat16, true>(p, stream)

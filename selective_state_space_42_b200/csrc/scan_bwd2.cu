@@ -1,5 +1,6 @@
 // scan_bwd2.cu -- gradient of the selective scan with two lanes per chain
-// (d_state ≤ 16 in one group, no conv front end, Δ·B·x input term).
+// (d_state ≤ 16 in one group, no conv front end, Δ·B·x input term, rows of
+// whole 16-byte chunks).
 //
 // Pages: "Mamba: co potrafią modele przestrzeni stanów", "Cena selekcji"
 // (the backward pass recomputes the intermediate states instead of storing
@@ -10,22 +11,27 @@
 // The sweeps and formulas are those of scan_bwd.cu (see its header): a
 // forward sweep storing the state entering every 8-token tile, then a reverse
 // sweep over the tiles that recomputes each tile's states from its checkpoint
-// and walks the tile backwards carrying λ = ∂loss/∂h. The thread layout
+// and walks the tile backwards carrying λ = ∂loss/∂h. The organisation
 // differs:
 //  * lanes l and l + 16 of a warp share one channel, the lower lane keeping
 //    the even states and the upper lane the odd ones (8 each), so a layer of
 //    20,480 chains puts two warps where scan_bwd.cu has one;
 //  * every per-token scalar (softplus and its derivative, silu(z) and its
 //    derivative, the decay base, Δ·x) is formed once per token by one of the
-//    two lanes (tokens 0–3 of a tile by the lower lane, 4–7 by the upper),
-//    which also writes that token's dx, ddelta and dz at the end of the tile;
+//    two lanes (the even tokens of a tile by the lower lane, the odd ones by
+//    the upper), which also forms that token's dx, ddelta and dz at the end
+//    of the tile;
+//  * a tile's inputs (x, delta, z, dy rows of the warp's 16 channels, the B
+//    and C rows, the checkpoint) arrive by cp.async into shared memory one
+//    tile ahead, and its dx, ddelta, dz leave as 16-byte row chunks;
 //  * the channel sums of dB and dC are formed per half tile, not per token:
 //    the walk stores λ_t, the recompute has already stored h_t, and 32 lanes
 //    each form 4 of the 4 tokens × 32 sums as Σ_c λ_t[c]·u_t[c] and
 //    Σ_c ds_t[c]·h_t[c] (the products dB = λ·u and dC = ds·h are never formed
 //    per chain); per tile the CTA's two warps add their rows and write one
-//    128-byte row per token to the partial buffer of scan_bwd.cu, which its
-//    reduction kernel sums over the channel tiles.
+//    128-byte row per token to the partial buffer of scan_bwd.cu, in the
+//    reducer's value order (part_lane_order), which its reduction kernel
+//    sums over the channel tiles.
 // With λa = λ_t·Abar_t (the λ carried to token t − 1), the per-state work of
 // the walk is six f32x2 operations per state pair: λ_t = ds·C + λa_{t+1},
 // du += λ_t·B, λa = λ_t·Abar_t, lh = λa·h_{t−1}, q += lh·A, dA += Δ·lh.
@@ -49,25 +55,35 @@ __device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a
 __device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
 __device__ __forceinline__ float2 dup2(float v) { return make_float2(v, v); }
 
+// 16 bytes global → shared, bypassing registers and L1; src_bytes = 0 fills
+// the 16 bytes with zeros (the source is then not read).
+__device__ __forceinline__ void cp_async16(void *dst, const void *src, int src_bytes) {
+    const unsigned s = (unsigned)__cvta_generic_to_shared(dst);
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(s), "l"(src),
+                 "r"(src_bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;\n" ::: "memory"); }
+
 // A warp's shared memory. hs and lam rows hold one float4 per (lane, half):
 // half 0 = state pairs 0, 1 of the lane, half 1 = pairs 2, 3; the slot of lane
 // l is l ^ (4·half + 2·(l ≥ 16) + is_h), so that the reducer's column reads
 // (8 lanes: both halves, both parities, λ and h, one channel) fall in 8
 // distinct bank quads, while a lane reads back only the slots it wrote.
-struct WarpSmem {
+template <typename T>
+struct alignas(128) WarpSmem {
+    T raw[4][kSeg][kCh];             // x, delta, z, dy rows of the next tile (cp.async target)
+    T bc[2][kSeg * kMaxN];           // B, C of the next tile as stored (8·N used)
+    float4 h0[2][2][32];             // checkpoints, by tile parity (slots as hs)
     float B[kSeg][kMaxN];            // float32; [0..7] the even states, [8..15] the odd ones
     float C[kSeg][kMaxN];
     float4 sc[kSeg][kCh + 1];        // Δ, u = Δ·x, ds = dy·silu(z), r = 2^(Δ·A[d,0]·log2 e)
-    float4 hs[kSeg + 1][2][32];      // hs[0]: state entering the tile; hs[t + 1]: after token t
+    float4 hs[kSeg][2][32];          // state after token t
     float4 lam[kOwn][2][32];         // λ of the half tile being reduced
-    float sv[kSeg][kCh];             // per token: s = Σ C·h (the D·x term is added later)
-    float du[kSeg][kCh];             //   Σ_n λ·B
-    float qp[kSeg][kCh];             //   Σ_n λ·Abar·h_{t−1}·A[n]
-    float4 row[2][kSeg][kVals / 4];  // per-warp channel sums of the tile, double buffered
-};
-
-struct __align__(128) Smem {
-    WarpSmem w[kWarps];
+    float tok[3][kSeg][kCh];         // per token: Σ C·h, Σ λ·B, Σ λ·Abar·h_{t−1}·A; then
+                                     // reused for the tile's dx, ddelta, dz rows (type T)
+    float4 row[kSeg][kVals / 4];     // per-warp channel sums of the tile, reducer order
 };
 
 __device__ __forceinline__ int slot(int lane, int half, int is_h) {
@@ -95,88 +111,116 @@ __device__ __forceinline__ void decay8(float dt, float r, bool odd, const float2
     }
 }
 
-// B and C of one tile: lane l fetches token l / 4, float4 slot l % 4 of the
-// shared rows (slots 0, 1: the even states; 2, 3: the odd ones), a tile ahead
-// into registers; C only in the reverse sweep.
+// Where a tile's rows are.
+struct TileGeo {
+    long long row0;  // batch row · seqlen + first token of the tile
+    long long t0;    // first token
+    long long d0;    // the warp's first channel
+};
+
+// cp.async of one tile's inputs into the warp's buffers: the rows of the
+// arrays in amask (bit a: 0 x, 1 delta, 2 z, 3 dy), B (and C when withC),
+// and the checkpoint (when ck is not null). Chunks past the sequence or the
+// channels are zero filled.
 template <typename T>
-__device__ __forceinline__ void fetch_bc(float (&vb)[4], float (&vc)[4], const BwdParams &p,
-                                         long long b, long long t0, int lane, bool withC) {
-    const int s = lane & 3;
+__device__ __forceinline__ void issue_tile(WarpSmem<T> &W, const BwdParams &p, const TileGeo &g,
+                                           int amask, bool withC, const float4 *ck, int hbuf,
+                                           bool active, int lane) {
+    constexpr int kPer = 16 / sizeof(T);        // elements per chunk
+    constexpr int kRowChunks = kCh / kPer;      // chunks per 16-channel row
+    constexpr int kArr = kSeg * kRowChunks;     // chunks per array
+#pragma unroll
+    for (int c0 = 0; c0 < 4 * kArr; c0 += 32) {
+        const int c = c0 + lane;
+        const int a = c / kArr;
+        if ((amask >> a) & 1) {
+            const int r = (c % kArr) / kRowChunks, q = c % kRowChunks;
+            const long long ch = g.d0 + q * kPer;
+            const bool ok = g.t0 + r < p.seqlen && ch < p.dim;
+            const void *arr = a == 0 ? p.x : a == 1 ? p.delta : a == 2 ? p.z : p.dy;
+            const T *s = static_cast<const T *>(arr) + (ok ? (g.row0 + r) * p.dim + ch : 0);
+            cp_async16(&W.raw[a][r][q * kPer], s, ok ? 16 : 0);
+        }
+    }
+    // B and C: the tile's 8·N elements are contiguous
+    const int nb = kSeg * p.dstate / kPer;      // chunks per matrix (whole: checked on the host)
+    const long long e0 = g.row0 * p.dstate;
+    const long long end = (g.row0 - g.t0 + p.seqlen) * p.dstate;  // end of the batch row
+    for (int c = lane; c < 2 * nb; c += 32) {
+        const int m = c >= nb;
+        if (m && !withC) break;
+        const int q = c - m * nb;
+        const long long e = e0 + q * kPer;
+        const bool ok = e < end;
+        const T *base = static_cast<const T *>(m ? p.C : p.B);
+        cp_async16(&W.bc[m][q * kPer], base + (ok ? e : 0), ok ? 16 : 0);
+    }
+    if (ck) {
+        cp_async16(&W.h0[hbuf][0][slot(lane, 0, 1)], ck, active ? 16 : 0);
+        cp_async16(&W.h0[hbuf][1][slot(lane, 1, 1)], ck + 1, active ? 16 : 0);
+    }
+    cp_async_commit();
+}
+
+// The landed B (and C) as float32 rows, even states then odd: lane l writes
+// token l / 4, float4 slot l % 4.
+template <typename T>
+__device__ __forceinline__ void convert_bc(WarpSmem<T> &W, int N, int lane, bool withC) {
+    const int t = lane >> 2, s = lane & 3;
     const int odd = s >> 1, i0 = (s & 1) * 4;
-    const long long tok = t0 + (lane >> 2);
+    float vb[4], vc[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
         const int n = 2 * (i0 + e) + odd;
-        const bool ok = tok < p.seqlen && n < p.dstate;
-        const long long idx = (b * p.seqlen + tok) * p.dstate + n;
-        vb[e] = ok ? ldg_f32(static_cast<const T *>(p.B) + idx) : 0.0f;
-        vc[e] = (ok && withC) ? ldg_f32(static_cast<const T *>(p.C) + idx) : 0.0f;
+        const bool ok = n < N;
+        vb[e] = ok ? to_f32(W.bc[0][t * N + n]) : 0.0f;
+        vc[e] = (ok && withC) ? to_f32(W.bc[1][t * N + n]) : 0.0f;
     }
-}
-
-__device__ __forceinline__ void store_bc(WarpSmem &W, const float (&vb)[4], const float (&vc)[4],
-                                         int lane, bool withC) {
-    const int t = lane >> 2, s = lane & 3;
     *reinterpret_cast<float4 *>(&W.B[t][4 * s]) = make_float4(vb[0], vb[1], vb[2], vb[3]);
     if (withC)
         *reinterpret_cast<float4 *>(&W.C[t][4 * s]) = make_float4(vc[0], vc[1], vc[2], vc[3]);
 }
 
-// Raw inputs of the lane's 4 owned tokens of a tile (x, delta; z, dy in the
-// reverse sweep), a tile ahead.
-template <typename T> struct Raw {
-    T x[kOwn], dl[kOwn], z[kOwn], dy[kOwn];
-};
-
-template <typename T, bool kGate, bool kBwd>
-__device__ __forceinline__ void load_raw(Raw<T> &r, const BwdParams &p, long long b,
-                                         long long tok0, long long d, bool active) {
-    const T zero = from_f32<T>(0.0f);
-    const long long i0 = (b * p.seqlen + tok0) * p.dim + d;
-#pragma unroll
-    for (int j = 0; j < kOwn; ++j) {
-        const bool ok = active && tok0 + j < p.seqlen;
-        const long long i = i0 + j * p.dim;
-        r.x[j] = ok ? __ldg(static_cast<const T *>(p.x) + i) : zero;
-        r.dl[j] = ok ? __ldg(static_cast<const T *>(p.delta) + i) : zero;
-        if (kBwd) {
-            r.dy[j] = ok ? __ldg(static_cast<const T *>(p.dy) + i) : zero;
-            if (kGate) r.z[j] = ok ? __ldg(static_cast<const T *>(p.z) + i) : zero;
-        }
-    }
-}
-
 // One half tile's channel sums: lane (j, v) forms, for token base + j, the 4
 // values of group v (v < 4: dB of states 8·(v & 1) + 2e + (v >> 1); v ≥ 4: dC
 // of the same states for v − 4) summed over the warp's 16 channels.
-__device__ __forceinline__ void reduce_half(WarpSmem &W, int buf, int base, int lane) {
+template <typename T>
+__device__ __forceinline__ void reduce_half(WarpSmem<T> &W, int base, int lane) {
     const int j = lane >> 3, v = lane & 7;
     const int is_h = v >> 2, par = (v >> 1) & 1, half = v & 1;
     const int t = base + j;
-    const float4 *src = is_h ? &W.hs[t + 1][half][0] : &W.lam[j][half][0];
+    const float4 *src = is_h ? &W.hs[t][half][0] : &W.lam[j][half][0];
     const float *w = reinterpret_cast<const float *>(&W.sc[t][0]) + 1 + is_h;  // u or ds
     const int mask = 4 * half + 2 * par + is_h;
-    float2 a01 = make_float2(0.f, 0.f), a23 = a01;
+    float2 a01 = make_float2(0.f, 0.f), a23 = a01, b01 = a01, b23 = a01;
 #pragma unroll
-    for (int c = 0; c < kCh; ++c) {
-        const float4 val = src[(16 * par + c) ^ mask];
-        const float2 wc = dup2(w[4 * c]);
-        a01 = fma2(make_float2(val.x, val.y), wc, a01);
-        a23 = fma2(make_float2(val.z, val.w), wc, a23);
+    for (int c = 0; c < kCh; c += 2) {
+        const float4 v0 = src[(16 * par + c) ^ mask];
+        const float4 v1 = src[(16 * par + c + 1) ^ mask];
+        const float2 w0 = dup2(w[4 * c]), w1 = dup2(w[4 * c + 4]);
+        a01 = fma2(make_float2(v0.x, v0.y), w0, a01);
+        a23 = fma2(make_float2(v0.z, v0.w), w0, a23);
+        b01 = fma2(make_float2(v1.x, v1.y), w1, b01);
+        b23 = fma2(make_float2(v1.z, v1.w), w1, b23);
     }
-    W.row[buf][t][v] = make_float4(a01.x, a01.y, a23.x, a23.y);
+    a01 = __fadd2_rn(a01, b01);
+    a23 = __fadd2_rn(a23, b23);
+    W.row[t][v] = make_float4(a01.x, a01.y, a23.x, a23.y);
 }
 
 template <typename T, bool kGate, bool kSoftplus, bool kStruct>
-__device__ __forceinline__ void bwd_pairs_body(Smem &S, const BwdParams &p) {
+__device__ __forceinline__ void bwd_pairs_body(WarpSmem<T> *S, const BwdParams &p) {
+    constexpr int kPer = 16 / sizeof(T);
+    constexpr int kRowChunks = kCh / kPer;
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const bool odd = lane >= 16;
     const int cl = lane & 15;
-    const int own0 = odd ? kOwn : 0;  // first owned token of a tile
-    WarpSmem &W = S.w[warp];
+    const int par = odd ? 1 : 0;  // the lane's owned tokens of a tile: 2j + par
+    WarpSmem<T> &W = S[warp];
     const long long b = blockIdx.y;
-    const long long d = (long long)blockIdx.x * (kWarps * kCh) + warp * kCh + cl;
+    const long long d0 = (long long)blockIdx.x * (kWarps * kCh) + warp * kCh;
+    const long long d = d0 + cl;
     const bool active = d < p.dim;
     const int N = p.dstate;
     const long long dd = active ? d : 0;
@@ -202,6 +246,13 @@ __device__ __forceinline__ void bwd_pairs_body(Smem &S, const BwdParams &p) {
     const long long ck_stride = p.dim * 4;
     const int hs0 = slot(lane, 0, 1), hs1 = slot(lane, 1, 1);
     const int lm0 = slot(lane, 0, 0), lm1 = slot(lane, 1, 0);
+    auto geo = [&](int k) {
+        TileGeo g;
+        g.t0 = (long long)k * kSeg;
+        g.row0 = b * p.seqlen + g.t0;
+        g.d0 = d0;
+        return g;
+    };
 
     // ---- 1. forward sweep: checkpoints ------------------------------------------
     {
@@ -213,30 +264,27 @@ __device__ __forceinline__ void bwd_pairs_body(Smem &S, const BwdParams &p) {
             h[q] = make_float2((active && p.h0 && n0 < N) ? h0[n0] : 0.f,
                                (active && p.h0 && n1 < N) ? h0[n1] : 0.f);
         }
-        Raw<T> cur, nxt;
-        float vb[4], vc[4];
-        load_raw<T, kGate, false>(cur, p, b, own0, dd, active);
-        fetch_bc<T>(vb, vc, p, b, 0, lane, false);
+        issue_tile(W, p, geo(0), 0x3, false, nullptr, 0, active, lane);
         for (int k = 0; k < K; ++k) {
             const long long t0 = (long long)k * kSeg;
+            cp_async_wait_all();
+            __syncwarp();
+            convert_bc(W, N, lane, false);
+#pragma unroll
+            for (int j = 0; j < kOwn; ++j) {
+                const int t = 2 * j + par;
+                const float v = to_f32(W.raw[1][t][cl]) + bias;
+                const bool live = active && t0 + t < p.seqlen;
+                const float dt = live ? (kSoftplus ? softplus_f32(v) : v) : 0.0f;
+                W.sc[t][cl] = make_float4(dt, dt * to_f32(W.raw[0][t][cl]), 0.0f,
+                                          ex2_approx(dt * A0l));
+            }
             if (active) {
                 ck[k * ck_stride] = make_float4(h[0].x, h[0].y, h[1].x, h[1].y);
                 ck[k * ck_stride + 1] = make_float4(h[2].x, h[2].y, h[3].x, h[3].y);
             }
-            store_bc(W, vb, vc, lane, false);
-            if (k + 1 < K) {
-                load_raw<T, kGate, false>(nxt, p, b, t0 + kSeg + own0, dd, active);
-                fetch_bc<T>(vb, vc, p, b, t0 + kSeg, lane, false);
-            }
-#pragma unroll
-            for (int j = 0; j < kOwn; ++j) {
-                const float v = to_f32(cur.dl[j]) + bias;
-                const bool live = active && t0 + own0 + j < p.seqlen;
-                const float dt = live ? (kSoftplus ? softplus_f32(v) : v) : 0.0f;
-                W.sc[own0 + j][cl] = make_float4(dt, dt * to_f32(cur.x[j]), 0.0f,
-                                                 ex2_approx(dt * A0l));
-            }
             __syncwarp();
+            if (k + 1 < K) issue_tile(W, p, geo(k + 1), 0x3, false, nullptr, 0, active, lane);
 #pragma unroll 2
             for (int t = 0; t < kSeg; ++t) {
                 const float4 sc = W.sc[t][cl];
@@ -250,10 +298,10 @@ __device__ __forceinline__ void bwd_pairs_body(Smem &S, const BwdParams &p) {
                 h[2] = fma2(a[2], h[2], mul2(u2, make_float2(b1.x, b1.y)));
                 h[3] = fma2(a[3], h[3], mul2(u2, make_float2(b1.z, b1.w)));
             }
-            __syncwarp();
-            cur = nxt;
         }
     }
+    // the checkpoints just written are read back below by the same threads
+    __threadfence_block();
 
     // ---- 2. reverse sweep ---------------------------------------------------------
     float2 lam[kPairs], dA[kPairs];
@@ -267,39 +315,29 @@ __device__ __forceinline__ void bwd_pairs_body(Smem &S, const BwdParams &p) {
     }
     float accD = 0.f, accBias = 0.f;
     float *part = p.part + (b * p.ctiles + blockIdx.x) * p.seqlen * kVals;
-    Raw<T> cur, nxt;
-    float vb[4], vc[4];
-    float4 hc0, hc1, hn0, hn1;
-    {
-        const long long t0 = (long long)(K - 1) * kSeg;
-        load_raw<T, kGate, true>(cur, p, b, t0 + own0, dd, active);
-        fetch_bc<T>(vb, vc, p, b, t0, lane, true);
-        hc0 = active ? ck[(K - 1) * ck_stride] : make_float4(0.f, 0.f, 0.f, 0.f);
-        hc1 = active ? ck[(K - 1) * ck_stride + 1] : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
+    const int amask = kGate ? 0xf : 0xb;
+    __syncwarp();
+    issue_tile(W, p, geo(K - 1), amask, true, ck + (K - 1) * ck_stride, (K - 1) & 1, active, lane);
     for (int k = K - 1; k >= 0; --k) {
         const long long t0 = (long long)k * kSeg;
         const int buf = k & 1;
-        store_bc(W, vb, vc, lane, true);
-        if (k > 0) {
-            load_raw<T, kGate, true>(nxt, p, b, t0 - kSeg + own0, dd, active);
-            fetch_bc<T>(vb, vc, p, b, t0 - kSeg, lane, true);
-            hn0 = active ? ck[(k - 1) * ck_stride] : make_float4(0.f, 0.f, 0.f, 0.f);
-            hn1 = active ? ck[(k - 1) * ck_stride + 1] : make_float4(0.f, 0.f, 0.f, 0.f);
-        }
+        cp_async_wait_all();
+        __syncthreads();  // also: both warps are done with the previous tile's sums
+        convert_bc(W, N, lane, true);
         // owned tokens' scalars; x, dy·silu'(z) and σ stay in registers for
         // the tile's epilogue
         float xo[kOwn], dyso[kOwn], sgo[kOwn];
 #pragma unroll
         for (int j = 0; j < kOwn; ++j) {
-            const bool live = active && t0 + own0 + j < p.seqlen;
-            const float xv = to_f32(cur.x[j]);
-            const float v = to_f32(cur.dl[j]) + bias;
+            const int t = 2 * j + par;
+            const bool live = active && t0 + t < p.seqlen;
+            const float xv = to_f32(W.raw[0][t][cl]);
+            const float v = to_f32(W.raw[1][t][cl]) + bias;
             const float dt = live ? (kSoftplus ? softplus_f32(v) : v) : 0.0f;
-            const float dyv = to_f32(cur.dy[j]);
+            const float dyv = to_f32(W.raw[3][t][cl]);
             float ds = dyv, dysz = 0.f;
             if (kGate) {
-                const float zv = to_f32(cur.z[j]);
+                const float zv = to_f32(W.raw[2][t][cl]);
                 const float sgz = sigmoid_f32(zv);
                 ds = dyv * zv * sgz;
                 dysz = dyv * sgz * fmaf(zv, 1.0f - sgz, 1.0f);
@@ -307,14 +345,15 @@ __device__ __forceinline__ void bwd_pairs_body(Smem &S, const BwdParams &p) {
             xo[j] = xv;
             dyso[j] = dysz;
             sgo[j] = kSoftplus ? sigmoid_f32(v) : 1.0f;
-            W.sc[own0 + j][cl] = make_float4(dt, dt * xv, ds, ex2_approx(dt * A0l));
+            W.sc[t][cl] = make_float4(dt, dt * xv, ds, ex2_approx(dt * A0l));
         }
-        W.hs[0][0][hs0] = hc0;
-        W.hs[0][1][hs1] = hc1;
         __syncwarp();
+        if (k > 0)
+            issue_tile(W, p, geo(k - 1), amask, true, ck + (k - 1) * ck_stride, buf ^ 1, active, lane);
 
         // recompute the tile's states (this lane's 8) and Σ C·h per token
         {
+            const float4 hc0 = W.h0[buf][0][hs0], hc1 = W.h0[buf][1][hs1];
             float2 h[kPairs] = {make_float2(hc0.x, hc0.y), make_float2(hc0.z, hc0.w),
                                 make_float2(hc1.x, hc1.y), make_float2(hc1.z, hc1.w)};
 #pragma unroll 2
@@ -329,8 +368,8 @@ __device__ __forceinline__ void bwd_pairs_body(Smem &S, const BwdParams &p) {
                 h[1] = fma2(a[1], h[1], mul2(u2, make_float2(b0.z, b0.w)));
                 h[2] = fma2(a[2], h[2], mul2(u2, make_float2(b1.x, b1.y)));
                 h[3] = fma2(a[3], h[3], mul2(u2, make_float2(b1.z, b1.w)));
-                W.hs[t + 1][0][hs0] = make_float4(h[0].x, h[0].y, h[1].x, h[1].y);
-                W.hs[t + 1][1][hs1] = make_float4(h[2].x, h[2].y, h[3].x, h[3].y);
+                W.hs[t][0][hs0] = make_float4(h[0].x, h[0].y, h[1].x, h[1].y);
+                W.hs[t][1][hs1] = make_float4(h[2].x, h[2].y, h[3].x, h[3].y);
                 if (kGate) {  // dz needs the pre-gate output s = Σ C·h + D·x
                     const float4 c0 = *reinterpret_cast<const float4 *>(&W.C[t][odd ? 8 : 0]);
                     const float4 c1 = *reinterpret_cast<const float4 *>(&W.C[t][odd ? 12 : 4]);
@@ -340,7 +379,7 @@ __device__ __forceinline__ void bwd_pairs_body(Smem &S, const BwdParams &p) {
                     sacc = fma2(make_float2(c1.z, c1.w), h[3], sacc);
                     float tot = sacc.x + sacc.y;
                     tot += __shfl_xor_sync(0xffffffffu, tot, 16);
-                    W.sv[t][cl] = tot;  // both lanes store the same sum
+                    W.tok[0][t][cl] = tot;  // both lanes store the same sum
                 }
             }
         }
@@ -352,7 +391,8 @@ __device__ __forceinline__ void bwd_pairs_body(Smem &S, const BwdParams &p) {
             float2 a[kPairs];
             decay8<kStruct>(sc.x, sc.w, odd, Al, a);
             const float2 ds2 = dup2(sc.z), dt2 = dup2(sc.x);
-            const float4 hp0 = W.hs[t][0][hs0], hp1 = W.hs[t][1][hs1];
+            const float4 *hp = t > 0 ? &W.hs[t - 1][0][0] : &W.h0[buf][0][0];  // h_{t−1}
+            const float4 hp0 = hp[hs0], hp1 = hp[32 + hs1];
             const float2 hprev[kPairs] = {make_float2(hp0.x, hp0.y), make_float2(hp0.z, hp0.w),
                                           make_float2(hp1.x, hp1.y), make_float2(hp1.z, hp1.w)};
             const float4 b0 = *reinterpret_cast<const float4 *>(&W.B[t][odd ? 8 : 0]);
@@ -380,60 +420,67 @@ __device__ __forceinline__ void bwd_pairs_body(Smem &S, const BwdParams &p) {
             float du = du2.x + du2.y, qs = qp2.x + qp2.y;
             du += __shfl_xor_sync(0xffffffffu, du, 16);
             qs += __shfl_xor_sync(0xffffffffu, qs, 16);
-            W.du[t][cl] = du;  // both lanes store the same sums
-            W.qp[t][cl] = kStruct ? qs * A0l * kLn2 : qs * kLn2;  // Σ_n λ·Abar·h·A[n]
+            W.tok[1][t][cl] = du;  // both lanes store the same sums
+            W.tok[2][t][cl] = kStruct ? qs * A0l * kLn2 : qs * kLn2;  // Σ_n λ·Abar·h·A[n]
             if ((t & 3) == 0) {  // a half tile is walked: its channel sums
                 __syncwarp();
-                reduce_half(W, buf, t, lane);
+                reduce_half(W, t, lane);
                 __syncwarp();
             }
         }
 
-        // the owned tokens' dx, ddelta, dz (the walk ended with a __syncwarp)
+        // the owned tokens' dx, ddelta, dz: formed from the per-token sums,
+        // then written over them as rows of T and stored in 16-byte chunks
         {
-            const long long tok0 = t0 + own0;
-            const long long i0 = (b * p.seqlen + tok0) * p.dim + d;
+            float sv[kOwn], du[kOwn], qp[kOwn];
+            float4 sc[kOwn];
 #pragma unroll
             for (int j = 0; j < kOwn; ++j) {
-                if (active && tok0 + j < p.seqlen) {
-                    const int t = own0 + j;
-                    const float4 sc = W.sc[t][cl];
-                    const float du = W.du[t][cl];
-                    const long long i = i0 + j * p.dim;
-                    const float dv = fmaf(du, xo[j], W.qp[t][cl]) * sgo[j];
-                    static_cast<T *>(p.dx)[i] = from_f32<T>(fmaf(du, sc.x, sc.z * Dv));
-                    static_cast<T *>(p.ddelta)[i] = from_f32<T>(dv);
-                    if (kGate)
-                        static_cast<T *>(p.dz)[i] =
-                            from_f32<T>(fmaf(Dv, xo[j], W.sv[t][cl]) * dyso[j]);
-                    accD = fmaf(sc.z, xo[j], accD);
+                sv[j] = W.tok[0][2 * j + par][cl];
+                du[j] = W.tok[1][2 * j + par][cl];
+                qp[j] = W.tok[2][2 * j + par][cl];
+                sc[j] = W.sc[2 * j + par][cl];
+            }
+            __syncwarp();
+            T *out = reinterpret_cast<T *>(&W.tok[0][0][0]);  // [3][kSeg][kCh]
+#pragma unroll
+            for (int j = 0; j < kOwn; ++j) {
+                const int t = 2 * j + par;
+                const float dv = fmaf(du[j], xo[j], qp[j]) * sgo[j];
+                out[(0 * kSeg + t) * kCh + cl] = from_f32<T>(fmaf(du[j], sc[j].x, sc[j].z * Dv));
+                out[(1 * kSeg + t) * kCh + cl] = from_f32<T>(dv);
+                if (kGate)
+                    out[(2 * kSeg + t) * kCh + cl] = from_f32<T>(fmaf(Dv, xo[j], sv[j]) * dyso[j]);
+                if (active && t0 + t < p.seqlen) {
+                    accD = fmaf(sc[j].z, xo[j], accD);
                     accBias += dv;
                 }
             }
+            __syncwarp();
+            constexpr int kArr = kSeg * kRowChunks;
+            const int nout = kGate ? 3 : 2;
+            const long long row0 = b * p.seqlen + t0;
+            for (int c = lane; c < nout * kArr; c += 32) {
+                const int a = c / kArr, r = (c % kArr) / kRowChunks, q = c % kRowChunks;
+                const long long ch = d0 + q * kPer;
+                void *arr = a == 0 ? p.dx : a == 1 ? p.ddelta : p.dz;
+                if (t0 + r < p.seqlen && ch < p.dim)
+                    *reinterpret_cast<uint4 *>(static_cast<T *>(arr) + (row0 + r) * p.dim + ch) =
+                        *reinterpret_cast<const uint4 *>(out + (a * kSeg + r) * kCh + q * kPer);
+            }
         }
-        // the two warps' sums: one 128-byte row per token of the channel tile
+        // the two warps' sums: one 128-byte row per token of the channel tile,
+        // in the reducer's order (the reduction kernel maps it to states)
         __syncthreads();
         {
             const int t = threadIdx.x >> 3, g = threadIdx.x & 7;
             const long long tok = t0 + t;
             if (tok < p.seqlen) {
-                const float *r0 = reinterpret_cast<const float *>(&S.w[0].row[buf][t][0]);
-                const float *r1 = reinterpret_cast<const float *>(&S.w[1].row[buf][t][0]);
-                float o[4];
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const int vv = 4 * g + i;  // natural index: 16·is_C + n
-                    const int n = vv & 15;
-                    const int e = 4 * (4 * (vv >> 4) + 2 * (n & 1) + (n >> 3)) + ((n >> 1) & 3);
-                    o[i] = r0[e] + r1[e];
-                }
+                const float4 r0 = S[0].row[t][g], r1 = S[1].row[t][g];
                 *reinterpret_cast<float4 *>(part + tok * kVals + 4 * g) =
-                    make_float4(o[0], o[1], o[2], o[3]);
+                    make_float4(r0.x + r1.x, r0.y + r1.y, r0.z + r1.z, r0.w + r1.w);
             }
         }
-        cur = nxt;
-        hc0 = hn0;
-        hc1 = hn1;
     }
 
     // the initial state's gradient: λ carried past the first token
@@ -467,7 +514,8 @@ __device__ __forceinline__ void bwd_pairs_body(Smem &S, const BwdParams &p) {
 
 template <typename T, bool kGate, bool kSoftplus>
 __global__ void __launch_bounds__(kWarps * 32, 5) scan_bwd_pairs_kernel(const BwdParams p) {
-    __shared__ Smem S;
+    extern __shared__ __align__(128) unsigned char smem[];
+    WarpSmem<T> *S = reinterpret_cast<WarpSmem<T> *>(smem);
     // A[d, n] == (n+1)·A[d, 0] for every state of every channel of the CTA
     // selects the power-ladder decay (two threads per channel check it)
     const long long d = (long long)blockIdx.x * (kWarps * kCh) + threadIdx.x / 2;
@@ -485,13 +533,16 @@ __global__ void __launch_bounds__(kWarps * 32, 5) scan_bwd_pairs_kernel(const Bw
 
 template <typename T, bool kGate, bool kSoftplus>
 cudaError_t launch_one(const BwdParams &p, cudaStream_t stream) {
+    const size_t smem = kWarps * sizeof(WarpSmem<T>);
+    auto *kern = scan_bwd_pairs_kernel<T, kGate, kSoftplus>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
     // five CTAs per SM need the largest shared-memory carveout
-    const cudaError_t e = cudaFuncSetAttribute(scan_bwd_pairs_kernel<T, kGate, kSoftplus>,
-                                               cudaFuncAttributePreferredSharedMemoryCarveout,
-                                               cudaSharedmemCarveoutMaxShared);
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return e;
     const dim3 grid((unsigned)p.ctiles, (unsigned)p.batch, 1);
-    scan_bwd_pairs_kernel<T, kGate, kSoftplus><<<grid, kWarps * 32, 0, stream>>>(p);
+    kern<<<grid, kWarps * 32, smem, stream>>>(p);
     return cudaGetLastError();
 }
 
@@ -500,10 +551,17 @@ cudaError_t launch_gate(const BwdParams &p, cudaStream_t stream) {
     return p.softplus ? launch_one<T, kGate, true>(p, stream) : launch_one<T, kGate, false>(p, stream);
 }
 
+bool aligned16(const void *ptr) { return ptr == nullptr || (reinterpret_cast<uintptr_t>(ptr) & 15) == 0; }
+
 }  // namespace
 
-bool bwd_pairs_supported(const BwdParams &p) {
-    return p.groups == 1 && p.dstate <= kMaxN && p.conv_width == 0 && !p.zoh;
+bool bwd_pairs_supported(const BwdParams &p, bool bf16) {
+    const long long es = bf16 ? 2 : 4;
+    return p.groups == 1 && p.dstate <= kMaxN && p.conv_width == 0 && !p.zoh &&
+           (p.dim * es) % 16 == 0 && (p.seqlen * p.dstate * es) % 16 == 0 &&
+           aligned16(p.x) && aligned16(p.delta) && aligned16(p.z) && aligned16(p.dy) &&
+           aligned16(p.B) && aligned16(p.C) && aligned16(p.dx) && aligned16(p.ddelta) &&
+           aligned16(p.dz) && aligned16(p.ckpt);
 }
 
 cudaError_t launch_scan_bwd_pairs(const BwdParams &p, bool bf16, cudaStream_t stream) {

@@ -73,6 +73,24 @@ def test_small_every_element(dtype, shape, gate):
     _compare_all(g, _oracle_bwd(inp, dy, df), dtype, f"{shape}")
 
 
+# Shapes whose rows are whole 16-byte chunks in both dtypes, so the two-lane
+# kernel takes them: ragged last tiles, channel tiles with one warp partly or
+# wholly past the channels, fewer than 16 states.
+PAIR_SHAPES = [(2, 37, 48, 16), (2, 61, 24, 16), (1, 46, 40, 4), (3, 9, 8, 8), (1, 8, 64, 16)]
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("shape", PAIR_SHAPES, ids=str)
+@pytest.mark.parametrize("gate", [True, False])
+@pytest.mark.parametrize("structured", [True, False])
+def test_chunked_rows_every_element(dtype, shape, gate, structured):
+    inp, dy, df = _inputs(*shape, dtype, gate, seed=41, structured=structured)
+    g = _gpu_bwd(inp, dy, df)
+    torch.cuda.synchronize()
+    _compare_all(g, _oracle_bwd(inp, dy, df), dtype,
+                 f"{shape} {dtype} gate={gate} structured={structured}")
+
+
 @pytest.mark.parametrize("structured", [True, False])
 @pytest.mark.parametrize("softplus", [True, False])
 def test_variants(structured, softplus):
@@ -96,8 +114,9 @@ def test_medium_130m_shape():
     _compare_all(g, _oracle_bwd(inp, dy, df), "bf16", "130m-shaped")
 
 
-def test_deterministic():
-    inp, dy, df = _inputs(2, 200, 100, 16, "bf16", True, seed=12)
+@pytest.mark.parametrize("dim", [100, 96])
+def test_deterministic(dim):
+    inp, dy, df = _inputs(2, 200, dim, 16, "bf16", True, seed=12)
     g1 = _gpu_bwd(inp, dy, df)
     g2 = _gpu_bwd(inp, dy, df)
     torch.cuda.synchronize()
@@ -192,12 +211,14 @@ def test_workspace_too_small_is_rejected():
 
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
-def test_initial_state_gradient(dtype):
+@pytest.mark.parametrize("dim", [70, 48])
+def test_initial_state_gradient(dtype, dim):
     """The gradient of the scan started from a given state: every gradient,
-    the initial state's included, against the oracle."""
-    inp, dy, df = _inputs(2, 90, 70, 16, dtype, True, seed=17)
+    the initial state's included, against the oracle (70 channels: rows that
+    are not whole 16-byte chunks; 48: the two-lane kernel)."""
+    inp, dy, df = _inputs(2, 90, dim, 16, dtype, True, seed=17)
     g = torch.Generator().manual_seed(18)
-    h0 = torch.randn(2, 70, 16, generator=g)
+    h0 = torch.randn(2, dim, 16, generator=g)
     d = {k: (None if v is None else v.to(DEV)) for k, v in inp.items()}
     got = ss.selscan_bwd(d["x"], d["delta"], d["A"], d["B"], d["C"], d["D"], d["z"],
                          d["delta_bias"], dy=dy.to(DEV), dfinal_state=df.to(DEV),
