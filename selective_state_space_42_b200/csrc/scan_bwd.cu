@@ -565,27 +565,46 @@ __global__ void bwd_groups_finish_kernel(const BwdParams p) {
 }
 
 // dB[b, t, n] and dC[b, t, n]: sums of the channel-tile partials (one
-// thread per (batch row, token, value, state group)).
+// thread per (batch row, token, four consecutive stored values, state
+// group); 16-byte loads). Stored value e of a row holds dB (c = 0) or dC
+// (c = 1) of state n: e = 16·c + n, or with part_lane_order
+// e = 4·(4c + 2·(n & 1) + n / 8) + (n / 2) % 4.
 __global__ void bwd_reduce_bc_kernel(const BwdParams p) {
     const long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-    const long long per = p.batch * p.seqlen * kVals;
+    constexpr int kQuads = kVals / 4;
+    const long long per = p.batch * p.seqlen * kQuads;
     if (e >= per * p.groups) return;
     const int g = (int)(e / per);
     const long long eg = e - g * per;
-    const long long b = eg / (p.seqlen * kVals);
-    const long long rest = eg - b * p.seqlen * kVals;  // tok * 32 + v
-    const int v = (int)(rest % kVals);
-    const long long tok = rest / kVals;
-    const int n = 16 * g + v % kMaxN;
-    if (n >= p.dstate) return;
-    const int m = v % kMaxN;
-    const int pv = p.part_lane_order ? 4 * (4 * (v / kMaxN) + 2 * (m & 1) + m / 8) + (m / 2) % 4 : v;
-    const float *src = p.part + ((long long)g * p.batch * p.ctiles + b * p.ctiles) * p.seqlen * kVals +
-                       tok * kVals + pv;
-    float sum = 0.f;
-    for (int c = 0; c < p.ctiles; ++c) sum += src[(long long)c * p.seqlen * kVals];
-    float *dst = v < kMaxN ? p.dB : p.dC;
-    dst[(b * p.seqlen + tok) * p.dstate + n] = sum;
+    const long long b = eg / (p.seqlen * kQuads);
+    const long long rest = eg - b * p.seqlen * kQuads;  // tok * 8 + f
+    const int f = (int)(rest % kQuads);
+    const long long tok = rest / kQuads;
+    const float4 *src = reinterpret_cast<const float4 *>(
+                            p.part + ((long long)g * p.batch * p.ctiles + b * p.ctiles) * p.seqlen * kVals) +
+                        rest;
+    float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int c = 0; c < p.ctiles; ++c) {
+        const float4 v = src[(long long)c * p.seqlen * kQuads];
+        sum.x += v.x;
+        sum.y += v.y;
+        sum.z += v.z;
+        sum.w += v.w;
+    }
+    const float s[4] = {sum.x, sum.y, sum.z, sum.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        int isC, m;
+        if (p.part_lane_order) {
+            isC = f >> 2;
+            m = 8 * (f & 1) + 2 * i + ((f >> 1) & 1);
+        } else {
+            isC = (4 * f + i) / kMaxN;
+            m = (4 * f + i) % kMaxN;
+        }
+        const int n = 16 * g + m;
+        if (n < p.dstate) (isC ? p.dC : p.dB)[(b * p.seqlen + tok) * p.dstate + n] = s[i];
+    }
 }
 
 // dA[d, n], dD[d], ddelta_bias[d]: sums over batch rows.
@@ -748,7 +767,7 @@ cudaError_t launch_scan_bwd(const BwdParams &params, bool bf16, cudaStream_t str
     else
         e = p.z ? launch_gate<float, true>(p, stream) : launch_gate<float, false>(p, stream);
     if (e != cudaSuccess) return e;
-    const long long nbc = p.batch * p.seqlen * kVals * p.groups;
+    const long long nbc = p.batch * p.seqlen * (kVals / 4) * p.groups;
     bwd_reduce_bc_kernel<<<(unsigned)((nbc + 255) / 256), 256, 0, stream>>>(p);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
