@@ -344,7 +344,7 @@ def time_calls(torch, stream, fn, n, flush=None):
 def extra_legs(args, torch, ss, wl, dev, stream, peak, over_ranks):
     """Other workloads of the path, timed the same way (not part of the
     headline metric): the other scan shapes, the general-A and ZOH variants
-    of the headline shape, the decode step and the SSD layer."""
+    of the headline shape, its gradient, the decode step and the SSD layer."""
     flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
     out = {}
 
@@ -378,6 +378,30 @@ def extra_legs(args, torch, ss, wl, dev, stream, peak, over_ranks):
     out["general_A"]["A"] = "-exp(log(n+1)) in float32 (not bit-exactly (n+1)*A[d,0]: general decay)"
     out["zoh"], _ = scan_leg("mamba2p8b_layer", 50, bbar="zoh", ref_ms=ref)
     out["zoh"]["input_term"] = "(exp(delta*A)-1)/A*B*x"
+
+    # the gradient of the headline shape (dy and a final-state gradient in;
+    # dx, ddelta, dz, dA, dB, dC, dD, ddelta_bias out)
+    gw = wl.WORKLOADS["mamba2p8b_layer"]
+    ginp = wl.make_scan_inputs(gw, device=dev)
+    gg = torch.Generator(device=dev)
+    gg.manual_seed(gw.seed + 1000)
+    gdy = torch.randn(gw.batch, gw.seqlen, gw.dim, generator=gg, device=dev).to(ginp["x"].dtype)
+    gdf = torch.randn(gw.batch, gw.dim, gw.dstate, generator=gg, device=dev)
+
+    def grad_call():
+        ss.selscan_bwd(ginp["x"], ginp["delta"], ginp["A"], ginp["B"], ginp["C"], ginp["D"],
+                       ginp["z"], ginp["delta_bias"], softplus=True, dy=gdy, dfinal_state=gdf,
+                       stream=stream)
+    b2b, cold = time_calls(torch, stream, grad_call, 10, flush)
+    b2b, cold = over_ranks(b2b), over_ranks(cold)
+    gnb = gw.backward_algorithmic_bytes()
+    out["gradient"] = {
+        "workload": gw.name, "bytes_per_call": gnb, "elements_per_call": gw.elements,
+        "us_back_to_back": b2b * 1e3, "us_after_l2_flush": cold * 1e3,
+        "GBps_back_to_back": gnb / b2b / 1e6, "frac_back_to_back": gnb / b2b / 1e6 / peak,
+        "time_vs_headline_shape": b2b / ref,
+        "kernels": "scan_bwd_pairs_kernel + bwd_reduce_bc_kernel + bwd_reduce_params_kernel"}
+    del ginp, gdy, gdf
 
     # the decode step (one token in place on the [256, 5120, 16] state); the
     # after-flush time is the headline: back to back the 84 MB state stays in L2
