@@ -141,6 +141,24 @@ def test_ssd_options(dtype):
     gh.compare(gh.to_np(h2), ho2, gh.RTOL[dtype], "no softplus, D, bias final state")
 
 
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_ssd_steep_decay_heads(dtype):
+    """Heads whose decay over a 128-token chunk leaves the float32 range of
+    2^(Acum_i − Acum_j) factored as 2^Acum_i · 2^(−Acum_j) (|A|·Δ large) next
+    to heads where it does not: the per-element decay path and the factored
+    one in the same calls, with an initial state so that C·h_in counts."""
+    inp = _inputs(2, 300, 5, 64, 128, dtype, seed=7700)
+    inp["A"] = torch.tensor([-0.5, -30.0, -1.0, -40.0, -12.0])
+    inp["dt_bias"] = torch.zeros(5)
+    g = torch.Generator().manual_seed(7701)
+    h0 = torch.randn(2, 5 * 64, 128, generator=g) * 0.3
+    y, hf = _gpu(inp, h0.to(DEV))
+    torch.cuda.synchronize()
+    yo, ho = _oracle(inp, 64, h0)
+    gh.compare(gh.to_np(y), yo, gh.RTOL[dtype], "steep decay y")
+    gh.compare(gh.to_np(hf), ho, gh.RTOL[dtype], "steep decay final state")
+
+
 @pytest.mark.parametrize("L", [127, 128, 129, 256, 257])
 def test_ssd_chunk_edges(L):
     """Sequence lengths at the 128-token chunk edges of the tensor-core path
