@@ -111,6 +111,24 @@ __device__ __forceinline__ void decay8(float dt, float r, bool odd, const float2
     }
 }
 
+// Δ = softplus(v) and its derivative σ(v). bfloat16 I/O: from one MUFU pair,
+// q = 1 + 2^(v·log2 e): Δ = log2(q)·ln 2 and σ = 2^(v·log2 e)/q (v and 1 above
+// v = 15); absolute error ~1e-7 of Δ, as in the forward kernel for bfloat16
+// I/O. float32 I/O: the accurate softplus and sigmoid.
+template <typename T>
+__device__ __forceinline__ void softplus_sigma(float v, float &dt, float &sg) {
+    if (sizeof(T) == 2) {
+        const float e = ex2_approx(v * kLog2e);
+        const float q = 1.0f + e;
+        const bool big = v > 15.0f;
+        dt = big ? v : lg2_approx(q) * kLn2;
+        sg = big ? 1.0f : e * rcp_approx(q);
+    } else {
+        dt = softplus_f32(v);
+        sg = sigmoid_f32(v);
+    }
+}
+
 // Where a tile's rows are.
 struct TileGeo {
     long long row0;  // batch row · seqlen + first token of the tile
@@ -270,12 +288,14 @@ __device__ __forceinline__ void bwd_pairs_body(WarpSmem<T> *S, const BwdParams &
             cp_async_wait_all();
             __syncwarp();
             convert_bc(W, N, lane, false);
+            const int nvalid = active ? (int)min((long long)kSeg, p.seqlen - t0) : 0;
 #pragma unroll
             for (int j = 0; j < kOwn; ++j) {
                 const int t = 2 * j + par;
                 const float v = to_f32(W.raw[1][t][cl]) + bias;
-                const bool live = active && t0 + t < p.seqlen;
-                const float dt = live ? (kSoftplus ? softplus_f32(v) : v) : 0.0f;
+                float dt = v, sg;
+                if (kSoftplus) softplus_sigma<T>(v, dt, sg);
+                dt = t < nvalid ? dt : 0.0f;
                 W.sc[t][cl] = make_float4(dt, dt * to_f32(W.raw[0][t][cl]), 0.0f,
                                           ex2_approx(dt * A0l));
             }
@@ -327,13 +347,15 @@ __device__ __forceinline__ void bwd_pairs_body(WarpSmem<T> *S, const BwdParams &
         // owned tokens' scalars; x, dy·silu'(z) and σ stay in registers for
         // the tile's epilogue
         float xo[kOwn], dyso[kOwn], sgo[kOwn];
+        const int nvalid = active ? (int)min((long long)kSeg, p.seqlen - t0) : 0;
 #pragma unroll
         for (int j = 0; j < kOwn; ++j) {
             const int t = 2 * j + par;
-            const bool live = active && t0 + t < p.seqlen;
             const float xv = to_f32(W.raw[0][t][cl]);
             const float v = to_f32(W.raw[1][t][cl]) + bias;
-            const float dt = live ? (kSoftplus ? softplus_f32(v) : v) : 0.0f;
+            float dt = v, sg = 1.0f;
+            if (kSoftplus) softplus_sigma<T>(v, dt, sg);
+            dt = t < nvalid ? dt : 0.0f;
             const float dyv = to_f32(W.raw[3][t][cl]);
             float ds = dyv, dysz = 0.f;
             if (kGate) {
@@ -344,7 +366,7 @@ __device__ __forceinline__ void bwd_pairs_body(WarpSmem<T> *S, const BwdParams &
             }
             xo[j] = xv;
             dyso[j] = dysz;
-            sgo[j] = kSoftplus ? sigmoid_f32(v) : 1.0f;
+            sgo[j] = sg;
             W.sc[t][cl] = make_float4(dt, dt * xv, ds, ex2_approx(dt * A0l));
         }
         __syncwarp();
@@ -451,7 +473,7 @@ __device__ __forceinline__ void bwd_pairs_body(WarpSmem<T> *S, const BwdParams &
                 out[(1 * kSeg + t) * kCh + cl] = from_f32<T>(dv);
                 if (kGate)
                     out[(2 * kSeg + t) * kCh + cl] = from_f32<T>(fmaf(Dv, xo[j], sv[j]) * dyso[j]);
-                if (active && t0 + t < p.seqlen) {
+                if (t < nvalid) {
                     accD = fmaf(sc[j].z, xo[j], accD);
                     accBias += dv;
                 }
