@@ -811,7 +811,7 @@ ssd_tc_out_kernel(const SsdParams p, const __grid_constant__ CUtensorMap tm_b,
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
                 float v = fmaf(dec, yo[8 * k8 + e], yd[8 * k8 + e]) + dsk * xv[e];
-                if (kGate) v *= silu_f32(zv[e]);
+                if (kGate) v *= silu_tanh(zv[e]);  // one MUFU op; bfloat16 output
                 o[e] = v;
             }
             if (p.vec_x && c0 + 8 <= P) {
