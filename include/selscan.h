@@ -184,9 +184,10 @@ typedef struct {
 
 /*
  * selscan_fwd_ex -- selscan_fwd with every option: an initial state, the
- * causal conv in front, and the input term. The zero-order-hold term runs on
- * the generic (non-TMA) kernels, which also serve every shape the TMA kernel
- * cannot take. options NULL: selscan_fwd. Unknown bbar_mode: SELSCAN_ERR_BAD_DIM.
+ * causal conv in front, and the input term (Δ·B·x or the zero-order-hold
+ * term, both on the TMA-staged kernel where the shape allows it, else on the
+ * generic kernels). options NULL: selscan_fwd. Unknown bbar_mode:
+ * SELSCAN_ERR_BAD_DIM.
  */
 SELSCAN_API int selscan_fwd_ex(const void *x, const void *delta, const float *A,
                                const void *B, const void *C, const float *D, const void *z,
