@@ -42,7 +42,7 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["selscan", "reference"], default="selscan")
     ap.add_argument("--workload", default=WORKLOAD)
-    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--e2e-steps", type=int, default=8)
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="target duration of the oracle CPU-baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -516,21 +516,45 @@ def main():
     args.headline_ms = ms / args.steps
 
     # end to end through the public call: pinned host inputs -> device ->
-    # selscan_fwd -> y and final state back to pinned host memory, every step
+    # selscan_fwd -> y and final state back to pinned host memory, every
+    # step. Two buffer sets on three streams, as a streaming caller would run
+    # it: step i + 1's inputs go up while step i computes and step i − 1's
+    # outputs come down (PCIe carries both directions at once).
     names = ["x", "delta", "z", "B", "C"]
     host = {k: inp[k].to("cpu").pin_memory() for k in names}
-    y_h = torch.empty(y.shape, dtype=y.dtype, pin_memory=True)
-    fs_h = torch.empty(fs.shape, dtype=fs.dtype, pin_memory=True)
-    dbuf = {k: torch.empty_like(inp[k]) for k in names}
+    nbuf = 2
+    y_h = [torch.empty(y.shape, dtype=y.dtype, pin_memory=True) for _ in range(nbuf)]
+    fs_h = [torch.empty(fs.shape, dtype=fs.dtype, pin_memory=True) for _ in range(nbuf)]
+    dbuf = [{k: torch.empty_like(inp[k]) for k in names} for _ in range(nbuf)]
+    ybuf = [y, torch.empty_like(y)]
+    fsbuf = [fs, torch.empty_like(fs)]
+    s_up, s_down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    up_done = [torch.cuda.Event() for _ in range(nbuf)]
+    comp_done = [torch.cuda.Event() for _ in range(nbuf)]
+    down_done = [torch.cuda.Event() for _ in range(nbuf)]
+    for e in comp_done + down_done:
+        e.record(stream)
+    k_step = [0]
 
     def e2e_step():
-        for k in names:
-            dbuf[k].copy_(host[k], non_blocking=True)
-        ss.selscan_fwd(dbuf["x"], dbuf["delta"], inp["A"], dbuf["B"], dbuf["C"],
-                       inp["D"], dbuf["z"], inp["delta_bias"], softplus=True, y=y,
-                       final_state=fs, stream=stream)
-        y_h.copy_(y, non_blocking=True)
-        fs_h.copy_(fs, non_blocking=True)
+        j = k_step[0] % nbuf
+        k_step[0] += 1
+        s_up.wait_event(comp_done[j])      # the last call that read this input set is done
+        with torch.cuda.stream(s_up):
+            for k in names:
+                dbuf[j][k].copy_(host[k], non_blocking=True)
+            up_done[j].record(s_up)
+        stream.wait_event(up_done[j])
+        stream.wait_event(down_done[j])    # this y / final-state set has been read back
+        ss.selscan_fwd(dbuf[j]["x"], dbuf[j]["delta"], inp["A"], dbuf[j]["B"], dbuf[j]["C"],
+                       inp["D"], dbuf[j]["z"], inp["delta_bias"], softplus=True, y=ybuf[j],
+                       final_state=fsbuf[j], stream=stream)
+        comp_done[j].record(stream)
+        s_down.wait_event(comp_done[j])
+        with torch.cuda.stream(s_down):
+            y_h[j].copy_(ybuf[j], non_blocking=True)
+            fs_h[j].copy_(fsbuf[j], non_blocking=True)
+            down_done[j].record(s_down)
 
     e2e_step()
     torch.cuda.synchronize(dev)
@@ -538,14 +562,18 @@ def main():
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
+    s_up.wait_event(e0)
+    s_down.wait_event(e0)
     for _ in range(args.e2e_steps):
         e2e_step()
+    stream.wait_stream(s_down)
+    stream.wait_stream(s_up)
     e1.record(stream)
     torch.cuda.synchronize(dev)
     barrier()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), dist if world > 1 else None, dev)
     h2d = sum(host[k].numel() * host[k].element_size() for k in names)
-    d2h = y_h.numel() * y_h.element_size() + fs_h.numel() * fs_h.element_size()
+    d2h = y_h[0].numel() * y_h[0].element_size() + fs_h[0].numel() * fs_h[0].element_size()
 
     peak, peak_kind = peaks()
     legs = extra_legs(args, torch, ss, wl, dev, stream, peak,
