@@ -48,6 +48,12 @@ int sm_count() {
     return sms;
 }
 
+// A set, non-"0" environment variable (tuning and testing switches).
+bool env_flag(const char *name) {
+    const char *v = getenv(name);
+    return v && *v && strcmp(v, "0") != 0;
+}
+
 int64_t env_int(const char *name) {
     const char *v = getenv(name);
     return (v && *v) ? atoll(v) : 0;
@@ -341,7 +347,7 @@ cudaError_t fwd_run(FwdPlan *plan, void *ws, cudaStream_t stream) {
 namespace {
 
 struct BwdLayout {
-    size_t ckpt, part, pA, pD, pbias, dxc, pconv, acc, total;
+    size_t ckpt, part, pA, pD, pbias, dxc, pconv, acc, tma, tma_bytes, total;
 };
 
 // 16-state groups the gradient walks per chain
@@ -379,6 +385,16 @@ BwdLayout bwd_layout(int64_t batch, int64_t seqlen, int64_t dim, int64_t dstate,
     }
     l.acc = off;
     if (G > 1) off = align256(off + 3 * (size_t)(G * batch * seqlen * dim) * sizeof(float));
+    // the one-pass TMA plan's counters, flags and handed-over states, for the
+    // checkpoint pass of the forward kernel (one 16-state group, no conv)
+    l.tma = off;
+    l.tma_bytes = 0;
+    if (G == 1 && !conv && dim >= selscan::tma_tile_channels()) {
+        const int64_t groups = batch * ceil_div64(dim, selscan::tma_tile_channels());
+        l.tma_bytes = align256(256 + 4 * 8 * (size_t)groups) +
+                      (size_t)groups * selscan::tma_tile_channels() * selscan::kMaxN * sizeof(float);
+        off = align256(off + l.tma_bytes);
+    }
     l.total = off;
     return l;
 }
@@ -653,7 +669,44 @@ int bwd_entry(const void *x, const void *delta, const float *A, const void *B, c
     p.acc = p.groups > 1 ? reinterpret_cast<float *>(w + l.acc) : nullptr;
     p.dxc = conv_width > 0 ? reinterpret_cast<float *>(w + l.dxc) : nullptr;
     p.pconv = conv_width > 0 ? reinterpret_cast<float *>(w + l.pconv) : nullptr;
-    e = selscan::launch_scan_bwd(p, dtype == SELSCAN_BF16, stream);
+    // With the two-lane gradient kernel and the forward's one-pass TMA plan
+    // both available, the TMA-staged forward kernel writes the checkpoints
+    // (no y) and the gradient kernel skips its own forward sweep.
+    const bool bf16 = dtype == SELSCAN_BF16;
+    if (l.tma_bytes > 0 && selscan::bwd_pairs_supported(p, bf16) &&
+        !env_flag("SELSCAN_BWD_OWN_SWEEP")) {
+        const bool aligned = !misaligned(x, 16) && !misaligned(delta, 16) &&
+                             !misaligned(B, 16) && !misaligned(C, 16);
+        selscan::FwdPlan fp{};
+        selscan::plan_for_sizes(batch, seqlen, dim, dstate, dtype, aligned, &fp);
+        if (fp.tma && fp.tp.mode == selscan::kModeSeq && fp.ws_bytes <= l.tma_bytes) {
+            selscan::TmaScanParams t = fp.tp;
+            t.B = B; t.C = C; t.A = A; t.Dskip = D; t.delta_bias = delta_bias;
+            t.y = nullptr; t.final_state = nullptr; t.h0 = h0;
+            t.conv_w = t.conv_b = t.conv_init = nullptr;
+            t.conv_width = 0;
+            t.zoh = 0;
+            t.batch = batch; t.seqlen = seqlen; t.dim = dim; t.dstate = (int)dstate;
+            t.softplus = p.softplus;
+            t.mode = selscan::kModeCkpt;
+            t.ckpt = p.ckpt;
+            t.ck_tiles = p.ktiles;
+            char *tw = w + l.tma;
+            e = cudaMemsetAsync(tw, 0, fp.ws_clear, stream);
+            int *tickets = reinterpret_cast<int *>(tw);
+            t.ticket = tickets;
+            t.abort_all = tickets + 2;
+            t.flags = reinterpret_cast<int *>(tw + 256);
+            t.ws_state = reinterpret_cast<float *>(tw + fp.ws_clear);
+            t.units = (int)(t.groups * t.nchunks);
+            if (e == cudaSuccess) e = selscan::launch_scan_tma(t, bf16, x, delta, nullptr, stream);
+            p.ckpt_ready = e == cudaSuccess ? 1 : 0;
+            // a tensor map the driver refused: nothing launched, the gradient
+            // kernel does its own forward sweep
+            if (e == cudaErrorInvalidValue) e = cudaSuccess;
+        }
+    }
+    if (e == cudaSuccess) e = selscan::launch_scan_bwd(p, bf16, stream);
     if (allocate) {
         cudaError_t ef = cudaFreeAsync(ws, stream);
         if (e == cudaSuccess) e = ef;

@@ -26,6 +26,8 @@ struct BwdParams {
                    // of dB (0..15), dC (16..31) of the group's states; with part_lane_order
                    // value 16·c + n (c = 1 for dC) sits at 4·(4c + 2·(n & 1) + n / 8) + (n / 2) % 4
     int part_lane_order;  // set by launch_scan_bwd for the kernel it runs
+    int ckpt_ready;       // ckpt already holds every tile's entering state (the two-lane
+                          // kernel then skips its forward sweep)
     float *pA;     // [groups][batch][dim][16]: Σ over tokens of dA
     float *acc;    // groups > 1: [groups][3][batch][seqlen][dim] float32: each group's part of
                    // dΔ (before the softplus derivative), dx and the pre-gate output

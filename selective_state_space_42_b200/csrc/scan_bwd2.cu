@@ -272,8 +272,8 @@ __device__ __forceinline__ void bwd_pairs_body(WarpSmem<T> *S, const BwdParams &
         return g;
     };
 
-    // ---- 1. forward sweep: checkpoints ------------------------------------------
-    {
+    // ---- 1. forward sweep: checkpoints (unless given) ----------------------------
+    if (!p.ckpt_ready) {
         float2 h[kPairs];
 #pragma unroll
         for (int q = 0; q < kPairs; ++q) {

@@ -471,6 +471,7 @@ struct Scal {
     float r1[kOwn];  // structured: r = 2^(Δ/ln 2 · A[d, 0])
     float dx[kOwn];  // D·x
     float zg[kOwn];  // silu(z), or 1 without a gate
+    float up;        // structured: u of the token before the sub-tile (after link_prev)
 };
 
 template <typename T, bool kGate, int kMode, bool kStruct, bool kSoftplus, bool kFull,
@@ -544,6 +545,7 @@ __device__ __forceinline__ void token_scalars(const Stage<T, kConv> &st, int sub
 __device__ __forceinline__ void link_prev(Scal &S, bool odd, float &ulast) {
     const float send = odd ? ulast : S.uu[kOwn - 1];
     const float prev = __shfl_xor_sync(0xffffffffu, send, 16);
+    S.up = odd ? ulast : prev;  // both lanes: u of the token before the sub-tile
     ulast = S.uu[kOwn - 1];
     S.rr[0] *= prev;
 #pragma unroll
@@ -616,7 +618,7 @@ __device__ __forceinline__ void recurrence(const Stage<T, kConv> &st, int sub, i
 #pragma unroll
             for (int q = 0; q < kHalf / 2; ++q) run.h[q] = fma2(a[q], run.h[q], bu[q]);
         }
-        if (kMode != kModeAgg) {
+        if (kMode != kModeAgg && kMode != kModeCkpt) {
             const float4 *C4 = reinterpret_cast<const float4 *>(&st.C[t][odd ? kHalf : 0]);
             const float4 c0 = C4[0], c1 = C4[1];
             float2 yv = mul2(make_float2(c0.x, c0.y), run.h[0]);
@@ -654,6 +656,18 @@ __device__ __forceinline__ void write_y(const Scal &S, const float (&part)[kSub]
     }
 }
 
+// kModeCkpt: the state entering sub-tile `sub`, this lane's 8 states, to the
+// gradient's checkpoint row of that 8-token tile. run.h is h/ln 2, in the
+// structured form also divided by the u of the token before the sub-tile.
+template <bool kStruct>
+__device__ __forceinline__ void store_ckpt(const Run &run, float up, float4 *ckp,
+                                           long long ckstride, int sub) {
+    const float sc = kLn2 * (kStruct ? up : 1.0f);
+    float4 *dst = ckp + (long long)(sub / kSub) * ckstride;
+    dst[0] = make_float4(run.h[0].x * sc, run.h[0].y * sc, run.h[1].x * sc, run.h[1].y * sc);
+    dst[1] = make_float4(run.h[2].x * sc, run.h[2].y * sc, run.h[3].x * sc, run.h[3].y * sc);
+}
+
 // One ring stage for this lane. kFull: the stage holds kTile valid tokens and
 // y goes to this warp's shared-memory tile `ys` (written to global memory by
 // one TMA store per warp); the sub-tiles are software-pipelined (the scalars
@@ -665,8 +679,10 @@ template <typename T, bool kGate, int kMode, bool kStruct, bool kSoftplus, bool 
 __device__ __forceinline__ void consume_tile(const Stage<T, kConv> &st, int nt, Run &run,
                                              const Chain &ch, const Offs &o, bool seq_start,
                                              const float *conv_init, T *ys, T *yp,
-                                             long long ybase, long long ystride, bool active) {
+                                             long long ybase, long long ystride, bool active,
+                                             float4 *ckp, long long ckstride) {
     constexpr int kTile = TileCfg<T>::kTile;
+    constexpr bool kCk = kMode == kModeCkpt;
     const bool odd = threadIdx.x & 16;
     if constexpr (kFull) {
         Scal S;
@@ -681,15 +697,17 @@ __device__ __forceinline__ void consume_tile(const Stage<T, kConv> &st, int nt, 
             token_scalars<T, kGate, kMode, kStruct, kSoftplus, true, kConv>(
                 st, sub + kSub, nt, ch, o, seq_start, conv_init, active, run, N);
             if (kStruct) link_prev(N, odd, run.ulast);
+            if (kCk && ckp) store_ckpt<kStruct>(run, S.up, ckp, ckstride, sub);
             recurrence<T, kMode, kStruct, true, kConv, kZoh>(st, sub, nt, P0, P1, ch, run, part);
-            if (kMode != kModeAgg)
+            if (kMode != kModeAgg && !kCk)
                 write_y<T, kStruct, true>(S, part, sub, nt, o, ys, yp, ybase, ystride, active);
             S = N;
         }
         float P0[kSub], P1[kSub], part[kSub];
         broadcast<kStruct>(S, P0, P1);
+        if (kCk && ckp) store_ckpt<kStruct>(run, S.up, ckp, ckstride, kTile - kSub);
         recurrence<T, kMode, kStruct, true, kConv, kZoh>(st, kTile - kSub, nt, P0, P1, ch, run, part);
-        if (kMode != kModeAgg)
+        if (kMode != kModeAgg && !kCk)
             write_y<T, kStruct, true>(S, part, kTile - kSub, nt, o, ys, yp, ybase, ystride,
                                       active);
     } else {
@@ -701,6 +719,7 @@ __device__ __forceinline__ void consume_tile(const Stage<T, kConv> &st, int nt, 
             if (kStruct) link_prev(S, odd, run.ulast);
             float P0[kSub], P1[kSub], part[kSub];
             broadcast<kStruct>(S, P0, P1);
+            if (kCk && ckp) store_ckpt<kStruct>(run, S.up, ckp, ckstride, sub);
             recurrence<T, kMode, kStruct, false, kConv, kZoh>(st, sub, nt, P0, P1, ch, run, part);
             // u of the sequence's last token (a partial tile ends the
             // sequence), for the state handed out of the unit
@@ -713,7 +732,7 @@ __device__ __forceinline__ void consume_tile(const Stage<T, kConv> &st, int nt, 
                     if (sub + hsub + j < nt) us = S.uu[j];
                 run.uend = __shfl_sync(0xffffffffu, us, (threadIdx.x & 15) + 16 * (tl / kOwn));
             }
-            if (kMode != kModeAgg)
+            if (kMode != kModeAgg && !kCk)
                 write_y<T, kStruct, false>(S, part, sub, nt, o, ys, yp, ybase, ystride, active);
         }
     }
@@ -795,7 +814,7 @@ __device__ void consume(Shared<T, kConv> &S, const TmaScanParams &p, const CUten
             float hs[kHalf];
 #pragma unroll
             for (int i = 0; i < kHalf; ++i) hs[i] = 0.0f;
-            if (kMode == kModeSeq && inf.chunk > 0) {
+            if ((kMode == kModeSeq || kMode == kModeCkpt) && inf.chunk > 0) {
                 // every lane acquires this warp's predecessor flag (bounded)
                 const int *flag = p.flags + g * kMaxConsumerWarps + warp;
                 const uint64_t start = global_ns();
@@ -815,7 +834,7 @@ __device__ void consume(Shared<T, kConv> &S, const TmaScanParams &p, const CUten
                     hs[0] = v0.x; hs[1] = v0.y; hs[2] = v0.z; hs[3] = v0.w;
                     hs[4] = v1.x; hs[5] = v1.y; hs[6] = v1.z; hs[7] = v1.w;
                 }
-            } else if (kMode == kModeSeq && p.h0 && active) {
+            } else if ((kMode == kModeSeq || kMode == kModeCkpt) && p.h0 && active) {
                 const float *src = p.h0 + (inf.b * p.dim + d) * p.dstate;
 #pragma unroll
                 for (int i = 0; i < kHalf; ++i) {
@@ -838,20 +857,28 @@ __device__ void consume(Shared<T, kConv> &S, const TmaScanParams &p, const CUten
         const float *cinit = (kConv && p.conv_init && active)
                                  ? p.conv_init + (inf.b * p.dim + d) * kHalo
                                  : nullptr;
+        // kModeCkpt: this lane's checkpoint slots of the tile's first 8 tokens
+        float4 *ckp = nullptr;
+        const long long ckstride = p.dim * 4;  // float4s between consecutive 8-token tiles
+        if (kMode == kModeCkpt && active)
+            ckp = reinterpret_cast<float4 *>(p.ckpt) +
+                  ((inf.b * p.ck_tiles + inf.t0 / kSub) * p.dim + d) * 4 + (odd ? 2 : 0);
         if (inf.nt == kTile) {
             T *ys = S.ybuf[warp][kbuf];
-            if (kMode != kModeAgg) {
+            if (kMode != kModeAgg && kMode != kModeCkpt) {
                 // the store that last read this staging tile has finished with it
                 if (lane == 0) bulk_wait_read<kYBufs - 1>();
                 __syncwarp();
             }
             if (!kZoh && structured)
                 consume_tile<T, kGate, kMode, true, kSoftplus, true, kConv, false>(
-                    S.stage[s], inf.nt, run, ch, offs, seq_start, cinit, ys, yp, ybase, p.dim, active);
+                    S.stage[s], inf.nt, run, ch, offs, seq_start, cinit, ys, yp, ybase, p.dim, active,
+                    ckp, ckstride);
             else
                 consume_tile<T, kGate, kMode, false, kSoftplus, true, kConv, kZoh>(
-                    S.stage[s], inf.nt, run, ch, offs, seq_start, cinit, ys, yp, ybase, p.dim, active);
-            if (kMode != kModeAgg) {
+                    S.stage[s], inf.nt, run, ch, offs, seq_start, cinit, ys, yp, ybase, p.dim, active,
+                    ckp, ckstride);
+            if (kMode != kModeAgg && kMode != kModeCkpt) {
                 fence_proxy_async_smem();
                 __syncwarp();
                 const int c0 = inf.tile * kChannels + warp * kWarpChannels;
@@ -865,11 +892,11 @@ __device__ void consume(Shared<T, kConv> &S, const TmaScanParams &p, const CUten
             if (!kZoh && structured)
                 consume_tile<T, kGate, kMode, true, kSoftplus, false, kConv, false>(
                     S.stage[s], inf.nt, run, ch, offs, seq_start, cinit, nullptr, yp, ybase, p.dim,
-                    active);
+                    active, ckp, ckstride);
             else
                 consume_tile<T, kGate, kMode, false, kSoftplus, false, kConv, kZoh>(
                     S.stage[s], inf.nt, run, ch, offs, seq_start, cinit, nullptr, yp, ybase, p.dim,
-                    active);
+                    active, ckp, ckstride);
         }
 
         if (inf.flags & kLast) {
@@ -905,7 +932,7 @@ __device__ void consume(Shared<T, kConv> &S, const TmaScanParams &p, const CUten
                         if (n < p.dstate) fs[n] = hf[i];
                     }
                 }
-            } else if (kMode == kModeSeq) {
+            } else if (kMode == kModeSeq || kMode == kModeCkpt) {
                 if (active) {
                     float *dst = p.ws_state + (g * kChannels + c) * kMaxN + (odd ? kHalf : 0);
                     st_cg_f4(dst, make_float4(hf[0], hf[1], hf[2], hf[3]));
@@ -1015,8 +1042,11 @@ cudaError_t launch_mode(const TmaScanParams &p, const void *x, const void *dl, c
                      CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_map<T>(&md, dl, rows, p.dim, kBoxCh, kTile, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_map<T>(&mb, p.B, rows, p.dstate, p.dstate, kTile, CU_TENSOR_MAP_SWIZZLE_NONE) ||
-        !make_map<T>(&mc, p.C, rows, p.dstate, p.dstate, kTile, CU_TENSOR_MAP_SWIZZLE_NONE) ||
-        !make_map<T>(&my, p.y, rows, p.dim, kWarpChannels, kTile, yswz))
+        !make_map<T>(&mc, p.C, rows, p.dstate, p.dstate, kTile, CU_TENSOR_MAP_SWIZZLE_NONE))
+        return cudaErrorInvalidValue;
+    if (kMode == kModeCkpt)
+        my = md;  // no y
+    else if (!make_map<T>(&my, p.y, rows, p.dim, kWarpChannels, kTile, yswz))
         return cudaErrorInvalidValue;
     if (kGate) {
         if (!make_map<T>(&mz, z, rows, p.dim, kBoxCh, kTile, CU_TENSOR_MAP_SWIZZLE_128B))
@@ -1050,6 +1080,11 @@ cudaError_t launch_conv(const TmaScanParams &p, const void *x, const void *dl, c
         return launch_mode<T, kGate, kModeSeq, kSoftplus, kConv, kZoh>(p, x, dl, z, stream);
     case kModeAgg:
         return launch_mode<T, false, kModeAgg, kSoftplus, kConv, kZoh>(p, x, dl, z, stream);
+    case kModeCkpt:  // the gradient's checkpoints: Δ·B·x term, no conv
+        if constexpr (!kConv && !kZoh)
+            return launch_mode<T, false, kModeCkpt, kSoftplus, false, false>(p, x, dl, z, stream);
+        else
+            return cudaErrorInvalidValue;
     default:
         return launch_mode<T, kGate, kModeRescan, kSoftplus, kConv, kZoh>(p, x, dl, z, stream);
     }

@@ -161,7 +161,9 @@ struct StepParams {
 cudaError_t device_status_address(int **p);
 
 // Persistent TMA-staged scan (scan_tma.cu).
-enum : int { kModeSeq = 0, kModeAgg = 1, kModeRescan = 2 };
+// kModeCkpt: the one-pass plan's hand-off without y, writing instead the
+// state entering every 8-token sub-tile (the gradient's checkpoints).
+enum : int { kModeSeq = 0, kModeAgg = 1, kModeRescan = 2, kModeCkpt = 3 };
 
 struct TmaScanParams {
     const void *B, *C;
@@ -192,6 +194,11 @@ struct TmaScanParams {
     unsigned long long timeout_ns;  // bound on every device-side wait
     int skip_release_chunk;  // fault-injection hook for tests: the kSeq units of this
                              // chunk publish no completion flag (-1: none)
+    // kModeCkpt: [batch][ck_tiles][dim][16] float32, per (batch row, 8-token
+    // tile, channel) the lower lane's states 0,2,4,6 | 8,10,12,14 then the upper
+    // lane's 1,3,5,7 | 9,11,13,15 (the gradient kernel's layout)
+    float *ckpt;
+    long long ck_tiles;
 };
 
 cudaError_t launch_scan_tma(const TmaScanParams &p, bool bf16, const void *x, const void *dl,

@@ -178,6 +178,36 @@ def test_bench_shape_sampled_and_identities():
     assert abs(lhs_b - rhs_b) <= 1e-3 * (abs(rhs_b) + abs(lhs_c)), (lhs_b, rhs_b)
 
 
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("structured", [True, False])
+def test_checkpoints_from_the_forward_kernel(dtype, structured, monkeypatch):
+    """The checkpoints written by the TMA-staged forward kernel (its one-pass
+    plan forced on a small shape, ragged last tile, with an initial state)
+    against the oracle, and against the gradient kernel's own forward sweep."""
+    inp, dy, df = _inputs(2, 301, 256, 16, dtype, True, seed=51, structured=structured)
+    g = torch.Generator().manual_seed(52)
+    h0 = torch.randn(2, 256, 16, generator=g)
+    d = {k: (None if v is None else v.to(DEV)) for k, v in inp.items()}
+
+    def run():
+        return ss.selscan_bwd(d["x"], d["delta"], d["A"], d["B"], d["C"], d["D"], d["z"],
+                              d["delta_bias"], dy=dy.to(DEV), dfinal_state=df.to(DEV),
+                              initial_state=h0.to(DEV))
+
+    monkeypatch.setenv("SELSCAN_PATH", "seq")
+    assert ss.selscan_fwd_plan(2, 301, 256, 16)["launches"] == 1  # the one-pass plan
+    got = run()
+    monkeypatch.setenv("SELSCAN_BWD_OWN_SWEEP", "1")
+    own = run()
+    torch.cuda.synchronize()
+    n = gh.to_np
+    o = oracle.default().bwd(n(inp["x"]), n(inp["delta"]), n(inp["A"]), n(inp["B"]), n(inp["C"]),
+                             n(inp["D"]), n(inp["z"]), n(inp["delta_bias"]), h0=n(h0), dy=n(dy),
+                             dfinal=n(df))
+    _compare_all(got, o, dtype, "forward-kernel checkpoints", names=GRADS + ("dh0",))
+    _compare_all(own, o, dtype, "own forward sweep", names=GRADS + ("dh0",))
+
+
 def test_long_sequence_sampled():
     """The 1M-token layer (1 × 1,048,576 × 2048, N = 16, bf16, gated): 131,072
     8-token tiles per chain, checkpoint and partial buffers of several GB;
