@@ -542,10 +542,11 @@ __device__ __forceinline__ void token_scalars(const Stage<T, kConv> &st, int sub
 // before it. For the first owned token that u lives on the other lane: for
 // the lower lane the upper lane's last token of the previous sub-tile
 // (`ulast`, updated here), for the upper lane the lower lane's token 3.
+template <bool kUp = false>
 __device__ __forceinline__ void link_prev(Scal &S, bool odd, float &ulast) {
     const float send = odd ? ulast : S.uu[kOwn - 1];
     const float prev = __shfl_xor_sync(0xffffffffu, send, 16);
-    S.up = odd ? ulast : prev;  // both lanes: u of the token before the sub-tile
+    if (kUp) S.up = odd ? ulast : prev;  // both lanes: u of the token before the sub-tile
     ulast = S.uu[kOwn - 1];
     S.rr[0] *= prev;
 #pragma unroll
@@ -688,7 +689,7 @@ __device__ __forceinline__ void consume_tile(const Stage<T, kConv> &st, int nt, 
         Scal S;
         token_scalars<T, kGate, kMode, kStruct, kSoftplus, true, kConv>(
             st, 0, nt, ch, o, seq_start, conv_init, active, run, S);
-        if (kStruct) link_prev(S, odd, run.ulast);
+        if (kStruct) link_prev<kCk>(S, odd, run.ulast);
 #pragma unroll 1
         for (int sub = 0; sub < kTile - kSub; sub += kSub) {
             float P0[kSub], P1[kSub], part[kSub];
@@ -696,7 +697,7 @@ __device__ __forceinline__ void consume_tile(const Stage<T, kConv> &st, int nt, 
             Scal N;
             token_scalars<T, kGate, kMode, kStruct, kSoftplus, true, kConv>(
                 st, sub + kSub, nt, ch, o, seq_start, conv_init, active, run, N);
-            if (kStruct) link_prev(N, odd, run.ulast);
+            if (kStruct) link_prev<kCk>(N, odd, run.ulast);
             if (kCk && ckp) store_ckpt<kStruct>(run, S.up, ckp, ckstride, sub);
             recurrence<T, kMode, kStruct, true, kConv, kZoh>(st, sub, nt, P0, P1, ch, run, part);
             if (kMode != kModeAgg && !kCk)
@@ -716,7 +717,7 @@ __device__ __forceinline__ void consume_tile(const Stage<T, kConv> &st, int nt, 
             Scal S;
             token_scalars<T, kGate, kMode, kStruct, kSoftplus, false, kConv>(
                 st, sub, nt, ch, o, seq_start, conv_init, active, run, S);
-            if (kStruct) link_prev(S, odd, run.ulast);
+            if (kStruct) link_prev<kCk>(S, odd, run.ulast);
             float P0[kSub], P1[kSub], part[kSub];
             broadcast<kStruct>(S, P0, P1);
             if (kCk && ckp) store_ckpt<kStruct>(run, S.up, ckp, ckstride, sub);
