@@ -247,7 +247,7 @@ __device__ __forceinline__ void fail(const TmaScanParams &p, int *abort, int cod
 // ones, zero for rows past nt and states past dstate; C is multiplied by
 // ln 2. Lane l handles float4 slots l, l + 32, ...: consecutive lanes write
 // consecutive 16-byte chunks.
-template <typename T, bool kConv>
+template <typename T, bool kConv, bool kNoC>
 __device__ __forceinline__ void convert_bc(Stage<T, kConv> &st, int nt, int dstate, int lane) {
     constexpr int kTile = TileCfg<T>::kTile;
     constexpr int kSlots = kTile * kMaxN / 4;
@@ -263,18 +263,19 @@ __device__ __forceinline__ void convert_bc(Stage<T, kConv> &st, int nt, int dsta
             const int n = 2 * (i0 + e) + odd;
             const bool ok = t < nt && n < dstate;
             vb[e] = ok ? to_f32(st.Bs[t * dstate + n]) : 0.0f;
-            vc[e] = ok ? to_f32(st.Cs[t * dstate + n]) * kLn2 : 0.0f;
+            vc[e] = (ok && !kNoC) ? to_f32(st.Cs[t * dstate + n]) * kLn2 : 0.0f;
         }
         reinterpret_cast<float4 *>(&st.B[0][0])[i] = make_float4(vb[0], vb[1], vb[2], vb[3]);
-        reinterpret_cast<float4 *>(&st.C[0][0])[i] = make_float4(vc[0], vc[1], vc[2], vc[3]);
+        if (!kNoC)
+            reinterpret_cast<float4 *>(&st.C[0][0])[i] = make_float4(vc[0], vc[1], vc[2], vc[3]);
     }
 }
 
 // The producer issues every TMA of a stage as soon as the stage is free and
 // converts its B/C kLag stages later, so it never waits on global memory
 // latency itself; the stage is handed to the consumers (32 arrivals on
-// `full`) after its conversion.
-template <typename T, bool kGate, bool kConv>
+// `full`) after its conversion. kNoC: the passes without y do not load C.
+template <typename T, bool kGate, bool kConv, bool kNoC>
 __device__ void produce(Shared<T, kConv> &S, const TmaScanParams &p, const CUtensorMap *tm_x,
                         const CUtensorMap *tm_d, const CUtensorMap *tm_z,
                         const CUtensorMap *tm_b, const CUtensorMap *tm_c) {
@@ -289,12 +290,12 @@ __device__ void produce(Shared<T, kConv> &S, const TmaScanParams &p, const CUten
         prefetch_tmap(tm_d);
         if (kGate) prefetch_tmap(tm_z);
         prefetch_tmap(tm_b);
-        prefetch_tmap(tm_c);
+        if (!kNoC) prefetch_tmap(tm_c);
     }
     constexpr uint32_t kTileBytes = kNB * kTile * 128;
     constexpr uint32_t kXBytes = kNB * kXRows * 128;
     const uint32_t tx_bytes = (kGate ? 2u : 1u) * kTileBytes + kXBytes;
-    const uint32_t bc_bytes = 2u * kTile * p.dstate * sizeof(T);
+    const uint32_t bc_bytes = (kNoC ? 1u : 2u) * kTile * p.dstate * sizeof(T);
     int s = 0;                 // next stage to fill
     uint32_t phase = 0;
     int cs = 0;                // oldest stage awaiting conversion
@@ -304,7 +305,7 @@ __device__ void produce(Shared<T, kConv> &S, const TmaScanParams &p, const CUten
     // converts the oldest pending stage and hands it to the consumers
     auto convert_oldest = [&]() -> bool {
         if (!mbar_wait(&S.bc[cs], cphase, &S.abort, p.timeout_ns)) return false;
-        convert_bc<T, kConv>(S.stage[cs], S.info[cs].nt, p.dstate, lane);
+        convert_bc<T, kConv, kNoC>(S.stage[cs], S.info[cs].nt, p.dstate, lane);
         __syncwarp();
         mbar_arrive(&S.full[cs]);
         if (++cs == kStages) {
@@ -377,7 +378,7 @@ __device__ void produce(Shared<T, kConv> &S, const TmaScanParams &p, const CUten
                 }
                 mbar_arrive_expect_tx(&S.bc[s], bc_bytes);
                 tma_load_2d(&st.Bs[0], tm_b, &S.bc[s], 0, c1);
-                tma_load_2d(&st.Cs[0], tm_c, &S.bc[s], 0, c1);
+                if (!kNoC) tma_load_2d(&st.Cs[0], tm_c, &S.bc[s], 0, c1);
             }
             __syncwarp();
             if (++s == kStages) {
@@ -981,7 +982,8 @@ scan_tma_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
     }
     __syncthreads();
     if (threadIdx.x >= kConsumers)
-        produce<T, kGate, kConv>(S, p, &tm_x, &tm_d, &tm_z, &tm_b, &tm_c);
+        produce<T, kGate, kConv, kMode == kModeAgg || kMode == kModeCkpt>(S, p, &tm_x, &tm_d,
+                                                                         &tm_z, &tm_b, &tm_c);
     else
         consume<T, kGate, kMode, kSoftplus, kConv, kZoh>(S, p, &tm_y);
 }
