@@ -509,68 +509,101 @@ ssd_tc_state_kernel(const SsdParams p, const __grid_constant__ CUtensorMap tm_b)
 // (or zero), written per chunk as the bfloat16 pair (high, low) in the
 // interleaved operand layout the output kernel's MMA reads: one 32 KB block
 // per (batch row, head, chunk) = high tile [state n][channel p] then low
-// tile. One thread per (batch row, head, state n, group of 8 channels).
-__global__ void ssd_tc_carry_kernel(const SsdParams p) {
-    const long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-    const long long per = (long long)kNp * (kPp / 8);
-    if (e >= (long long)p.batch * p.nheads * per) return;
-    const long long bh = e / per;
-    const int n = (int)((e % per) / (kPp / 8)), pg = (int)(e % (kPp / 8));
+// tile. One CTA per (batch row, head, slab of 16 states): the slab of every
+// chunk state (16 × 64 float32 = 4 KB, contiguous) streams through a ring of
+// kCarryStages bulk copies, so that many chunks' loads are in flight without
+// holding registers; thread t carries state n0 + t/16, channels 4·(t mod 16)
+// to + 3, across the chunks.
+constexpr int kCarryRows = 16, kCarryStages = 8, kCarryThreads = 256;
+constexpr uint32_t kCarrySlab = kCarryRows * kPp * 4;
+struct CarrySmem {
+    float4 slab[kCarryStages][kCarryThreads];
+    float dec[kCarryThreads];  // the decays of the next kCarryThreads chunks
+    uint64_t full[kCarryStages];
+};
+
+__global__ void __launch_bounds__(kCarryThreads) ssd_tc_carry_kernel(const SsdParams p) {
+    __shared__ __align__(128) CarrySmem S;
+    constexpr int kSlabs = kNp / kCarryRows;
+    const long long bh = blockIdx.x / kSlabs;
+    const int n0 = (int)(blockIdx.x % kSlabs) * kCarryRows;
+    const int t = threadIdx.x, n = n0 + t / 16, p0 = 4 * (t % 16);
     const long long b = bh / p.nheads;
     const int h = (int)(bh % p.nheads);
-    const int N = p.dstate, P = p.headdim;
-    float st[8];
+    const int N = p.dstate, P = p.headdim, nc = p.nchunks;
+    const char *src0 = reinterpret_cast<const char *>(p.chunk_state) +
+                       ((bh * nc * kNp + n0) * kPp) * 4ll;
+    const long long chunk_bytes = (long long)kNp * kPp * 4;
+    const int first = min(nc, kCarryStages);
+    if (t == 0) {
+        for (int s = 0; s < kCarryStages; ++s) mbar_init(&S.full[s], 1);
+        fence_barrier_init();
+        for (int c = 0; c < first; ++c) {
+            mbar_arrive_expect_tx(&S.full[c], kCarrySlab);
+            bulk_load(&S.slab[c][0], src0 + c * chunk_bytes, kCarrySlab, &S.full[c]);
+        }
+    }
+    float st[4];
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-        const int pp = 8 * pg + k;
+    for (int k = 0; k < 4; ++k) {
+        const int pp = p0 + k;
         st[k] = (p.h0 && n < N && pp < P)
                     ? p.h0[((b * p.nheads + h) * (long long)P + pp) * N + n] : 0.0f;
     }
-    const uint32_t off = core_off<kPp>(n, 8 * pg);
-    char *blk0 = reinterpret_cast<char *>(p.state_in) + bh * p.nchunks * 32768ll;
-    const float *cs0 = p.chunk_state + (bh * p.nchunks * 128 + n) * 64 + 8 * pg;
-    const float *dec0 = p.chunk_decay + bh * p.nchunks;
-    // groups of kAhead chunks in two alternating register sets: the loads of
-    // the next group are in flight while the current group's dependent
-    // updates run (loads past the last chunk re-read it and are not used)
-    constexpr int kAhead = 4;
-    float4 ua[kAhead], va[kAhead], ub[kAhead], vb[kAhead];
-    float da[kAhead], db[kAhead];
-    auto load = [&](float4 (&u)[kAhead], float4 (&v)[kAhead], float (&d)[kAhead], int c0) {
-#pragma unroll
-        for (int k = 0; k < kAhead; ++k) {
-            const int c = min(c0 + k, p.nchunks - 1);
-            u[k] = __ldg(reinterpret_cast<const float4 *>(cs0 + (long long)c * 128 * 64));
-            v[k] = __ldg(reinterpret_cast<const float4 *>(cs0 + (long long)c * 128 * 64 + 4));
-            d[k] = __ldg(dec0 + c);
+    __syncthreads();  // barriers initialised
+    const uint32_t off = core_off<kPp>(n, p0);
+    char *blk0 = reinterpret_cast<char *>(p.state_in) + bh * nc * 32768ll;
+    const float *dec0 = p.chunk_decay + bh * nc;
+    int c = 0;
+    bool ok = true;
+    for (; c < nc; ++c) {
+        const int s = c % kCarryStages;
+        if (c % kCarryThreads == 0) {  // one load per thread brings the next block of decays
+            __syncthreads();
+            S.dec[t] = c + t < nc ? dec0[c + t] : 0.0f;
+            __syncthreads();
         }
-    };
-    auto update = [&](const float4 (&u)[kAhead], const float4 (&v)[kAhead],
-                      const float (&d)[kAhead], int c0) {
-#pragma unroll
-        for (int k = 0; k < kAhead; ++k) {
-            if (c0 + k >= p.nchunks) break;
-            uint4 hi, lo;
-            split8(st, hi, lo);
-            char *blk = blk0 + (long long)(c0 + k) * 32768;
-            *reinterpret_cast<uint4 *>(blk + off) = hi;
-            *reinterpret_cast<uint4 *>(blk + 16384 + off) = lo;
-            const float s8[8] = {u[k].x, u[k].y, u[k].z, u[k].w, v[k].x, v[k].y, v[k].z, v[k].w};
-#pragma unroll
-            for (int e = 0; e < 8; ++e) st[e] = fmaf(d[k], st[e], s8[e]);
+        const float d = S.dec[c % kCarryThreads];
+        const bool got = mbar_wait(&S.full[s], (uint32_t)(c / kCarryStages) & 1, &kNoAbortTc,
+                                   kWaitNs);
+        float4 u = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (got) u = S.slab[s][t];
+        // h_in of chunk c, then the state after it
+        float v8[8] = {st[0], st[1], st[2], st[3], 0.f, 0.f, 0.f, 0.f};
+        uint4 hi, lo;
+        split8(v8, hi, lo);
+        char *blk = blk0 + (long long)c * 32768;
+        *reinterpret_cast<uint2 *>(blk + off) = make_uint2(hi.x, hi.y);
+        *reinterpret_cast<uint2 *>(blk + 16384 + off) = make_uint2(lo.x, lo.y);
+        st[0] = fmaf(d, st[0], u.x);
+        st[1] = fmaf(d, st[1], u.y);
+        st[2] = fmaf(d, st[2], u.z);
+        st[3] = fmaf(d, st[3], u.w);
+        // every thread has read stage s: refill it with chunk c + kCarryStages
+        ok = __syncthreads_and(got) != 0;
+        if (!ok) break;
+        if (t == 0 && c + kCarryStages < nc) {
+            mbar_arrive_expect_tx(&S.full[s], kCarrySlab);
+            bulk_load(&S.slab[s][0], src0 + (c + kCarryStages) * chunk_bytes, kCarrySlab,
+                      &S.full[s]);
         }
-    };
-    load(ua, va, da, 0);
-    for (int c0 = 0; c0 < p.nchunks; c0 += 2 * kAhead) {
-        load(ub, vb, db, c0 + kAhead);
-        update(ua, va, da, c0);
-        load(ua, va, da, c0 + 2 * kAhead);
-        update(ub, vb, db, c0 + kAhead);
+    }
+    if (!ok) {
+        // a wait gave up: record it, then let the copies still in flight into
+        // this CTA's ring land (bounded) before the CTA exits
+        if (t == 0) {
+            if (p.status) atomicCAS(p.status, 0, kStatusMmaWait);
+            for (int k = c; k < min(nc, c + kCarryStages); ++k)
+                mbar_wait(&S.full[k % kCarryStages], (uint32_t)(k / kCarryStages) & 1,
+                          &kNoAbortTc, kWaitNs);
+        }
+        __syncthreads();
+        return;
     }
     if (p.final_state && n < N) {
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-            const int pp = 8 * pg + k;
+        for (int k = 0; k < 4; ++k) {
+            const int pp = p0 + k;
             if (pp < P) p.final_state[((b * p.nheads + h) * (long long)P + pp) * N + n] = st[k];
         }
     }
@@ -897,8 +930,8 @@ cudaError_t launch_ssd_tc_state(const SsdParams &p, cudaStream_t stream) {
 }
 
 cudaError_t launch_ssd_tc_carry(const SsdParams &p, cudaStream_t stream) {
-    const long long n = (long long)p.batch * p.nheads * kNp * (kPp / 8);
-    ssd_tc_carry_kernel<<<(unsigned)((n + 255) / 256), 256, 0, stream>>>(p);
+    const long long n = (long long)p.batch * p.nheads * (kNp / kCarryRows);
+    ssd_tc_carry_kernel<<<(unsigned)n, kCarryThreads, 0, stream>>>(p);
     return cudaGetLastError();
 }
 

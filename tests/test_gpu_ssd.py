@@ -77,6 +77,21 @@ def test_ssd_initial_state_and_no_gate():
     gh.compare(gh.to_np(hf), ho, gh.RTOL["f32"], "h0 final state")
 
 
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_ssd_long_sequence_from_a_state(dtype):
+    """More chunks than the carry stages its decays for at a time (258 chunks
+    of 128 tokens), from an initial state."""
+    H, P, N = 2, 16, 16
+    inp = _inputs(1, 33000, H, P, N, dtype, seed=7150)
+    g = torch.Generator().manual_seed(7151)
+    h0 = torch.randn(1, H * P, N, generator=g)
+    y, hf = _gpu(inp, h0.to(DEV))
+    torch.cuda.synchronize()
+    yo, ho = _oracle(inp, P, h0)
+    gh.compare(gh.to_np(y), yo, gh.RTOL[dtype], "long y")
+    gh.compare(gh.to_np(hf), ho, gh.RTOL[dtype], "long final state")
+
+
 def test_ssd_equals_wide_scan_on_a_head_layer():
     """A Mamba-2-sized layer (2 × 2048 tokens, 32 heads of 64, d_state 128):
     the chunked form against the recurrence of the wide-state scan kernel
