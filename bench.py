@@ -197,9 +197,13 @@ def oracle_sample(w, inp, target_s, cores):
     elements per pass, description)."""
     import oracle
     orc = oracle.default()
-    probe = max(cores, 8)
+    # the probe's inputs are prepared, and its threads started once, outside
+    # the timed call: the rate is the oracle's own
+    probe = min(w.dim, 4 * max(cores, 8))
+    pargs = _oracle_args(inp, (0,), probe)
+    orc.fwd(*pargs, softplus=True, threads=cores)
     t = time.perf_counter()
-    orc.fwd(*_oracle_args(inp, (0,), probe), softplus=True, threads=cores)
+    orc.fwd(*pargs, softplus=True, threads=cores)
     rate = probe * w.seqlen * w.dstate / max(time.perf_counter() - t, 1e-9)
     row_s = w.dim * w.seqlen * w.dstate / rate
     if row_s >= target_s:
@@ -311,6 +315,9 @@ def smi_id(torch, dev, local):
         return str(local)
 
 
+HOLD_CYCLES = 2_000_000  # device clock cycles (~1 ms at 1.965 GHz)
+
+
 def time_calls(torch, stream, fn, n, flush=None):
     """CUDA-event time of one call in ms: the mean of n back-to-back calls,
     and (with `flush`, a buffer larger than L2 written before each call) the
@@ -331,6 +338,10 @@ def time_calls(torch, stream, fn, n, flush=None):
     cold = []
     for _ in range(10):
         flush.zero_()
+        # ~1 ms of device-side spinning after the flush, so that the call is
+        # already queued when the start event fires: the interval then holds
+        # the call's device time, not the host's time to launch it
+        torch.cuda._sleep(HOLD_CYCLES)
         c0 = torch.cuda.Event(enable_timing=True)
         c1 = torch.cuda.Event(enable_timing=True)
         c0.record(stream)

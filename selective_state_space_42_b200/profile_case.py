@@ -127,6 +127,9 @@ def main(argv=None) -> int:
         cold = []
         for i in range(20):
             flush.zero_()
+            # device-side spin so that the launch is queued before e0 fires:
+            # the interval holds the kernels, not the host's launch time
+            torch.cuda._sleep(2_000_000)
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record()
             launch(i)
