@@ -232,10 +232,16 @@ def test_long_sequence_sampled():
         assert torch.isfinite(grads[k]).all(), k
 
 
-def test_library_allocated_workspace_matches():
+@pytest.mark.parametrize("shape,path", [((2, 77, 70), None), ((2, 301, 256), "seq")],
+                         ids=["own-sweep", "forward-kernel-checkpoints"])
+def test_library_allocated_workspace_matches(shape, path, monkeypatch):
     """selscan_bwd (workspace allocated on the stream by the library) and
-    selscan_bwd_workspace (torch-allocated workspace) give identical results."""
-    inp, dy, df = _inputs(2, 77, 70, 16, "bf16", True, seed=15)
+    selscan_bwd_workspace (torch-allocated workspace) give identical results,
+    also where the workspace holds the forward kernel's checkpoint-pass
+    region (one-pass plan forced)."""
+    if path:
+        monkeypatch.setenv("SELSCAN_PATH", path)
+    inp, dy, df = _inputs(*shape, 16, "bf16", True, seed=15)
     d = {k: (None if v is None else v.to(DEV)) for k, v in inp.items()}
     args = (d["x"], d["delta"], d["A"], d["B"], d["C"], d["D"], d["z"], d["delta_bias"])
     g1 = ss.selscan_bwd(*args, dy=dy.to(DEV), dfinal_state=df.to(DEV))
