@@ -515,7 +515,8 @@ SELSCAN_API int64_t selscan_ssd_workspace_bytes(int64_t batch, int64_t seqlen, i
  * wait has given up; otherwise the code of the first one that did (1: a
  * sequence chunk waited too long for its predecessor's state; 2, 3: a
  * pipeline stage waited too long; 4: a tensor-core MMA or its operand copy
- * of selscan_ssd_fwd did not complete in time). Every device-side wait in the library is
+ * of selscan_ssd_fwd did not complete in time; 5: the state copy of a
+ * selscan_state_update step did not complete in time). Every device-side wait in the library is
  * bounded (2 s); a wait that gives up records its code here and the kernel
  * returns instead of hanging, leaving its outputs undefined. `clear` nonzero
  * resets the word to 0 after reading it.

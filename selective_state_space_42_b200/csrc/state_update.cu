@@ -9,12 +9,15 @@
 // is read and written once, everything else is small. Lanes work in quads:
 // the four lanes of a quad hold the four 16-byte quarters of one chain's
 // 16 states, so each warp-wide access covers 8 whole chains = 512 contiguous
-// bytes. Every lane serves kChainsPerLane chains (8 chains apart), issuing
-// all of their state loads before any arithmetic so that enough bytes are in
-// flight to cover DRAM latency. The partial outputs Σ_n C[n]·h[n] are
-// combined across a quad with two xor-shuffles. Each state element is read
-// and written by the same thread, which makes the in-place update safe.
+// bytes. Every lane serves kChainsPerLane chains (8 chains apart). A CTA's
+// 256 chains have contiguous states (16 KB): one bulk copy into shared
+// memory, issued before anything else, brings them in, so the bytes in
+// flight are not bounded by registers. The partial outputs Σ_n C[n]·h[n] are
+// combined across a quad with two xor-shuffles. Each state element is
+// written by the thread that read it, after the copy has landed, which makes
+// the in-place update safe.
 #include "selscan_device.cuh"
+#include "tma_util.cuh"
 
 namespace selscan {
 namespace {
@@ -23,6 +26,21 @@ constexpr int kThreads = 256;
 constexpr int kLanesPerChain = 4;
 constexpr int kChainsPerLane = 4;                 // chains per lane, 8 apart
 constexpr int kChainsPerWarp = 32 / kLanesPerChain * kChainsPerLane;  // 32
+constexpr int kChainsPerCta = kThreads / 32 * kChainsPerWarp;          // 256
+constexpr int kMinCtas = 6;                       // resident CTAs per SM the registers allow
+constexpr int kStatusStateCopy = 5;               // device error code: the state copy timed out
+constexpr uint64_t kStepWaitNs = 2000000000ull;   // bounded wait for the copy (2 s)
+__device__ const int kNoAbortStep = 0;
+
+// Contiguous global -> shared bulk copy (16-byte aligned, size a multiple of
+// 16) completing on an mbarrier's transaction count.
+__device__ __forceinline__ void bulk_copy_in(void *dst, const void *src, uint32_t bytes,
+                                             uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        ::"r"(smem_addr(dst)), "l"(src), "r"(bytes), "r"(smem_addr(bar))
+        : "memory");
+}
 
 // The causal conv + SiLU for one chain's token: reads the chain's window of
 // the previous inputs, writes it back shifted by the new input.
@@ -76,24 +94,29 @@ __device__ __forceinline__ float4 ld4_f32(const __nv_bfloat16 *p) {
 // reduction of Σ_n C[n]·h[n] every lane of the quad has the sum, and the
 // owner writes the chain's y.
 template <typename T, bool kGate, bool kConv, bool kZoh>
-__global__ void __launch_bounds__(kThreads)
-state_update_vec_kernel(const StepParams p) {
+__global__ void __launch_bounds__(kThreads, kMinCtas)
+state_update_vec_kernel(const StepParams p, int *status) {
+    __shared__ __align__(128) float4 sst[kChainsPerCta * 4];  // the CTA's states, 16 KB
+    __shared__ uint64_t bar;
     const int lane = threadIdx.x & 31;
     const int q = lane & 3;
     const int j = lane >> 2;
     const int quad0 = lane & ~3;
+    const int wl = threadIdx.x >> 5;  // warp within the CTA
     const int64_t warp = ((int64_t)blockIdx.x * kThreads + threadIdx.x) >> 5;
     const int64_t total = p.batch * p.dim;
     const int64_t base = warp * kChainsPerWarp;
+    const int64_t cta0 = (int64_t)blockIdx.x * kChainsPerCta;
 
-    // state loads first, so that they are all in flight together
-    float4 st[kChainsPerLane];
-#pragma unroll
-    for (int k = 0; k < kChainsPerLane; ++k) {
-        const int64_t chain = base + 8 * k + j;
-        st[k] = chain < total ? *reinterpret_cast<const float4 *>(p.state + chain * kMaxN + 4 * q)
-                              : make_float4(0.f, 0.f, 0.f, 0.f);
+    // the CTA's states first: one copy of its contiguous chains
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        fence_barrier_init();
+        const uint32_t bytes = (uint32_t)(min((int64_t)kChainsPerCta, total - cta0) * kMaxN * 4);
+        mbar_arrive_expect_tx(&bar, bytes);
+        bulk_copy_in(sst, p.state + cta0 * kMaxN, bytes, &bar);
     }
+    __syncthreads();
 
     // (b, d) of chain base + j by one division, then of base + 8k + j by steps of 8
     int64_t bk[kChainsPerLane], dk[kChainsPerLane];
@@ -129,6 +152,13 @@ state_update_vec_kernel(const StepParams p) {
 
     const T *Bp = static_cast<const T *>(p.B);
     const T *Cp = static_cast<const T *>(p.C);
+    if (!__all_sync(0xffffffffu, mbar_wait(&bar, 0, &kNoAbortStep, kStepWaitNs))) {
+        // the warp agrees to give up: record it, give the copy one more
+        // bounded wait to land, and leave the warp's chains as they were
+        if (status) atomicCAS(status, 0, kStatusStateCopy);
+        mbar_wait(&bar, 0, &kNoAbortStep, kStepWaitNs);
+        return;
+    }
     float mine = 0.f;
 #pragma unroll
     for (int k = 0; k < kChainsPerLane; ++k) {
@@ -141,7 +171,7 @@ state_update_vec_kernel(const StepParams p) {
             const float4 b4 = ld4_f32(Bp + bk[k] * kMaxN + 4 * q);
             const float4 c4 = ld4_f32(Cp + bk[k] * kMaxN + 4 * q);
             const float dl = dt * kLog2e;
-            float4 h = st[k];
+            float4 h = sst[(wl * kChainsPerWarp + 8 * k + j) * 4 + q];
             const float e0 = ex2_approx(dl * a4.x), e1 = ex2_approx(dl * a4.y);
             const float e2 = ex2_approx(dl * a4.z), e3 = ex2_approx(dl * a4.w);
             float4 bz = b4;
@@ -224,9 +254,12 @@ cudaError_t launch_zoh(const StepParams &p, cudaStream_t stream) {
                      (reinterpret_cast<uintptr_t>(p.B) & bc_align) == 0 &&
                      (reinterpret_cast<uintptr_t>(p.C) & bc_align) == 0;
     if (vec) {
+        int *status = nullptr;
+        const cudaError_t e = device_status_address(&status);
+        if (e != cudaSuccess) return e;
         const int64_t warps = (chains + kChainsPerWarp - 1) / kChainsPerWarp;
         const unsigned blocks = (unsigned)((warps * 32 + kThreads - 1) / kThreads);
-        state_update_vec_kernel<T, kGate, kConv, kZoh><<<blocks, kThreads, 0, stream>>>(p);
+        state_update_vec_kernel<T, kGate, kConv, kZoh><<<blocks, kThreads, 0, stream>>>(p, status);
     } else {
         const int64_t threads = chains * kLanesPerChain;
         const unsigned blocks = (unsigned)((threads + kThreads - 1) / kThreads);
