@@ -8,6 +8,7 @@ the device) and to give quick CUDA-event timings without one:
     python -m selective_state_space_42_b200.profile_case bwd mamba2p8b_layer --launches 2
     python -m selective_state_space_42_b200.profile_case bwd mamba2p8b_layer --seqlen 1024
     python -m selective_state_space_42_b200.profile_case ssd --launches 3
+    python -m selective_state_space_42_b200.profile_case decode --launches 4 --flushed 3
 
 ``scan`` calls selscan_fwd on a scan workload; ``bwd`` calls selscan_bwd on
 it (with a seeded dy and final-state gradient); ``decode`` calls
@@ -15,6 +16,9 @@ selscan_state_update on the decode workload; ``ssd`` calls selscan_ssd_fwd
 on the Mamba-2-shaped head workload. With ``--time`` it also prints
 the median CUDA-event time per launch, cold (a 512 MiB buffer is written
 between launches, which evicts L2) and back to back, as one JSON line.
+``--flushed N`` adds N launches after the back-to-back ones, each after a
+512 MiB write (for DRAM counters of launches that find L2 full of another
+buffer's dirty lines).
 """
 from __future__ import annotations
 
@@ -103,6 +107,8 @@ def main(argv=None) -> int:
                     help="scan workload name (ignored for decode)")
     ap.add_argument("--launches", type=int, default=2)
     ap.add_argument("--time", action="store_true")
+    ap.add_argument("--flushed", type=int, default=0,
+                    help="launches after the back-to-back ones, each after a 512 MiB write")
     ap.add_argument("--seqlen", type=int, default=None,
                     help="scan and bwd: the workload cut (or grown) to this many tokens")
     args = ap.parse_args(argv)
@@ -117,6 +123,12 @@ def main(argv=None) -> int:
         launch, nbytes = _decode_case()
     for i in range(args.launches):
         launch(i)
+    if args.flushed > 0:
+        buf = torch.empty(512 << 20, dtype=torch.uint8, device="cuda")
+        for i in range(args.flushed):
+            buf.zero_()
+            launch(args.launches + i)
+        del buf
     torch.cuda.synchronize()
     out = {"kernel": args.kernel, "launches": args.launches,
            "workload": {"decode": wl.DECODE.name, "ssd": wl.SSD.name}.get(args.kernel,
