@@ -242,6 +242,23 @@ __device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t b
         : "memory");
 }
 
+// Contiguous shared -> global bulk copy in this thread's bulk group, and the
+// waits for the group: its shared-memory reads done, or the whole copy done.
+__device__ __forceinline__ void bulk_store(void *dst, const void *src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;"
+                 ::"l"(dst), "r"(smem_addr(src)), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() {
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_read() {
+    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_all() {
+    asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+
 constexpr int kThrTc = 256;  // threads of the two MMA kernels
 
 // Work item k of this thread in a cooperative pass over a kQ-row tile with
@@ -358,7 +375,12 @@ __device__ __forceinline__ bool wait_mma(uint64_t *bar, uint32_t parity, int *st
 // accumulator alternate between two buffers, so that the MMAs of head k run
 // while head k − 1's result is stored and head k + 1's x is in flight.
 // 256 threads; in the epilogue thread t reads state row n = t mod 128
-// (tensor-memory lane n), column half t / 128.
+// (tensor-memory lane n), column half t / 128, into the operand pair its
+// head no longer needs (rows 0..63 over the high part, 64..127 over the low
+// part), and one thread sends the 32 KB to global memory by two bulk copies.
+// The chunk state is stored in 16-byte units swizzled within each row: the
+// channels 4u .. 4u + 3 of state n sit at unit u ^ (n mod 8) of the row, so
+// that the 32 rows a warp stages at once spread over all banks.
 
 struct TcStateSmem {
     bf16 Bt[kQ * kNp];     // rows token j, columns state n
@@ -417,6 +439,9 @@ ssd_tc_state_kernel(const SsdParams p, const __grid_constant__ CUtensorMap tm_b)
 
     for (int k = 0; k <= nh; ++k) {
         float aend2 = 0.0f;
+        // the operand pair written below was sent out as head k − 2's state:
+        // its copy must have read it (the barriers in chunk_delta publish this)
+        if (t == 0 && k >= 2) bulk_wait_read();
         if (k < nh) {
             const int h = h_first + k;
             chunk_delta(p, h, nq, dt_raw, S.dt, S.acum2, S.wsum);
@@ -482,24 +507,34 @@ ssd_tc_state_kernel(const SsdParams p, const __grid_constant__ CUtensorMap tm_b)
             ok = __syncthreads_and(ok && wait_mma(&S.bar[kk & 1], (kk >> 1) & 1, p.status));
             tc_fence_after();
             if (ok) {
-                // lane r holds state row n = r: this thread stores S[n][32·hh .. 32·hh + 31]
-                float *dst = p.chunk_state +
-                             (((b * p.nheads + h) * p.nchunks + c) * 128 + r) * 64 + 32 * hh;
+                // lane r holds state row n = r: this thread stages S[n][32·hh .. 32·hh + 31]
                 float v[32];
                 tmem_ld32(tmem + ((uint32_t)((warp & 3) * 32) << 16) + 64u * (uint32_t)(kk & 1) +
                               32 * hh,
                           v);
+                float4 *row = reinterpret_cast<float4 *>(r < 64 ? S.Xw[kk & 1] : S.Xl[kk & 1]) +
+                              (r & 63) * 16;
 #pragma unroll
-                for (int q = 0; q < 32; q += 4)
-                    *reinterpret_cast<float4 *>(dst + q) =
-                        make_float4(v[q], v[q + 1], v[q + 2], v[q + 3]);
+                for (int i = 0; i < 8; ++i)
+                    row[(8 * hh + i) ^ (r & 7)] =
+                        make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
                 if (t == 0)
                     p.chunk_decay[(b * p.nheads + h) * p.nchunks + c] = ex2_approx(aend_prev);
             }
             tc_fence_before();
+            fence_proxy_async_smem();
+            __syncthreads();
+            if (t == 0 && ok) {
+                char *dst = reinterpret_cast<char *>(
+                    p.chunk_state + ((b * p.nheads + h) * p.nchunks + c) * 128ll * 64);
+                bulk_store(dst, S.Xw[kk & 1], 16384);
+                bulk_store(dst + 16384, S.Xl[kk & 1], 16384);
+                bulk_commit();
+            }
         }
         aend_prev = aend2;
     }
+    if (t == 0) bulk_wait_all();  // the last states are out before the CTA ends
     __syncthreads();
     if (warp == 0) tmem_dealloc(tmem, 128);
 }
@@ -567,7 +602,7 @@ __global__ void __launch_bounds__(kCarryThreads) ssd_tc_carry_kernel(const SsdPa
         const bool got = mbar_wait(&S.full[s], (uint32_t)(c / kCarryStages) & 1, &kNoAbortTc,
                                    kWaitNs);
         float4 u = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (got) u = S.slab[s][t];
+        if (got) u = S.slab[s][(t & ~15) | ((t & 15) ^ (n & 7))];  // the rows' 16-byte swizzle
         // h_in of chunk c, then the state after it
         float v8[8] = {st[0], st[1], st[2], st[3], 0.f, 0.f, 0.f, 0.f};
         uint4 hi, lo;
