@@ -242,21 +242,12 @@ __device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t b
         : "memory");
 }
 
-// Contiguous shared -> global bulk copy in this thread's bulk group, and the
-// waits for the group: its shared-memory reads done, or the whole copy done.
+// Contiguous shared -> global bulk copy (16-byte aligned, size a multiple of
+// 16) in this thread's bulk group.
 __device__ __forceinline__ void bulk_store(void *dst, const void *src, uint32_t bytes) {
     asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;"
                  ::"l"(dst), "r"(smem_addr(src)), "r"(bytes)
                  : "memory");
-}
-__device__ __forceinline__ void bulk_commit() {
-    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-}
-__device__ __forceinline__ void bulk_wait_read() {
-    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-}
-__device__ __forceinline__ void bulk_wait_all() {
-    asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 
 constexpr int kThrTc = 256;  // threads of the two MMA kernels
@@ -441,7 +432,7 @@ ssd_tc_state_kernel(const SsdParams p, const __grid_constant__ CUtensorMap tm_b)
         float aend2 = 0.0f;
         // the operand pair written below was sent out as head k − 2's state:
         // its copy must have read it (the barriers in chunk_delta publish this)
-        if (t == 0 && k >= 2) bulk_wait_read();
+        if (t == 0 && k >= 2) bulk_wait_read<0>();
         if (k < nh) {
             const int h = h_first + k;
             chunk_delta(p, h, nq, dt_raw, S.dt, S.acum2, S.wsum);
@@ -534,7 +525,7 @@ ssd_tc_state_kernel(const SsdParams p, const __grid_constant__ CUtensorMap tm_b)
         }
         aend_prev = aend2;
     }
-    if (t == 0) bulk_wait_all();  // the last states are out before the CTA ends
+    if (t == 0) bulk_wait<0>();  // the last states are out before the CTA ends
     __syncthreads();
     if (warp == 0) tmem_dealloc(tmem, 128);
 }
