@@ -936,16 +936,31 @@ cudaError_t launch_ssd_tc_state(const SsdParams &p, cudaStream_t stream) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
+    static int sms_of[64] = {0};
     if (dev >= 0 && dev < 64 && !configured[dev]) {
         e = set_smem(ssd_tc_state_kernel, sizeof(TcStateSmem) + 1024);
+        if (e == cudaSuccess)
+            e = cudaDeviceGetAttribute(&sms_of[dev], cudaDevAttrMultiProcessorCount, dev);
         if (e != cudaSuccess) return e;
         configured[dev] = true;
     }
-    // heads per CTA: as many as keep about two waves of CTAs on 148 SMs (two
-    // CTAs each), at most 8
+    const int sms = (dev >= 0 && dev < 64 && sms_of[dev] > 0) ? sms_of[dev] : 148;
+    // heads per CTA (1..8): the fewest estimated CTA-time units, a CTA of g
+    // heads taking (setup + g) with the setup (TMEM, barriers, the B tile)
+    // about half a head, and the CTAs running in waves of two per SM
     SsdParams q = p;
-    const long long items = (long long)p.nchunks * p.nheads * p.batch;
-    q.heads_per_cta = (int)std::min<long long>(8, std::max<long long>(1, items / (2 * 2 * 148)));
+    int best = 1;
+    double best_cost = 1e300;
+    for (int g = 1; g <= 8; ++g) {
+        const long long ctas = (long long)p.nchunks * ((p.nheads + g - 1) / g) * p.batch;
+        const long long waves = (ctas + 2LL * sms - 1) / (2LL * sms);
+        const double cost = (double)waves * (0.5 + g);
+        if (cost < best_cost) {
+            best_cost = cost;
+            best = g;
+        }
+    }
+    q.heads_per_cta = best;
     const dim3 grid((unsigned)p.nchunks,
                     (unsigned)((p.nheads + q.heads_per_cta - 1) / q.heads_per_cta),
                     (unsigned)p.batch);

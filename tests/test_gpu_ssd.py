@@ -92,12 +92,14 @@ def test_ssd_long_sequence_from_a_state(dtype):
     gh.compare(gh.to_np(hf), ho, gh.RTOL[dtype], "long final state")
 
 
-def test_ssd_equals_wide_scan_on_a_head_layer():
-    """A Mamba-2-sized layer (2 × 2048 tokens, 32 heads of 64, d_state 128):
-    the chunked form against the recurrence of the wide-state scan kernel
-    with the same inputs broadcast to channels, and a channel sample against
-    the oracle."""
-    inp = _inputs(2, 2048, 32, 64, 128, "bf16", seed=7200)
+@pytest.mark.parametrize("L,H", [(2048, 32), (4096, 37)], ids=["32-heads", "37-heads"])
+def test_ssd_equals_wide_scan_on_a_head_layer(L, H):
+    """A Mamba-2-sized layer (2 × L tokens, H heads of 64, d_state 128): the
+    chunked form against the recurrence of the wide-state scan kernel with
+    the same inputs broadcast to channels, and a channel sample against the
+    oracle. The state kernel groups 4 heads per CTA for the first shape and
+    3 for the second, whose last group holds one head."""
+    inp = _inputs(2, L, H, 64, 128, "bf16", seed=7200 + H)
     y, hf = _gpu(inp)
     d = {k: (None if v is None else v.to(DEV)) for k, v in inp.items()}
     rep = lambda v: v.repeat_interleave(64, dim=-1).contiguous()  # noqa: E731
@@ -107,7 +109,7 @@ def test_ssd_equals_wide_scan_on_a_head_layer():
     torch.cuda.synchronize()
     gh.compare(gh.to_np(y), gh.to_np(yw), 2e-2, "ssd vs recurrence y")
     gh.compare(gh.to_np(hf), gh.to_np(hw), 2e-2, "ssd vs recurrence state")
-    chans = list(wl.channel_subset(2048, 64))
+    chans = list(wl.channel_subset(H * 64, 64))
     n = gh.to_np
     heads = [c // 64 for c in chans]
     A_s = np.repeat(n(inp["A"])[heads][:, None], 128, axis=1)
