@@ -301,13 +301,6 @@ __device__ __forceinline__ void load_tile_regs(uint4 (&v)[tile_items<kCols>()], 
     }
 }
 
-// Δ_t of the chunk's tokens t (zero past the sequence end; from chunk_dt_raw)
-// into dt[], and the
-// inclusive prefix sums of Δ·A over the chunk, times log2(e), into acum2[]
-// (so exp(Acum_i − Acum_j) = 2^(acum2_i − acum2_j)). With F given, also
-// F[t] = 2^(−acum2_t)·Δ_t and the per-warp maxima of |acum2| in wmax[4].
-// Threads 0..kQ−1 compute; every thread of the block takes part in the two
-// barriers.
 // dt + dt_bias of this thread's token (threads 0..kQ−1 of a chunk with nq
 // tokens; 0 otherwise): issued early, consumed by chunk_delta.
 __device__ __forceinline__ float chunk_dt_raw(const SsdParams &p, long long b, int h, long long t0,
@@ -318,6 +311,12 @@ __device__ __forceinline__ float chunk_dt_raw(const SsdParams &p, long long b, i
            (p.dt_bias ? p.dt_bias[h] : 0.0f);
 }
 
+// Δ_t of the chunk's tokens t (zero past the sequence end; from chunk_dt_raw)
+// into dt[], and the inclusive prefix sums of Δ·A over the chunk, times
+// log2(e), into acum2[] (so exp(Acum_i − Acum_j) = 2^(acum2_i − acum2_j)).
+// With F given, also F[t] = 2^(−acum2_t)·Δ_t and the per-warp maxima of
+// |acum2| in wmax[4]. Threads 0..kQ−1 compute; every thread of the block
+// takes part in the two barriers.
 __device__ __forceinline__ void chunk_delta(const SsdParams &p, int h, int nq, float raw, float *dt,
                                             float *acum2, float *wsum, float *F = nullptr,
                                             float *wmax = nullptr) {
