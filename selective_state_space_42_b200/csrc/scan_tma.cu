@@ -178,16 +178,16 @@ __device__ __forceinline__ float2 exp2_poly2(float2 e) {
 // Zero-order-hold input factor (exp(z) − 1)/z of a pair, z = Δ·A (here
 // e·ln 2 with e the log2 exponent), given a = exp(z): below |z| = 1/32 the
 // series 1 + z/2 + z²/6 + z³/24 (truncation under z⁴/120 < 1e-8 relative),
-// above (a − 1)/z with the MUFU reciprocal.
-__device__ __forceinline__ float2 zoh_factor2(float2 e, float2 a) {
+// above (a − 1)·iz with iz = 1/z given.
+__device__ __forceinline__ float2 zoh_factor2(float2 e, float2 a, float2 iz) {
     const float2 z = __fmul2_rn(e, make_float2(kLn2, kLn2));
     float2 sr = __ffma2_rn(z, make_float2(1.0f / 24.0f, 1.0f / 24.0f),
                            make_float2(1.0f / 6.0f, 1.0f / 6.0f));
     sr = __ffma2_rn(z, sr, make_float2(0.5f, 0.5f));
     sr = __ffma2_rn(z, sr, make_float2(1.0f, 1.0f));
     const float2 am1 = __fadd2_rn(a, make_float2(-1.0f, -1.0f));
-    return make_float2(fabsf(z.x) < 0.03125f ? sr.x : am1.x * rcp_approx(z.x),
-                       fabsf(z.y) < 0.03125f ? sr.y : am1.y * rcp_approx(z.y));
+    return make_float2(fabsf(z.x) < 0.03125f ? sr.x : am1.x * iz.x,
+                       fabsf(z.y) < 0.03125f ? sr.y : am1.y * iz.y);
 }
 
 #ifndef SELSCAN_POLY_PAIRS
@@ -409,6 +409,7 @@ __device__ __forceinline__ float signed_tiny(float v) {
 struct Chain {
     float A0;               // A[d, 0]
     float An[kHalf];        // A[d, n] of this lane's states (n = 2i + odd)
+    float iAn[kHalf];       // 1 / A[d, n] (the ZOH term)
     float dskip, bias, biasl;  // D[d], delta_bias[d], delta_bias[d]·log2 e
     float cw[kMaxConv], cb;    // conv taps
 };
@@ -614,8 +615,14 @@ __device__ __forceinline__ void recurrence(const Stage<T, kConv> &st, int sub, i
                                     mul2(u2, make_float2(b1.x, b1.y)),
                                     mul2(u2, make_float2(b1.z, b1.w))};
             if (kZoh) {
+                // 1/z = 1/(Δ·A[d, n]) from one reciprocal per token (P0 = Δ·log2 e)
+                const float r0s = rcp_approx(P0[k]) * kLog2e;
+                const float2 r0 = make_float2(r0s, r0s);
 #pragma unroll
-                for (int q = 0; q < kHalf / 2; ++q) bu[q] = mul2(bu[q], zoh_factor2(e[q], a[q]));
+                for (int q = 0; q < kHalf / 2; ++q)
+                    bu[q] = mul2(bu[q], zoh_factor2(e[q], a[q],
+                                                    mul2(r0, make_float2(ch.iAn[2 * q],
+                                                                         ch.iAn[2 * q + 1]))));
             }
 #pragma unroll
             for (int q = 0; q < kHalf / 2; ++q) run.h[q] = fma2(a[q], run.h[q], bu[q]);
@@ -787,6 +794,7 @@ __device__ void consume(Shared<T, kConv> &S, const TmaScanParams &p, const CUten
                         const int n = 2 * i + (odd ? 1 : 0);
                         const float an = n < p.dstate ? Ar[n] : 0.0f;
                         ch.An[i] = an;
+                        if (kZoh) ch.iAn[i] = 1.0f / an;
                         if (n < p.dstate) ok &= (an == (float)(n + 1) * ch.A0);
                     }
                     ch.dskip = p.Dskip ? p.Dskip[d] : 0.0f;
@@ -798,7 +806,7 @@ __device__ void consume(Shared<T, kConv> &S, const TmaScanParams &p, const CUten
                 } else {
                     ch.A0 = 0.0f;
 #pragma unroll
-                    for (int i = 0; i < kHalf; ++i) ch.An[i] = 0.0f;
+                    for (int i = 0; i < kHalf; ++i) ch.An[i] = ch.iAn[i] = 0.0f;
                     ch.dskip = ch.bias = 0.0f;
                     if (kConv) {
 #pragma unroll
