@@ -385,8 +385,11 @@ def extra_legs(args, torch, ss, wl, dev, stream, peak, over_ranks):
     out["mamba130m_layer"], _ = scan_leg("mamba130m_layer", 200)
     out["long_1m"], _ = scan_leg("long_1m", 5)
     ref = args.headline_ms
-    out["general_A"], _ = scan_leg("mamba2p8b_layer_expA", 100, ref_ms=ref)
-    out["general_A"]["A"] = "-exp(log(n+1)) in float32 (not bit-exactly (n+1)*A[d,0]: general decay)"
+    out["pages_A"], _ = scan_leg("mamba2p8b_layer_expA", 100, ref_ms=ref)
+    out["pages_A"]["A"] = ("-exp(log(n+1)) in float32 (within a few ulps of (n+1)*A[d,0]: "
+                           "power-ladder decay)")
+    out["general_A"], _ = scan_leg("mamba2p8b_layer_trainedA", 100, ref_ms=ref)
+    out["general_A"]["A"] = "-exp(log(n+1) + 0.1*N(0,1)) per (d, n) in float32: general decay"
     out["zoh"], _ = scan_leg("mamba2p8b_layer", 50, bbar="zoh", ref_ms=ref)
     out["zoh"]["input_term"] = "(exp(delta*A)-1)/A*B*x"
 

@@ -506,8 +506,8 @@ __device__ __forceinline__ void bwd_body(BwdSmem &S, const BwdParams &p, int g) 
     }
 }
 
-// A[d, n] == (n+1)·A[d, 0] for every state of every channel of the warp
-// selects the power-ladder decay (the A = −(1..N) initialisation).
+// A[d, n] = (n+1)·A[d, 0] (ladder_state) for every state of every channel of
+// the warp selects the power-ladder decay (the A = −(1..N) initialisation).
 template <typename T, bool kGate, bool kSoftplus, bool kConv, bool kZoh>
 __global__ void __launch_bounds__(kChains, 6) scan_bwd_kernel(const BwdParams p) {
     __shared__ BwdSmem S;
@@ -516,7 +516,7 @@ __global__ void __launch_bounds__(kChains, 6) scan_bwd_kernel(const BwdParams p)
     if (ok && d < p.dim) {
         const float a0 = p.A[d * p.dstate];
         for (int n = 1; n < p.dstate; ++n)
-            if (p.A[d * p.dstate + n] != (float)(n + 1) * a0) ok = false;
+            if (!ladder_state(p.A[d * p.dstate + n], a0, n)) ok = false;
     }
     if (__all_sync(0xffffffffu, ok))
         bwd_body<T, kGate, kSoftplus, true, kConv, kZoh>(S, p, 0);

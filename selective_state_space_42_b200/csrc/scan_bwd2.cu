@@ -538,14 +538,14 @@ template <typename T, bool kGate, bool kSoftplus>
 __global__ void __launch_bounds__(kWarps * 32, 5) scan_bwd_pairs_kernel(const BwdParams p) {
     extern __shared__ __align__(128) unsigned char smem[];
     WarpSmem<T> *S = reinterpret_cast<WarpSmem<T> *>(smem);
-    // A[d, n] == (n+1)·A[d, 0] for every state of every channel of the CTA
-    // selects the power-ladder decay (two threads per channel check it)
+    // A[d, n] = (n+1)·A[d, 0] (ladder_state) for every state of every channel
+    // of the CTA selects the power-ladder decay (two threads per channel check it)
     const long long d = (long long)blockIdx.x * (kWarps * kCh) + threadIdx.x / 2;
     bool ok = true;
     if (d < p.dim) {
         const float a0 = p.A[d * p.dstate];
         for (int n = 1 + (threadIdx.x & 1); n < p.dstate; n += 2)
-            if (p.A[d * p.dstate + n] != (float)(n + 1) * a0) ok = false;
+            if (!ladder_state(p.A[d * p.dstate + n], a0, n)) ok = false;
     }
     if (__syncthreads_and(ok))
         bwd_pairs_body<T, kGate, kSoftplus, true>(S, p);

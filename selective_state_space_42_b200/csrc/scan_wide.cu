@@ -14,7 +14,7 @@
 // 128 / kLanes consecutive channels of one batch row; B and C of a 16-token
 // tile are staged in shared memory as float32. One pass over the whole
 // sequence per CTA (no chunking). The exponent strategy follows scan.cu: with
-// A[d, n] == (n+1)·A[d, 0] on every channel of the CTA, Abar[n] = r^(n+1) is
+// A[d, n] = (n+1)·A[d, 0] (ladder_state) on every channel of the CTA, Abar[n] = r^(n+1) is
 // a lane's base power r^(16·slice) times a ladder; otherwise one ex2 per
 // element. Optional: initial state, causal conv in front, ZOH input term.
 #include "selscan_device.cuh"
@@ -62,7 +62,7 @@ scan_wide_kernel(const ScanParams p) {
             const float an = n < N ? p.A[d * N + n] : 0.0f;
             A2[i] = an * kLog2e;
             if (n < N) {
-                structured &= (an == (float)(n + 1) * a0);
+                structured &= ladder_state(an, a0, n);
                 constant &= (an == a0);
             }
         }

@@ -14,6 +14,16 @@ constexpr int kMaxConv = 4;         // widest causal conv in front of the scan
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
+// A[d, n] is taken as (n + 1)·A[d, 0], so that a token's decay factors are
+// powers of one base, when the two differ by at most 2^−21 of A[d, n] (4 to
+// 8 float32 ulps). exp(Δ·A) then changes by a relative Δ·|A|·2^−21: no more
+// than the MUFU exponential's own error while Δ·|A| ≤ 1/2, and beyond that
+// only in factors below e^−1/2. The pages' A = −exp(log(1..N)), which float32
+// rounds a few ulps off the integers, qualifies.
+__host__ __device__ __forceinline__ bool ladder_state(float an, float a0, int n) {
+    return fabsf(an - (float)(n + 1) * a0) <= 0x1p-21f * fabsf(an);
+}
+
 // ---- element I/O -------------------------------------------------------------
 __device__ __forceinline__ float to_f32(float v) { return v; }
 __device__ __forceinline__ float to_f32(__nv_bfloat16 v) { return __bfloat162float(v); }

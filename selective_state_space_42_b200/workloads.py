@@ -40,7 +40,8 @@ class ScanWorkload:
     final_state: bool = True
     # A[d, n]: "ladder" −(n+1); "exp_log" −exp(log(n+1)) evaluated in float32
     # (the pages' A = −exp(A_log) with A_log = log(1..N)), which is −(n+1)
-    # only up to rounding
+    # only up to rounding; "trained" −exp(log(n+1) + 0.1·N(0,1)) per (d, n),
+    # a general A such as training leaves
     a_init: str = "ladder"
 
     @property
@@ -157,9 +158,12 @@ WORKLOADS: Dict[str, ScanWorkload] = {
     "long_1m": ScanWorkload("long_1m", 1, 1 << 20, 2048, 16, "bf16",
                             gate=True, seed=3),
 }
-# the 2.8B layer with the pages' A = −exp(A_log) parametrisation
+# the 2.8B layer with the pages' A = −exp(A_log) parametrisation, and with a
+# general (per channel and state) A
 WORKLOADS["mamba2p8b_layer_expA"] = WORKLOADS["mamba2p8b_layer"].scaled(
     name="mamba2p8b_layer_expA", a_init="exp_log")
+WORKLOADS["mamba2p8b_layer_trainedA"] = WORKLOADS["mamba2p8b_layer"].scaled(
+    name="mamba2p8b_layer_trainedA", a_init="trained")
 
 DECODE = DecodeWorkload("decode_b256", 256, 5120, 16, 1000, "bf16", gate=True,
                         seed=4)
@@ -177,13 +181,18 @@ def _randn(shape, g, device, scale=1.0) -> torch.Tensor:
 
 
 def a_matrix(dim: int, dstate: int, a_init: str = "ladder", device="cpu") -> torch.Tensor:
-    """A [dim, dstate]: −(n+1), or −exp(log(n+1)) evaluated in float32 on the
-    CPU (so that every device sees the same values)."""
+    """A [dim, dstate]: −(n+1), −exp(log(n+1)), or −exp(log(n+1) + 0.1·N(0,1))
+    with a fixed seed, evaluated in float32 on the CPU (so that every device
+    sees the same values)."""
     n1 = torch.arange(1, dstate + 1, dtype=torch.float32)
     if a_init == "exp_log":
         row = -torch.exp(torch.log(n1))
     elif a_init == "ladder":
         row = -n1
+    elif a_init == "trained":
+        g = torch.Generator().manual_seed(20250)
+        noise = 0.1 * torch.randn(dim, dstate, generator=g, dtype=torch.float32)
+        return (-torch.exp(torch.log(n1)[None, :] + noise)).contiguous().to(device)
     else:
         raise ValueError(a_init)
     return row.repeat(dim, 1).contiguous().to(device)

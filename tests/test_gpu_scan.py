@@ -189,9 +189,16 @@ def test_mamba2p8b_layer_sampled():
 
 def test_mamba2p8b_layer_expA_sampled():
     """The benchmark's workload with the pages' A = −exp(log(1..16)) in float32,
-    which misses the exact-ladder test and takes the general decay (one exp
-    per state, part of them on the FMA pipe)."""
+    a few ulps off the integers: within the ladder test's bound, so it takes
+    the power-ladder decay of (n+1)·A[d, 0]."""
     _full_size_sampled("mamba2p8b_layer_expA", 160)
+
+
+def test_mamba2p8b_layer_trainedA_sampled():
+    """The benchmark's workload with a general A (−exp(log(n+1) + 0.1·N(0,1))
+    per channel and state): the general decay, one exp per state, part of
+    them on the FMA pipe."""
+    _full_size_sampled("mamba2p8b_layer_trainedA", 160)
 
 
 @pytest.mark.parametrize("a_init", ["exp_log", "random"])

@@ -142,3 +142,17 @@ def test_ragged_shapes_span_tiles_with_tails():
     assert shapes
     assert any(s[1] % 32 for s in shapes) and any(s[2] % 32 for s in shapes)
     assert any(s[1] > 32 for s in shapes) and any(s[2] > 128 for s in shapes)
+
+
+def test_a_initialisations():
+    """The three A recipes: −(n+1) exactly; the pages' −exp(log(n+1)) within
+    2^−21 of it (the kernels' ladder bound); the trained-like A negative and
+    off the ladder by far more than that bound."""
+    ladder = wl.a_matrix(8, 16, "ladder")
+    assert torch.equal(ladder, -torch.arange(1, 17, dtype=torch.float32).repeat(8, 1))
+    pages = wl.a_matrix(8, 16, "exp_log")
+    assert float(((pages - ladder).abs() / ladder.abs()).max()) <= 2.0 ** -21
+    trained = wl.a_matrix(8, 16, "trained")
+    assert bool((trained < 0).all())
+    assert float(((trained - ladder).abs() / ladder.abs()).min()) > 2.0 ** -21
+    assert torch.equal(trained, wl.a_matrix(8, 16, "trained"))  # seeded
