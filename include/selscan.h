@@ -304,7 +304,7 @@ SELSCAN_API int selscan_state_update(float *state, const void *x, const void *de
  * (fixed summation order, no atomics). Outputs must not overlap any input.
  * Takes a stream-ordered device workspace (cudaMallocAsync / cudaFreeAsync
  * on `stream`) of selscan_bwd_workspace_bytes() bytes: the state entering
- * every 8-token tile of every chain, and per-32-channel partial sums of dB
+ * every 8-token tile of every chain, and per-channel-tile partial sums of dB
  * and dC. Above 16 states the states go in groups of 16 computed side by
  * side; the workspace then holds every group's checkpoints and partials and
  * three float32 [batch, seqlen, dim] arrays per group, summed in group

@@ -44,8 +44,12 @@ struct BwdParams {
 
 cudaError_t launch_scan_bwd(const BwdParams &p, bool bf16, cudaStream_t stream);
 // Two lanes per chain (scan_bwd2.cu): one 16-state group, no conv, Δ·B·x input.
+// Its CTAs cover bwd_pairs_tile_channels() channels (no fewer than the
+// one-lane kernel's, so the workspace's partial rows suffice): the channel
+// tiles of its partial sums when it runs.
 bool bwd_pairs_supported(const BwdParams &p, bool bf16);
 cudaError_t launch_scan_bwd_pairs(const BwdParams &p, bool bf16, cudaStream_t stream);
+int bwd_pairs_tile_channels();
 int bwd_tile_tokens();
 int bwd_tile_channels();
 int bwd_conv_tile_tokens();

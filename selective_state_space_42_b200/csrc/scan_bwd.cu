@@ -759,8 +759,11 @@ cudaError_t launch_scan_bwd(const BwdParams &params, bool bf16, cudaStream_t str
     cudaError_t e;
     BwdParams p = params;
     p.part_lane_order = bwd_pairs_supported(p, bf16) ? 1 : 0;
-    if (p.part_lane_order)
+    if (p.part_lane_order) {
+        // the two-lane kernel's channel tiles (its partial rows)
+        p.ctiles = (int)((p.dim + bwd_pairs_tile_channels() - 1) / bwd_pairs_tile_channels());
         e = launch_scan_bwd_pairs(p, bf16, stream);
+    }
     else if (bf16)
         e = p.z ? launch_gate<__nv_bfloat16, true>(p, stream)
                 : launch_gate<__nv_bfloat16, false>(p, stream);

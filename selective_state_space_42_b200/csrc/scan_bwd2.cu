@@ -28,7 +28,7 @@
 //    the walk stores λ_t, the recompute has already stored h_t, and 32 lanes
 //    each form 4 of the 4 tokens × 32 sums as Σ_c λ_t[c]·u_t[c] and
 //    Σ_c ds_t[c]·h_t[c] (the products dB = λ·u and dC = ds·h are never formed
-//    per chain); per tile the CTA's two warps add their rows and write one
+//    per chain); per tile the CTA's warps add their rows and write one
 //    128-byte row per token to the partial buffer of scan_bwd.cu, in the
 //    reducer's value order (part_lane_order), which its reduction kernel
 //    sums over the channel tiles.
@@ -36,9 +36,11 @@
 // the walk is six f32x2 operations per state pair: λ_t = ds·C + λa_{t+1},
 // du += λ_t·B, λa = λ_t·Abar_t, lh = λa·h_{t−1}, q += lh·A, dA += Δ·lh.
 //
-// A CTA is two warps = 32 consecutive channels of one batch row, the channel
-// tile of scan_bwd.cu: the checkpoint, partial and per-channel buffers keep
-// their sizes.
+// A CTA is three warps = 48 consecutive channels of one batch row, three
+// CTAs per SM: the time follows the busiest SM, and 48-channel tiles put at
+// most 9 warps on an SM where 32-channel ones put 10 (at the 2.8B layer's
+// 4 × 5120 channels). Its partial-sum tiles are wider than scan_bwd.cu's
+// 32-channel ones, so the workspace's partial buffer suffices.
 #include "bwd_params.cuh"
 
 namespace selscan {
@@ -46,7 +48,8 @@ namespace {
 
 constexpr int kSeg = 8;     // tokens per tile (checkpoint interval)
 constexpr int kOwn = 4;     // tokens per tile whose scalars one lane forms
-constexpr int kWarps = 2;   // warps per CTA
+constexpr int kWarps = 3;   // warps per CTA
+constexpr int kCtasPerSm = 9 / kWarps;  // resident CTAs per SM (shared memory bound)
 constexpr int kCh = 16;     // channels per warp
 constexpr int kVals = 2 * kMaxN;
 constexpr int kPairs = 4;   // f32x2 registers holding a lane's 8 states
@@ -491,16 +494,21 @@ __device__ __forceinline__ void bwd_pairs_body(WarpSmem<T> *S, const BwdParams &
                         *reinterpret_cast<const uint4 *>(out + (a * kSeg + r) * kCh + q * kPer);
             }
         }
-        // the two warps' sums: one 128-byte row per token of the channel tile,
-        // in the reducer's order (the reduction kernel maps it to states)
+        // the CTA's sums (its warps' rows added): one 128-byte row per token
+        // of the channel tile, in the reducer's order (the reduction kernel
+        // maps it to states)
         __syncthreads();
-        {
-            const int t = threadIdx.x >> 3, g = threadIdx.x & 7;
+        for (int i = threadIdx.x; i < kSeg * 8; i += kWarps * 32) {
+            const int t = i >> 3, g = i & 7;
             const long long tok = t0 + t;
             if (tok < p.seqlen) {
-                const float4 r0 = S[0].row[t][g], r1 = S[1].row[t][g];
-                *reinterpret_cast<float4 *>(part + tok * kVals + 4 * g) =
-                    make_float4(r0.x + r1.x, r0.y + r1.y, r0.z + r1.z, r0.w + r1.w);
+                float4 r = S[0].row[t][g];
+#pragma unroll
+                for (int w = 1; w < kWarps; ++w) {
+                    const float4 o = S[w].row[t][g];
+                    r = make_float4(r.x + o.x, r.y + o.y, r.z + o.z, r.w + o.w);
+                }
+                *reinterpret_cast<float4 *>(part + tok * kVals + 4 * g) = r;
             }
         }
     }
@@ -535,7 +543,7 @@ __device__ __forceinline__ void bwd_pairs_body(WarpSmem<T> *S, const BwdParams &
 }
 
 template <typename T, bool kGate, bool kSoftplus>
-__global__ void __launch_bounds__(kWarps * 32, 5) scan_bwd_pairs_kernel(const BwdParams p) {
+__global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) scan_bwd_pairs_kernel(const BwdParams p) {
     extern __shared__ __align__(128) unsigned char smem[];
     WarpSmem<T> *S = reinterpret_cast<WarpSmem<T> *>(smem);
     // A[d, n] = (n+1)·A[d, 0] (ladder_state) for every state of every channel
@@ -559,7 +567,7 @@ cudaError_t launch_one(const BwdParams &p, cudaStream_t stream) {
     auto *kern = scan_bwd_pairs_kernel<T, kGate, kSoftplus>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    // five CTAs per SM need the largest shared-memory carveout
+    // kCtasPerSm CTAs per SM need the largest shared-memory carveout
     e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
                              cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return e;
@@ -585,6 +593,8 @@ bool bwd_pairs_supported(const BwdParams &p, bool bf16) {
            aligned16(p.B) && aligned16(p.C) && aligned16(p.dx) && aligned16(p.ddelta) &&
            aligned16(p.dz) && aligned16(p.ckpt);
 }
+
+int bwd_pairs_tile_channels() { return kWarps * kCh; }
 
 cudaError_t launch_scan_bwd_pairs(const BwdParams &p, bool bf16, cudaStream_t stream) {
     if (bf16)
