@@ -240,29 +240,75 @@ scan_kernel(const ScanParams p) {
     }
 }
 
-// Chunk carry: one thread per (b, d, n), sequential over chunks,
-// hin_0 = 0, hin_{c+1} = P_c · hin_c + H_c; hin_c overwrites H_c in place.
-// Only the aggregates of chunks 0 .. nchunks-2 are read (pass 1 skips the
-// last chunk), so every workspace element is written before it is read.
+// Chunk carry: hin_0 = h0 (or 0), hin_{c+1} = P_c · hin_c + H_c, hin_c
+// written over H_c in place. Each chunk's aggregate is the affine map
+// h ↦ P_c·h + H_c, and the maps compose associatively (later ∘ earlier:
+// (P2, H2)∘(P1, H1) = (P2·P1, P2·H1 + H2)), so one warp per (b, d, group of
+// 4 states) takes 32 chunks at a time, lane c chunk c0 + c: a warp-shuffle
+// inclusive scan gives each lane the map from the block's start through its
+// chunk, the exclusive map (the lane below's) applied to the state entering
+// the block is its chunk's hin, and lane 31's map carries that state to the
+// next block. Only the aggregates of chunks 0 .. nchunks-2 are read (pass 1
+// skips the last chunk, which takes the identity map), so every workspace
+// element is written before it is read.
+__device__ __forceinline__ float4 fma4(float4 a, float4 b, float4 c) {
+    return make_float4(fmaf(a.x, b.x, c.x), fmaf(a.y, b.y, c.y), fmaf(a.z, b.z, c.z),
+                       fmaf(a.w, b.w, c.w));
+}
+__device__ __forceinline__ float4 mul4(float4 a, float4 b) {
+    return make_float4(a.x * b.x, a.y * b.y, a.z * b.z, a.w * b.w);
+}
+__device__ __forceinline__ float4 shfl_up4(float4 v, int off) {
+    return make_float4(__shfl_up_sync(0xffffffffu, v.x, off), __shfl_up_sync(0xffffffffu, v.y, off),
+                       __shfl_up_sync(0xffffffffu, v.z, off), __shfl_up_sync(0xffffffffu, v.w, off));
+}
+__device__ __forceinline__ float4 shfl4(float4 v, int src) {
+    return make_float4(__shfl_sync(0xffffffffu, v.x, src), __shfl_sync(0xffffffffu, v.y, src),
+                       __shfl_sync(0xffffffffu, v.z, src), __shfl_sync(0xffffffffu, v.w, src));
+}
+
+constexpr int kCarryGroup = 4;  // states per lane
+
 __global__ void carry_kernel(const ScanParams p) {
-    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    const int64_t total = p.batch * p.dim * kMaxN;
-    if (i >= total) return;
-    const int64_t n = i % kMaxN;
-    const int64_t bd = i / kMaxN;
-    const int64_t d = bd % p.dim;
-    const int64_t b = bd / p.dim;
-    float h = (p.h0 && n < p.dstate) ? p.h0[(b * p.dim + d) * p.dstate + n] : 0.0f;
-    for (int c = 0; c < p.nchunks; ++c) {
-        const size_t idx = (((size_t)b * p.nchunks + c) * p.dim + d) * kMaxN + n;
+    const int lane = threadIdx.x & 31;
+    const int64_t gw = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    constexpr int kGroups = kMaxN / kCarryGroup;
+    if (gw >= p.batch * p.dim * kGroups) return;  // whole warps
+    const int n0 = (int)(gw % kGroups) * kCarryGroup;
+    const int64_t bd = gw / kGroups;
+    const int64_t d = bd % p.dim, b = bd / p.dim;
+    float hv[kCarryGroup];
+#pragma unroll
+    for (int k = 0; k < kCarryGroup; ++k)
+        hv[k] = (p.h0 && n0 + k < p.dstate) ? p.h0[(b * p.dim + d) * p.dstate + n0 + k] : 0.0f;
+    float4 h = make_float4(hv[0], hv[1], hv[2], hv[3]);
+    const float4 one = make_float4(1.f, 1.f, 1.f, 1.f), zero = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int c0 = 0; c0 < p.nchunks; c0 += 32) {
+        const int c = c0 + lane;
+        const size_t idx = (((size_t)b * p.nchunks + c) * p.dim + d) * kMaxN + n0;
+        float4 P = one, H = zero;
         if (c + 1 < p.nchunks) {
-            const float P = p.ws_P[idx];
-            const float H = p.ws_H[idx];
-            p.ws_H[idx] = h;
-            h = fmaf(P, h, H);
-        } else {
-            p.ws_H[idx] = h;
+            P = *reinterpret_cast<const float4 *>(p.ws_P + idx);
+            H = *reinterpret_cast<const float4 *>(p.ws_H + idx);
         }
+        // inclusive scan: lane c holds the map of chunks c0 .. c
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const float4 Pp = shfl_up4(P, off), Hp = shfl_up4(H, off);
+            if (lane >= off) {
+                H = fma4(P, Hp, H);
+                P = mul4(P, Pp);
+            }
+        }
+        // exclusive: the map of chunks c0 .. c − 1, applied to the state
+        // entering the block
+        float4 Pe = shfl_up4(P, 1), He = shfl_up4(H, 1);
+        if (lane == 0) {
+            Pe = one;
+            He = zero;
+        }
+        if (c < p.nchunks) *reinterpret_cast<float4 *>(p.ws_H + idx) = fma4(Pe, h, He);
+        h = fma4(shfl4(P, 31), h, shfl4(H, 31));
     }
 }
 
@@ -279,8 +325,8 @@ cudaError_t launch_typed(const ScanParams &p, cudaStream_t stream) {
     if (p.nchunks > 1) {
         e = launch_one<T, false, kModeAggregate>(p, blocks, stream);
         if (e != cudaSuccess) return e;
-        const int64_t total = p.batch * p.dim * kMaxN;
-        carry_kernel<<<(unsigned)((total + 255) / 256), 256, 0, stream>>>(p);
+        const int64_t threads = p.batch * p.dim * (kMaxN / kCarryGroup) * 32;
+        carry_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, stream>>>(p);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
@@ -292,8 +338,8 @@ cudaError_t launch_typed(const ScanParams &p, cudaStream_t stream) {
 }  // namespace
 
 cudaError_t launch_carry(const ScanParams &p, cudaStream_t stream) {
-    const int64_t total = p.batch * p.dim * kMaxN;
-    carry_kernel<<<(unsigned)((total + 255) / 256), 256, 0, stream>>>(p);
+    const int64_t threads = p.batch * p.dim * (kMaxN / kCarryGroup) * 32;
+    carry_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, stream>>>(p);
     return cudaGetLastError();
 }
 
